@@ -1,0 +1,119 @@
+"""The chunked form of the IA recurrence, in numpy fp64 -- test infrastructure.
+
+The paper runs the S4D recurrence chunkwise (paperlayer.ai summary of
+'Interdomain Attention', sec. 3.2 and sec. A.2: parallel work inside chunks of
+64 tokens, states passed across chunk boundaries, a second pass recomputing
+each chunk from its corrected initial state).  This file writes out the exact
+re-association that the tensor-core kernels use, so that the algebra itself is
+checked on the CPU against the sequential oracle (pin P7) before any kernel
+runs.  It imports nothing from the CUDA path and the CUDA path imports nothing
+from here.
+
+Per (b,h), chunk length C, centre c = C // 2, positions i (query) and j (key)
+in [0, C), tables per head:
+    E'[j,m] = b_m lambda_m^(c-j)          s[i,m] = |lambda_m|^(2(i-c))
+The running state is kept scaled, S_hat = lambda^-(C-c-1) S (U, Gamma, eta), so
+that the state carried into a chunk and the decayed state it adds to are the
+same product R = lambda^C S_hat0 = lambda^(c+1) S0.  For one chunk:
+    a~[i]  = sum_{j<=i} S_ij E'[j] + R_U xi(q_i)          (a_i = lambda^(i-c) a~_i)
+    X[i]   = s[i] conj(a~[i])                              (= conj(a_i) lambda^(i-c))
+    P_ij   = Re sum_m X[i,m] E'[j,m],  masked j <= i
+    num_i  = sum_j P_ij v_j + Re sum_m X[i,m] R_Gamma[m]
+    den_i  = sum_j P_ij     + Re sum_m X[i,m] R_eta[m]
+    S_hat1 = R + sum_j E'[j] x_j^T          (x = xi(k), v, 1)
+A ragged last chunk is zero-padded; its padded tokens add nothing but still
+decay the state, which the end state undoes with lambda^(n_valid - C).
+Segments: the local end states of equal segments of L tokens combine as
+S_in(s+1) = lambda^L S_in(s) + S_local(s).
+"""
+import numpy as np
+
+
+def feat(x):
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def tables(lam, b, C):
+    c = C // 2
+    j = np.arange(C)
+    Ep = b[None, :] * lam[None, :] ** (c - j[:, None])          # [C, M]
+    s = np.abs(lam[None, :]) ** (2.0 * (j[:, None] - c))        # [C, M]
+    return Ep, s, c
+
+
+def chunk_pass(fq, fk, v, lam, b, C, S0=None, with_outputs=True, rnd=None):
+    """One (b,h) sequence.  fq, fk [N,d], v [N,dv]; S0 = (U, G, eta) unscaled.
+
+    rnd, if given, is a function applied to every tensor-core operand (to
+    emulate fp16/bf16 rounding); accumulations stay fp64 here.
+    Returns (o, num, den, (U, G, eta)) with the end state unscaled."""
+    N, d = fq.shape
+    dv = v.shape[1]
+    M = lam.shape[0]
+    r = rnd if rnd is not None else (lambda x: x)
+    Ep, s, c = tables(lam, b, C)
+    sc = lam ** (C - c - 1)        # = lambda^(c-1) when C = 2c
+    if S0 is None:
+        Uh = np.zeros((M, d), complex); Gh = np.zeros((M, dv), complex); eh = np.zeros(M, complex)
+    else:
+        Uh, Gh, eh = (S0[0] / sc[:, None], S0[1] / sc[:, None], S0[2] / sc)
+    lamC = lam ** C
+    o = np.zeros((N, dv)); num = np.zeros((N, dv)); den = np.zeros(N)
+    ii = np.arange(C)
+    causal = ii[None, :] <= ii[:, None]                      # [i, j]
+    Epr = r(Ep.real) + 1j * r(Ep.imag)
+    nv = C
+    for n0 in range(0, N, C):
+        nv = min(C, N - n0)
+        Q = np.zeros((C, d)); K = np.zeros((C, d)); V = np.zeros((C, dv)); one = np.zeros(C)
+        Q[:nv] = fq[n0:n0 + nv]; K[:nv] = fk[n0:n0 + nv]; V[:nv] = v[n0:n0 + nv]; one[:nv] = 1.0
+        Q, K, V = r(Q), r(K), r(V)
+        RU, RG, Re_ = lamC[:, None] * Uh, lamC[:, None] * Gh, lamC * eh
+        if with_outputs:
+            S = Q @ K.T
+            Sb = r(np.where(causal & (ii[None, :] < nv), S, 0.0))
+            RUr = r(RU.real) + 1j * r(RU.imag)
+            at = Sb @ Epr + Q @ RUr.T                            # a~ [C, M]
+            X = s * np.conj(at)
+            Xr = r(X.real) + 1j * r(X.imag)
+            P = np.where(causal, (Xr @ Epr.T).real, 0.0)
+            Pr = r(P)
+            RGr = r(RG.real) + 1j * r(RG.imag)
+            Rer = r(Re_.real) + 1j * r(Re_.imag)
+            nm = Pr @ V + (Xr @ RGr).real
+            dn = Pr @ one + (Xr @ Rer).real
+            o[n0:n0 + nv] = nm[:nv] / dn[:nv, None]
+            num[n0:n0 + nv] = nm[:nv]
+            den[n0:n0 + nv] = dn[:nv]
+        Uh = RU + Epr.T @ K
+        Gh = RG + Epr.T @ V
+        eh = Re_ + Epr.T @ one
+    fix = lam ** (nv - C) if N > 0 else np.ones_like(lam)
+    end = (sc[:, None] * fix[:, None] * Uh, sc[:, None] * fix[:, None] * Gh, sc * fix * eh)
+    return o, num, den, end
+
+
+def segmented_pass(fq, fk, v, lam, b, C, L):
+    """Two-pass form over segments of L tokens (L a multiple of C):
+    local end states from zero, an exclusive scan of the carries, then every
+    segment recomputed from its carry-in."""
+    N = fq.shape[0]
+    starts = list(range(0, N, L))
+    local = []
+    for s0 in starts[:-1]:
+        _, _, _, end = chunk_pass(fq[s0:s0 + L], fk[s0:s0 + L], v[s0:s0 + L], lam, b, C,
+                                  with_outputs=False)
+        local.append(end)
+    M, d, dv = lam.shape[0], fq.shape[1], v.shape[1]
+    carry = (np.zeros((M, d), complex), np.zeros((M, dv), complex), np.zeros(M, complex))
+    lamL = lam ** L
+    outs = []
+    for si, s0 in enumerate(starts):
+        o, num, den, end = chunk_pass(fq[s0:s0 + L], fk[s0:s0 + L], v[s0:s0 + L], lam, b, C, S0=carry)
+        outs.append((o, num, den))
+        if si < len(local):
+            carry = tuple(lamL.reshape((-1,) + (1,) * (x.ndim - 1)) * x + y
+                          for x, y in zip(carry, local[si]))
+    o = np.concatenate([x[0] for x in outs]); num = np.concatenate([x[1] for x in outs])
+    den = np.concatenate([x[2] for x in outs])
+    return o, num, den, end

@@ -1,0 +1,56 @@
+"""Pin P7: the chunked re-association used by the kernels equals the plain
+sequential recurrence (paperlayer.ai summary of 'Interdomain Attention',
+sec. 3.2 and sec. A.2: chunkwise execution with state passing and a second
+pass from corrected initial states).  fp64, CPU only."""
+import numpy as np
+import pytest
+
+from chunk_algebra import chunk_pass, feat, segmented_pass
+
+
+def rel(x, r):
+    return float(np.max(np.abs(np.asarray(x) - np.asarray(r))) / np.max(np.abs(r)))
+
+
+def case(seed, N, d=3, dv=2, M=5, delta=0.07):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 1, N, d)); k = rng.standard_normal((1, 1, N, d))
+    v = rng.standard_normal((1, 1, N, dv))
+    return q, k, v, np.array([delta]), M
+
+
+@pytest.mark.parametrize("C", [1, 2, 3, 16, 64])
+@pytest.mark.parametrize("N", [1, 5, 64, 77, 130])
+def test_p7_chunked_equals_sequential(oracle_mod, C, N):
+    q, k, v, delta, M = case(C * 1000 + N, N)
+    ref = oracle_mod.forward(q, k, v, delta, M)
+    lam, b = oracle_mod.params(M, delta[0])
+    o, num, den, (U, G, e) = chunk_pass(feat(q[0, 0]), feat(k[0, 0]), v[0, 0], lam, b, C)
+    assert rel(num, ref["num"][0, 0]) < 1e-11
+    assert rel(den, ref["den"][0, 0]) < 1e-11
+    Ur, Gr, er = oracle_mod.split_state(ref["state"], 1, 1, M, q.shape[-1], v.shape[-1])
+    assert rel(U, Ur[0, 0]) < 1e-11 and rel(G, Gr[0, 0]) < 1e-11 and rel(e, er[0, 0]) < 1e-11
+
+
+def test_p7_chunked_with_state_in_and_fast_modes(oracle_mod):
+    q, k, v, delta, M = case(3, 150, d=4, dv=3, M=64, delta=0.1)
+    pre = oracle_mod.forward(q[:, :, :40], k[:, :, :40], v[:, :, :40], delta, M)
+    ref = oracle_mod.forward(q[:, :, 40:], k[:, :, 40:], v[:, :, 40:], delta, M, state_in=pre["state"])
+    U0, G0, e0 = oracle_mod.split_state(pre["state"], 1, 1, M, 4, 3)
+    lam, b = oracle_mod.params(M, delta[0])
+    o, num, den, _ = chunk_pass(feat(q[0, 0, 40:]), feat(k[0, 0, 40:]), v[0, 0, 40:], lam, b, 64,
+                                S0=(U0[0, 0], G0[0, 0], e0[0, 0]))
+    assert rel(num, ref["num"][0, 0]) < 1e-10
+    assert rel(den, ref["den"][0, 0]) < 1e-10
+
+
+@pytest.mark.parametrize("L,N", [(64, 200), (128, 384), (192, 500)])
+def test_p7_segmented_two_pass(oracle_mod, L, N):
+    q, k, v, delta, M = case(L + N, N, M=8, delta=0.02)
+    ref = oracle_mod.forward(q, k, v, delta, M)
+    lam, b = oracle_mod.params(M, delta[0])
+    o, num, den, (U, G, e) = segmented_pass(feat(q[0, 0]), feat(k[0, 0]), v[0, 0], lam, b, 64, L)
+    assert rel(num, ref["num"][0, 0]) < 1e-11
+    assert rel(den, ref["den"][0, 0]) < 1e-11
+    Ur, Gr, er = oracle_mod.split_state(ref["state"], 1, 1, M, 3, 2)
+    assert rel(U, Ur[0, 0]) < 1e-11 and rel(e, er[0, 0]) < 1e-11
