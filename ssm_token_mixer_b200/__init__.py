@@ -1,0 +1,193 @@
+"""Interdomain Attention (IA) layer hot path for NVIDIA B200 -- Python binding.
+
+This module only marshals torch tensors (device memory and the current CUDA
+stream) into the C-ABI of ``lib/libia.so`` (declared in ``include/ia.h``);
+every step of the layer runs in that library's sm_100a kernels.  There is no
+CPU or PyTorch fallback: if the library is missing or a call fails, the call
+raises.
+
+Entry points (same names as the C-ABI):
+  prefill_fwd(q, k, v, delta, M, ...)   causal prefill, returns o (+ num, den, state)
+  fwd_bwd(q, k, v, delta, dO, M, ...)   training step: o, dq, dk, dv, dDelta
+  decode_step(q, k, v, delta, state, M)  one recurrent step, state updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["IAError", "load_library", "state_bytes", "prefill_workspace_bytes",
+           "fwd_bwd_workspace_bytes", "prefill_fwd", "fwd_bwd", "decode_step",
+           "check_device_errors", "library_path", "IA_F32", "IA_BF16"]
+
+IA_F32, IA_BF16 = 0, 1
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "lib", "libia.so")
+_lib = None
+
+STATUS = {0: "IA_OK", 1: "IA_ERR_INVALID_ARG", 2: "IA_ERR_UNSUPPORTED", 3: "IA_ERR_WORKSPACE",
+          4: "IA_ERR_CUDA", 5: "IA_ERR_TIMEOUT"}
+
+
+class IAError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = _lib.ia_status_string(status).decode() if _lib else STATUS.get(status, str(status))
+        super().__init__(f"{where}: {msg}")
+
+
+class IAShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("d_xi", ctypes.c_int), ("d_v", ctypes.c_int), ("M", ctypes.c_int),
+                ("in_dtype", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libia.so (built by ssm_token_mixer_b200.build); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m ssm_token_mixer_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, S = ctypes.c_void_p, ctypes.POINTER(IAShape)
+    for name in ("ia_state_bytes", "ia_prefill_workspace_bytes", "ia_fwd_bwd_workspace_bytes"):
+        getattr(lib, name).restype = ctypes.c_size_t
+        getattr(lib, name).argtypes = [S]
+    lib.ia_prefill_fwd.restype = ctypes.c_int
+    lib.ia_prefill_fwd.argtypes = [S] + [P] * 10 + [P, ctypes.c_size_t, P]
+    lib.ia_fwd_bwd.restype = ctypes.c_int
+    lib.ia_fwd_bwd.argtypes = [S] + [P] * 11 + [P, ctypes.c_size_t, P]
+    lib.ia_decode_step.restype = ctypes.c_int
+    lib.ia_decode_step.argtypes = [S] + [P] * 9 + [P]
+    lib.ia_check_device_errors.restype = ctypes.c_int
+    lib.ia_check_device_errors.argtypes = [P]
+    lib.ia_status_string.restype = ctypes.c_char_p
+    lib.ia_status_string.argtypes = [ctypes.c_int]
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return IA_F32
+    if t.dtype == torch.bfloat16:
+        return IA_BF16
+    raise TypeError(f"unsupported input dtype {t.dtype} (float32 or bfloat16)")
+
+
+def make_shape(B, H, N, d_xi, d_v, M, dtype) -> IAShape:
+    code = dtype if isinstance(dtype, int) else (IA_BF16 if dtype in (torch.bfloat16, "bf16") else IA_F32)
+    return IAShape(int(B), int(H), int(N), int(d_xi), int(d_v), int(M), code)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, where):
+    if status != 0:
+        raise IAError(status, where)
+
+
+def state_bytes(B, H, M, d_xi, d_v) -> int:
+    return int(load_library().ia_state_bytes(ctypes.byref(make_shape(B, H, 1, d_xi, d_v, M, IA_F32))))
+
+
+def prefill_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
+    return int(load_library().ia_prefill_workspace_bytes(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
+
+
+def fwd_bwd_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
+    return int(load_library().ia_fwd_bwd_workspace_bytes(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
+
+
+def _workspace(nbytes, device, workspace):
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def prefill_fwd(q, k, v, delta, M, A=None, state_in=None, want_num_den=False, want_state=False,
+                o=None, workspace=None, stream=None):
+    """Causal IA prefill.  q,k [B,H,N,d_xi], v [B,H,N,d_v] (fp32 or bf16), delta [H] fp32.
+
+    Returns dict with o [B,H,N,d_v] fp32 and, on request, num, den, state (flat fp32)."""
+    lib = load_library()
+    B, H, N, d_xi = q.shape
+    d_v = v.shape[-1]
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    dev = q.device
+    if o is None:
+        o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    num = torch.empty_like(o) if want_num_den else None
+    den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
+    st = torch.empty(lib.ia_state_bytes(ctypes.byref(shp)) // 4, dtype=torch.float32, device=dev) if want_state else None
+    need = lib.ia_prefill_workspace_bytes(ctypes.byref(shp))
+    ws = _workspace(need, dev, workspace)
+    rc = lib.ia_prefill_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
+                            _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _ptr(ws),
+                            ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream))
+    _check(rc, "ia_prefill_fwd")
+    return {"o": o, "num": num, "den": den, "state": st}
+
+
+def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
+    """Forward + reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta)."""
+    lib = load_library()
+    B, H, N, d_xi = q.shape
+    d_v = v.shape[-1]
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    dev = q.device
+    o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    dq = torch.empty(B, H, N, d_xi, dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    dD = torch.empty(H, dtype=torch.float32, device=dev)
+    need = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(shp))
+    ws = _workspace(need, dev, workspace)
+    rc = lib.ia_fwd_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A), _ptr(dO),
+                        _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dD), _ptr(ws),
+                        ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream))
+    _check(rc, "ia_fwd_bwd")
+    return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD}
+
+
+def decode_step(q, k, v, delta, state, M, A=None, o=None, want_num_den=False, stream=None):
+    """One decode step.  q,k [B,H,d_xi], v [B,H,d_v]; state (flat fp32) updated in place."""
+    lib = load_library()
+    B, H, d_xi = q.shape
+    d_v = v.shape[-1]
+    shp = make_shape(B, H, 1, d_xi, d_v, M, _dtype_code(q))
+    dev = q.device
+    if o is None:
+        o = torch.empty(B, H, d_v, dtype=torch.float32, device=dev)
+    num = torch.empty_like(o) if want_num_den else None
+    den = torch.empty(B, H, dtype=torch.float32, device=dev) if want_num_den else None
+    rc = lib.ia_decode_step(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
+                            _ptr(state), _ptr(o), _ptr(num), _ptr(den), _stream(stream))
+    _check(rc, "ia_decode_step")
+    return {"o": o, "num": num, "den": den}
+
+
+def check_device_errors(stream=None):
+    """Synchronise the stream and raise if a device-side bounded wait expired."""
+    _check(load_library().ia_check_device_errors(_stream(stream)), "ia_check_device_errors")

@@ -1,0 +1,190 @@
+// C-ABI of libia: argument validation on the host (before any launch),
+// workspace sizing and dispatch to the kernels.  See include/ia.h for the
+// contract of every entry point.
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "ia_device.cuh"
+#include "ia_internal.h"
+#include "ia_tables.cuh"
+
+namespace ia {
+
+// Raised by device-side bounded waits that expire (bit 0); read and cleared
+// by ia_check_device_errors().
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr size_t kMaxSmem = 232448;   // 227 KB opt-in shared memory per block on sm_100
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool env_set(const char* name) {
+  const char* s = std::getenv(name);
+  return s && s[0] && std::strcmp(s, "0") != 0;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();   // clear a sticky "no device" error; plan for a B200
+    return 148;
+  }
+  return n;
+}
+
+bool valid_dims(const ia_shape_t* s, bool need_n) {
+  if (!s) return false;
+  if (s->B <= 0 || s->H <= 0 || s->d_xi <= 0 || s->d_v <= 0 || s->M <= 0) return false;
+  if (need_n && s->N <= 0) return false;
+  if (s->in_dtype != IA_F32 && s->in_dtype != IA_BF16) return false;
+  // element counts must stay addressable with 64-bit indices and int grid sizes
+  const long long BH = static_cast<long long>(s->B) * s->H;
+  if (BH > (1LL << 31) - 1) return false;
+  return true;
+}
+
+bool use_tc(const ia_shape_t& s) {
+  if (env_set("IA_PREFILL_SIMT")) return false;   // debug switch: force the CUDA-core path
+  return tc_prefill_supported(s);
+}
+
+ia_status_t map_cuda(cudaError_t e) { return e == cudaSuccess ? IA_OK : IA_ERR_CUDA; }
+
+}  // namespace
+
+int* device_error_ptr() {
+  constexpr int kMaxDev = 64;
+  static int* cache[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+int read_and_clear_device_error(cudaStream_t st, cudaError_t* err) {
+  int flag = 0;
+  *err = cudaStreamSynchronize(st);
+  if (*err != cudaSuccess) return 0;
+  *err = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int));
+  if (*err != cudaSuccess) return 0;
+  if (flag) {
+    int zero = 0;
+    *err = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  }
+  return flag;
+}
+
+}  // namespace ia
+
+using namespace ia;
+
+extern "C" {
+
+size_t ia_state_bytes(const ia_shape_t* s) {
+  if (!valid_dims(s, false)) return 0;
+  return sizeof(float) * 2 * static_cast<size_t>(s->B) * s->H * s->M *
+         (static_cast<size_t>(s->d_xi) + s->d_v + 1);
+}
+
+size_t ia_prefill_workspace_bytes(const ia_shape_t* s) {
+  if (!valid_dims(s, true)) return 0;
+  if (!use_tc(*s)) return 0;
+  return tc_workspace_bytes(*s, tc_plan(*s, num_sms()));
+}
+
+size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* s) {
+  if (!valid_dims(s, true)) return 0;
+  return sizeof(float2) * static_cast<size_t>(s->B) * s->H *
+             seq_bwd_ws_per_bh(s->N, s->d_xi, s->d_v, s->M) + 256;
+}
+
+ia_status_t ia_prefill_fwd(const ia_shape_t* s, const void* q, const void* k, const void* v,
+                           const float* delta, const float* A, const void* state_in, float* o,
+                           float* num, float* den, void* state_out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!valid_dims(s, true)) return IA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !delta || !o) return IA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, delta, A, state_in, o, num, den, state_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
+  if (state_in && state_in == state_out) return IA_ERR_INVALID_ARG;
+  const bool tc = use_tc(*s);
+  size_t need = 0;
+  TcPlan plan{1, 1};
+  if (tc) {
+    plan = tc_plan(*s, num_sms());
+    need = tc_workspace_bytes(*s, plan);
+  } else if (seq_fwd_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) {
+    return IA_ERR_UNSUPPORTED;
+  }
+  if (need > 0 && (!workspace || workspace_bytes < need)) return IA_ERR_WORKSPACE;
+  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc)
+    return map_cuda(launch_tc_prefill(*s, plan, q, k, v, delta, A, state_in, o, num, den,
+                                      state_out, workspace, st));
+  return map_cuda(launch_seq_fwd(*s, q, k, v, delta, A, state_in, o, num, den, state_out, st));
+}
+
+ia_status_t ia_fwd_bwd(const ia_shape_t* s, const void* q, const void* k, const void* v,
+                       const float* delta, const float* A, const void* dO, float* o, float* dq,
+                       float* dk, float* dv, float* dDelta, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (!valid_dims(s, true)) return IA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !delta || !dO || !o || !dq || !dk || !dv || !dDelta)
+    return IA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
+  if (seq_bwd_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  const size_t need = ia_fwd_bwd_workspace_bytes(s);
+  if (!workspace || workspace_bytes < need) return IA_ERR_WORKSPACE;
+  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  return map_cuda(launch_seq_bwd(*s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, const void* v,
+                           const float* delta, const float* A, void* state, float* o, float* num,
+                           float* den, void* stream) {
+  if (!valid_dims(s, false)) return IA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !delta || !state || !o) return IA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, delta, A, state, o, num, den};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
+  if ((s->d_xi & 1) || (s->d_v & 1)) return IA_ERR_UNSUPPORTED;   // 16-byte state vectors
+  const size_t smem = sizeof(float) * (2 * s->d_xi + 9 * s->d_v + 8) + 2 * sizeof(float2) * s->M + 16;
+  if (smem > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  return map_cuda(launch_decode(*s, q, k, v, delta, A, state, o, num, den,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+ia_status_t ia_check_device_errors(void* stream) {
+  cudaError_t e;
+  int flag = read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);
+  if (e != cudaSuccess) return IA_ERR_CUDA;
+  return flag ? IA_ERR_TIMEOUT : IA_OK;
+}
+
+const char* ia_status_string(ia_status_t st) {
+  switch (st) {
+    case IA_OK: return "IA_OK: success";
+    case IA_ERR_INVALID_ARG: return "IA_ERR_INVALID_ARG: null, misaligned or inconsistent argument";
+    case IA_ERR_UNSUPPORTED: return "IA_ERR_UNSUPPORTED: shape or dtype not implemented";
+    case IA_ERR_WORKSPACE: return "IA_ERR_WORKSPACE: workspace missing or too small";
+    case IA_ERR_CUDA: return "IA_ERR_CUDA: CUDA runtime or launch failure";
+    case IA_ERR_TIMEOUT: return "IA_ERR_TIMEOUT: a device-side bounded wait expired";
+  }
+  return "unknown ia_status_t";
+}
+
+}  // extern "C"

@@ -1,0 +1,193 @@
+// One recurrent decode step of the IA layer (paperlayer.ai summary of
+// 'Interdomain Attention', sec. 3.2: a fixed state of size O(M(R + d)) and
+// constant work per generated token; sec. F.3: graphed decode whose latency
+// does not depend on the prefix length).  For every (b,h):
+//   U <- lambda U + b xi(k)^T,  Gamma <- lambda Gamma + b v^T,  eta <- lambda eta + b
+//   a = U xi(q),  o = Re(a^H Gamma) / Re(a^H eta)
+//
+// The step is bound by state bytes: every state entry is read and written
+// once in fp32.  A thread-block cluster serves one (b,h); each CTA of the
+// cluster streams a group of modes with 16-byte loads and stores, keeps its
+// partial num/den in shared memory, and the cluster's rank-0 CTA sums the
+// partials over distributed shared memory and writes o.
+#include <cooperative_groups.h>
+
+#include "ia_device.cuh"
+#include "ia_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace ia {
+namespace {
+
+constexpr int kDecThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ float ldx(const T* p);
+template <>
+__device__ __forceinline__ float ldx<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ldx<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+__device__ __forceinline__ float xi_acc(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// shared: fq [DX] | fk [DX] | vv [DV] | part [8 warps][DV] | pden [8] | lam,b [MG] float2
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads) decode_kernel(
+    int H, int DX, int DV, int M, int MG, const T* __restrict__ q, const T* __restrict__ k,
+    const T* __restrict__ v, const float* __restrict__ delta, const float* __restrict__ A,
+    float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
+    float* __restrict__ den, long long BH) {
+  extern __shared__ float4 dsm[];
+  float* fq = reinterpret_cast<float*>(dsm);
+  float* fk = fq + DX;
+  float* vv = fk + DX;
+  float* part = vv + DV;                    // [8][DV]
+  float* pden = part + 8 * DV;              // [8]
+  float2* lamb = reinterpret_cast<float2*>(pden + 8);   // [MG] lambda, [MG] b
+  float2* bb = lamb + MG;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int g = static_cast<int>(cluster.block_rank());
+  const int G = static_cast<int>(cluster.num_blocks());
+  const long long bh = blockIdx.y;
+  const int h = static_cast<int>(bh % H);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = g * MG;
+
+  for (int f = tid; f < DX; f += kDecThreads) {
+    fq[f] = xi_acc(ldx(q + bh * DX + f));
+    fk[f] = xi_acc(ldx(k + bh * DX + f));
+  }
+  for (int f = tid; f < DV; f += kDecThreads) vv[f] = ldx(v + bh * DV + f);
+  for (int i = tid; i < MG; i += kDecThreads) {
+    const int m = m0 + i;
+    double ar = A ? static_cast<double>(A[2 * m]) : -0.5;
+    double ai = A ? static_cast<double>(A[2 * m + 1]) : 3.14159265358979323846 * m;
+    double d = static_cast<double>(delta[h]), e = exp(d * ar), s, c;
+    sincos(d * ai, &s, &c);
+    double lr = e * c, li = e * s, nr = lr - 1.0, dd = ar * ar + ai * ai;
+    lamb[i] = make_float2(static_cast<float>(lr), static_cast<float>(li));
+    bb[i] = make_float2(static_cast<float>((nr * ar + li * ai) / dd),
+                        static_cast<float>((li * ar - nr * ai) / dd));
+  }
+  for (int i = tid; i < 8 * DV + 8; i += kDecThreads) part[i] = 0.f;
+  __syncthreads();
+
+  float2* Ub = state + bh * M * DX;
+  float2* Gb = state + BH * M * DX + bh * M * DV;
+  float2* Eb = state + BH * M * (DX + DV) + bh * M;
+  float* mypart = part + warp * DV;
+  float dpart = 0.f;
+
+  for (int mi = warp; mi < MG && m0 + mi < M; mi += kDecThreads / 32) {
+    const int m = m0 + mi;
+    const float2 L = lamb[mi], Bm = bb[mi];
+    float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
+    float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
+    float ar = 0.f, ai = 0.f;
+    for (int p = lane; p < DX / 2; p += 32) {
+      float4 u = Ur[p];
+      const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
+      float4 w;
+      w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
+      w.y = fmaf(L.x, u.y, fmaf(L.y, u.x, Bm.y * x0));
+      w.z = fmaf(L.x, u.z, fmaf(-L.y, u.w, Bm.x * x1));
+      w.w = fmaf(L.x, u.w, fmaf(L.y, u.z, Bm.y * x1));
+      Ur[p] = w;
+      ar = fmaf(w.x, fq[2 * p], fmaf(w.z, fq[2 * p + 1], ar));
+      ai = fmaf(w.y, fq[2 * p], fmaf(w.w, fq[2 * p + 1], ai));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ar += __shfl_xor_sync(0xffffffffu, ar, off);
+      ai += __shfl_xor_sync(0xffffffffu, ai, off);
+    }
+    for (int p = lane; p < DV / 2; p += 32) {
+      float4 gv = Gr[p];
+      const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
+      float4 w;
+      w.x = fmaf(L.x, gv.x, fmaf(-L.y, gv.y, Bm.x * x0));
+      w.y = fmaf(L.x, gv.y, fmaf(L.y, gv.x, Bm.y * x0));
+      w.z = fmaf(L.x, gv.z, fmaf(-L.y, gv.w, Bm.x * x1));
+      w.w = fmaf(L.x, gv.w, fmaf(L.y, gv.z, Bm.y * x1));
+      Gr[p] = w;
+      mypart[2 * p] += fmaf(ar, w.x, ai * w.y);       // Re(conj(a) Gamma)
+      mypart[2 * p + 1] += fmaf(ar, w.z, ai * w.w);
+    }
+    if (lane == 0) {
+      float2 e = Eb[m];
+      float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
+      Eb[m] = w;
+      dpart += fmaf(ar, w.x, ai * w.y);
+    }
+  }
+  if (lane == 0) pden[warp] = dpart;
+  __syncthreads();
+  // CTA partial: fold the 8 warp rows into row 0
+  for (int f = tid; f < DV; f += kDecThreads) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += part[w * DV + f];
+    part[f] = s;
+  }
+  if (tid == 0) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += pden[w];
+    pden[0] = s;
+  }
+  cluster.sync();
+  if (g == 0) {
+    float dn = 0.f;
+    for (int r = 0; r < G; ++r) dn += cluster.map_shared_rank(pden, r)[0];
+    for (int f = tid; f < DV; f += kDecThreads) {
+      float s = 0.f;
+      for (int r = 0; r < G; ++r) s += cluster.map_shared_rank(part, r)[f];
+      o[bh * DV + f] = s / dn;
+      if (num) num[bh * DV + f] = s;
+    }
+    if (den && tid == 0) den[bh] = dn;
+  }
+  cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
+}
+
+template <typename T>
+cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const void* v,
+                        const float* delta, const float* A, void* state, float* o, float* num,
+                        float* den, cudaStream_t st) {
+  int G = (s.M + 15) / 16;
+  if (G > 8) G = 8;
+  const int MG = (s.M + G - 1) / G;
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + 8 * s.d_v + 8) + sizeof(float2) * 2 * MG + 16;
+  auto kern = decode_kernel<T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G, static_cast<unsigned>(BH), 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, MG, static_cast<const T*>(q),
+                            static_cast<const T*>(k), static_cast<const T*>(v), delta, A,
+                            static_cast<float2*>(state), o, num, den, BH);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
+                          const float* delta, const float* A, void* state, float* o, float* num,
+                          float* den, cudaStream_t st) {
+  if (s.in_dtype == IA_F32) return decode_impl<float>(s, q, k, v, delta, A, state, o, num, den, st);
+  return decode_impl<__nv_bfloat16>(s, q, k, v, delta, A, state, o, num, den, st);
+}
+
+}  // namespace ia

@@ -1,0 +1,54 @@
+// Internal launch interface between the C-ABI layer (ia_api.cu) and the
+// kernel translation units.  Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/ia.h"
+
+namespace ia {
+
+struct HeadTables;
+
+cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
+                                cudaStream_t st);
+
+size_t seq_fwd_smem(int DX, int DV, int M);
+cudaError_t launch_seq_fwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
+                           const float* delta, const float* A, const void* state_in, float* o,
+                           float* num, float* den, void* state_out, cudaStream_t st);
+
+size_t seq_bwd_smem(int DX, int DV, int M);
+size_t seq_bwd_ws_per_bh(int N, int DX, int DV, int M);   // in float2 units
+cudaError_t launch_seq_bwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
+                           const float* delta, const float* A, const void* dO, float* o, float* dq,
+                           float* dk, float* dv, float* dDelta, void* ws, cudaStream_t st);
+
+cudaError_t launch_segment_scan(int B, int H, int DX, int DV, int nseg, int L,
+                                const HeadTables* tabs, const void* state_in, float* ws_state,
+                                float* ws_eta, cudaStream_t st);
+
+// Tensor-core chunked prefill (bf16 inputs, M = 64).
+bool tc_prefill_supported(const ia_shape_t& s);
+struct TcPlan {
+  int nseg;        // segments per (b,h) sequence
+  int seg_chunks;  // chunks per segment (all but the last)
+};
+TcPlan tc_plan(const ia_shape_t& s, int num_sms);
+size_t tc_workspace_bytes(const ia_shape_t& s, const TcPlan& p);
+cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
+                              const void* v, const float* delta, const float* A,
+                              const void* state_in, float* o, float* num, float* den,
+                              void* state_out, void* ws, cudaStream_t st);
+
+// Decode step.
+cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
+                          const float* delta, const float* A, void* state, float* o, float* num,
+                          float* den, cudaStream_t st);
+
+// Device address of the library's error flag on the current device (looked
+// up once per device), or nullptr if the lookup fails.
+int* device_error_ptr();
+int read_and_clear_device_error(cudaStream_t st, cudaError_t* err);
+
+}  // namespace ia

@@ -1,0 +1,105 @@
+"""C-ABI contract checks that need no GPU: the library loads, exports every
+symbol include/ia.h declares, and rejects bad arguments on the host before
+any launch (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ssm_token_mixer_b200 import build
+    build.build()
+    import ssm_token_mixer_b200 as ia
+    return ia.load_library()
+
+
+def declared_symbols():
+    syms = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            syms |= set(re.findall(r"IA_API\s+[\w\s\*]+?\b(ia_\w+)\s*\(", text))
+    return syms
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert {"ia_prefill_fwd", "ia_fwd_bwd", "ia_decode_step"} <= syms
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def shape(B=2, H=3, N=100, dx=64, dv=64, M=64, dt=1):
+    import ssm_token_mixer_b200 as ia
+    return ia.IAShape(B, H, N, dx, dv, M, dt)
+
+
+FAKE = ctypes.c_void_p(0x10000)      # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def prefill(lib, s, q=FAKE, o=FAKE, state_in=None, state_out=None, ws=None, wsb=0):
+    return lib.ia_prefill_fwd(ctypes.byref(s) if s is not None else None, q, FAKE, FAKE, FAKE, None,
+                              state_in, o, None, None, state_out, ws, ctypes.c_size_t(wsb), None)
+
+
+def test_state_bytes(lib):
+    s = shape(B=2, H=3, dx=5, dv=7, M=11)
+    assert lib.ia_state_bytes(ctypes.byref(s)) == 8 * 2 * 3 * 11 * (5 + 7 + 1)
+
+
+def test_invalid_arguments(lib):
+    assert prefill(lib, None) == 1
+    for bad in (dict(B=0), dict(H=-1), dict(N=0), dict(dx=0), dict(M=0), dict(dt=7)):
+        assert prefill(lib, shape(**bad)) == 1, bad
+    assert prefill(lib, shape(), q=None) == 1
+    assert prefill(lib, shape(), o=None) == 1
+    assert prefill(lib, shape(), q=MISALIGNED) == 1
+    assert prefill(lib, shape(), state_in=FAKE, state_out=FAKE) == 1
+
+
+def test_workspace_checked_before_launch(lib):
+    s = shape()
+    need = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
+    assert need > 0                                     # tensor-core path uses tables
+    assert prefill(lib, s) == 3
+    assert prefill(lib, s, ws=FAKE, wsb=need - 1) == 3
+    fb = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(s))
+    rc = lib.ia_fwd_bwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                        FAKE, FAKE, ctypes.c_size_t(fb - 1), None)
+    assert rc == 3
+
+
+def test_decode_validation(lib):
+    s = shape(dx=63)
+    rc = lib.ia_decode_step(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, None)
+    assert rc == 2
+    rc = lib.ia_decode_step(ctypes.byref(shape()), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None, None)
+    assert rc == 1
+
+
+def test_injected_launch_failure(lib, monkeypatch):
+    monkeypatch.setenv("IA_INJECT_LAUNCH_FAILURE", "1")
+    s = shape(dt=0, dx=16, dv=16, M=4)                 # CUDA-core path: no workspace
+    assert prefill(lib, s) == 4
+    rc = lib.ia_decode_step(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, None)
+    assert rc == 4
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.ia_status_string(code).startswith(b"IA_")
+    assert b"unknown" in lib.ia_status_string(99)
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    import ssm_token_mixer_b200 as ia
+    monkeypatch.setattr(ia, "_lib", None)
+    monkeypatch.setattr(ia, "_LIB_PATH", "/nonexistent/libia.so")
+    with pytest.raises(RuntimeError):
+        ia.load_library()
