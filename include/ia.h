@@ -78,6 +78,11 @@ IA_API size_t ia_prefill_workspace_bytes(const ia_shape_t* shape);
 /* Workspace bytes ia_fwd_bwd needs for this shape. */
 IA_API size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* shape);
 
+/* Number of kernel launches one ia_prefill_fwd call makes for this shape
+ * (the tensor-core path adds a state-only pass and a carry scan when it
+ * splits sequences into segments); 0 for an invalid shape. */
+IA_API int ia_prefill_launches(const ia_shape_t* shape);
+
 /*
  * Causal prefill over N tokens (paperlayer.ai summary sec. 3.2 and sec. A.2:
  * chunkwise execution, chunk 64, with state passing; sec. F.2: chunked
@@ -117,6 +122,17 @@ IA_API ia_status_t ia_fwd_bwd(const ia_shape_t* shape, const void* q, const void
 IA_API ia_status_t ia_decode_step(const ia_shape_t* shape, const void* q, const void* k,
                            const void* v, const float* delta, const float* A, void* state,
                            float* o, float* num, float* den, void* stream);
+
+/*
+ * Profiling aid (no counterpart in the paper): registers two caller-owned
+ * CUDA events (cudaEvent_t handles).  While set, every later entry-point call
+ * records `begin` on its stream immediately before launching its dominant
+ * kernel (the full chunk pass of the prefill, the reverse-mode kernel of the
+ * training step, the decode kernel) and `end` immediately after it, so the
+ * caller can time that kernel alone.  Pass NULL, NULL to stop.  The events
+ * are not owned or destroyed by the library.
+ */
+IA_API ia_status_t ia_set_launch_events(void* begin, void* end);
 
 /* Synchronises `stream`, then reports (and clears) the device error flag
  * that bounded waits set when they expire: IA_OK or IA_ERR_TIMEOUT. */

@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["IAError", "load_library", "state_bytes", "prefill_workspace_bytes",
            "fwd_bwd_workspace_bytes", "prefill_fwd", "fwd_bwd", "decode_step",
-           "check_device_errors", "library_path", "IA_F32", "IA_BF16"]
+           "check_device_errors", "set_launch_events", "library_path", "IA_F32", "IA_BF16"]
 
 IA_F32, IA_BF16 = 0, 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -61,12 +61,16 @@ def load_library():
     for name in ("ia_state_bytes", "ia_prefill_workspace_bytes", "ia_fwd_bwd_workspace_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [S]
+    lib.ia_prefill_launches.restype = ctypes.c_int
+    lib.ia_prefill_launches.argtypes = [S]
     lib.ia_prefill_fwd.restype = ctypes.c_int
     lib.ia_prefill_fwd.argtypes = [S] + [P] * 10 + [P, ctypes.c_size_t, P]
     lib.ia_fwd_bwd.restype = ctypes.c_int
     lib.ia_fwd_bwd.argtypes = [S] + [P] * 11 + [P, ctypes.c_size_t, P]
     lib.ia_decode_step.restype = ctypes.c_int
     lib.ia_decode_step.argtypes = [S] + [P] * 9 + [P]
+    lib.ia_set_launch_events.restype = ctypes.c_int
+    lib.ia_set_launch_events.argtypes = [P, P]
     lib.ia_check_device_errors.restype = ctypes.c_int
     lib.ia_check_device_errors.argtypes = [P]
     lib.ia_status_string.restype = ctypes.c_char_p
@@ -112,6 +116,10 @@ def state_bytes(B, H, M, d_xi, d_v) -> int:
 
 def prefill_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
     return int(load_library().ia_prefill_workspace_bytes(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
+
+
+def prefill_launches(B, H, N, d_xi, d_v, M, dtype) -> int:
+    return int(load_library().ia_prefill_launches(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
 
 
 def fwd_bwd_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
@@ -186,6 +194,14 @@ def decode_step(q, k, v, delta, state, M, A=None, o=None, want_num_den=False, st
                             _ptr(state), _ptr(o), _ptr(num), _ptr(den), _stream(stream))
     _check(rc, "ia_decode_step")
     return {"o": o, "num": num, "den": den}
+
+
+def set_launch_events(begin=None, end=None):
+    """Bracket every later call's dominant kernel launch with two torch.cuda.Events
+    (profiling aid); call with no arguments to stop."""
+    b = ctypes.c_void_p(begin.cuda_event) if begin is not None else None
+    e = ctypes.c_void_p(end.cuda_event) if end is not None else None
+    _check(load_library().ia_set_launch_events(b, e), "ia_set_launch_events")
 
 
 def check_device_errors(stream=None):

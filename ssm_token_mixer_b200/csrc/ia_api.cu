@@ -54,7 +54,16 @@ bool use_tc(const ia_shape_t& s) {
 
 ia_status_t map_cuda(cudaError_t e) { return e == cudaSuccess ? IA_OK : IA_ERR_CUDA; }
 
+cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
+
 }  // namespace
+
+void mark_launch_begin(cudaStream_t st) {
+  if (g_ev_begin) cudaEventRecord(g_ev_begin, st);
+}
+void mark_launch_end(cudaStream_t st) {
+  if (g_ev_end) cudaEventRecord(g_ev_end, st);
+}
 
 int* device_error_ptr() {
   constexpr int kMaxDev = 64;
@@ -98,6 +107,12 @@ size_t ia_prefill_workspace_bytes(const ia_shape_t* s) {
   if (!valid_dims(s, true)) return 0;
   if (!use_tc(*s)) return 0;
   return tc_workspace_bytes(*s, tc_plan(*s, num_sms()));
+}
+
+int ia_prefill_launches(const ia_shape_t* s) {
+  if (!valid_dims(s, true)) return 0;
+  if (!use_tc(*s)) return 1;
+  return tc_plan(*s, num_sms()).nseg > 1 ? 4 : 2;   // tables [+ state-only pass + scan] + full pass
 }
 
 size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* s) {
@@ -166,6 +181,13 @@ ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, co
   if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
   return map_cuda(launch_decode(*s, q, k, v, delta, A, state, o, num, den,
                                 static_cast<cudaStream_t>(stream)));
+}
+
+ia_status_t ia_set_launch_events(void* begin, void* end) {
+  if ((begin == nullptr) != (end == nullptr)) return IA_ERR_INVALID_ARG;
+  g_ev_begin = static_cast<cudaEvent_t>(begin);
+  g_ev_end = static_cast<cudaEvent_t>(end);
+  return IA_OK;
 }
 
 ia_status_t ia_check_device_errors(void* stream) {

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   cg::cluster_group cluster = cg::this_cluster();
   const int g = static_cast<int>(cluster.block_rank());
   const int G = static_cast<int>(cluster.num_blocks());
-  const long long bh = blockIdx.y;
+  const long long bh = blockIdx.x / G;
   const int h = static_cast<int>(bh % H);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = g * MG;
@@ -165,7 +165,7 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G, static_cast<unsigned>(BH), 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(G * BH), 1, 1);
   cfg.blockDim = dim3(kDecThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -176,9 +176,12 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, MG, static_cast<const T*>(q),
-                            static_cast<const T*>(k), static_cast<const T*>(v), delta, A,
-                            static_cast<float2*>(state), o, num, den, BH);
+  mark_launch_begin(st);
+  e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, MG, static_cast<const T*>(q),
+                         static_cast<const T*>(k), static_cast<const T*>(v), delta, A,
+                         static_cast<float2*>(state), o, num, den, BH);
+  mark_launch_end(st);
+  return e;
 }
 
 }  // namespace

@@ -46,6 +46,10 @@ cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, con
                           const float* delta, const float* A, void* state, float* o, float* num,
                           float* den, cudaStream_t st);
 
+// Caller-registered events bracketing the dominant kernel launch (profiling).
+void mark_launch_begin(cudaStream_t st);
+void mark_launch_end(cudaStream_t st);
+
 // Device address of the library's error flag on the current device (looked
 // up once per device), or nullptr if the lookup fails.
 int* device_error_ptr();

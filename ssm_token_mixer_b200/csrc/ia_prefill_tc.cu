@@ -38,6 +38,7 @@
 // pass recomputes every segment from its carried-in state -- the two
 // parallel passes around a sequential carry pass of the summary's sec. A.2.
 #include <cmath>
+#include <cstdlib>
 
 #include "ia_device.cuh"
 #include "ia_internal.h"
@@ -578,8 +579,11 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
   auto k3 = tc_prefill_kernel<DX, DV, true>;
   e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
+  mark_launch_begin(st);
   k3<<<static_cast<unsigned>(args.BH * p.nseg), NTHR, K::SMEM, st>>>(args);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  mark_launch_end(st);
+  return e;
 }
 
 }  // namespace
@@ -593,16 +597,27 @@ bool tc_prefill_supported(const ia_shape_t& s) {
 TcPlan tc_plan(const ia_shape_t& s, int num_sms) {
   const long long BH = static_cast<long long>(s.B) * s.H;
   const int nch = (s.N + C - 1) / C;
-  const double alpha = 0.35;   // cost of a state-only chunk relative to a full one
+  // Forced segment count (tuning and tests): IA_PREFILL_SEGMENTS=n.
+  if (const char* env = std::getenv("IA_PREFILL_SEGMENTS")) {
+    const int n = std::atoi(env);
+    if (n >= 1 && n <= nch) {
+      const int L = (nch + n - 1) / n;
+      return TcPlan{(nch + L - 1) / L, L};
+    }
+  }
+  // Cost in units of one full chunk pass: waves x (chunks per CTA + per-CTA
+  // prologue/epilogue), a state-only chunk costing alpha, plus the scan.
+  const double alpha = 0.35, cta_overhead = 1.0, scan = 1.0;
+  const int min_len = 4;   // shorter segments spend more on state round trips than they save
   TcPlan best{1, nch};
   double best_t = 1e300;
   for (int nseg = 1; nseg <= 32 && nseg <= nch; ++nseg) {
     const int L = (nch + nseg - 1) / nseg;
-    const int used = (nch + L - 1) / L;   // segments actually holding chunks
-    if (used != nseg) continue;
+    if ((nch + L - 1) / L != nseg) continue;
+    if (nseg > 1 && L < min_len) continue;
     const double w1 = nseg > 1 ? std::ceil(static_cast<double>(BH * (nseg - 1)) / num_sms) : 0.0;
     const double w3 = std::ceil(static_cast<double>(BH * nseg) / num_sms);
-    const double t = w1 * L * alpha + w3 * L + (nseg > 1 ? 1.0 : 0.0);
+    const double t = w1 * (L * alpha + cta_overhead) + w3 * (L + cta_overhead) + (nseg > 1 ? scan : 0.0);
     if (t < best_t - 1e-9) {
       best_t = t;
       best = TcPlan{nseg, L};

@@ -535,11 +535,14 @@ static cudaError_t seq_fwd_impl(const ia_shape_t& s, const void* q, const void* 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   long long BH = static_cast<long long>(s.B) * s.H;
+  mark_launch_begin(st);
   kern<<<static_cast<unsigned>(BH), 256, smem, st>>>(
       s.H, s.N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
       static_cast<const T*>(v), delta, A, static_cast<const float2*>(state_in), o, num, den,
       static_cast<float2*>(state_out), BH);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  mark_launch_end(st);
+  return e;
 }
 
 cudaError_t launch_seq_fwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
@@ -574,11 +577,14 @@ static cudaError_t seq_bwd_impl(const ia_shape_t& s, const void* q, const void* 
   e = cudaMemsetAsync(dDelta, 0, sizeof(float) * s.H, st);
   if (e != cudaSuccess) return e;
   long long BH = static_cast<long long>(s.B) * s.H;
+  mark_launch_begin(st);
   kern<<<static_cast<unsigned>(BH), 256, smem, st>>>(
       s.H, s.N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
       static_cast<const T*>(v), static_cast<const T*>(dO), delta, A, o, dq, dk, dv, dDelta,
       static_cast<float2*>(ws), static_cast<long long>(seq_bwd_ws_per_bh(s.N, s.d_xi, s.d_v, s.M)));
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  mark_launch_end(st);
+  return e;
 }
 
 cudaError_t launch_seq_bwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
