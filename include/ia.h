@@ -100,6 +100,30 @@ IA_API ia_status_t ia_prefill_fwd(const ia_shape_t* shape, const void* q, const 
                            void* stream);
 
 /*
+ * ia_prefill_fwd for callers that cannot allocate device memory, for example
+ * a plugin inside another framework whose memory pool owns the device, or a
+ * serving loop that must never reach cudaMalloc/cudaFree because those calls
+ * can synchronise the device.  No counterpart in the paper: same arguments
+ * and results as ia_prefill_fwd, minus the workspace.
+ *   - Scratch lives in a fixed 2 MiB array compiled into the library, held by
+ *     every GPU that loads the library until the process exits.  It holds
+ *     the per-head tables of unsplit sequences: up to 97 heads.  More heads
+ *     return IA_ERR_WORKSPACE and launch nothing.
+ *   - Only the tensor-core shapes run here (bf16 inputs, M = 64, d_xi and d_v
+ *     in {64, 128}); other shapes return IA_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address;
+ *     make that first call before any stream capture.
+ *   - Every call shares the array and it keeps the last call's contents.
+ *     Calls that overlap on the GPU (different streams, unordered host
+ *     threads) race on it; the caller must serialise them.
+ *   - Never calls cudaMalloc, cudaFree or any other allocating routine.
+ */
+IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* shape, const void* q, const void* k,
+                                         const void* v, const float* delta, const float* A,
+                                         const void* state_in, float* o, float* num, float* den,
+                                         void* state_out, void* stream);
+
+/*
  * Training step of the layer from a zero state (paperlayer.ai summary
  * sec. A.3 and App. G: bf16 mixed-precision training).  Given the upstream
  * gradient dO [B,H,N,d_v] (input dtype), writes o, and the gradients

@@ -19,7 +19,7 @@ import os
 import torch
 
 __all__ = ["IAError", "load_library", "state_bytes", "prefill_workspace_bytes",
-           "fwd_bwd_workspace_bytes", "prefill_fwd", "fwd_bwd", "decode_step",
+           "fwd_bwd_workspace_bytes", "prefill_fwd", "prefill_fwd_static", "fwd_bwd", "decode_step",
            "check_device_errors", "set_launch_events", "library_path", "IA_F32", "IA_BF16"]
 
 IA_F32, IA_BF16 = 0, 1
@@ -65,6 +65,8 @@ def load_library():
     lib.ia_prefill_launches.argtypes = [S]
     lib.ia_prefill_fwd.restype = ctypes.c_int
     lib.ia_prefill_fwd.argtypes = [S] + [P] * 10 + [P, ctypes.c_size_t, P]
+    lib.ia_prefill_fwd_static.restype = ctypes.c_int
+    lib.ia_prefill_fwd_static.argtypes = [S] + [P] * 10 + [P]
     lib.ia_fwd_bwd.restype = ctypes.c_int
     lib.ia_fwd_bwd.argtypes = [S] + [P] * 11 + [P, ctypes.c_size_t, P]
     lib.ia_decode_step.restype = ctypes.c_int
@@ -155,6 +157,28 @@ def prefill_fwd(q, k, v, delta, M, A=None, state_in=None, want_num_den=False, wa
                             _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _ptr(ws),
                             ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream))
     _check(rc, "ia_prefill_fwd")
+    return {"o": o, "num": num, "den": den, "state": st}
+
+
+def prefill_fwd_static(q, k, v, delta, M, A=None, state_in=None, want_num_den=False,
+                       want_state=False, o=None, stream=None):
+    """prefill_fwd for callers that cannot allocate device memory: the library
+    keeps its scratch in a fixed per-GPU array instead of a workspace (see
+    ia_prefill_fwd_static in include/ia.h).  Output tensors are still the
+    caller's; pass `o` (and use want_* = False) to allocate nothing here."""
+    lib = load_library()
+    B, H, N, d_xi = q.shape
+    d_v = v.shape[-1]
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    dev = q.device
+    if o is None:
+        o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    num = torch.empty_like(o) if want_num_den else None
+    den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
+    st = torch.empty(lib.ia_state_bytes(ctypes.byref(shp)) // 4, dtype=torch.float32, device=dev) if want_state else None
+    rc = lib.ia_prefill_fwd_static(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
+                                   _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _stream(stream))
+    _check(rc, "ia_prefill_fwd_static")
     return {"o": o, "num": num, "den": den, "state": st}
 
 
