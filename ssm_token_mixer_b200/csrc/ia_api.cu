@@ -52,6 +52,11 @@ bool use_tc(const ia_shape_t& s) {
   return tc_prefill_supported(s);
 }
 
+bool use_tc_bwd(const ia_shape_t& s) {
+  if (env_set("IA_BWD_SIMT")) return false;       // debug switch: force the CUDA-core adjoint
+  return tc_bwd_supported(s);
+}
+
 ia_status_t map_cuda(cudaError_t e) { return e == cudaSuccess ? IA_OK : IA_ERR_CUDA; }
 
 cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
@@ -117,6 +122,7 @@ int ia_prefill_launches(const ia_shape_t* s) {
 
 size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* s) {
   if (!valid_dims(s, true)) return 0;
+  if (use_tc_bwd(*s)) return tc_fwd_bwd_workspace_bytes(*s, tc_plan(*s, num_sms()));
   return sizeof(float2) * static_cast<size_t>(s->B) * s->H *
              seq_bwd_ws_per_bh(s->N, s->d_xi, s->d_v, s->M) + 256;
 }
@@ -159,12 +165,16 @@ ia_status_t ia_fwd_bwd(const ia_shape_t* s, const void* q, const void* k, const 
   const void* ptrs[] = {q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
-  if (seq_bwd_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  const bool tc = use_tc_bwd(*s);
+  if (!tc && seq_bwd_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
   const size_t need = ia_fwd_bwd_workspace_bytes(s);
   if (!workspace || workspace_bytes < need) return IA_ERR_WORKSPACE;
   if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
-  return map_cuda(launch_seq_bwd(*s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace,
-                                 static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc)
+    return map_cuda(launch_tc_fwd_bwd(*s, tc_plan(*s, num_sms()), q, k, v, delta, A, dO, o, dq, dk,
+                                      dv, dDelta, workspace, st));
+  return map_cuda(launch_seq_bwd(*s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace, st));
 }
 
 ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, const void* v,
@@ -176,6 +186,8 @@ ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, co
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
   if ((s->d_xi & 1) || (s->d_v & 1)) return IA_ERR_UNSUPPORTED;   // 16-byte state vectors
+  if (s->d_xi > 256 || s->d_v > 256) return IA_ERR_UNSUPPORTED;     // one register pass per row
+  if (s->M > 128) return IA_ERR_UNSUPPORTED;                        // at most 8 CTAs x 16 modes
   const size_t smem = sizeof(float) * (2 * s->d_xi + 9 * s->d_v + 8) + 2 * sizeof(float2) * s->M + 16;
   if (smem > kMaxSmem) return IA_ERR_UNSUPPORTED;
   if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;

@@ -1,0 +1,674 @@
+// Reverse mode of the chunked IA layer on tcgen05 tensor cores (training
+// step: dq, dk, dv, dDelta) for bf16 inputs, M = 64 modes, d_xi = d_v = 64.
+//
+// The layer is the causal IA layer of 'Interdomain Attention: Beyond
+// Token-Level Key-Value Memory' (paperlayer.ai summary sec. 3.1-3.2, chunkwise
+// execution per sec. A.2; bf16 training per sec. A.3 and App. G).  The
+// backward differentiates the same chunk algorithm the forward runs, in the
+// real-row form (rows k = 2m re, 2m+1 im; E'' = E' split into rows; x = [xi(K)|V]):
+//
+//   forward per chunk:  R = lambda^C S_hat0;  a~ = S E'' + xi(Q) R_U^T;  X = s * a~
+//                       P = mask(X E''^T);  num = P V + X R_G;  den = P 1 + X R_eta
+//                       S_hat1 = R + E''^T x
+//   reverse per chunk (from dO and the adjoint dS1 of S_hat1, chunks last to first):
+//     dnum = dO/den, dden = -(dO.o)/den           dP = mask(dnum V^T + dden 1^T)
+//     dX^T = E''^T dP^T + R_G dnum^T + R_eta dden   da~ = s * dX
+//     dS = mask(da~ E''^T)
+//     dxi(Q) = dS xi(K) + da~ R_U      dxi(K) = dS^T xi(Q) + E'' dS1_U
+//     dV = P^T dnum + E'' dS1_G        dR = dS1 + [da~^T xi(Q) | X^T dnum | X^T dden]
+//     dS_hat0 = conj(lambda^C) dR
+//   Delta enters only through the per-head tables, so their adjoints are
+//   gathered over all chunks and contracted once with the tables' derivatives:
+//     dE''^T += da~^T S + X^T dP + dS1 x^T    (accumulated in TMEM)
+//     ds     += dX * a~,  dlambda^C += sum dR conj(S_hat0)
+//     d(b lambda^n)/dDelta = (lambda + n A b) lambda^n,  ds/dDelta = 2 Re(A)(i-c) s,
+//     d(lambda^C)/dDelta = C A lambda^C.
+// The forward pass (the prefill kernel) stores R and den for every chunk.
+//
+// TMEM columns: [0,128) adjoint of the state (dS1, then dR, then dS_hat0);
+// [128,192) dE''^T; [192,256) a~^T then dK; [256,320) dX^T then dV;
+// [320,384) S^T, P, dP, dS (M=64 layout); [384,448) dQ.
+#include <cmath>
+
+#include "ia_device.cuh"
+#include "ia_internal.h"
+#include "ia_tables.cuh"
+#include "ia_tc_common.cuh"
+
+namespace ia {
+namespace {
+
+using namespace tc;
+
+struct B {
+  static constexpr int DX = 64, DV = 64, F = 128;
+  static constexpr uint32_t T_ADJ = 0, T_EBAR = 128, T_A = 192, T_DK = 192, T_DX = 256,
+                            T_DV = 256, T_SP = 320, T_DQ = 384;
+  static constexpr uint32_t TILE64 = C * 64 * 2;     // 8 KB: [64 rows][64 cols] fp16
+  static constexpr uint32_t TILE128 = KR * 64 * 2;   // 16 KB: [128 rows][64 cols] fp16
+  static constexpr uint32_t STG_Q = 0;
+  static constexpr uint32_t STG_K = STG_Q + TILE64;
+  static constexpr uint32_t STG_V = STG_K + TILE64;
+  static constexpr uint32_t STG_G = STG_V + TILE64;
+  static constexpr uint32_t S_Q = STG_G + TILE64;
+  static constexpr uint32_t S_K = S_Q + TILE64;
+  static constexpr uint32_t S_V = S_K + TILE64;
+  static constexpr uint32_t S_E = S_V + TILE64;
+  static constexpr uint32_t S_S = S_E + TILE128;
+  static constexpr uint32_t S_X = S_S + TILE64;
+  static constexpr uint32_t S_P = S_X + TILE128;
+  static constexpr uint32_t S_DP = S_P + TILE64;
+  static constexpr uint32_t S_DA = S_DP + TILE64;
+  static constexpr uint32_t S_DS = S_DA + TILE128;
+  static constexpr uint32_t S_DN = S_DS + TILE64;
+  static constexpr uint32_t S_RU = S_DN + TILE64;
+  static constexpr uint32_t S_RG = S_RU + TILE128;
+  static constexpr uint32_t S_DS1 = S_RG + TILE128;          // [128][F] fp16
+  static constexpr uint32_t S_DD = S_DS1 + KR * F * 2;       // dden [64] fp32
+  static constexpr uint32_t S_RED = S_DD + C * 4;            // dR_eta halves [2][128] fp32
+  static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;
+  static constexpr uint32_t S_TMEMH = S_BAR + 32;
+  static constexpr uint32_t SMEM = S_TMEMH + 16;
+};
+
+struct BwdArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* dO;
+  const float* o;
+  const float* den;
+  const float* A;
+  const HeadTables* tabs;
+  const float* R;    // [BH][nch][128][F]
+  const float* Re;   // [BH][nch][128]
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dDelta;
+  int* err;
+  int H, N;
+  long long BH;
+};
+
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  return make_uint4(pack_half2(x[0], x[1]), pack_half2(x[2], x[3]), pack_half2(x[4], x[5]),
+                    pack_half2(x[6], x[7]));
+}
+
+__global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
+  constexpr int DX = B::DX, DV = B::DV, F = B::F;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
+  const long long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % a.H);
+  const HeadTables* T = a.tabs + h;
+  const int nch = (a.N + C - 1) / C;
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + B::S_BAR);
+  uint64_t* bar_mma = bar_tma + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + B::S_TMEMH);
+  float* sDD = reinterpret_cast<float*>(smem + B::S_DD);
+  float* sRED = reinterpret_cast<float*>(smem + B::S_RED);
+  const uint32_t sb = smem_u32(smem);
+
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_tma, 1);
+    mbar_init(bar_mma, 1);
+    fence_barrier_init();
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(T->E);
+    uint4* dst = reinterpret_cast<uint4*>(smem + B::S_E);
+    for (int i = tid; i < static_cast<int>(B::TILE128 / 16); i += NTHR) dst[i] = src[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int k = 32 * quad + lane;   // state row: mode m, component comp
+  const int m = k >> 1, comp = k & 1;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+  const float2 lamC = T->lamC[m];
+  const float ReA = a.A ? a.A[2 * m] : -0.5f;
+  const float ImA = a.A ? a.A[2 * m + 1] : static_cast<float>(3.14159265358979323846 * m);
+  const float r2 = T->r2[m];
+  const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
+  const float sgn = comp ? 1.f : -1.f;
+  // sum over j of d(E'[j,m])/dDelta = lambda^(c-j) (lambda + (c-j) A b), this row's component
+  float dEsum_c;
+  {
+    const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
+    const double Ar = ReA, Ai = ImA;
+    double sr = 0.0, si = 0.0;
+    for (int j = 0; j < C; ++j) {
+      const double n = C / 2 - j;
+      const double e = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
+      double sn, cs;
+      sincos(ph, &sn, &cs);
+      const double pr = e * cs, pi = e * sn;
+      const double fr = lr + n * (Ar * br - Ai * bi), fi = li + n * (Ar * bi + Ai * br);
+      sr += pr * fr - pi * fi;
+      si += pr * fi + pi * fr;
+    }
+    dEsum_c = static_cast<float>(comp ? si : sr);
+  }
+
+  // zero the state adjoint and the table adjoint
+  {
+    uint32_t z[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) z[e] = 0u;
+    for (int cb = 0; cb < F / 2; cb += 16) tmem_st16(trow + B::T_ADJ + half * (F / 2) + cb, z);
+    for (int cb = 0; cb < 32; cb += 16) tmem_st16(trow + B::T_EBAR + half * 32 + cb, z);
+    tmem_st_wait();
+  }
+  float de_c = 0.f;     // adjoint of the eta channel of the chunk-end state (this row)
+  float dD = 0.f;       // this thread's share of dDelta
+
+  auto issue_load = [&](int ch) {
+    const int n0 = ch * C;
+    const int nv = min(C, a.N - n0);
+    const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
+    mbar_arrive_expect_tx(bar_tma, 2 * bq + 2 * bv);
+    const long long row = bh * a.N + n0;
+    bulk_g2s(smem + B::STG_Q, a.q + row * DX, bq, bar_tma);
+    bulk_g2s(smem + B::STG_K, a.k + row * DX, bq, bar_tma);
+    bulk_g2s(smem + B::STG_V, a.v + row * DV, bv, bar_tma);
+    bulk_g2s(smem + B::STG_G, a.dO + row * DV, bv, bar_tma);
+  };
+  if (tid == 0) issue_load(nch - 1);
+  bool tma_pending = true;
+  uint32_t ph_tma = 0, ph_mma = 0;
+  bool aborted = false;
+  auto mma_sync = [&]() -> bool {
+    bool ok = mbar_wait(bar_mma, ph_mma, a.err);
+    ph_mma ^= 1u;
+    tc_fence_after();
+    return !__syncthreads_or(!ok);
+  };
+  auto to_tc = [&]() {
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  };
+
+  for (int ch = nch - 1; ch >= 0; --ch) {
+    const int n0 = ch * C;
+    const int nv = min(C, a.N - n0);
+    {
+      bool ok = mbar_wait(bar_tma, ph_tma, a.err);
+      ph_tma ^= 1u;
+      if (__syncthreads_or(!ok)) { aborted = true; break; }
+      tma_pending = false;
+    }
+    // ---- P0: operands of this chunk
+    convert_tile<DX, true>(smem + B::STG_Q, smem + B::S_Q, nv, warp, lane);
+    convert_tile<DX, true>(smem + B::STG_K, smem + B::S_K, nv, warp, lane);
+    convert_tile<DV, false>(smem + B::STG_V, smem + B::S_V, nv, warp, lane);
+    {  // dnum = dO / den (fp16 tile [i][f]), dden = -(dO . o) / den
+      const int i = tid >> 2, part = tid & 3;
+      const long long row = bh * a.N + n0 + i;
+      float g[16];
+      float dot = 0.f, rden = 0.f;
+      if (i < nv) {
+        rden = 1.0f / a.den[row];
+        const __nv_bfloat162* gs =
+            reinterpret_cast<const __nv_bfloat162*>(smem + B::STG_G + i * DV * 2 + part * 32);
+        const float4* op = reinterpret_cast<const float4*>(a.o + row * DV + part * 16);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float2 x = __bfloat1622float2(gs[e]);
+          g[2 * e] = x.x;
+          g[2 * e + 1] = x.y;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 ov = op[e];
+          dot = fmaf(g[4 * e], ov.x, fmaf(g[4 * e + 1], ov.y, fmaf(g[4 * e + 2], ov.z, fmaf(g[4 * e + 3], ov.w, dot))));
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) g[e] *= rden;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) g[e] = 0.f;
+      }
+      dot += __shfl_xor_sync(kFull, dot, 1);
+      dot += __shfl_xor_sync(kFull, dot, 2);
+      *reinterpret_cast<uint4*>(smem + B::S_DN + tile_off(i, part * 16, DV * 16)) = pack8(g);
+      *reinterpret_cast<uint4*>(smem + B::S_DN + tile_off(i, part * 16 + 8, DV * 16)) = pack8(g + 8);
+      if (part == 0) sDD[i] = i < nv ? -dot * rden : 0.f;
+    }
+    __syncthreads();   // staging consumed
+    if (tid == 0 && ch > 0) issue_load(ch - 1);
+    tma_pending = ch > 0;
+    const float* Rrow = a.R + ((bh * nch + ch) * KR + k) * F;
+    const float Reta = a.Re[(bh * nch + ch) * KR + k];
+    {  // R -> fp16 operands R_U (half 0) / R_G (half 1); dS1 -> fp16
+      const float4* src = reinterpret_cast<const float4*>(Rrow + half * 64);
+      uint8_t* dst = smem + (half == 0 ? B::S_RU : B::S_RG);
+#pragma unroll
+      for (int g8 = 0; g8 < 8; ++g8) {
+        const float4 x0 = src[2 * g8], x1 = src[2 * g8 + 1];
+        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        *reinterpret_cast<uint4*>(dst + tile_off(k, 8 * g8, 64 * 16)) = pack8(xs);
+      }
+      for (int cb = 0; cb < 64; cb += 16) {
+        const int col0 = half * 64 + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_ADJ + col0, r);
+        tmem_ld_wait16(r);
+        float xs[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) xs[e] = __uint_as_float(r[e]);
+        *reinterpret_cast<uint4*>(smem + B::S_DS1 + tile_off(k, col0, F * 16)) = pack8(xs);
+        *reinterpret_cast<uint4*>(smem + B::S_DS1 + tile_off(k, col0 + 8, F * 16)) = pack8(xs + 8);
+      }
+    }
+    to_tc();
+    if (tid == 0) {   // F1: S^T = xi(K) xi(Q)^T
+      tc_fence_after();
+      gemm(tmem + B::T_SP, sb + B::S_K, kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), sb + B::S_Q,
+           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(64, 64, 0, 0), DX / 16, false);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E1: masked S^T -> [j][i]
+      const int j = 16 * quad + lane;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int i0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + i0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            xs[e] = (j < nv && i0 + e >= j) ? __uint_as_float(r[e]) : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
+    }
+    to_tc();
+    if (tid == 0) {   // F2: a~^T = E''^T S^T + R_U xi(Q)^T
+      tc_fence_after();
+      gemm(tmem + B::T_A, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S,
+           mn_lbo(64), mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, false);
+      gemm(tmem + B::T_A, sb + B::S_RU, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_Q,
+           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16, true);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E2: X = s a~  (rows k), dR_eta partial = sum_i X dden_i
+      float s = s_start, acc = 0.f;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int i0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_A + i0, r);
+        tmem_ld_wait16(r);
+        float xs[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          xs[e] = __uint_as_float(r[e]) * s;
+          acc = fmaf(xs[e], sDD[i0 + e], acc);
+          s *= r2;
+        }
+        *reinterpret_cast<uint4*>(smem + B::S_X + tile_off(k, i0, 1024)) = pack8(xs);
+        *reinterpret_cast<uint4*>(smem + B::S_X + tile_off(k, i0 + 8, 1024)) = pack8(xs + 8);
+      }
+      sRED[half * KR + k] = acc;
+    }
+    to_tc();
+    if (tid == 0) {   // F4: P = X E''^T
+      tc_fence_after();
+      gemm(tmem + B::T_SP, sb + B::S_X, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_E, mn_lbo(64),
+           mn_sbo(), mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E3: masked P -> [i][j]
+      const int i = 16 * quad + lane;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
+    }
+    to_tc();
+    if (tid == 0) {   // B1: dP = dnum V^T
+      tc_fence_after();
+      gemm(tmem + B::T_SP, sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), sb + B::S_V,
+           kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(64, 64, 0, 0), DV / 16, false);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E_dP: + dden_i, mask j <= i -> [i][j]
+      const int i = 16 * quad + lane;
+      const float ddi = lane < 16 ? sDD[i] : 0.f;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) + ddi : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
+    }
+    to_tc();
+    if (tid == 0) {   // B2: dX^T = E''^T dP^T + R_G dnum^T
+      tc_fence_after();
+      gemm(tmem + B::T_DX, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP,
+           kmaj_lbo(), kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, false);
+      gemm(tmem + B::T_DX, sb + B::S_RG, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DN,
+           kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16, true);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E_dX: dX += R_eta dden; da~ = s dX; dDelta += dX a~ ds/dDelta
+      float s = s_start;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int i0 = 32 * half + cb;
+        uint32_t rx[16], ra[16];
+        tmem_ld16(trow + B::T_DX + i0, rx);
+        tmem_ld_wait16(rx);
+        tmem_ld16(trow + B::T_A + i0, ra);
+        tmem_ld_wait16(ra);
+        float xs[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = i0 + e;
+          const float dx = fmaf(Reta, sDD[i], __uint_as_float(rx[e]));
+          xs[e] = dx * s;
+          dD = fmaf(dx * __uint_as_float(ra[e]), 2.f * ReA * static_cast<float>(i - C / 2) * s, dD);
+          s *= r2;
+        }
+        *reinterpret_cast<uint4*>(smem + B::S_DA + tile_off(k, i0, 1024)) = pack8(xs);
+        *reinterpret_cast<uint4*>(smem + B::S_DA + tile_off(k, i0 + 8, 1024)) = pack8(xs + 8);
+      }
+    }
+    to_tc();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sDA = sb + B::S_DA, sX = sb + B::S_X, sE = sb + B::S_E;
+      // B3: dS = da~ E''^T
+      gemm(tmem + B::T_SP, sDA, mn_lbo(64), mn_sbo(), mn_step(64), sE, mn_lbo(64), mn_sbo(),
+           mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
+      // B4, B5: dR += [da~^T xi(Q) | X^T dnum]
+      gemm(tmem + B::T_ADJ, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_Q, mn_lbo(DX),
+           mn_sbo(), mn_step(DX), idesc_f16(128, DX, 0, 1), C / 16, true);
+      gemm(tmem + B::T_ADJ + DX, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DN,
+           mn_lbo(DV), mn_sbo(), mn_step(DV), idesc_f16(128, DV, 0, 1), C / 16, true);
+      // table adjoint: dE''^T += da~^T S + X^T dP + dS1 x^T
+      gemm(tmem + B::T_EBAR, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S, kmaj_lbo(),
+           kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, true);
+      gemm(tmem + B::T_EBAR, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP, mn_lbo(64),
+           mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, true);
+      gemm(tmem + B::T_EBAR, sb + B::S_DS1, kmaj_lbo(), kmaj_sbo(F), kmaj_step(), sb + B::S_K,
+           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16, true);
+      gemm(tmem + B::T_EBAR, sb + B::S_DS1 + (DX / 8) * 128, kmaj_lbo(), kmaj_sbo(F), kmaj_step(),
+           sb + B::S_V, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16,
+           true);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // E_dS: mask (j <= i, j < nv) -> [i][j]
+      const int i = 16 * quad + lane;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            xs[e] = (j0 + e <= i && j0 + e < nv) ? __uint_as_float(r[e]) : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
+    }
+    to_tc();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sDS = sb + B::S_DS, sDA = sb + B::S_DA, sE = sb + B::S_E, sDS1 = sb + B::S_DS1;
+      // dQ = dS xi(K) + da~ R_U
+      gemm(tmem + B::T_DQ, sDS, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_K, mn_lbo(DX),
+           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 0, 1), C / 16, false);
+      gemm(tmem + B::T_DQ, sDA, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_RU, mn_lbo(64),
+           mn_sbo(), mn_step(64), idesc_f16(64, DX, 1, 1), KR / 16, true);
+      // dK = dS^T xi(Q) + E'' dS1_U
+      gemm(tmem + B::T_DK, sDS, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_Q, mn_lbo(DX),
+           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 1, 1), C / 16, false);
+      gemm(tmem + B::T_DK, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1, mn_lbo(F), mn_sbo(),
+           mn_step(F), idesc_f16(64, DX, 1, 1), KR / 16, true);
+      // dV = P^T dnum + E'' dS1_G
+      gemm(tmem + B::T_DV, sb + B::S_P, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_DN, mn_lbo(DV),
+           mn_sbo(), mn_step(DV), idesc_f16(64, DV, 1, 1), C / 16, false);
+      gemm(tmem + B::T_DV, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1 + (DX / 8) * 128, mn_lbo(F),
+           mn_sbo(), mn_step(F), idesc_f16(64, DV, 1, 1), KR / 16, true);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1)
+      const int i = 16 * quad + lane;
+      const bool valid = lane < 16 && i < nv;
+      const long long row = bh * a.N + n0 + i;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int f0 = 32 * half + cb;
+        uint32_t rq[16], rk[16], rv[16];
+        tmem_ld16(trow + B::T_DQ + f0, rq);
+        tmem_ld_wait16(rq);
+        tmem_ld16(trow + B::T_DK + f0, rk);
+        tmem_ld_wait16(rk);
+        tmem_ld16(trow + B::T_DV + f0, rv);
+        tmem_ld_wait16(rv);
+        if (valid) {
+          const __half* xq = reinterpret_cast<const __half*>(smem + B::S_Q);
+          const __half* xk = reinterpret_cast<const __half*>(smem + B::S_K);
+          float4* pq = reinterpret_cast<float4*>(a.dq + row * DX + f0);
+          float4* pk = reinterpret_cast<float4*>(a.dk + row * DX + f0);
+          float4* pv = reinterpret_cast<float4*>(a.dv + row * DV + f0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float oq[4], ok[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int f = f0 + 4 * g + e;
+              const float fq = __half2float(xq[tile_off(i, f, DX * 16) / 2]);
+              const float fk = __half2float(xk[tile_off(i, f, DX * 16) / 2]);
+              oq[e] = __uint_as_float(rq[4 * g + e]) * fminf(fq, 1.f);
+              ok[e] = __uint_as_float(rk[4 * g + e]) * fminf(fk, 1.f);
+            }
+            pq[g] = make_float4(oq[0], oq[1], oq[2], oq[3]);
+            pk[g] = make_float4(ok[0], ok[1], ok[2], ok[3]);
+            pv[g] = make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
+                                __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
+          }
+        }
+      }
+    }
+    {  // adjoint carry: dS_hat0 = conj(lambda^C) dR;  dDelta += C Re(conj(sum dR conj(R)) A)
+      for (int cb = 0; cb < 64; cb += 16) {
+        const int col0 = half * 64 + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_ADJ + col0, r);
+        tmem_ld_wait16(r);
+        const float4* rp = reinterpret_cast<const float4*>(Rrow + col0);
+        float rv[16];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 x = rp[g];
+          rv[4 * g] = x.x; rv[4 * g + 1] = x.y; rv[4 * g + 2] = x.z; rv[4 * g + 3] = x.w;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x = __uint_as_float(r[e]);
+          const float y = __shfl_xor_sync(kFull, x, 1);
+          const float rpart = __shfl_xor_sync(kFull, rv[e], 1);
+          dD = fmaf(static_cast<float>(C), fmaf(ReA, x * rv[e], ImA * sgn * x * rpart), dD);
+          w[e] = __float_as_uint(fmaf(lamC.x, x, -sgn * lamC.y * y));
+        }
+        tmem_st16(trow + B::T_ADJ + col0, w);
+      }
+      tmem_st_wait();
+      // eta channel (each row once: half 0 counts the Delta terms)
+      const float dRe = de_c + sRED[k] + sRED[KR + k];
+      const float y = __shfl_xor_sync(kFull, dRe, 1);
+      const float Rp = __shfl_xor_sync(kFull, Reta, 1);
+      float dEpart = dEsum_c;
+      if (nv < C) {   // ragged chunk: only the valid keys carry the constant channel
+        const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
+        double sr = 0.0, si = 0.0;
+        for (int j = 0; j < nv; ++j) {
+          const double n = C / 2 - j;
+          const double e = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
+          double sn, cs;
+          sincos(ph, &sn, &cs);
+          const double pr = e * cs, pi = e * sn;
+          const double fr = lr + n * (ReA * br - ImA * bi), fi = li + n * (ReA * bi + ImA * br);
+          sr += pr * fr - pi * fi;
+          si += pr * fi + pi * fr;
+        }
+        dEpart = static_cast<float>(comp ? si : sr);
+      }
+      if (half == 0) {
+        dD = fmaf(static_cast<float>(C), fmaf(ReA, dRe * Reta, ImA * sgn * dRe * Rp), dD);
+        dD = fmaf(de_c, dEpart, dD);
+      }
+      de_c = fmaf(lamC.x, dRe, -sgn * lamC.y * y);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (!aborted) {
+    // contract the table adjoint with d(E'')/dDelta
+    const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
+#pragma unroll
+    for (int cb = 0; cb < 32; cb += 16) {
+      const int j0 = 32 * half + cb;
+      uint32_t r[16];
+      tmem_ld16(trow + B::T_EBAR + j0, r);
+      tmem_ld_wait16(r);
+      for (int e = 0; e < 16; ++e) {
+        const double n = C / 2 - (j0 + e);
+        const double ex = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
+        double sn, cs;
+        sincos(ph, &sn, &cs);
+        const double pr = ex * cs, pi = ex * sn;
+        const double fr = lr + n * (ReA * br - ImA * bi), fi = li + n * (ReA * bi + ImA * br);
+        const double dE = comp ? pr * fi + pi * fr : pr * fr - pi * fi;
+        dD = fmaf(__uint_as_float(r[e]), static_cast<float>(dE), dD);
+      }
+    }
+    // block reduction -> one atomic per CTA
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dD += __shfl_xor_sync(kFull, dD, off);
+    __syncthreads();
+    if (lane == 0) sRED[warp] = dD;
+    __syncthreads();
+    if (tid == 0) {
+      float s = 0.f;
+      for (int w = 0; w < NTHR / 32; ++w) s += sRED[w];
+      atomicAdd(a.dDelta + h, s);
+    }
+  } else if (tma_pending) {
+    mbar_wait(bar_tma, ph_tma, a.err);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const ia_shape_t& s) {
+  return s.in_dtype == IA_BF16 && s.M == kModesTC && s.d_xi == 64 && s.d_v == 64;
+}
+
+size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t nch = (s.N + C - 1) / C;
+  size_t bytes = tc_workspace_bytes(s, p);
+  bytes = (bytes + 255) & ~static_cast<size_t>(255);
+  bytes += BH * nch * KR * (s.d_xi + s.d_v) * sizeof(float);   // R per chunk
+  bytes += BH * nch * KR * sizeof(float);                      // R_eta per chunk
+  bytes += BH * s.N * sizeof(float) + 256;                     // den
+  return bytes + 256;
+}
+
+cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
+                              const void* v, const float* delta, const float* A, const void* dO,
+                              float* o, float* dq, float* dk, float* dv, float* dDelta, void* ws,
+                              cudaStream_t st) {
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t nch = (s.N + C - 1) / C;
+  uint8_t* base = reinterpret_cast<uint8_t*>(tc_tables(ws));
+  size_t off = (tc_workspace_bytes(s, p) + 255) & ~static_cast<size_t>(255);
+  float* dumpR = reinterpret_cast<float*>(base + off);
+  float* dumpRe = dumpR + BH * nch * KR * (s.d_xi + s.d_v);
+  float* den = dumpRe + BH * nch * KR;
+  den = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(den) + 255) & ~static_cast<uintptr_t>(255));
+  cudaError_t e = launch_tc_prefill(s, p, q, k, v, delta, A, nullptr, o, nullptr, den, nullptr, ws,
+                                    st, dumpR, dumpRe);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(dDelta, 0, sizeof(float) * s.H, st);
+  if (e != cudaSuccess) return e;
+  BwdArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.dO = static_cast<const __nv_bfloat16*>(dO);
+  a.o = o;
+  a.den = den;
+  a.A = A;
+  a.tabs = tc_tables(ws);
+  a.R = dumpR;
+  a.Re = dumpRe;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dDelta = dDelta;
+  a.err = device_error_ptr();
+  if (!a.err) return cudaErrorInvalidSymbol;
+  a.H = s.H;
+  a.N = s.N;
+  a.BH = static_cast<long long>(BH);
+  e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B::SMEM);
+  if (e != cudaSuccess) return e;
+  mark_launch_begin(st);
+  tc_bwd_kernel<<<static_cast<unsigned>(BH), NTHR, B::SMEM, st>>>(a);
+  e = cudaGetLastError();
+  mark_launch_end(st);
+  return e;
+}
+
+}  // namespace ia

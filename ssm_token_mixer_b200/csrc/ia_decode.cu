@@ -21,6 +21,8 @@ namespace ia {
 namespace {
 
 constexpr int kDecThreads = 256;
+constexpr int kVecPerLane = 4;   // rows up to 256 complex entries (d <= 256)
+constexpr int kModesPerWarp = 2;  // up to 16 modes per CTA
 
 template <typename T>
 __device__ __forceinline__ float ldx(const T* p);
@@ -56,6 +58,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   const int h = static_cast<int>(bh % H);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = g * MG;
+  const int nu = DX / 2, ng = DV / 2;   // 16-byte vectors (two complex entries) per row
+
+  float2* Ub = state + bh * M * DX;
+  float2* Gb = state + BH * M * DX + bh * M * DV;
+  float2* Eb = state + BH * M * (DX + DV) + bh * M;
+
+  // Issue every state load of this warp's modes first, so that HBM latency
+  // overlaps the parameter and feature set-up below.
+  float4 uv[kModesPerWarp][kVecPerLane], gv[kModesPerWarp][kVecPerLane];
+  float2 ev[kModesPerWarp];
+#pragma unroll
+  for (int r = 0; r < kModesPerWarp; ++r) {
+    const int mi = warp + 8 * r, m = m0 + mi;
+    const bool ok = mi < MG && m < M;
+    const float4* Ur = reinterpret_cast<const float4*>(Ub + static_cast<long long>(m) * DX);
+    const float4* Gr = reinterpret_cast<const float4*>(Gb + static_cast<long long>(m) * DV);
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (ok && p < nu) uv[r][i] = Ur[p];
+      if (ok && p < ng) gv[r][i] = Gr[p];
+    }
+    ev[r] = (ok && lane == 0) ? Eb[m] : make_float2(0.f, 0.f);
+  }
 
   for (int f = tid; f < DX; f += kDecThreads) {
     fq[f] = xi_acc(ldx(q + bh * DX + f));
@@ -76,50 +102,56 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   for (int i = tid; i < 8 * DV + 8; i += kDecThreads) part[i] = 0.f;
   __syncthreads();
 
-  float2* Ub = state + bh * M * DX;
-  float2* Gb = state + BH * M * DX + bh * M * DV;
-  float2* Eb = state + BH * M * (DX + DV) + bh * M;
   float* mypart = part + warp * DV;
   float dpart = 0.f;
-
-  for (int mi = warp; mi < MG && m0 + mi < M; mi += kDecThreads / 32) {
-    const int m = m0 + mi;
+#pragma unroll
+  for (int r = 0; r < kModesPerWarp; ++r) {
+    const int mi = warp + 8 * r, m = m0 + mi;
+    if (mi >= MG || m >= M) break;
     const float2 L = lamb[mi], Bm = bb[mi];
     float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
     float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
     float ar = 0.f, ai = 0.f;
-    for (int p = lane; p < DX / 2; p += 32) {
-      float4 u = Ur[p];
-      const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
-      float4 w;
-      w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
-      w.y = fmaf(L.x, u.y, fmaf(L.y, u.x, Bm.y * x0));
-      w.z = fmaf(L.x, u.z, fmaf(-L.y, u.w, Bm.x * x1));
-      w.w = fmaf(L.x, u.w, fmaf(L.y, u.z, Bm.y * x1));
-      Ur[p] = w;
-      ar = fmaf(w.x, fq[2 * p], fmaf(w.z, fq[2 * p + 1], ar));
-      ai = fmaf(w.y, fq[2 * p], fmaf(w.w, fq[2 * p + 1], ai));
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (p < nu) {
+        const float4 u = uv[r][i];
+        const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
+        float4 w;
+        w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
+        w.y = fmaf(L.x, u.y, fmaf(L.y, u.x, Bm.y * x0));
+        w.z = fmaf(L.x, u.z, fmaf(-L.y, u.w, Bm.x * x1));
+        w.w = fmaf(L.x, u.w, fmaf(L.y, u.z, Bm.y * x1));
+        Ur[p] = w;
+        ar = fmaf(w.x, fq[2 * p], fmaf(w.z, fq[2 * p + 1], ar));
+        ai = fmaf(w.y, fq[2 * p], fmaf(w.w, fq[2 * p + 1], ai));
+      }
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       ar += __shfl_xor_sync(0xffffffffu, ar, off);
       ai += __shfl_xor_sync(0xffffffffu, ai, off);
     }
-    for (int p = lane; p < DV / 2; p += 32) {
-      float4 gv = Gr[p];
-      const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
-      float4 w;
-      w.x = fmaf(L.x, gv.x, fmaf(-L.y, gv.y, Bm.x * x0));
-      w.y = fmaf(L.x, gv.y, fmaf(L.y, gv.x, Bm.y * x0));
-      w.z = fmaf(L.x, gv.z, fmaf(-L.y, gv.w, Bm.x * x1));
-      w.w = fmaf(L.x, gv.w, fmaf(L.y, gv.z, Bm.y * x1));
-      Gr[p] = w;
-      mypart[2 * p] += fmaf(ar, w.x, ai * w.y);       // Re(conj(a) Gamma)
-      mypart[2 * p + 1] += fmaf(ar, w.z, ai * w.w);
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (p < ng) {
+        const float4 gq = gv[r][i];
+        const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
+        float4 w;
+        w.x = fmaf(L.x, gq.x, fmaf(-L.y, gq.y, Bm.x * x0));
+        w.y = fmaf(L.x, gq.y, fmaf(L.y, gq.x, Bm.y * x0));
+        w.z = fmaf(L.x, gq.z, fmaf(-L.y, gq.w, Bm.x * x1));
+        w.w = fmaf(L.x, gq.w, fmaf(L.y, gq.z, Bm.y * x1));
+        Gr[p] = w;
+        mypart[2 * p] += fmaf(ar, w.x, ai * w.y);       // Re(conj(a) Gamma)
+        mypart[2 * p + 1] += fmaf(ar, w.z, ai * w.w);
+      }
     }
     if (lane == 0) {
-      float2 e = Eb[m];
-      float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
+      const float2 e = ev[r];
+      const float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
       Eb[m] = w;
       dpart += fmaf(ar, w.x, ai * w.y);
     }
@@ -156,8 +188,8 @@ template <typename T>
 cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const void* v,
                         const float* delta, const float* A, void* state, float* o, float* num,
                         float* den, cudaStream_t st) {
-  int G = (s.M + 15) / 16;
-  if (G > 8) G = 8;
+  // 16 modes (two per warp) per CTA, up to 8 CTAs per cluster
+  const int G = (s.M + 15) / 16;
   const int MG = (s.M + G - 1) / G;
   const long long BH = static_cast<long long>(s.B) * s.H;
   const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + 8 * s.d_v + 8) + sizeof(float2) * 2 * MG + 16;

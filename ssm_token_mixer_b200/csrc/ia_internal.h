@@ -39,7 +39,18 @@ size_t tc_workspace_bytes(const ia_shape_t& s, const TcPlan& p);
 cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
-                              void* state_out, void* ws, cudaStream_t st);
+                              void* state_out, void* ws, cudaStream_t st,
+                              float* dump_R = nullptr, float* dump_Re = nullptr);
+// Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
+HeadTables* tc_tables(void* ws);
+
+// Tensor-core training step (bf16, M = 64, d_xi = d_v = 64).
+bool tc_bwd_supported(const ia_shape_t& s);
+size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p);
+cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
+                              const void* v, const float* delta, const float* A, const void* dO,
+                              float* o, float* dq, float* dk, float* dv, float* dDelta, void* ws,
+                              cudaStream_t st);
 
 // Decode step.
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,

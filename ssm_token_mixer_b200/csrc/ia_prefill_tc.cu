@@ -43,14 +43,12 @@
 #include "ia_device.cuh"
 #include "ia_internal.h"
 #include "ia_tables.cuh"
+#include "ia_tc_common.cuh"
 
 namespace ia {
 namespace {
 
-constexpr int C = kChunk;          // 64 tokens per chunk
-constexpr int KR = 2 * kModesTC;   // 128 real rows (mode, re/im)
-constexpr int NTHR = 256;          // 8 warps: warp w owns TMEM lane quadrant w%4, column half w/4
-constexpr uint32_t kFull = 0xffffffffu;
+using namespace tc;
 
 template <int DX, int DV>
 struct Cfg {
@@ -91,56 +89,11 @@ struct TcArgs {
   float* den;
   float2* state_out;
   int* err;                 // device error flag
+  float* dump_R;            // optional: R = lambda^C S_hat at every chunk start, [BH][nch][128][F]
+  float* dump_Re;           // optional: the eta part, [BH][nch][128]
   int H, N, nseg, seg_chunks;
   long long BH;
 };
-
-__device__ __forceinline__ uint32_t tile_off(int r, int x, uint32_t rs) {
-  return static_cast<uint32_t>((r >> 3) * rs + (x >> 3) * 128 + (r & 7) * 16 + (x & 7) * 2);
-}
-
-// D (+)= A * B^T over ksteps of K = 16; A and B described by (addr, lbo, sbo,
-// byte advance per K step).
-__device__ __forceinline__ void gemm(uint32_t dtm, uint32_t a, uint32_t alb, uint32_t asb,
-                                     uint32_t ast, uint32_t b, uint32_t blb, uint32_t bsb,
-                                     uint32_t bst, uint32_t idesc, int ksteps, bool acc) {
-  for (int kk = 0; kk < ksteps; ++kk) {
-    mma_f16(dtm, smem_desc(a + kk * ast, alb, asb), smem_desc(b + kk * bst, blb, bsb), idesc,
-            (kk > 0 || acc) ? 1u : 0u);
-  }
-}
-
-// bf16 staging rows [C][W] (row-major, contiguous) -> fp16 canonical tile,
-// applying xi when FEAT; rows >= nv become zero.  One warp iteration moves 8
-// rows x 4 column groups; the column group is rotated by the row so that
-// both the staging reads and the tile writes are bank-conflict free.
-template <int W, bool FEAT>
-__device__ __forceinline__ void convert_tile(const uint8_t* stg, uint8_t* dst, int nv, int warp,
-                                             int lane) {
-  constexpr int NCG = W / 8;            // 16-byte column groups per row
-  constexpr int ITERS = (C / 8) * (NCG / 4);
-  const int r8 = lane & 7, slot = lane >> 3;
-  for (int it = warp; it < ITERS; it += NTHR / 32) {
-    const int rb = it & 7, rest = it >> 3;
-    const int cb8 = rest >> 1, sub = rest & 1;
-    const int r = rb * 8 + r8;
-    const int cg = cb8 * 8 + ((slot + 4 * sub + r8) & 7);
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nv) {
-      uint4 in = *reinterpret_cast<const uint4*>(stg + r * (W * 2) + cg * 16);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&in);
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 f = __bfloat1622float2(p[e]);
-        if (FEAT) { f.x = feat(f.x); f.y = feat(f.y); }
-        w[e] = pack_half2(f.x, f.y);
-      }
-      out = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    *reinterpret_cast<uint4*>(dst + tile_off(r, cg * 8, W * 16)) = out;
-  }
-}
 
 template <int DX, int DV, bool FULL>
 __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
@@ -296,6 +249,13 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
         w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
       }
       tmem_st16(trow + K::T_STATE + col0, w);
+      if (FULL && a.dump_R) {
+        float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + ch) * KR + k) * F + col0);
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
+                              __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
+      }
       if (FULL) {
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -316,6 +276,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     {  // eta: R_eta = lambda^C eta_hat;  eta_hat <- R_eta + sum_{j<nv} E'[j]
       const float y = __shfl_xor_sync(kFull, eta_c, 1);
       const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
+      if (FULL && half == 0 && a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
       if (FULL && half == 0)
         *reinterpret_cast<uint4*>(smem + K::S_RE + tile_off(k, 0, 256)) =
             make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
@@ -478,6 +439,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
       tmem_ld16(trow + K::T_DEN, rd);
       tmem_ld_wait16(rd);
       const float dn = __uint_as_float(rd[0]);
+      const float rdn = 1.0f / dn;
       const long long row = bh * a.N + n0 + i;
       const bool valid = lane < 16 && i < nv;
       if (valid && a.den && half == 0) a.den[row] = dn;
@@ -491,8 +453,8 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
           float4* op = reinterpret_cast<float4*>(a.o + row * DV + f0);
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            op[g] = make_float4(__uint_as_float(r[4 * g]) / dn, __uint_as_float(r[4 * g + 1]) / dn,
-                                __uint_as_float(r[4 * g + 2]) / dn, __uint_as_float(r[4 * g + 3]) / dn);
+            op[g] = make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                                __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
           if (a.num) {
             float4* np = reinterpret_cast<float4*>(a.num + row * DV + f0);
 #pragma unroll
@@ -635,10 +597,15 @@ size_t tc_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
   return bytes + 256;
 }
 
+HeadTables* tc_tables(void* ws) {
+  return reinterpret_cast<HeadTables*>((reinterpret_cast<uintptr_t>(ws) + 255) & ~static_cast<uintptr_t>(255));
+}
+
 cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
-                              void* state_out, void* ws, cudaStream_t st) {
+                              void* state_out, void* ws, cudaStream_t st, float* dump_R,
+                              float* dump_Re) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 255) & ~static_cast<uintptr_t>(255));
   HeadTables* tabs = reinterpret_cast<HeadTables*>(w);
@@ -660,6 +627,8 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
   args.den = den;
   args.state_out = static_cast<float2*>(state_out);
   args.err = device_error_ptr();
+  args.dump_R = dump_R;
+  args.dump_Re = dump_Re;
   if (!args.err) return cudaErrorInvalidSymbol;
   args.H = s.H;
   args.N = s.N;

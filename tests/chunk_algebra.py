@@ -117,3 +117,135 @@ def segmented_pass(fq, fk, v, lam, b, C, L):
     o = np.concatenate([x[0] for x in outs]); num = np.concatenate([x[1] for x in outs])
     den = np.concatenate([x[2] for x in outs])
     return o, num, den, end
+
+
+# ----------------------------------------------------------------------------
+# Reverse mode of the chunked form, in the real-row representation the
+# kernels use: complex rows become k = 2m (re), 2m+1 (im); the per-mode decay
+# rotation Rot(z) acts on each (re, im) row pair.  Per chunk, with x = [xi(K) | V]:
+#   R = Rot(lambda^C) S_hat0;  a~ = S E'' + xi(Q) R_U^T;  X = s * a~
+#   P = mask(X E''^T);  num = P V + X R_G;  den = P 1 + X R_eta;  o = num/den
+#   S_hat1 = R + E''^T x
+# Backward from dO and the adjoint of S_hat1 (the reverse carry):
+#   dnum = dO/den;  dden = -(dO . o)/den;  dP = mask(dnum V^T + dden 1^T)
+#   dV = P^T dnum + E'' dS1_G;   dX = dP E'' + dnum R_G^T + dden R_eta^T
+#   dR_G = X^T dnum;  dR_eta = X^T dden;  da~ = s * dX;  dS = mask(da~ E''^T)
+#   dxiQ = dS xi(K) + da~ R_U;  dxiK = dS^T xi(Q) + E'' dS1_U;  dR_U = da~^T xi(Q)
+#   dS_hat0 = Rot(lambda^C)^T (dS1 + [dR_U | dR_G | dR_eta])
+# Delta enters only through the per-head tables, so their adjoints are summed
+# over every chunk and contracted once with the tables' Delta-derivatives:
+#   dE'' += S^T da~ + dP^T X + x dS1^T,  ds += dX * a~,  dlambda^C += sum R conj(S_hat0)
+#   d(b lambda^n)/dDelta = (lambda + n A b) lambda^n,  ds/dDelta = 2 Re(A)(i-c) s,
+#   d(lambda^C)/dDelta = C A lambda^C.
+# ----------------------------------------------------------------------------
+def _rows(z):
+    """complex [..., M] -> real rows [..., 2M] interleaved (re, im)."""
+    out = np.empty(z.shape[:-1] + (2 * z.shape[-1],))
+    out[..., 0::2] = z.real
+    out[..., 1::2] = z.imag
+    return out
+
+
+def _rot(z, Y):
+    """Apply the per-mode complex factor z [M] to real rows Y [2M, F]."""
+    re, im = Y[0::2], Y[1::2]
+    zr, zi = z.real[:, None], z.imag[:, None]
+    out = np.empty_like(Y)
+    out[0::2] = zr * re - zi * im
+    out[1::2] = zi * re + zr * im
+    return out
+
+
+def chunk_backward(fq, fk, v, dO, lam, b, A, delta, C=64):
+    """Reverse mode of chunk_pass from a zero state for one (b,h) sequence.
+
+    Returns (o, dxiQ, dxiK, dV, dDelta) -- the feature gradients before the
+    xi' factor."""
+    N, d = fq.shape
+    dv_ = v.shape[1]
+    M = lam.shape[0]
+    c = C // 2
+    j = np.arange(C)
+    Ep = b[None, :] * lam[None, :] ** (c - j[:, None])
+    E2 = _rows(Ep)                                           # [C, 2M]
+    s = np.abs(lam[None, :]) ** (2.0 * (j[:, None] - c))
+    s2 = np.repeat(s, 2, axis=1)                             # [C, 2M]
+    lamC = lam ** C
+    causal = (j[None, :] <= j[:, None]).astype(float)
+    nch = (N + C - 1) // C
+    # forward, keeping the state at every chunk start
+    Sh = np.zeros((2 * M, d + dv_))
+    eh = np.zeros(2 * M)
+    starts = []
+    o = np.zeros((N, dv_))
+    for ch in range(nch):
+        n0 = ch * C
+        nv = min(C, N - n0)
+        starts.append((Sh.copy(), eh.copy()))
+        Q = np.zeros((C, d)); K = np.zeros((C, d)); V = np.zeros((C, dv_)); one = np.zeros(C)
+        Q[:nv] = fq[n0:n0 + nv]; K[:nv] = fk[n0:n0 + nv]; V[:nv] = v[n0:n0 + nv]; one[:nv] = 1
+        R = _rot(lamC, Sh)
+        Re = _rot(lamC, eh[:, None])[:, 0]
+        Mk = causal * (j[None, :] < nv)
+        Sb = (Q @ K.T) * Mk
+        at = Sb @ E2 + Q @ R[:, :d].T
+        X = s2 * at
+        P = (X @ E2.T) * causal
+        num = P @ V + X @ R[:, d:]
+        den = P @ one + X @ Re
+        o[n0:n0 + nv] = num[:nv] / den[:nv, None]
+        Sh = R + E2.T @ np.concatenate([K, V], axis=1)
+        eh = Re + E2.T @ one
+    # backward
+    dq = np.zeros((N, d)); dk = np.zeros((N, d)); dvv = np.zeros((N, dv_))
+    dS1 = np.zeros((2 * M, d + dv_)); de1 = np.zeros(2 * M)
+    dE2 = np.zeros_like(E2); ds2 = np.zeros_like(s2); dlamC = np.zeros(M, complex)
+    for ch in reversed(range(nch)):
+        n0 = ch * C
+        nv = min(C, N - n0)
+        Sh0, eh0 = starts[ch]
+        Q = np.zeros((C, d)); K = np.zeros((C, d)); V = np.zeros((C, dv_)); one = np.zeros(C)
+        G = np.zeros((C, dv_)); Oc = np.zeros((C, dv_))
+        Q[:nv] = fq[n0:n0 + nv]; K[:nv] = fk[n0:n0 + nv]; V[:nv] = v[n0:n0 + nv]; one[:nv] = 1
+        G[:nv] = dO[n0:n0 + nv]; Oc[:nv] = o[n0:n0 + nv]
+        R = _rot(lamC, Sh0)
+        Re = _rot(lamC, eh0[:, None])[:, 0]
+        Mk = causal * (j[None, :] < nv)
+        Sb = (Q @ K.T) * Mk
+        at = Sb @ E2 + Q @ R[:, :d].T
+        X = s2 * at
+        P = (X @ E2.T) * causal
+        den = P @ one + X @ Re
+        den_safe = np.where(np.arange(C) < nv, den, 1.0)
+        dnum = G / den_safe[:, None]
+        dden = -(G * Oc).sum(1) / den_safe
+        dP = (dnum @ V.T + dden[:, None] * one[None, :]) * causal
+        dV = P.T @ dnum + E2 @ dS1[:, d:]
+        dX = dP @ E2 + dnum @ R[:, d:].T + dden[:, None] * Re[None, :]
+        dRG = X.T @ dnum
+        dRe = X.T @ dden
+        dat = s2 * dX
+        dSm = (dat @ E2.T) * Mk
+        dRU = dat.T @ Q
+        dQ = dSm @ K + dat @ R[:, :d]
+        dK = dSm.T @ Q + E2 @ dS1[:, :d]
+        x = np.concatenate([K, V], axis=1)
+        dE2 += Sb.T @ dat + dP.T @ X + x @ dS1.T + one[:, None] * de1[None, :]
+        ds2 += dX * at
+        dR = dS1 + np.concatenate([dRU, dRG], axis=1)
+        dRe_tot = de1 + dRe
+        # adjoint of R = lambda^C S_hat0:  dlambda^C += sum conj(S_hat0) dR  (complex form)
+        Sc = Sh0[0::2] + 1j * Sh0[1::2]
+        Rc = dR[0::2] + 1j * dR[1::2]
+        dlamC += (Rc * np.conj(Sc)).sum(1) + (dRe_tot[0::2] + 1j * dRe_tot[1::2]) * np.conj(eh0[0::2] + 1j * eh0[1::2])
+        dS1 = _rot(np.conj(lamC), dR)
+        de1 = _rot(np.conj(lamC), dRe_tot[:, None])[:, 0]
+        dq[n0:n0 + nv] = dQ[:nv]; dk[n0:n0 + nv] = dK[:nv]; dvv[n0:n0 + nv] = dV[:nv]
+    # Delta through the tables
+    dEc = dE2[:, 0::2] + 1j * dE2[:, 1::2]
+    dEp = lam[None, :] * lam[None, :] ** (c - j[:, None]) + (c - j[:, None]) * A[None, :] * Ep
+    ds = ds2[:, 0::2] + ds2[:, 1::2]
+    dsd = 2.0 * A.real[None, :] * (j[:, None] - c) * s
+    dD = float(np.sum((np.conj(dEc) * dEp).real) + np.sum(ds * dsd)
+               + np.sum((np.conj(dlamC) * C * A * lamC).real))
+    return o, dq, dk, dvv, dD

@@ -54,3 +54,25 @@ def test_p7_segmented_two_pass(oracle_mod, L, N):
     assert rel(den, ref["den"][0, 0]) < 1e-11
     Ur, Gr, er = oracle_mod.split_state(ref["state"], 1, 1, M, 3, 2)
     assert rel(U, Ur[0, 0]) < 1e-11 and rel(e, er[0, 0]) < 1e-11
+
+
+@pytest.mark.parametrize("N,C", [(150, 64), (64, 64), (37, 16), (100, 8)])
+def test_p7_chunked_reverse_mode_equals_oracle_adjoint(oracle_mod, N, C):
+    # the reverse mode of the chunked algorithm (table adjoints for Delta)
+    # reproduces the oracle's sequential adjoint
+    from chunk_algebra import chunk_backward
+    rng = np.random.default_rng(N + C)
+    d, dv, M = 5, 3, 7
+    q = rng.standard_normal((1, 1, N, d)); k = rng.standard_normal((1, 1, N, d))
+    v = rng.standard_normal((1, 1, N, dv)); dO = rng.standard_normal((1, 1, N, dv))
+    delta = np.array([0.06])
+    ref = oracle_mod.backward(q, k, v, delta, dO, M)
+    lam, b = oracle_mod.params(M, delta[0])
+    A = -0.5 + 1j * np.pi * np.arange(M)
+    o, dxq, dxk, dvv, dD = chunk_backward(feat(q[0, 0]), feat(k[0, 0]), v[0, 0], dO[0, 0], lam, b, A, delta[0], C)
+    dfeat = lambda x: np.where(x > 0, 1.0, np.exp(np.minimum(x, 0.0)))
+    assert rel(o, ref["o"][0, 0]) < 1e-10
+    assert rel(dxq * dfeat(q[0, 0]), ref["dq"][0, 0]) < 1e-9
+    assert rel(dxk * dfeat(k[0, 0]), ref["dk"][0, 0]) < 1e-9
+    assert rel(dvv, ref["dv"][0, 0]) < 1e-9
+    assert abs(dD - ref["dDelta"][0]) < 1e-9 * max(1.0, abs(ref["dDelta"][0]))

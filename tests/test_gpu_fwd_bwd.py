@@ -50,3 +50,25 @@ def test_fwd_bwd_training_shape_reduced_batch(oracle_mod, dev):
     r = run(inp, w.M, dev)
     g = oracle_mod.backward(inp["q"], inp["k"], inp["v"], inp["delta"], inp["dO"], w.M)
     compare(r, g, TOL_BF16)
+
+
+@pytest.mark.parametrize("N", [64, 150, 333])
+def test_fwd_bwd_tensor_core_path(oracle_mod, dev, N):
+    # bf16, M = 64, d = 64 runs the tensor-core reverse-mode kernel; ragged N
+    B, H, d, M = 2, 3, 64, 64
+    inp = synthetic.layer_inputs(B, H, N, d, d, "bf16", seed=41 + N, with_grad=True)
+    r = run(inp, M, dev)
+    g = oracle_mod.backward(inp["q"], inp["k"], inp["v"], inp["delta"], inp["dO"], M)
+    assert slice_rel(r["o"], g["o"], (-2, -1)) < TOL_BF16
+    compare(r, g, TOL_BF16)
+
+
+def test_fwd_bwd_tensor_core_matches_cuda_core(dev, monkeypatch):
+    inp = synthetic.layer_inputs(2, 2, 200, 64, 64, "bf16", seed=77, with_grad=True)
+    r_tc = run(inp, 64, dev)
+    monkeypatch.setenv("IA_BWD_SIMT", "1")
+    r_ref = run(inp, 64, dev)
+    for key in ("dq", "dk", "dv"):
+        assert slice_rel(r_tc[key], r_ref[key], (-2, -1)) < TOL_BF16, key
+    dd = (r_tc["dDelta"] - r_ref["dDelta"]).abs().max() / r_ref["dDelta"].abs().max()
+    assert dd.item() < TOL_BF16
