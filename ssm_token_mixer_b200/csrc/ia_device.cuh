@@ -65,6 +65,48 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   return true;
 }
 
+// Arrive once (release semantics) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that also gives up as soon as another thread of the CTA has
+// raised *abort (a shared flag); raises it itself on expiry.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, int* err,
+                                                   volatile int* abort) {
+  if (mbar_test(bar, parity)) return true;
+  unsigned long long t0 = global_ns();
+  while (!mbar_test(bar, parity)) {
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(err, 1);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// Named barrier among `count` threads that also ORs a predicate across them:
+// returns true if any participating thread passed true.
+__device__ __forceinline__ bool named_sync_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Named barrier among `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ------------------------------------------------------------- bulk copies
 // Contiguous global -> shared copy completing on an mbarrier (transaction
 // bytes).  dst, src 16-byte aligned; bytes a multiple of 16.

@@ -50,13 +50,21 @@ namespace {
 
 using namespace tc;
 
+constexpr int NT = 512;            // 16 warps: warp w owns TMEM lane quadrant w%4, column quarter w/4
+constexpr int NWARP = NT / 32;
+
 template <int DX, int DV>
 struct Cfg {
   static constexpr int F = DX + DV;
-  static constexpr uint32_t RSX = DX * 16;   // row-group stride of an [r][DX] fp16 tile
-  static constexpr uint32_t RSV = DV * 16;
-  static constexpr uint32_t T_STATE = 0, T_A = F, T_DEN = F, T_SP = F + 64, T_NUM = F + 128;
-  static_assert(F + 128 + DV <= 512, "TMEM budget");
+  // den rides along the value contractions as an extra column when TMEM has room
+  static constexpr bool MERGE = F + 128 + DV + 16 <= 512;
+  static constexpr int WV = MERGE ? DV + 16 : DV;   // width of the V and R_Gamma tiles
+  static constexpr int NV = MERGE ? DV + 16 : DV;   // N of the value contractions
+  static constexpr uint32_t RSX = DX * 16;          // row-group stride of an [r][DX] fp16 tile
+  static constexpr uint32_t RSV = WV * 16;
+  static constexpr uint32_t T_STATE = 0, T_A = F, T_SP = F + 64, T_NUM = F + 128;
+  static constexpr uint32_t T_DEN = MERGE ? T_NUM + DV : F;
+  static_assert(F + 128 + NV <= 512, "TMEM budget");
   static_assert(DX % 64 == 0 && DV % 64 == 0, "feature widths must be multiples of 64");
   static constexpr uint32_t STG_Q = 0;
   static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
@@ -64,16 +72,20 @@ struct Cfg {
   static constexpr uint32_t S_Q = STG_V + C * DV * 2;
   static constexpr uint32_t S_K = S_Q + C * DX * 2;
   static constexpr uint32_t S_V = S_K + C * DX * 2;
-  static constexpr uint32_t S_E = S_V + C * DV * 2;
+  static constexpr uint32_t S_E = S_V + C * WV * 2;
   static constexpr uint32_t S_SP = S_E + KR * C * 2;
   static constexpr uint32_t S_X = S_SP + C * C * 2;
   static constexpr uint32_t S_RU = S_X + KR * C * 2;
   static constexpr uint32_t S_RG = S_RU + KR * DX * 2;
-  static constexpr uint32_t S_RE = S_RG + KR * DV * 2;
-  static constexpr uint32_t S_ONES = S_RE + KR * 16 * 2;
-  static constexpr uint32_t S_BAR = S_ONES + C * 16 * 2;
+  static constexpr uint32_t S_RE = S_RG + KR * WV * 2;
+  static constexpr uint32_t S_ONES = S_RE + (MERGE ? 0 : KR * 16 * 2);
+  static constexpr uint32_t S_BAR = S_ONES + (MERGE ? 0 : C * 16 * 2);
   static constexpr uint32_t S_TMEMH = S_BAR + 32;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
+  // o of one chunk is staged (fp32, swizzled) over the sX and sRU tiles, both
+  // free while the output is written
+  static constexpr uint32_t S_OUT = S_X;
+  static_assert(KR * C * 2 + KR * DX * 2 >= C * DV * 4, "output staging fits");
 };
 
 struct TcArgs {
@@ -95,13 +107,62 @@ struct TcArgs {
   long long BH;
 };
 
+// bf16 staging rows [C][W] (row-major) -> fp16 canonical tile of row width WD,
+// applying xi when FEAT; rows >= nv become zero.  Work is split into warp
+// iterations of 8 rows x 4 column groups, the column group rotated by the row
+// so that staging reads and tile writes are bank-conflict free; all loads of
+// a thread are issued before any conversion.
+template <int W, int WD, bool FEAT>
+__device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, int nv, int warp, int lane) {
+  constexpr int NCG = W / 8;
+  constexpr int ITERS = (C / 8) * (NCG / 4);
+  constexpr int PER = (ITERS + NWARP - 1) / NWARP;
+  const int r8 = lane & 7, slot = lane >> 3;
+  uint4 in[PER];
+  int rr[PER], cc[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int it = warp + u * NWARP;
+    const int rb = it & 7, rest = it >> 3;
+    rr[u] = rb * 8 + r8;
+    cc[u] = (rest >> 1) * 8 + ((slot + 4 * (rest & 1) + r8) & 7);
+    in[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (it < ITERS && rr[u] < nv) in[u] = *reinterpret_cast<const uint4*>(stg + rr[u] * (W * 2) + cc[u] * 16);
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int it = warp + u * NWARP;
+    if (it >= ITERS) break;
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (rr[u] < nv) {
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 f = __bfloat1622float2(p[e]);
+        if (FEAT) { f.x = feat(f.x); f.y = feat(f.y); }
+        w[e] = pack_half2(f.x, f.y);
+      }
+      out = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *reinterpret_cast<uint4*>(dst + tile_off(rr[u], cc[u] * 8, WD * 16)) = out;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8f(const uint32_t* r, float scale) {
+  return make_uint4(pack_half2(__uint_as_float(r[0]) * scale, __uint_as_float(r[1]) * scale),
+                    pack_half2(__uint_as_float(r[2]) * scale, __uint_as_float(r[3]) * scale),
+                    pack_half2(__uint_as_float(r[4]) * scale, __uint_as_float(r[5]) * scale),
+                    pack_half2(__uint_as_float(r[6]) * scale, __uint_as_float(r[7]) * scale));
+}
+
 template <int DX, int DV, bool FULL>
-__global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
+__global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
   using K = Cfg<DX, DV>;
   constexpr int F = K::F;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
+  const int quad = warp & 3, part = warp >> 2;   // lane quadrant, column quarter
   const int nrun = FULL ? a.nseg : a.nseg - 1;
   const long long bh = blockIdx.x / nrun;
   const int seg = static_cast<int>(blockIdx.x % nrun);
@@ -128,13 +189,26 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
   {  // E' table -> shared (already in canonical layout), constant tiles
     const uint4* src = reinterpret_cast<const uint4*>(T->E);
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += NTHR) dst[i] = src[i];
+    for (int i = tid; i < KR * C * 2 / 16; i += NT) dst[i] = src[i];
     if (FULL) {
-      uint4* ones = reinterpret_cast<uint4*>(smem + K::S_ONES);
       const uint32_t one2 = 0x3C003C00u;   // two fp16 ones
-      for (int i = tid; i < C * 16 * 2 / 16; i += NTHR) ones[i] = make_uint4(one2, one2, one2, one2);
-      uint4* re = reinterpret_cast<uint4*>(smem + K::S_RE);
-      for (int i = tid; i < KR * 16 * 2 / 16; i += NTHR) re[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (K::MERGE) {
+        // V's extra column DV is 1 (gives den = P 1), R_Gamma's extra columns
+        // start at zero (column DV receives R_eta every chunk)
+        for (int r = tid; r < C; r += NT) {
+          *reinterpret_cast<uint4*>(smem + K::S_V + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(smem + K::S_V + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int r = tid; r < KR; r += NT) {
+          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+        uint4* ones = reinterpret_cast<uint4*>(smem + K::S_ONES);
+        for (int i = tid; i < C * 16 * 2 / 16; i += NT) ones[i] = make_uint4(one2, one2, one2, one2);
+        uint4* re = reinterpret_cast<uint4*>(smem + K::S_RE);
+        for (int i = tid; i < KR * 16 * 2 / 16; i += NT) re[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
   }
   tc_fence_before();
@@ -148,9 +222,10 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
   const float2 lamC = T->lamC[m];
   const float sgnLi = comp ? lamC.y : -lamC.y;
   const float r2 = T->r2[m];
-  const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
+  const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (16.0 * part - C / 2)));
   const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
   const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+  constexpr int FQ = F / 4;    // state columns per thread
 
   // Initial (scaled) state into TMEM rows.
   float eta_c = 0.f;
@@ -163,8 +238,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     }
     const bool from_in = FULL && seg == 0 && a.state_in != nullptr;
     const float2 si = T->sc_inv[m];
-    for (int cb = 0; cb < F / 2; cb += 16) {
-      const int col0 = half * (F / 2) + cb;
+#pragma unroll
+    for (int cb = 0; cb < FQ; cb += 16) {
+      const int col0 = part * FQ + cb;
       uint32_t r[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -228,16 +304,17 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
       if (__syncthreads_or(!ok)) { aborted = true; break; }
       tma_pending = false;
     }
-    if (FULL) convert_tile<DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
-    convert_tile<DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
-    convert_tile<DV, false>(smem + K::STG_V, smem + K::S_V, nv, warp, lane);
+    if (FULL) convert_all<DX, DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
+    convert_all<DX, DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
+    convert_all<DV, K::WV, false>(smem + K::STG_V, smem + K::S_V, nv, warp, lane);
     __syncthreads();   // staging consumed
     if (tid == 0 && ch + 1 < ch1) issue_load(ch + 1);
     tma_pending = ch + 1 < ch1;
 
     // ---- state: R = lambda^C S_hat -> TMEM (for GEMM7) and fp16 operands
-    for (int cb = 0; cb < F / 2; cb += 16) {
-      const int col0 = half * (F / 2) + cb;
+#pragma unroll
+    for (int cb = 0; cb < FQ; cb += 16) {
+      const int col0 = part * FQ + cb;
       uint32_t r[16];
       tmem_ld16(trow + K::T_STATE + col0, r);
       tmem_ld_wait16(r);
@@ -259,11 +336,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
       if (FULL) {
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          uint4 pk;
-          pk.x = pack_half2(__uint_as_float(w[8 * g + 0]), __uint_as_float(w[8 * g + 1]));
-          pk.y = pack_half2(__uint_as_float(w[8 * g + 2]), __uint_as_float(w[8 * g + 3]));
-          pk.z = pack_half2(__uint_as_float(w[8 * g + 4]), __uint_as_float(w[8 * g + 5]));
-          pk.w = pack_half2(__uint_as_float(w[8 * g + 6]), __uint_as_float(w[8 * g + 7]));
+          const uint4 pk = pack8f(w + 8 * g, 1.f);
           const int f = col0 + 8 * g;
           if (f < DX)
             *reinterpret_cast<uint4*>(smem + K::S_RU + tile_off(k, f, K::RSX)) = pk;
@@ -276,21 +349,24 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     {  // eta: R_eta = lambda^C eta_hat;  eta_hat <- R_eta + sum_{j<nv} E'[j]
       const float y = __shfl_xor_sync(kFull, eta_c, 1);
       const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
-      if (FULL && half == 0 && a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
-      if (FULL && half == 0)
-        *reinterpret_cast<uint4*>(smem + K::S_RE + tile_off(k, 0, 256)) =
-            make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
+      if (FULL && part == 0) {
+        if (a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
+        const uint4 pk = make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
+        if (K::MERGE)
+          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(k, DV, K::RSV)) = pk;
+        else
+          *reinterpret_cast<uint4*>(smem + K::S_RE + tile_off(k, 0, 256)) = pk;
+      }
       float add = esum_c;
       if (nv < C) {   // ragged last chunk: partial sum of E' over the valid keys
-        double pr, pi, sr = 0.0, si = 0.0;
+        double sr = 0.0, si = 0.0;
         const double br = T->b[m].x, bi = T->b[m].y;
         for (int j = 0; j < nv; ++j) {
-          double e = exp((C / 2 - j) * T->re_dA[m]);
-          double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
-          double s, c;
-          sincos(ph, &s, &c);
-          pr = e * c;
-          pi = e * s;
+          const double e = exp((C / 2 - j) * T->re_dA[m]);
+          const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
+          double sn, cs;
+          sincos(ph, &sn, &cs);
+          const double pr = e * cs, pi = e * sn;
           sr += br * pr - bi * pi;
           si += br * pi + bi * pr;
         }
@@ -316,31 +392,20 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     if (!mma_sync()) { aborted = true; break; }
     if (!FULL) continue;
 
+    const int i0 = 16 * part;     // this thread's 16 columns of the 64-wide tiles
     // ---- E1: S^T (M=64 rows j) -> masked fp16, MN-major B of GEMM2
     {
       const int j = 16 * quad + lane;
+      uint32_t r[16];
+      tmem_ld16(trow + K::T_SP + i0, r);
+      tmem_ld_wait16(r);
+      if (lane < 16) {
+        const bool keep = j < nv;
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int i0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_SP + i0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = i0 + 8 * g + 2 * e;
-              const bool keep = j < nv;
-              float x0 = (keep && i >= j) ? __uint_as_float(r[8 * g + 2 * e]) : 0.f;
-              float x1 = (keep && i + 1 >= j) ? __uint_as_float(r[8 * g + 2 * e + 1]) : 0.f;
-              w[e] = pack_half2(x0, x1);
-            }
-            *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, i0 + 8 * g, 1024)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+        for (int e = 0; e < 16; ++e)
+          if (!(keep && i0 + e >= j)) r[e] = 0u;
+        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, i0, 1024)) = pack8f(r, 1.f);
+        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
       }
     }
     to_tensor_core();
@@ -358,28 +423,17 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
 
     // ---- E2: X = |lambda|^(2(i-c)) a~  (rows k, columns i) -> MN-major A of GEMM4/6
     {
+      uint32_t r[16];
+      tmem_ld16(trow + K::T_A + i0, r);
+      tmem_ld_wait16(r);
       float s = s_start;
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int i0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_A + i0, r);
-        tmem_ld_wait16(r);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(r[8 * g + 2 * e]) * s;
-            s *= r2;
-            const float x1 = __uint_as_float(r[8 * g + 2 * e + 1]) * s;
-            s *= r2;
-            w[e] = pack_half2(x0, x1);
-          }
-          *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 8 * g, 1024)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
+      for (int e = 0; e < 16; ++e) {
+        r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
+        s *= r2;
       }
+      *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0, 1024)) = pack8f(r, 1.f);
+      *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
     }
     to_tensor_core();
     if (tid == 0) {
@@ -393,27 +447,15 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     // ---- E3: P (M=64 rows i) -> masked fp16, K-major A of GEMM5
     {
       const int i = 16 * quad + lane;
+      uint32_t r[16];
+      tmem_ld16(trow + K::T_SP + i0, r);
+      tmem_ld_wait16(r);
+      if (lane < 16) {
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_SP + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = j0 + 8 * g + 2 * e;
-              float x0 = j <= i ? __uint_as_float(r[8 * g + 2 * e]) : 0.f;
-              float x1 = j + 1 <= i ? __uint_as_float(r[8 * g + 2 * e + 1]) : 0.f;
-              w[e] = pack_half2(x0, x1);
-            }
-            *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, j0 + 8 * g, 1024)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+        for (int e = 0; e < 16; ++e)
+          if (i0 + e > i) r[e] = 0u;
+        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, i0, 1024)) = pack8f(r, 1.f);
+        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
       }
     }
     to_tensor_core();
@@ -421,18 +463,20 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
       tc_fence_after();
       const uint32_t sSP = sbase + K::S_SP, sX = sbase + K::S_X;
       gemm(tmem + K::T_NUM, sSP, 128, 1024, 256, sbase + K::S_V, K::RSV, 128, 2 * K::RSV,
-           idesc_f16(64, DV, 0, 1), C / 16, false);   // GEMM5: P V
-      gemm(tmem + K::T_DEN, sSP, 128, 1024, 256, sbase + K::S_ONES, 256, 128, 512,
-           idesc_f16(64, 16, 0, 1), C / 16, false);   // GEMM5b: P 1
+           idesc_f16(64, K::NV, 0, 1), C / 16, false);   // GEMM5: P [V | 1]
       gemm(tmem + K::T_NUM, sX, 1024, 128, 2048, sbase + K::S_RG, K::RSV, 128, 2 * K::RSV,
-           idesc_f16(64, DV, 1, 1), KR / 16, true);   // GEMM6: X R_Gamma
-      gemm(tmem + K::T_DEN, sX, 1024, 128, 2048, sbase + K::S_RE, 256, 128, 512,
-           idesc_f16(64, 16, 1, 1), KR / 16, true);   // GEMM6b: X R_eta
+           idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // GEMM6: X [R_Gamma | R_eta]
+      if (!K::MERGE) {
+        gemm(tmem + K::T_DEN, sSP, 128, 1024, 256, sbase + K::S_ONES, 256, 128, 512,
+             idesc_f16(64, 16, 0, 1), C / 16, false);   // GEMM5b: P 1
+        gemm(tmem + K::T_DEN, sX, 1024, 128, 2048, sbase + K::S_RE, 256, 128, 512,
+             idesc_f16(64, 16, 1, 1), KR / 16, true);   // GEMM6b: X R_eta
+      }
       mma_commit(bar_mma);
     }
     if (!mma_sync()) { aborted = true; break; }
 
-    // ---- E4: o = num / den (M=64 rows i)
+    // ---- E4: o = num / den, staged in shared memory, then written coalesced
     {
       const int i = 16 * quad + lane;
       uint32_t rd[16];
@@ -442,20 +486,23 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
       const float rdn = 1.0f / dn;
       const long long row = bh * a.N + n0 + i;
       const bool valid = lane < 16 && i < nv;
-      if (valid && a.den && half == 0) a.den[row] = dn;
+      if (valid && a.den && part == 0) a.den[row] = dn;
+      constexpr int DQ = DV / 4;   // value columns per thread
 #pragma unroll
-      for (int cb = 0; cb < DV / 2; cb += 16) {
-        const int f0 = half * (DV / 2) + cb;
+      for (int cb = 0; cb < DQ; cb += 16) {
+        const int f0 = part * DQ + cb;
         uint32_t r[16];
         tmem_ld16(trow + K::T_NUM + f0, r);
         tmem_ld_wait16(r);
-        if (valid) {
-          float4* op = reinterpret_cast<float4*>(a.o + row * DV + f0);
+        if (lane < 16) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            op[g] = make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                                __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-          if (a.num) {
+          for (int g = 0; g < 4; ++g) {
+            const int chunk = (f0 >> 2) + g;
+            *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
+                make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                            __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
+          }
+          if (valid && a.num) {
             float4* np = reinterpret_cast<float4*>(a.num + row * DV + f0);
 #pragma unroll
             for (int g = 0; g < 4; ++g)
@@ -463,6 +510,14 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
                                   __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
           }
         }
+      }
+      __syncthreads();
+      constexpr int CPR = DV / 4;  // 16-byte chunks per row
+      float* obase = a.o + (bh * a.N + n0) * DV;
+      for (int c = tid; c < nv * CPR; c += NT) {
+        const int rr = c / CPR, g = c % CPR;
+        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
+        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
       }
     }
     tc_fence_before();
@@ -473,14 +528,14 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
     if (FULL) {
       if (a.state_out && seg == a.nseg - 1) {
         // state after the last token: sc * lambda^(nv - C) * S_hat = lambda^(nv-c-1) S_hat
-        double pr, pi, e = exp((nv - C / 2 - 1) * T->re_dA[m]);
-        double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925), s, c;
-        sincos(ph, &s, &c);
-        pr = e * c;
-        pi = e * s;
-        const float fr = static_cast<float>(pr), fi = static_cast<float>(pi);
-        for (int cb = 0; cb < F / 2; cb += 16) {
-          const int col0 = half * (F / 2) + cb;
+        const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
+        const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
+        double sn, cs;
+        sincos(ph, &sn, &cs);
+        const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
+#pragma unroll
+        for (int cb = 0; cb < FQ; cb += 16) {
+          const int col0 = part * FQ + cb;
           uint32_t r[16];
           tmem_ld16(trow + K::T_STATE + col0, r);
           tmem_ld_wait16(r);
@@ -497,14 +552,15 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
           }
         }
         const float y = __shfl_xor_sync(kFull, eta_c, 1);
-        if (comp == 0 && half == 0)
+        if (comp == 0 && part == 0)
           a.state_out[a.BH * 64 * F + bh * 64 + m] =
               make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
       }
     } else {
       float* dst = a.seg_state + ((bh * (a.nseg - 1) + seg) * KR + k) * F;
-      for (int cb = 0; cb < F / 2; cb += 16) {
-        const int col0 = half * (F / 2) + cb;
+#pragma unroll
+      for (int cb = 0; cb < FQ; cb += 16) {
+        const int col0 = part * FQ + cb;
         uint32_t r[16];
         tmem_ld16(trow + K::T_STATE + col0, r);
         tmem_ld_wait16(r);
@@ -514,10 +570,463 @@ __global__ void __launch_bounds__(NTHR, 1) tc_prefill_kernel(const TcArgs a) {
           d4[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
                               __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
       }
-      if (half == 0) a.seg_eta[(bh * (a.nseg - 1) + seg) * KR + k] = eta_c;
+      if (part == 0) a.seg_eta[(bh * (a.nseg - 1) + seg) * KR + k] = eta_c;
     }
   } else if (tma_pending) {
     mbar_wait(bar_tma, ph_tma, a.err);   // bounded: let our own copy land before exiting
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// Warp-specialized full pass for d_xi = d_v = 64.  tcgen05.mma issue blocks
+// the issuing thread for about as long as the tensor core works, so the
+// contractions are issued by a dedicated warp (warp 16, which also issues the
+// bulk copies) while 16 epilogue warps do the elementwise phases.  The two
+// sides hand over through mbarriers: "ready" barriers (512 epilogue-thread
+// arrivals after their shared/TMEM writes) and "done" barriers (one
+// tcgen05.commit).  Chunks are software-pipelined: the tail of chunk t-1
+// (mask P, value contractions, output) is interleaved with the head of chunk
+// t (Gram, decay contractions, readout scale), so the tensor core works on
+// one chunk while the epilogue warps work on the other.  V, R_Gamma and R_eta
+// are double-buffered; S, P, a~, num have their own TMEM tiles.
+constexpr int WS_EW = 16;                   // epilogue warps
+constexpr int WS_ET = WS_EW * 32;           // epilogue threads
+constexpr int WS_NT = WS_ET + 32;           // + one MMA / copy warp
+
+struct WCfg {
+  static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
+  static constexpr uint32_t RSX = DX * 16, RSV = WV * 16;
+  static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
+                            T_DEN = 320 + 64;
+  static constexpr uint32_t STG_Q = 0;
+  static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
+  static constexpr uint32_t STG_V = STG_K + C * DX * 2;
+  static constexpr uint32_t S_Q = STG_V + C * DV * 2;
+  static constexpr uint32_t S_K = S_Q + C * DX * 2;
+  static constexpr uint32_t S_V0 = S_K + C * DX * 2;
+  static constexpr uint32_t S_V1 = S_V0 + C * WV * 2;
+  static constexpr uint32_t S_E = S_V1 + C * WV * 2;
+  static constexpr uint32_t S_S = S_E + KR * C * 2;
+  static constexpr uint32_t S_P = S_S + C * C * 2;
+  static constexpr uint32_t S_X = S_P + C * C * 2;
+  static constexpr uint32_t S_RU = S_X + KR * C * 2;
+  static constexpr uint32_t S_RG0 = S_RU + KR * DX * 2;
+  static constexpr uint32_t S_RG1 = S_RG0 + KR * WV * 2;
+  static constexpr uint32_t S_BAR = S_RG1 + KR * WV * 2;    // 10 mbarriers
+  static constexpr uint32_t S_FLAG = S_BAR + 80;
+  static constexpr uint32_t S_TMEMH = S_FLAG + 16;
+  static constexpr uint32_t SMEM = S_TMEMH + 16;
+  static constexpr uint32_t S_OUT = S_X;   // o of chunk t-1 is staged while sX is free
+  static_assert(KR * C * 2 >= C * DV * 4, "output staging fits in sX");
+};
+
+__global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a) {
+  using K = WCfg;
+  constexpr int DX = K::DX, DV = K::DV, F = K::F;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool mma_warp = warp == WS_EW;
+  const int quad = warp & 3, part = (warp >> 2) & 3;
+  const long long bh = blockIdx.x / a.nseg;
+  const int seg = static_cast<int>(blockIdx.x % a.nseg);
+  const int h = static_cast<int>(bh % a.H);
+  const HeadTables* T = a.tabs + h;
+  const int nch_total = (a.N + C - 1) / C;
+  const int ch0 = seg * a.seg_chunks;
+  const int ch1 = min(ch0 + a.seg_chunks, nch_total);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* bar_tma = bars + 0;
+  uint64_t* rdy = bars + 1;     // rdy[0..3]: ready for G1+G7, G2+G3, G4, G5+G6
+  uint64_t* dne = bars + 5;     // dne[0..3]: done   "
+  uint64_t* bar_drain = bars + 9;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
+  const uint32_t sbase = smem_u32(smem);
+
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_tma, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(rdy + i, WS_ET);
+      mbar_init(dne + i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(T->E);
+    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
+    for (int i = tid; i < KR * C * 2 / 16; i += WS_NT) dst[i] = src[i];
+    // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
+    for (int r = tid; r < C; r += WS_NT) {
+      for (int p = 0; p < 2; ++p) {
+        const uint32_t sv = p ? K::S_V1 : K::S_V0;
+        *reinterpret_cast<uint4*>(smem + sv + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sv + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    for (int r = tid; r < KR; r += WS_NT) {
+      for (int p = 0; p < 2; ++p) {
+        const uint32_t sr = p ? K::S_RG1 : K::S_RG0;
+        *reinterpret_cast<uint4*>(smem + sr + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sr + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (mma_warp) {
+    // ------------------------------------------------ MMA and copy issuer
+    if (lane == 0) {
+      uint32_t pr[4] = {0u, 0u, 0u, 0u};
+      int issued = 0;
+      bool ok = true;
+      auto issue_load = [&](int ch) {
+        const int n0 = ch * C;
+        const int nv = min(C, a.N - n0);
+        const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
+        mbar_arrive_expect_tx(bar_tma, 2 * bq + bv);
+        const long long row = bh * a.N + n0;
+        bulk_g2s(smem + K::STG_Q, a.q + row * DX, bq, bar_tma);
+        bulk_g2s(smem + K::STG_K, a.k + row * DX, bq, bar_tma);
+        bulk_g2s(smem + K::STG_V, a.v + row * DV, bv, bar_tma);
+        ++issued;
+      };
+      auto wait_rdy = [&](int i) -> bool {
+        const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
+        pr[i] ^= 1u;
+        tc_fence_after();
+        return r;
+      };
+      auto g5g6 = [&](int pp) {
+        const uint32_t sv = sbase + (pp ? K::S_V1 : K::S_V0), srg = sbase + (pp ? K::S_RG1 : K::S_RG0);
+        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sv, K::RSV, 128, 2 * K::RSV,
+             idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
+        gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, srg, K::RSV, 128, 2 * K::RSV,
+             idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
+        mma_commit(dne + 3);
+      };
+      if (ch0 < ch1) issue_load(ch0);
+      for (int t = ch0; t < ch1; ++t) {
+        const int p = (t - ch0) & 1;
+        if (!(ok = wait_rdy(0))) break;
+        if (t + 1 < ch1) issue_load(t + 1);   // staging was consumed before ready(0)
+        const uint32_t sv = sbase + (p ? K::S_V1 : K::S_V0);
+        gemm(tmem + K::T_S, sbase + K::S_K, 128, K::RSX, 256, sbase + K::S_Q, 128, K::RSX, 256,
+             idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
+        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + K::S_K, K::RSX, 128,
+             2 * K::RSX, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
+        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sv, K::RSV, 128, 2 * K::RSV,
+             idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
+        mma_commit(dne + 0);
+        if (t > ch0) {
+          if (!(ok = wait_rdy(3))) break;
+          g5g6(p ^ 1);
+        }
+        if (!(ok = wait_rdy(1))) break;
+        gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
+             idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
+        gemm(tmem + K::T_A, sbase + K::S_RU, 128, K::RSX, 256, sbase + K::S_Q, 128, K::RSX, 256,
+             idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
+        mma_commit(dne + 1);
+        if (!(ok = wait_rdy(2))) break;
+        gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
+             idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
+        mma_commit(dne + 2);
+      }
+      if (ok && ch0 < ch1) {
+        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) & 1);
+      }
+      if (!ok) {
+        // drain: every tensor-core group issued so far, and the last copy
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0u, a.err);
+        if (issued > 0) mbar_wait(bar_tma, static_cast<uint32_t>((issued - 1) & 1), a.err);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue warps
+    const int k = 32 * quad + lane;
+    const int m = k >> 1, comp = k & 1;
+    const float2 lamC = T->lamC[m];
+    const float sgnLi = comp ? lamC.y : -lamC.y;
+    const float r2 = T->r2[m];
+    const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (16.0 * part - C / 2)));
+    const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    constexpr int FQ = F / 4;
+    const int i0 = 16 * part;
+    uint32_t pd[4] = {0u, 0u, 0u, 0u};
+    uint32_t ptma = 0u;
+    auto wait_dne = [&](int i) -> bool {   // outcome made uniform across the epilogue warps
+      const bool r = mbar_wait_or_abort(dne + i, pd[i], a.err, abort_flag);
+      pd[i] ^= 1u;
+      tc_fence_after();
+      return !named_sync_or(2, WS_ET, !r);
+    };
+    auto signal = [&](int i) {   // my shared / TMEM writes are done: ready(i)
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(rdy + i);
+    };
+
+    float eta_c = 0.f;
+    {  // initial (scaled) state
+      const float* carry = nullptr;
+      const float* carry_eta = nullptr;
+      if (seg > 0) {
+        carry = a.seg_state + ((bh * (a.nseg - 1) + (seg - 1)) * KR + k) * F;
+        carry_eta = a.seg_eta + (bh * (a.nseg - 1) + (seg - 1)) * KR + k;
+      }
+      const bool from_in = seg == 0 && a.state_in != nullptr;
+      const float2 si = T->sc_inv[m];
+#pragma unroll
+      for (int cb = 0; cb < FQ; cb += 16) {
+        const int col0 = part * FQ + cb;
+        uint32_t r[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float val = 0.f;
+          const int f = col0 + e;
+          if (carry) {
+            val = carry[f];
+          } else if (from_in) {
+            float2 x = f < DX ? a.state_in[(bh * 64 + m) * DX + f]
+                              : a.state_in[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)];
+            val = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
+          }
+          r[e] = __float_as_uint(val);
+        }
+        tmem_st16(trow + K::T_STATE + col0, r);
+      }
+      if (carry_eta) {
+        eta_c = *carry_eta;
+      } else if (from_in) {
+        float2 x = a.state_in[a.BH * 64 * F + bh * 64 + m];
+        eta_c = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
+      }
+      tmem_st_wait();
+    }
+
+    int nv_last = C;
+    // chunk ch, buffer parity p: convert inputs, rotate the state, signal ready(0)
+    auto prepare = [&](int ch, int p) -> bool {
+      const int nv = min(C, a.N - ch * C);
+      nv_last = nv;
+      const bool r = mbar_wait_or_abort(bar_tma, ptma, a.err, abort_flag);
+      ptma ^= 1u;
+      if (named_sync_or(2, WS_ET, !r)) return false;
+      const uint32_t sv = p ? K::S_V1 : K::S_V0, srg = p ? K::S_RG1 : K::S_RG0;
+      convert_all<DX, DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
+      convert_all<DX, DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
+      convert_all<DV, K::WV, false>(smem + K::STG_V, smem + sv, nv, warp, lane);
+#pragma unroll
+      for (int cb = 0; cb < FQ; cb += 16) {
+        const int col0 = part * FQ + cb;
+        uint32_t rr[16];
+        tmem_ld16(trow + K::T_STATE + col0, rr);
+        tmem_ld_wait16(rr);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x = __uint_as_float(rr[e]);
+          const float y = __shfl_xor_sync(kFull, x, 1);
+          w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
+        }
+        tmem_st16(trow + K::T_STATE + col0, w);
+        if (a.dump_R) {
+          float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + ch) * KR + k) * F + col0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
+                                __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
+        }
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint4 pk = pack8f(w + 8 * g, 1.f);
+          const int f = col0 + 8 * g;
+          if (f < DX)
+            *reinterpret_cast<uint4*>(smem + K::S_RU + tile_off(k, f, K::RSX)) = pk;
+          else
+            *reinterpret_cast<uint4*>(smem + srg + tile_off(k, f - DX, K::RSV)) = pk;
+        }
+      }
+      tmem_st_wait();
+      {
+        const float y = __shfl_xor_sync(kFull, eta_c, 1);
+        const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
+        if (part == 0) {
+          if (a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
+          *reinterpret_cast<uint4*>(smem + srg + tile_off(k, DV, K::RSV)) =
+              make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
+        }
+        float add = esum_c;
+        if (nv < C) {
+          double sr = 0.0, si = 0.0;
+          const double br = T->b[m].x, bi = T->b[m].y;
+          for (int j = 0; j < nv; ++j) {
+            const double e = exp((C / 2 - j) * T->re_dA[m]);
+            const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
+            double sn, cs;
+            sincos(ph, &sn, &cs);
+            const double pr = e * cs, pi = e * sn;
+            sr += br * pr - bi * pi;
+            si += br * pi + bi * pr;
+          }
+          add = static_cast<float>(comp ? si : sr);
+        }
+        eta_c = Re + add;
+      }
+      signal(0);
+      return true;
+    };
+    auto e3 = [&]() {   // masked P -> [i][j]
+      const int i = 16 * quad + lane;
+      uint32_t r[16];
+      tmem_ld16(trow + K::T_P + i0, r);
+      tmem_ld_wait16(r);
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (i0 + e > i) r[e] = 0u;
+        *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0, 1024)) = pack8f(r, 1.f);
+        *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
+      }
+      signal(3);
+    };
+    auto e4 = [&](int ch, int nv) {   // o = num / den, staged then written coalesced
+      const int n0 = ch * C;
+      const int i = 16 * quad + lane;
+      uint32_t rd[16];
+      tmem_ld16(trow + K::T_DEN, rd);
+      tmem_ld_wait16(rd);
+      uint32_t r[16];
+      tmem_ld16(trow + K::T_NUM + i0, r);
+      tmem_ld_wait16(r);
+      const float dn = __uint_as_float(rd[0]);
+      const float rdn = 1.0f / dn;
+      const long long row = bh * a.N + n0 + i;
+      if (lane < 16) {
+        if (i < nv && a.den && part == 0) a.den[row] = dn;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int chunk = (i0 >> 2) + g;
+          *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
+              make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                          __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
+        }
+        if (i < nv && a.num) {
+          float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+        }
+      }
+      named_sync(1, WS_ET);
+      constexpr int CPR = DV / 4;
+      float* obase = a.o + (bh * a.N + n0) * DV;
+      for (int c = tid; c < nv * CPR; c += WS_ET) {
+        const int rr = c / CPR, g = c % CPR;
+        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
+        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
+      }
+      named_sync(1, WS_ET);   // staging (sX) is read before E2 of the next chunk writes it
+    };
+
+    bool ok = true;
+    int prev = -1, prev_nv = C;
+    if (ch0 < ch1) ok = prepare(ch0, 0);
+    for (int t = ch0; ok && t < ch1; ++t) {
+      const int nv = min(C, a.N - t * C);
+      if (prev >= 0) {
+        if (!(ok = wait_dne(2))) break;   // G4(t-1)
+        e3();
+      }
+      if (!(ok = wait_dne(0))) break;     // G1 + G7(t)
+      {  // E1(t): masked S^T -> [j][i]
+        const int j = 16 * quad + lane;
+        uint32_t r[16];
+        tmem_ld16(trow + K::T_S + i0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          const bool keep = j < nv;
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (!(keep && i0 + e >= j)) r[e] = 0u;
+          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0, 1024)) = pack8f(r, 1.f);
+          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
+        }
+        signal(1);
+      }
+      if (prev >= 0) {
+        if (!(ok = wait_dne(3))) break;   // G5 + G6(t-1)
+        e4(prev, prev_nv);
+      }
+      if (!(ok = wait_dne(1))) break;     // G2 + G3(t)
+      {  // E2(t): X = |lambda|^(2(i-c)) a~
+        uint32_t r[16];
+        tmem_ld16(trow + K::T_A + i0, r);
+        tmem_ld_wait16(r);
+        float s = s_start;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
+          s *= r2;
+        }
+        *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0, 1024)) = pack8f(r, 1.f);
+        *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
+        signal(2);
+      }
+      prev = t;
+      prev_nv = nv;
+      if (t + 1 < ch1) ok = prepare(t + 1, (t + 1 - ch0) & 1);
+    }
+    if (ok && prev >= 0) {
+      if ((ok = wait_dne(2))) e3();
+      if (ok && (ok = wait_dne(3))) e4(prev, prev_nv);
+    }
+    if (ok && a.state_out && seg == a.nseg - 1) {
+      const int nv = nv_last;
+      const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
+      const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
+      double sn, cs;
+      sincos(ph, &sn, &cs);
+      const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
+#pragma unroll
+      for (int cb = 0; cb < FQ; cb += 16) {
+        const int col0 = part * FQ + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + K::T_STATE + col0, r);
+        tmem_ld_wait16(r);
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float x = __uint_as_float(r[e2]);
+          const float y = __shfl_xor_sync(kFull, x, 1);
+          if (comp == 0) {
+            const float2 z = make_float2(fr * x - fi * y, fr * y + fi * x);
+            const int f = col0 + e2;
+            if (f < DX) a.state_out[(bh * 64 + m) * DX + f] = z;
+            else a.state_out[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)] = z;
+          }
+        }
+      }
+      const float y = __shfl_xor_sync(kFull, eta_c, 1);
+      if (comp == 0 && part == 0)
+        a.state_out[a.BH * 64 * F + bh * 64 + m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -532,17 +1041,28 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
     auto k1 = tc_prefill_kernel<DX, DV, false>;
     e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
     if (e != cudaSuccess) return e;
-    k1<<<static_cast<unsigned>(args.BH * (p.nseg - 1)), NTHR, K::SMEM, st>>>(args);
+    k1<<<static_cast<unsigned>(args.BH * (p.nseg - 1)), NT, K::SMEM, st>>>(args);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = launch_segment_scan(s.B, s.H, DX, DV, p.nseg, p.seg_chunks * C, args.tabs, args.state_in,
                             args.seg_state, args.seg_eta, st);
     if (e != cudaSuccess) return e;
   }
+  if constexpr (DX == 64 && DV == 64) {
+    if (!std::getenv("IA_PREFILL_NO_WS")) {   // tuning switch: the single-role chunk loop
+      e = cudaFuncSetAttribute(tc_prefill_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WCfg::SMEM);
+      if (e != cudaSuccess) return e;
+      mark_launch_begin(st);
+      tc_prefill_ws_kernel<<<static_cast<unsigned>(args.BH * p.nseg), WS_NT, WCfg::SMEM, st>>>(args);
+      e = cudaGetLastError();
+      mark_launch_end(st);
+      return e;
+    }
+  }
   auto k3 = tc_prefill_kernel<DX, DV, true>;
   e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
   mark_launch_begin(st);
-  k3<<<static_cast<unsigned>(args.BH * p.nseg), NTHR, K::SMEM, st>>>(args);
+  k3<<<static_cast<unsigned>(args.BH * p.nseg), NT, K::SMEM, st>>>(args);
   e = cudaGetLastError();
   mark_launch_end(st);
   return e;
