@@ -89,15 +89,22 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   }
   for (int f = tid; f < DV; f += kDecThreads) vv[f] = ldx(v + bh * DV + f);
   for (int i = tid; i < MG; i += kDecThreads) {
+    // lambda = exp(Delta A), b = (lambda - 1)/A in fp32; lambda - 1 is formed
+    // as expm1(x) cos(y) - 2 sin^2(y/2) + i e^x sin(y) so it keeps its
+    // relative accuracy for small Delta.
     const int m = m0 + i;
-    double ar = A ? static_cast<double>(A[2 * m]) : -0.5;
-    double ai = A ? static_cast<double>(A[2 * m + 1]) : 3.14159265358979323846 * m;
-    double d = static_cast<double>(delta[h]), e = exp(d * ar), s, c;
-    sincos(d * ai, &s, &c);
-    double lr = e * c, li = e * s, nr = lr - 1.0, dd = ar * ar + ai * ai;
-    lamb[i] = make_float2(static_cast<float>(lr), static_cast<float>(li));
-    bb[i] = make_float2(static_cast<float>((nr * ar + li * ai) / dd),
-                        static_cast<float>((li * ar - nr * ai) / dd));
+    const float ar = A ? A[2 * m] : -0.5f;
+    const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
+    const float d = delta[h];
+    const float x = d * ar, y = d * ai;
+    float sy, cy, sh, ch;
+    sincosf(y, &sy, &cy);
+    sincosf(0.5f * y, &sh, &ch);
+    const float ex = expf(x), em1 = expm1f(x);
+    const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;   // lambda - 1
+    const float dd = fmaf(ar, ar, ai * ai);
+    lamb[i] = make_float2(ex * cy, ex * sy);
+    bb[i] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
   }
   for (int i = tid; i < 8 * DV + 8; i += kDecThreads) part[i] = 0.f;
   __syncthreads();
@@ -184,10 +191,173 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
   cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
 }
 
+// Large-batch variant: one CTA per (b,h) covers all modes, so no cluster and
+// no cross-CTA reduction is needed; each warp walks its modes with the next
+// mode's U / Gamma rows already in flight (one-deep prefetch), and keeps its
+// partial Re(a^H Gamma) in registers.
+constexpr int kBhWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
+    int H, int DX, int DV, int M, const T* __restrict__ q, const T* __restrict__ k,
+    const T* __restrict__ v, const float* __restrict__ delta, const float* __restrict__ A,
+    float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
+    float* __restrict__ den, long long BH) {
+  extern __shared__ float4 dsm[];
+  float* fq = reinterpret_cast<float*>(dsm);
+  float* fk = fq + DX;
+  float* vv = fk + DX;
+  float* part = vv + DV;                    // [8][DV]
+  float* pden = part + kBhWarps * DV;       // [8]
+  float2* lamb = reinterpret_cast<float2*>(pden + kBhWarps);   // [M]
+  float2* bb = lamb + M;
+  const long long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nu = DX / 2, ng = DV / 2;
+  float2* Ub = state + bh * M * DX;
+  float2* Gb = state + BH * M * DX + bh * M * DV;
+  float2* Eb = state + BH * M * (DX + DV) + bh * M;
+
+  float4 cu[kVecPerLane], cg[kVecPerLane], nu4[kVecPerLane], ng4[kVecPerLane];
+  auto load_mode = [&](int m, float4 (&u)[kVecPerLane], float4 (&g)[kVecPerLane]) {
+    const float4* Ur = reinterpret_cast<const float4*>(Ub + static_cast<long long>(m) * DX);
+    const float4* Gr = reinterpret_cast<const float4*>(Gb + static_cast<long long>(m) * DV);
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (p < nu) u[i] = Ur[p];
+      if (p < ng) g[i] = Gr[p];
+    }
+  };
+  if (warp < M) load_mode(warp, cu, cg);
+
+  for (int f = tid; f < DX; f += kBhWarps * 32) {
+    fq[f] = xi_acc(ldx(q + bh * DX + f));
+    fk[f] = xi_acc(ldx(k + bh * DX + f));
+  }
+  for (int f = tid; f < DV; f += kBhWarps * 32) vv[f] = ldx(v + bh * DV + f);
+  for (int m = tid; m < M; m += kBhWarps * 32) {
+    const float ar = A ? A[2 * m] : -0.5f;
+    const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
+    const float d = delta[h];
+    const float x = d * ar, y = d * ai;
+    float sy, cy, sh, ch;
+    sincosf(y, &sy, &cy);
+    sincosf(0.5f * y, &sh, &ch);
+    const float ex = expf(x), em1 = expm1f(x);
+    const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;
+    const float dd = fmaf(ar, ar, ai * ai);
+    lamb[m] = make_float2(ex * cy, ex * sy);
+    bb[m] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
+  }
+  __syncthreads();
+
+  float acc[2 * kVecPerLane];
+#pragma unroll
+  for (int i = 0; i < 2 * kVecPerLane; ++i) acc[i] = 0.f;
+  float dpart = 0.f;
+  for (int m = warp; m < M; m += kBhWarps) {
+    const bool more = m + kBhWarps < M;
+    if (more) load_mode(m + kBhWarps, nu4, ng4);
+    float2 e = make_float2(0.f, 0.f);
+    if (lane == 0) e = Eb[m];
+    const float2 L = lamb[m], Bm = bb[m];
+    float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
+    float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
+    float ar = 0.f, ai = 0.f;
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (p < nu) {
+        const float4 u = cu[i];
+        const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
+        float4 w;
+        w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
+        w.y = fmaf(L.x, u.y, fmaf(L.y, u.x, Bm.y * x0));
+        w.z = fmaf(L.x, u.z, fmaf(-L.y, u.w, Bm.x * x1));
+        w.w = fmaf(L.x, u.w, fmaf(L.y, u.z, Bm.y * x1));
+        Ur[p] = w;
+        ar = fmaf(w.x, fq[2 * p], fmaf(w.z, fq[2 * p + 1], ar));
+        ai = fmaf(w.y, fq[2 * p], fmaf(w.w, fq[2 * p + 1], ai));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      ar += __shfl_xor_sync(0xffffffffu, ar, off);
+      ai += __shfl_xor_sync(0xffffffffu, ai, off);
+    }
+#pragma unroll
+    for (int i = 0; i < kVecPerLane; ++i) {
+      const int p = lane + 32 * i;
+      if (p < ng) {
+        const float4 g = cg[i];
+        const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
+        float4 w;
+        w.x = fmaf(L.x, g.x, fmaf(-L.y, g.y, Bm.x * x0));
+        w.y = fmaf(L.x, g.y, fmaf(L.y, g.x, Bm.y * x0));
+        w.z = fmaf(L.x, g.z, fmaf(-L.y, g.w, Bm.x * x1));
+        w.w = fmaf(L.x, g.w, fmaf(L.y, g.z, Bm.y * x1));
+        Gr[p] = w;
+        acc[2 * i] = fmaf(ar, w.x, fmaf(ai, w.y, acc[2 * i]));        // Re(conj(a) Gamma)
+        acc[2 * i + 1] = fmaf(ar, w.z, fmaf(ai, w.w, acc[2 * i + 1]));
+      }
+    }
+    if (lane == 0) {
+      const float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
+      Eb[m] = w;
+      dpart = fmaf(ar, w.x, fmaf(ai, w.y, dpart));
+    }
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < kVecPerLane; ++i) {
+        cu[i] = nu4[i];
+        cg[i] = ng4[i];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kVecPerLane; ++i) {
+    const int p = lane + 32 * i;
+    if (p < ng) {
+      part[warp * DV + 2 * p] = acc[2 * i];
+      part[warp * DV + 2 * p + 1] = acc[2 * i + 1];
+    }
+  }
+  if (lane == 0) pden[warp] = dpart;
+  __syncthreads();
+  float dn = 0.f;
+  for (int w = 0; w < kBhWarps; ++w) dn += pden[w];
+  for (int f = tid; f < DV; f += kBhWarps * 32) {
+    float s = 0.f;
+    for (int w = 0; w < kBhWarps; ++w) s += part[w * DV + f];
+    o[bh * DV + f] = s / dn;
+    if (num) num[bh * DV + f] = s;
+  }
+  if (den && tid == 0) den[bh] = dn;
+}
+
 template <typename T>
 cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const void* v,
                         const float* delta, const float* A, void* state, float* o, float* num,
                         float* den, cudaStream_t st) {
+  const long long BHc = static_cast<long long>(s.B) * s.H;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (BHc >= 2LL * sms) {   // enough (b,h) pairs to fill the GPU without splitting modes
+    const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
+                        sizeof(float2) * 2 * s.M + 16;
+    auto kern = decode_bh_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    mark_launch_begin(st);
+    kern<<<static_cast<unsigned>(BHc), kBhWarps * 32, smem, st>>>(
+        s.H, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
+        static_cast<const T*>(v), delta, A, static_cast<float2*>(state), o, num, den, BHc);
+    e = cudaGetLastError();
+    mark_launch_end(st);
+    return e;
+  }
   // 16 modes (two per warp) per CTA, up to 8 CTAs per cluster
   const int G = (s.M + 15) / 16;
   const int MG = (s.M + G - 1) / G;
