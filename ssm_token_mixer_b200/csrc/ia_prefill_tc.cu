@@ -112,17 +112,17 @@ struct TcArgs {
 // iterations of 8 rows x 4 column groups, the column group rotated by the row
 // so that staging reads and tile writes are bank-conflict free; all loads of
 // a thread are issued before any conversion.
-template <int W, int WD, bool FEAT>
+template <int W, int WD, bool FEAT, int NW = NWARP>
 __device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, int nv, int warp, int lane) {
   constexpr int NCG = W / 8;
   constexpr int ITERS = (C / 8) * (NCG / 4);
-  constexpr int PER = (ITERS + NWARP - 1) / NWARP;
+  constexpr int PER = (ITERS + NW - 1) / NW;
   const int r8 = lane & 7, slot = lane >> 3;
   uint4 in[PER];
   int rr[PER], cc[PER];
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const int it = warp + u * NWARP;
+    const int it = warp + u * NW;
     const int rb = it & 7, rest = it >> 3;
     rr[u] = rb * 8 + r8;
     cc[u] = (rest >> 1) * 8 + ((slot + 4 * (rest & 1) + r8) & 7);
@@ -131,7 +131,7 @@ __device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, in
   }
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const int it = warp + u * NWARP;
+    const int it = warp + u * NW;
     if (it >= ITERS) break;
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (rr[u] < nv) {
@@ -832,12 +832,16 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
       convert_all<DX, DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
       convert_all<DX, DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
       convert_all<DV, K::WV, false>(smem + K::STG_V, smem + sv, nv, warp, lane);
+      static_assert(FQ == 32, "two 16-column blocks per thread");
+      uint32_t rs[2][16];
+      tmem_ld16(trow + K::T_STATE + part * FQ, rs[0]);
+      tmem_ld16(trow + K::T_STATE + part * FQ + 16, rs[1]);
+      tmem_ld_wait16(rs[0]);
+      tmem_ld_wait16(rs[1]);
 #pragma unroll
       for (int cb = 0; cb < FQ; cb += 16) {
         const int col0 = part * FQ + cb;
-        uint32_t rr[16];
-        tmem_ld16(trow + K::T_STATE + col0, rr);
-        tmem_ld_wait16(rr);
+        uint32_t (&rr)[16] = rs[cb / 16];
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -909,11 +913,10 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
     auto e4 = [&](int ch, int nv) {   // o = num / den, staged then written coalesced
       const int n0 = ch * C;
       const int i = 16 * quad + lane;
-      uint32_t rd[16];
+      uint32_t rd[16], r[16];
       tmem_ld16(trow + K::T_DEN, rd);
-      tmem_ld_wait16(rd);
-      uint32_t r[16];
       tmem_ld16(trow + K::T_NUM + i0, r);
+      tmem_ld_wait16(rd);
       tmem_ld_wait16(r);
       const float dn = __uint_as_float(rd[0]);
       const float rdn = 1.0f / dn;
@@ -1033,6 +1036,490 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------------------
+// Two-group warp-specialized full pass for d_xi = d_v = 64.  Three roles run
+// concurrently: 8 "prepare" warps (0-7) convert chunk t's inputs and rotate
+// the carried state into R(t); 8 "output" warps (8-15) run the masks,
+// readout scale and o = num/den of chunks t and t-1; warp 16 issues the
+// bulk copies and every tensor-core contraction.  Handover is by mbarriers:
+// ready(0) from the prepare warps, ready(1..3) from the output warps,
+// done(0..3) and the buffer releases (freeQK, freeVR) from tcgen05.commit.
+// Inputs, R_U, R_Gamma and R_eta are double-buffered by chunk parity; a
+// buffer is rewritten only after the commit that follows its last reader.
+constexpr int W2_GW = 8;                       // warps per epilogue group
+constexpr int W2_GT = W2_GW * 32;              // threads per epilogue group
+constexpr int W2_NT = 2 * W2_GT + 32;          // + one MMA / copy warp
+
+struct W2Cfg {
+  static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
+  static constexpr uint32_t RSX = DX * 16, RSV = WV * 16;
+  static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
+                            T_DEN = 320 + 64;
+  static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRU = KR * DX * 2, TRG = KR * WV * 2;
+  static constexpr uint32_t STG_Q = 0;
+  static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
+  static constexpr uint32_t STG_V = STG_K + C * DX * 2;
+  static constexpr uint32_t S_Q = STG_V + C * DV * 2;      // [2]
+  static constexpr uint32_t S_K = S_Q + 2 * TQ;            // [2]
+  static constexpr uint32_t S_V = S_K + 2 * TQ;            // [2]
+  static constexpr uint32_t S_E = S_V + 2 * TV;
+  static constexpr uint32_t S_S = S_E + KR * C * 2;
+  static constexpr uint32_t S_P = S_S + C * C * 2;
+  static constexpr uint32_t S_X = S_P + C * C * 2;
+  static constexpr uint32_t S_RU = S_X + KR * C * 2;       // [2]
+  static constexpr uint32_t S_RG = S_RU + 2 * TRU;         // [2]
+  static constexpr uint32_t S_BAR = S_RG + 2 * TRG;        // 14 mbarriers
+  static constexpr uint32_t S_FLAG = S_BAR + 128;
+  static constexpr uint32_t S_TMEMH = S_FLAG + 16;
+  static constexpr uint32_t SMEM = S_TMEMH + 16;
+  static constexpr uint32_t S_OUT = S_X;
+  static_assert(KR * C * 2 >= C * DV * 4, "output staging fits in sX");
+};
+
+__global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a) {
+  using K = W2Cfg;
+  constexpr int DX = K::DX, DV = K::DV, F = K::F;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int role = warp < W2_GW ? 0 : (warp < 2 * W2_GW ? 1 : 2);   // prepare, output, mma
+  const int gw = warp & (W2_GW - 1);          // warp index within its epilogue group
+  const int quad = warp & 3, half = gw >> 2;
+  const long long bh = blockIdx.x / a.nseg;
+  const int seg = static_cast<int>(blockIdx.x % a.nseg);
+  const int h = static_cast<int>(bh % a.H);
+  const HeadTables* T = a.tabs + h;
+  const int nch_total = (a.N + C - 1) / C;
+  const int ch0 = seg * a.seg_chunks;
+  const int ch1 = min(ch0 + a.seg_chunks, nch_total);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* bar_tma = bars + 0;
+  uint64_t* rdy = bars + 1;       // [4]
+  uint64_t* dne = bars + 5;       // [4]
+  uint64_t* freeQK = bars + 9;    // [2]: sQ, sK, sR_U of that parity may be rewritten
+  uint64_t* freeVR = bars + 11;   // [2]: sV, sR_Gamma of that parity may be rewritten
+  uint64_t* bar_drain = bars + 13;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
+  const uint32_t sbase = smem_u32(smem);
+  auto sQ = [&](int p) { return K::S_Q + p * K::TQ; };
+  auto sK = [&](int p) { return K::S_K + p * K::TQ; };
+  auto sV = [&](int p) { return K::S_V + p * K::TV; };
+  auto sRU = [&](int p) { return K::S_RU + p * K::TRU; };
+  auto sRG = [&](int p) { return K::S_RG + p * K::TRG; };
+
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_tma, 1);
+    mbar_init(rdy + 0, W2_GT);
+    for (int i = 1; i < 4; ++i) mbar_init(rdy + i, W2_GT);
+    for (int i = 0; i < 4; ++i) mbar_init(dne + i, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(freeQK + i, 1);
+      mbar_init(freeVR + i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(T->E);
+    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
+    for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
+    for (int r = tid; r < C; r += W2_NT) {
+      for (int p = 0; p < 2; ++p) {
+        *reinterpret_cast<uint4*>(smem + sV(p) + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sV(p) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    for (int r = tid; r < KR; r += W2_NT) {
+      for (int p = 0; p < 2; ++p) {
+        *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (role == 2) {
+    // ------------------------------------------------ MMA and copy issuer
+    if (lane == 0) {
+      uint32_t pr[4] = {0u, 0u, 0u, 0u};
+      int issued = 0;
+      bool ok = true;
+      auto issue_load = [&](int ch) {
+        const int n0 = ch * C;
+        const int nv = min(C, a.N - n0);
+        const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
+        mbar_arrive_expect_tx(bar_tma, 2 * bq + bv);
+        const long long row = bh * a.N + n0;
+        bulk_g2s(smem + K::STG_Q, a.q + row * DX, bq, bar_tma);
+        bulk_g2s(smem + K::STG_K, a.k + row * DX, bq, bar_tma);
+        bulk_g2s(smem + K::STG_V, a.v + row * DV, bv, bar_tma);
+        ++issued;
+      };
+      auto wait_rdy = [&](int i) -> bool {
+        const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
+        pr[i] ^= 1u;
+        tc_fence_after();
+        return r;
+      };
+      auto g5g6 = [&](int pp) {
+        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(pp), K::RSV, 128, 2 * K::RSV,
+             idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
+        gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, sbase + sRG(pp), K::RSV, 128, 2 * K::RSV,
+             idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
+        mma_commit(dne + 3);
+        mma_commit(freeVR + pp);
+      };
+      if (ch0 < ch1) issue_load(ch0);
+      for (int t = ch0; t < ch1; ++t) {
+        const int p = (t - ch0) & 1;
+        if (!(ok = wait_rdy(0))) break;
+        if (t + 1 < ch1) issue_load(t + 1);   // the prepare warps have consumed the staging
+        gemm(tmem + K::T_S, sbase + sK(p), 128, K::RSX, 256, sbase + sQ(p), 128, K::RSX, 256,
+             idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
+        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(p), K::RSX, 128,
+             2 * K::RSX, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
+        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(p), K::RSV, 128,
+             2 * K::RSV, idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
+        mma_commit(dne + 0);
+        if (t > ch0) {
+          if (!(ok = wait_rdy(3))) break;
+          g5g6(p ^ 1);
+        }
+        if (!(ok = wait_rdy(1))) break;
+        gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
+             idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
+        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(p), 128, K::RSX, 256,
+             idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
+        mma_commit(dne + 1);
+        mma_commit(freeQK + p);
+        if (!(ok = wait_rdy(2))) break;
+        gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
+             idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
+        mma_commit(dne + 2);
+      }
+      if (ok && ch0 < ch1) {
+        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) & 1);
+      }
+      if (!ok) {
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0u, a.err);
+        if (issued > 0) mbar_wait(bar_tma, static_cast<uint32_t>((issued - 1) & 1), a.err);
+      }
+    }
+    __syncwarp();
+  } else if (role == 0) {
+    // ------------------------------------------------ prepare warps
+    const int k = 32 * quad + lane;
+    const int m = k >> 1, comp = k & 1;
+    const float2 lamC = T->lamC[m];
+    const float sgnLi = comp ? lamC.y : -lamC.y;
+    const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    constexpr int FH = F / 2;   // state columns per thread
+    uint32_t ptma = 0u, pd0 = 0u, pfq[2] = {0u, 0u}, pfv[2] = {0u, 0u};
+    auto waitA = [&](uint64_t* bar, uint32_t& ph) -> bool {   // uniform over the prepare group
+      const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
+      ph ^= 1u;
+      tc_fence_after();
+      return !named_sync_or(2, W2_GT, !r);
+    };
+    float eta_c = 0.f;
+    {  // initial (scaled) state
+      const float* carry = nullptr;
+      const float* carry_eta = nullptr;
+      if (seg > 0) {
+        carry = a.seg_state + ((bh * (a.nseg - 1) + (seg - 1)) * KR + k) * F;
+        carry_eta = a.seg_eta + (bh * (a.nseg - 1) + (seg - 1)) * KR + k;
+      }
+      const bool from_in = seg == 0 && a.state_in != nullptr;
+      const float2 si = T->sc_inv[m];
+#pragma unroll
+      for (int cb = 0; cb < FH; cb += 16) {
+        const int col0 = half * FH + cb;
+        uint32_t r[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float val = 0.f;
+          const int f = col0 + e;
+          if (carry) {
+            val = carry[f];
+          } else if (from_in) {
+            float2 x = f < DX ? a.state_in[(bh * 64 + m) * DX + f]
+                              : a.state_in[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)];
+            val = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
+          }
+          r[e] = __float_as_uint(val);
+        }
+        tmem_st16(trow + K::T_STATE + col0, r);
+      }
+      if (carry_eta) {
+        eta_c = *carry_eta;
+      } else if (from_in) {
+        float2 x = a.state_in[a.BH * 64 * F + bh * 64 + m];
+        eta_c = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
+      }
+      tmem_st_wait();
+    }
+    bool ok = true;
+    int nv_last = C;
+    for (int t = ch0; t < ch1; ++t) {
+      const int rel = t - ch0, p = rel & 1;
+      const int nv = min(C, a.N - t * C);
+      nv_last = nv;
+      if (rel >= 2) {
+        if (!(ok = waitA(freeQK + p, pfq[p]))) break;
+        if (!(ok = waitA(freeVR + p, pfv[p]))) break;
+      }
+      if (!(ok = waitA(bar_tma, ptma))) break;
+      convert_all<DX, DX, true, W2_GW>(smem + K::STG_Q, smem + sQ(p), nv, gw, lane);
+      convert_all<DX, DX, true, W2_GW>(smem + K::STG_K, smem + sK(p), nv, gw, lane);
+      convert_all<DV, K::WV, false, W2_GW>(smem + K::STG_V, smem + sV(p), nv, gw, lane);
+      if (rel >= 1 && !(ok = waitA(dne + 0, pd0))) break;   // G7(t-1): the state is current
+#pragma unroll
+      for (int b = 0; b < FH / 16; ++b) {
+        const int col0 = half * FH + 16 * b;
+        uint32_t rs[16], w[16];
+        tmem_ld16(trow + K::T_STATE + col0, rs);
+        tmem_ld_wait16(rs);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float x = __uint_as_float(rs[e]);
+          const float y = __shfl_xor_sync(kFull, x, 1);
+          w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
+        }
+        tmem_st16(trow + K::T_STATE + col0, w);
+        if (a.dump_R) {
+          float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + t) * KR + k) * F + col0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
+                                __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
+        }
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint4 pk = pack8f(w + 8 * g, 1.f);
+          const int f = col0 + 8 * g;
+          if (f < DX)
+            *reinterpret_cast<uint4*>(smem + sRU(p) + tile_off(k, f, K::RSX)) = pk;
+          else
+            *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(k, f - DX, K::RSV)) = pk;
+        }
+      }
+      tmem_st_wait();
+      {
+        const float y = __shfl_xor_sync(kFull, eta_c, 1);
+        const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
+        if (half == 0) {
+          if (a.dump_Re) a.dump_Re[(bh * nch_total + t) * KR + k] = Re;
+          *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(k, DV, K::RSV)) =
+              make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
+        }
+        float add = esum_c;
+        if (nv < C) {
+          double sr = 0.0, si = 0.0;
+          const double br = T->b[m].x, bi = T->b[m].y;
+          for (int j = 0; j < nv; ++j) {
+            const double e = exp((C / 2 - j) * T->re_dA[m]);
+            const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
+            double sn, cs;
+            sincos(ph, &sn, &cs);
+            const double pr = e * cs, pi = e * sn;
+            sr += br * pr - bi * pi;
+            si += br * pi + bi * pr;
+          }
+          add = static_cast<float>(comp ? si : sr);
+        }
+        eta_c = Re + add;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(rdy + 0);
+    }
+    if (ok && ch0 < ch1 && a.state_out && seg == a.nseg - 1) {
+      ok = waitA(dne + 0, pd0);   // G7 of the last chunk
+      if (ok) {
+        const int nv = nv_last;
+        const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
+        const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
+        double sn, cs;
+        sincos(ph, &sn, &cs);
+        const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
+#pragma unroll
+        for (int cb = 0; cb < FH; cb += 16) {
+          const int col0 = half * FH + cb;
+          uint32_t r[16];
+          tmem_ld16(trow + K::T_STATE + col0, r);
+          tmem_ld_wait16(r);
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float x = __uint_as_float(r[e2]);
+            const float y = __shfl_xor_sync(kFull, x, 1);
+            if (comp == 0) {
+              const float2 z = make_float2(fr * x - fi * y, fr * y + fi * x);
+              const int f = col0 + e2;
+              if (f < DX) a.state_out[(bh * 64 + m) * DX + f] = z;
+              else a.state_out[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)] = z;
+            }
+          }
+        }
+        const float y = __shfl_xor_sync(kFull, eta_c, 1);
+        if (comp == 0 && half == 0)
+          a.state_out[a.BH * 64 * F + bh * 64 + m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
+      }
+    }
+  } else {
+    // ------------------------------------------------ output warps
+    const int btid = tid - W2_GT;
+    const int k = 32 * quad + lane;
+    const int m = k >> 1;
+    const float r2 = T->r2[m];
+    const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
+    const int i0 = 32 * half;     // this thread's 32 columns of the 64-wide tiles
+    uint32_t pd[4] = {0u, 0u, 0u, 0u};
+    auto waitB = [&](int i) -> bool {
+      const bool r = mbar_wait_or_abort(dne + i, pd[i], a.err, abort_flag);
+      pd[i] ^= 1u;
+      tc_fence_after();
+      return !named_sync_or(3, W2_GT, !r);
+    };
+    auto signalB = [&](int i) {
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(rdy + i);
+    };
+    auto e3 = [&]() {   // masked P -> [i][j]
+      const int i = 16 * quad + lane;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        uint32_t r[16];
+        tmem_ld16(trow + K::T_P + i0 + 16 * b, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (i0 + 16 * b + e > i) r[e] = 0u;
+          *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
+          *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
+        }
+      }
+      signalB(3);
+    };
+    auto e4 = [&](int ch, int nv) {   // o = num / den, staged then written coalesced
+      const int n0 = ch * C;
+      const int i = 16 * quad + lane;
+      uint32_t rd;
+      tmem_ld1(trow + K::T_DEN, rd);
+      tmem_ld_wait1(rd);
+      const float dn = __uint_as_float(rd);
+      const float rdn = 1.0f / dn;
+      const long long row = bh * a.N + n0 + i;
+      if (lane < 16 && i < nv && a.den && half == 0) a.den[row] = dn;
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        uint32_t r[16];
+        tmem_ld16(trow + K::T_NUM + i0 + 16 * b, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int chunk = ((i0 + 16 * b) >> 2) + g;
+            *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
+                make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                            __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
+          }
+          if (i < nv && a.num) {
+            float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0 + 16 * b);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                  __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+          }
+        }
+      }
+      named_sync(1, W2_GT);
+      constexpr int CPR = DV / 4;
+      float* obase = a.o + (bh * a.N + n0) * DV;
+      for (int c = btid; c < nv * CPR; c += W2_GT) {
+        const int rr = c / CPR, g = c % CPR;
+        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
+        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
+      }
+      named_sync(1, W2_GT);   // staging (sX) is read before E2 writes it
+    };
+    bool ok = true;
+    int prev = -1, prev_nv = C;
+    // t == ch1 runs only the tail (E3, E4) of the last chunk
+    for (int t = ch0; ok && t <= ch1 && ch0 < ch1; ++t) {
+      const bool head = t < ch1;
+      const int nv = head ? min(C, a.N - t * C) : 0;
+      if (prev >= 0) {
+        if (!(ok = waitB(2))) break;   // G4(t-1)
+        e3();
+      }
+      if (head) {
+        if (!(ok = waitB(0))) break;   // G1 + G7(t)
+        {  // E1(t): masked S^T -> [j][i]
+          const int j = 16 * quad + lane;
+          const bool keep = j < nv;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            uint32_t r[16];
+            tmem_ld16(trow + K::T_S + i0 + 16 * b, r);
+            tmem_ld_wait16(r);
+            if (lane < 16) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                if (!(keep && i0 + 16 * b + e >= j)) r[e] = 0u;
+              *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
+              *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
+            }
+          }
+          signalB(1);
+        }
+      }
+      if (prev >= 0) {
+        if (!(ok = waitB(3))) break;   // G5 + G6(t-1)
+        e4(prev, prev_nv);
+      }
+      if (head) {
+        if (!(ok = waitB(1))) break;   // G2 + G3(t)
+        {  // E2(t): X = |lambda|^(2(i-c)) a~
+          float s = s_start;
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            uint32_t r[16];
+            tmem_ld16(trow + K::T_A + i0 + 16 * b, r);
+            tmem_ld_wait16(r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
+              s *= r2;
+            }
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
+          }
+          signalB(2);
+        }
+      }
+      prev = t;
+      prev_nv = nv;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 template <int DX, int DV>
 cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p, cudaStream_t st) {
   using K = Cfg<DX, DV>;
@@ -1048,7 +1535,17 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
     if (e != cudaSuccess) return e;
   }
   if constexpr (DX == 64 && DV == 64) {
-    if (!std::getenv("IA_PREFILL_NO_WS")) {   // tuning switch: the single-role chunk loop
+    const char* ws = std::getenv("IA_PREFILL_WS");   // tuning switch: 0 plain loop, 1 one epilogue group
+    if (!ws || std::atoi(ws) >= 2) {
+      e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
+      if (e != cudaSuccess) return e;
+      mark_launch_begin(st);
+      tc_prefill_ws2_kernel<<<static_cast<unsigned>(args.BH * p.nseg), W2_NT, W2Cfg::SMEM, st>>>(args);
+      e = cudaGetLastError();
+      mark_launch_end(st);
+      return e;
+    }
+    if (std::atoi(ws) == 1) {
       e = cudaFuncSetAttribute(tc_prefill_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WCfg::SMEM);
       if (e != cudaSuccess) return e;
       mark_launch_begin(st);

@@ -95,6 +95,29 @@ def test_state_in_and_split_prefill(oracle_mod, dev, dtype, tol):
     check_state(r2["state"], oracle_mod.split_state(ref["state"], B, H, M, d, d), B, H, M, d, d, tol)
 
 
+@pytest.mark.parametrize("variant", ["0", "1", "2"])
+@pytest.mark.parametrize("N,with_state", [(1, False), (37, True), (200, False), (1000, True)])
+def test_d64_chunk_pass_variants(oracle_mod, dev, monkeypatch, variant, N, with_state):
+    # the three d=64 full-pass kernels (one role for all warps, one epilogue
+    # group beside the MMA warp, two epilogue groups) against the oracle, on
+    # ragged lengths, a carried state and (N=1000, B*H=2) split segments
+    monkeypatch.setenv("IA_PREFILL_WS", variant)
+    B, H, d, M = 1, 2, 64, 64
+    N0 = 75 if with_state else 0
+    inp = synthetic.layer_inputs(B, H, N0 + N, d, d, "bf16", seed=31 + N)
+    st = None
+    if with_state:
+        head = {k: (v[:, :, :N0].contiguous() if k != "delta" else v) for k, v in inp.items()}
+        st = gpu_prefill(head, M, dev)["state"].to(dev)
+    tail = {k: (v[:, :, N0:].contiguous() if k != "delta" else v) for k, v in inp.items()}
+    r = gpu_prefill(tail, M, dev, state_in=st)
+    ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
+    ref_tail = {"num": ref["num"][:, :, N0:], "den": ref["den"][:, :, N0:], "o": ref["o"][:, :, N0:]}
+    rep = report(r["num"], r["den"], r["o"], ref_tail)
+    assert max(rep.values()) < TOL_BF16, rep
+    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, d, d), B, H, M, d, d, TOL_BF16)
+
+
 def test_first_token_returns_v(dev):
     # P3 on the GPU path: o_1 = v_1 whatever q_1 and k_1
     inp = synthetic.layer_inputs(3, 4, 70, 64, 64, "bf16", seed=3)
