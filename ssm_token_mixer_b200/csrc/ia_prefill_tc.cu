@@ -149,6 +149,56 @@ __device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, in
   }
 }
 
+// convert_all for the three input tiles of one chunk at once (q and k through
+// the feature map, v plain): every load is issued before the first convert,
+// so the shared-memory latency is paid once.
+template <int D, int WDV, int NW>
+__device__ __forceinline__ void convert_qkv(const uint8_t* stg_q, const uint8_t* stg_k,
+                                            const uint8_t* stg_v, uint8_t* dq, uint8_t* dk,
+                                            uint8_t* dv, int nv, int warp, int lane) {
+  constexpr int NCG = D / 8;
+  constexpr int ITERS = (C / 8) * (NCG / 4);
+  static_assert(ITERS % NW == 0, "whole iterations per warp");
+  constexpr int PER = ITERS / NW;
+  const int r8 = lane & 7, slot = lane >> 3;
+  uint4 in[3][PER];
+  int rr[PER], cc[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int it = warp + u * NW;
+    const int rb = it & 7, rest = it >> 3;
+    rr[u] = rb * 8 + r8;
+    cc[u] = (rest >> 1) * 8 + ((slot + 4 * (rest & 1) + r8) & 7);
+    const int off = rr[u] * (D * 2) + cc[u] * 16;
+    const bool live = rr[u] < nv;
+    in[0][u] = live ? *reinterpret_cast<const uint4*>(stg_q + off) : make_uint4(0u, 0u, 0u, 0u);
+    in[1][u] = live ? *reinterpret_cast<const uint4*>(stg_k + off) : make_uint4(0u, 0u, 0u, 0u);
+    in[2][u] = live ? *reinterpret_cast<const uint4*>(stg_v + off) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int tsel = 0; tsel < 3; ++tsel) {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      uint4 out = make_uint4(0u, 0u, 0u, 0u);
+      if (rr[u] < nv) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&in[tsel][u]);
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = __bfloat1622float2(p[e]);
+          if (tsel < 2) { f.x = feat(f.x); f.y = feat(f.y); }
+          w[e] = pack_half2(f.x, f.y);
+        }
+        out = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (tsel == 2)
+        *reinterpret_cast<uint4*>(dv + tile_off(rr[u], cc[u] * 8, WDV * 16)) = out;
+      else
+        *reinterpret_cast<uint4*>((tsel ? dk : dq) + tile_off(rr[u], cc[u] * 8, D * 16)) = out;
+    }
+  }
+}
+
 __device__ __forceinline__ uint4 pack8f(const uint32_t* r, float scale) {
   return make_uint4(pack_half2(__uint_as_float(r[0]) * scale, __uint_as_float(r[1]) * scale),
                     pack_half2(__uint_as_float(r[2]) * scale, __uint_as_float(r[3]) * scale),
@@ -1037,18 +1087,21 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
 }
 
 // ---------------------------------------------------------------------------
-// Two-group warp-specialized full pass for d_xi = d_v = 64.  Three roles run
-// concurrently: 8 "prepare" warps (0-7) convert chunk t's inputs and rotate
-// the carried state into R(t); 8 "output" warps (8-15) run the masks,
-// readout scale and o = num/den of chunks t and t-1; warp 16 issues the
-// bulk copies and every tensor-core contraction.  Handover is by mbarriers:
-// ready(0) from the prepare warps, ready(1..3) from the output warps,
-// done(0..3) and the buffer releases (freeQK, freeVR) from tcgen05.commit.
-// Inputs, R_U, R_Gamma and R_eta are double-buffered by chunk parity; a
-// buffer is rewritten only after the commit that follows its last reader.
+// Two-group warp-specialized full pass for d_xi = d_v = 64.  Four roles run
+// concurrently: 8 "prepare" warps (0-7) convert the inputs and rotate the
+// carried state into R(t); 8 "output" warps (8-15) run the masks, readout
+// scale and o = num/den of chunks t and t-1; warp 16 issues every
+// tensor-core contraction; warp 17 copies q, k, v rows with cp.async straight
+// into the operand layout, where the prepare warps convert them in place, so
+// there is no staging area.  q, k, v and R_Gamma have three buffer sets and
+// R_U two: the fetch warp refills a set as soon as the contractions of the
+// chunk it held are done, about two chunks ahead of its use.  Handover is by
+// mbarriers: loaded(set) from the copies, ready(0) from the prepare warps,
+// ready(1..3) from the output warps, done(0..3) and the buffer releases
+// (freeQK after G2+G3, freeVR after G5+G6) from tcgen05.commit.
 constexpr int W2_GW = 8;                       // warps per epilogue group
 constexpr int W2_GT = W2_GW * 32;              // threads per epilogue group
-constexpr int W2_NT = 2 * W2_GT + 32;          // + one MMA / copy warp
+constexpr int W2_NT = 2 * W2_GT + 64;          // + the MMA warp and the fetch warp
 
 struct W2Cfg {
   static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
@@ -1056,32 +1109,29 @@ struct W2Cfg {
   static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
                             T_DEN = 320 + 64;
   static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRU = KR * DX * 2, TRG = KR * WV * 2;
-  static constexpr uint32_t STG_Q = 0;
-  static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
-  static constexpr uint32_t STG_V = STG_K + C * DX * 2;
-  static constexpr uint32_t S_Q = STG_V + C * DV * 2;      // [2]
-  static constexpr uint32_t S_K = S_Q + 2 * TQ;            // [2]
-  static constexpr uint32_t S_V = S_K + 2 * TQ;            // [2]
-  static constexpr uint32_t S_E = S_V + 2 * TV;
+  static constexpr int NB = 3;                             // q, k, v and R_Gamma buffer sets
+  static constexpr uint32_t S_Q = 0;                       // [NB]
+  static constexpr uint32_t S_K = S_Q + NB * TQ;           // [NB]
+  static constexpr uint32_t S_V = S_K + NB * TQ;           // [NB]
+  static constexpr uint32_t S_E = S_V + NB * TV;
   static constexpr uint32_t S_S = S_E + KR * C * 2;
   static constexpr uint32_t S_P = S_S + C * C * 2;
   static constexpr uint32_t S_X = S_P + C * C * 2;
   static constexpr uint32_t S_RU = S_X + KR * C * 2;       // [2]
-  static constexpr uint32_t S_RG = S_RU + 2 * TRU;         // [2]
-  static constexpr uint32_t S_BAR = S_RG + 2 * TRG;        // 14 mbarriers
-  static constexpr uint32_t S_FLAG = S_BAR + 128;
+  static constexpr uint32_t S_RG = S_RU + 2 * TRU;         // [NB]
+  static constexpr uint32_t S_BAR = S_RG + NB * TRG;       // 18 mbarriers
+  static constexpr uint32_t S_FLAG = S_BAR + 256;
   static constexpr uint32_t S_TMEMH = S_FLAG + 16;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
-  static constexpr uint32_t S_OUT = S_X;
-  static_assert(KR * C * 2 >= C * DV * 4, "output staging fits in sX");
+  static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
 };
 
 __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a) {
   using K = W2Cfg;
-  constexpr int DX = K::DX, DV = K::DV, F = K::F;
+  constexpr int DX = K::DX, DV = K::DV, F = K::F, NB = K::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int role = warp < W2_GW ? 0 : (warp < 2 * W2_GW ? 1 : 2);   // prepare, output, mma
+  const int role = warp < 2 * W2_GW ? warp / W2_GW : warp - 2 * W2_GW + 2;   // prepare, output, mma, fetch
   const int gw = warp & (W2_GW - 1);          // warp index within its epilogue group
   const int quad = warp & 3, half = gw >> 2;
   const long long bh = blockIdx.x / a.nseg;
@@ -1093,33 +1143,34 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
   const int ch1 = min(ch0 + a.seg_chunks, nch_total);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
-  uint64_t* bar_tma = bars + 0;
-  uint64_t* rdy = bars + 1;       // [4]
-  uint64_t* dne = bars + 5;       // [4]
-  uint64_t* freeQK = bars + 9;    // [2]: sQ, sK, sR_U of that parity may be rewritten
-  uint64_t* freeVR = bars + 11;   // [2]: sV, sR_Gamma of that parity may be rewritten
-  uint64_t* bar_drain = bars + 13;
+  uint64_t* rdy = bars + 0;       // [4]
+  uint64_t* dne = bars + 4;       // [4]
+  uint64_t* freeQK = bars + 8;    // [NB]: sQ, sK of that set (and the sR_U it was read with) reusable
+  uint64_t* freeVR = bars + 11;   // [NB]: sV, sR_Gamma of that set reusable
+  uint64_t* bar_drain = bars + 14;
+  uint64_t* loaded = bars + 15;   // [NB]: that set's q, k, v rows have landed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
   const uint32_t sbase = smem_u32(smem);
-  auto sQ = [&](int p) { return K::S_Q + p * K::TQ; };
-  auto sK = [&](int p) { return K::S_K + p * K::TQ; };
-  auto sV = [&](int p) { return K::S_V + p * K::TV; };
+  auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
+  auto sK = [&](int b) { return K::S_K + b * K::TQ; };
+  auto sV = [&](int b) { return K::S_V + b * K::TV; };
   auto sRU = [&](int p) { return K::S_RU + p * K::TRU; };
-  auto sRG = [&](int p) { return K::S_RG + p * K::TRG; };
+  auto sRG = [&](int b) { return K::S_RG + b * K::TRG; };
 
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar_tma, 1);
-    mbar_init(rdy + 0, W2_GT);
-    for (int i = 1; i < 4; ++i) mbar_init(rdy + i, W2_GT);
-    for (int i = 0; i < 4; ++i) mbar_init(dne + i, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(rdy + i, W2_GT);
+      mbar_init(dne + i, 1);
+    }
+    for (int i = 0; i < NB; ++i) {
       mbar_init(freeQK + i, 1);
       mbar_init(freeVR + i, 1);
+      mbar_init(loaded + i, 32);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -1129,16 +1180,17 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
     const uint4* src = reinterpret_cast<const uint4*>(T->E);
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
     for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
+    // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
     for (int r = tid; r < C; r += W2_NT) {
-      for (int p = 0; p < 2; ++p) {
-        *reinterpret_cast<uint4*>(smem + sV(p) + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sV(p) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      for (int b = 0; b < NB; ++b) {
+        *reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     for (int r = tid; r < KR; r += W2_NT) {
-      for (int p = 0; p < 2; ++p) {
-        *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      for (int b = 0; b < NB; ++b) {
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
@@ -1148,71 +1200,56 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
   const uint32_t tmem = *tmem_holder;
 
   if (role == 2) {
-    // ------------------------------------------------ MMA and copy issuer
+    // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t pr[4] = {0u, 0u, 0u, 0u};
-      int issued = 0;
       bool ok = true;
-      auto issue_load = [&](int ch) {
-        const int n0 = ch * C;
-        const int nv = min(C, a.N - n0);
-        const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
-        mbar_arrive_expect_tx(bar_tma, 2 * bq + bv);
-        const long long row = bh * a.N + n0;
-        bulk_g2s(smem + K::STG_Q, a.q + row * DX, bq, bar_tma);
-        bulk_g2s(smem + K::STG_K, a.k + row * DX, bq, bar_tma);
-        bulk_g2s(smem + K::STG_V, a.v + row * DV, bv, bar_tma);
-        ++issued;
-      };
       auto wait_rdy = [&](int i) -> bool {
         const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
         pr[i] ^= 1u;
         tc_fence_after();
         return r;
       };
-      auto g5g6 = [&](int pp) {
-        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(pp), K::RSV, 128, 2 * K::RSV,
+      auto g5g6 = [&](int bb) {
+        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(bb), K::RSV, 128, 2 * K::RSV,
              idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
-        gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, sbase + sRG(pp), K::RSV, 128, 2 * K::RSV,
+        gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, sbase + sRG(bb), K::RSV, 128, 2 * K::RSV,
              idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
         mma_commit(dne + 3);
-        mma_commit(freeVR + pp);
+        mma_commit(freeVR + bb);
       };
-      if (ch0 < ch1) issue_load(ch0);
       for (int t = ch0; t < ch1; ++t) {
-        const int p = (t - ch0) & 1;
+        const int rel = t - ch0, b = rel % NB, p = rel & 1;
         if (!(ok = wait_rdy(0))) break;
-        if (t + 1 < ch1) issue_load(t + 1);   // the prepare warps have consumed the staging
-        gemm(tmem + K::T_S, sbase + sK(p), 128, K::RSX, 256, sbase + sQ(p), 128, K::RSX, 256,
+        gemm(tmem + K::T_S, sbase + sK(b), 128, K::RSX, 256, sbase + sQ(b), 128, K::RSX, 256,
              idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
-        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(p), K::RSX, 128,
+        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(b), K::RSX, 128,
              2 * K::RSX, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
-        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(p), K::RSV, 128,
+        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(b), K::RSV, 128,
              2 * K::RSV, idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
         mma_commit(dne + 0);
         if (t > ch0) {
           if (!(ok = wait_rdy(3))) break;
-          g5g6(p ^ 1);
+          g5g6((rel + NB - 1) % NB);
         }
         if (!(ok = wait_rdy(1))) break;
         gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
              idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
-        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(p), 128, K::RSX, 256,
+        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(b), 128, K::RSX, 256,
              idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
         mma_commit(dne + 1);
-        mma_commit(freeQK + p);
+        mma_commit(freeQK + b);
         if (!(ok = wait_rdy(2))) break;
         gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
              idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
         mma_commit(dne + 2);
       }
       if (ok && ch0 < ch1) {
-        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) & 1);
+        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) % NB);
       }
-      if (!ok) {
+      if (!ok) {   // drain every tensor-core group issued so far
         mma_commit(bar_drain);
         mbar_wait(bar_drain, 0u, a.err);
-        if (issued > 0) mbar_wait(bar_tma, static_cast<uint32_t>((issued - 1) & 1), a.err);
       }
     }
     __syncwarp();
@@ -1225,12 +1262,46 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
     const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     constexpr int FH = F / 2;   // state columns per thread
-    uint32_t ptma = 0u, pd0 = 0u, pfq[2] = {0u, 0u}, pfv[2] = {0u, 0u};
+    uint32_t pd0 = 0u, pld[NB] = {0u, 0u, 0u};
     auto waitA = [&](uint64_t* bar, uint32_t& ph) -> bool {   // uniform over the prepare group
       const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
       ph ^= 1u;
       tc_fence_after();
       return !named_sync_or(2, W2_GT, !r);
+    };
+    // 16-byte pieces of a 64 x 64 input tile: piece = row%8 | col-block << 3 | row/8 << 6
+    auto piece = [](int pc, int& r, int& cb) {
+      r = (pc >> 6) * 8 + (pc & 7);
+      cb = (pc >> 3) & 7;
+    };
+    // bf16 -> fp16 in place (q, k through the feature map); rows past the
+    // sequence become 0
+    auto convert = [&](int nv, int b) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        int r, cb;
+        piece(tid + u * W2_GT, r, cb);   // this thread converts pieces tid, tid + 256
+        uint4* ptr[3] = {reinterpret_cast<uint4*>(smem + sQ(b) + tile_off(r, cb * 8, K::RSX)),
+                         reinterpret_cast<uint4*>(smem + sK(b) + tile_off(r, cb * 8, K::RSX)),
+                         reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, cb * 8, K::RSV))};
+        uint4 in[3] = {*ptr[0], *ptr[1], *ptr[2]};
+#pragma unroll
+        for (int tsel = 0; tsel < 3; ++tsel) {
+          uint4 out = make_uint4(0u, 0u, 0u, 0u);
+          if (r < nv) {
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[tsel]);
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float2 f = __bfloat1622float2(x2[e]);
+              if (tsel < 2) { f.x = feat(f.x); f.y = feat(f.y); }
+              w[e] = pack_half2(f.x, f.y);
+            }
+            out = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          *ptr[tsel] = out;
+        }
+      }
     };
     float eta_c = 0.f;
     {  // initial (scaled) state
@@ -1272,21 +1343,15 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
     bool ok = true;
     int nv_last = C;
     for (int t = ch0; t < ch1; ++t) {
-      const int rel = t - ch0, p = rel & 1;
+      const int rel = t - ch0, b = rel % NB, p = rel & 1;
       const int nv = min(C, a.N - t * C);
       nv_last = nv;
-      if (rel >= 2) {
-        if (!(ok = waitA(freeQK + p, pfq[p]))) break;
-        if (!(ok = waitA(freeVR + p, pfv[p]))) break;
-      }
-      if (!(ok = waitA(bar_tma, ptma))) break;
-      convert_all<DX, DX, true, W2_GW>(smem + K::STG_Q, smem + sQ(p), nv, gw, lane);
-      convert_all<DX, DX, true, W2_GW>(smem + K::STG_K, smem + sK(p), nv, gw, lane);
-      convert_all<DV, K::WV, false, W2_GW>(smem + K::STG_V, smem + sV(p), nv, gw, lane);
+      if (!(ok = waitA(loaded + b, pld[b]))) break;
+      convert(nv, b);
       if (rel >= 1 && !(ok = waitA(dne + 0, pd0))) break;   // G7(t-1): the state is current
 #pragma unroll
-      for (int b = 0; b < FH / 16; ++b) {
-        const int col0 = half * FH + 16 * b;
+      for (int blk = 0; blk < FH / 16; ++blk) {
+        const int col0 = half * FH + 16 * blk;
         uint32_t rs[16], w[16];
         tmem_ld16(trow + K::T_STATE + col0, rs);
         tmem_ld_wait16(rs);
@@ -1311,7 +1376,7 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
           if (f < DX)
             *reinterpret_cast<uint4*>(smem + sRU(p) + tile_off(k, f, K::RSX)) = pk;
           else
-            *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(k, f - DX, K::RSV)) = pk;
+            *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, f - DX, K::RSV)) = pk;
         }
       }
       tmem_st_wait();
@@ -1320,7 +1385,7 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
         const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
         if (half == 0) {
           if (a.dump_Re) a.dump_Re[(bh * nch_total + t) * KR + k] = Re;
-          *reinterpret_cast<uint4*>(smem + sRG(p) + tile_off(k, DV, K::RSV)) =
+          *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, DV, K::RSV)) =
               make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
         }
         float add = esum_c;
@@ -1376,9 +1441,8 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
           a.state_out[a.BH * 64 * F + bh * 64 + m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
       }
     }
-  } else {
+  } else if (role == 1) {
     // ------------------------------------------------ output warps
-    const int btid = tid - W2_GT;
     const int k = 32 * quad + lane;
     const int m = k >> 1;
     const float r2 = T->r2[m];
@@ -1414,30 +1478,28 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
       }
       signalB(3);
     };
-    auto e4 = [&](int ch, int nv) {   // o = num / den, staged then written coalesced
-      const int n0 = ch * C;
+    auto e4 = [&](int ch, int nv) {   // o = num / den, written straight from registers
       const int i = 16 * quad + lane;
       uint32_t rd;
       tmem_ld1(trow + K::T_DEN, rd);
       tmem_ld_wait1(rd);
       const float dn = __uint_as_float(rd);
       const float rdn = 1.0f / dn;
-      const long long row = bh * a.N + n0 + i;
-      if (lane < 16 && i < nv && a.den && half == 0) a.den[row] = dn;
+      const long long row = bh * a.N + ch * C + i;
+      const bool live = lane < 16 && i < nv;
+      if (live && a.den && half == 0) a.den[row] = dn;
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         uint32_t r[16];
         tmem_ld16(trow + K::T_NUM + i0 + 16 * b, r);
         tmem_ld_wait16(r);
-        if (lane < 16) {
+        if (live) {
+          float4* op = reinterpret_cast<float4*>(a.o + row * DV + i0 + 16 * b);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int chunk = ((i0 + 16 * b) >> 2) + g;
-            *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
-                make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                            __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-          }
-          if (i < nv && a.num) {
+          for (int g = 0; g < 4; ++g)
+            op[g] = make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                                __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
+          if (a.num) {
             float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0 + 16 * b);
 #pragma unroll
             for (int g = 0; g < 4; ++g)
@@ -1446,15 +1508,6 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
           }
         }
       }
-      named_sync(1, W2_GT);
-      constexpr int CPR = DV / 4;
-      float* obase = a.o + (bh * a.N + n0) * DV;
-      for (int c = btid; c < nv * CPR; c += W2_GT) {
-        const int rr = c / CPR, g = c % CPR;
-        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
-        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
-      }
-      named_sync(1, W2_GT);   // staging (sX) is read before E2 writes it
     };
     bool ok = true;
     int prev = -1, prev_nv = C;
@@ -1514,6 +1567,34 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
       prev = t;
       prev_nv = nv;
     }
+  }
+  if (role == 3) {
+    // ------------------------------------------------ fetch warp
+    uint32_t pfq[NB] = {0u, 0u, 0u}, pfv[NB] = {0u, 0u, 0u};
+    for (int t = ch0; t < ch1; ++t) {
+      const int rel = t - ch0, b = rel % NB;
+      if (rel >= NB) {   // set b last held chunk t-3: wait until its contractions are done
+        bool ok = mbar_wait_or_abort(freeQK + b, pfq[b], a.err, abort_flag);
+        pfq[b] ^= 1u;
+        if (ok) ok = mbar_wait_or_abort(freeVR + b, pfv[b], a.err, abort_flag);
+        pfv[b] ^= 1u;
+        if (!__all_sync(kFull, ok)) break;
+      }
+      const int n0 = t * C;
+      const int nv = min(C, a.N - n0);
+#pragma unroll 4
+      for (int u = 0; u < C * DX / 8 / 32; ++u) {
+        const int pc = lane + 32 * u;
+        const int r = (pc >> 6) * 8 + (pc & 7), cb = (pc >> 3) & 7;
+        const uint32_t bytes = r < nv ? 16u : 0u;   // rows past the sequence are zero-filled
+        const long long g = (bh * a.N + n0 + (r < nv ? r : 0)) * DX + cb * 8;
+        cp_async16(sbase + sQ(b) + tile_off(r, cb * 8, K::RSX), a.q + g, bytes);
+        cp_async16(sbase + sK(b) + tile_off(r, cb * 8, K::RSX), a.k + g, bytes);
+        cp_async16(sbase + sV(b) + tile_off(r, cb * 8, K::RSV), a.v + g, bytes);
+      }
+      cp_async_mbar_arrive(loaded + b);
+    }
+    cp_async_wait_all();   // nothing of ours lands after the block exits
   }
   tc_fence_before();
   __syncthreads();
