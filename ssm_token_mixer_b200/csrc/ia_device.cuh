@@ -134,6 +134,19 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 // Waits for every cp.async this thread has committed.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// TMA tensor load of one box (4-D tensor map) into shared memory, completing
+// on an mbarrier with the box's bytes as transaction count.  tmap is the
+// address of a __grid_constant__ CUtensorMap parameter; c0 * element size is
+// a multiple of 16 bytes.  Plain (non-multicast) form.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

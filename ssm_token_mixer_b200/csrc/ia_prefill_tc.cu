@@ -37,6 +37,8 @@
 // combines them (S_in(s+1) = lambda^L S_in(s) + S_local(s)), and the full
 // pass recomputes every segment from its carried-in state -- the two
 // parallel passes around a sequential carry pass of the summary's sec. A.2.
+#include <cuda.h>
+
 #include <cmath>
 #include <cstdlib>
 
@@ -1091,9 +1093,12 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
 // concurrently: 8 "prepare" warps (0-7) convert the inputs and rotate the
 // carried state into R(t); 8 "output" warps (8-15) run the masks, readout
 // scale and o = num/den of chunks t and t-1; warp 16 issues every
-// tensor-core contraction; warp 17 copies q, k, v rows with cp.async straight
-// into the operand layout, where the prepare warps convert them in place, so
-// there is no staging area.  q, k, v and R_Gamma have three buffer sets and
+// tensor-core contraction; warp 17 brings q, k, v in with TMA tensor loads
+// that land directly in the operand layout, where the prepare warps convert
+// them in place, so there is no staging area.  The tensor map views a
+// [rows][64] bf16 input as [column block][row][8 elements], so a 64-row box
+// arrives as core matrices of 8 rows x 16 bytes: row groups 128 bytes apart,
+// column blocks 1024 bytes apart.  Rows past the sequence arrive as zeros.  q, k, v and R_Gamma have three buffer sets and
 // R_U two: the fetch warp refills a set as soon as the contractions of the
 // chunk it held are done, about two chunks ahead of its use.  Handover is by
 // mbarriers: loaded(set) from the copies, ready(0) from the prepare warps,
@@ -1110,6 +1115,11 @@ struct W2Cfg {
                             T_DEN = 320 + 64;
   static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRU = KR * DX * 2, TRG = KR * WV * 2;
   static constexpr int NB = 3;                             // q, k, v and R_Gamma buffer sets
+  static constexpr uint32_t TIN = C * 64 * 2;              // bytes of one TMA box (64 rows x 64 bf16)
+  // q, k, v tiles: column block cb of row r at cb * 1024 + r * 16; K-major
+  // operands step 1024 bytes along K and 128 along M/N, MN-major ones 128
+  // along K and 1024 along M/N
+  static constexpr uint32_t IN_CB = C * 16, IN_RG = 128;
   static constexpr uint32_t S_Q = 0;                       // [NB]
   static constexpr uint32_t S_K = S_Q + NB * TQ;           // [NB]
   static constexpr uint32_t S_V = S_K + NB * TQ;           // [NB]
@@ -1126,7 +1136,9 @@ struct W2Cfg {
   static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
 };
 
-__global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a) {
+__global__ void __launch_bounds__(W2_NT, 1)
+    tc_prefill_ws2_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using K = W2Cfg;
   constexpr int DX = K::DX, DV = K::DV, F = K::F, NB = K::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1170,7 +1182,7 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
     for (int i = 0; i < NB; ++i) {
       mbar_init(freeQK + i, 1);
       mbar_init(freeVR + i, 1);
-      mbar_init(loaded + i, 32);
+      mbar_init(loaded + i, 1);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -1181,10 +1193,10 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
     for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
     // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
-    for (int r = tid; r < C; r += W2_NT) {
+    for (int r = tid; r < C; r += W2_NT) {   // column blocks 8, 9 of V: the ones column, then zeros
       for (int b = 0; b < NB; ++b) {
-        *reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sV(b) + 8 * K::IN_CB + r * 16) = make_uint4(0x00003C00u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sV(b) + 9 * K::IN_CB + r * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     for (int r = tid; r < KR; r += W2_NT) {
@@ -1211,8 +1223,8 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
         return r;
       };
       auto g5g6 = [&](int bb) {
-        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(bb), K::RSV, 128, 2 * K::RSV,
-             idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
+        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(bb), K::IN_RG, K::IN_CB,
+             2 * K::IN_RG, idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
         gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, sbase + sRG(bb), K::RSV, 128, 2 * K::RSV,
              idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
         mma_commit(dne + 3);
@@ -1221,12 +1233,12 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
       for (int t = ch0; t < ch1; ++t) {
         const int rel = t - ch0, b = rel % NB, p = rel & 1;
         if (!(ok = wait_rdy(0))) break;
-        gemm(tmem + K::T_S, sbase + sK(b), 128, K::RSX, 256, sbase + sQ(b), 128, K::RSX, 256,
-             idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
-        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(b), K::RSX, 128,
-             2 * K::RSX, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
-        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(b), K::RSV, 128,
-             2 * K::RSV, idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
+        gemm(tmem + K::T_S, sbase + sK(b), K::IN_CB, K::IN_RG, 2 * K::IN_CB, sbase + sQ(b), K::IN_CB,
+             K::IN_RG, 2 * K::IN_CB, idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
+        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(b), K::IN_RG, K::IN_CB,
+             2 * K::IN_RG, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
+        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(b), K::IN_RG, K::IN_CB,
+             2 * K::IN_RG, idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
         mma_commit(dne + 0);
         if (t > ch0) {
           if (!(ok = wait_rdy(3))) break;
@@ -1235,8 +1247,8 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
         if (!(ok = wait_rdy(1))) break;
         gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
              idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
-        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(b), 128, K::RSX, 256,
-             idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
+        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(b), K::IN_CB, K::IN_RG,
+             2 * K::IN_CB, idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
         mma_commit(dne + 1);
         mma_commit(freeQK + b);
         if (!(ok = wait_rdy(2))) break;
@@ -1269,10 +1281,11 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
       tc_fence_after();
       return !named_sync_or(2, W2_GT, !r);
     };
-    // 16-byte pieces of a 64 x 64 input tile: piece = row%8 | col-block << 3 | row/8 << 6
+    // 16-byte pieces of a 64 x 64 input tile, numbered in address order:
+    // piece = row | column block << 6
     auto piece = [](int pc, int& r, int& cb) {
-      r = (pc >> 6) * 8 + (pc & 7);
-      cb = (pc >> 3) & 7;
+      r = pc & (C - 1);
+      cb = pc >> 6;
     };
     // bf16 -> fp16 in place (q, k through the feature map); rows past the
     // sequence become 0
@@ -1281,9 +1294,10 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
       for (int u = 0; u < 2; ++u) {
         int r, cb;
         piece(tid + u * W2_GT, r, cb);   // this thread converts pieces tid, tid + 256
-        uint4* ptr[3] = {reinterpret_cast<uint4*>(smem + sQ(b) + tile_off(r, cb * 8, K::RSX)),
-                         reinterpret_cast<uint4*>(smem + sK(b) + tile_off(r, cb * 8, K::RSX)),
-                         reinterpret_cast<uint4*>(smem + sV(b) + tile_off(r, cb * 8, K::RSV))};
+        const uint32_t off = cb * K::IN_CB + r * 16;
+        uint4* ptr[3] = {reinterpret_cast<uint4*>(smem + sQ(b) + off),
+                         reinterpret_cast<uint4*>(smem + sK(b) + off),
+                         reinterpret_cast<uint4*>(smem + sV(b) + off)};
         uint4 in[3] = {*ptr[0], *ptr[1], *ptr[2]};
 #pragma unroll
         for (int tsel = 0; tsel < 3; ++tsel) {
@@ -1570,35 +1584,65 @@ __global__ void __launch_bounds__(W2_NT, 1) tc_prefill_ws2_kernel(const TcArgs a
   }
   if (role == 3) {
     // ------------------------------------------------ fetch warp
-    uint32_t pfq[NB] = {0u, 0u, 0u}, pfv[NB] = {0u, 0u, 0u};
-    for (int t = ch0; t < ch1; ++t) {
-      const int rel = t - ch0, b = rel % NB;
-      if (rel >= NB) {   // set b last held chunk t-3: wait until its contractions are done
-        bool ok = mbar_wait_or_abort(freeQK + b, pfq[b], a.err, abort_flag);
-        pfq[b] ^= 1u;
-        if (ok) ok = mbar_wait_or_abort(freeVR + b, pfv[b], a.err, abort_flag);
-        pfv[b] ^= 1u;
-        if (!__all_sync(kFull, ok)) break;
+    if (lane == 0) {
+      uint32_t pfq[NB] = {0u, 0u, 0u}, pfv[NB] = {0u, 0u, 0u};
+      int issued[NB] = {0, 0, 0};
+      for (int t = ch0; t < ch1; ++t) {
+        const int rel = t - ch0, b = rel % NB;
+        if (rel >= NB) {   // set b last held chunk t-3: wait until its contractions are done
+          bool ok = mbar_wait_or_abort(freeQK + b, pfq[b], a.err, abort_flag);
+          pfq[b] ^= 1u;
+          if (ok) ok = mbar_wait_or_abort(freeVR + b, pfv[b], a.err, abort_flag);
+          pfv[b] ^= 1u;
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(loaded + b, 3 * K::TIN);
+        tma_load_4d(sbase + sQ(b), &tm_q, 0, t * C, 0, static_cast<int>(bh), loaded + b);
+        tma_load_4d(sbase + sK(b), &tm_k, 0, t * C, 0, static_cast<int>(bh), loaded + b);
+        tma_load_4d(sbase + sV(b), &tm_v, 0, t * C, 0, static_cast<int>(bh), loaded + b);
+        ++issued[b];
       }
-      const int n0 = t * C;
-      const int nv = min(C, a.N - n0);
-#pragma unroll 4
-      for (int u = 0; u < C * DX / 8 / 32; ++u) {
-        const int pc = lane + 32 * u;
-        const int r = (pc >> 6) * 8 + (pc & 7), cb = (pc >> 3) & 7;
-        const uint32_t bytes = r < nv ? 16u : 0u;   // rows past the sequence are zero-filled
-        const long long g = (bh * a.N + n0 + (r < nv ? r : 0)) * DX + cb * 8;
-        cp_async16(sbase + sQ(b) + tile_off(r, cb * 8, K::RSX), a.q + g, bytes);
-        cp_async16(sbase + sK(b) + tile_off(r, cb * 8, K::RSX), a.k + g, bytes);
-        cp_async16(sbase + sV(b) + tile_off(r, cb * 8, K::RSV), a.v + g, bytes);
-      }
-      cp_async_mbar_arrive(loaded + b);
+      for (int b = 0; b < NB; ++b)   // no copy of ours lands after the block exits
+        if (issued[b] > 0) mbar_wait(loaded + b, static_cast<uint32_t>((issued[b] - 1) & 1), a.err);
     }
-    cp_async_wait_all();   // nothing of ours lands after the block exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links no driver stub).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// q, k or v [BH][N][64] bf16 viewed as [BH][column block 0..7][row 0..N-1][8
+// elements]; one box is 8 column blocks x 64 rows of one (b,h), 8 KB, landing
+// column-block-major.  Rows >= N lie outside the map and read as zero.
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {8, static_cast<cuuint64_t>(N), 8, static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[3] = {64 * 2, 16, static_cast<cuuint64_t>(N) * 64 * 2};
+  const cuuint32_t box[4] = {8, static_cast<cuuint32_t>(C), 8, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int DX, int DV>
@@ -1618,10 +1662,15 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
   if constexpr (DX == 64 && DV == 64) {
     const char* ws = std::getenv("IA_PREFILL_WS");   // tuning switch: 0 plain loop, 1 one epilogue group
     if (!ws || std::atoi(ws) >= 2) {
+      CUtensorMap tm_q, tm_k, tm_v;
+      if (!encode_input_map(&tm_q, args.q, args.BH, args.N) || !encode_input_map(&tm_k, args.k, args.BH, args.N) ||
+          !encode_input_map(&tm_v, args.v, args.BH, args.N))
+        return cudaErrorNotSupported;
       e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
       if (e != cudaSuccess) return e;
       mark_launch_begin(st);
-      tc_prefill_ws2_kernel<<<static_cast<unsigned>(args.BH * p.nseg), W2_NT, W2Cfg::SMEM, st>>>(args);
+      tc_prefill_ws2_kernel<<<static_cast<unsigned>(args.BH * p.nseg), W2_NT, W2Cfg::SMEM, st>>>(args, tm_q, tm_k,
+                                                                                               tm_v);
       e = cudaGetLastError();
       mark_launch_end(st);
       return e;
