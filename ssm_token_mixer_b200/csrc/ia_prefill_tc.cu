@@ -1098,7 +1098,10 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
 // them in place, so there is no staging area.  The tensor map views a
 // [rows][64] bf16 input as [column block][row][8 elements], so a 64-row box
 // arrives as core matrices of 8 rows x 16 bytes: row groups 128 bytes apart,
-// column blocks 1024 bytes apart.  Rows past the sequence arrive as zeros.  q, k, v and R_Gamma have three buffer sets and
+// column blocks 1024 bytes apart.  Rows past the sequence arrive as zeros.
+// R_U, the A operand of G3, is written to tensor memory as fp16 pairs, and o
+// leaves through TMA tensor stores from a double-buffered staging area, so
+// neither waits on the other side.  q, k, v and R_Gamma have three buffer sets and
 // R_U two: the fetch warp refills a set as soon as the contractions of the
 // chunk it held are done, about two chunks ahead of its use.  Handover is by
 // mbarriers: loaded(set) from the copies, ready(0) from the prepare warps,
@@ -1110,10 +1113,11 @@ constexpr int W2_NT = 2 * W2_GT + 64;          // + the MMA warp and the fetch w
 
 struct W2Cfg {
   static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
-  static constexpr uint32_t RSX = DX * 16, RSV = WV * 16;
+  static constexpr uint32_t RSV = WV * 16;
   static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
-                            T_DEN = 320 + 64;
-  static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRU = KR * DX * 2, TRG = KR * WV * 2;
+                            T_DEN = 320 + 64, T_RU = 400;   // T_RU: [2] x 32 columns of fp16 pairs
+  static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRG = KR * WV * 2;
+  static constexpr uint32_t TO = C * DV * 4;               // o of one chunk: two 64 x 128-byte boxes
   static constexpr int NB = 3;                             // q, k, v and R_Gamma buffer sets
   static constexpr uint32_t TIN = C * 64 * 2;              // bytes of one TMA box (64 rows x 64 bf16)
   // q, k, v tiles: column block cb of row r at cb * 1024 + r * 16; K-major
@@ -1127,18 +1131,20 @@ struct W2Cfg {
   static constexpr uint32_t S_S = S_E + KR * C * 2;
   static constexpr uint32_t S_P = S_S + C * C * 2;
   static constexpr uint32_t S_X = S_P + C * C * 2;
-  static constexpr uint32_t S_RU = S_X + KR * C * 2;       // [2]
-  static constexpr uint32_t S_RG = S_RU + 2 * TRU;         // [NB]
+  static constexpr uint32_t S_O = S_X + KR * C * 2;        // [2] o staging, 128-byte swizzled
+  static constexpr uint32_t S_RG = S_O + 2 * TO;           // [NB]
   static constexpr uint32_t S_BAR = S_RG + NB * TRG;       // 18 mbarriers
   static constexpr uint32_t S_FLAG = S_BAR + 256;
   static constexpr uint32_t S_TMEMH = S_FLAG + 16;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
   static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
+  static_assert(S_O % 1024 == 0, "o boxes start on the 128-byte swizzle period");
 };
 
 __global__ void __launch_bounds__(W2_NT, 1)
     tc_prefill_ws2_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
-                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o) {
   using K = W2Cfg;
   constexpr int DX = K::DX, DV = K::DV, F = K::F, NB = K::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1167,7 +1173,6 @@ __global__ void __launch_bounds__(W2_NT, 1)
   auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
   auto sK = [&](int b) { return K::S_K + b * K::TQ; };
   auto sV = [&](int b) { return K::S_V + b * K::TV; };
-  auto sRU = [&](int p) { return K::S_RU + p * K::TRU; };
   auto sRG = [&](int b) { return K::S_RG + b * K::TRG; };
 
   if (warp == 0) {
@@ -1247,8 +1252,9 @@ __global__ void __launch_bounds__(W2_NT, 1)
         if (!(ok = wait_rdy(1))) break;
         gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
              idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
-        gemm(tmem + K::T_A, sbase + sRU(p), 128, K::RSX, 256, sbase + sQ(b), K::IN_CB, K::IN_RG,
-             2 * K::IN_CB, idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
+        for (int kk = 0; kk < DX / 16; ++kk)   // G3: A = R_U from tensor memory
+          mma_f16_ts(tmem + K::T_A, tmem + K::T_RU + 32 * p + 8 * kk,
+                     smem_desc(sbase + sQ(b) + kk * 2 * K::IN_CB, K::IN_CB, K::IN_RG), idesc_f16(128, 64, 0, 0), 1u);
         mma_commit(dne + 1);
         mma_commit(freeQK + b);
         if (!(ok = wait_rdy(2))) break;
@@ -1363,6 +1369,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
       if (!(ok = waitA(loaded + b, pld[b]))) break;
       convert(nv, b);
       if (rel >= 1 && !(ok = waitA(dne + 0, pd0))) break;   // G7(t-1): the state is current
+      uint32_t ru[16];
 #pragma unroll
       for (int blk = 0; blk < FH / 16; ++blk) {
         const int col0 = half * FH + 16 * blk;
@@ -1383,14 +1390,16 @@ __global__ void __launch_bounds__(W2_NT, 1)
             d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
                                 __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
         }
+        if (half == 0) {   // R_U: fp16 pairs into tensor memory, 16 columns per two blocks
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint4 pk = pack8f(w + 8 * g, 1.f);
-          const int f = col0 + 8 * g;
-          if (f < DX)
-            *reinterpret_cast<uint4*>(smem + sRU(p) + tile_off(k, f, K::RSX)) = pk;
-          else
-            *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, f - DX, K::RSV)) = pk;
+          for (int e = 0; e < 8; ++e)
+            ru[(blk & 1) * 8 + e] = pack_half2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+          if (blk & 1) tmem_st16(trow + K::T_RU + 32 * p + 16 * (blk >> 1), ru);
+        } else {           // R_Gamma: shared memory, B operand of G6
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+            *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, col0 - DX + 8 * g, K::RSV)) =
+                pack8f(w + 8 * g, 1.f);
         }
       }
       tmem_st_wait();
@@ -1492,35 +1501,52 @@ __global__ void __launch_bounds__(W2_NT, 1)
       }
       signalB(3);
     };
-    auto e4 = [&](int ch, int nv) {   // o = num / den, written straight from registers
+    // o = num / den, staged as two boxes of 64 rows x 128 bytes (columns 0-31
+    // and 32-63) in the 128-byte swizzled layout, which keeps the row-per-lane
+    // writes free of bank conflicts, then written by one TMA store per box.
+    // Rows past the sequence lie outside the tensor map and are not written.
+    // Staging alternates between two buffers; before one is reused, the
+    // issuing thread has seen its previous store finish reading it.
+    auto e4 = [&](int ch, int nv) {
       const int i = 16 * quad + lane;
-      uint32_t rd;
+      uint32_t rd, rr[2][16];
       tmem_ld1(trow + K::T_DEN, rd);
+      tmem_ld16(trow + K::T_NUM + i0, rr[0]);
+      tmem_ld16(trow + K::T_NUM + i0 + 16, rr[1]);
       tmem_ld_wait1(rd);
+      tmem_ld_wait16(rr[0]);
+      tmem_ld_wait16(rr[1]);
       const float dn = __uint_as_float(rd);
       const float rdn = 1.0f / dn;
       const long long row = bh * a.N + ch * C + i;
-      const bool live = lane < 16 && i < nv;
-      if (live && a.den && half == 0) a.den[row] = dn;
+      const uint32_t stage = K::S_O + ((ch - ch0) & 1) * K::TO;
+      if (lane < 16) {
+        if (i < nv && a.den && half == 0) a.den[row] = dn;
+        uint8_t* box = smem + stage + half * (K::TO / 2) + i * 128;
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_NUM + i0 + 16 * b, r);
-        tmem_ld_wait16(r);
-        if (live) {
-          float4* op = reinterpret_cast<float4*>(a.o + row * DV + i0 + 16 * b);
+        for (int b = 0; b < 2; ++b) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            op[g] = make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                                __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-          if (a.num) {
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t* r = rr[b] + 4 * g;
+            *reinterpret_cast<float4*>(box + (((4 * b + g) ^ (i & 7)) << 4)) =
+                make_float4(__uint_as_float(r[0]) * rdn, __uint_as_float(r[1]) * rdn,
+                            __uint_as_float(r[2]) * rdn, __uint_as_float(r[3]) * rdn);
+          }
+          if (i < nv && a.num) {
             float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0 + 16 * b);
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-              np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                                  __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
+              np[g] = make_float4(__uint_as_float(rr[b][4 * g]), __uint_as_float(rr[b][4 * g + 1]),
+                                  __uint_as_float(rr[b][4 * g + 2]), __uint_as_float(rr[b][4 * g + 3]));
           }
         }
+      }
+      fence_async_smem();
+      named_sync(1, W2_GT);
+      if (tid == W2_GT) {
+        tma_store_3d(&tm_o, sbase + stage, 0, ch * C, static_cast<int>(bh));
+        tma_store_3d(&tm_o, sbase + stage + K::TO / 2, 32, ch * C, static_cast<int>(bh));
+        bulk_commit();
       }
     };
     bool ok = true;
@@ -1555,6 +1581,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
         }
       }
       if (prev >= 0) {
+        if (tid == W2_GT) bulk_wait_read_1();   // the staging buffer e4 is about to fill is free
         if (!(ok = waitB(3))) break;   // G5 + G6(t-1)
         e4(prev, prev_nv);
       }
@@ -1581,6 +1608,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
       prev = t;
       prev_nv = nv;
     }
+    if (tid == W2_GT) bulk_wait_all();   // o is in global memory before the block exits
   }
   if (role == 3) {
     // ------------------------------------------------ fetch warp
@@ -1645,6 +1673,20 @@ bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// o [BH][N][64] fp32 seen as boxes of 32 columns x 64 rows of one (b,h),
+// 128-byte swizzled in shared memory; rows >= N lie outside the map.
+bool encode_o_map(CUtensorMap* m, float* o, long long BH, int N) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {64 * sizeof(float), static_cast<cuuint64_t>(N) * 64 * sizeof(float)};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(C), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DX, int DV>
 cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p, cudaStream_t st) {
   using K = Cfg<DX, DV>;
@@ -1662,15 +1704,15 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
   if constexpr (DX == 64 && DV == 64) {
     const char* ws = std::getenv("IA_PREFILL_WS");   // tuning switch: 0 plain loop, 1 one epilogue group
     if (!ws || std::atoi(ws) >= 2) {
-      CUtensorMap tm_q, tm_k, tm_v;
+      CUtensorMap tm_q, tm_k, tm_v, tm_o;
       if (!encode_input_map(&tm_q, args.q, args.BH, args.N) || !encode_input_map(&tm_k, args.k, args.BH, args.N) ||
-          !encode_input_map(&tm_v, args.v, args.BH, args.N))
+          !encode_input_map(&tm_v, args.v, args.BH, args.N) || !encode_o_map(&tm_o, args.o, args.BH, args.N))
         return cudaErrorNotSupported;
       e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
       if (e != cudaSuccess) return e;
       mark_launch_begin(st);
       tc_prefill_ws2_kernel<<<static_cast<unsigned>(args.BH * p.nseg), W2_NT, W2Cfg::SMEM, st>>>(args, tm_q, tm_k,
-                                                                                               tm_v);
+                                                                                               tm_v, tm_o);
       e = cudaGetLastError();
       mark_launch_end(st);
       return e;
