@@ -134,16 +134,16 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
 // Waits for every cp.async this thread has committed.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// TMA tensor load of one box (4-D tensor map) into shared memory, completing
+// TMA tensor load of one box (3-D tensor map) into shared memory, completing
 // on an mbarrier with the box's bytes as transaction count.  tmap is the
 // address of a __grid_constant__ CUtensorMap parameter; c0 * element size is
 // a multiple of 16 bytes.  Plain (non-multicast) form.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int c0, int c1, int c2, int c3,
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int c0, int c1, int c2,
                                             uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -271,6 +271,17 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   return d;
+}
+
+// Same for a tile in the 128-byte swizzled layout (rows of 128 bytes whose
+// 16-byte chunks are XOR-permuted by row % 8, atoms of 8 rows = 1024 bytes,
+// atoms 1024-byte aligned); layout type 2 in bits [61,64).  K-major: sbo is
+// the distance between 8-row groups along M/N and lbo is not used; stepping
+// K by 16 elements adds 32 bytes to the start address.  MN-major: lbo is the
+// distance between 64-element blocks along M/N, sbo between 8-row groups
+// along K.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo) | (static_cast<uint64_t>(2) << 61);
 }
 
 // Instruction descriptor for kind::f16 with fp16 A and B, fp32 D.

@@ -1095,10 +1095,10 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
 // scale and o = num/den of chunks t and t-1; warp 16 issues every
 // tensor-core contraction; warp 17 brings q, k, v in with TMA tensor loads
 // that land directly in the operand layout, where the prepare warps convert
-// them in place, so there is no staging area.  The tensor map views a
-// [rows][64] bf16 input as [column block][row][8 elements], so a 64-row box
-// arrives as core matrices of 8 rows x 16 bytes: row groups 128 bytes apart,
-// column blocks 1024 bytes apart.  Rows past the sequence arrive as zeros.
+// them in place, so there is no staging area.  A 64-row box arrives as 64
+// rows of 128 bytes in the 128-byte swizzled layout, which the tensor core
+// reads as a K-major (features along K) or an MN-major (tokens along K)
+// operand alike.  Rows past the sequence arrive as zeros.
 // R_U, the A operand of G3, is written to tensor memory as fp16 pairs, and o
 // leaves through TMA tensor stores from a double-buffered staging area, so
 // neither waits on the other side.  q, k, v and R_Gamma have three buffer sets and
@@ -1116,18 +1116,16 @@ struct W2Cfg {
   static constexpr uint32_t RSV = WV * 16;
   static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
                             T_DEN = 320 + 64, T_RU = 400;   // T_RU: [2] x 32 columns of fp16 pairs
-  static constexpr uint32_t TQ = C * DX * 2, TV = C * WV * 2, TRG = KR * WV * 2;
+  static constexpr uint32_t TQ = C * DX * 2, TV = C * DV * 2, TRG = KR * WV * 2;
   static constexpr uint32_t TO = C * DV * 4;               // o of one chunk: two 64 x 128-byte boxes
   static constexpr int NB = 3;                             // q, k, v and R_Gamma buffer sets
   static constexpr uint32_t TIN = C * 64 * 2;              // bytes of one TMA box (64 rows x 64 bf16)
-  // q, k, v tiles: column block cb of row r at cb * 1024 + r * 16; K-major
-  // operands step 1024 bytes along K and 128 along M/N, MN-major ones 128
-  // along K and 1024 along M/N
-  static constexpr uint32_t IN_CB = C * 16, IN_RG = 128;
+  static constexpr uint32_t SW = 1024;                     // one swizzle atom: 8 rows x 128 bytes
   static constexpr uint32_t S_Q = 0;                       // [NB]
   static constexpr uint32_t S_K = S_Q + NB * TQ;           // [NB]
   static constexpr uint32_t S_V = S_K + NB * TQ;           // [NB]
-  static constexpr uint32_t S_E = S_V + NB * TV;
+  static constexpr uint32_t S_ONES = S_V + NB * TV;        // [V | 1]: MN-block 64..127 of G5's B operand
+  static constexpr uint32_t S_E = S_ONES + TV;
   static constexpr uint32_t S_S = S_E + KR * C * 2;
   static constexpr uint32_t S_P = S_S + C * C * 2;
   static constexpr uint32_t S_X = S_P + C * C * 2;
@@ -1138,7 +1136,8 @@ struct W2Cfg {
   static constexpr uint32_t S_TMEMH = S_FLAG + 16;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
   static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
-  static_assert(S_O % 1024 == 0, "o boxes start on the 128-byte swizzle period");
+  static_assert(S_O % 1024 == 0 && S_K % 1024 == 0 && S_V % 1024 == 0 && S_ONES % 1024 == 0,
+                "swizzled tiles start on the 128-byte swizzle period");
 };
 
 __global__ void __launch_bounds__(W2_NT, 1)
@@ -1198,11 +1197,12 @@ __global__ void __launch_bounds__(W2_NT, 1)
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
     for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
     // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
-    for (int r = tid; r < C; r += W2_NT) {   // column blocks 8, 9 of V: the ones column, then zeros
-      for (int b = 0; b < NB; ++b) {
-        *reinterpret_cast<uint4*>(smem + sV(b) + 8 * K::IN_CB + r * 16) = make_uint4(0x00003C00u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sV(b) + 9 * K::IN_CB + r * 16) = make_uint4(0u, 0u, 0u, 0u);
-      }
+    // the ones column after V: MN element 64 (first of the second 64-block)
+    // is 1 in every row, the rest 0, in the swizzled layout
+    for (int i = tid; i < C * 8; i += W2_NT) {
+      const int r = i >> 3, c = i & 7;
+      *reinterpret_cast<uint4*>(smem + K::S_ONES + r * 128 + c * 16) =
+          make_uint4((c == (r & 7)) ? 0x00003C00u : 0u, 0u, 0u, 0u);
     }
     for (int r = tid; r < KR; r += W2_NT) {
       for (int b = 0; b < NB; ++b) {
@@ -1227,9 +1227,17 @@ __global__ void __launch_bounds__(W2_NT, 1)
         tc_fence_after();
         return r;
       };
+      // contraction over ksteps K-steps of 16 with prebuilt descriptors; the
+      // start addresses advance by astep / bstep bytes per step
+      auto gemm_d = [&](uint32_t d, uint64_t ad, uint32_t astep, uint64_t bd, uint32_t bstep, uint32_t idesc,
+                        int ksteps, bool acc) {
+        for (int kk = 0; kk < ksteps; ++kk)
+          mma_f16(d, ad + ((kk * astep) >> 4), bd + ((kk * bstep) >> 4), idesc, (kk > 0 || acc) ? 1u : 0u);
+      };
       auto g5g6 = [&](int bb) {
-        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sbase + sV(bb), K::IN_RG, K::IN_CB,
-             2 * K::IN_RG, idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
+        gemm_d(tmem + K::T_NUM, smem_desc(sbase + K::S_P, 128, 1024), 256,
+               smem_desc_sw128(sbase + sV(bb), K::S_ONES - sV(bb), K::SW), 2 * K::SW,
+               idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
         gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, sbase + sRG(bb), K::RSV, 128, 2 * K::RSV,
              idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
         mma_commit(dne + 3);
@@ -1238,12 +1246,15 @@ __global__ void __launch_bounds__(W2_NT, 1)
       for (int t = ch0; t < ch1; ++t) {
         const int rel = t - ch0, b = rel % NB, p = rel & 1;
         if (!(ok = wait_rdy(0))) break;
-        gemm(tmem + K::T_S, sbase + sK(b), K::IN_CB, K::IN_RG, 2 * K::IN_CB, sbase + sQ(b), K::IN_CB,
-             K::IN_RG, 2 * K::IN_CB, idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
-        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + sK(b), K::IN_RG, K::IN_CB,
-             2 * K::IN_RG, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
-        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sbase + sV(b), K::IN_RG, K::IN_CB,
-             2 * K::IN_RG, idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
+        gemm_d(tmem + K::T_S, smem_desc_sw128(sbase + sK(b), 16, K::SW), 32,
+               smem_desc_sw128(sbase + sQ(b), 16, K::SW), 32, idesc_f16(64, 64, 0, 0), DX / 16,
+               false);   // G1: S^T
+        gemm_d(tmem + K::T_STATE, smem_desc(sbase + K::S_E, 128, 1024), 256,
+               smem_desc_sw128(sbase + sK(b), K::TQ, K::SW), 2 * K::SW, idesc_f16(128, DX, 0, 1), C / 16,
+               true);   // G7: U carry
+        gemm_d(tmem + K::T_STATE + DX, smem_desc(sbase + K::S_E, 128, 1024), 256,
+               smem_desc_sw128(sbase + sV(b), K::S_ONES - sV(b), K::SW), 2 * K::SW, idesc_f16(128, DV, 0, 1),
+               C / 16, true);   // G7: Gamma carry
         mma_commit(dne + 0);
         if (t > ch0) {
           if (!(ok = wait_rdy(3))) break;
@@ -1254,7 +1265,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
              idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
         for (int kk = 0; kk < DX / 16; ++kk)   // G3: A = R_U from tensor memory
           mma_f16_ts(tmem + K::T_A, tmem + K::T_RU + 32 * p + 8 * kk,
-                     smem_desc(sbase + sQ(b) + kk * 2 * K::IN_CB, K::IN_CB, K::IN_RG), idesc_f16(128, 64, 0, 0), 1u);
+                     smem_desc_sw128(sbase + sQ(b) + 32 * kk, 16, K::SW), idesc_f16(128, 64, 0, 0), 1u);
         mma_commit(dne + 1);
         mma_commit(freeQK + b);
         if (!(ok = wait_rdy(2))) break;
@@ -1287,20 +1298,20 @@ __global__ void __launch_bounds__(W2_NT, 1)
       tc_fence_after();
       return !named_sync_or(2, W2_GT, !r);
     };
-    // 16-byte pieces of a 64 x 64 input tile, numbered in address order:
-    // piece = row | column block << 6
-    auto piece = [](int pc, int& r, int& cb) {
-      r = pc & (C - 1);
-      cb = pc >> 6;
+    // 16-byte pieces of a 64 x 64 input tile in address order (piece =
+    // row * 8 + slot); the map is elementwise, so the swizzle does not matter
+    auto piece = [](int pc, int& r, int& slot) {
+      r = pc >> 3;
+      slot = pc & 7;
     };
     // bf16 -> fp16 in place (q, k through the feature map); rows past the
     // sequence become 0
     auto convert = [&](int nv, int b) {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        int r, cb;
-        piece(tid + u * W2_GT, r, cb);   // this thread converts pieces tid, tid + 256
-        const uint32_t off = cb * K::IN_CB + r * 16;
+        int r, slot;
+        piece(tid + u * W2_GT, r, slot);   // this thread converts pieces tid, tid + 256
+        const uint32_t off = r * 128 + slot * 16;
         uint4* ptr[3] = {reinterpret_cast<uint4*>(smem + sQ(b) + off),
                          reinterpret_cast<uint4*>(smem + sK(b) + off),
                          reinterpret_cast<uint4*>(smem + sV(b) + off)};
@@ -1625,9 +1636,9 @@ __global__ void __launch_bounds__(W2_NT, 1)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(loaded + b, 3 * K::TIN);
-        tma_load_4d(sbase + sQ(b), &tm_q, 0, t * C, 0, static_cast<int>(bh), loaded + b);
-        tma_load_4d(sbase + sK(b), &tm_k, 0, t * C, 0, static_cast<int>(bh), loaded + b);
-        tma_load_4d(sbase + sV(b), &tm_v, 0, t * C, 0, static_cast<int>(bh), loaded + b);
+        tma_load_3d(sbase + sQ(b), &tm_q, 0, t * C, static_cast<int>(bh), loaded + b);
+        tma_load_3d(sbase + sK(b), &tm_k, 0, t * C, static_cast<int>(bh), loaded + b);
+        tma_load_3d(sbase + sV(b), &tm_v, 0, t * C, static_cast<int>(bh), loaded + b);
         ++issued[b];
       }
       for (int b = 0; b < NB; ++b)   // no copy of ours lands after the block exits
@@ -1658,18 +1669,18 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// q, k or v [BH][N][64] bf16 viewed as [BH][column block 0..7][row 0..N-1][8
-// elements]; one box is 8 column blocks x 64 rows of one (b,h), 8 KB, landing
-// column-block-major.  Rows >= N lie outside the map and read as zero.
+// q, k or v [BH][N][64] bf16: one box is 64 rows x 64 columns (128 bytes) of
+// one (b,h), 128-byte swizzled in shared memory.  Rows >= N lie outside the
+// map and read as zero.
 bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
   const EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
-  const cuuint64_t dims[4] = {8, static_cast<cuuint64_t>(N), 8, static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[3] = {64 * 2, 16, static_cast<cuuint64_t>(N) * 64 * 2};
-  const cuuint32_t box[4] = {8, static_cast<cuuint32_t>(C), 8, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {64 * 2, static_cast<cuuint64_t>(N) * 64 * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(C), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
