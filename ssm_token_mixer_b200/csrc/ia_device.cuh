@@ -300,4 +300,39 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// xi on a pair of inputs, returned as fp16 pairs: max(x, 0) + 2^(min(x, 0) *
+// log2(e)), which is x + 1 for x > 0 and e^x for x <= 0 (one of the two
+// terms is always 0 or 1).  The power of two is the hardware approximation on
+// fp16 pairs (ex2.approx.f16x2), so the argument is rounded to fp16 first;
+// the operand the tensor core reads is fp16 either way.
+__device__ __forceinline__ uint32_t feat_h2(float x0, float x1) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const __half2 zero = __float2half2_rn(0.f);
+  const __half2 arg = __hmul2(__hmin2(h, zero), __float2half2_rn(1.4426950408889634f));
+  uint32_t e;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(*reinterpret_cast<const uint32_t*>(&arg)));
+  const __half2 r = __hadd2(__hmax2(h, zero), *reinterpret_cast<const __half2*>(&e));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// Packed fp32 pair arithmetic (one instruction for both lanes of a float2).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {   // a * b + c
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 }  // namespace ia

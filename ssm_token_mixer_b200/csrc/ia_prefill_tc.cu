@@ -1288,6 +1288,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
     const int m = k >> 1, comp = k & 1;
     const float2 lamC = T->lamC[m];
     const float sgnLi = comp ? lamC.y : -lamC.y;
+    const uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
     const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     constexpr int FH = F / 2;   // state columns per thread
@@ -1324,9 +1325,8 @@ __global__ void __launch_bounds__(W2_NT, 1)
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              float2 f = __bfloat1622float2(x2[e]);
-              if (tsel < 2) { f.x = feat(f.x); f.y = feat(f.y); }
-              w[e] = pack_half2(f.x, f.y);
+              const float2 f = __bfloat1622float2(x2[e]);
+              w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
             }
             out = make_uint4(w[0], w[1], w[2], w[3]);
           }
@@ -1388,10 +1388,13 @@ __global__ void __launch_bounds__(W2_NT, 1)
         tmem_ld16(trow + K::T_STATE + col0, rs);
         tmem_ld_wait16(rs);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float x = __uint_as_float(rs[e]);
-          const float y = __shfl_xor_sync(kFull, x, 1);
-          w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
+        for (int e = 0; e < 16; e += 2) {   // w = Re/Im of lambda^C times the partner row, two columns at once
+          const float x0 = __uint_as_float(rs[e]), x1 = __uint_as_float(rs[e + 1]);
+          const uint64_t y = f2_pack(__shfl_xor_sync(kFull, x0, 1), __shfl_xor_sync(kFull, x1, 1));
+          float w0, w1;
+          f2_unpack(f2_fma(lamC2, f2_pack(x0, x1), f2_mul(sgnLi2, y)), w0, w1);
+          w[e] = __float_as_uint(w0);
+          w[e + 1] = __float_as_uint(w1);
         }
         tmem_st16(trow + K::T_STATE + col0, w);
         if (a.dump_R) {
@@ -1529,6 +1532,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
       tmem_ld_wait16(rr[1]);
       const float dn = __uint_as_float(rd);
       const float rdn = 1.0f / dn;
+      const uint64_t rdn2 = f2_pack(rdn, rdn);
       const long long row = bh * a.N + ch * C + i;
       const uint32_t stage = K::S_O + ((ch - ch0) & 1) * K::TO;
       if (lane < 16) {
@@ -1539,9 +1543,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const uint32_t* r = rr[b] + 4 * g;
-            *reinterpret_cast<float4*>(box + (((4 * b + g) ^ (i & 7)) << 4)) =
-                make_float4(__uint_as_float(r[0]) * rdn, __uint_as_float(r[1]) * rdn,
-                            __uint_as_float(r[2]) * rdn, __uint_as_float(r[3]) * rdn);
+            float4 q;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(r[0]), __uint_as_float(r[1])), rdn2), q.x, q.y);
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2]), __uint_as_float(r[3])), rdn2), q.z, q.w);
+            *reinterpret_cast<float4*>(box + (((4 * b + g) ^ (i & 7)) << 4)) = q;
           }
           if (i < nv && a.num) {
             float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0 + 16 * b);
@@ -1599,16 +1604,20 @@ __global__ void __launch_bounds__(W2_NT, 1)
       if (head) {
         if (!(ok = waitB(1))) break;   // G2 + G3(t)
         {  // E2(t): X = |lambda|^(2(i-c)) a~
-          float s = s_start;
+          uint64_t s2 = f2_pack(s_start, s_start * r2);   // scales of two adjacent columns
+          const uint64_t r4 = f2_pack(r2 * r2, r2 * r2);
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             uint32_t r[16];
             tmem_ld16(trow + K::T_A + i0 + 16 * b, r);
             tmem_ld_wait16(r);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
-              s *= r2;
+            for (int e = 0; e < 16; e += 2) {
+              float x0, x1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), s2), x0, x1);
+              r[e] = __float_as_uint(x0);
+              r[e + 1] = __float_as_uint(x1);
+              s2 = f2_mul(s2, r4);
             }
             *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
             *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
