@@ -79,49 +79,61 @@ __device__ __forceinline__ float warp_sum(float x) {
 }  // namespace
 
 // ------------------------------------------------------------------------
-// Parameter prologue for the tensor-core path: one block per head, one thread
-// per mode.  The powers lambda^(c-j) come from an fp64 recurrence started at
-// lambda^c (relative error ~C * 2^-53), the E' table is staged in shared
-// memory and written out with coalesced 16-byte stores.
-__global__ void param_tables_kernel(int H, const float* __restrict__ delta,
-                                    const float* __restrict__ A, HeadTables* __restrict__ tabs) {
+// Parameter prologue for the tensor-core path: one block per head, four
+// threads per mode.  Each thread covers 16 consecutive j: the powers
+// lambda^(c-j) come from an fp64 recurrence started at a directly computed
+// power (relative error ~16 * 2^-53); the sum of E' over the chunk is reduced
+// across the four threads, and the remaining per-mode powers are shared out
+// among them.  The E' table is staged in shared memory and written out with
+// coalesced 16-byte stores.
+__global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const float* __restrict__ delta,
+                                                                    const float* __restrict__ A,
+                                                                    HeadTables* __restrict__ tabs) {
   __shared__ __align__(16) __half Es[2 * kModesTC * kChunk];
   const int h = blockIdx.x;
   HeadTables* T = tabs + h;
   const float dl = delta[h];
-  constexpr int C = kChunk, c = kChunk / 2;
-  const int m = threadIdx.x;
-  if (m < kModesTC) {
-    ModeD md = mode_consts(dl, A, m);
-    const double rdA = dl * md.ar, idA = dl * md.ai;
-    double pr, pi, ir, ii;
-    cpow_d(rdA, idA, c, &pr, &pi);      // lambda^c
-    cpow_d(rdA, idA, -1.0, &ir, &ii);   // lambda^-1
-    double sr = 0.0, si = 0.0;
-    char* base = reinterpret_cast<char*>(Es);
-    for (int j = 0; j < C; ++j) {       // E'[j] = b lambda^(c-j)
-      const double er = md.br * pr - md.bi * pi, ei = md.br * pi + md.bi * pr;
-      *reinterpret_cast<__half*>(base + etab_offset(2 * m, j)) = __double2half(er);
-      *reinterpret_cast<__half*>(base + etab_offset(2 * m + 1, j)) = __double2half(ei);
-      sr += er;
-      si += ei;
-      const double nr = pr * ir - pi * ii;
-      pi = pr * ii + pi * ir;
-      pr = nr;
-    }
+  constexpr int C = kChunk, c = kChunk / 2, JS = kChunk / 4;
+  const int m = threadIdx.x >> 2, part = threadIdx.x & 3;   // four threads per mode, adjacent lanes
+  ModeD md = mode_consts(dl, A, m);
+  const double rdA = dl * md.ar, idA = dl * md.ai;
+  double pr, pi, ir, ii;
+  cpow_d(rdA, idA, c - JS * part, &pr, &pi);   // lambda^(c-j) at this thread's first j
+  cpow_d(rdA, idA, -1.0, &ir, &ii);            // lambda^-1
+  double sr = 0.0, si = 0.0;
+  char* base = reinterpret_cast<char*>(Es);
+  for (int j = JS * part; j < JS * (part + 1); ++j) {   // E'[j] = b lambda^(c-j)
+    const double er = md.br * pr - md.bi * pi, ei = md.br * pi + md.bi * pr;
+    *reinterpret_cast<__half*>(base + etab_offset(2 * m, j)) = __double2half(er);
+    *reinterpret_cast<__half*>(base + etab_offset(2 * m + 1, j)) = __double2half(ei);
+    sr += er;
+    si += ei;
+    const double nr = pr * ir - pi * ii;
+    pi = pr * ii + pi * ir;
+    pr = nr;
+  }
+  // sum of E' over the chunk: the four partial sums of this mode
+  for (int off = 1; off < 4; off <<= 1) {
+    sr += __shfl_xor_sync(0xffffffffu, sr, off);
+    si += __shfl_xor_sync(0xffffffffu, si, off);
+  }
+  if (part == 0) {
     T->lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
     T->b[m] = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
-    cpow_d(rdA, idA, C, &pr, &pi);
-    T->lamC[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
-    cpow_d(rdA, idA, C - c - 1, &pr, &pi);
-    T->sc[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
-    cpow_d(rdA, idA, -(C - c - 1), &pr, &pi);
-    T->sc_inv[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
     T->esum[m] = make_float2(static_cast<float>(sr), static_cast<float>(si));
-    T->r2[m] = static_cast<float>(exp(2.0 * rdA));
-    T->s0[m] = static_cast<float>(exp(-2.0 * c * rdA));
     T->re_dA[m] = rdA;
     T->im_dA[m] = idA;
+  } else if (part == 1) {
+    cpow_d(rdA, idA, C, &pr, &pi);
+    T->lamC[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
+    T->r2[m] = static_cast<float>(exp(2.0 * rdA));
+  } else if (part == 2) {
+    cpow_d(rdA, idA, C - c - 1, &pr, &pi);
+    T->sc[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
+    T->s0[m] = static_cast<float>(exp(-2.0 * c * rdA));
+  } else {
+    cpow_d(rdA, idA, -(C - c - 1), &pr, &pi);
+    T->sc_inv[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
   }
   __syncthreads();
   const uint4* src = reinterpret_cast<const uint4*>(Es);
@@ -525,7 +537,7 @@ __global__ void segment_scan_kernel(int H, int DX, int DV, int nseg, int L,
 // host-side launchers
 cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
                                 cudaStream_t st) {
-  param_tables_kernel<<<H, 128, 0, st>>>(H, delta, A, tabs);
+  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs);
   return cudaGetLastError();
 }
 
