@@ -23,7 +23,9 @@
 //     ds     += dX * a~,  dlambda^C += sum dR conj(S_hat0)
 //     d(b lambda^n)/dDelta = (lambda + n A b) lambda^n,  ds/dDelta = 2 Re(A)(i-c) s,
 //     d(lambda^C)/dDelta = C A lambda^C.
-// The forward pass (the prefill kernel) stores R and den for every chunk.
+// The forward pass (the prefill kernel) stores R (fp16 tiles R_U, R_Gamma in
+// the 128-byte swizzled operand layout, loaded here with one bulk copy per
+// chunk, one chunk ahead), R_eta (fp32) and den for every chunk.
 //
 // TMEM columns: [0,128) adjoint of the state (dS1, then dR, then dS_hat0);
 // [128,192) dE''^T; [192,256) a~^T then dK; [256,320) dX^T then dV;
@@ -66,8 +68,10 @@ struct B {
   static constexpr uint32_t S_DS1 = S_RG + TILE128;          // [128][F] fp16
   static constexpr uint32_t S_DD = S_DS1 + KR * F * 2;       // dden [64] fp32
   static constexpr uint32_t S_RED = S_DD + C * 4;            // dR_eta halves [2][128] fp32
-  static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;
+  static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;    // bar_tma, bar_mma, bar_r
   static constexpr uint32_t S_TMEMH = S_BAR + 32;
+  static constexpr uint32_t RT = KR * 64 * 2;                // one fp16 R tile: 16 KB
+  static_assert(S_RG == S_RU + RT && S_RU % 1024 == 0, "R tiles adjacent, on the swizzle period");
   static constexpr uint32_t SMEM = S_TMEMH + 16;
 };
 
@@ -80,7 +84,7 @@ struct BwdArgs {
   const float* den;
   const float* A;
   const HeadTables* tabs;
-  const float* R;    // [BH][nch][128][F]
+  const uint8_t* R;  // [BH][nch] x (R_U, R_Gamma) fp16 swizzled tiles of 16 KB
   const float* Re;   // [BH][nch][128]
   float* dq;
   float* dk;
@@ -107,6 +111,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
   const int nch = (a.N + C - 1) / C;
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + B::S_BAR);
   uint64_t* bar_mma = bar_tma + 1;
+  uint64_t* bar_r = bar_tma + 2;   // the R tiles of the next chunk to process
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + B::S_TMEMH);
   float* sDD = reinterpret_cast<float*>(smem + B::S_DD);
   float* sRED = reinterpret_cast<float*>(smem + B::S_RED);
@@ -119,6 +124,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_r, 1);
     fence_barrier_init();
   }
   {
@@ -182,9 +188,16 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     bulk_g2s(smem + B::STG_V, a.v + row * DV, bv, bar_tma);
     bulk_g2s(smem + B::STG_G, a.dO + row * DV, bv, bar_tma);
   };
-  if (tid == 0) issue_load(nch - 1);
-  bool tma_pending = true;
-  uint32_t ph_tma = 0, ph_mma = 0;
+  auto issue_r = [&](int ch) {   // both R tiles of chunk ch: 32 KB contiguous
+    mbar_arrive_expect_tx(bar_r, 2 * B::RT);
+    bulk_g2s(smem + B::S_RU, a.R + (bh * nch + ch) * 2 * B::RT, 2 * B::RT, bar_r);
+  };
+  if (tid == 0) {
+    issue_load(nch - 1);
+    issue_r(nch - 1);
+  }
+  bool tma_pending = true, r_pending = true;
+  uint32_t ph_tma = 0, ph_mma = 0, ph_r = 0;
   bool aborted = false;
   auto mma_sync = [&]() -> bool {
     bool ok = mbar_wait(bar_mma, ph_mma, a.err);
@@ -247,17 +260,12 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     __syncthreads();   // staging consumed
     if (tid == 0 && ch > 0) issue_load(ch - 1);
     tma_pending = ch > 0;
-    const float* Rrow = a.R + ((bh * nch + ch) * KR + k) * F;
     const float Reta = a.Re[(bh * nch + ch) * KR + k];
-    {  // R -> fp16 operands R_U (half 0) / R_G (half 1); dS1 -> fp16
-      const float4* src = reinterpret_cast<const float4*>(Rrow + half * 64);
-      uint8_t* dst = smem + (half == 0 ? B::S_RU : B::S_RG);
-#pragma unroll
-      for (int g8 = 0; g8 < 8; ++g8) {
-        const float4 x0 = src[2 * g8], x1 = src[2 * g8 + 1];
-        const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        *reinterpret_cast<uint4*>(dst + tile_off(k, 8 * g8, 64 * 16)) = pack8(xs);
-      }
+    {  // the R tiles of this chunk have landed; dS1 -> fp16
+      bool ok = mbar_wait(bar_r, ph_r, a.err);
+      ph_r ^= 1u;
+      if (__syncthreads_or(!ok)) { aborted = true; break; }
+      r_pending = false;
       for (int cb = 0; cb < 64; cb += 16) {
         const int col0 = half * 64 + cb;
         uint32_t r[16];
@@ -301,8 +309,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
       tc_fence_after();
       gemm(tmem + B::T_A, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S,
            mn_lbo(64), mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, false);
-      gemm(tmem + B::T_A, sb + B::S_RU, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_Q,
-           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16, true);
+      gemm_dd(tmem + B::T_A, smem_desc_sw128(sb + B::S_RU, 16, 1024), 32,
+              smem_desc(sb + B::S_Q, kmaj_lbo(), kmaj_sbo(DX)), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16,
+              true);
       mma_commit(bar_mma);
     }
     if (!mma_sync()) { aborted = true; break; }
@@ -382,8 +391,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
       tc_fence_after();
       gemm(tmem + B::T_DX, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP,
            kmaj_lbo(), kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, false);
-      gemm(tmem + B::T_DX, sb + B::S_RG, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DN,
-           kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16, true);
+      gemm_dd(tmem + B::T_DX, smem_desc_sw128(sb + B::S_RG, 16, 1024), 32,
+              smem_desc(sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV)), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16,
+              true);
       mma_commit(bar_mma);
     }
     if (!mma_sync()) { aborted = true; break; }
@@ -435,97 +445,26 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
       mma_commit(bar_mma);
     }
     if (!mma_sync()) { aborted = true; break; }
-    {  // E_dS: mask (j <= i, j < nv) -> [i][j]
-      const int i = 16 * quad + lane;
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            xs[e] = (j0 + e <= i && j0 + e < nv) ? __uint_as_float(r[e]) : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
-    }
-    to_tc();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sDS = sb + B::S_DS, sDA = sb + B::S_DA, sE = sb + B::S_E, sDS1 = sb + B::S_DS1;
-      // dQ = dS xi(K) + da~ R_U
-      gemm(tmem + B::T_DQ, sDS, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_K, mn_lbo(DX),
-           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 0, 1), C / 16, false);
-      gemm(tmem + B::T_DQ, sDA, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_RU, mn_lbo(64),
-           mn_sbo(), mn_step(64), idesc_f16(64, DX, 1, 1), KR / 16, true);
-      // dK = dS^T xi(Q) + E'' dS1_U
-      gemm(tmem + B::T_DK, sDS, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_Q, mn_lbo(DX),
-           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 1, 1), C / 16, false);
-      gemm(tmem + B::T_DK, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1, mn_lbo(F), mn_sbo(),
-           mn_step(F), idesc_f16(64, DX, 1, 1), KR / 16, true);
-      // dV = P^T dnum + E'' dS1_G
-      gemm(tmem + B::T_DV, sb + B::S_P, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_DN, mn_lbo(DV),
-           mn_sbo(), mn_step(DV), idesc_f16(64, DV, 1, 1), C / 16, false);
-      gemm(tmem + B::T_DV, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1 + (DX / 8) * 128, mn_lbo(F),
-           mn_sbo(), mn_step(F), idesc_f16(64, DV, 1, 1), KR / 16, true);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-    {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1)
-      const int i = 16 * quad + lane;
-      const bool valid = lane < 16 && i < nv;
-      const long long row = bh * a.N + n0 + i;
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int f0 = 32 * half + cb;
-        uint32_t rq[16], rk[16], rv[16];
-        tmem_ld16(trow + B::T_DQ + f0, rq);
-        tmem_ld_wait16(rq);
-        tmem_ld16(trow + B::T_DK + f0, rk);
-        tmem_ld_wait16(rk);
-        tmem_ld16(trow + B::T_DV + f0, rv);
-        tmem_ld_wait16(rv);
-        if (valid) {
-          const __half* xq = reinterpret_cast<const __half*>(smem + B::S_Q);
-          const __half* xk = reinterpret_cast<const __half*>(smem + B::S_K);
-          float4* pq = reinterpret_cast<float4*>(a.dq + row * DX + f0);
-          float4* pk = reinterpret_cast<float4*>(a.dk + row * DX + f0);
-          float4* pv = reinterpret_cast<float4*>(a.dv + row * DV + f0);
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float oq[4], ok[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int f = f0 + 4 * g + e;
-              const float fq = __half2float(xq[tile_off(i, f, DX * 16) / 2]);
-              const float fk = __half2float(xk[tile_off(i, f, DX * 16) / 2]);
-              oq[e] = __uint_as_float(rq[4 * g + e]) * fminf(fq, 1.f);
-              ok[e] = __uint_as_float(rk[4 * g + e]) * fminf(fk, 1.f);
-            }
-            pq[g] = make_float4(oq[0], oq[1], oq[2], oq[3]);
-            pk[g] = make_float4(ok[0], ok[1], ok[2], ok[3]);
-            pv[g] = make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
-                                __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
-          }
-        }
-      }
-    }
+    // dR of this chunk is complete: Delta terms, then the carry to the previous chunk
     {  // adjoint carry: dS_hat0 = conj(lambda^C) dR;  dDelta += C Re(conj(sum dR conj(R)) A)
       for (int cb = 0; cb < 64; cb += 16) {
         const int col0 = half * 64 + cb;
         uint32_t r[16];
         tmem_ld16(trow + B::T_ADJ + col0, r);
         tmem_ld_wait16(r);
-        const float4* rp = reinterpret_cast<const float4*>(Rrow + col0);
+        // R of this row, columns col0..col0+15, from the fp16 swizzled tile
+        const uint8_t* rrow = smem + B::S_RU + half * B::RT + k * 128;
         float rv[16];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 x = rp[g];
-          rv[4 * g] = x.x; rv[4 * g + 1] = x.y; rv[4 * g + 2] = x.z; rv[4 * g + 3] = x.w;
+        for (int g = 0; g < 2; ++g) {
+          const uint4 x = *reinterpret_cast<const uint4*>(rrow + ((((cb >> 3) + g) ^ (k & 7)) << 4));
+          const __half2* h2 = reinterpret_cast<const __half2*>(&x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h2[e]);
+            rv[8 * g + 2 * e] = f.x;
+            rv[8 * g + 2 * e + 1] = f.y;
+          }
         }
         uint32_t w[16];
 #pragma unroll
@@ -567,6 +506,89 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     }
     tc_fence_before();
     __syncthreads();
+    {  // E_dS: mask (j <= i, j < nv) -> [i][j]
+      const int i = 16 * quad + lane;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            xs[e] = (j0 + e <= i && j0 + e < nv) ? __uint_as_float(r[e]) : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
+    }
+    to_tc();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sDS = sb + B::S_DS, sDA = sb + B::S_DA, sE = sb + B::S_E, sDS1 = sb + B::S_DS1;
+      // dQ = dS xi(K) + da~ R_U
+      gemm(tmem + B::T_DQ, sDS, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_K, mn_lbo(DX),
+           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 0, 1), C / 16, false);
+      gemm_dd(tmem + B::T_DQ, smem_desc(sDA, mn_lbo(64), mn_sbo()), mn_step(64),
+              smem_desc_sw128(sb + B::S_RU, 16, 1024), 2048, idesc_f16(64, DX, 1, 1), KR / 16, true);
+      // dK = dS^T xi(Q) + E'' dS1_U
+      gemm(tmem + B::T_DK, sDS, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_Q, mn_lbo(DX),
+           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 1, 1), C / 16, false);
+      gemm(tmem + B::T_DK, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1, mn_lbo(F), mn_sbo(),
+           mn_step(F), idesc_f16(64, DX, 1, 1), KR / 16, true);
+      // dV = P^T dnum + E'' dS1_G
+      gemm(tmem + B::T_DV, sb + B::S_P, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_DN, mn_lbo(DV),
+           mn_sbo(), mn_step(DV), idesc_f16(64, DV, 1, 1), C / 16, false);
+      gemm(tmem + B::T_DV, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1 + (DX / 8) * 128, mn_lbo(F),
+           mn_sbo(), mn_step(F), idesc_f16(64, DV, 1, 1), KR / 16, true);
+      mma_commit(bar_mma);
+    }
+    if (!mma_sync()) { aborted = true; break; }
+    if (tid == 0 && ch > 0) issue_r(ch - 1);   // R tiles are free: every contraction reading them is done
+    r_pending = ch > 0;
+    {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1)
+      const int i = 16 * quad + lane;
+      const bool valid = lane < 16 && i < nv;
+      const long long row = bh * a.N + n0 + i;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int f0 = 32 * half + cb;
+        uint32_t rq[16], rk[16], rv[16];
+        tmem_ld16(trow + B::T_DQ + f0, rq);
+        tmem_ld_wait16(rq);
+        tmem_ld16(trow + B::T_DK + f0, rk);
+        tmem_ld_wait16(rk);
+        tmem_ld16(trow + B::T_DV + f0, rv);
+        tmem_ld_wait16(rv);
+        if (valid) {
+          const __half* xq = reinterpret_cast<const __half*>(smem + B::S_Q);
+          const __half* xk = reinterpret_cast<const __half*>(smem + B::S_K);
+          float4* pq = reinterpret_cast<float4*>(a.dq + row * DX + f0);
+          float4* pk = reinterpret_cast<float4*>(a.dk + row * DX + f0);
+          float4* pv = reinterpret_cast<float4*>(a.dv + row * DV + f0);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            float oq[4], ok[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int f = f0 + 4 * g + e;
+              const float fq = __half2float(xq[tile_off(i, f, DX * 16) / 2]);
+              const float fk = __half2float(xk[tile_off(i, f, DX * 16) / 2]);
+              oq[e] = __uint_as_float(rq[4 * g + e]) * fminf(fq, 1.f);
+              ok[e] = __uint_as_float(rk[4 * g + e]) * fminf(fk, 1.f);
+            }
+            pq[g] = make_float4(oq[0], oq[1], oq[2], oq[3]);
+            pk[g] = make_float4(ok[0], ok[1], ok[2], ok[3]);
+            pv[g] = make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
+                                __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
   }
 
   if (!aborted) {
@@ -600,8 +622,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
       for (int w = 0; w < NTHR / 32; ++w) s += sRED[w];
       atomicAdd(a.dDelta + h, s);
     }
-  } else if (tma_pending) {
-    mbar_wait(bar_tma, ph_tma, a.err);
+  } else {   // let our own copies land before exiting (bounded)
+    if (tma_pending) mbar_wait(bar_tma, ph_tma, a.err);
+    if (r_pending) mbar_wait(bar_r, ph_r, a.err);
   }
   tc_fence_before();
   __syncthreads();
@@ -619,7 +642,7 @@ size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
   const size_t nch = (s.N + C - 1) / C;
   size_t bytes = tc_workspace_bytes(s, p);
   bytes = (bytes + 255) & ~static_cast<size_t>(255);
-  bytes += BH * nch * KR * (s.d_xi + s.d_v) * sizeof(float);   // R per chunk
+  bytes += BH * nch * 2 * KR * 64 * 2;                        // R per chunk: two fp16 tiles
   bytes += BH * nch * KR * sizeof(float);                      // R_eta per chunk
   bytes += BH * s.N * sizeof(float) + 256;                     // den
   return bytes + 256;
@@ -633,8 +656,8 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   const size_t nch = (s.N + C - 1) / C;
   uint8_t* base = reinterpret_cast<uint8_t*>(tc_tables(ws));
   size_t off = (tc_workspace_bytes(s, p) + 255) & ~static_cast<size_t>(255);
-  float* dumpR = reinterpret_cast<float*>(base + off);
-  float* dumpRe = dumpR + BH * nch * KR * (s.d_xi + s.d_v);
+  uint8_t* dumpR = base + off;   // 32 KB per chunk, 256-byte aligned
+  float* dumpRe = reinterpret_cast<float*>(dumpR + BH * nch * 2 * B::RT);
   float* den = dumpRe + BH * nch * KR;
   den = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(den) + 255) & ~static_cast<uintptr_t>(255));
   cudaError_t e = launch_tc_prefill(s, p, q, k, v, delta, A, nullptr, o, nullptr, den, nullptr, ws,

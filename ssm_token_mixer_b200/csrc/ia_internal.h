@@ -40,7 +40,7 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st,
-                              float* dump_R = nullptr, float* dump_Re = nullptr);
+                              void* dump_R = nullptr, float* dump_Re = nullptr);
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
 

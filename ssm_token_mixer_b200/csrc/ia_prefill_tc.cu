@@ -103,8 +103,8 @@ struct TcArgs {
   float* den;
   float2* state_out;
   int* err;                 // device error flag
-  float* dump_R;            // optional: R = lambda^C S_hat at every chunk start, [BH][nch][128][F]
-  float* dump_Re;           // optional: the eta part, [BH][nch][128]
+  uint8_t* dump_R;          // optional: R = lambda^C S_hat at every chunk start, fp16 tiles (dump_r16)
+  float* dump_Re;           // optional: the eta part, [BH][nch][128] fp32
   int H, N, nseg, seg_chunks;
   long long BH;
 };
@@ -206,6 +206,20 @@ __device__ __forceinline__ uint4 pack8f(const uint32_t* r, float scale) {
                     pack_half2(__uint_as_float(r[2]) * scale, __uint_as_float(r[3]) * scale),
                     pack_half2(__uint_as_float(r[4]) * scale, __uint_as_float(r[5]) * scale),
                     pack_half2(__uint_as_float(r[6]) * scale, __uint_as_float(r[7]) * scale));
+}
+
+// R for the reverse pass: per chunk two fp16 tiles, R_U then R_Gamma, each
+// 128 rows (k) x 64 columns in the 128-byte swizzled layout (16-byte chunk c
+// of row k at byte k * 128 + (c ^ (k % 8)) * 16), 32 KB per chunk, so that a
+// plain bulk copy lands them ready to serve as tensor-core operands.  Stores
+// columns col0..col0+15 (col0 a multiple of 16) of row k of chunk `chunk`.
+constexpr uint32_t kDumpTile = KR * 64 * 2;
+__device__ __forceinline__ void dump_r16(uint8_t* base, long long chunk, int k, int col0, const uint32_t* w) {
+  uint8_t* row = base + (chunk * 2 + (col0 >= 64 ? 1 : 0)) * kDumpTile + k * 128;
+  const int c0 = (col0 & 63) >> 3;
+#pragma unroll
+  for (int g = 0; g < 2; ++g)
+    *reinterpret_cast<uint4*>(row + (((c0 + g) ^ (k & 7)) << 4)) = pack8f(w + 8 * g, 1.f);
 }
 
 template <int DX, int DV, bool FULL>
@@ -378,13 +392,7 @@ __global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
         w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
       }
       tmem_st16(trow + K::T_STATE + col0, w);
-      if (FULL && a.dump_R) {
-        float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + ch) * KR + k) * F + col0);
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-          d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
-                              __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
-      }
+      if (FULL && a.dump_R) dump_r16(a.dump_R, bh * nch_total + ch, k, col0, w);
       if (FULL) {
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -902,13 +910,7 @@ __global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a)
           w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
         }
         tmem_st16(trow + K::T_STATE + col0, w);
-        if (a.dump_R) {
-          float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + ch) * KR + k) * F + col0);
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-            d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
-                                __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
-        }
+        if (a.dump_R) dump_r16(a.dump_R, bh * nch_total + ch, k, col0, w);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           const uint4 pk = pack8f(w + 8 * g, 1.f);
@@ -1397,13 +1399,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
           w[e + 1] = __float_as_uint(w1);
         }
         tmem_st16(trow + K::T_STATE + col0, w);
-        if (a.dump_R) {
-          float4* d4 = reinterpret_cast<float4*>(a.dump_R + ((bh * nch_total + t) * KR + k) * F + col0);
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-            d4[g] = make_float4(__uint_as_float(w[4 * g]), __uint_as_float(w[4 * g + 1]),
-                                __uint_as_float(w[4 * g + 2]), __uint_as_float(w[4 * g + 3]));
-        }
+        if (a.dump_R) dump_r16(a.dump_R, bh * nch_total + t, k, col0, w);
         if (half == 0) {   // R_U: fp16 pairs into tensor memory, 16 columns per two blocks
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -1813,7 +1809,7 @@ HeadTables* tc_tables(void* ws) {
 cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
-                              void* state_out, void* ws, cudaStream_t st, float* dump_R,
+                              void* state_out, void* ws, cudaStream_t st, void* dump_R,
                               float* dump_Re) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 255) & ~static_cast<uintptr_t>(255));
@@ -1836,7 +1832,7 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
   args.den = den;
   args.state_out = static_cast<float2*>(state_out);
   args.err = device_error_ptr();
-  args.dump_R = dump_R;
+  args.dump_R = static_cast<uint8_t*>(dump_R);
   args.dump_Re = dump_Re;
   if (!args.err) return cudaErrorInvalidSymbol;
   args.H = s.H;

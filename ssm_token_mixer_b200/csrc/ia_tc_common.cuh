@@ -42,6 +42,14 @@ __device__ __forceinline__ void gemm(uint32_t dtm, uint32_t a, uint32_t alb, uin
   }
 }
 
+// Same with prebuilt descriptors (e.g. swizzled tiles): the start addresses
+// advance by astep / bstep bytes per K-step of 16.
+__device__ __forceinline__ void gemm_dd(uint32_t dtm, uint64_t adesc, uint32_t astep, uint64_t bdesc,
+                                        uint32_t bstep, uint32_t idesc, int ksteps, bool acc) {
+  for (int kk = 0; kk < ksteps; ++kk)
+    mma_f16(dtm, adesc + ((kk * astep) >> 4), bdesc + ((kk * bstep) >> 4), idesc, (kk > 0 || acc) ? 1u : 0u);
+}
+
 // bf16 staging rows [C][W] (row-major, contiguous) -> fp16 canonical tile,
 // applying xi when FEAT; rows >= nv become zero.  One warp iteration moves 8
 // rows x 4 column groups; the column group is rotated by the row so that
