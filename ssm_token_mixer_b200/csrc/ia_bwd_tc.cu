@@ -70,9 +70,17 @@ struct B {
   static constexpr uint32_t S_RED = S_DD + C * 4;            // dR_eta halves [2][128] fp32
   static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;    // bar_tma, bar_mma, bar_r
   static constexpr uint32_t S_TMEMH = S_BAR + 32;
+  static constexpr uint32_t S_OST = S_TMEMH + 16;            // o rows of the chunk, fp32 [64][64]
   static constexpr uint32_t RT = KR * 64 * 2;                // one fp16 R tile: 16 KB
+  // dq, dk, dv leave by TMA stores from tiles that are free between the
+  // gradient contractions and the next chunk's readout (E2, E3, dP, dX):
+  // each as two 64-row x 128-byte boxes in the 128-byte swizzled layout
+  static constexpr uint32_t O_DQ = S_X, O_DK = S_P, O_DV = S_DA, OBOX = C * 128;
+  static_assert(S_DP == S_P + OBOX && O_DQ % 1024 == 0 && O_DK % 1024 == 0 && O_DV % 1024 == 0,
+                "output staging: three 16 KB areas on the swizzle period");
   static_assert(S_RG == S_RU + RT && S_RU % 1024 == 0, "R tiles adjacent, on the swizzle period");
-  static constexpr uint32_t SMEM = S_TMEMH + 16;
+  static constexpr uint32_t SMEM = S_OST + C * 64 * 4;
+  static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
 };
 
 struct BwdArgs {
@@ -100,7 +108,9 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
                     pack_half2(x[6], x[7]));
 }
 
-__global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(NTHR, 1)
+    tc_bwd_kernel(const __grid_constant__ BwdArgs a, const __grid_constant__ CUtensorMap tm_dq,
+                  const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv) {
   constexpr int DX = B::DX, DV = B::DV, F = B::F;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -181,12 +191,14 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     const int n0 = ch * C;
     const int nv = min(C, a.N - n0);
     const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
-    mbar_arrive_expect_tx(bar_tma, 2 * bq + 2 * bv);
+    const uint32_t bo = static_cast<uint32_t>(nv * DV * 4);
+    mbar_arrive_expect_tx(bar_tma, 2 * bq + 2 * bv + bo);
     const long long row = bh * a.N + n0;
     bulk_g2s(smem + B::STG_Q, a.q + row * DX, bq, bar_tma);
     bulk_g2s(smem + B::STG_K, a.k + row * DX, bq, bar_tma);
     bulk_g2s(smem + B::STG_V, a.v + row * DV, bv, bar_tma);
     bulk_g2s(smem + B::STG_G, a.dO + row * DV, bv, bar_tma);
+    bulk_g2s(smem + B::S_OST, a.o + row * DV, bo, bar_tma);   // row * 256 bytes: 16-byte aligned
   };
   auto issue_r = [&](int ch) {   // both R tiles of chunk ch: 32 KB contiguous
     mbar_arrive_expect_tx(bar_r, 2 * B::RT);
@@ -196,6 +208,12 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     issue_load(nch - 1);
     issue_r(nch - 1);
   }
+  // den of row tid/4 of the next chunk to process, loaded a chunk ahead
+  auto load_den = [&](int ch) -> float {
+    const int i = tid >> 2;
+    return i < a.N - ch * C ? a.den[bh * a.N + ch * C + i] : 1.f;
+  };
+  float den_next = load_den(nch - 1);
   bool tma_pending = true, r_pending = true;
   uint32_t ph_tma = 0, ph_mma = 0, ph_r = 0;
   bool aborted = false;
@@ -226,14 +244,13 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     convert_tile<DV, false>(smem + B::STG_V, smem + B::S_V, nv, warp, lane);
     {  // dnum = dO / den (fp16 tile [i][f]), dden = -(dO . o) / den
       const int i = tid >> 2, part = tid & 3;
-      const long long row = bh * a.N + n0 + i;
       float g[16];
       float dot = 0.f, rden = 0.f;
       if (i < nv) {
-        rden = 1.0f / a.den[row];
+        rden = 1.0f / den_next;
         const __nv_bfloat162* gs =
             reinterpret_cast<const __nv_bfloat162*>(smem + B::STG_G + i * DV * 2 + part * 32);
-        const float4* op = reinterpret_cast<const float4*>(a.o + row * DV + part * 16);
+        const float4* op = reinterpret_cast<const float4*>(smem + B::S_OST + i * DV * 4 + part * 64);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float2 x = __bfloat1622float2(gs[e]);
@@ -257,6 +274,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
       *reinterpret_cast<uint4*>(smem + B::S_DN + tile_off(i, part * 16 + 8, DV * 16)) = pack8(g + 8);
       if (part == 0) sDD[i] = i < nv ? -dot * rden : 0.f;
     }
+    if (ch > 0) den_next = load_den(ch - 1);
     __syncthreads();   // staging consumed
     if (tid == 0 && ch > 0) issue_load(ch - 1);
     tma_pending = ch > 0;
@@ -307,6 +325,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     to_tc();
     if (tid == 0) {   // F2: a~^T = E''^T S^T + R_U xi(Q)^T
       tc_fence_after();
+      bulk_wait_read_0();   // last chunk's dq/dk/dv staging (sX, sP, sDP, sDA) has been read
       gemm(tmem + B::T_A, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S,
            mn_lbo(64), mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, false);
       gemm_dd(tmem + B::T_A, smem_desc_sw128(sb + B::S_RU, 16, 1024), 32,
@@ -548,43 +567,67 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     if (!mma_sync()) { aborted = true; break; }
     if (tid == 0 && ch > 0) issue_r(ch - 1);   // R tiles are free: every contraction reading them is done
     r_pending = ch > 0;
-    {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1)
+    {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1).  Staged as
+       // swizzled boxes (rows past the sequence are clipped by the tensor maps)
       const int i = 16 * quad + lane;
-      const bool valid = lane < 16 && i < nv;
-      const long long row = bh * a.N + n0 + i;
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 16) {
         const int f0 = 32 * half + cb;
         uint32_t rq[16], rk[16], rv[16];
         tmem_ld16(trow + B::T_DQ + f0, rq);
-        tmem_ld_wait16(rq);
         tmem_ld16(trow + B::T_DK + f0, rk);
-        tmem_ld_wait16(rk);
         tmem_ld16(trow + B::T_DV + f0, rv);
+        tmem_ld_wait16(rq);
+        tmem_ld_wait16(rk);
         tmem_ld_wait16(rv);
-        if (valid) {
-          const __half* xq = reinterpret_cast<const __half*>(smem + B::S_Q);
-          const __half* xk = reinterpret_cast<const __half*>(smem + B::S_K);
-          float4* pq = reinterpret_cast<float4*>(a.dq + row * DX + f0);
-          float4* pk = reinterpret_cast<float4*>(a.dk + row * DX + f0);
-          float4* pv = reinterpret_cast<float4*>(a.dv + row * DV + f0);
+        if (lane < 16) {
+          // xi(q), xi(k) of this row, columns f0..f0+15, from the fp16 operand tiles
+          float fq[16], fk[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float oq[4], ok[4];
+          for (int g = 0; g < 2; ++g) {
+            const uint4 xq = *reinterpret_cast<const uint4*>(smem + B::S_Q + tile_off(i, f0 + 8 * g, DX * 16));
+            const uint4 xk = *reinterpret_cast<const uint4*>(smem + B::S_K + tile_off(i, f0 + 8 * g, DX * 16));
+            const __half2* hq = reinterpret_cast<const __half2*>(&xq);
+            const __half2* hk = reinterpret_cast<const __half2*>(&xk);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int f = f0 + 4 * g + e;
-              const float fq = __half2float(xq[tile_off(i, f, DX * 16) / 2]);
-              const float fk = __half2float(xk[tile_off(i, f, DX * 16) / 2]);
-              oq[e] = __uint_as_float(rq[4 * g + e]) * fminf(fq, 1.f);
-              ok[e] = __uint_as_float(rk[4 * g + e]) * fminf(fk, 1.f);
+              const float2 a2 = __half22float2(hq[e]), b2 = __half22float2(hk[e]);
+              fq[8 * g + 2 * e] = a2.x; fq[8 * g + 2 * e + 1] = a2.y;
+              fk[8 * g + 2 * e] = b2.x; fk[8 * g + 2 * e + 1] = b2.y;
             }
-            pq[g] = make_float4(oq[0], oq[1], oq[2], oq[3]);
-            pk[g] = make_float4(ok[0], ok[1], ok[2], ok[3]);
-            pv[g] = make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
-                                __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
+          }
+          const uint32_t rowoff = half * B::OBOX + i * 128;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t pos = rowoff + ((((cb >> 2) + g) ^ (i & 7)) << 4);
+            float4 oq, ok;
+            oq.x = __uint_as_float(rq[4 * g]) * fminf(fq[4 * g], 1.f);
+            oq.y = __uint_as_float(rq[4 * g + 1]) * fminf(fq[4 * g + 1], 1.f);
+            oq.z = __uint_as_float(rq[4 * g + 2]) * fminf(fq[4 * g + 2], 1.f);
+            oq.w = __uint_as_float(rq[4 * g + 3]) * fminf(fq[4 * g + 3], 1.f);
+            ok.x = __uint_as_float(rk[4 * g]) * fminf(fk[4 * g], 1.f);
+            ok.y = __uint_as_float(rk[4 * g + 1]) * fminf(fk[4 * g + 1], 1.f);
+            ok.z = __uint_as_float(rk[4 * g + 2]) * fminf(fk[4 * g + 2], 1.f);
+            ok.w = __uint_as_float(rk[4 * g + 3]) * fminf(fk[4 * g + 3], 1.f);
+            *reinterpret_cast<float4*>(smem + B::O_DQ + pos) = oq;
+            *reinterpret_cast<float4*>(smem + B::O_DK + pos) = ok;
+            *reinterpret_cast<float4*>(smem + B::O_DV + pos) =
+                make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
+                            __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
           }
         }
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        const int y = n0, z = static_cast<int>(bh);
+        tma_store_3d(&tm_dq, sb + B::O_DQ, 0, y, z);
+        tma_store_3d(&tm_dq, sb + B::O_DQ + B::OBOX, 32, y, z);
+        tma_store_3d(&tm_dk, sb + B::O_DK, 0, y, z);
+        tma_store_3d(&tm_dk, sb + B::O_DK + B::OBOX, 32, y, z);
+        tma_store_3d(&tm_dv, sb + B::O_DV, 0, y, z);
+        tma_store_3d(&tm_dv, sb + B::O_DV + B::OBOX, 32, y, z);
+        bulk_commit();
       }
     }
     tc_fence_before();
@@ -626,6 +669,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_bwd_kernel(const BwdArgs a) {
     if (tma_pending) mbar_wait(bar_tma, ph_tma, a.err);
     if (r_pending) mbar_wait(bar_r, ph_r, a.err);
   }
+  if (tid == 0) bulk_wait_all();   // dq, dk, dv are in global memory before the block exits
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -685,10 +729,14 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   a.H = s.H;
   a.N = s.N;
   a.BH = static_cast<long long>(BH);
+  CUtensorMap tm_dq, tm_dk, tm_dv;
+  if (!encode_rows64_f32_map(&tm_dq, dq, a.BH, s.N) || !encode_rows64_f32_map(&tm_dk, dk, a.BH, s.N) ||
+      !encode_rows64_f32_map(&tm_dv, dv, a.BH, s.N))
+    return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B::SMEM);
   if (e != cudaSuccess) return e;
   mark_launch_begin(st);
-  tc_bwd_kernel<<<static_cast<unsigned>(BH), NTHR, B::SMEM, st>>>(a);
+  tc_bwd_kernel<<<static_cast<unsigned>(BH), NTHR, B::SMEM, st>>>(a, tm_dq, tm_dk, tm_dv);
   e = cudaGetLastError();
   mark_launch_end(st);
   return e;

@@ -206,6 +206,8 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// No committed bulk store group of this thread is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // At most one committed bulk store group of this thread is still reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Every committed bulk store of this thread is complete.

@@ -2,6 +2,7 @@
 // kernel translation units.  Not part of the public header.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/ia.h"
@@ -43,6 +44,12 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               void* dump_R = nullptr, float* dump_Re = nullptr);
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
+
+// TMA tensor maps (ia_prefill_tc.cu): an fp32 [BH][N][64] array as
+// 32-column x 64-row boxes, 128-byte swizzled; q/k/v bf16 [BH][N][64] as
+// 64 x 64 boxes, 128-byte swizzled.  False if the driver refuses the map.
+bool encode_rows64_f32_map(CUtensorMap* m, float* x, long long BH, int N);
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N);
 
 // Tensor-core training step (bf16, M = 64, d_xi = d_v = 64).
 bool tc_bwd_supported(const ia_shape_t& s);

@@ -48,6 +48,55 @@
 #include "ia_tc_common.cuh"
 
 namespace ia {
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links no driver stub).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// q, k or v [BH][N][64] bf16: one box is 64 rows x 64 columns (128 bytes) of
+// one (b,h), 128-byte swizzled in shared memory.  Rows >= N lie outside the
+// map and read as zero.
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {64 * 2, static_cast<cuuint64_t>(N) * 64 * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kChunk), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An fp32 [BH][N][64] array (o, dq, dk, dv) seen as boxes of 32 columns x 64
+// rows of one (b,h), 128-byte swizzled in shared memory; rows >= N lie
+// outside the map (TMA stores skip them).
+bool encode_rows64_f32_map(CUtensorMap* m, float* o, long long BH, int N) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {64 * sizeof(float), static_cast<cuuint64_t>(N) * 64 * sizeof(float)};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kChunk), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 using namespace tc;
@@ -1656,53 +1705,6 @@ __global__ void __launch_bounds__(W2_NT, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
-// (the library links no driver stub).
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-EncodeTiledFn encode_tiled() {
-  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(f);
-  }();
-  return fn;
-}
-
-// q, k or v [BH][N][64] bf16: one box is 64 rows x 64 columns (128 bytes) of
-// one (b,h), 128-byte swizzled in shared memory.  Rows >= N lie outside the
-// map and read as zero.
-bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
-  const EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {64 * 2, static_cast<cuuint64_t>(N) * 64 * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(C), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// o [BH][N][64] fp32 seen as boxes of 32 columns x 64 rows of one (b,h),
-// 128-byte swizzled in shared memory; rows >= N lie outside the map.
-bool encode_o_map(CUtensorMap* m, float* o, long long BH, int N) {
-  const EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {64 * sizeof(float), static_cast<cuuint64_t>(N) * 64 * sizeof(float)};
-  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(C), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int DX, int DV>
 cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p, cudaStream_t st) {
   using K = Cfg<DX, DV>;
@@ -1722,7 +1724,7 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
     if (!ws || std::atoi(ws) >= 2) {
       CUtensorMap tm_q, tm_k, tm_v, tm_o;
       if (!encode_input_map(&tm_q, args.q, args.BH, args.N) || !encode_input_map(&tm_k, args.k, args.BH, args.N) ||
-          !encode_input_map(&tm_v, args.v, args.BH, args.N) || !encode_o_map(&tm_o, args.o, args.BH, args.N))
+          !encode_input_map(&tm_v, args.v, args.BH, args.N) || !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N))
         return cudaErrorNotSupported;
       e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
       if (e != cudaSuccess) return e;
