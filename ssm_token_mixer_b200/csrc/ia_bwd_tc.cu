@@ -94,6 +94,7 @@ struct BwdArgs {
   const HeadTables* tabs;
   const uint8_t* R;  // [BH][nch] x (R_U, R_Gamma) fp16 swizzled tiles of 16 KB
   const float* Re;   // [BH][nch][128]
+  const float* dtab; // [H][128][64] d(E'')/dDelta rows, then [H][128] row sums
   float* dq;
   float* dk;
   float* dv;
@@ -156,24 +157,9 @@ __global__ void __launch_bounds__(NTHR, 1)
   const float r2 = T->r2[m];
   const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
   const float sgn = comp ? 1.f : -1.f;
-  // sum over j of d(E'[j,m])/dDelta = lambda^(c-j) (lambda + (c-j) A b), this row's component
-  float dEsum_c;
-  {
-    const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
-    const double Ar = ReA, Ai = ImA;
-    double sr = 0.0, si = 0.0;
-    for (int j = 0; j < C; ++j) {
-      const double n = C / 2 - j;
-      const double e = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
-      double sn, cs;
-      sincos(ph, &sn, &cs);
-      const double pr = e * cs, pi = e * sn;
-      const double fr = lr + n * (Ar * br - Ai * bi), fi = li + n * (Ar * bi + Ai * br);
-      sr += pr * fr - pi * fi;
-      si += pr * fi + pi * fr;
-    }
-    dEsum_c = static_cast<float>(comp ? si : sr);
-  }
+  // this row of d(E'')/dDelta over j (from the table prologue) and its sum
+  const float* dErow = a.dtab + (static_cast<size_t>(h) * KR + k) * C;
+  const float dEsum_c = a.dtab[static_cast<size_t>(a.H) * KR * C + static_cast<size_t>(h) * KR + k];
 
   // zero the state adjoint and the table adjoint
   {
@@ -503,19 +489,9 @@ __global__ void __launch_bounds__(NTHR, 1)
       const float Rp = __shfl_xor_sync(kFull, Reta, 1);
       float dEpart = dEsum_c;
       if (nv < C) {   // ragged chunk: only the valid keys carry the constant channel
-        const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
-        double sr = 0.0, si = 0.0;
-        for (int j = 0; j < nv; ++j) {
-          const double n = C / 2 - j;
-          const double e = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
-          double sn, cs;
-          sincos(ph, &sn, &cs);
-          const double pr = e * cs, pi = e * sn;
-          const double fr = lr + n * (ReA * br - ImA * bi), fi = li + n * (ReA * bi + ImA * br);
-          sr += pr * fr - pi * fi;
-          si += pr * fi + pi * fr;
-        }
-        dEpart = static_cast<float>(comp ? si : sr);
+        float acc = 0.f;
+        for (int j = 0; j < nv; ++j) acc += dErow[j];
+        dEpart = acc;
       }
       if (half == 0) {
         dD = fmaf(static_cast<float>(C), fmaf(ReA, dRe * Reta, ImA * sgn * dRe * Rp), dD);
@@ -636,22 +612,20 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (!aborted) {
     // contract the table adjoint with d(E'')/dDelta
-    const double lr = T->lam[m].x, li = T->lam[m].y, br = T->b[m].x, bi = T->b[m].y;
 #pragma unroll
     for (int cb = 0; cb < 32; cb += 16) {
       const int j0 = 32 * half + cb;
       uint32_t r[16];
       tmem_ld16(trow + B::T_EBAR + j0, r);
       tmem_ld_wait16(r);
-      for (int e = 0; e < 16; ++e) {
-        const double n = C / 2 - (j0 + e);
-        const double ex = exp(n * T->re_dA[m]), ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
-        double sn, cs;
-        sincos(ph, &sn, &cs);
-        const double pr = ex * cs, pi = ex * sn;
-        const double fr = lr + n * (ReA * br - ImA * bi), fi = li + n * (ReA * bi + ImA * br);
-        const double dE = comp ? pr * fi + pi * fr : pr * fr - pi * fi;
-        dD = fmaf(__uint_as_float(r[e]), static_cast<float>(dE), dD);
+      const float4* dq4 = reinterpret_cast<const float4*>(dErow + j0);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 d = dq4[g];
+        dD = fmaf(__uint_as_float(r[4 * g]), d.x, dD);
+        dD = fmaf(__uint_as_float(r[4 * g + 1]), d.y, dD);
+        dD = fmaf(__uint_as_float(r[4 * g + 2]), d.z, dD);
+        dD = fmaf(__uint_as_float(r[4 * g + 3]), d.w, dD);
       }
     }
     // block reduction -> one atomic per CTA
@@ -689,6 +663,7 @@ size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
   bytes += BH * nch * 2 * KR * 64 * 2;                        // R per chunk: two fp16 tiles
   bytes += BH * nch * KR * sizeof(float);                      // R_eta per chunk
   bytes += BH * s.N * sizeof(float) + 256;                     // den
+  bytes += static_cast<size_t>(s.H) * KR * (C + 1) * sizeof(float) + 256;   // dE/dDelta table
   return bytes + 256;
 }
 
@@ -704,8 +679,10 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   float* dumpRe = reinterpret_cast<float*>(dumpR + BH * nch * 2 * B::RT);
   float* den = dumpRe + BH * nch * KR;
   den = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(den) + 255) & ~static_cast<uintptr_t>(255));
+  float* dtab = den + BH * s.N;
+  dtab = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(dtab) + 255) & ~static_cast<uintptr_t>(255));
   cudaError_t e = launch_tc_prefill(s, p, q, k, v, delta, A, nullptr, o, nullptr, den, nullptr, ws,
-                                    st, dumpR, dumpRe);
+                                    st, dumpR, dumpRe, dtab);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(dDelta, 0, sizeof(float) * s.H, st);
   if (e != cudaSuccess) return e;
@@ -720,6 +697,7 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   a.tabs = tc_tables(ws);
   a.R = dumpR;
   a.Re = dumpRe;
+  a.dtab = dtab;
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;

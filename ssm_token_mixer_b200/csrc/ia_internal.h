@@ -12,7 +12,7 @@ namespace ia {
 struct HeadTables;
 
 cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
-                                cudaStream_t st);
+                                cudaStream_t st, float* dtab = nullptr);
 
 size_t seq_fwd_smem(int DX, int DV, int M);
 cudaError_t launch_seq_fwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
@@ -41,7 +41,8 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st,
-                              void* dump_R = nullptr, float* dump_Re = nullptr);
+                              void* dump_R = nullptr, float* dump_Re = nullptr,
+                              float* dtab = nullptr);
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
 

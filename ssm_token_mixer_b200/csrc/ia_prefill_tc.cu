@@ -1812,14 +1812,14 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st, void* dump_R,
-                              float* dump_Re) {
+                              float* dump_Re, float* dtab) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 255) & ~static_cast<uintptr_t>(255));
   HeadTables* tabs = reinterpret_cast<HeadTables*>(w);
   float* seg_state = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   float* seg_eta = seg_state + BH * (p.nseg > 1 ? p.nseg - 1 : 0) * KR * (s.d_xi + s.d_v);
-  cudaError_t e = launch_param_tables(s.H, delta, A, tabs, st);
+  cudaError_t e = launch_param_tables(s.H, delta, A, tabs, st, dtab);
   if (e != cudaSuccess) return e;
   TcArgs args;
   args.q = static_cast<const __nv_bfloat16*>(q);

@@ -85,10 +85,14 @@ __device__ __forceinline__ float warp_sum(float x) {
 // power (relative error ~16 * 2^-53); the sum of E' over the chunk is reduced
 // across the four threads, and the remaining per-mode powers are shared out
 // among them.  The E' table is staged in shared memory and written out with
-// coalesced 16-byte stores.
+// coalesced 16-byte stores.  With dtab, also the derivative table for the
+// reverse pass: dtab[h][k][j] = component (k & 1) of dE'[j, k/2]/dDelta =
+// lambda^n (lambda + n A b), n = c - j, fp32, followed by the row sums
+// dtab[H*128*64 + h*128 + k].
 __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const float* __restrict__ delta,
                                                                     const float* __restrict__ A,
-                                                                    HeadTables* __restrict__ tabs) {
+                                                                    HeadTables* __restrict__ tabs,
+                                                                    float* __restrict__ dtab) {
   __shared__ __align__(16) __half Es[2 * kModesTC * kChunk];
   const int h = blockIdx.x;
   HeadTables* T = tabs + h;
@@ -100,14 +104,24 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
   double pr, pi, ir, ii;
   cpow_d(rdA, idA, c - JS * part, &pr, &pi);   // lambda^(c-j) at this thread's first j
   cpow_d(rdA, idA, -1.0, &ir, &ii);            // lambda^-1
-  double sr = 0.0, si = 0.0;
+  double sr = 0.0, si = 0.0, dsr = 0.0, dsi = 0.0;
   char* base = reinterpret_cast<char*>(Es);
+  float* drow = dtab ? dtab + (static_cast<size_t>(h) * 2 * kModesTC + 2 * m) * C : nullptr;
   for (int j = JS * part; j < JS * (part + 1); ++j) {   // E'[j] = b lambda^(c-j)
     const double er = md.br * pr - md.bi * pi, ei = md.br * pi + md.bi * pr;
     *reinterpret_cast<__half*>(base + etab_offset(2 * m, j)) = __double2half(er);
     *reinterpret_cast<__half*>(base + etab_offset(2 * m + 1, j)) = __double2half(ei);
     sr += er;
     si += ei;
+    if (drow) {   // dE'[j]/dDelta = lambda^n (lambda + n A b), n = c - j
+      const double n = c - j;
+      const double fr = md.lr + n * (md.ar * md.br - md.ai * md.bi), fi = md.li + n * (md.ar * md.bi + md.ai * md.br);
+      const double dr = pr * fr - pi * fi, di = pr * fi + pi * fr;
+      drow[j] = static_cast<float>(dr);
+      drow[C + j] = static_cast<float>(di);
+      dsr += dr;
+      dsi += di;
+    }
     const double nr = pr * ir - pi * ii;
     pi = pr * ii + pi * ir;
     pr = nr;
@@ -116,6 +130,13 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
   for (int off = 1; off < 4; off <<= 1) {
     sr += __shfl_xor_sync(0xffffffffu, sr, off);
     si += __shfl_xor_sync(0xffffffffu, si, off);
+    dsr += __shfl_xor_sync(0xffffffffu, dsr, off);
+    dsi += __shfl_xor_sync(0xffffffffu, dsi, off);
+  }
+  if (dtab && part == 0) {   // row sums after the [H][128][64] table
+    float* dsum = dtab + static_cast<size_t>(H) * 2 * kModesTC * C + static_cast<size_t>(h) * 2 * kModesTC;
+    dsum[2 * m] = static_cast<float>(dsr);
+    dsum[2 * m + 1] = static_cast<float>(dsi);
   }
   if (part == 0) {
     T->lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
@@ -536,8 +557,8 @@ __global__ void segment_scan_kernel(int H, int DX, int DV, int nseg, int L,
 // ------------------------------------------------------------------------
 // host-side launchers
 cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
-                                cudaStream_t st) {
-  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs);
+                                cudaStream_t st, float* dtab) {
+  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs, dtab);
   return cudaGetLastError();
 }
 
