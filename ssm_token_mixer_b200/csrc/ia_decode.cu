@@ -10,6 +10,7 @@
 // cluster streams a group of modes with 16-byte loads and stores, keeps its
 // partial num/den in shared memory, and the cluster's rank-0 CTA sums the
 // partials over distributed shared memory and writes o.
+#include <cstdlib>
 #include <cooperative_groups.h>
 
 #include "ia_device.cuh"
@@ -344,7 +345,10 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   const long long BHc = static_cast<long long>(s.B) * s.H;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (BHc >= 2LL * sms) {   // enough (b,h) pairs to fill the GPU without splitting modes
+  // tuning switch: the smallest B*H that takes the one-CTA-per-(b,h) kernel
+  const char* thr_env = std::getenv("IA_DECODE_BH_MIN");
+  const long long thr = thr_env ? std::atoll(thr_env) : static_cast<long long>(sms);
+  if (BHc >= thr) {   // at least one (b,h) per SM: no need to split the modes across CTAs
     const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
                         sizeof(float2) * 2 * s.M + 16;
     auto kern = decode_bh_kernel<T>;

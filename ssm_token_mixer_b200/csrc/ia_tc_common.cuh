@@ -51,9 +51,10 @@ __device__ __forceinline__ void gemm_dd(uint32_t dtm, uint64_t adesc, uint32_t a
 }
 
 // bf16 staging rows [C][W] (row-major, contiguous) -> fp16 canonical tile,
-// applying xi when FEAT; rows >= nv become zero.  One warp iteration moves 8
-// rows x 4 column groups; the column group is rotated by the row so that
-// both the staging reads and the tile writes are bank-conflict free.
+// applying xi (on fp16 pairs, as the forward does) when FEAT; rows >= nv
+// become zero.  One warp iteration moves 8 rows x 4 column groups; the column
+// group is rotated by the row so that both the staging reads and the tile
+// writes are bank-conflict free.
 template <int W, bool FEAT>
 __device__ __forceinline__ void convert_tile(const uint8_t* stg, uint8_t* dst, int nv, int warp,
                                              int lane) {
@@ -72,9 +73,8 @@ __device__ __forceinline__ void convert_tile(const uint8_t* stg, uint8_t* dst, i
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float2 f = __bfloat1622float2(p[e]);
-        if (FEAT) { f.x = feat(f.x); f.y = feat(f.y); }
-        w[e] = pack_half2(f.x, f.y);
+        const float2 f = __bfloat1622float2(p[e]);
+        w[e] = FEAT ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
       }
       out = make_uint4(w[0], w[1], w[2], w[3]);
     }
