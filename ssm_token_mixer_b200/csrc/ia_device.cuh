@@ -118,22 +118,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// 16-byte global -> shared copy by one thread (cp.async, L2 only).  Copies
-// src_bytes (16 or 0) bytes and zero-fills the rest, so src_bytes = 0 writes
-// 16 zero bytes and reads nothing.  dst and src 16-byte aligned.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the barrier's expected count must include this arrival).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Waits for every cp.async this thread has committed.
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // TMA tensor load of one box (3-D tensor map) into shared memory, completing
 // on an mbarrier with the box's bytes as transaction count.  tmap is the
 // address of a __grid_constant__ CUtensorMap parameter; c0 * element size is

@@ -200,56 +200,6 @@ __device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, in
   }
 }
 
-// convert_all for the three input tiles of one chunk at once (q and k through
-// the feature map, v plain): every load is issued before the first convert,
-// so the shared-memory latency is paid once.
-template <int D, int WDV, int NW>
-__device__ __forceinline__ void convert_qkv(const uint8_t* stg_q, const uint8_t* stg_k,
-                                            const uint8_t* stg_v, uint8_t* dq, uint8_t* dk,
-                                            uint8_t* dv, int nv, int warp, int lane) {
-  constexpr int NCG = D / 8;
-  constexpr int ITERS = (C / 8) * (NCG / 4);
-  static_assert(ITERS % NW == 0, "whole iterations per warp");
-  constexpr int PER = ITERS / NW;
-  const int r8 = lane & 7, slot = lane >> 3;
-  uint4 in[3][PER];
-  int rr[PER], cc[PER];
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int it = warp + u * NW;
-    const int rb = it & 7, rest = it >> 3;
-    rr[u] = rb * 8 + r8;
-    cc[u] = (rest >> 1) * 8 + ((slot + 4 * (rest & 1) + r8) & 7);
-    const int off = rr[u] * (D * 2) + cc[u] * 16;
-    const bool live = rr[u] < nv;
-    in[0][u] = live ? *reinterpret_cast<const uint4*>(stg_q + off) : make_uint4(0u, 0u, 0u, 0u);
-    in[1][u] = live ? *reinterpret_cast<const uint4*>(stg_k + off) : make_uint4(0u, 0u, 0u, 0u);
-    in[2][u] = live ? *reinterpret_cast<const uint4*>(stg_v + off) : make_uint4(0u, 0u, 0u, 0u);
-  }
-#pragma unroll
-  for (int tsel = 0; tsel < 3; ++tsel) {
-#pragma unroll
-    for (int u = 0; u < PER; ++u) {
-      uint4 out = make_uint4(0u, 0u, 0u, 0u);
-      if (rr[u] < nv) {
-        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&in[tsel][u]);
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 f = __bfloat1622float2(p[e]);
-          if (tsel < 2) { f.x = feat(f.x); f.y = feat(f.y); }
-          w[e] = pack_half2(f.x, f.y);
-        }
-        out = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      if (tsel == 2)
-        *reinterpret_cast<uint4*>(dv + tile_off(rr[u], cc[u] * 8, WDV * 16)) = out;
-      else
-        *reinterpret_cast<uint4*>((tsel ? dk : dq) + tile_off(rr[u], cc[u] * 8, D * 16)) = out;
-    }
-  }
-}
-
 __device__ __forceinline__ uint4 pack8f(const uint32_t* r, float scale) {
   return make_uint4(pack_half2(__uint_as_float(r[0]) * scale, __uint_as_float(r[1]) * scale),
                     pack_half2(__uint_as_float(r[2]) * scale, __uint_as_float(r[3]) * scale),
