@@ -257,7 +257,7 @@ def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
     launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
     fl = flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
     by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
-    traffic = recorded_traffic("tc_prefill_full_125m.md", "ssm_token_mixer_b200/csrc/ia_prefill_tc.cu")
+    traffic = recorded_traffic("tc_prefill_ws2_125m.md", "ssm_token_mixer_b200/csrc/ia_prefill_tc.cu")
     rf = roofline(by, fl, kern_ms, peaks, peak_kind, traffic, sustained=False)
     # end to end through the public API with host buffers: H2D inputs, call, D2H o
     qh, kh, vh = (x.pin_memory() for x in (inp["q"], inp["k"], inp["v"]))
@@ -306,12 +306,24 @@ def leg_fwd_bwd(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
     barrier(dev)
     total = max_over_ranks(sum(step_ms), dev)
     tokens = w.B * w.N
-    fl = 3 * flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
-    by = bytes_fwd_bwd(w.d_xi, w.d_v) * tokens * w.H
+    # the dominant kernel is the reverse pass: its own algorithmic work is the
+    # step's minus the forward's (re-read q, k, v; read dO, o; write dq, dk, dv;
+    # two forward-sized contraction chains by the convention of 3x forward flops)
+    fl_step = 3 * flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
+    by_step = bytes_fwd_bwd(w.d_xi, w.d_v) * tokens * w.H
+    fl = 2 * flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
+    by = (bytes_fwd_bwd(w.d_xi, w.d_v) - bytes_fwd(w.d_xi, w.d_v)) * tokens * w.H
+    traffic = recorded_traffic("tc_bwd_350m.md", "ssm_token_mixer_b200/csrc/ia_bwd_tc.cu")
+    rf = roofline(by, fl, kern_ms, peaks, peak_kind, traffic, sustained=False)
+    rf["kernel"] = "reverse pass (tc_bwd_kernel)"
+    step_s = total / steps * 1e-3
+    rf["step"] = {"algorithmic_bytes": by_step, "algorithmic_flops": fl_step,
+                  "achieved_gbs": by_step / step_s / 1e9, "frac_hbm": by_step / step_s / 1e9 / float(peaks["hbm_gbs"])}
+    launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16") + 1
     res = {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
            "value": world * tokens * steps / (total * 1e-3), "unit": "tokens/s",
-           "ms_per_step": total / steps, "steps": steps, "gpu_launches": steps,
-           "roofline": roofline(by, fl, kern_ms, peaks, peak_kind, None, sustained=False)}
+           "ms_per_step": total / steps, "steps": steps, "gpu_launches": launches * steps,
+           "roofline": rf}
     if cpu_leg and rank == 0 and world == 1:
         import oracle
         sub = synthetic.workload_inputs(w, B=1)
