@@ -193,25 +193,32 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
 }
 
 // Large-batch variant: one CTA per (b,h) covers all modes, so no cluster and
-// no cross-CTA reduction is needed; each warp walks its modes with the next
-// mode's U / Gamma rows already in flight (one-deep prefetch), and keeps its
-// partial Re(a^H Gamma) in registers.
+// no cross-CTA reduction is needed.  Each warp walks its modes (warp, warp+8,
+// ...) through a ring of D shared-memory slots: bulk copies bring the U and
+// Gamma rows of the next D modes while it updates the current one, so each SM
+// keeps enough bytes in flight to cover the memory latency; the updated rows
+// go straight back to HBM and the partial Re(a^H Gamma) stays in registers.
 constexpr int kBhWarps = 8;
 
 template <typename T>
-__global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
-    int H, int DX, int DV, int M, const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
+    int H, int DX, int DV, int M, int D, const T* __restrict__ q, const T* __restrict__ k,
     const T* __restrict__ v, const float* __restrict__ delta, const float* __restrict__ A,
     float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
-    float* __restrict__ den, long long BH) {
+    float* __restrict__ den, long long BH, int* err) {
   extern __shared__ float4 dsm[];
-  float* fq = reinterpret_cast<float*>(dsm);
+  const uint32_t rowU = static_cast<uint32_t>(DX) * 8, rowG = static_cast<uint32_t>(DV) * 8, slot = rowU + rowG;
+  // ring of D mode rows (U row then Gamma row) per warp, then its mbarriers
+  uint8_t* ring = reinterpret_cast<uint8_t*>(dsm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + kBhWarps * D * slot);
+  float* fq = reinterpret_cast<float*>(bars + kBhWarps * D);
   float* fk = fq + DX;
   float* vv = fk + DX;
   float* part = vv + DV;                    // [8][DV]
   float* pden = part + kBhWarps * DV;       // [8]
   float2* lamb = reinterpret_cast<float2*>(pden + kBhWarps);   // [M]
   float2* bb = lamb + M;
+  float2* eta = bb + M;
   const long long bh = blockIdx.x;
   const int h = static_cast<int>(bh % H);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -219,19 +226,24 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
   float2* Ub = state + bh * M * DX;
   float2* Gb = state + BH * M * DX + bh * M * DV;
   float2* Eb = state + BH * M * (DX + DV) + bh * M;
+  uint8_t* myring = ring + warp * D * slot;
+  uint64_t* mybar = bars + warp * D;
+  const int nj = warp < M ? (M - warp + kBhWarps - 1) / kBhWarps : 0;   // modes warp, warp + 8, ...
 
-  float4 cu[kVecPerLane], cg[kVecPerLane], nu4[kVecPerLane], ng4[kVecPerLane];
-  auto load_mode = [&](int m, float4 (&u)[kVecPerLane], float4 (&g)[kVecPerLane]) {
-    const float4* Ur = reinterpret_cast<const float4*>(Ub + static_cast<long long>(m) * DX);
-    const float4* Gr = reinterpret_cast<const float4*>(Gb + static_cast<long long>(m) * DV);
-#pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i) {
-      const int p = lane + 32 * i;
-      if (p < nu) u[i] = Ur[p];
-      if (p < ng) g[i] = Gr[p];
-    }
+  // each warp streams its own modes' state rows through its ring, D rows ahead
+  auto issue = [&](int j) {
+    const int m = warp + kBhWarps * j, s = j % D;
+    mbar_arrive_expect_tx(mybar + s, slot);
+    bulk_g2s(myring + s * slot, Ub + static_cast<long long>(m) * DX, rowU, mybar + s);
+    bulk_g2s(myring + s * slot + rowU, Gb + static_cast<long long>(m) * DV, rowG, mybar + s);
   };
-  if (warp < M) load_mode(warp, cu, cg);
+  int issued = 0;
+  if (lane == 0) {
+    for (int s = 0; s < D; ++s) mbar_init(mybar + s, 1);
+    fence_barrier_init();
+    for (; issued < D && issued < nj; ++issued) issue(issued);
+  }
+  __syncwarp();
 
   for (int f = tid; f < DX; f += kBhWarps * 32) {
     fq[f] = xi_acc(ldx(q + bh * DX + f));
@@ -251,6 +263,7 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
     const float dd = fmaf(ar, ar, ai * ai);
     lamb[m] = make_float2(ex * cy, ex * sy);
     bb[m] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
+    eta[m] = Eb[m];
   }
   __syncthreads();
 
@@ -258,11 +271,15 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
 #pragma unroll
   for (int i = 0; i < 2 * kVecPerLane; ++i) acc[i] = 0.f;
   float dpart = 0.f;
-  for (int m = warp; m < M; m += kBhWarps) {
-    const bool more = m + kBhWarps < M;
-    if (more) load_mode(m + kBhWarps, nu4, ng4);
-    float2 e = make_float2(0.f, 0.f);
-    if (lane == 0) e = Eb[m];
+  bool ok = true;
+  for (int j = 0; j < nj; ++j) {
+    const int m = warp + kBhWarps * j, s = j % D;
+    if (!mbar_wait(mybar + s, static_cast<uint32_t>((j / D) & 1), err)) {
+      ok = false;
+      break;
+    }
+    const float4* us = reinterpret_cast<const float4*>(myring + s * slot);
+    const float4* gs = reinterpret_cast<const float4*>(myring + s * slot + rowU);
     const float2 L = lamb[m], Bm = bb[m];
     float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
     float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
@@ -271,7 +288,7 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
     for (int i = 0; i < kVecPerLane; ++i) {
       const int p = lane + 32 * i;
       if (p < nu) {
-        const float4 u = cu[i];
+        const float4 u = us[p];
         const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
         float4 w;
         w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
@@ -292,7 +309,7 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
     for (int i = 0; i < kVecPerLane; ++i) {
       const int p = lane + 32 * i;
       if (p < ng) {
-        const float4 g = cg[i];
+        const float4 g = gs[p];
         const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
         float4 w;
         w.x = fmaf(L.x, g.x, fmaf(-L.y, g.y, Bm.x * x0));
@@ -305,17 +322,21 @@ __global__ void __launch_bounds__(kBhWarps * 32, 2) decode_bh_kernel(
       }
     }
     if (lane == 0) {
+      const float2 e = eta[m];
       const float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
       Eb[m] = w;
       dpart = fmaf(ar, w.x, fmaf(ai, w.y, dpart));
     }
-    if (more) {
-#pragma unroll
-      for (int i = 0; i < kVecPerLane; ++i) {
-        cu[i] = nu4[i];
-        cg[i] = ng4[i];
-      }
+    __syncwarp();   // every lane has read slot s
+    if (lane == 0 && issued < nj) {
+      fence_async_smem();   // the generic reads of the slot come before the copy that refills it
+      issue(issued++);
     }
+  }
+  if (!ok) {   // let this warp's copies in flight land (bounded) before the block exits
+    if (lane == 0)
+      for (int j = 0; j < issued; ++j) mbar_wait(mybar + j % D, static_cast<uint32_t>((j / D) & 1), err);
+    __syncwarp();
   }
 #pragma unroll
   for (int i = 0; i < kVecPerLane; ++i) {
@@ -349,15 +370,20 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   const char* thr_env = std::getenv("IA_DECODE_BH_MIN");
   const long long thr = thr_env ? std::atoll(thr_env) : static_cast<long long>(sms);
   if (BHc >= thr) {   // at least one (b,h) per SM: no need to split the modes across CTAs
-    const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
-                        sizeof(float2) * 2 * s.M + 16;
+    // ring depth: four mode rows per warp while several CTAs still fit on an SM
+    const size_t row = static_cast<size_t>(s.d_xi + s.d_v) * 8;
+    const int D = kBhWarps * 4 * row <= 96 * 1024 ? 4 : 2;
+    const size_t smem = kBhWarps * D * (row + 8) + sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
+                        sizeof(float2) * 3 * s.M + 16;
+    int* err = device_error_ptr();
+    if (!err) return cudaErrorInvalidSymbol;
     auto kern = decode_bh_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     mark_launch_begin(st);
     kern<<<static_cast<unsigned>(BHc), kBhWarps * 32, smem, st>>>(
-        s.H, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
-        static_cast<const T*>(v), delta, A, static_cast<float2*>(state), o, num, den, BHc);
+        s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q), static_cast<const T*>(k),
+        static_cast<const T*>(v), delta, A, static_cast<float2*>(state), o, num, den, BHc, err);
     e = cudaGetLastError();
     mark_launch_end(st);
     return e;
