@@ -23,6 +23,11 @@
 //     ds     += dX * a~,  dlambda^C += sum dR conj(S_hat0)
 //     d(b lambda^n)/dDelta = (lambda + n A b) lambda^n,  ds/dDelta = 2 Re(A)(i-c) s,
 //     d(lambda^C)/dDelta = C A lambda^C.
+// A dedicated MMA warp issues the contraction groups (tcgen05.mma blocks its
+// issuing thread) on ready barriers from the 8 epilogue warps, in the order
+// F1+B1, F2, B2, F4, B3-B5, dQ/dK/dV, so the readout chain (S, a~, P) and the
+// adjoint chain (dP, dX) overlap: each epilogue runs while the other chain's
+// contraction executes; dP and dS use their own TMEM tile (T_X2).
 // The forward pass (the prefill kernel) stores R (fp16 tiles R_U, R_Gamma in
 // the 128-byte swizzled operand layout, loaded here with one bulk copy per
 // chunk, one chunk ahead), R_eta (fp32) and den for every chunk.
@@ -45,7 +50,7 @@ using namespace tc;
 struct B {
   static constexpr int DX = 64, DV = 64, F = 128;
   static constexpr uint32_t T_ADJ = 0, T_EBAR = 128, T_A = 192, T_DK = 192, T_DX = 256,
-                            T_DV = 256, T_SP = 320, T_DQ = 384;
+                            T_DV = 256, T_SP = 320, T_DQ = 384, T_X2 = 448;
   static constexpr uint32_t TILE64 = C * 64 * 2;     // 8 KB: [64 rows][64 cols] fp16
   static constexpr uint32_t TILE128 = KR * 64 * 2;   // 16 KB: [128 rows][64 cols] fp16
   static constexpr uint32_t STG_Q = 0;
@@ -68,8 +73,9 @@ struct B {
   static constexpr uint32_t S_DS1 = S_RG + TILE128;          // [128][F] fp16
   static constexpr uint32_t S_DD = S_DS1 + KR * F * 2;       // dden [64] fp32
   static constexpr uint32_t S_RED = S_DD + C * 4;            // dR_eta halves [2][128] fp32
-  static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;    // bar_tma, bar_mma, bar_r
-  static constexpr uint32_t S_TMEMH = S_BAR + 32;
+  static constexpr uint32_t S_BAR = S_RED + 2 * KR * 4;    // 17 mbarriers (see the kernel)
+  static constexpr uint32_t S_FLAG = S_BAR + 17 * 8;       // abort flag
+  static constexpr uint32_t S_TMEMH = S_FLAG + 8;
   static constexpr uint32_t S_OST = S_TMEMH + 16;            // o rows of the chunk, fp32 [64][64]
   static constexpr uint32_t RT = KR * 64 * 2;                // one fp16 R tile: 16 KB
   // dq, dk, dv leave by TMA stores from tiles that are free between the
@@ -109,7 +115,10 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
                     pack_half2(x[6], x[7]));
 }
 
-__global__ void __launch_bounds__(NTHR, 1)
+constexpr int NEPI = NTHR;        // epilogue threads (warps 0-7)
+constexpr int NBWD = NEPI + 32;   // + one MMA warp
+
+__global__ void __launch_bounds__(NBWD, 1)
     tc_bwd_kernel(const __grid_constant__ BwdArgs a, const __grid_constant__ CUtensorMap tm_dq,
                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv) {
   constexpr int DX = B::DX, DV = B::DV, F = B::F;
@@ -120,9 +129,12 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int h = static_cast<int>(bh % a.H);
   const HeadTables* T = a.tabs + h;
   const int nch = (a.N + C - 1) / C;
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + B::S_BAR);
-  uint64_t* bar_mma = bar_tma + 1;
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + B::S_BAR);   // q, k, v, dO, o of a chunk
+  uint64_t* bar_drain = bar_tma + 1;
   uint64_t* bar_r = bar_tma + 2;   // the R tiles of the next chunk to process
+  uint64_t* rdy = bar_tma + 3;     // [6] epilogue -> MMA warp: operands of group i are in place
+  uint64_t* dn = bar_tma + 9;      // [7] MMA warp -> epilogue: F1, B1, F2, B2, F4, B3-B5, G done
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + B::S_FLAG);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + B::S_TMEMH);
   float* sDD = reinterpret_cast<float*>(smem + B::S_DD);
   float* sRED = reinterpret_cast<float*>(smem + B::S_RED);
@@ -134,14 +146,17 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   if (tid == 0) {
     mbar_init(bar_tma, 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar_drain, 1);
     mbar_init(bar_r, 1);
+    for (int i = 0; i < 6; ++i) mbar_init(rdy + i, NEPI);
+    for (int i = 0; i < 7; ++i) mbar_init(dn + i, 1);
+    *abort_flag = 0;
     fence_barrier_init();
   }
   {
     const uint4* src = reinterpret_cast<const uint4*>(T->E);
     uint4* dst = reinterpret_cast<uint4*>(smem + B::S_E);
-    for (int i = tid; i < static_cast<int>(B::TILE128 / 16); i += NTHR) dst[i] = src[i];
+    for (int i = tid; i < static_cast<int>(B::TILE128 / 16); i += NBWD) dst[i] = src[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -162,7 +177,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   const float dEsum_c = a.dtab[static_cast<size_t>(a.H) * KR * C + static_cast<size_t>(h) * KR + k];
 
   // zero the state adjoint and the table adjoint
-  {
+  if (warp < NEPI / 32) {
     uint32_t z[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) z[e] = 0u;
@@ -197,31 +212,125 @@ __global__ void __launch_bounds__(NTHR, 1)
   // den of row tid/4 of the next chunk to process, loaded a chunk ahead
   auto load_den = [&](int ch) -> float {
     const int i = tid >> 2;
-    return i < a.N - ch * C ? a.den[bh * a.N + ch * C + i] : 1.f;
+    return tid < NEPI && i < a.N - ch * C ? a.den[bh * a.N + ch * C + i] : 1.f;
   };
   float den_next = load_den(nch - 1);
   bool tma_pending = true, r_pending = true;
-  uint32_t ph_tma = 0, ph_mma = 0, ph_r = 0;
+  uint32_t ph_tma = 0, ph_r = 0;
   bool aborted = false;
-  auto mma_sync = [&]() -> bool {
-    bool ok = mbar_wait(bar_mma, ph_mma, a.err);
-    ph_mma ^= 1u;
-    tc_fence_after();
-    return !__syncthreads_or(!ok);
-  };
-  auto to_tc = [&]() {
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-  };
-
+  if (warp == NEPI / 32) {
+    // ------------------------------------------------ MMA warp: the contraction groups, in order
+    if (lane == 0) {
+      uint32_t pr[6] = {0u, 0u, 0u, 0u, 0u, 0u};
+      bool ok = true;
+      auto wait_rdy = [&](int i) -> bool {
+        const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
+        pr[i] ^= 1u;
+        tc_fence_after();
+        return r;
+      };
+      for (int ch = nch - 1; ch >= 0; --ch) {
+        if (!(ok = wait_rdy(0))) break;   // operands, R, dS1 of the chunk
+        // F1: S^T = xi(K) xi(Q)^T
+        gemm(tmem + B::T_SP, sb + B::S_K, kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), sb + B::S_Q,
+             kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(64, 64, 0, 0), DX / 16, false);
+        mma_commit(dn + 0);
+        // B1: dP = dnum V^T
+        gemm(tmem + B::T_X2, sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), sb + B::S_V,
+             kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(64, 64, 0, 0), DV / 16, false);
+        mma_commit(dn + 1);
+        if (!(ok = wait_rdy(1))) break;   // E1 done
+        // F2: a~^T = E''^T S^T + R_U xi(Q)^T
+        gemm(tmem + B::T_A, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S,
+             mn_lbo(64), mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, false);
+        gemm_dd(tmem + B::T_A, smem_desc_sw128(sb + B::S_RU, 16, 1024), 32,
+                smem_desc(sb + B::S_Q, kmaj_lbo(), kmaj_sbo(DX)), kmaj_step(), idesc_f16(128, 64, 0, 0),
+                DX / 16, true);
+        mma_commit(dn + 2);
+        if (!(ok = wait_rdy(2))) break;   // dP done
+        // B2: dX^T = E''^T dP^T + R_G dnum^T
+        gemm(tmem + B::T_DX, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP,
+             kmaj_lbo(), kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, false);
+        gemm_dd(tmem + B::T_DX, smem_desc_sw128(sb + B::S_RG, 16, 1024), 32,
+                smem_desc(sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV)), kmaj_step(), idesc_f16(128, 64, 0, 0),
+                DV / 16, true);
+        mma_commit(dn + 3);
+        if (!(ok = wait_rdy(3))) break;   // E2 done
+        // F4: P = X E''^T
+        gemm(tmem + B::T_SP, sb + B::S_X, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_E, mn_lbo(64),
+             mn_sbo(), mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
+        mma_commit(dn + 4);
+        if (!(ok = wait_rdy(4))) break;   // dX done
+        {
+        const uint32_t sDA = sb + B::S_DA, sX = sb + B::S_X, sE = sb + B::S_E;
+        // B3: dS = da~ E''^T
+        gemm(tmem + B::T_X2, sDA, mn_lbo(64), mn_sbo(), mn_step(64), sE, mn_lbo(64), mn_sbo(),
+             mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
+        // B4, B5: dR += [da~^T xi(Q) | X^T dnum]
+        gemm(tmem + B::T_ADJ, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_Q, mn_lbo(DX),
+             mn_sbo(), mn_step(DX), idesc_f16(128, DX, 0, 1), C / 16, true);
+        gemm(tmem + B::T_ADJ + DX, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DN,
+             mn_lbo(DV), mn_sbo(), mn_step(DV), idesc_f16(128, DV, 0, 1), C / 16, true);
+        // table adjoint: dE''^T += da~^T S + X^T dP + dS1 x^T
+        gemm(tmem + B::T_EBAR, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S, kmaj_lbo(),
+             kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, true);
+        gemm(tmem + B::T_EBAR, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP, mn_lbo(64),
+             mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, true);
+        gemm(tmem + B::T_EBAR, sb + B::S_DS1, kmaj_lbo(), kmaj_sbo(F), kmaj_step(), sb + B::S_K,
+             kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16, true);
+        gemm(tmem + B::T_EBAR, sb + B::S_DS1 + (DX / 8) * 128, kmaj_lbo(), kmaj_sbo(F), kmaj_step(),
+             sb + B::S_V, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16,
+             true);
+        }
+        mma_commit(dn + 5);
+        if (!(ok = wait_rdy(5))) break;   // E3, carry and dS done
+        {
+        const uint32_t sDS = sb + B::S_DS, sDA = sb + B::S_DA, sE = sb + B::S_E, sDS1 = sb + B::S_DS1;
+        // dQ = dS xi(K) + da~ R_U
+        gemm(tmem + B::T_DQ, sDS, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_K, mn_lbo(DX),
+             mn_sbo(), mn_step(DX), idesc_f16(64, DX, 0, 1), C / 16, false);
+        gemm_dd(tmem + B::T_DQ, smem_desc(sDA, mn_lbo(64), mn_sbo()), mn_step(64),
+                smem_desc_sw128(sb + B::S_RU, 16, 1024), 2048, idesc_f16(64, DX, 1, 1), KR / 16, true);
+        // dK = dS^T xi(Q) + E'' dS1_U
+        gemm(tmem + B::T_DK, sDS, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_Q, mn_lbo(DX),
+             mn_sbo(), mn_step(DX), idesc_f16(64, DX, 1, 1), C / 16, false);
+        gemm(tmem + B::T_DK, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1, mn_lbo(F), mn_sbo(),
+             mn_step(F), idesc_f16(64, DX, 1, 1), KR / 16, true);
+        // dV = P^T dnum + E'' dS1_G
+        gemm(tmem + B::T_DV, sb + B::S_P, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_DN, mn_lbo(DV),
+             mn_sbo(), mn_step(DV), idesc_f16(64, DV, 1, 1), C / 16, false);
+        gemm(tmem + B::T_DV, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1 + (DX / 8) * 128, mn_lbo(F),
+             mn_sbo(), mn_step(F), idesc_f16(64, DV, 1, 1), KR / 16, true);
+        }
+        mma_commit(dn + 6);
+      }
+      if (!ok) {   // drain every group issued so far
+        mma_commit(bar_drain);
+        mbar_wait(bar_drain, 0u, a.err);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue warps
+    uint32_t pd[7] = {0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    auto wait_dn = [&](int i) -> bool {   // outcome uniform over the epilogue warps
+      const bool r = mbar_wait_or_abort(dn + i, pd[i], a.err, abort_flag);
+      pd[i] ^= 1u;
+      tc_fence_after();
+      return !named_sync_or(1, NEPI, !r);
+    };
+    auto signal = [&](int i) {   // this thread's shared / TMEM writes are done
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(rdy + i);
+    };
   for (int ch = nch - 1; ch >= 0; --ch) {
     const int n0 = ch * C;
     const int nv = min(C, a.N - n0);
     {
-      bool ok = mbar_wait(bar_tma, ph_tma, a.err);
+      bool ok = mbar_wait_or_abort(bar_tma, ph_tma, a.err, abort_flag);
       ph_tma ^= 1u;
-      if (__syncthreads_or(!ok)) { aborted = true; break; }
+      if (named_sync_or(1, NEPI, !ok)) { aborted = true; break; }
       tma_pending = false;
     }
     // ---- P0: operands of this chunk
@@ -261,14 +370,14 @@ __global__ void __launch_bounds__(NTHR, 1)
       if (part == 0) sDD[i] = i < nv ? -dot * rden : 0.f;
     }
     if (ch > 0) den_next = load_den(ch - 1);
-    __syncthreads();   // staging consumed
+    named_sync(1, NEPI);   // staging consumed
     if (tid == 0 && ch > 0) issue_load(ch - 1);
     tma_pending = ch > 0;
     const float Reta = a.Re[(bh * nch + ch) * KR + k];
     {  // the R tiles of this chunk have landed; dS1 -> fp16
-      bool ok = mbar_wait(bar_r, ph_r, a.err);
+      bool ok = mbar_wait_or_abort(bar_r, ph_r, a.err, abort_flag);
       ph_r ^= 1u;
-      if (__syncthreads_or(!ok)) { aborted = true; break; }
+      if (named_sync_or(1, NEPI, !ok)) { aborted = true; break; }
       r_pending = false;
       for (int cb = 0; cb < 64; cb += 16) {
         const int col0 = half * 64 + cb;
@@ -282,14 +391,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         *reinterpret_cast<uint4*>(smem + B::S_DS1 + tile_off(k, col0 + 8, F * 16)) = pack8(xs + 8);
       }
     }
-    to_tc();
-    if (tid == 0) {   // F1: S^T = xi(K) xi(Q)^T
-      tc_fence_after();
-      gemm(tmem + B::T_SP, sb + B::S_K, kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), sb + B::S_Q,
-           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(64, 64, 0, 0), DX / 16, false);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
+    signal(0);
+    if (!wait_dn(0)) { aborted = true; break; }   // F1
     {  // E1: masked S^T -> [j][i]
       const int j = 16 * quad + lane;
 #pragma unroll
@@ -308,18 +411,29 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
       }
     }
-    to_tc();
-    if (tid == 0) {   // F2: a~^T = E''^T S^T + R_U xi(Q)^T
-      tc_fence_after();
-      bulk_wait_read_0();   // last chunk's dq/dk/dv staging (sX, sP, sDP, sDA) has been read
-      gemm(tmem + B::T_A, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S,
-           mn_lbo(64), mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, false);
-      gemm_dd(tmem + B::T_A, smem_desc_sw128(sb + B::S_RU, 16, 1024), 32,
-              smem_desc(sb + B::S_Q, kmaj_lbo(), kmaj_sbo(DX)), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16,
-              true);
-      mma_commit(bar_mma);
+    signal(1);
+    if (tid == 0) bulk_wait_read_0();   // last chunk's dq/dk/dv staging (sX, sP, sDP, sDA) has been read
+    if (!wait_dn(1)) { aborted = true; break; }   // B1
+    {  // E_dP: + dden_i, mask j <= i -> [i][j]
+      const int i = 16 * quad + lane;
+      const float ddi = lane < 16 ? sDD[i] : 0.f;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_X2 + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) + ddi : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
     }
-    if (!mma_sync()) { aborted = true; break; }
+    signal(2);
+    if (!wait_dn(2)) { aborted = true; break; }   // F2
     {  // E2: X = s a~  (rows k), dR_eta partial = sum_i X dden_i
       float s = s_start, acc = 0.f;
 #pragma unroll
@@ -340,68 +454,8 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       sRED[half * KR + k] = acc;
     }
-    to_tc();
-    if (tid == 0) {   // F4: P = X E''^T
-      tc_fence_after();
-      gemm(tmem + B::T_SP, sb + B::S_X, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_E, mn_lbo(64),
-           mn_sbo(), mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-    {  // E3: masked P -> [i][j]
-      const int i = 16 * quad + lane;
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
-    }
-    to_tc();
-    if (tid == 0) {   // B1: dP = dnum V^T
-      tc_fence_after();
-      gemm(tmem + B::T_SP, sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), sb + B::S_V,
-           kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(64, 64, 0, 0), DV / 16, false);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-    {  // E_dP: + dden_i, mask j <= i -> [i][j]
-      const int i = 16 * quad + lane;
-      const float ddi = lane < 16 ? sDD[i] : 0.f;
-#pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) + ddi : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
-    }
-    to_tc();
-    if (tid == 0) {   // B2: dX^T = E''^T dP^T + R_G dnum^T
-      tc_fence_after();
-      gemm(tmem + B::T_DX, sb + B::S_E, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP,
-           kmaj_lbo(), kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, false);
-      gemm_dd(tmem + B::T_DX, smem_desc_sw128(sb + B::S_RG, 16, 1024), 32,
-              smem_desc(sb + B::S_DN, kmaj_lbo(), kmaj_sbo(DV)), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16,
-              true);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
+    signal(3);
+    if (!wait_dn(3)) { aborted = true; break; }   // B2
     {  // E_dX: dX += R_eta dden; da~ = s dX; dDelta += dX a~ ds/dDelta
       float s = s_start;
 #pragma unroll
@@ -425,31 +479,26 @@ __global__ void __launch_bounds__(NTHR, 1)
         *reinterpret_cast<uint4*>(smem + B::S_DA + tile_off(k, i0 + 8, 1024)) = pack8(xs + 8);
       }
     }
-    to_tc();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sDA = sb + B::S_DA, sX = sb + B::S_X, sE = sb + B::S_E;
-      // B3: dS = da~ E''^T
-      gemm(tmem + B::T_SP, sDA, mn_lbo(64), mn_sbo(), mn_step(64), sE, mn_lbo(64), mn_sbo(),
-           mn_step(64), idesc_f16(64, 64, 1, 1), KR / 16, false);
-      // B4, B5: dR += [da~^T xi(Q) | X^T dnum]
-      gemm(tmem + B::T_ADJ, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_Q, mn_lbo(DX),
-           mn_sbo(), mn_step(DX), idesc_f16(128, DX, 0, 1), C / 16, true);
-      gemm(tmem + B::T_ADJ + DX, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DN,
-           mn_lbo(DV), mn_sbo(), mn_step(DV), idesc_f16(128, DV, 0, 1), C / 16, true);
-      // table adjoint: dE''^T += da~^T S + X^T dP + dS1 x^T
-      gemm(tmem + B::T_EBAR, sDA, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_S, kmaj_lbo(),
-           kmaj_sbo(64), kmaj_step(), idesc_f16(128, 64, 0, 0), C / 16, true);
-      gemm(tmem + B::T_EBAR, sX, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_DP, mn_lbo(64),
-           mn_sbo(), mn_step(64), idesc_f16(128, 64, 0, 1), C / 16, true);
-      gemm(tmem + B::T_EBAR, sb + B::S_DS1, kmaj_lbo(), kmaj_sbo(F), kmaj_step(), sb + B::S_K,
-           kmaj_lbo(), kmaj_sbo(DX), kmaj_step(), idesc_f16(128, 64, 0, 0), DX / 16, true);
-      gemm(tmem + B::T_EBAR, sb + B::S_DS1 + (DX / 8) * 128, kmaj_lbo(), kmaj_sbo(F), kmaj_step(),
-           sb + B::S_V, kmaj_lbo(), kmaj_sbo(DV), kmaj_step(), idesc_f16(128, 64, 0, 0), DV / 16,
-           true);
-      mma_commit(bar_mma);
+    signal(4);
+    if (!wait_dn(4)) { aborted = true; break; }   // F4
+    {  // E3: masked P -> [i][j]
+      const int i = 16 * quad + lane;
+#pragma unroll
+      for (int cb = 0; cb < 32; cb += 16) {
+        const int j0 = 32 * half + cb;
+        uint32_t r[16];
+        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld_wait16(r);
+        if (lane < 16) {
+          float xs[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) : 0.f;
+          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0, 1024)) = pack8(xs);
+          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
+        }
+      }
     }
-    if (!mma_sync()) { aborted = true; break; }
+    if (!wait_dn(5)) { aborted = true; break; }   // B3-B5, table adjoint
     // dR of this chunk is complete: Delta terms, then the carry to the previous chunk
     {  // adjoint carry: dS_hat0 = conj(lambda^C) dR;  dDelta += C Re(conj(sum dR conj(R)) A)
       for (int cb = 0; cb < 64; cb += 16) {
@@ -500,14 +549,14 @@ __global__ void __launch_bounds__(NTHR, 1)
       de_c = fmaf(lamC.x, dRe, -sgn * lamC.y * y);
     }
     tc_fence_before();
-    __syncthreads();
+    named_sync(1, NEPI);
     {  // E_dS: mask (j <= i, j < nv) -> [i][j]
       const int i = 16 * quad + lane;
 #pragma unroll
       for (int cb = 0; cb < 32; cb += 16) {
         const int j0 = 32 * half + cb;
         uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + j0, r);
+        tmem_ld16(trow + B::T_X2 + j0, r);
         tmem_ld_wait16(r);
         if (lane < 16) {
           float xs[16];
@@ -519,28 +568,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
       }
     }
-    to_tc();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sDS = sb + B::S_DS, sDA = sb + B::S_DA, sE = sb + B::S_E, sDS1 = sb + B::S_DS1;
-      // dQ = dS xi(K) + da~ R_U
-      gemm(tmem + B::T_DQ, sDS, kmaj_lbo(), kmaj_sbo(64), kmaj_step(), sb + B::S_K, mn_lbo(DX),
-           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 0, 1), C / 16, false);
-      gemm_dd(tmem + B::T_DQ, smem_desc(sDA, mn_lbo(64), mn_sbo()), mn_step(64),
-              smem_desc_sw128(sb + B::S_RU, 16, 1024), 2048, idesc_f16(64, DX, 1, 1), KR / 16, true);
-      // dK = dS^T xi(Q) + E'' dS1_U
-      gemm(tmem + B::T_DK, sDS, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_Q, mn_lbo(DX),
-           mn_sbo(), mn_step(DX), idesc_f16(64, DX, 1, 1), C / 16, false);
-      gemm(tmem + B::T_DK, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1, mn_lbo(F), mn_sbo(),
-           mn_step(F), idesc_f16(64, DX, 1, 1), KR / 16, true);
-      // dV = P^T dnum + E'' dS1_G
-      gemm(tmem + B::T_DV, sb + B::S_P, mn_lbo(64), mn_sbo(), mn_step(64), sb + B::S_DN, mn_lbo(DV),
-           mn_sbo(), mn_step(DV), idesc_f16(64, DV, 1, 1), C / 16, false);
-      gemm(tmem + B::T_DV, sE, mn_lbo(64), mn_sbo(), mn_step(64), sDS1 + (DX / 8) * 128, mn_lbo(F),
-           mn_sbo(), mn_step(F), idesc_f16(64, DV, 1, 1), KR / 16, true);
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
+    signal(5);
+    if (!wait_dn(6)) { aborted = true; break; }   // dQ, dK, dV
     if (tid == 0 && ch > 0) issue_r(ch - 1);   // R tiles are free: every contraction reading them is done
     r_pending = ch > 0;
     {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1).  Staged as
@@ -594,7 +623,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
       }
       fence_async_smem();
-      __syncthreads();
+      named_sync(1, NEPI);
       if (tid == 0) {
         const int y = n0, z = static_cast<int>(bh);
         tma_store_3d(&tm_dq, sb + B::O_DQ, 0, y, z);
@@ -607,7 +636,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
     }
     tc_fence_before();
-    __syncthreads();
+    named_sync(1, NEPI);
   }
 
   if (!aborted) {
@@ -631,19 +660,20 @@ __global__ void __launch_bounds__(NTHR, 1)
     // block reduction -> one atomic per CTA
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dD += __shfl_xor_sync(kFull, dD, off);
-    __syncthreads();
+    named_sync(1, NEPI);
     if (lane == 0) sRED[warp] = dD;
-    __syncthreads();
+    named_sync(1, NEPI);
     if (tid == 0) {
       float s = 0.f;
-      for (int w = 0; w < NTHR / 32; ++w) s += sRED[w];
+      for (int w = 0; w < NEPI / 32; ++w) s += sRED[w];
       atomicAdd(a.dDelta + h, s);
     }
   } else {   // let our own copies land before exiting (bounded)
-    if (tma_pending) mbar_wait(bar_tma, ph_tma, a.err);
-    if (r_pending) mbar_wait(bar_r, ph_r, a.err);
+    if (tid == 0 && tma_pending) mbar_wait(bar_tma, ph_tma, a.err);
+    if (tid == 0 && r_pending) mbar_wait(bar_r, ph_r, a.err);
   }
-  if (tid == 0) bulk_wait_all();   // dq, dk, dv are in global memory before the block exits
+    if (tid == 0) bulk_wait_all();   // dq, dk, dv are in global memory before the block exits
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -714,7 +744,7 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B::SMEM);
   if (e != cudaSuccess) return e;
   mark_launch_begin(st);
-  tc_bwd_kernel<<<static_cast<unsigned>(BH), NTHR, B::SMEM, st>>>(a, tm_dq, tm_dk, tm_dv);
+  tc_bwd_kernel<<<static_cast<unsigned>(BH), NBWD, B::SMEM, st>>>(a, tm_dq, tm_dk, tm_dv);
   e = cudaGetLastError();
   mark_launch_end(st);
   return e;
