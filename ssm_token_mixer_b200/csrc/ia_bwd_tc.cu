@@ -34,7 +34,7 @@
 //
 // TMEM columns: [0,128) adjoint of the state (dS1, then dR, then dS_hat0);
 // [128,192) dE''^T; [192,256) a~^T then dK; [256,320) dX^T then dV;
-// [320,384) S^T, P, dP, dS (M=64 layout); [384,448) dQ.
+// [320,384) S^T, then P (M=64 layout); [384,448) dQ; [448,512) dP, then dS.
 #include <cmath>
 
 #include "ia_device.cuh"
