@@ -7,10 +7,12 @@ A step is one call of the layer over one batch of synthetic, seeded input
 with the inputs already resident in HBM.  The headline value is the prefill
 forward of the 125M-layer shape (B=8, H=12, N=2048, d_xi=d_v=64, M=64, bf16
 inputs): every row of the forward path (parameter tables, feature map, chunk
-Gram/decay contractions, carried-state reads, readout, chunk carries and the
-segment scan) runs in each step.  The same line carries the training step
-(forward + reverse mode, 350M-layer shape) and the graphed decode step
-(1.3B-layer shape, B = 1/16/64) as separate legs, each timed the same way.
+Gram/decay contractions, carried-state reads, readout, chunk carries) runs in
+each step.  The same line carries, as separate legs timed the same way, the
+training step (forward + reverse mode, 350M-layer shape), the graphed decode
+step (1.3B-layer shape, B = 1/16/64) and a long-context prefill (1.3B-layer
+shape, B=1, N=7168) whose 16 sequences the planner splits into segments, so
+its steps also run the state-only pass and the inter-segment carry scan.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream, with the L2 flushed (a 256 MB write) between steps
@@ -292,6 +294,37 @@ def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
     return res
 
 
+def leg_prefill_long(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world):
+    """Long-context prefill of few sequences: the planner splits them into
+    segments, so a step runs the table prologue, the state-only pass, the
+    carry scan and the full chunk pass (the dominant kernel, timed live)."""
+    import torch
+    import ssm_token_mixer_b200 as ia
+    from ssm_token_mixer_b200 import synthetic
+    inp = synthetic.workload_inputs(w)
+    q, k, v, delta = (inp[n].to(dev) for n in ("q", "k", "v", "delta"))
+    o = torch.empty(w.B, w.H, w.N, w.d_v, dtype=torch.float32, device=dev)
+    need = ia.prefill_workspace_bytes(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    fn = lambda: ia.prefill_fwd(q, k, v, delta, w.M, o=o, workspace=ws)
+    barrier(dev)
+    step_ms, kern_ms = timer.run(fn, steps, warmup)
+    barrier(dev)
+    total = max_over_ranks(sum(step_ms), dev)
+    tokens = w.B * w.N
+    launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
+    fl = flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
+    by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
+    rf = roofline(by, fl, kern_ms, peaks, peak_kind, None, sustained=False)
+    rf["kernel"] = "full chunk pass"
+    step_s = total / steps * 1e-3
+    rf["step"] = {"achieved_gbs": by / step_s / 1e9, "frac_hbm": by / step_s / 1e9 / float(peaks["hbm_gbs"])}
+    return {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
+            "value": world * tokens * steps / (total * 1e-3), "unit": "tokens/s",
+            "ms_per_step": total / steps, "steps": steps, "launches_per_step": launches,
+            "gpu_launches": launches * steps, "roofline": rf}
+
+
 def leg_fwd_bwd(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_leg):
     import torch
     import ssm_token_mixer_b200 as ia
@@ -470,7 +503,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--legs", default="prefill,fwd_bwd,decode",
+    ap.add_argument("--legs", default="prefill,fwd_bwd,decode,prefill_long",
                     help="comma list of legs to run (prefill is the headline)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--workload", default="prefill_125m", help="headline prefill workload")
@@ -526,6 +559,11 @@ def main():
             r = leg_decode(dev, WORKLOADS["decode_1p3b"], args.steps, args.warmup, timer, peaks, peak_kind,
                            rank, world, cpu)
             line["decode"] = r
+        if "prefill_long" in legs:
+            r = leg_prefill_long(dev, WORKLOADS["prefill_1p3b_7168"], args.steps, args.warmup, timer, peaks,
+                                 peak_kind, rank, world)
+            line["prefill_long"] = r
+            extra_launches += r["gpu_launches"]
         line["gpu_launches_all_legs"] = line.get("gpu_launches", 0) + extra_launches + sum(
             b["gpu_launches"] for b in line.get("decode", {}).get("batches", {}).values())
     finally:
