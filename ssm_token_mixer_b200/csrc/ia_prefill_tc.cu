@@ -1514,8 +1514,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
     // and 32-63) in the 128-byte swizzled layout, which keeps the row-per-lane
     // writes free of bank conflicts, then written by one TMA store per box.
     // Rows past the sequence lie outside the tensor map and are not written.
-    // Staging alternates between two buffers; before one is reused, the
-    // issuing thread has seen its previous store finish reading it.
+    // Staging alternates between two buffers.  Before the barrier that
+    // precedes each store, the issuing thread waits until the store before it
+    // has finished reading its buffer; every thread passes that barrier before
+    // it writes that buffer again one chunk later.
     auto e4 = [&](int ch, int nv) {
       const int i = 16 * quad + lane;
       uint32_t rd, rr[2][16];
@@ -1553,6 +1555,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
         }
       }
       fence_async_smem();
+      if (tid == W2_GT) bulk_wait_read_0();
       named_sync(1, W2_GT);
       if (tid == W2_GT) {
         tma_store_3d(&tm_o, sbase + stage, 0, ch * C, static_cast<int>(bh));
@@ -1562,6 +1565,7 @@ __global__ void __launch_bounds__(W2_NT, 1)
     };
     bool ok = true;
     int prev = -1, prev_nv = C;
+    // E2(t) comes before E4(t-1) so that G4(t) can start while E4 runs;
     // t == ch1 runs only the tail (E3, E4) of the last chunk
     for (int t = ch0; ok && t <= ch1 && ch0 < ch1; ++t) {
       const bool head = t < ch1;
@@ -1591,11 +1595,6 @@ __global__ void __launch_bounds__(W2_NT, 1)
           signalB(1);
         }
       }
-      if (prev >= 0) {
-        if (tid == W2_GT) bulk_wait_read_1();   // the staging buffer e4 is about to fill is free
-        if (!(ok = waitB(3))) break;   // G5 + G6(t-1)
-        e4(prev, prev_nv);
-      }
       if (head) {
         if (!(ok = waitB(1))) break;   // G2 + G3(t)
         {  // E2(t): X = |lambda|^(2(i-c)) a~
@@ -1619,6 +1618,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
           }
           signalB(2);
         }
+      }
+      if (prev >= 0) {
+        if (!(ok = waitB(3))) break;   // G5 + G6(t-1)
+        e4(prev, prev_nv);
       }
       prev = t;
       prev_nv = nv;
