@@ -125,6 +125,9 @@ __global__ void __launch_bounds__(NBWD, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
+  // The M = 64 accumulators fill lanes 0-15 of each quadrant: thread t of an
+  // epilogue warp takes row 16 * quad + t % 16 and 16 of the warp's 32 columns.
+  const int r16 = 16 * quad + (lane & 15), c16 = 32 * half + 16 * (lane >> 4);
   const long long bh = blockIdx.x;
   const int h = static_cast<int>(bh % a.H);
   const HeadTables* T = a.tabs + h;
@@ -394,43 +397,31 @@ __global__ void __launch_bounds__(NBWD, 1)
     signal(0);
     if (!wait_dn(0)) { aborted = true; break; }   // F1
     {  // E1: masked S^T -> [j][i]
-      const int j = 16 * quad + lane;
+      const int j = r16, i0 = c16;
+      uint32_t r[16];
+      tmem_ld16_halves<16>(trow + B::T_SP + 32 * half, r);
+      tmem_ld_wait16(r);
+      float xs[16];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int i0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + i0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            xs[e] = (j < nv && i0 + e >= j) ? __uint_as_float(r[e]) : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
+      for (int e = 0; e < 16; ++e)
+        xs[e] = (j < nv && i0 + e >= j) ? __uint_as_float(r[e]) : 0.f;
+      *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0, 1024)) = pack8(xs);
+      *reinterpret_cast<uint4*>(smem + B::S_S + tile_off(j, i0 + 8, 1024)) = pack8(xs + 8);
     }
     signal(1);
     if (tid == 0) bulk_wait_read_0();   // last chunk's dq/dk/dv staging (sX, sP, sDP, sDA) has been read
     if (!wait_dn(1)) { aborted = true; break; }   // B1
     {  // E_dP: + dden_i, mask j <= i -> [i][j]
-      const int i = 16 * quad + lane;
-      const float ddi = lane < 16 ? sDD[i] : 0.f;
+      const int i = r16, j0 = c16;
+      const float ddi = sDD[i];
+      uint32_t r[16];
+      tmem_ld16_halves<16>(trow + B::T_X2 + 32 * half, r);
+      tmem_ld_wait16(r);
+      float xs[16];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_X2 + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) + ddi : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
+      for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) + ddi : 0.f;
+      *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0, 1024)) = pack8(xs);
+      *reinterpret_cast<uint4*>(smem + B::S_DP + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
     }
     signal(2);
     if (!wait_dn(2)) { aborted = true; break; }   // F2
@@ -482,21 +473,15 @@ __global__ void __launch_bounds__(NBWD, 1)
     signal(4);
     if (!wait_dn(4)) { aborted = true; break; }   // F4
     {  // E3: masked P -> [i][j]
-      const int i = 16 * quad + lane;
+      const int i = r16, j0 = c16;
+      uint32_t r[16];
+      tmem_ld16_halves<16>(trow + B::T_SP + 32 * half, r);
+      tmem_ld_wait16(r);
+      float xs[16];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_SP + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
+      for (int e = 0; e < 16; ++e) xs[e] = (j0 + e <= i) ? __uint_as_float(r[e]) : 0.f;
+      *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0, 1024)) = pack8(xs);
+      *reinterpret_cast<uint4*>(smem + B::S_P + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
     }
     if (!wait_dn(5)) { aborted = true; break; }   // B3-B5, table adjoint
     // dR of this chunk is complete: Delta terms, then the carry to the previous chunk
@@ -551,22 +536,16 @@ __global__ void __launch_bounds__(NBWD, 1)
     tc_fence_before();
     named_sync(1, NEPI);
     {  // E_dS: mask (j <= i, j < nv) -> [i][j]
-      const int i = 16 * quad + lane;
+      const int i = r16, j0 = c16;
+      uint32_t r[16];
+      tmem_ld16_halves<16>(trow + B::T_X2 + 32 * half, r);
+      tmem_ld_wait16(r);
+      float xs[16];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int j0 = 32 * half + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + B::T_X2 + j0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          float xs[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            xs[e] = (j0 + e <= i && j0 + e < nv) ? __uint_as_float(r[e]) : 0.f;
-          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0, 1024)) = pack8(xs);
-          *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
-        }
-      }
+      for (int e = 0; e < 16; ++e)
+        xs[e] = (j0 + e <= i && j0 + e < nv) ? __uint_as_float(r[e]) : 0.f;
+      *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0, 1024)) = pack8(xs);
+      *reinterpret_cast<uint4*>(smem + B::S_DS + tile_off(i, j0 + 8, 1024)) = pack8(xs + 8);
     }
     signal(5);
     if (!wait_dn(6)) { aborted = true; break; }   // dQ, dK, dV
@@ -574,53 +553,47 @@ __global__ void __launch_bounds__(NBWD, 1)
     r_pending = ch > 0;
     {  // outputs: dq = dxi(Q) xi'(q), dk likewise, dv; xi'(x) = min(xi(x), 1).  Staged as
        // swizzled boxes (rows past the sequence are clipped by the tensor maps)
-      const int i = 16 * quad + lane;
+      const int i = r16, f0 = c16, cg = 4 * (lane >> 4);
+      uint32_t rq[16], rk[16], rv[16];
+      tmem_ld16_halves<16>(trow + B::T_DQ + 32 * half, rq);
+      tmem_ld16_halves<16>(trow + B::T_DK + 32 * half, rk);
+      tmem_ld16_halves<16>(trow + B::T_DV + 32 * half, rv);
+      tmem_ld_wait16(rq);
+      tmem_ld_wait16(rk);
+      tmem_ld_wait16(rv);
+      // xi(q), xi(k) of this row, columns f0..f0+15, from the fp16 operand tiles
+      float fq[16], fk[16];
 #pragma unroll
-      for (int cb = 0; cb < 32; cb += 16) {
-        const int f0 = 32 * half + cb;
-        uint32_t rq[16], rk[16], rv[16];
-        tmem_ld16(trow + B::T_DQ + f0, rq);
-        tmem_ld16(trow + B::T_DK + f0, rk);
-        tmem_ld16(trow + B::T_DV + f0, rv);
-        tmem_ld_wait16(rq);
-        tmem_ld_wait16(rk);
-        tmem_ld_wait16(rv);
-        if (lane < 16) {
-          // xi(q), xi(k) of this row, columns f0..f0+15, from the fp16 operand tiles
-          float fq[16], fk[16];
+      for (int g = 0; g < 2; ++g) {
+        const uint4 xq = *reinterpret_cast<const uint4*>(smem + B::S_Q + tile_off(i, f0 + 8 * g, DX * 16));
+        const uint4 xk = *reinterpret_cast<const uint4*>(smem + B::S_K + tile_off(i, f0 + 8 * g, DX * 16));
+        const __half2* hq = reinterpret_cast<const __half2*>(&xq);
+        const __half2* hk = reinterpret_cast<const __half2*>(&xk);
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const uint4 xq = *reinterpret_cast<const uint4*>(smem + B::S_Q + tile_off(i, f0 + 8 * g, DX * 16));
-            const uint4 xk = *reinterpret_cast<const uint4*>(smem + B::S_K + tile_off(i, f0 + 8 * g, DX * 16));
-            const __half2* hq = reinterpret_cast<const __half2*>(&xq);
-            const __half2* hk = reinterpret_cast<const __half2*>(&xk);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 a2 = __half22float2(hq[e]), b2 = __half22float2(hk[e]);
-              fq[8 * g + 2 * e] = a2.x; fq[8 * g + 2 * e + 1] = a2.y;
-              fk[8 * g + 2 * e] = b2.x; fk[8 * g + 2 * e + 1] = b2.y;
-            }
-          }
-          const uint32_t rowoff = half * B::OBOX + i * 128;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t pos = rowoff + ((((cb >> 2) + g) ^ (i & 7)) << 4);
-            float4 oq, ok;
-            oq.x = __uint_as_float(rq[4 * g]) * fminf(fq[4 * g], 1.f);
-            oq.y = __uint_as_float(rq[4 * g + 1]) * fminf(fq[4 * g + 1], 1.f);
-            oq.z = __uint_as_float(rq[4 * g + 2]) * fminf(fq[4 * g + 2], 1.f);
-            oq.w = __uint_as_float(rq[4 * g + 3]) * fminf(fq[4 * g + 3], 1.f);
-            ok.x = __uint_as_float(rk[4 * g]) * fminf(fk[4 * g], 1.f);
-            ok.y = __uint_as_float(rk[4 * g + 1]) * fminf(fk[4 * g + 1], 1.f);
-            ok.z = __uint_as_float(rk[4 * g + 2]) * fminf(fk[4 * g + 2], 1.f);
-            ok.w = __uint_as_float(rk[4 * g + 3]) * fminf(fk[4 * g + 3], 1.f);
-            *reinterpret_cast<float4*>(smem + B::O_DQ + pos) = oq;
-            *reinterpret_cast<float4*>(smem + B::O_DK + pos) = ok;
-            *reinterpret_cast<float4*>(smem + B::O_DV + pos) =
-                make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
-                            __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 a2 = __half22float2(hq[e]), b2 = __half22float2(hk[e]);
+          fq[8 * g + 2 * e] = a2.x; fq[8 * g + 2 * e + 1] = a2.y;
+          fk[8 * g + 2 * e] = b2.x; fk[8 * g + 2 * e + 1] = b2.y;
         }
+      }
+      const uint32_t rowoff = half * B::OBOX + i * 128;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t pos = rowoff + (((cg + g) ^ (i & 7)) << 4);
+        float4 oq, ok;
+        oq.x = __uint_as_float(rq[4 * g]) * fminf(fq[4 * g], 1.f);
+        oq.y = __uint_as_float(rq[4 * g + 1]) * fminf(fq[4 * g + 1], 1.f);
+        oq.z = __uint_as_float(rq[4 * g + 2]) * fminf(fq[4 * g + 2], 1.f);
+        oq.w = __uint_as_float(rq[4 * g + 3]) * fminf(fq[4 * g + 3], 1.f);
+        ok.x = __uint_as_float(rk[4 * g]) * fminf(fk[4 * g], 1.f);
+        ok.y = __uint_as_float(rk[4 * g + 1]) * fminf(fk[4 * g + 1], 1.f);
+        ok.z = __uint_as_float(rk[4 * g + 2]) * fminf(fk[4 * g + 2], 1.f);
+        ok.w = __uint_as_float(rk[4 * g + 3]) * fminf(fk[4 * g + 3], 1.f);
+        *reinterpret_cast<float4*>(smem + B::O_DQ + pos) = oq;
+        *reinterpret_cast<float4*>(smem + B::O_DK + pos) = ok;
+        *reinterpret_cast<float4*>(smem + B::O_DV + pos) =
+            make_float4(__uint_as_float(rv[4 * g]), __uint_as_float(rv[4 * g + 1]),
+                        __uint_as_float(rv[4 * g + 2]), __uint_as_float(rv[4 * g + 3]));
       }
       fence_async_smem();
       named_sync(1, NEPI);

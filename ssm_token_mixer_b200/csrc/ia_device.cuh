@@ -225,6 +225,21 @@ __device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
                :
                : "memory");
 }
+// 16 lanes x 32 bit read by the two half-warps (16x32bx2.x16): thread t reads
+// lane t % 16 of the warp's quadrant, 16 consecutive columns starting at the
+// address's column for t < 16 and OFF columns further on for t >= 16.  This is
+// the shape for M = 64 accumulators, which fill lanes 0-15 of each quadrant.
+// Values valid after tmem_ld_wait16.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16_halves(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr), "n"(OFF));
+}
 // One column of 32 lanes (32x32b.x1); value valid after tmem_ld_wait1.
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));

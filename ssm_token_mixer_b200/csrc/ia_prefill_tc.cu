@@ -1493,21 +1493,20 @@ __global__ void __launch_bounds__(W2_NT, 1)
       tc_fence_before();
       mbar_arrive(rdy + i);
     };
+    // The M = 64 accumulators (S^T, P, num) fill lanes 0-15 of each quadrant:
+    // thread t takes row 16 * quad + t % 16 and columns c0 .. c0 + 15 of the
+    // warp's 32, the two half-warps splitting them.
+    const int r16 = 16 * quad + (lane & 15);
+    const int c0 = i0 + 16 * (lane >> 4);
     auto e3 = [&]() {   // masked P -> [i][j]
-      const int i = 16 * quad + lane;
+      uint32_t r[16];
+      tmem_ld16_halves<16>(trow + K::T_P + i0, r);
+      tmem_ld_wait16(r);
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_P + i0 + 16 * b, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (i0 + 16 * b + e > i) r[e] = 0u;
-          *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
-          *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
-        }
-      }
+      for (int e = 0; e < 16; ++e)
+        if (c0 + e > r16) r[e] = 0u;
+      *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(r16, c0, 1024)) = pack8f(r, 1.f);
+      *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(r16, c0 + 8, 1024)) = pack8f(r + 8, 1.f);
       signalB(3);
     };
     // o = num / den, staged as two boxes of 64 rows x 128 bytes (columns 0-31
@@ -1519,40 +1518,33 @@ __global__ void __launch_bounds__(W2_NT, 1)
     // has finished reading its buffer; every thread passes that barrier before
     // it writes that buffer again one chunk later.
     auto e4 = [&](int ch, int nv) {
-      const int i = 16 * quad + lane;
-      uint32_t rd, rr[2][16];
-      tmem_ld1(trow + K::T_DEN, rd);
-      tmem_ld16(trow + K::T_NUM + i0, rr[0]);
-      tmem_ld16(trow + K::T_NUM + i0 + 16, rr[1]);
+      const int i = r16, hb = lane >> 4;
+      uint32_t rd, rr[16];
+      tmem_ld1(trow + K::T_DEN, rd);   // one column of all 32 lanes: rows in lanes 0-15
+      tmem_ld16_halves<16>(trow + K::T_NUM + i0, rr);
       tmem_ld_wait1(rd);
-      tmem_ld_wait16(rr[0]);
-      tmem_ld_wait16(rr[1]);
-      const float dn = __uint_as_float(rd);
+      tmem_ld_wait16(rr);
+      const float dn = __shfl_sync(kFull, __uint_as_float(rd), lane & 15);
       const float rdn = 1.0f / dn;
       const uint64_t rdn2 = f2_pack(rdn, rdn);
       const long long row = bh * a.N + ch * C + i;
       const uint32_t stage = K::S_O + ((ch - ch0) & 1) * K::TO;
-      if (lane < 16) {
-        if (i < nv && a.den && half == 0) a.den[row] = dn;
-        uint8_t* box = smem + stage + half * (K::TO / 2) + i * 128;
+      if (i < nv && a.den && half == 0 && hb == 0) a.den[row] = dn;
+      uint8_t* box = smem + stage + half * (K::TO / 2) + i * 128;
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t* r = rr + 4 * g;
+        float4 q;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(r[0]), __uint_as_float(r[1])), rdn2), q.x, q.y);
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2]), __uint_as_float(r[3])), rdn2), q.z, q.w);
+        *reinterpret_cast<float4*>(box + (((4 * hb + g) ^ (i & 7)) << 4)) = q;
+      }
+      if (i < nv && a.num) {
+        float4* np = reinterpret_cast<float4*>(a.num + row * DV + c0);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t* r = rr[b] + 4 * g;
-            float4 q;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(r[0]), __uint_as_float(r[1])), rdn2), q.x, q.y);
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2]), __uint_as_float(r[3])), rdn2), q.z, q.w);
-            *reinterpret_cast<float4*>(box + (((4 * b + g) ^ (i & 7)) << 4)) = q;
-          }
-          if (i < nv && a.num) {
-            float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0 + 16 * b);
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-              np[g] = make_float4(__uint_as_float(rr[b][4 * g]), __uint_as_float(rr[b][4 * g + 1]),
-                                  __uint_as_float(rr[b][4 * g + 2]), __uint_as_float(rr[b][4 * g + 3]));
-          }
-        }
+        for (int g = 0; g < 4; ++g)
+          np[g] = make_float4(__uint_as_float(rr[4 * g]), __uint_as_float(rr[4 * g + 1]),
+                              __uint_as_float(rr[4 * g + 2]), __uint_as_float(rr[4 * g + 3]));
       }
       fence_async_smem();
       if (tid == W2_GT) bulk_wait_read_0();
@@ -1577,21 +1569,16 @@ __global__ void __launch_bounds__(W2_NT, 1)
       if (head) {
         if (!(ok = waitB(0))) break;   // G1 + G7(t)
         {  // E1(t): masked S^T -> [j][i]
-          const int j = 16 * quad + lane;
+          const int j = r16;
           const bool keep = j < nv;
+          uint32_t r[16];
+          tmem_ld16_halves<16>(trow + K::T_S + i0, r);
+          tmem_ld_wait16(r);
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            uint32_t r[16];
-            tmem_ld16(trow + K::T_S + i0 + 16 * b, r);
-            tmem_ld_wait16(r);
-            if (lane < 16) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (!(keep && i0 + 16 * b + e >= j)) r[e] = 0u;
-              *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
-              *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
-            }
-          }
+          for (int e = 0; e < 16; ++e)
+            if (!(keep && c0 + e >= j)) r[e] = 0u;
+          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, c0, 1024)) = pack8f(r, 1.f);
+          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, c0 + 8, 1024)) = pack8f(r + 8, 1.f);
           signalB(1);
         }
       }
