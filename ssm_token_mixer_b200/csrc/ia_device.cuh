@@ -240,6 +240,22 @@ __device__ __forceinline__ void tmem_ld16_halves(uint32_t taddr, uint32_t (&r)[1
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr), "n"(OFF));
 }
+// Same shape with 8 columns per half-warp (16x32bx2.x8); valid after
+// tmem_ld_wait8.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld8_halves(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr), "n"(OFF));
+}
+__device__ __forceinline__ void tmem_ld_wait8(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7])
+               :
+               : "memory");
+}
 // One column of 32 lanes (32x32b.x1); value valid after tmem_ld_wait1.
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));

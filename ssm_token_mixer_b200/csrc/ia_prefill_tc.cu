@@ -451,21 +451,23 @@ __global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
     if (!mma_sync()) { aborted = true; break; }
     if (!FULL) continue;
 
-    const int i0 = 16 * part;     // this thread's 16 columns of the 64-wide tiles
+    const int i0 = 16 * part;     // this warp's 16 columns of the 64-wide tiles
+    // The M = 64 accumulators (S^T, P, num) fill lanes 0-15 of each quadrant:
+    // thread t takes row 16 * quad + t % 16, the two half-warps splitting the
+    // warp's columns.
+    const int r16 = 16 * quad + (lane & 15), hb = lane >> 4;
+    const int c8 = i0 + 8 * hb;   // this thread's 8 columns
     // ---- E1: S^T (M=64 rows j) -> masked fp16, MN-major B of GEMM2
     {
-      const int j = 16 * quad + lane;
-      uint32_t r[16];
-      tmem_ld16(trow + K::T_SP + i0, r);
-      tmem_ld_wait16(r);
-      if (lane < 16) {
-        const bool keep = j < nv;
+      const int j = r16;
+      uint32_t r[8];
+      tmem_ld8_halves<8>(trow + K::T_SP + i0, r);
+      tmem_ld_wait8(r);
+      const bool keep = j < nv;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (!(keep && i0 + e >= j)) r[e] = 0u;
-        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, i0, 1024)) = pack8f(r, 1.f);
-        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-      }
+      for (int e = 0; e < 8; ++e)
+        if (!(keep && c8 + e >= j)) r[e] = 0u;
+      *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, c8, 1024)) = pack8f(r, 1.f);
     }
     to_tensor_core();
     if (tid == 0) {
@@ -505,17 +507,14 @@ __global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
 
     // ---- E3: P (M=64 rows i) -> masked fp16, K-major A of GEMM5
     {
-      const int i = 16 * quad + lane;
-      uint32_t r[16];
-      tmem_ld16(trow + K::T_SP + i0, r);
-      tmem_ld_wait16(r);
-      if (lane < 16) {
+      const int i = r16;
+      uint32_t r[8];
+      tmem_ld8_halves<8>(trow + K::T_SP + i0, r);
+      tmem_ld_wait8(r);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (i0 + e > i) r[e] = 0u;
-        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, i0, 1024)) = pack8f(r, 1.f);
-        *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-      }
+      for (int e = 0; e < 8; ++e)
+        if (c8 + e > i) r[e] = 0u;
+      *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, c8, 1024)) = pack8f(r, 1.f);
     }
     to_tensor_core();
     if (tid == 0) {
@@ -537,38 +536,40 @@ __global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
 
     // ---- E4: o = num / den, staged in shared memory, then written coalesced
     {
-      const int i = 16 * quad + lane;
-      uint32_t rd[16];
-      tmem_ld16(trow + K::T_DEN, rd);
-      tmem_ld_wait16(rd);
-      const float dn = __uint_as_float(rd[0]);
+      const int i = r16;
+      uint32_t rd;
+      tmem_ld1(trow + K::T_DEN, rd);   // one column of all 32 lanes: rows in lanes 0-15
+      tmem_ld_wait1(rd);
+      const float dn = __shfl_sync(kFull, __uint_as_float(rd), lane & 15);
       const float rdn = 1.0f / dn;
       const long long row = bh * a.N + n0 + i;
-      const bool valid = lane < 16 && i < nv;
-      if (valid && a.den && part == 0) a.den[row] = dn;
-      constexpr int DQ = DV / 4;   // value columns per thread
-#pragma unroll
-      for (int cb = 0; cb < DQ; cb += 16) {
-        const int f0 = part * DQ + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_NUM + f0, r);
+      const bool valid = i < nv;
+      if (valid && a.den && part == 0 && hb == 0) a.den[row] = dn;
+      constexpr int DQ = DV / 4;   // value columns per warp
+      static_assert(DQ == 16 || DQ == 32, "a warp's value columns split into two halves of 8 or 16");
+      constexpr int PH = DQ / 2;   // value columns per thread
+      const int f0 = part * DQ + PH * hb;
+      uint32_t r[PH];
+      if constexpr (PH == 16) {
+        tmem_ld16_halves<16>(trow + K::T_NUM + part * DQ, r);
         tmem_ld_wait16(r);
-        if (lane < 16) {
+      } else {
+        tmem_ld8_halves<8>(trow + K::T_NUM + part * DQ, r);
+        tmem_ld_wait8(r);
+      }
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int chunk = (f0 >> 2) + g;
-            *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
-                make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                            __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-          }
-          if (valid && a.num) {
-            float4* np = reinterpret_cast<float4*>(a.num + row * DV + f0);
+      for (int g = 0; g < PH / 4; ++g) {
+        const int chunk = (f0 >> 2) + g;
+        *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
+            make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
+                        __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
+      }
+      if (valid && a.num) {
+        float4* np = reinterpret_cast<float4*>(a.num + row * DV + f0);
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-              np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                                  __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
-          }
-        }
+        for (int g = 0; g < PH / 4; ++g)
+          np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                              __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
       }
       __syncthreads();
       constexpr int CPR = DV / 4;  // 16-byte chunks per row
