@@ -315,7 +315,8 @@ def leg_prefill_long(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world
     launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
     fl = flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
     by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
-    rf = roofline(by, fl, kern_ms, peaks, peak_kind, None, sustained=False)
+    traffic = recorded_traffic("tc_prefill_1p3b_7168.md", "ssm_token_mixer_b200/csrc/ia_prefill_tc.cu")
+    rf = roofline(by, fl, kern_ms, peaks, peak_kind, traffic, sustained=False)
     rf["kernel"] = "full chunk pass"
     step_s = total / steps * 1e-3
     rf["step"] = {"achieved_gbs": by / step_s / 1e9, "frac_hbm": by / step_s / 1e9 / float(peaks["hbm_gbs"])}
