@@ -1195,9 +1195,6 @@ __global__ void __launch_bounds__(W2_NT, 1)
     fence_barrier_init();
   }
   {
-    const uint4* src = reinterpret_cast<const uint4*>(T->E);
-    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
     // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
     // the ones column after V: MN element 64 (first of the second 64-block)
     // is 1 in every row, the rest 0, in the swizzled layout
@@ -1212,6 +1209,15 @@ __global__ void __launch_bounds__(W2_NT, 1)
         *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    // Everything above touches only this CTA's own resources.  The kernel may
+    // have been launched while the previous kernel of the stream (the table
+    // prologue, or the segment carry scan) still runs: every global read of
+    // the tables, carries and inputs comes after this wait, and nothing global
+    // is written before it.
+    griddep_wait();
+    const uint4* src = reinterpret_cast<const uint4*>(T->E);
+    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
+    for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -1646,6 +1652,13 @@ __global__ void __launch_bounds__(W2_NT, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// Tuning switch IA_PREFILL_WS for d = 64: 0 the one-role loop, 1 one epilogue
+// group, unset or 2 the four-role kernel.
+bool ws2_selected() {
+  const char* ws = std::getenv("IA_PREFILL_WS");
+  return !ws || std::atoi(ws) >= 2;
+}
+
 template <int DX, int DV>
 cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p, cudaStream_t st) {
   using K = Cfg<DX, DV>;
@@ -1661,21 +1674,32 @@ cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p
     if (e != cudaSuccess) return e;
   }
   if constexpr (DX == 64 && DV == 64) {
-    const char* ws = std::getenv("IA_PREFILL_WS");   // tuning switch: 0 plain loop, 1 one epilogue group
-    if (!ws || std::atoi(ws) >= 2) {
+    if (ws2_selected()) {
       CUtensorMap tm_q, tm_k, tm_v, tm_o;
       if (!encode_input_map(&tm_q, args.q, args.BH, args.N) || !encode_input_map(&tm_k, args.k, args.BH, args.N) ||
           !encode_input_map(&tm_v, args.v, args.BH, args.N) || !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N))
         return cudaErrorNotSupported;
       e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
       if (e != cudaSuccess) return e;
-      mark_launch_begin(st);
-      tc_prefill_ws2_kernel<<<static_cast<unsigned>(args.BH * p.nseg), W2_NT, W2Cfg::SMEM, st>>>(args, tm_q, tm_k,
-                                                                                               tm_v, tm_o);
-      e = cudaGetLastError();
+      // Programmatic dependent launch: the CTAs set up barriers, TMEM and
+      // constant tiles while the previous kernel finishes (see griddep_wait).
+      // Straight after the table kernel, the timing mark was set before it.
+      if (p.nseg > 1) mark_launch_begin(st);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(args.BH * p.nseg));
+      cfg.blockDim = dim3(W2_NT);
+      cfg.dynamicSmemBytes = W2Cfg::SMEM;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, tc_prefill_ws2_kernel, args, tm_q, tm_k, tm_v, tm_o);
       mark_launch_end(st);
       return e;
     }
+    const char* ws = std::getenv("IA_PREFILL_WS");
     if (std::atoi(ws) == 1) {
       e = cudaFuncSetAttribute(tc_prefill_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WCfg::SMEM);
       if (e != cudaSuccess) return e;
@@ -1760,6 +1784,9 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
   float* seg_state = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   float* seg_eta = seg_state + BH * (p.nseg > 1 ? p.nseg - 1 : 0) * KR * (s.d_xi + s.d_v);
+  // the four-role d = 64 kernel directly after the tables overlaps them, so
+  // its timing mark goes before the table kernel
+  if (s.d_xi == 64 && s.d_v == 64 && p.nseg == 1 && ws2_selected()) mark_launch_begin(st);
   cudaError_t e = launch_param_tables(s.H, delta, A, tabs, st, dtab);
   if (e != cudaSuccess) return e;
   TcArgs args;

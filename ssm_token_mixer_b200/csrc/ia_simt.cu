@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
                                                                     HeadTables* __restrict__ tabs,
                                                                     float* __restrict__ dtab) {
   __shared__ __align__(16) __half Es[2 * kModesTC * kChunk];
+  griddep_launch_dependents();   // the chunk pass may start its table-free prologue now
   const int h = blockIdx.x;
   HeadTables* T = tabs + h;
   const float dl = delta[h];
