@@ -153,7 +153,10 @@ IA_API ia_status_t ia_decode_step(const ia_shape_t* shape, const void* q, const 
  * records `begin` on its stream immediately before launching its dominant
  * kernel (the full chunk pass of the prefill, the reverse-mode kernel of the
  * training step, the decode kernel) and `end` immediately after it, so the
- * caller can time that kernel alone.  Pass NULL, NULL to stop.  The events
+ * caller can time that kernel alone.  One exception: the unsplit d = 64
+ * chunk pass starts while the per-head table kernel before it still runs
+ * (programmatic dependent launch), so there `begin` precedes the table
+ * kernel and the interval covers both.  Pass NULL, NULL to stop.  The events
  * are not owned or destroyed by the library.
  */
 IA_API ia_status_t ia_set_launch_events(void* begin, void* end);
