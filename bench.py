@@ -467,6 +467,14 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
     return out
 
 
+def workload_config(w):
+    """The JSON line's config: the workload and how it is timed (both arms)."""
+    return {"workload": f"{w.name} prefill (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, "
+                        f"bf16 inputs, fp32 state/output)",
+            "l2": "flushed (256 MB write) between timed steps",
+            "per_gpu": "each rank runs the full workload (weak scaling)"}
+
+
 # ---------------------------------------------------------------- reference arm (oracle)
 def run_reference(args):
     rank, world, _ = dist_env()
@@ -475,8 +483,8 @@ def run_reference(args):
     import oracle
     from ssm_token_mixer_b200 import synthetic
     from ssm_token_mixer_b200.workloads import WORKLOADS
-    w = WORKLOADS["prefill_125m"]
-    inp = synthetic.workload_inputs(w, B=1)     # one batch element (12 heads x 2048 tokens) per step
+    w = WORKLOADS[args.workload]
+    inp = synthetic.workload_inputs(w, B=1)     # one batch element (H heads x N tokens) per step
     ms = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -490,10 +498,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ms),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
-                   "sample_per_step": "batch element 0 (H12 x N2048)"},
+        "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": "batch element 0 of prefill_125m per step, fp64 sequential recurrence"},
+                         "sample": f"batch element 0 of {w.name} (H{w.H} x N{w.N}) per step, fp64 sequential "
+                                   f"recurrence on the host cores; tokens/s counts that element's N tokens"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -540,10 +548,7 @@ def main():
     line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16xf16->f32 (bf16 inputs)", "data": "synthetic (seeded N(0,1) q/k/v, log-uniform Delta)",
-            "config": {"workload": f"{w.name} prefill (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, "
-                                   f"bf16 inputs, fp32 state/output)",
-                       "l2": "flushed (256 MB write) between timed steps",
-                       "per_gpu": "each rank runs the full workload (weak scaling)"}}
+            "config": workload_config(w)}
     cpu = not args.no_cpu
     try:
         if "prefill" in legs:

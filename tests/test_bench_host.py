@@ -53,3 +53,20 @@ def test_recorded_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     src.write_text("// kernel, changed since the capture\n")
     assert bench.recorded_traffic("k.md", "kernel.cu") is None
     assert bench.recorded_traffic("missing.md", "kernel.cu") is None
+
+
+def test_reference_arm_reports_the_gpu_arms_config(capsys, monkeypatch):
+    # the oracle arm times one batch element per step on the host cores and
+    # labels its line with the same workload config as the GPU arm
+    import argparse
+    import json
+    from ssm_token_mixer_b200.workloads import WORKLOADS
+    monkeypatch.delenv("RANK", raising=False)
+    args = argparse.Namespace(steps=1, warmup=0, gpus=1, workload="prefill_125m")
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config(WORKLOADS["prefill_125m"])
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
