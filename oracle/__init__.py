@@ -30,16 +30,24 @@ _LIB = os.path.join(_HERE, "libia_oracle.so")
 _lib = None
 
 
+def compile_source(src: str, out: str) -> str:
+    """Compile an oracle source file into a shared library at ``out`` with the
+    oracle's flags (gcc, -O2, OpenMP, IEEE fp64 with no contraction).  The
+    mutation test uses it to build copies that carry a planted mistake."""
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile ia_oracle.c into libia_oracle.so (gcc, -O2, OpenMP, IEEE fp64)."""
+    """Compile ia_oracle.c into libia_oracle.so."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
         os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "ia_oracle.h"))
     ):
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
-        subprocess.check_call(cmd)
-        os.replace(tmp, _LIB)
+        compile_source(_SRC, _LIB)
     return _LIB
 
 
