@@ -103,3 +103,40 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(ia, "_LIB_PATH", "/nonexistent/libia.so")
     with pytest.raises(RuntimeError):
         ia.load_library()
+
+
+def _segments(lib, s, monkeypatch):
+    """Segments per sequence of the tensor-core plan, read from the workspace
+    size: each boundary between segments keeps one carried state per (b,h)."""
+    ws = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
+    monkeypatch.setenv("IA_PREFILL_SEGMENTS", "1")
+    ws1 = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
+    monkeypatch.delenv("IA_PREFILL_SEGMENTS")
+    per_bh = lib.ia_state_bytes(ctypes.byref(s)) // (s.B * s.H)
+    extra = ws - ws1
+    assert extra % (s.B * s.H * per_bh) == 0
+    return 1 + extra // (s.B * s.H * per_bh)
+
+
+@pytest.mark.parametrize("B,H,N,d,nseg", [
+    (8, 12, 2048, 64, 1),    # 125M prefill: 96 sequences, one pass
+    (8, 16, 2048, 64, 1),    # 350M training shape: 128 sequences
+    (4, 16, 2048, 128, 2),   # 1.3B prefill: 64 sequences of 32 chunks -> 2 x 16 chunks on 128 CTAs
+    (1, 16, 7168, 128, 9),   # 1.3B long context: 16 x 112 chunks -> 9 x 13 chunks on 144 CTAs
+])
+def test_segment_plan_on_148_sms(lib, monkeypatch, B, H, N, d, nseg):
+    # With no GPU the planner assumes a B200's 148 SMs.  Splitting pays when
+    # the sequences alone leave SMs idle: a state-only pass and the carry scan
+    # then precede the full pass (4 launches instead of tables + full pass).
+    s = shape(B=B, H=H, N=N, dx=d, dv=d, M=64, dt=1)
+    assert _segments(lib, s, monkeypatch) == nseg
+    assert lib.ia_prefill_launches(ctypes.byref(s)) == (4 if nseg > 1 else 2)
+
+
+def test_segment_override_and_cuda_core_path(lib, monkeypatch):
+    s = shape(B=8, H=12, N=2048, dx=64, dv=64, M=64, dt=1)
+    monkeypatch.setenv("IA_PREFILL_SEGMENTS", "4")
+    assert lib.ia_prefill_launches(ctypes.byref(s)) == 4
+    monkeypatch.delenv("IA_PREFILL_SEGMENTS")
+    # fp32 inputs run the sequential CUDA-core kernel: one launch, no segments
+    assert lib.ia_prefill_launches(ctypes.byref(shape(B=1, H=2, N=256, dx=16, dv=16, M=16, dt=0))) == 1
