@@ -136,26 +136,105 @@ def _workspace(nbytes, device, workspace):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+# The library receives raw device pointers and cannot see tensor sizes, so the
+# binding checks every tensor against the shape before the call: a short or
+# misplaced buffer is an error here rather than an out-of-bounds access on the
+# GPU.  Shapes and dtypes are checked first, the device last.
+def _need(name, t, shape=None, dtype=None, numel=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+
+
+def _cuda_device(named):
+    """The one CUDA device all given tensors live on (None entries skipped)."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if t.device.type != "cuda":
+            raise ValueError(f"{name} is on {t.device}; the library takes CUDA tensors")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
+    return dev
+
+
+def _check_sequence_args(q, k, v, delta, M, A, dO=None):
+    """q, k [B,H,N,d_xi], v and dO [B,H,N,d_v] in one input dtype, delta [H]
+    fp32, A [M] complex as 2M fp32 (or None).  Returns (B, H, N, d_xi, d_v)."""
+    _need("q", q)
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B,H,N,d_xi], got shape {tuple(q.shape)}")
+    _dtype_code(q)
+    B, H, N, d_xi = q.shape
+    _need("k", k, (B, H, N, d_xi), q.dtype)
+    _need("v", v, dtype=q.dtype)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, H, N):
+        raise ValueError(f"v must be [B,H,N,d_v] = [{B},{H},{N},d_v], got {tuple(v.shape)}")
+    d_v = v.shape[3]
+    _need("delta", delta, (H,), torch.float32)
+    if A is not None:
+        _need("A", A, dtype=torch.float32, numel=2 * int(M))
+    if dO is not None:
+        _need("dO", dO, (B, H, N, d_v), q.dtype)
+    return B, H, N, d_xi, d_v
+
+
+def _check_token_args(q, k, v, delta, M, A):
+    """Decode: q, k [B,H,d_xi], v [B,H,d_v].  Returns (B, H, d_xi, d_v)."""
+    _need("q", q)
+    if q.dim() != 3:
+        raise ValueError(f"q must be [B,H,d_xi], got shape {tuple(q.shape)}")
+    _dtype_code(q)
+    B, H, d_xi = q.shape
+    _need("k", k, (B, H, d_xi), q.dtype)
+    _need("v", v, dtype=q.dtype)
+    if v.dim() != 3 or tuple(v.shape[:2]) != (B, H):
+        raise ValueError(f"v must be [B,H,d_v] = [{B},{H},d_v], got {tuple(v.shape)}")
+    _need("delta", delta, (H,), torch.float32)
+    if A is not None:
+        _need("A", A, dtype=torch.float32, numel=2 * int(M))
+    return B, H, d_xi, v.shape[2]
+
+
 def prefill_fwd(q, k, v, delta, M, A=None, state_in=None, want_num_den=False, want_state=False,
                 o=None, workspace=None, stream=None):
     """Causal IA prefill.  q,k [B,H,N,d_xi], v [B,H,N,d_v] (fp32 or bf16), delta [H] fp32.
 
     Returns dict with o [B,H,N,d_v] fp32 and, on request, num, den, state (flat fp32)."""
     lib = load_library()
-    B, H, N, d_xi = q.shape
-    d_v = v.shape[-1]
+    B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A)
     shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
-    dev = q.device
+    n_state = lib.ia_state_bytes(ctypes.byref(shp)) // 4
+    if state_in is not None:
+        _need("state_in", state_in, dtype=torch.float32, numel=n_state)
+    if o is not None:
+        _need("o", o, (B, H, N, d_v), torch.float32)
+    if workspace is not None:
+        _need("workspace", workspace)
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("state_in", state_in),
+                        ("o", o), ("workspace", workspace)])
     if o is None:
         o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
     num = torch.empty_like(o) if want_num_den else None
     den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
-    st = torch.empty(lib.ia_state_bytes(ctypes.byref(shp)) // 4, dtype=torch.float32, device=dev) if want_state else None
+    st = torch.empty(n_state, dtype=torch.float32, device=dev) if want_state else None
     need = lib.ia_prefill_workspace_bytes(ctypes.byref(shp))
     ws = _workspace(need, dev, workspace)
     rc = lib.ia_prefill_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
                             _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _ptr(ws),
-                            ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream))
+                            ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check(rc, "ia_prefill_fwd")
     return {"o": o, "num": num, "den": den, "state": st}
 
@@ -167,15 +246,20 @@ def prefill_fwd_static(q, k, v, delta, M, A=None, state_in=None, want_num_den=Fa
     ia_prefill_fwd_static in include/ia.h).  Output tensors are still the
     caller's; pass `o` (and use want_* = False) to allocate nothing here."""
     lib = load_library()
-    B, H, N, d_xi = q.shape
-    d_v = v.shape[-1]
+    B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A)
     shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
-    dev = q.device
+    n_state = lib.ia_state_bytes(ctypes.byref(shp)) // 4
+    if state_in is not None:
+        _need("state_in", state_in, dtype=torch.float32, numel=n_state)
+    if o is not None:
+        _need("o", o, (B, H, N, d_v), torch.float32)
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("state_in", state_in),
+                        ("o", o)])
     if o is None:
         o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
     num = torch.empty_like(o) if want_num_den else None
     den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
-    st = torch.empty(lib.ia_state_bytes(ctypes.byref(shp)) // 4, dtype=torch.float32, device=dev) if want_state else None
+    st = torch.empty(n_state, dtype=torch.float32, device=dev) if want_state else None
     rc = lib.ia_prefill_fwd_static(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
                                    _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _stream(stream))
     _check(rc, "ia_prefill_fwd_static")
@@ -185,10 +269,12 @@ def prefill_fwd_static(q, k, v, delta, M, A=None, state_in=None, want_num_den=Fa
 def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
     """Forward + reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta)."""
     lib = load_library()
-    B, H, N, d_xi = q.shape
-    d_v = v.shape[-1]
+    B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A, dO=dO)
     shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
-    dev = q.device
+    if workspace is not None:
+        _need("workspace", workspace)
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("dO", dO),
+                        ("workspace", workspace)])
     o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
     dq = torch.empty(B, H, N, d_xi, dtype=torch.float32, device=dev)
     dk = torch.empty_like(dq)
@@ -198,7 +284,7 @@ def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
     ws = _workspace(need, dev, workspace)
     rc = lib.ia_fwd_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A), _ptr(dO),
                         _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dD), _ptr(ws),
-                        ctypes.c_size_t(ws.numel() if ws is not None else 0), _stream(stream))
+                        ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check(rc, "ia_fwd_bwd")
     return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD}
 
@@ -206,10 +292,12 @@ def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
 def decode_step(q, k, v, delta, state, M, A=None, o=None, want_num_den=False, stream=None):
     """One decode step.  q,k [B,H,d_xi], v [B,H,d_v]; state (flat fp32) updated in place."""
     lib = load_library()
-    B, H, d_xi = q.shape
-    d_v = v.shape[-1]
+    B, H, d_xi, d_v = _check_token_args(q, k, v, delta, M, A)
     shp = make_shape(B, H, 1, d_xi, d_v, M, _dtype_code(q))
-    dev = q.device
+    _need("state", state, dtype=torch.float32, numel=lib.ia_state_bytes(ctypes.byref(shp)) // 4)
+    if o is not None:
+        _need("o", o, (B, H, d_v), torch.float32)
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("state", state), ("o", o)])
     if o is None:
         o = torch.empty(B, H, d_v, dtype=torch.float32, device=dev)
     num = torch.empty_like(o) if want_num_den else None
