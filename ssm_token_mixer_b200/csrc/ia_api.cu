@@ -63,6 +63,8 @@ cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
 
 }  // namespace
 
+bool inject_launch_failure() { return env_set("IA_INJECT_LAUNCH_FAILURE"); }
+
 void mark_launch_begin(cudaStream_t st) {
   if (g_ev_begin) cudaEventRecord(g_ev_begin, st);
 }
@@ -147,7 +149,7 @@ ia_status_t ia_prefill_fwd(const ia_shape_t* s, const void* q, const void* k, co
     return IA_ERR_UNSUPPORTED;
   }
   if (need > 0 && (!workspace || workspace_bytes < need)) return IA_ERR_WORKSPACE;
-  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  if (inject_launch_failure()) return IA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc)
     return map_cuda(launch_tc_prefill(*s, plan, q, k, v, delta, A, state_in, o, num, den,
@@ -169,7 +171,7 @@ ia_status_t ia_fwd_bwd(const ia_shape_t* s, const void* q, const void* k, const 
   if (!tc && seq_bwd_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
   const size_t need = ia_fwd_bwd_workspace_bytes(s);
   if (!workspace || workspace_bytes < need) return IA_ERR_WORKSPACE;
-  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  if (inject_launch_failure()) return IA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc)
     return map_cuda(launch_tc_fwd_bwd(*s, tc_plan(*s, num_sms()), q, k, v, delta, A, dO, o, dq, dk,
@@ -190,7 +192,7 @@ ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, co
   if (s->M > 128) return IA_ERR_UNSUPPORTED;                        // at most 8 CTAs x 16 modes
   const size_t smem = sizeof(float) * (2 * s->d_xi + 9 * s->d_v + 8) + 2 * sizeof(float2) * s->M + 16;
   if (smem > kMaxSmem) return IA_ERR_UNSUPPORTED;
-  if (env_set("IA_INJECT_LAUNCH_FAILURE")) return IA_ERR_CUDA;
+  if (inject_launch_failure()) return IA_ERR_CUDA;
   return map_cuda(launch_decode(*s, q, k, v, delta, A, state, o, num, den,
                                 static_cast<cudaStream_t>(stream)));
 }

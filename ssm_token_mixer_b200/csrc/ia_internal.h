@@ -65,6 +65,11 @@ cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, con
                           const float* delta, const float* A, void* state, float* o, float* num,
                           float* den, cudaStream_t st);
 
+// Failure injection for host tests: with IA_INJECT_LAUNCH_FAILURE set (and
+// not "0"), every entry point returns IA_ERR_CUDA after its argument checks,
+// launching nothing.
+bool inject_launch_failure();
+
 // Caller-registered events bracketing the dominant kernel launch (profiling).
 void mark_launch_begin(cudaStream_t st);
 void mark_launch_end(cudaStream_t st);

@@ -75,6 +75,7 @@ extern "C" IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* s, const v
   const int nch = (s->N + kChunk - 1) / kChunk;
   const TcPlan plan{1, nch};
   if (tc_workspace_bytes(*s, plan) > kStaticScratchBytes) return IA_ERR_WORKSPACE;
+  if (inject_launch_failure()) return IA_ERR_CUDA;
   cudaError_t e;
   void* scratch = static_scratch_on_current_device(&e);
   if (!scratch) return IA_ERR_CUDA;

@@ -84,11 +84,24 @@ def test_decode_validation(lib):
 
 
 def test_injected_launch_failure(lib, monkeypatch):
+    # every entry point, given valid arguments, reports the injected launch
+    # failure after its checks and launches nothing (no pointer is touched)
     monkeypatch.setenv("IA_INJECT_LAUNCH_FAILURE", "1")
     s = shape(dt=0, dx=16, dv=16, M=4)                 # CUDA-core path: no workspace
     assert prefill(lib, s) == 4
     rc = lib.ia_decode_step(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, None)
     assert rc == 4
+    need = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(s))
+    rc = lib.ia_fwd_bwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                        FAKE, ctypes.c_size_t(need), None)
+    assert rc == 4
+    t = shape(B=1, H=2, N=100, dx=64, dv=64, M=64, dt=1)   # the no-allocation entry point: bf16, M = 64
+    rc = lib.ia_prefill_fwd_static(ctypes.byref(t), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None,
+                                   None, None)
+    assert rc == 4
+    # without the switch, argument errors still come first
+    monkeypatch.setenv("IA_INJECT_LAUNCH_FAILURE", "0")
+    assert prefill(lib, shape(B=0)) == 1
 
 
 def test_status_strings(lib):
