@@ -100,6 +100,19 @@ def barrier(device=None):
             dist.barrier()
 
 
+def rank_workload(w, rank, world, scaling):
+    """This rank's workload and the batch the whole job processes.  Weak
+    scaling: every rank runs the full workload (its own batch of the same
+    size); strong: the workload's batch is split over the ranks."""
+    import dataclasses
+    if scaling == "weak" or world == 1:
+        return w, world * w.B
+    if w.B < world:
+        raise SystemExit(f"--scaling strong needs B >= ranks ({w.name}: B={w.B}, {world} ranks)")
+    lo, hi = shard_units(w.B, rank, world)
+    return dataclasses.replace(w, B=hi - lo), w.B
+
+
 # ---------------------------------------------------------------- environment
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -238,7 +251,10 @@ def roofline(bytes_per_launch, flops_per_launch, kern_ms, peaks, peak_kind, traf
 
 
 # ---------------------------------------------------------------- legs
-def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_leg):
+def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_leg,
+                profile="tc_prefill_ws2_125m.md", job_B=None):
+    """Prefill of one workload: step time, the chunk pass timed live, e2e, and
+    the oracle on the full batch."""
     import torch
     import ssm_token_mixer_b200 as ia
     from ssm_token_mixer_b200 import synthetic
@@ -255,15 +271,21 @@ def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
     barrier(dev)
     total = max_over_ranks(sum(step_ms), dev)
     tokens = w.B * w.N
-    value = world * tokens * steps / (total * 1e-3)
+    job_tokens = (job_B or world * w.B) * w.N
+    value = job_tokens * steps / (total * 1e-3)
     launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
     fl = flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H
     by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
-    traffic = recorded_traffic("tc_prefill_ws2_125m.md", "ssm_token_mixer_b200/csrc/ia_prefill_tc.cu")
+    traffic = recorded_traffic(profile, "ssm_token_mixer_b200/csrc/ia_prefill_tc.cu")
     rf = roofline(by, fl, kern_ms, peaks, peak_kind, traffic, sustained=False)
-    # the chunk pass starts under the table kernel (programmatic dependent
-    # launch), so its events bracket both: kernel_ms is an upper bound
-    rf["kernel"] = "chunk pass, timed from the table kernel it overlaps"
+    if launches == 2:
+        # unsplit: the chunk pass starts under the table kernel (programmatic
+        # dependent launch), so its events bracket both: an upper bound
+        rf["kernel"] = "chunk pass, timed from the table kernel it overlaps"
+    else:
+        rf["kernel"] = "full chunk pass (after the state-only pass and the carry scan)"
+    step_s = total / steps * 1e-3
+    rf["step"] = {"achieved_gbs": by / step_s / 1e9, "frac_hbm": by / step_s / 1e9 / float(peaks["hbm_gbs"])}
     # end to end through the public API with host buffers: H2D inputs, call, D2H o
     qh, kh, vh = (x.pin_memory() for x in (inp["q"], inp["k"], inp["v"]))
     oh = torch.empty(o.shape, dtype=torch.float32).pin_memory()
@@ -278,9 +300,10 @@ def leg_prefill(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
     e2e_ms, _ = timer.run(e2e, steps, warmup, kernel_events=False)
     e2e_total = max_over_ranks(sum(e2e_ms), dev)
     res = {
-        "value": value, "ms_per_step": total / steps, "roofline": rf,
-        "gpu_launches": launches * steps,
-        "e2e": {"value": world * tokens * steps / (e2e_total * 1e-3), "unit": "tokens/s",
+        "workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
+        "value": value, "unit": "tokens/s", "ms_per_step": total / steps, "roofline": rf,
+        "launches_per_step": launches, "gpu_launches": launches * steps,
+        "e2e": {"value": job_tokens * steps / (e2e_total * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in (qh, kh, vh))),
                 "d2h_bytes_per_step": int(oh.numel() * 4)},
         "algorithmic": {"flops": fl, "bytes": by},
@@ -329,15 +352,17 @@ def leg_prefill_long(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world
             "gpu_launches": launches * steps, "roofline": rf}
 
 
-def leg_fwd_bwd(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_leg):
+def leg_fwd_bwd(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_leg, job_B=None):
+    """Training step; with several ranks each step ends with the all-reduce
+    of dDelta over NCCL (the one exchange data-parallel training needs)."""
     import torch
     import ssm_token_mixer_b200 as ia
-    from ssm_token_mixer_b200 import synthetic
+    from ssm_token_mixer_b200 import parallel, synthetic
     inp = synthetic.workload_inputs(w)
     d = {n: inp[n].to(dev) for n in ("q", "k", "v", "delta", "dO")}
     need = ia.fwd_bwd_workspace_bytes(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16")
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
-    fn = lambda: ia.fwd_bwd(d["q"], d["k"], d["v"], d["delta"], d["dO"], w.M, workspace=ws)
+    fn = lambda: parallel.fwd_bwd_sharded(d["q"], d["k"], d["v"], d["delta"], d["dO"], w.M, workspace=ws)
     barrier(dev)
     step_ms, kern_ms = timer.run(fn, steps, warmup)
     barrier(dev)
@@ -358,7 +383,7 @@ def leg_fwd_bwd(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu
                   "achieved_gbs": by_step / step_s / 1e9, "frac_hbm": by_step / step_s / 1e9 / float(peaks["hbm_gbs"])}
     launches = ia.prefill_launches(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16") + 1
     res = {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
-           "value": world * tokens * steps / (total * 1e-3), "unit": "tokens/s",
+           "value": (job_B or world * w.B) * w.N * steps / (total * 1e-3), "unit": "tokens/s",
            "ms_per_step": total / steps, "steps": steps, "gpu_launches": launches * steps,
            "roofline": rf}
     if cpu_leg and rank == 0 and world == 1:
@@ -467,12 +492,14 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
     return out
 
 
-def workload_config(w):
+def workload_config(w, scaling="weak"):
     """The JSON line's config: the workload and how it is timed (both arms)."""
     return {"workload": f"{w.name} prefill (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, "
                         f"bf16 inputs, fp32 state/output)",
             "l2": "flushed (256 MB write) between timed steps",
-            "per_gpu": "each rank runs the full workload (weak scaling)"}
+            "per_gpu": "each rank runs the full workload (weak scaling)" if scaling == "weak" else
+                       "the batch is split over the ranks (strong scaling); decode and the long prefill "
+                       "stay per rank"}
 
 
 # ---------------------------------------------------------------- reference arm (oracle)
@@ -484,7 +511,7 @@ def run_reference(args):
     from ssm_token_mixer_b200 import synthetic
     from ssm_token_mixer_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]
-    inp = synthetic.workload_inputs(w, B=1)     # one batch element (H heads x N tokens) per step
+    inp = synthetic.workload_inputs(w)          # the full batch per step, as the GPU arm
     ms = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -492,7 +519,7 @@ def run_reference(args):
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             ms.append(dt * 1e3)
-    value = w.N * len(ms) / (sum(ms) * 1e-3)
+    value = w.B * w.N * len(ms) / (sum(ms) * 1e-3)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.mean(ms),
@@ -500,8 +527,8 @@ def run_reference(args):
         "data": "synthetic",
         "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"batch element 0 of {w.name} (H{w.H} x N{w.N}) per step, fp64 sequential "
-                                   f"recurrence on the host cores; tokens/s counts that element's N tokens"},
+                         "sample": f"full {w.name} batch (B{w.B} H{w.H} N{w.N}) per step, fp64 sequential "
+                                   f"recurrence, OpenMP over the (b,h) sequences on the host cores"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -515,10 +542,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--legs", default="prefill,fwd_bwd,decode,prefill_long",
+    ap.add_argument("--legs", default="prefill,prefill_1p3b,fwd_bwd,decode,prefill_long",
                     help="comma list of legs to run (prefill is the headline)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--workload", default="prefill_125m", help="headline prefill workload")
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="weak: every rank runs the full batch; strong: the batch is split over the ranks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -546,22 +575,32 @@ def main():
     clocks.start()
     w = WORKLOADS[args.workload]
     line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None,
             "dtype": "f16xf16->f32 (bf16 inputs)", "data": "synthetic (seeded N(0,1) q/k/v, log-uniform Delta)",
-            "config": workload_config(w)}
+            "config": workload_config(w, args.scaling)}
+    w_loc, job_B = rank_workload(w, rank, world, args.scaling)
     cpu = not args.no_cpu
     try:
         if "prefill" in legs:
-            r = leg_prefill(dev, w, args.steps, args.warmup, timer, peaks, peak_kind, rank, world, cpu)
+            r = leg_prefill(dev, w_loc, args.steps, args.warmup, timer, peaks, peak_kind, rank, world, cpu,
+                            job_B=job_B)
             line.update(value=r["value"], ms_per_step=r["ms_per_step"], roofline=r["roofline"],
                         e2e=r["e2e"], gpu_launches=r["gpu_launches"])
             if "cpu_baseline" in r:
                 line["cpu_baseline"] = r["cpu_baseline"]
             line["algorithmic_per_step"] = r["algorithmic"]
         extra_launches = 0
+        if "prefill_1p3b" in legs:
+            wl, jb = rank_workload(WORKLOADS["prefill_1p3b"], rank, world, args.scaling)
+            r = leg_prefill(dev, wl, args.steps, args.warmup, timer, peaks, peak_kind,
+                            rank, world, cpu, profile="tc_prefill_1p3b.md", job_B=jb)
+            r.pop("algorithmic", None)
+            line["prefill_1p3b"] = r
+            extra_launches += r["gpu_launches"]
         if "fwd_bwd" in legs:
-            r = leg_fwd_bwd(dev, WORKLOADS["train_350m"], args.steps, args.warmup, timer, peaks, peak_kind,
-                            rank, world, cpu)
+            wl, jb = rank_workload(WORKLOADS["train_350m"], rank, world, args.scaling)
+            r = leg_fwd_bwd(dev, wl, args.steps, args.warmup, timer, peaks, peak_kind,
+                            rank, world, cpu, job_B=jb)
             line["fwd_bwd"] = r
             extra_launches += r["gpu_launches"]
         if "decode" in legs:

@@ -35,6 +35,16 @@
  *   - A launch failure returns IA_ERR_CUDA.  Device-side bounded waits that
  *     expire set a device flag, reported as IA_ERR_TIMEOUT by
  *     ia_check_device_errors().
+ *   - The tensor-core path holds the per-mode decay over half a chunk,
+ *     |lambda_m|^(-32) = exp(32 Delta_h |Re A_m|), in fp16 operands.  A head
+ *     whose factor exceeds 64 (Delta > 0.26 for S4D-Lin, whose
+ *     initialisation range [1e-3, 1e-1] gives at most 5), or whose Delta is
+ *     not positive, sets the device flag reported as IA_ERR_PARAM_RANGE by
+ *     ia_check_device_errors(); its outputs are then not to be used.  The
+ *     CUDA-core paths compute in fp32 and have no such limit.
+ *   - The library caches the device addresses of its own __device__
+ *     variables per device, keyed on the current context, so a context that
+ *     cudaDeviceReset replaced is looked up again.
  */
 #ifndef IA_H
 #define IA_H
@@ -57,8 +67,16 @@ typedef enum {
   IA_ERR_UNSUPPORTED = 2,   /* shape or dtype outside what the kernels implement */
   IA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the query says */
   IA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
-  IA_ERR_TIMEOUT = 5        /* a device-side bounded wait expired (see ia_check_device_errors) */
+  IA_ERR_TIMEOUT = 5,       /* a device-side bounded wait expired (see ia_check_device_errors) */
+  IA_ERR_PARAM_RANGE = 6    /* Delta or A outside what the tensor-core path holds (see above) */
 } ia_status_t;
+
+/* Which kernels a shape runs on (see ia_prefill_path, ia_fwd_bwd_path). */
+typedef enum {
+  IA_PATH_NONE = 0,          /* invalid shape */
+  IA_PATH_TENSOR_CORE = 1,   /* chunked tcgen05 kernels, chunk length 64 */
+  IA_PATH_SEQUENTIAL = 2     /* token-serial fp32 CUDA-core kernel, one CTA per (b,h) */
+} ia_path_t;
 
 typedef enum { IA_F32 = 0, IA_BF16 = 1 } ia_dtype_t;
 
@@ -77,6 +95,18 @@ IA_API size_t ia_prefill_workspace_bytes(const ia_shape_t* shape);
 
 /* Workspace bytes ia_fwd_bwd needs for this shape. */
 IA_API size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* shape);
+
+/* Path of ia_prefill_fwd for this shape.  The tensor-core path takes bf16
+ * inputs with M = 64 and d_xi, d_v in {64, 128}; every other shape (and fp32
+ * input) runs the token-serial CUDA-core kernel, which is correct for any
+ * shape whose state fits in shared memory but one to two orders of
+ * magnitude slower on long sequences. */
+IA_API ia_path_t ia_prefill_path(const ia_shape_t* shape);
+
+/* Path of ia_fwd_bwd for this shape.  The tensor-core reverse pass takes
+ * bf16 inputs with M = 64 and d_xi = d_v = 64; every other shape, d = 128
+ * included, runs the token-serial CUDA-core adjoint. */
+IA_API ia_path_t ia_fwd_bwd_path(const ia_shape_t* shape);
 
 /* Number of kernel launches one ia_prefill_fwd call makes for this shape
  * (the tensor-core path adds a state-only pass and a carry scan when it
@@ -107,8 +137,9 @@ IA_API ia_status_t ia_prefill_fwd(const ia_shape_t* shape, const void* q, const 
  * and results as ia_prefill_fwd, minus the workspace.
  *   - Scratch lives in a fixed 2 MiB array compiled into the library, held by
  *     every GPU that loads the library until the process exits.  It holds
- *     the per-head tables of unsplit sequences: up to 97 heads.  More heads
- *     return IA_ERR_WORKSPACE and launch nothing.
+ *     the per-head tables of unsplit sequences (20,992 bytes per head): up
+ *     to ia_prefill_static_max_heads() = 99 heads.  More heads return
+ *     IA_ERR_WORKSPACE and launch nothing.
  *   - Only the tensor-core shapes run here (bf16 inputs, M = 64, d_xi and d_v
  *     in {64, 128}); other shapes return IA_ERR_UNSUPPORTED.
  *   - The first call on each device looks up the array's device address;
@@ -118,6 +149,9 @@ IA_API ia_status_t ia_prefill_fwd(const ia_shape_t* shape, const void* q, const 
  *     threads) race on it; the caller must serialise them.
  *   - Never calls cudaMalloc, cudaFree or any other allocating routine.
  */
+/* Largest H that ia_prefill_fwd_static accepts (99). */
+IA_API int ia_prefill_static_max_heads(void);
+
 IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* shape, const void* q, const void* k,
                                          const void* v, const float* delta, const float* A,
                                          const void* state_in, float* o, float* num, float* den,
@@ -161,9 +195,24 @@ IA_API ia_status_t ia_decode_step(const ia_shape_t* shape, const void* q, const 
  */
 IA_API ia_status_t ia_set_launch_events(void* begin, void* end);
 
-/* Synchronises `stream`, then reports (and clears) the device error flag
- * that bounded waits set when they expire: IA_OK or IA_ERR_TIMEOUT. */
+/* Synchronises `stream`, then reports (and clears) the device error flag:
+ * IA_ERR_TIMEOUT if a bounded wait expired, else IA_ERR_PARAM_RANGE if a
+ * tensor-core call met an out-of-range Delta, else IA_OK. */
 IA_API ia_status_t ia_check_device_errors(void* stream);
+
+/*
+ * Self-test of the bounded waits (a diagnostic with no counterpart in the
+ * paper).  Launches one small kernel on `stream` that waits on shared-memory
+ * barriers nobody completes, with nothing else in flight: one plain bounded
+ * wait and one abortable wait that expire after limit_ns (1e3 .. 1e9 ns),
+ * and one abortable wait with the full one-second limit that must give up as
+ * soon as the other raises the CTA's abort flag.  out (device, 6 x u64):
+ * per waiter, 1 if its barrier completed (it never does) and the ns its wait
+ * took.  After the kernel, ia_check_device_errors() returns IA_ERR_TIMEOUT
+ * once and clears the flag.  Faults, traps and hangs nothing.
+ */
+IA_API ia_status_t ia_selftest_wait_expiry(unsigned long long limit_ns, unsigned long long* out,
+                                           void* stream);
 
 /* Static description of a status code. */
 IA_API const char* ia_status_string(ia_status_t status);

@@ -19,8 +19,9 @@ import os
 import torch
 
 __all__ = ["IAError", "load_library", "state_bytes", "prefill_workspace_bytes",
-           "fwd_bwd_workspace_bytes", "prefill_fwd", "prefill_fwd_static", "fwd_bwd", "decode_step",
-           "check_device_errors", "set_launch_events", "library_path", "IA_F32", "IA_BF16"]
+           "fwd_bwd_workspace_bytes", "prefill_path", "fwd_bwd_path", "prefill_static_max_heads",
+           "prefill_fwd", "prefill_fwd_static", "fwd_bwd", "decode_step", "check_device_errors",
+           "selftest_wait_expiry", "set_launch_events", "library_path", "IA_F32", "IA_BF16"]
 
 IA_F32, IA_BF16 = 0, 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,8 @@ _LIB_PATH = os.path.join(_HERE, "lib", "libia.so")
 _lib = None
 
 STATUS = {0: "IA_OK", 1: "IA_ERR_INVALID_ARG", 2: "IA_ERR_UNSUPPORTED", 3: "IA_ERR_WORKSPACE",
-          4: "IA_ERR_CUDA", 5: "IA_ERR_TIMEOUT"}
+          4: "IA_ERR_CUDA", 5: "IA_ERR_TIMEOUT", 6: "IA_ERR_PARAM_RANGE"}
+PATHS = {0: None, 1: "tensor_core", 2: "sequential"}
 
 
 class IAError(RuntimeError):
@@ -61,8 +63,13 @@ def load_library():
     for name in ("ia_state_bytes", "ia_prefill_workspace_bytes", "ia_fwd_bwd_workspace_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [S]
-    lib.ia_prefill_launches.restype = ctypes.c_int
-    lib.ia_prefill_launches.argtypes = [S]
+    for name in ("ia_prefill_launches", "ia_prefill_path", "ia_fwd_bwd_path"):
+        getattr(lib, name).restype = ctypes.c_int
+        getattr(lib, name).argtypes = [S]
+    lib.ia_prefill_static_max_heads.restype = ctypes.c_int
+    lib.ia_prefill_static_max_heads.argtypes = []
+    lib.ia_selftest_wait_expiry.restype = ctypes.c_int
+    lib.ia_selftest_wait_expiry.argtypes = [ctypes.c_ulonglong, P, P]
     lib.ia_prefill_fwd.restype = ctypes.c_int
     lib.ia_prefill_fwd.argtypes = [S] + [P] * 10 + [P, ctypes.c_size_t, P]
     lib.ia_prefill_fwd_static.restype = ctypes.c_int
@@ -122,6 +129,20 @@ def prefill_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
 
 def prefill_launches(B, H, N, d_xi, d_v, M, dtype) -> int:
     return int(load_library().ia_prefill_launches(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
+
+
+def prefill_path(B, H, N, d_xi, d_v, M, dtype):
+    """'tensor_core' or 'sequential': the kernels ia_prefill_fwd runs for this shape."""
+    return PATHS[load_library().ia_prefill_path(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype)))]
+
+
+def fwd_bwd_path(B, H, N, d_xi, d_v, M, dtype):
+    """'tensor_core' or 'sequential': the reverse-pass kernels ia_fwd_bwd runs for this shape."""
+    return PATHS[load_library().ia_fwd_bwd_path(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype)))]
+
+
+def prefill_static_max_heads() -> int:
+    return int(load_library().ia_prefill_static_max_heads())
 
 
 def fwd_bwd_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
@@ -317,5 +338,17 @@ def set_launch_events(begin=None, end=None):
 
 
 def check_device_errors(stream=None):
-    """Synchronise the stream and raise if a device-side bounded wait expired."""
+    """Synchronise the stream and raise if a device-side bounded wait expired
+    (IA_ERR_TIMEOUT) or a tensor-core call met an out-of-range Delta
+    (IA_ERR_PARAM_RANGE); the flag is cleared either way."""
     _check(load_library().ia_check_device_errors(_stream(stream)), "ia_check_device_errors")
+
+
+def selftest_wait_expiry(limit_ns, device=None, stream=None):
+    """Run the library's bounded-wait self-test kernel (see include/ia.h) and
+    return its six u64 results: per waiter, completed flag and ns waited."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    out = torch.zeros(6, dtype=torch.int64, device=dev)
+    _check(load_library().ia_selftest_wait_expiry(ctypes.c_ulonglong(int(limit_ns)), _ptr(out), _stream(stream)),
+           "ia_selftest_wait_expiry")
+    return out

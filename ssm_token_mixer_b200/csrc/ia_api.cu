@@ -36,17 +36,6 @@ int num_sms() {
   return n;
 }
 
-bool valid_dims(const ia_shape_t* s, bool need_n) {
-  if (!s) return false;
-  if (s->B <= 0 || s->H <= 0 || s->d_xi <= 0 || s->d_v <= 0 || s->M <= 0) return false;
-  if (need_n && s->N <= 0) return false;
-  if (s->in_dtype != IA_F32 && s->in_dtype != IA_BF16) return false;
-  // element counts must stay addressable with 64-bit indices and int grid sizes
-  const long long BH = static_cast<long long>(s->B) * s->H;
-  if (BH > (1LL << 31) - 1) return false;
-  return true;
-}
-
 bool use_tc(const ia_shape_t& s) {
   if (env_set("IA_PREFILL_SIMT")) return false;   // debug switch: force the CUDA-core path
   return tc_prefill_supported(s);
@@ -63,7 +52,59 @@ cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
 
 }  // namespace
 
+bool valid_dims(const ia_shape_t* s, bool need_n) {
+  if (!s) return false;
+  if (s->B <= 0 || s->H <= 0 || s->d_xi <= 0 || s->d_v <= 0 || s->M <= 0) return false;
+  if (need_n && s->N <= 0) return false;
+  if (s->in_dtype != IA_F32 && s->in_dtype != IA_BF16) return false;
+  // element counts must stay addressable with 64-bit indices and int grid sizes
+  const long long BH = static_cast<long long>(s->B) * s->H;
+  if (BH > (1LL << 31) - 1) return false;
+  return true;
+}
+
 bool inject_launch_failure() { return env_set("IA_INJECT_LAUNCH_FAILURE"); }
+
+// The current context, through the driver entry point (the library links no
+// driver stub); nullptr if there is none or the lookup fails.
+void* current_context() {
+  using GetCtxFn = int (*)(void**);   // CUresult cuCtxGetCurrent(CUcontext*)
+  static const GetCtxFn fn = []() -> GetCtxFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<GetCtxFn>(f);
+  }();
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+void* SymbolCache::get(const void* symbol, cudaError_t* err) {
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  void* ctx = current_context();
+  if (addr[dev] && ctx && ctx == ctx_of[dev]) {
+    *err = cudaSuccess;
+    return addr[dev];
+  }
+  // First use on this device, or its context was replaced (cudaDeviceReset
+  // unloads the module): look the address up again.  The lookup creates the
+  // primary context if there is none yet, so the key is read after it.
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, symbol);
+  if (*err != cudaSuccess) return nullptr;
+  addr[dev] = p;
+  ctx_of[dev] = current_context();
+  return p;
+}
 
 void mark_launch_begin(cudaStream_t st) {
   if (g_ev_begin) cudaEventRecord(g_ev_begin, st);
@@ -73,16 +114,9 @@ void mark_launch_end(cudaStream_t st) {
 }
 
 int* device_error_ptr() {
-  constexpr int kMaxDev = 64;
-  static int* cache[kMaxDev] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-  if (!cache[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int*>(p);
-  }
-  return cache[dev];
+  static SymbolCache cache;
+  cudaError_t e;
+  return static_cast<int*>(cache.get(&g_device_error, &e));
 }
 
 int read_and_clear_device_error(cudaStream_t st, cudaError_t* err) {
@@ -208,7 +242,19 @@ ia_status_t ia_check_device_errors(void* stream) {
   cudaError_t e;
   int flag = read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);
   if (e != cudaSuccess) return IA_ERR_CUDA;
-  return flag ? IA_ERR_TIMEOUT : IA_OK;
+  if (flag & kErrTimeout) return IA_ERR_TIMEOUT;
+  if (flag & kErrParamRange) return IA_ERR_PARAM_RANGE;
+  return IA_OK;
+}
+
+ia_path_t ia_prefill_path(const ia_shape_t* s) {
+  if (!valid_dims(s, true)) return IA_PATH_NONE;
+  return use_tc(*s) ? IA_PATH_TENSOR_CORE : IA_PATH_SEQUENTIAL;
+}
+
+ia_path_t ia_fwd_bwd_path(const ia_shape_t* s) {
+  if (!valid_dims(s, true)) return IA_PATH_NONE;
+  return use_tc_bwd(*s) ? IA_PATH_TENSOR_CORE : IA_PATH_SEQUENTIAL;
 }
 
 const char* ia_status_string(ia_status_t st) {
@@ -219,6 +265,8 @@ const char* ia_status_string(ia_status_t st) {
     case IA_ERR_WORKSPACE: return "IA_ERR_WORKSPACE: workspace missing or too small";
     case IA_ERR_CUDA: return "IA_ERR_CUDA: CUDA runtime or launch failure";
     case IA_ERR_TIMEOUT: return "IA_ERR_TIMEOUT: a device-side bounded wait expired";
+    case IA_ERR_PARAM_RANGE:
+      return "IA_ERR_PARAM_RANGE: Delta or A outside the range the tensor-core path holds in fp16";
   }
   return "unknown ia_status_t";
 }

@@ -50,15 +50,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete, for at most one
-// second.  On expiry sets bit 0 of *err (the library's device error flag,
-// read and cleared by ia_check_device_errors) and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Device error flag bits (the library's flag, read and cleared by
+// ia_check_device_errors): a bounded wait expired; a parameter was outside
+// the range the tensor-core operands hold.
+constexpr int kErrTimeout = 1;
+constexpr int kErrParamRange = 2;
+
+// Waits for the phase with the given parity to complete, for at most
+// limit_ns (one second unless a caller passes less).  On expiry sets
+// kErrTimeout in *err and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   unsigned long long t0 = global_ns();
   while (!mbar_test(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicOr(err, 1);
+    if (global_ns() - t0 > limit_ns) {
+      atomicOr(err, kErrTimeout);
       return false;
     }
   }
@@ -73,13 +80,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // Bounded wait that also gives up as soon as another thread of the CTA has
 // raised *abort (a shared flag); raises it itself on expiry.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, int* err,
-                                                   volatile int* abort) {
+                                                   volatile int* abort,
+                                                   unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   unsigned long long t0 = global_ns();
   while (!mbar_test(bar, parity)) {
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicOr(err, 1);
+    if (global_ns() - t0 > limit_ns) {
+      atomicOr(err, kErrTimeout);
       *abort = 1;
       return false;
     }

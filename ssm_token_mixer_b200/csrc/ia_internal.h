@@ -74,8 +74,24 @@ bool inject_launch_failure();
 void mark_launch_begin(cudaStream_t st);
 void mark_launch_end(cudaStream_t st);
 
-// Device address of the library's error flag on the current device (looked
-// up once per device), or nullptr if the lookup fails.
+// Shape check shared by every entry point: positive dims (N only when
+// need_n), a known dtype, and B*H within int range.
+bool valid_dims(const ia_shape_t* s, bool need_n);
+
+// Device address of a __device__ variable of this library on the current
+// device.  In host code the variable's name is only a host-side stand-in, so
+// the address is looked up with the device current and cached per device,
+// keyed on the device's current context: a context created after
+// cudaDeviceReset triggers a fresh lookup.
+struct SymbolCache {
+  static constexpr int kMaxDevices = 64;
+  void* addr[kMaxDevices] = {};
+  void* ctx_of[kMaxDevices] = {};
+  void* get(const void* symbol, cudaError_t* err);
+};
+
+// Device address of the library's error flag on the current device, or
+// nullptr if the lookup fails.
 int* device_error_ptr();
 int read_and_clear_device_error(cudaStream_t st, cudaError_t* err);
 

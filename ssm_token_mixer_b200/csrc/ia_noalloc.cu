@@ -12,7 +12,8 @@
 // the library until the process exits).  It never allocates.
 //
 // It always runs the sequences unsplit (one CTA per (b,h)), so the scratch
-// only holds the per-head tables: 21.5 KB per head, up to 97 heads.
+// only holds the per-head tables: sizeof(HeadTables) per head plus 256 bytes
+// of alignment slack, kStaticMaxHeads heads at most.
 #include <cstdint>
 
 #include "ia_internal.h"
@@ -22,34 +23,16 @@ namespace ia {
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(2) << 20;   // 2 MiB per GPU
-constexpr int kMaxDevices = 64;
+// The per-head tables of an unsplit prefill take sizeof(HeadTables) per head
+// after a 256-byte alignment allowance (tc_workspace_bytes with one segment).
+constexpr int kStaticMaxHeads = static_cast<int>((kStaticScratchBytes - 256) / sizeof(HeadTables));
+static_assert(sizeof(HeadTables) == 20992 && kStaticMaxHeads == 99,
+              "the head limit stated in include/ia.h follows the table size");
 
 // Shared by every call on a device; it keeps the last call's contents.  The
 // tables are rewritten at the start of every call, so nothing in it has to
 // start at zero.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
-
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-void* static_scratch_on_current_device(cudaError_t* err) {
-  static void* cache[kMaxDevices] = {};
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return nullptr;
-  if (dev < 0 || dev >= kMaxDevices) {
-    *err = cudaErrorInvalidDevice;
-    return nullptr;
-  }
-  if (!cache[dev]) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (*err != cudaSuccess) return nullptr;
-    cache[dev] = p;
-  }
-  *err = cudaSuccess;
-  return cache[dev];
-}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -58,14 +41,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 using namespace ia;
 
+extern "C" IA_API int ia_prefill_static_max_heads(void) { return kStaticMaxHeads; }
+
 extern "C" IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* s, const void* q,
                                                     const void* k, const void* v,
                                                     const float* delta, const float* A,
                                                     const void* state_in, float* o, float* num,
                                                     float* den, void* state_out, void* stream) {
-  if (!s || s->B <= 0 || s->H <= 0 || s->N <= 0 || s->d_xi <= 0 || s->d_v <= 0 || s->M <= 0)
-    return IA_ERR_INVALID_ARG;
-  if (s->in_dtype != IA_F32 && s->in_dtype != IA_BF16) return IA_ERR_INVALID_ARG;
+  if (!valid_dims(s, true)) return IA_ERR_INVALID_ARG;
   if (!q || !k || !v || !delta || !o) return IA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, delta, A, state_in, o, num, den, state_out};
   for (const void* p : ptrs)
@@ -76,8 +59,12 @@ extern "C" IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* s, const v
   const TcPlan plan{1, nch};
   if (tc_workspace_bytes(*s, plan) > kStaticScratchBytes) return IA_ERR_WORKSPACE;
   if (inject_launch_failure()) return IA_ERR_CUDA;
+  // Device address of the scratch array: in host code its name is only a
+  // host-side stand-in, so it is looked up with the device current, once per
+  // device (again after a device reset), and cached.
+  static SymbolCache scratch_cache;
   cudaError_t e;
-  void* scratch = static_scratch_on_current_device(&e);
+  void* scratch = scratch_cache.get(&g_static_scratch, &e);
   if (!scratch) return IA_ERR_CUDA;
   e = launch_tc_prefill(*s, plan, q, k, v, delta, A, state_in, o, num, den, state_out, scratch,
                         static_cast<cudaStream_t>(stream));

@@ -89,10 +89,18 @@ __device__ __forceinline__ float warp_sum(float x) {
 // reverse pass: dtab[h][k][j] = component (k & 1) of dE'[j, k/2]/dDelta =
 // lambda^n (lambda + n A b), n = c - j, fp32, followed by the row sums
 // dtab[H*128*64 + h*128 + k].
+// The tensor-core operands carry factors up to |lambda_m|^(-C/2) =
+// exp(Delta |Re A_m| C/2) in fp16 (the centred decay table and the readout
+// scale); a head whose factor exceeds kMaxHalfChunkGrowth, or whose Delta is
+// not positive, raises kErrParamRange in *err instead of returning numbers
+// that may have overflowed.
+constexpr double kMaxHalfChunkGrowth = 64.0;
+
 __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const float* __restrict__ delta,
                                                                     const float* __restrict__ A,
                                                                     HeadTables* __restrict__ tabs,
-                                                                    float* __restrict__ dtab) {
+                                                                    float* __restrict__ dtab,
+                                                                    int* __restrict__ err) {
   __shared__ __align__(16) __half Es[2 * kModesTC * kChunk];
   griddep_launch_dependents();   // the chunk pass may start its table-free prologue now
   const int h = blockIdx.x;
@@ -102,6 +110,7 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
   const int m = threadIdx.x >> 2, part = threadIdx.x & 3;   // four threads per mode, adjacent lanes
   ModeD md = mode_consts(dl, A, m);
   const double rdA = dl * md.ar, idA = dl * md.ai;
+  if (part == 0 && !(dl > 0.f && fabs(rdA) * (C / 2) <= log(kMaxHalfChunkGrowth))) atomicOr(err, kErrParamRange);
   double pr, pi, ir, ii;
   cpow_d(rdA, idA, c - JS * part, &pr, &pi);   // lambda^(c-j) at this thread's first j
   cpow_d(rdA, idA, -1.0, &ir, &ii);            // lambda^-1
@@ -559,7 +568,9 @@ __global__ void segment_scan_kernel(int H, int DX, int DV, int nseg, int L,
 // host-side launchers
 cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
                                 cudaStream_t st, float* dtab) {
-  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs, dtab);
+  int* err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs, dtab, err);
   return cudaGetLastError();
 }
 

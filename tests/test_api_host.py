@@ -104,8 +104,46 @@ def test_injected_launch_failure(lib, monkeypatch):
     assert prefill(lib, shape(B=0)) == 1
 
 
+def test_no_alloc_head_limit_and_shape_checks(lib, monkeypatch):
+    # The limit follows the table size: 99 heads of 20,992 bytes fit the
+    # 2 MiB array after its 256-byte alignment allowance.  H = 99 passes every
+    # check (the injected failure then stops it before any launch), H = 100
+    # is refused as too large for the array.
+    assert lib.ia_prefill_static_max_heads() == 99
+    monkeypatch.setenv("IA_INJECT_LAUNCH_FAILURE", "1")
+
+    def static(s):
+        return lib.ia_prefill_fwd_static(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None,
+                                         None, None, None)
+    assert static(shape(B=1, H=99, N=64, dx=64, dv=64, M=64, dt=1)) == 4
+    assert static(shape(B=1, H=100, N=64, dx=64, dv=64, M=64, dt=1)) == 3
+    # the same shape checks as ia_prefill_fwd: B*H beyond int range is invalid
+    assert static(shape(B=1 << 16, H=1 << 16, N=64, dx=64, dv=64, M=64, dt=1)) == 1
+    assert prefill(lib, shape(B=1 << 16, H=1 << 16, N=64)) == 1
+    assert static(shape(B=1, H=2, N=64, dx=32, dv=64, M=64, dt=1)) == 2   # not a tensor-core shape
+
+
+def test_path_queries(lib):
+    def paths(**kw):
+        s = shape(**kw)
+        return lib.ia_prefill_path(ctypes.byref(s)), lib.ia_fwd_bwd_path(ctypes.byref(s))
+    TC, SEQ = 1, 2
+    assert paths(B=8, H=12, N=2048, dx=64, dv=64, M=64, dt=1) == (TC, TC)
+    assert paths(B=4, H=16, N=2048, dx=128, dv=128, M=64, dt=1) == (TC, SEQ)   # d = 128 training: CUDA cores
+    assert paths(B=1, H=2, N=256, dx=16, dv=16, M=16, dt=0) == (SEQ, SEQ)     # fp32 inputs
+    assert paths(B=1, H=2, N=256, dx=64, dv=64, M=32, dt=1) == (SEQ, SEQ)     # M != 64
+    assert paths(B=0) == (0, 0)
+
+
+def test_selftest_argument_checks(lib):
+    assert lib.ia_selftest_wait_expiry(ctypes.c_ulonglong(1000000), None, None) == 1
+    assert lib.ia_selftest_wait_expiry(ctypes.c_ulonglong(10), FAKE, None) == 1          # limit too short
+    assert lib.ia_selftest_wait_expiry(ctypes.c_ulonglong(2 * 10 ** 9), FAKE, None) == 1  # above one second
+    assert lib.ia_selftest_wait_expiry(ctypes.c_ulonglong(1000000), ctypes.c_void_p(0x10004), None) == 1
+
+
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert lib.ia_status_string(code).startswith(b"IA_")
     assert b"unknown" in lib.ia_status_string(99)
 

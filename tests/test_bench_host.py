@@ -70,3 +70,15 @@ def test_reference_arm_reports_the_gpu_arms_config(capsys, monkeypatch):
     assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
     assert line["e2e"]["value"] == line["value"] == line["cpu_baseline"]["value"]
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+
+
+def test_rank_workload_weak_and_strong():
+    import bench
+    from ssm_token_mixer_b200.workloads import WORKLOADS
+    w = WORKLOADS["prefill_125m"]
+    assert bench.rank_workload(w, 0, 1, "strong") == (w, 8)
+    assert bench.rank_workload(w, 1, 4, "weak") == (w, 32)          # every rank: the full batch of 8
+    parts = [bench.rank_workload(w, r, 3, "strong") for r in range(3)]
+    assert [p[0].B for p in parts] == [3, 3, 2] and {p[1] for p in parts} == {8}
+    with pytest.raises(SystemExit):
+        bench.rank_workload(WORKLOADS["prefill_1p3b_7168"], 0, 2, "strong")   # B = 1 cannot split
