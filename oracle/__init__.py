@@ -61,12 +61,12 @@ def _load():
         lib.iao_state_len.restype = ctypes.c_long
         lib.iao_state_len.argtypes = [i] * 5
         lib.iao_params.argtypes = [i, ctypes.c_double, P, P, P]
-        lib.iao_forward.argtypes = [i] * 6 + [P] * 10
+        lib.iao_forward.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 6
         lib.iao_forward_features.argtypes = [i] * 6 + [P] * 10
-        lib.iao_decode_step.argtypes = [i] * 5 + [P] * 9
-        lib.iao_brute.argtypes = [i] * 6 + [P] * 8
-        lib.iao_backward.argtypes = [i] * 6 + [P] * 11
-        lib.iao_jvp.argtypes = [i] * 6 + [P] * 10
+        lib.iao_decode_step.argtypes = [i] * 5 + [P] * 4 + [i] + [P] * 5
+        lib.iao_brute.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 4
+        lib.iao_backward.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 8
+        lib.iao_jvp.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 7
         lib.iao_num_threads.restype = i
         for name in ("iao_params", "iao_forward", "iao_forward_features", "iao_decode_step",
                      "iao_brute", "iao_backward", "iao_jvp"):
@@ -85,6 +85,11 @@ def _f64(x):
 
 def _p(x):
     return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dpm(delta):
+    """1 if delta holds one value per head and mode ([H,M]), 0 for one per head ([H])."""
+    return 1 if delta.ndim == 2 else 0
 
 
 def _check(rc, name):
@@ -120,7 +125,7 @@ def params(M, delta, A=None):
 
 
 def forward(q, k, v, delta, M, A=None, state_in=None, want_state=True):
-    """Sequential recurrence.  q,k [B,H,N,d_xi], v [B,H,N,d_v], delta [H], M modes.
+    """Sequential recurrence.  q,k [B,H,N,d_xi], v [B,H,N,d_v], delta [H] or [H,M], M modes.
 
     Returns dict(o, num, den, state) in fp64 (state flat, see split_state)."""
     q, k, v, delta, A, state_in = map(_f64, (q, k, v, delta, A, state_in))
@@ -134,7 +139,7 @@ def _forward(q, k, v, delta, A, state_in, want_state, M):
     num = np.zeros((B, H, N, d_v))
     den = np.zeros((B, H, N))
     st = np.zeros(state_len(B, H, M, d_xi, d_v)) if want_state else None
-    rc = _load().iao_forward(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _p(A),
+    rc = _load().iao_forward(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _dpm(delta), _p(A),
                              _p(state_in), _p(o), _p(num), _p(den), _p(st))
     _check(rc, "forward")
     return {"o": o, "num": num, "den": den, "state": st}
@@ -167,7 +172,7 @@ def decode_step(q, k, v, delta, M, state, A=None):
     o = np.zeros((B, H, d_v))
     num = np.zeros((B, H, d_v))
     den = np.zeros((B, H))
-    rc = _load().iao_decode_step(B, H, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _p(A),
+    rc = _load().iao_decode_step(B, H, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _dpm(delta), _p(A),
                                  _p(st), _p(o), _p(num), _p(den))
     _check(rc, "decode_step")
     return o, num, den, st
@@ -180,14 +185,17 @@ def brute(q, k, v, delta, M, A=None):
     o = np.zeros((B, H, N, d_v))
     num = np.zeros((B, H, N, d_v))
     den = np.zeros((B, H, N))
-    rc = _load().iao_brute(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _p(A),
+    rc = _load().iao_brute(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _dpm(delta), _p(A),
                            _p(o), _p(num), _p(den))
     _check(rc, "brute")
     return {"o": o, "num": num, "den": den}
 
 
 def backward(q, k, v, delta, dO, M, A=None):
-    """Reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta)."""
+    """Reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta, dA).
+
+    dDelta has delta's shape ([H] or [H,M]); dA is [2M] as (dL/dRe A_m,
+    dL/dIm A_m) pairs, summed over batch, heads and time."""
     q, k, v, delta, dO, A = map(_f64, (q, k, v, delta, dO, A))
     B, H, N, d_xi = q.shape
     d_v = v.shape[-1]
@@ -195,19 +203,22 @@ def backward(q, k, v, delta, dO, M, A=None):
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
-    dD = np.zeros(H)
-    rc = _load().iao_backward(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _p(A),
-                              _p(dO), _p(o), _p(dq), _p(dk), _p(dv), _p(dD))
+    dD = np.zeros(delta.shape)
+    dA = np.zeros(2 * M)
+    rc = _load().iao_backward(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _dpm(delta), _p(A),
+                              _p(dO), _p(o), _p(dq), _p(dk), _p(dv), _p(dD), _p(dA))
     _check(rc, "backward")
-    return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD}
+    return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD, "dA": dA}
 
 
-def jvp(q, k, v, delta, tq, tk, tv, tdelta, M, A=None):
-    q, k, v, delta, tq, tk, tv, tdelta, A = map(_f64, (q, k, v, delta, tq, tk, tv, tdelta, A))
+def jvp(q, k, v, delta, tq, tk, tv, tdelta, M, A=None, tA=None):
+    """Output tangent along (tq, tk, tv, tdelta[, tA]); tdelta has delta's shape,
+    tA is [2M] (re, im) pairs or None."""
+    q, k, v, delta, tq, tk, tv, tdelta, A, tA = map(_f64, (q, k, v, delta, tq, tk, tv, tdelta, A, tA))
     B, H, N, d_xi = q.shape
     d_v = v.shape[-1]
     to = np.zeros((B, H, N, d_v))
-    rc = _load().iao_jvp(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _p(A),
-                         _p(tq), _p(tk), _p(tv), _p(tdelta), _p(to))
+    rc = _load().iao_jvp(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), _p(delta), _dpm(delta), _p(A),
+                         _p(tq), _p(tk), _p(tv), _p(tdelta), _p(tA), _p(to))
     _check(rc, "jvp")
     return to

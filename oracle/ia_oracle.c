@@ -15,8 +15,9 @@
  *     num_t = Re(a_t^H Gamma_t), den_t = Re(a_t^H eta_t), a_t = U_t xi(q_t).
  * Readings where the pages are silent: xi = elu + 1 (alpha = 1); S4D-Lin
  * A_m = -1/2 + i*pi*m, m = 0..M-1; zero-order-hold b = (lambda - 1)/A; one
- * Delta per head shared by all modes; the state is updated with token t
- * before query t reads it (inclusive causality); no epsilon in o = num/den.
+ * Delta per head shared by all modes, or (flag dpm) one Delta per head and
+ * mode, Delta[h][m]; the state is updated with token t before query t reads
+ * it (inclusive causality); no epsilon in o = num/den.
  *
  * All arithmetic is IEEE fp64 in the order written; no blocking or fusion.
  */
@@ -45,6 +46,11 @@ static cd mode_A(const double* A, int m) {
   return -0.5 + I * (kPi * (double)m);          /* S4D-Lin */
 }
 
+/* Delta of head h and mode m: one per head, or one per (head, mode) with dpm. */
+static double delta_hm(const double* delta, int dpm, int M, int h, int m) {
+  return dpm ? delta[(long)h * M + m] : delta[h];
+}
+
 static cd ld_c(const double* p) { return p[0] + I * p[1]; }
 static void st_c(double* p, cd z) { p[0] = creal(z); p[1] = cimag(z); }
 
@@ -60,14 +66,20 @@ int iao_num_threads(void) {
 #endif
 }
 
-/* Zero-order hold of dx/dt = A x + u over a step Delta. */
+/* Zero-order hold of dx/dt = A x + u over a step Delta:
+ * lambda = exp(Delta A), b = (lambda - 1) / A. */
+static void zoh(double delta, cd a, cd* l, cd* bm) {
+  *l = cexp(delta * a);
+  *bm = (*l - 1.0) / a;
+}
+
 int iao_params(int M, double delta, const double* A, double* lam, double* b) {
   if (M <= 0 || !(delta > 0.0) || !lam || !b) return -1;
   for (int m = 0; m < M; ++m) {
-    cd a = mode_A(A, m);
-    cd l = cexp(delta * a);
+    cd l, bm;
+    zoh(delta, mode_A(A, m), &l, &bm);
     st_c(lam + 2 * m, l);
-    st_c(b + 2 * m, (l - 1.0) / a);
+    st_c(b + 2 * m, bm);
   }
   return 0;
 }
@@ -194,24 +206,31 @@ static int forward_impl(int B, int H, int N, int d_xi, int d_v, int M,
   return err;
 }
 
-static int head_tables(int H, int M, const double* delta, const double* A,
+static int head_tables(int H, int M, const double* delta, int dpm, const double* A,
                        double** lamtab, double** btab) {
   *lamtab = malloc(sizeof(double) * 2 * (size_t)H * M);
   *btab = malloc(sizeof(double) * 2 * (size_t)H * M);
   if (!*lamtab || !*btab) return -2;
   for (int h = 0; h < H; ++h) {
-    if (iao_params(M, delta[h], A, *lamtab + 2L * h * M, *btab + 2L * h * M)) return -1;
+    for (int m = 0; m < M; ++m) {
+      double dl = delta_hm(delta, dpm, M, h, m);
+      if (!(dl > 0.0)) return -1;
+      cd l, bm;
+      zoh(dl, mode_A(A, m), &l, &bm);
+      st_c(*lamtab + 2L * ((long)h * M + m), l);
+      st_c(*btab + 2L * ((long)h * M + m), bm);
+    }
   }
   return 0;
 }
 
 int iao_forward(int B, int H, int N, int d_xi, int d_v, int M,
                 const double* q, const double* k, const double* v,
-                const double* delta, const double* A, const double* state_in,
+                const double* delta, int dpm, const double* A, const double* state_in,
                 double* o, double* num, double* den, double* state_out) {
   if (bad_dims(B, H, N, d_xi, d_v, M) || !delta) return -1;
   double *lt = NULL, *bt = NULL;
-  int err = head_tables(H, M, delta, A, &lt, &bt);
+  int err = head_tables(H, M, delta, dpm, A, &lt, &bt);
   if (!err)
     err = forward_impl(B, H, N, d_xi, d_v, M, q, k, 1, v, lt, bt, state_in, o, num, den,
                        state_out);
@@ -229,7 +248,7 @@ int iao_forward_features(int B, int H, int N, int d_xi, int d_v, int M,
 
 int iao_decode_step(int B, int H, int d_xi, int d_v, int M,
                     const double* q, const double* k, const double* v,
-                    const double* delta, const double* A, double* state,
+                    const double* delta, int dpm, const double* A, double* state,
                     double* o, double* num, double* den) {
   if (!state) return -1;
   /* One iteration of the loop body, reading and writing the same state. */
@@ -237,7 +256,7 @@ int iao_decode_step(int B, int H, int d_xi, int d_v, int M,
   double* tmp = malloc(sizeof(double) * (size_t)n);
   if (!tmp) return -2;
   memcpy(tmp, state, sizeof(double) * (size_t)n);
-  int err = iao_forward(B, H, 1, d_xi, d_v, M, q, k, v, delta, A, tmp, o, num, den, state);
+  int err = iao_forward(B, H, 1, d_xi, d_v, M, q, k, v, delta, dpm, A, tmp, o, num, den, state);
   free(tmp);
   return err;
 }
@@ -251,7 +270,7 @@ int iao_decode_step(int B, int H, int d_xi, int d_v, int M,
  */
 int iao_brute(int B, int H, int N, int d_xi, int d_v, int M,
               const double* q, const double* k, const double* v,
-              const double* delta, const double* A,
+              const double* delta, int dpm, const double* A,
               double* o, double* num, double* den) {
   if (bad_dims(B, H, N, d_xi, d_v, M) || !q || !k || !v || !delta || !o) return -1;
   long BH = (long)B * H;
@@ -266,13 +285,14 @@ int iao_brute(int B, int H, int N, int d_xi, int d_v, int M,
     for (int t = 0; t < N; ++t) {
       for (int m = 0; m < M; ++m) {
         cd Am = mode_A(A, m);
-        cd bm = (cexp(delta[h] * Am) - 1.0) / Am;
+        double dl = delta_hm(delta, dpm, M, h, m);
+        cd bm = (cexp(dl * Am) - 1.0) / Am;
         cd acc = 0.0;
         for (int n = 0; n <= t; ++n) {
           double s = 0.0;
           for (int f = 0; f < d_xi; ++f)
             s += feat(qb[(long)t * d_xi + f]) * feat(kb[(long)n * d_xi + f]);
-          acc += cexp((double)(t - n) * delta[h] * Am) * s;
+          acc += cexp((double)(t - n) * dl * Am) * s;
         }
         a[m] = bm * acc;
       }
@@ -281,8 +301,9 @@ int iao_brute(int B, int H, int N, int d_xi, int d_v, int M,
         double wt = 0.0;
         for (int m = 0; m < M; ++m) {
           cd Am = mode_A(A, m);
-          cd bm = (cexp(delta[h] * Am) - 1.0) / Am;
-          wt += creal(conj(a[m]) * bm * cexp((double)(t - n) * delta[h] * Am));
+          double dl = delta_hm(delta, dpm, M, h, m);
+          cd bm = (cexp(dl * Am) - 1.0) / Am;
+          wt += creal(conj(a[m]) * bm * cexp((double)(t - n) * dl * Am));
         }
         w[n] = wt;
         dn += wt;
@@ -310,25 +331,33 @@ int iao_brute(int B, int H, int N, int d_xi, int d_v, int M,
  *   reverse scans:  G_t = g_t + conj(lambda) G_{t+1}   (U, Gamma, eta alike)
  *   dxi(k_t)[f] = Re sum_m conj(b_m) G^U_t[m,f],  dv_t[f] likewise with G^Gamma
  *   gbar_lambda_m = sum_t G_t . conj(S_{t-1}),  gbar_b_m = sum_t G_t . x_t
- *   dDelta_h = sum_m Re(conj(gbar_lambda_m) A_m lambda_m + conj(gbar_b_m) lambda_m)
+ *   dDelta_hm = Re(conj(gbar_lambda_m) A_m lambda_m + conj(gbar_b_m) lambda_m)
+ *     (summed over the batch, and over m when one Delta serves all modes)
+ *   dA_m = sum over batch and heads of conj(dlambda/dA) gbar_lambda_m
+ *          + conj(db/dA) gbar_b_m,  dlambda/dA = Delta lambda,
+ *          db/dA = (Delta lambda - b) / A     (lambda = exp(Delta A), b = (lambda - 1)/A)
  *   dq = dxi(q) * xi'(q),  dk = dxi(k) * xi'(k).
- * Complex adjoints use the convention g = dL/dRe + i dL/dIm.  States are
- * recomputed forward from checkpoints every CK steps.
+ * Complex adjoints use the convention g = dL/dRe + i dL/dIm (so dA_m holds
+ * dL/dRe A_m and dL/dIm A_m).  States are recomputed forward from
+ * checkpoints every CK steps.
  */
 #define CK 64
 
 int iao_backward(int B, int H, int N, int d_xi, int d_v, int M,
                  const double* q, const double* k, const double* v,
-                 const double* delta, const double* A, const double* dO,
-                 double* o_out, double* dq, double* dk, double* dv, double* dDelta) {
+                 const double* delta, int dpm, const double* A, const double* dO,
+                 double* o_out, double* dq, double* dk, double* dv, double* dDelta,
+                 double* dA) {
   if (bad_dims(B, H, N, d_xi, d_v, M) || !q || !k || !v || !delta || !dO || !dq || !dk ||
       !dv || !dDelta)
     return -1;
   long BH = (long)B * H;
   long S1 = (long)M * d_xi, S2 = (long)M * d_v;
   long SL = S1 + S2 + M;                       /* complex entries per state */
-  double* part = calloc((size_t)BH, sizeof(double));
-  if (!part) return -2;
+  /* per (b,h,m): dL/dDelta_hm and the complex dL/dA_m of that sequence */
+  double* part = calloc((size_t)BH * M, sizeof(double));
+  cd* partA = calloc((size_t)BH * M, sizeof(cd));
+  if (!part || !partA) { free(part); free(partA); return -2; }
   int err = 0;
 #pragma omp parallel for schedule(dynamic, 1)
   for (long bh = 0; bh < BH; ++bh) {
@@ -359,7 +388,7 @@ int iao_backward(int B, int H, int N, int d_xi, int d_v, int M,
     } else {
       for (int m = 0; m < M; ++m) {
         Am[m] = mode_A(A, m);
-        lam[m] = cexp(delta[h] * Am[m]);
+        lam[m] = cexp(delta_hm(delta, dpm, M, h, m) * Am[m]);
         bb[m] = (lam[m] - 1.0) / Am[m];
       }
       for (long i = 0; i < (long)N * d_xi; ++i) { fq[i] = feat(qb[i]); fk[i] = feat(kb[i]); }
@@ -457,23 +486,34 @@ int iao_backward(int B, int H, int N, int d_xi, int d_v, int M,
           }
         }
       }
-      double dd = 0.0;
-      for (int m = 0; m < M; ++m)
-        dd += creal(conj(glam[m]) * Am[m] * lam[m] + conj(gb_[m]) * lam[m]);
-      part[bh] = dd;
+      for (int m = 0; m < M; ++m) {
+        double dl = delta_hm(delta, dpm, M, h, m);
+        part[bh * M + m] = creal(conj(glam[m]) * Am[m] * lam[m] + conj(gb_[m]) * lam[m]);
+        partA[bh * M + m] = conj(dl * lam[m]) * glam[m] + conj((dl * lam[m] - bb[m]) / Am[m]) * gb_[m];
+      }
     }
     free(lam); free(bb); free(Am); free(ck); free(blk); free(G); free(ga); free(a);
     free(glam); free(gb_); free(fq); free(fk); free(o); free(den);
   }
-  for (int h = 0; h < H; ++h) dDelta[h] = 0.0;
-  for (long bh = 0; bh < BH; ++bh) dDelta[bh % H] += part[bh];
-  free(part);
+  long nD = dpm ? (long)H * M : H;
+  for (long i = 0; i < nD; ++i) dDelta[i] = 0.0;
+  for (long bh = 0; bh < BH; ++bh)
+    for (int m = 0; m < M; ++m)
+      dDelta[dpm ? (bh % H) * M + m : bh % H] += part[bh * M + m];
+  if (dA) {
+    for (int m = 0; m < M; ++m) {
+      cd acc = 0.0;
+      for (long bh = 0; bh < BH; ++bh) acc += partA[bh * M + m];
+      st_c(dA + 2 * m, acc);
+    }
+  }
+  free(part); free(partA);
   return err;
 }
 
 /*
- * Tangent (forward-mode) recurrence along (tq, tk, tv, tdelta):
- *   lambda' = A lambda delta',  b' = lambda delta'
+ * Tangent (forward-mode) recurrence along (tq, tk, tv, tdelta, tA):
+ *   lambda' = lambda (A delta' + Delta A'),  b' = lambda delta' + (Delta lambda - b)/A A'
  *   U'_t = lambda U'_{t-1} + lambda' U_{t-1} + b' xi(k_t) + b xi'(k_t) tk_t   (Gamma, eta alike)
  *   a'_t = U'_t xi(q_t) + U_t (xi'(q_t) tq_t)
  *   num' = Re(conj(a') Gamma + conj(a) Gamma'),  den' likewise with eta
@@ -481,9 +521,9 @@ int iao_backward(int B, int H, int N, int d_xi, int d_v, int M,
  */
 int iao_jvp(int B, int H, int N, int d_xi, int d_v, int M,
             const double* q, const double* k, const double* v,
-            const double* delta, const double* A,
+            const double* delta, int dpm, const double* A,
             const double* tq, const double* tk, const double* tv, const double* tdelta,
-            double* to_) {
+            const double* tA, double* to_) {
   if (bad_dims(B, H, N, d_xi, d_v, M) || !q || !k || !v || !delta || !tq || !tk || !tv ||
       !tdelta || !to_)
     return -1;
@@ -502,10 +542,16 @@ int iao_jvp(int B, int H, int N, int d_xi, int d_v, int M,
     cd* ta = malloc(sizeof(cd) * M);
     for (int m = 0; m < M; ++m) {
       cd Am = mode_A(A, m);
-      lam[m] = cexp(delta[h] * Am);
+      double de = delta_hm(delta, dpm, M, h, m), tde = delta_hm(tdelta, dpm, M, h, m);
+      lam[m] = cexp(de * Am);
       bb[m] = (lam[m] - 1.0) / Am;
-      dl[m] = Am * lam[m] * tdelta[h];
-      dbb[m] = lam[m] * tdelta[h];
+      dl[m] = Am * lam[m] * tde;
+      dbb[m] = lam[m] * tde;
+      if (tA) {
+        cd ta = ld_c(tA + 2 * m);
+        dl[m] += de * lam[m] * ta;
+        dbb[m] += (de * lam[m] - bb[m]) / Am * ta;
+      }
     }
     for (int t = 0; t < N; ++t) {
       long rq = (bh * N + t) * (long)d_xi, rv = (bh * N + t) * (long)d_v;

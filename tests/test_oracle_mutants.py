@@ -45,11 +45,11 @@ MUTANTS = [
      "return x > 0.0 ? x + 1.0 : exp(x); }",
      "return x > 0.0 ? x : exp(x); }"),
     ("zero-order hold without 1/A",
-     "st_c(b + 2 * m, (l - 1.0) / a);",
-     "st_c(b + 2 * m, l - 1.0);"),
+     "*bm = (*l - 1.0) / a;",
+     "*bm = *l - 1.0;"),
     ("decay exp(-Delta A)",
-     "cd l = cexp(delta * a);",
-     "cd l = cexp(-delta * a);"),
+     "*l = cexp(delta * a);",
+     "*l = cexp(-delta * a);"),
     ("S4D-Lin frequencies shifted by one",
      "return -0.5 + I * (kPi * (double)m);",
      "return -0.5 + I * (kPi * (double)(m + 1));"),
@@ -61,8 +61,24 @@ MUTANTS = [
      "cd cl = conj(lam[m]);",
      "cd cl = lam[m];"),
     ("dDelta without the b term",
-     "dd += creal(conj(glam[m]) * Am[m] * lam[m] + conj(gb_[m]) * lam[m]);",
-     "dd += creal(conj(glam[m]) * Am[m] * lam[m]);"),
+     "part[bh * M + m] = creal(conj(glam[m]) * Am[m] * lam[m] + conj(gb_[m]) * lam[m]);",
+     "part[bh * M + m] = creal(conj(glam[m]) * Am[m] * lam[m]);"),
+    # trainable A and per-(head, mode) Delta
+    ("per-mode Delta read from the head's first mode",
+     "return dpm ? delta[(long)h * M + m] : delta[h];",
+     "return dpm ? delta[(long)h * M] : delta[h];"),
+    ("dA without the b term",
+     "partA[bh * M + m] = conj(dl * lam[m]) * glam[m] + conj((dl * lam[m] - bb[m]) / Am[m]) * gb_[m];",
+     "partA[bh * M + m] = conj(dl * lam[m]) * glam[m];"),
+    ("dA with dlambda/dA taken as A lambda",
+     "partA[bh * M + m] = conj(dl * lam[m]) * glam[m] + conj((dl * lam[m] - bb[m]) / Am[m]) * gb_[m];",
+     "partA[bh * M + m] = conj(Am[m] * lam[m]) * glam[m] + conj((dl * lam[m] - bb[m]) / Am[m]) * gb_[m];"),
+    ("db/dA without the -b term",
+     "partA[bh * M + m] = conj(dl * lam[m]) * glam[m] + conj((dl * lam[m] - bb[m]) / Am[m]) * gb_[m];",
+     "partA[bh * M + m] = conj(dl * lam[m]) * glam[m] + conj(dl * lam[m] / Am[m]) * gb_[m];"),
+    ("per-mode dDelta summed into the head's first mode",
+     "dDelta[dpm ? (bh % H) * M + m : bh % H] += part[bh * M + m];",
+     "dDelta[dpm ? (bh % H) * M : bh % H] += part[bh * M + m];"),
     ("dk without conj(b)",
      "s += creal(conj(bb[m]) * G[m * d_xi + f]);",
      "s += creal(bb[m] * G[m * d_xi + f]);"),
@@ -95,6 +111,10 @@ PINS = [
     ("p9 tangent/adjoint", P.test_p9_tangent_adjoint_dot_product, {}),
     ("dDelta batch sum", P.test_backward_batch_sum_of_ddelta, {}),
     ("p1 mpmath", P.test_p1_mpmath_brute_force, {}),
+    ("p1 per-mode Delta brute force", P.test_p1_per_mode_delta_brute_force, {}),
+    ("p1 per-mode Delta mpmath", P.test_p1_per_mode_delta_mpmath, {}),
+    ("p8 modes and A", P.test_p8_finite_differences_per_mode_delta_and_A, {}),
+    ("p9 modes and A", P.test_p9_dot_product_per_mode_delta_and_A, {}),
 ]
 
 

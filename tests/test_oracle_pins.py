@@ -52,8 +52,9 @@ def test_p1_brute_force_matches_recurrence(oracle_mod):
     assert rel(r["o"], b["o"]) < 1e-10
 
 
-def _mp_brute(q, k, v, delta, M):
-    """Quadratic form in 40-digit mpmath, one (b,h) slice, zero state."""
+def _mp_brute(q, k, v, delta, M, A=None):
+    """Quadratic form in 40-digit mpmath, one (b,h) slice, zero state.  delta
+    is one step for all modes or one per mode; A defaults to S4D-Lin."""
     import mpmath as mp
     mp.mp.dps = 40
     N, d = q.shape
@@ -65,9 +66,12 @@ def _mp_brute(q, k, v, delta, M):
 
     fq = [[xi(q[t, f]) for f in range(d)] for t in range(N)]
     fk = [[xi(k[t, f]) for f in range(d)] for t in range(N)]
-    A = [mp.mpc(-0.5, mp.pi * m) for m in range(M)]
-    D = mp.mpf(float(delta))
-    lam = [mp.e ** (D * a) for a in A]
+    if A is None:
+        A = [mp.mpc(-0.5, mp.pi * m) for m in range(M)]
+    else:
+        A = [mp.mpc(float(A[2 * m]), float(A[2 * m + 1])) for m in range(M)]
+    D = [mp.mpf(float(x)) for x in np.broadcast_to(np.asarray(delta, dtype=float), (M,))]
+    lam = [mp.e ** (D[m] * A[m]) for m in range(M)]
     bb = [(lam[m] - 1) / A[m] for m in range(M)]
     out = []
     for t in range(N):
@@ -294,3 +298,85 @@ def test_backward_batch_sum_of_ddelta(oracle_mod):
     cat = lambda x: np.concatenate([x, x], axis=0)
     g2 = oracle_mod.backward(cat(q), cat(k), cat(v), delta, cat(dO), M)
     assert rel(g2["dDelta"], 2 * g1["dDelta"]) < 1e-13
+
+
+# ---------------------------------------------------------------- trainable A, Delta per (head, mode)
+def _modes_case(seed, B=1, H=2, N=14, d=3, dv=2, M=4):
+    """Inputs with one Delta per (head, mode) and a general A (decaying modes
+    at other frequencies than S4D-Lin)."""
+    q, k, v, _, _ = small_case(seed=seed, B=B, H=H, N=N, d=d, dv=dv, M=M)
+    rng = np.random.default_rng(seed + 50)
+    delta = 0.02 + 0.1 * rng.random((H, M))
+    A = np.empty(2 * M)
+    A[0::2] = -0.2 - 0.6 * rng.random(M)
+    A[1::2] = np.pi * np.arange(M) + 0.7 * rng.random(M)
+    return q, k, v, delta, A, M
+
+
+def test_p1_per_mode_delta_brute_force(oracle_mod):
+    q, k, v, delta, A, M = _modes_case(31, B=2, H=2, N=33, M=5)
+    r = oracle_mod.forward(q, k, v, delta, M, A=A)
+    b = oracle_mod.brute(q, k, v, delta, M, A=A)
+    assert rel(r["num"], b["num"]) < 1e-12 and rel(r["den"], b["den"]) < 1e-12
+    # one Delta per head is the special case of equal per-mode steps
+    dh = np.array([0.05, 0.11])
+    r1 = oracle_mod.forward(q, k, v, dh, M, A=A)
+    r2 = oracle_mod.forward(q, k, v, np.repeat(dh[:, None], M, axis=1), M, A=A)
+    assert rel(r2["o"], r1["o"]) < 1e-15 and rel(r2["state"], r1["state"]) < 1e-15
+
+
+def test_p1_per_mode_delta_mpmath(oracle_mod):
+    q, k, v, delta, A, M = _modes_case(37, B=1, H=1, N=8, d=2, dv=2, M=3)
+    r = oracle_mod.forward(q, k, v, delta, M, A=A)
+    ref = _mp_brute(q[0, 0], k[0, 0], v[0, 0], delta[0], M, A=A)
+    assert rel(r["o"][0, 0], ref) < 1e-12
+
+
+def test_p8_finite_differences_per_mode_delta_and_A(oracle_mod):
+    q, k, v, delta, A, M = _modes_case(41)
+    H = delta.shape[0]
+    dO = rnd(v.shape, 43)
+    g = oracle_mod.backward(q, k, v, delta, dO, M, A=A)
+    assert g["dDelta"].shape == delta.shape and g["dA"].shape == (2 * M,)
+
+    def loss(d_, A_):
+        return float(np.sum(dO * oracle_mod.forward(q, k, v, d_, M, A=A_)["o"]))
+
+    h = 1e-7
+    for hh in range(H):
+        for m in range(M):
+            dp = delta.copy(); dp[hh, m] += h
+            dm = delta.copy(); dm[hh, m] -= h
+            fd = (loss(dp, A) - loss(dm, A)) / (2 * h)
+            assert abs(fd - g["dDelta"][hh, m]) <= 1e-6 * max(1.0, abs(fd)), (hh, m, fd, g["dDelta"][hh, m])
+    for i in range(2 * M):      # d/dRe A_m and d/dIm A_m
+        ap = A.copy(); ap[i] += h
+        am = A.copy(); am[i] -= h
+        fd = (loss(delta, ap) - loss(delta, am)) / (2 * h)
+        assert abs(fd - g["dA"][i]) <= 1e-6 * max(1.0, abs(fd)), (i, fd, g["dA"][i])
+    # S4D-Lin A as well (the default when A is not given)
+    gl = oracle_mod.backward(q, k, v, delta, dO, M)
+    A0 = np.empty(2 * M); A0[0::2] = -0.5; A0[1::2] = np.pi * np.arange(M)
+    for i in (0, 3):
+        ap = A0.copy(); ap[i] += h
+        am = A0.copy(); am[i] -= h
+        fd = (loss(delta, ap) - loss(delta, am)) / (2 * h)
+        assert abs(fd - gl["dA"][i]) <= 1e-6 * max(1.0, abs(fd)), (i, fd, gl["dA"][i])
+
+
+def test_p9_dot_product_per_mode_delta_and_A(oracle_mod):
+    q, k, v, delta, A, M = _modes_case(47, B=2, H=3, N=70, d=4, dv=3, M=6)   # crosses a checkpoint
+    dO = rnd(v.shape, 48)
+    tq, tk, tv = rnd(q.shape, 49), rnd(k.shape, 50), rnd(v.shape, 51)
+    td, tA = rnd(delta.shape, 52), rnd((2 * M,), 53)
+    to = oracle_mod.jvp(q, k, v, delta, tq, tk, tv, td, M, A=A, tA=tA)
+    g = oracle_mod.backward(q, k, v, delta, dO, M, A=A)
+    lhs = float(np.sum(dO * to))
+    rhs = float(np.sum(g["dq"] * tq) + np.sum(g["dk"] * tk) + np.sum(g["dv"] * tv)
+                + np.sum(g["dDelta"] * td) + np.sum(g["dA"] * tA))
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs)), (lhs, rhs)
+    # per-head Delta: the per-mode gradient summed over modes
+    dh = delta[:, 0].copy()
+    gh = oracle_mod.backward(q, k, v, dh, dO, M, A=A)
+    gm = oracle_mod.backward(q, k, v, np.repeat(dh[:, None], M, axis=1), dO, M, A=A)
+    assert rel(gm["dDelta"].sum(axis=1), gh["dDelta"]) < 1e-12 and rel(gm["dA"], gh["dA"]) < 1e-12
