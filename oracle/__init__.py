@@ -67,9 +67,10 @@ def _load():
         lib.iao_brute.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 4
         lib.iao_backward.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 8
         lib.iao_jvp.argtypes = [i] * 6 + [P] * 4 + [i] + [P] * 7
+        lib.iao_forward_ex.argtypes = [i] * 6 + [P] * 3 + [i, P, i] + [P] * 4 + [ctypes.c_double] + [P] * 6
         lib.iao_num_threads.restype = i
         for name in ("iao_params", "iao_forward", "iao_forward_features", "iao_decode_step",
-                     "iao_brute", "iao_backward", "iao_jvp"):
+                     "iao_brute", "iao_backward", "iao_jvp", "iao_forward_ex"):
             getattr(lib, name).restype = i
         _lib = lib
     return _lib
@@ -222,3 +223,44 @@ def jvp(q, k, v, delta, tq, tk, tv, tdelta, M, A=None, tA=None):
                          _p(tq), _p(tk), _p(tv), _p(tdelta), _p(tA), _p(to))
     _check(rc, "jvp")
     return to
+
+
+def forward_ex(q, k, v, M, delta=None, A=None, delta_t=None, gain=None, bias=None, eps=1e-6, W=None,
+               state_in=None, map_features=True):
+    """The layer with its optional parts (see iao_forward_ex): RMSNorm gain and
+    bias [H, d_xi+d_v] on the SSM input, a step per token delta_t [B,H,N], a
+    complex readout matrix W [H,M,M] (complex array or [H,M,M,2] reals).
+    Returns dict(o, num, den, state)."""
+    q, k, v, delta, A, delta_t, gain, bias, state_in = map(
+        _f64, (q, k, v, delta, A, delta_t, gain, bias, state_in))
+    if W is not None:
+        W = np.asarray(W)
+        W = np.ascontiguousarray(W.astype(np.complex128) if np.iscomplexobj(W) else
+                                 W.reshape(W.shape[:-1] + (2,)).astype(np.float64).view(np.complex128)[..., 0])
+        W = W.view(np.float64)
+    B, H, N, d_xi = q.shape
+    d_v = v.shape[-1]
+    o = np.zeros((B, H, N, d_v))
+    num = np.zeros((B, H, N, d_v))
+    den = np.zeros((B, H, N))
+    st = np.zeros(state_len(B, H, M, d_xi, d_v))
+    dpm = 0 if delta is None else _dpm(delta)
+    rc = _load().iao_forward_ex(B, H, N, d_xi, d_v, M, _p(q), _p(k), _p(v), 1 if map_features else 0,
+                                _p(delta), dpm, _p(A), _p(delta_t), _p(gain), _p(bias), float(eps), _p(W),
+                                _p(state_in), _p(o), _p(num), _p(den), _p(st))
+    _check(rc, "forward_ex")
+    return {"o": o, "num": num, "den": den, "state": st}
+
+
+def forward_bidirectional(q, k, v, M, **kw):
+    """The bidirectional layer (summary sec. 5.2: Caduceus-IA keeps Caduceus'
+    bidirectional handling): the causal layer on the sequence plus the causal
+    layer on the time-reversed sequence, reversed back: o = f(x) + flip(f(flip x)).
+    Per-token arrays in kw (delta_t) are reversed with the inputs."""
+    fwd = forward_ex(q, k, v, M, **kw)["o"]
+    flip = lambda x: None if x is None else np.ascontiguousarray(np.flip(_f64(x), axis=2))
+    kw_r = dict(kw)
+    if kw.get("delta_t") is not None:
+        kw_r["delta_t"] = flip(kw["delta_t"])
+    rev = forward_ex(flip(q), flip(k), flip(v), M, **kw_r)["o"]
+    return fwd + np.flip(rev, axis=2)

@@ -262,6 +262,120 @@ int iao_decode_step(int B, int H, int d_xi, int d_v, int M,
 }
 
 /*
+ * Extended layer forward: the optional parts of the layer, each off when its
+ * argument is NULL (with all of them off this is iao_forward).
+ *
+ *   Input stabilisation (AI-radio page, "Implementation Details": the SSM
+ *   input z_t = (xi(k_t), v_t) passes an RMSNorm with a learnable per-head
+ *   bias before the SSM): with gain or bias given,
+ *       z_t <- z_t / sqrt(mean_f z_t[f]^2 + eps) * gain_h + bias_h,
+ *   over the d_xi + d_v entries of z_t; gain, bias [H, d_xi + d_v] (NULL gain
+ *   = 1, NULL bias = 0).  The query features are not normalised.
+ *
+ *   Selective writing and memory decay (summary sec. 3.3 and sec. 5.3): with
+ *   delta_t [B,H,N] given, token t of sequence (b,h) uses its own step,
+ *   lambda_t = exp(delta_t A), b_t = (lambda_t - 1)/A, for all modes: a small
+ *   step writes little and forgets little.
+ *
+ *   Full complex readout matrix (summary sec. A.3, and the M^2 term of the
+ *   decode cost in sec. 3.2): with W [H,M,M] complex given (W[h][m][m'],
+ *   row m, column m'), the query's mode coefficients are mixed before the
+ *   readout: a~_t = W_h a_t, num_t = Re(a~_t^H Gamma_t), den_t = Re(a~_t^H eta_t).
+ *
+ * map_features = 0 takes q and k as already-mapped features (xi is then
+ * skipped), which lets a pin scale the SSM input directly.
+ */
+int iao_forward_ex(int B, int H, int N, int d_xi, int d_v, int M,
+                   const double* q, const double* k, const double* v, int map_features,
+                   const double* delta, int dpm, const double* A, const double* delta_t,
+                   const double* gain, const double* bias, double eps, const double* W,
+                   const double* state_in, double* o, double* num, double* den,
+                   double* state_out) {
+  if (bad_dims(B, H, N, d_xi, d_v, M) || !q || !k || !v || !o || (!delta && !delta_t)) return -1;
+  long BH = (long)B * H;
+  int D = d_xi + d_v;
+  int norm = gain || bias;
+  int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long bh = 0; bh < BH; ++bh) {
+    int h = (int)(bh % H);
+    cd* Am = malloc(sizeof(cd) * M);
+    cd* lam = malloc(sizeof(cd) * M);
+    cd* bb = malloc(sizeof(cd) * M);
+    cd* U = malloc(sizeof(cd) * (size_t)M * d_xi);
+    cd* G = malloc(sizeof(cd) * (size_t)M * d_v);
+    cd* eta = malloc(sizeof(cd) * M);
+    cd* a = malloc(sizeof(cd) * M);
+    cd* at = malloc(sizeof(cd) * M);
+    double* z = malloc(sizeof(double) * (size_t)D);
+    double* fq = malloc(sizeof(double) * (size_t)d_xi);
+    if (!Am || !lam || !bb || !U || !G || !eta || !a || !at || !z || !fq) {
+#pragma omp atomic write
+      err = -2;
+    } else {
+      for (int m = 0; m < M; ++m) {
+        Am[m] = mode_A(A, m);
+        if (!delta_t) zoh(delta_hm(delta, dpm, M, h, m), Am[m], &lam[m], &bb[m]);
+      }
+      load_state(state_in, B, H, M, d_xi, d_v, (int)bh, U, G, eta);
+      for (int t = 0; t < N; ++t) {
+        long rq = (bh * N + t) * (long)d_xi, rv = (bh * N + t) * (long)d_v;
+        /* the SSM input z_t = (xi(k_t), v_t), normalised if asked */
+        for (int f = 0; f < d_xi; ++f) {
+          z[f] = map_features ? feat(k[rq + f]) : k[rq + f];
+          fq[f] = map_features ? feat(q[rq + f]) : q[rq + f];
+        }
+        for (int f = 0; f < d_v; ++f) z[d_xi + f] = v[rv + f];
+        if (norm) {
+          double ss = 0.0;
+          for (int f = 0; f < D; ++f) ss += z[f] * z[f];
+          double r = 1.0 / sqrt(ss / (double)D + eps);
+          for (int f = 0; f < D; ++f) {
+            double g = gain ? gain[(long)h * D + f] : 1.0;
+            double c = bias ? bias[(long)h * D + f] : 0.0;
+            z[f] = z[f] * r * g + c;
+          }
+        }
+        /* this token's step */
+        if (delta_t)
+          for (int m = 0; m < M; ++m) zoh(delta_t[bh * N + t], Am[m], &lam[m], &bb[m]);
+        /* recurrence, then the query's mode coefficients */
+        for (int m = 0; m < M; ++m) {
+          cd am = 0.0;
+          for (int f = 0; f < d_xi; ++f) {
+            U[(long)m * d_xi + f] = lam[m] * U[(long)m * d_xi + f] + bb[m] * z[f];
+            am += U[(long)m * d_xi + f] * fq[f];
+          }
+          for (int f = 0; f < d_v; ++f)
+            G[(long)m * d_v + f] = lam[m] * G[(long)m * d_v + f] + bb[m] * z[d_xi + f];
+          eta[m] = lam[m] * eta[m] + bb[m];
+          a[m] = am;
+        }
+        /* readout matrix */
+        for (int m = 0; m < M; ++m) {
+          if (!W) { at[m] = a[m]; continue; }
+          cd acc = 0.0;
+          for (int mp = 0; mp < M; ++mp) acc += ld_c(W + 2 * (((long)h * M + m) * M + mp)) * a[mp];
+          at[m] = acc;
+        }
+        double dn = 0.0;
+        for (int m = 0; m < M; ++m) dn += creal(conj(at[m]) * eta[m]);
+        for (int f = 0; f < d_v; ++f) {
+          double nf = 0.0;
+          for (int m = 0; m < M; ++m) nf += creal(conj(at[m]) * G[(long)m * d_v + f]);
+          if (num) num[rv + f] = nf;
+          o[rv + f] = nf / dn;
+        }
+        if (den) den[bh * N + t] = dn;
+      }
+      if (state_out) store_state(state_out, B, H, M, d_xi, d_v, (int)bh, U, G, eta);
+    }
+    free(Am); free(lam); free(bb); free(U); free(G); free(eta); free(a); free(at); free(z); free(fq);
+  }
+  return err;
+}
+
+/*
  * Brute force from a zero state.  Unrolling the recurrence gives
  *   a_tm  = b_m sum_{n<=t} lambda_m^(t-n) s_tn,     s_tn = xi(q_t).xi(k_n)
  *   w_tn  = Re sum_m conj(a_tm) b_m lambda_m^(t-n)

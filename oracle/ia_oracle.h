@@ -91,6 +91,19 @@ int iao_jvp(int B, int H, int N, int d_xi, int d_v, int M,
             const double* tq, const double* tk, const double* tv, const double* tdelta,
             const double* tA, double* to_);
 
+/* Extended forward: the layer with its optional parts, each off when its
+ * argument is NULL (all off = iao_forward): RMSNorm with per-head gain and
+ * bias [H, d_xi+d_v] on the SSM input (xi(k_t), v_t); a step per token
+ * delta_t [B,H,N] (selective writing and memory decay; delta then unused);
+ * a complex readout matrix W [H,M,M] mixing the query's mode coefficients.
+ * map_features = 0 takes q, k as already-mapped features. */
+int iao_forward_ex(int B, int H, int N, int d_xi, int d_v, int M,
+                   const double* q, const double* k, const double* v, int map_features,
+                   const double* delta, int dpm, const double* A, const double* delta_t,
+                   const double* gain, const double* bias, double eps, const double* W,
+                   const double* state_in, double* o, double* num, double* den,
+                   double* state_out);
+
 /* Threads the OpenMP loops will use (for reporting). */
 int iao_num_threads(void);
 

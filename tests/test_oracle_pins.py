@@ -380,3 +380,152 @@ def test_p9_dot_product_per_mode_delta_and_A(oracle_mod):
     gh = oracle_mod.backward(q, k, v, dh, dO, M, A=A)
     gm = oracle_mod.backward(q, k, v, np.repeat(dh[:, None], M, axis=1), dO, M, A=A)
     assert rel(gm["dDelta"].sum(axis=1), gh["dDelta"]) < 1e-12 and rel(gm["dA"], gh["dA"]) < 1e-12
+
+
+# ---------------------------------------------------------------- optional parts of the layer
+def test_extended_forward_with_everything_off_is_the_layer(oracle_mod):
+    q, k, v, delta, M = small_case(seed=60, N=45, M=6)
+    a = oracle_mod.forward(q, k, v, delta, M)
+    b = oracle_mod.forward_ex(q, k, v, M, delta=delta)
+    assert rel(b["o"], a["o"]) < 1e-15 and rel(b["state"], a["state"]) < 1e-15
+
+
+def _mp_brute_ex(q, k, v, M, steps, W=None):
+    """Quadratic form in 40-digit mpmath for one (b,h) slice with one step per
+    token (steps [N]) and an optional readout matrix W [M,M] complex:
+        a_t[m]  = sum_{n<=t} b_n[m] exp(A_m sum_{s=n+1..t} Delta_s) s_tn
+        a~_t    = W a_t
+        w_tn    = Re sum_m conj(a~_t[m]) b_n[m] exp(A_m sum_{s=n+1..t} Delta_s)
+        o_t     = sum_n w_tn v_n / sum_n w_tn."""
+    import mpmath as mp
+    mp.mp.dps = 40
+    N, d = q.shape
+    dv = v.shape[1]
+
+    def xi(x):
+        x = mp.mpf(float(x))
+        return x + 1 if x > 0 else mp.e ** x
+
+    fq = [[xi(q[t, f]) for f in range(d)] for t in range(N)]
+    fk = [[xi(k[t, f]) for f in range(d)] for t in range(N)]
+    A = [mp.mpc(-0.5, mp.pi * m) for m in range(M)]
+    D = [mp.mpf(float(x)) for x in steps]
+    cum = [mp.mpf(0)]
+    for x in D:
+        cum.append(cum[-1] + x)        # cum[t+1] = sum_{s<=t} Delta_s
+    bn = [[(mp.e ** (D[n] * A[m]) - 1) / A[m] for m in range(M)] for n in range(N)]
+    Wm = None if W is None else [[mp.mpc(float(W[i, j].real), float(W[i, j].imag)) for j in range(M)]
+                                 for i in range(M)]
+    out = []
+    for t in range(N):
+        s = [sum(fq[t][f] * fk[n][f] for f in range(d)) for n in range(t + 1)]
+        dec = [[mp.e ** (A[m] * (cum[t + 1] - cum[n + 1])) for m in range(M)] for n in range(t + 1)]
+        a = [sum(bn[n][m] * dec[n][m] * s[n] for n in range(t + 1)) for m in range(M)]
+        at = a if Wm is None else [sum(Wm[i][j] * a[j] for j in range(M)) for i in range(M)]
+        w = [sum((mp.conj(at[m]) * bn[n][m] * dec[n][m]).real for m in range(M)) for n in range(t + 1)]
+        den = sum(w)
+        out.append([float(sum(w[n] * v[n, j] for n in range(t + 1)) / den) for j in range(dv)])
+    return np.array(out)
+
+
+def test_selective_steps_mpmath(oracle_mod):
+    q, k, v, _, M = small_case(seed=61, B=1, H=1, N=8, d=2, dv=2, M=3)
+    steps = 0.01 + 0.3 * np.random.default_rng(62).random((1, 1, 8))
+    r = oracle_mod.forward_ex(q, k, v, M, delta_t=steps)
+    ref = _mp_brute_ex(q[0, 0], k[0, 0], v[0, 0], M, steps[0, 0])
+    assert rel(r["o"][0, 0], ref) < 1e-12
+
+
+def test_selective_constant_steps_reduce_to_per_head_delta(oracle_mod):
+    q, k, v, delta, M = small_case(seed=63, N=40, M=5)
+    B, H, N = q.shape[:3]
+    steps = np.broadcast_to(delta[None, :, None], (B, H, N)).copy()
+    a = oracle_mod.forward(q, k, v, delta, M)
+    b = oracle_mod.forward_ex(q, k, v, M, delta_t=steps)
+    assert rel(b["o"], a["o"]) < 1e-14 and rel(b["state"], a["state"]) < 1e-13
+
+
+def test_selective_zero_step_skips_the_token(oracle_mod):
+    # A token whose step goes to zero writes nothing (b -> 0) and leaves the
+    # memory where it was (lambda -> 1): the other tokens' outputs match the
+    # sequence with that token removed.
+    q, k, v, _, M = small_case(seed=64, B=1, H=2, N=30, M=4)
+    rng = np.random.default_rng(65)
+    steps = 0.02 + 0.08 * rng.random((1, 2, 30))
+    t0 = 12
+    steps_gate = steps.copy()
+    steps_gate[:, :, t0] = 1e-13
+    r = oracle_mod.forward_ex(q, k, v, M, delta_t=steps_gate)
+    drop = lambda x: np.delete(x, t0, axis=2)
+    s = oracle_mod.forward_ex(drop(q), drop(k), drop(v), M, delta_t=drop(steps))
+    # tokens before t0 are untouched; after t0 the skipped token's write is ~1e-13
+    assert rel(np.delete(r["o"], t0, axis=2), s["o"]) < 1e-9
+
+
+def test_readout_matrix_mpmath_and_identity(oracle_mod):
+    q, k, v, _, M = small_case(seed=66, B=1, H=1, N=7, d=2, dv=2, M=3)
+    rng = np.random.default_rng(67)
+    W = rng.standard_normal((1, M, M)) + 1j * rng.standard_normal((1, M, M))
+    delta = np.array([0.2])
+    r = oracle_mod.forward_ex(q, k, v, M, delta=delta, W=W)
+    ref = _mp_brute_ex(q[0, 0], k[0, 0], v[0, 0], M, np.full(7, 0.2), W=W[0])
+    assert rel(r["o"][0, 0], ref) < 1e-11
+    # the identity matrix is the plain readout
+    q, k, v, delta, M = small_case(seed=68, N=30, M=5)
+    eye = np.broadcast_to(np.eye(M, dtype=complex), (2, M, M)).copy()
+    a = oracle_mod.forward(q, k, v, delta, M)
+    b = oracle_mod.forward_ex(q, k, v, M, delta=delta, W=eye)
+    assert rel(b["num"], a["num"]) < 1e-14 and rel(b["den"], a["den"]) < 1e-14
+
+
+def test_readout_matrix_linear_and_scale_free(oracle_mod):
+    q, k, v, delta, M = small_case(seed=69, N=33, M=4)
+    rng = np.random.default_rng(70)
+    W1 = rng.standard_normal((2, M, M)) + 1j * rng.standard_normal((2, M, M))
+    W2 = rng.standard_normal((2, M, M)) + 1j * rng.standard_normal((2, M, M))
+    f = lambda W: oracle_mod.forward_ex(q, k, v, M, delta=delta, W=W)
+    r1, r2, r12 = f(W1), f(W2), f(W1 + W2)
+    assert rel(r12["num"], r1["num"] + r2["num"]) < 1e-12 and rel(r12["den"], r1["den"] + r2["den"]) < 1e-12
+    r3 = f(-2.5 * W1)                      # a real scale multiplies num and den alike
+    assert rel(r3["num"], -2.5 * r1["num"]) < 1e-13 and rel(r3["o"], r1["o"]) < 1e-12
+
+
+def test_input_norm_bias_alone_gives_the_bias(oracle_mod):
+    # gain 0: the SSM input is the constant bias (beta_k, beta_v), so
+    # Gamma_t = eta_t beta_v^T and num_t = den_t beta_v: o_t = beta_v for every t
+    q, k, v, delta, M = small_case(seed=71, N=25, M=5)
+    H, dx, dv = q.shape[1], q.shape[-1], v.shape[-1]
+    bias = np.random.default_rng(72).standard_normal((H, dx + dv))
+    r = oracle_mod.forward_ex(q, k, v, M, delta=delta, gain=np.zeros((H, dx + dv)), bias=bias)
+    expect = np.broadcast_to(bias[None, :, None, dx:], r["o"].shape)
+    assert rel(r["o"], expect) < 1e-12
+
+
+def test_input_norm_is_scale_free(oracle_mod):
+    # without bias, RMSNorm removes any positive per-token scale of the SSM
+    # input (features given directly so that both halves scale together);
+    # eps is negligible against the inputs' size
+    q, k, v, delta, M = small_case(seed=73, N=28, M=4)
+    fq, fk = feat(q), feat(k)
+    H, dx, dv = q.shape[1], q.shape[-1], v.shape[-1]
+    gain = 0.5 + np.random.default_rng(74).random((H, dx + dv))
+    c = np.exp(np.random.default_rng(75).standard_normal(q.shape[:3] + (1,)))
+    f = lambda kk, vv: oracle_mod.forward_ex(fq, kk, vv, M, delta=delta, gain=gain, eps=1e-30,
+                                             map_features=False)["o"]
+    assert rel(f(fk * c, v * c), f(fk, v)) < 1e-12
+    # and it is not the identity: without the norm the scale matters
+    plain = lambda kk, vv: oracle_mod.forward_ex(fq, kk, vv, M, delta=delta, map_features=False)["o"]
+    assert rel(plain(fk * c, v * c), plain(fk, v)) > 1e-3
+
+
+def test_bidirectional_time_reversal_and_first_token(oracle_mod):
+    q, k, v, delta, M = small_case(seed=76, N=21, M=4)
+    rng = np.random.default_rng(77)
+    steps = 0.01 + 0.1 * rng.random(q.shape[:3])
+    flip = lambda x: np.flip(x, axis=2).copy()
+    o = oracle_mod.forward_bidirectional(q, k, v, M, delta_t=steps)
+    o_r = oracle_mod.forward_bidirectional(flip(q), flip(k), flip(v), M, delta_t=flip(steps))
+    assert rel(flip(o_r), o) < 1e-14
+    # one token: each direction returns v (P3), so the sum is 2 v
+    o1 = oracle_mod.forward_bidirectional(q[:, :, :1], k[:, :, :1], v[:, :, :1], M, delta=delta)
+    assert rel(o1, 2 * v[:, :, :1]) < 1e-14
