@@ -492,6 +492,46 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
     return out
 
 
+def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world):
+    """The layer's optional parts (RMSNorm on the SSM input, a step per token,
+    the complex readout matrix, the bidirectional layer) through
+    ia_prefill_fwd_ex on the same workload: the token-serial CUDA-core kernel,
+    one CTA per (b,h).  Each part is timed alone and all together."""
+    import torch
+    import ssm_token_mixer_b200 as ia
+    from ssm_token_mixer_b200 import synthetic
+    inp = synthetic.workload_inputs(w)
+    q, k, v, delta = (inp[n].to(dev) for n in ("q", "k", "v", "delta"))
+    g = torch.Generator().manual_seed(w.seed + 500)
+    D = w.d_xi + w.d_v
+    parts = {
+        "selective": {"delta_t": torch.exp(math.log(5e-3) + torch.rand(w.B, w.H, w.N, generator=g) *
+                                           (math.log(1e-1) - math.log(5e-3))).to(dev)},
+        "norm": {"gain": (0.5 + torch.rand(w.H, D, generator=g)).to(dev),
+                 "bias": (0.3 * torch.randn(w.H, D, generator=g)).to(dev)},
+        "readout": {"W": (torch.randn(w.H, w.M, w.M, 2, generator=g) / math.sqrt(w.M)).to(dev)},
+        "bidirectional": {"bidirectional": True},
+    }
+    parts["all"] = {**parts["selective"], **parts["norm"], **parts["readout"]}
+    tokens = w.B * w.N
+    by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
+    out = {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
+           "unit": "tokens/s", "kernel": "token-serial CUDA-core layer (ia_prefill_fwd_ex)", "parts": {}}
+    for name, kw in parts.items():
+        d = None if "delta_t" in kw else delta
+        fn = lambda: ia.prefill_fwd_ex(q, k, v, w.M, delta=d, **kw)
+        barrier(dev)
+        step_ms, kern_ms = timer.run(fn, steps, warmup)
+        barrier(dev)
+        total = max_over_ranks(sum(step_ms), dev)
+        passes = 2 if kw.get("bidirectional") else 1
+        rf = roofline(by * passes, flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H * passes, kern_ms, peaks,
+                      peak_kind, None, sustained=False)
+        out["parts"][name] = {"value": world * tokens * steps / (total * 1e-3), "ms_per_step": total / steps,
+                              "roofline": rf, "gpu_launches": passes * steps}
+    return out
+
+
 def workload_config(w, scaling="weak"):
     """The JSON line's config: the workload and how it is timed (both arms)."""
     return {"workload": f"{w.name} prefill (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, "
@@ -542,7 +582,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--legs", default="prefill,prefill_1p3b,fwd_bwd,decode,prefill_long",
+    ap.add_argument("--legs", default="prefill,prefill_1p3b,fwd_bwd,decode,prefill_long,optional_parts",
                     help="comma list of legs to run (prefill is the headline)")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--workload", default="prefill_125m", help="headline prefill workload")
@@ -612,6 +652,11 @@ def main():
                                  peak_kind, rank, world)
             line["prefill_long"] = r
             extra_launches += r["gpu_launches"]
+        if "optional_parts" in legs:
+            r = leg_optional_parts(dev, WORKLOADS["prefill_125m"], min(args.steps, 3), 3, timer, peaks,
+                                   peak_kind, rank, world)
+            line["optional_parts"] = r
+            extra_launches += sum(p["gpu_launches"] for p in r["parts"].values())
         line["gpu_launches_all_legs"] = line.get("gpu_launches", 0) + extra_launches + sum(
             b["gpu_launches"] for b in line.get("decode", {}).get("batches", {}).values())
     finally:

@@ -23,9 +23,11 @@
  *     comes from a caller-provided workspace sized by the *_workspace_bytes
  *     queries.  Tensor pointers must be 16-byte aligned.
  *   - q, k: [B,H,N,d_xi]; v: [B,H,N,d_v]; o, num: [B,H,N,d_v] fp32;
- *     den: [B,H,N] fp32; delta: [H] fp32 (> 0); A: [M] complex fp32 stored as
- *     (re, im) pairs, or NULL for S4D-Lin.  The input dtype (IA_F32 or
- *     IA_BF16) applies to q, k, v and dO; all outputs are fp32.
+ *     den: [B,H,N] fp32; delta: [H] fp32 (> 0), or [H,M] when
+ *     shape->delta_per_mode = 1 (lambda_hm = exp(Delta_hm A_m)); A: [M]
+ *     complex fp32 stored as (re, im) pairs, shared by all heads, or NULL
+ *     for S4D-Lin.  The input dtype (IA_F32 or IA_BF16) applies to q, k, v
+ *     and dO; all outputs are fp32.
  *   - State: one buffer of ia_state_bytes() bytes, complex fp32 stored as
  *     (re, im): U [B,H,M,d_xi] | Gamma [B,H,M,d_v] | eta [B,H,M].
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -85,6 +87,9 @@ typedef struct {
   int d_xi, d_v;     /* feature width of q/k, value width */
   int M;             /* complex S4D modes */
   ia_dtype_t in_dtype;
+  int delta_per_mode;   /* 0: delta [H], one step per head (S4D-Lin init, paper's
+                           default); 1: delta [H,M], one step per head and mode.
+                           Zero when the struct is aggregate-initialised without it. */
 } ia_shape_t;
 
 /* Bytes of one state buffer: 8 * B * H * M * (d_xi + d_v + 1). */
@@ -108,10 +113,19 @@ IA_API ia_path_t ia_prefill_path(const ia_shape_t* shape);
  * included, runs the token-serial CUDA-core adjoint. */
 IA_API ia_path_t ia_fwd_bwd_path(const ia_shape_t* shape);
 
-/* Number of kernel launches one ia_prefill_fwd call makes for this shape
- * (the tensor-core path adds a state-only pass and a carry scan when it
- * splits sequences into segments); 0 for an invalid shape. */
+/* Number of kernel launches one ia_prefill_fwd call makes for this shape:
+ * 2 on the tensor-core path (per-head tables, then the chunk pass), 1 on
+ * the sequential path; 0 for an invalid shape. */
 IA_API int ia_prefill_launches(const ia_shape_t* shape);
+
+/* CTAs of the tensor-core chunk pass for this shape (0 off that path).  The
+ * pass cuts the value columns into blocks of 64 (a "stream" is one (b,h) and
+ * value block) and gives every CTA an equal contiguous range of the
+ * (stream, chunk) space, at most one CTA per SM.  A range that starts inside
+ * a stream takes its carried state from its predecessors (see
+ * ia_prefill_fwd); the workspace then also holds two states per CTA.
+ * IA_PREFILL_GRID=n forces n CTAs (tuning and tests). */
+IA_API int ia_prefill_grid(const ia_shape_t* shape);
 
 /*
  * Causal prefill over N tokens (paperlayer.ai summary sec. 3.2 and sec. A.2:
@@ -159,14 +173,18 @@ IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* shape, const void* q,
 
 /*
  * Training step of the layer from a zero state (paperlayer.ai summary
- * sec. A.3 and App. G: bf16 mixed-precision training).  Given the upstream
- * gradient dO [B,H,N,d_v] (input dtype), writes o, and the gradients
- * dq, dk [B,H,N,d_xi], dv [B,H,N,d_v] (fp32) and dDelta [H] (fp32, summed
- * over batch and time; overwritten).
+ * sec. A.3 and App. G: bf16 mixed-precision training; sec. 3.2: the S4D
+ * recurrence, whose A and step Delta train with the model).  Given the
+ * upstream gradient dO [B,H,N,d_v] (input dtype), writes o, the gradients
+ * dq, dk [B,H,N,d_xi], dv [B,H,N,d_v] (fp32), dDelta (fp32, delta's shape:
+ * [H] or [H,M]; summed over batch and time) and, when dA is not NULL, dA [M]
+ * complex as (dL/dRe A_m, dL/dIm A_m) fp32 pairs, summed over batch, heads
+ * and time (A itself may still be NULL = S4D-Lin).  dDelta and dA are
+ * overwritten, reduced in a fixed order (bitwise reproducible run to run).
  */
 IA_API ia_status_t ia_fwd_bwd(const ia_shape_t* shape, const void* q, const void* k, const void* v,
                        const float* delta, const float* A, const void* dO, float* o,
-                       float* dq, float* dk, float* dv, float* dDelta, void* workspace,
+                       float* dq, float* dk, float* dv, float* dDelta, float* dA, void* workspace,
                        size_t workspace_bytes, void* stream);
 
 /*
@@ -180,6 +198,60 @@ IA_API ia_status_t ia_fwd_bwd(const ia_shape_t* shape, const void* q, const void
 IA_API ia_status_t ia_decode_step(const ia_shape_t* shape, const void* q, const void* k,
                            const void* v, const float* delta, const float* A, void* state,
                            float* o, float* num, float* den, void* stream);
+
+/*
+ * Optional parts of the layer that the pages name beside the plain readout.
+ * Every pointer is a caller-owned device array; NULL (or 0) leaves that part
+ * out, so an all-zero ia_options_t is the plain layer.
+ *   delta_t [B,H,N] fp32 (> 0): selective writing and memory decay
+ *       (paperlayer.ai summary sec. 3.3 and sec. 5.3): token t uses its own
+ *       step, lambda_t = exp(delta_t A), b_t = (lambda_t - 1)/A, for every
+ *       mode; a small step writes little and forgets little.  `delta` is then
+ *       not read (it may be NULL).  For a decode step: [B,H].
+ *   gain, bias [H, d_xi + d_v] fp32: input stabilisation (AI-radio page,
+ *       "Implementation Details"): the SSM input z_t = (xi(k_t), v_t) passes
+ *       an RMSNorm over its d_xi + d_v entries with a per-head gain and bias,
+ *       z <- z / sqrt(mean(z^2) + eps) * gain_h + bias_h, before the
+ *       recurrence (NULL gain = 1, NULL bias = 0; the norm is on when either
+ *       is given).  The query features are not normalised.
+ *   eps: the RMSNorm epsilon (>= 0).
+ *   W [H,M,M] complex fp32 ((re, im) pairs; W[h][m][m'] row m, column m'):
+ *       the full complex readout matrix (summary sec. A.3; the M^2 term of
+ *       the decode cost, sec. 3.2): a~_t = W_h a_t replaces a_t in
+ *       num = Re(a~^H Gamma) and den = Re(a~^H eta).
+ *   bidirectional: 1 for the bidirectional layer of the genomics models
+ *       (summary sec. 5.2: Caduceus-IA keeps Caduceus' bidirectional
+ *       handling): o = f(x) + flip(f(flip x)), f the causal layer, flip the
+ *       time reversal.  Prefill only, with no state_in, state_out, num, den.
+ */
+typedef struct {
+  const float* delta_t;
+  const float* gain;
+  const float* bias;
+  float eps;
+  const float* W;
+  int bidirectional;
+} ia_options_t;
+
+/*
+ * ia_prefill_fwd with the optional parts (NULL opt = the plain layer).
+ * Runs the token-serial fp32 CUDA-core kernel (one CTA per (b,h), any input
+ * dtype; the tensor-core chunk pass does not take these options), so it is
+ * correct for every shape whose state fits in shared memory but slower than
+ * ia_prefill_fwd.  Needs no workspace.
+ */
+IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* shape, const ia_options_t* opt, const void* q,
+                                     const void* k, const void* v, const float* delta, const float* A,
+                                     const void* state_in, float* o, float* num, float* den,
+                                     void* state_out, void* stream);
+
+/*
+ * ia_decode_step with the optional parts (bidirectional excluded: that layer
+ * is not causal).  delta_t, if given, is [B,H]: this token's step.
+ */
+IA_API ia_status_t ia_decode_step_ex(const ia_shape_t* shape, const ia_options_t* opt, const void* q,
+                                     const void* k, const void* v, const float* delta, const float* A,
+                                     void* state, float* o, float* num, float* den, void* stream);
 
 /*
  * Profiling aid (no counterpart in the paper): registers two caller-owned
@@ -213,6 +285,12 @@ IA_API ia_status_t ia_check_device_errors(void* stream);
  */
 IA_API ia_status_t ia_selftest_wait_expiry(unsigned long long limit_ns, unsigned long long* out,
                                            void* stream);
+
+/* The CUDA error (a cudaError_t value; 0 if none) behind the last
+ * IA_ERR_CUDA that an entry point returned on the calling thread, and its
+ * description.  A diagnostic with no counterpart in the paper. */
+IA_API int ia_last_cuda_error(void);
+IA_API const char* ia_last_cuda_error_string(void);
 
 /* Static description of a status code. */
 IA_API const char* ia_status_string(ia_status_t status);

@@ -20,7 +20,8 @@ import torch
 
 __all__ = ["IAError", "load_library", "state_bytes", "prefill_workspace_bytes",
            "fwd_bwd_workspace_bytes", "prefill_path", "fwd_bwd_path", "prefill_static_max_heads",
-           "prefill_fwd", "prefill_fwd_static", "fwd_bwd", "decode_step", "check_device_errors",
+           "prefill_fwd", "prefill_fwd_static", "prefill_fwd_ex", "fwd_bwd", "decode_step",
+           "decode_step_ex", "check_device_errors",
            "selftest_wait_expiry", "set_launch_events", "library_path", "IA_F32", "IA_BF16"]
 
 IA_F32, IA_BF16 = 0, 1
@@ -37,13 +38,20 @@ class IAError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
         msg = _lib.ia_status_string(status).decode() if _lib else STATUS.get(status, str(status))
+        if _lib and status == 4:   # IA_ERR_CUDA: name the CUDA error behind it
+            msg += f" ({_lib.ia_last_cuda_error_string().decode()}, code {_lib.ia_last_cuda_error()})"
         super().__init__(f"{where}: {msg}")
 
 
 class IAShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
                 ("d_xi", ctypes.c_int), ("d_v", ctypes.c_int), ("M", ctypes.c_int),
-                ("in_dtype", ctypes.c_int)]
+                ("in_dtype", ctypes.c_int), ("delta_per_mode", ctypes.c_int)]
+
+
+class IAOptions(ctypes.Structure):
+    _fields_ = [("delta_t", ctypes.c_void_p), ("gain", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("eps", ctypes.c_float), ("W", ctypes.c_void_p), ("bidirectional", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -63,7 +71,7 @@ def load_library():
     for name in ("ia_state_bytes", "ia_prefill_workspace_bytes", "ia_fwd_bwd_workspace_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [S]
-    for name in ("ia_prefill_launches", "ia_prefill_path", "ia_fwd_bwd_path"):
+    for name in ("ia_prefill_launches", "ia_prefill_grid", "ia_prefill_path", "ia_fwd_bwd_path"):
         getattr(lib, name).restype = ctypes.c_int
         getattr(lib, name).argtypes = [S]
     lib.ia_prefill_static_max_heads.restype = ctypes.c_int
@@ -75,15 +83,24 @@ def load_library():
     lib.ia_prefill_fwd_static.restype = ctypes.c_int
     lib.ia_prefill_fwd_static.argtypes = [S] + [P] * 10 + [P]
     lib.ia_fwd_bwd.restype = ctypes.c_int
-    lib.ia_fwd_bwd.argtypes = [S] + [P] * 11 + [P, ctypes.c_size_t, P]
+    lib.ia_fwd_bwd.argtypes = [S] + [P] * 12 + [P, ctypes.c_size_t, P]
     lib.ia_decode_step.restype = ctypes.c_int
     lib.ia_decode_step.argtypes = [S] + [P] * 9 + [P]
+    O = ctypes.POINTER(IAOptions)
+    lib.ia_prefill_fwd_ex.restype = ctypes.c_int
+    lib.ia_prefill_fwd_ex.argtypes = [S, O] + [P] * 10 + [P]
+    lib.ia_decode_step_ex.restype = ctypes.c_int
+    lib.ia_decode_step_ex.argtypes = [S, O] + [P] * 9 + [P]
     lib.ia_set_launch_events.restype = ctypes.c_int
     lib.ia_set_launch_events.argtypes = [P, P]
     lib.ia_check_device_errors.restype = ctypes.c_int
     lib.ia_check_device_errors.argtypes = [P]
     lib.ia_status_string.restype = ctypes.c_char_p
     lib.ia_status_string.argtypes = [ctypes.c_int]
+    lib.ia_last_cuda_error.restype = ctypes.c_int
+    lib.ia_last_cuda_error.argtypes = []
+    lib.ia_last_cuda_error_string.restype = ctypes.c_char_p
+    lib.ia_last_cuda_error_string.argtypes = []
     _lib = lib
     return lib
 
@@ -96,9 +113,9 @@ def _dtype_code(t):
     raise TypeError(f"unsupported input dtype {t.dtype} (float32 or bfloat16)")
 
 
-def make_shape(B, H, N, d_xi, d_v, M, dtype) -> IAShape:
+def make_shape(B, H, N, d_xi, d_v, M, dtype, delta_per_mode=False) -> IAShape:
     code = dtype if isinstance(dtype, int) else (IA_BF16 if dtype in (torch.bfloat16, "bf16") else IA_F32)
-    return IAShape(int(B), int(H), int(N), int(d_xi), int(d_v), int(M), code)
+    return IAShape(int(B), int(H), int(N), int(d_xi), int(d_v), int(M), code, int(bool(delta_per_mode)))
 
 
 def _ptr(t):
@@ -129,6 +146,11 @@ def prefill_workspace_bytes(B, H, N, d_xi, d_v, M, dtype) -> int:
 
 def prefill_launches(B, H, N, d_xi, d_v, M, dtype) -> int:
     return int(load_library().ia_prefill_launches(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
+
+
+def prefill_grid(B, H, N, d_xi, d_v, M, dtype) -> int:
+    """CTAs of the tensor-core chunk pass for this shape (0 off that path)."""
+    return int(load_library().ia_prefill_grid(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype))))
 
 
 def prefill_path(B, H, N, d_xi, d_v, M, dtype):
@@ -191,9 +213,20 @@ def _cuda_device(named):
     return dev
 
 
+def _check_delta(delta, H, M):
+    """delta [H] (one step per head) or [H,M] (one per head and mode), fp32.
+    Returns True for the per-mode form."""
+    _need("delta", delta, dtype=torch.float32)
+    if tuple(delta.shape) == (H,):
+        return False
+    if tuple(delta.shape) == (H, int(M)):
+        return True
+    raise ValueError(f"delta has shape {tuple(delta.shape)}, expected ({H},) or ({H}, {int(M)})")
+
+
 def _check_sequence_args(q, k, v, delta, M, A, dO=None):
     """q, k [B,H,N,d_xi], v and dO [B,H,N,d_v] in one input dtype, delta [H]
-    fp32, A [M] complex as 2M fp32 (or None).  Returns (B, H, N, d_xi, d_v)."""
+    or [H,M] fp32, A [M] complex as 2M fp32 (or None).  Returns (B, H, N, d_xi, d_v)."""
     _need("q", q)
     if q.dim() != 4:
         raise ValueError(f"q must be [B,H,N,d_xi], got shape {tuple(q.shape)}")
@@ -204,7 +237,7 @@ def _check_sequence_args(q, k, v, delta, M, A, dO=None):
     if v.dim() != 4 or tuple(v.shape[:3]) != (B, H, N):
         raise ValueError(f"v must be [B,H,N,d_v] = [{B},{H},{N},d_v], got {tuple(v.shape)}")
     d_v = v.shape[3]
-    _need("delta", delta, (H,), torch.float32)
+    _check_delta(delta, H, M)
     if A is not None:
         _need("A", A, dtype=torch.float32, numel=2 * int(M))
     if dO is not None:
@@ -223,7 +256,7 @@ def _check_token_args(q, k, v, delta, M, A):
     _need("v", v, dtype=q.dtype)
     if v.dim() != 3 or tuple(v.shape[:2]) != (B, H):
         raise ValueError(f"v must be [B,H,d_v] = [{B},{H},d_v], got {tuple(v.shape)}")
-    _need("delta", delta, (H,), torch.float32)
+    _check_delta(delta, H, M)
     if A is not None:
         _need("A", A, dtype=torch.float32, numel=2 * int(M))
     return B, H, d_xi, v.shape[2]
@@ -236,7 +269,7 @@ def prefill_fwd(q, k, v, delta, M, A=None, state_in=None, want_num_den=False, wa
     Returns dict with o [B,H,N,d_v] fp32 and, on request, num, den, state (flat fp32)."""
     lib = load_library()
     B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A)
-    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q), delta.dim() == 2)
     n_state = lib.ia_state_bytes(ctypes.byref(shp)) // 4
     if state_in is not None:
         _need("state_in", state_in, dtype=torch.float32, numel=n_state)
@@ -268,7 +301,7 @@ def prefill_fwd_static(q, k, v, delta, M, A=None, state_in=None, want_num_den=Fa
     caller's; pass `o` (and use want_* = False) to allocate nothing here."""
     lib = load_library()
     B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A)
-    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q), delta.dim() == 2)
     n_state = lib.ia_state_bytes(ctypes.byref(shp)) // 4
     if state_in is not None:
         _need("state_in", state_in, dtype=torch.float32, numel=n_state)
@@ -288,10 +321,14 @@ def prefill_fwd_static(q, k, v, delta, M, A=None, state_in=None, want_num_den=Fa
 
 
 def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
-    """Forward + reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta)."""
+    """Forward + reverse mode from a zero state: returns dict(o, dq, dk, dv, dDelta, dA).
+
+    delta is [H] (one step per head) or [H,M] (one per head and mode); dDelta
+    has its shape.  dA [2M] holds (dL/dRe A_m, dL/dIm A_m), for A as given or
+    for the S4D-Lin default when A is None."""
     lib = load_library()
     B, H, N, d_xi, d_v = _check_sequence_args(q, k, v, delta, M, A, dO=dO)
-    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q))
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q), delta.dim() == 2)
     if workspace is not None:
         _need("workspace", workspace)
     dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("dO", dO),
@@ -300,21 +337,22 @@ def fwd_bwd(q, k, v, delta, dO, M, A=None, workspace=None, stream=None):
     dq = torch.empty(B, H, N, d_xi, dtype=torch.float32, device=dev)
     dk = torch.empty_like(dq)
     dv = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
-    dD = torch.empty(H, dtype=torch.float32, device=dev)
+    dD = torch.empty(tuple(delta.shape), dtype=torch.float32, device=dev)
+    dA = torch.empty(2 * int(M), dtype=torch.float32, device=dev)
     need = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(shp))
     ws = _workspace(need, dev, workspace)
     rc = lib.ia_fwd_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A), _ptr(dO),
-                        _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dD), _ptr(ws),
+                        _ptr(o), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dD), _ptr(dA), _ptr(ws),
                         ctypes.c_size_t(_nbytes(ws)), _stream(stream))
     _check(rc, "ia_fwd_bwd")
-    return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD}
+    return {"o": o, "dq": dq, "dk": dk, "dv": dv, "dDelta": dD, "dA": dA}
 
 
 def decode_step(q, k, v, delta, state, M, A=None, o=None, want_num_den=False, stream=None):
     """One decode step.  q,k [B,H,d_xi], v [B,H,d_v]; state (flat fp32) updated in place."""
     lib = load_library()
     B, H, d_xi, d_v = _check_token_args(q, k, v, delta, M, A)
-    shp = make_shape(B, H, 1, d_xi, d_v, M, _dtype_code(q))
+    shp = make_shape(B, H, 1, d_xi, d_v, M, _dtype_code(q), delta.dim() == 2)
     _need("state", state, dtype=torch.float32, numel=lib.ia_state_bytes(ctypes.byref(shp)) // 4)
     if o is not None:
         _need("o", o, (B, H, d_v), torch.float32)
@@ -326,6 +364,85 @@ def decode_step(q, k, v, delta, state, M, A=None, o=None, want_num_den=False, st
     rc = lib.ia_decode_step(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(delta), _ptr(A),
                             _ptr(state), _ptr(o), _ptr(num), _ptr(den), _stream(stream))
     _check(rc, "ia_decode_step")
+    return {"o": o, "num": num, "den": den}
+
+
+def _options(named_shapes, delta_t, gain, bias, eps, W, bidirectional, B, H, M, d_xi, d_v, tokens):
+    """Check the optional parts and build the C options struct."""
+    if delta_t is not None:
+        _need("delta_t", delta_t, (B, H) + tokens, torch.float32)
+    for name, t in (("gain", gain), ("bias", bias)):
+        if t is not None:
+            _need(name, t, (H, d_xi + d_v), torch.float32)
+    if W is not None:
+        _need("W", W, dtype=torch.float32, numel=2 * H * int(M) * int(M))
+    opt = IAOptions(_ptr(delta_t), _ptr(gain), _ptr(bias), float(eps), _ptr(W), int(bool(bidirectional)))
+    return opt
+
+
+def prefill_fwd_ex(q, k, v, M, delta=None, A=None, delta_t=None, gain=None, bias=None, eps=1e-6, W=None,
+                   bidirectional=False, state_in=None, want_num_den=False, want_state=False, stream=None):
+    """The layer with its optional parts (see ia_prefill_fwd_ex in include/ia.h):
+    delta_t [B,H,N] a step per token, gain/bias [H, d_xi+d_v] the RMSNorm on the
+    SSM input, W [H,M,M,2] (re, im) the complex readout matrix, bidirectional
+    the two-direction layer.  Returns dict(o, num, den, state)."""
+    lib = load_library()
+    _need("q", q)
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B,H,N,d_xi], got shape {tuple(q.shape)}")
+    B, H, N, d_xi = q.shape
+    _need("k", k, (B, H, N, d_xi), q.dtype)
+    _need("v", v, dtype=q.dtype)
+    if v.dim() != 4 or tuple(v.shape[:3]) != (B, H, N):
+        raise ValueError(f"v must be [B,H,N,d_v], got {tuple(v.shape)}")
+    d_v = v.shape[3]
+    dpm = _check_delta(delta, H, M) if delta is not None else False
+    if delta is None and delta_t is None:
+        raise ValueError("either delta or delta_t is needed")
+    if A is not None:
+        _need("A", A, dtype=torch.float32, numel=2 * int(M))
+    shp = make_shape(B, H, N, d_xi, d_v, M, _dtype_code(q), dpm)
+    n_state = lib.ia_state_bytes(ctypes.byref(shp)) // 4
+    if state_in is not None:
+        _need("state_in", state_in, dtype=torch.float32, numel=n_state)
+    opt = _options(None, delta_t, gain, bias, eps, W, bidirectional, B, H, M, d_xi, d_v, (N,))
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("delta_t", delta_t),
+                        ("gain", gain), ("bias", bias), ("W", W), ("state_in", state_in)])
+    o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    num = torch.empty_like(o) if want_num_den else None
+    den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
+    st = torch.empty(n_state, dtype=torch.float32, device=dev) if want_state else None
+    rc = lib.ia_prefill_fwd_ex(ctypes.byref(shp), ctypes.byref(opt), _ptr(q), _ptr(k), _ptr(v), _ptr(delta),
+                               _ptr(A), _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _stream(stream))
+    _check(rc, "ia_prefill_fwd_ex")
+    return {"o": o, "num": num, "den": den, "state": st}
+
+
+def decode_step_ex(q, k, v, state, M, delta=None, A=None, delta_t=None, gain=None, bias=None, eps=1e-6,
+                   W=None, want_num_den=False, stream=None):
+    """One decode step with the optional parts; delta_t is [B,H] here."""
+    lib = load_library()
+    _need("q", q)
+    if q.dim() != 3:
+        raise ValueError(f"q must be [B,H,d_xi], got shape {tuple(q.shape)}")
+    B, H, d_xi = q.shape
+    _need("k", k, (B, H, d_xi), q.dtype)
+    _need("v", v, dtype=q.dtype)
+    d_v = v.shape[2]
+    dpm = _check_delta(delta, H, M) if delta is not None else False
+    if delta is None and delta_t is None:
+        raise ValueError("either delta or delta_t is needed")
+    shp = make_shape(B, H, 1, d_xi, d_v, M, _dtype_code(q), dpm)
+    _need("state", state, dtype=torch.float32, numel=lib.ia_state_bytes(ctypes.byref(shp)) // 4)
+    opt = _options(None, delta_t, gain, bias, eps, W, False, B, H, M, d_xi, d_v, ())
+    dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("state", state),
+                        ("delta_t", delta_t), ("gain", gain), ("bias", bias), ("W", W)])
+    o = torch.empty(B, H, d_v, dtype=torch.float32, device=dev)
+    num = torch.empty_like(o) if want_num_den else None
+    den = torch.empty(B, H, dtype=torch.float32, device=dev) if want_num_den else None
+    rc = lib.ia_decode_step_ex(ctypes.byref(shp), ctypes.byref(opt), _ptr(q), _ptr(k), _ptr(v), _ptr(delta),
+                               _ptr(A), _ptr(state), _ptr(o), _ptr(num), _ptr(den), _stream(stream))
+    _check(rc, "ia_decode_step_ex")
     return {"o": o, "num": num, "den": den}
 
 

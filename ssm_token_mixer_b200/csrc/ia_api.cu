@@ -46,8 +46,6 @@ bool use_tc_bwd(const ia_shape_t& s) {
   return tc_bwd_supported(s);
 }
 
-ia_status_t map_cuda(cudaError_t e) { return e == cudaSuccess ? IA_OK : IA_ERR_CUDA; }
-
 cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
 
 }  // namespace
@@ -57,10 +55,20 @@ bool valid_dims(const ia_shape_t* s, bool need_n) {
   if (s->B <= 0 || s->H <= 0 || s->d_xi <= 0 || s->d_v <= 0 || s->M <= 0) return false;
   if (need_n && s->N <= 0) return false;
   if (s->in_dtype != IA_F32 && s->in_dtype != IA_BF16) return false;
+  if (s->delta_per_mode != 0 && s->delta_per_mode != 1) return false;
   // element counts must stay addressable with 64-bit indices and int grid sizes
   const long long BH = static_cast<long long>(s->B) * s->H;
   if (BH > (1LL << 31) - 1) return false;
   return true;
+}
+
+// The CUDA error behind this thread's last IA_ERR_CUDA (see ia_last_cuda_error).
+thread_local int g_last_cuda_error = 0;
+
+ia_status_t map_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return IA_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return IA_ERR_CUDA;
 }
 
 bool inject_launch_failure() { return env_set("IA_INJECT_LAUNCH_FAILURE"); }
@@ -150,17 +158,21 @@ size_t ia_prefill_workspace_bytes(const ia_shape_t* s) {
   return tc_workspace_bytes(*s, tc_plan(*s, num_sms()));
 }
 
+int ia_prefill_grid(const ia_shape_t* s) {
+  if (!valid_dims(s, true) || !use_tc(*s)) return 0;
+  return tc_plan(*s, num_sms()).grid;
+}
+
 int ia_prefill_launches(const ia_shape_t* s) {
   if (!valid_dims(s, true)) return 0;
   if (!use_tc(*s)) return 1;
-  return tc_plan(*s, num_sms()).nseg > 1 ? 4 : 2;   // tables [+ state-only pass + scan] + full pass
+  return 2;   // the table kernel and the chunk pass
 }
 
 size_t ia_fwd_bwd_workspace_bytes(const ia_shape_t* s) {
   if (!valid_dims(s, true)) return 0;
   if (use_tc_bwd(*s)) return tc_fwd_bwd_workspace_bytes(*s, tc_plan(*s, num_sms()));
-  return sizeof(float2) * static_cast<size_t>(s->B) * s->H *
-             seq_bwd_ws_per_bh(s->N, s->d_xi, s->d_v, s->M) + 256;
+  return seq_bwd_workspace_bytes(*s);
 }
 
 ia_status_t ia_prefill_fwd(const ia_shape_t* s, const void* q, const void* k, const void* v,
@@ -175,7 +187,7 @@ ia_status_t ia_prefill_fwd(const ia_shape_t* s, const void* q, const void* k, co
   if (state_in && state_in == state_out) return IA_ERR_INVALID_ARG;
   const bool tc = use_tc(*s);
   size_t need = 0;
-  TcPlan plan{1, 1};
+  TcPlan plan{1};
   if (tc) {
     plan = tc_plan(*s, num_sms());
     need = tc_workspace_bytes(*s, plan);
@@ -193,12 +205,12 @@ ia_status_t ia_prefill_fwd(const ia_shape_t* s, const void* q, const void* k, co
 
 ia_status_t ia_fwd_bwd(const ia_shape_t* s, const void* q, const void* k, const void* v,
                        const float* delta, const float* A, const void* dO, float* o, float* dq,
-                       float* dk, float* dv, float* dDelta, void* workspace,
+                       float* dk, float* dv, float* dDelta, float* dA, void* workspace,
                        size_t workspace_bytes, void* stream) {
   if (!valid_dims(s, true)) return IA_ERR_INVALID_ARG;
   if (!q || !k || !v || !delta || !dO || !o || !dq || !dk || !dv || !dDelta)
     return IA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace};
+  const void* ptrs[] = {q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, dA, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
   const bool tc = use_tc_bwd(*s);
@@ -209,8 +221,8 @@ ia_status_t ia_fwd_bwd(const ia_shape_t* s, const void* q, const void* k, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc)
     return map_cuda(launch_tc_fwd_bwd(*s, tc_plan(*s, num_sms()), q, k, v, delta, A, dO, o, dq, dk,
-                                      dv, dDelta, workspace, st));
-  return map_cuda(launch_seq_bwd(*s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, workspace, st));
+                                      dv, dDelta, dA, workspace, st));
+  return map_cuda(launch_seq_bwd(*s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, dA, workspace, st));
 }
 
 ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, const void* v,
@@ -241,7 +253,7 @@ ia_status_t ia_set_launch_events(void* begin, void* end) {
 ia_status_t ia_check_device_errors(void* stream) {
   cudaError_t e;
   int flag = read_and_clear_device_error(static_cast<cudaStream_t>(stream), &e);
-  if (e != cudaSuccess) return IA_ERR_CUDA;
+  if (e != cudaSuccess) return map_cuda(e);
   if (flag & kErrTimeout) return IA_ERR_TIMEOUT;
   if (flag & kErrParamRange) return IA_ERR_PARAM_RANGE;
   return IA_OK;
@@ -255,6 +267,12 @@ ia_path_t ia_prefill_path(const ia_shape_t* s) {
 ia_path_t ia_fwd_bwd_path(const ia_shape_t* s) {
   if (!valid_dims(s, true)) return IA_PATH_NONE;
   return use_tc_bwd(*s) ? IA_PATH_TENSOR_CORE : IA_PATH_SEQUENTIAL;
+}
+
+int ia_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* ia_last_cuda_error_string(void) {
+  return g_last_cuda_error ? cudaGetErrorString(static_cast<cudaError_t>(g_last_cuda_error)) : "no error";
 }
 
 const char* ia_status_string(ia_status_t st) {

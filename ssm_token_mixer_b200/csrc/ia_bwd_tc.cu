@@ -17,12 +17,16 @@
 //     dxi(Q) = dS xi(K) + da~ R_U      dxi(K) = dS^T xi(Q) + E'' dS1_U
 //     dV = P^T dnum + E'' dS1_G        dR = dS1 + [da~^T xi(Q) | X^T dnum | X^T dden]
 //     dS_hat0 = conj(lambda^C) dR
-//   Delta enters only through the per-head tables, so their adjoints are
+//   Delta and A enter only through the per-head tables, so their adjoints are
 //   gathered over all chunks and contracted once with the tables' derivatives:
 //     dE''^T += da~^T S + X^T dP + dS1 x^T    (accumulated in TMEM)
 //     ds     += dX * a~,  dlambda^C += sum dR conj(S_hat0)
 //     d(b lambda^n)/dDelta = (lambda + n A b) lambda^n,  ds/dDelta = 2 Re(A)(i-c) s,
-//     d(lambda^C)/dDelta = C A lambda^C.
+//     d(lambda^C)/dDelta = C A lambda^C;  along A_m the same with
+//     d(b lambda^n)/dA = ((Delta lambda - b)/A + n Delta b) lambda^n,
+//     ds/dRe A = 2 Delta (i-c) s,  d(lambda^C)/dA = C Delta lambda^C.
+//   Each CTA writes its (b,h)'s per-mode sums of dL/dDelta, dL/dRe A and
+//   dL/dIm A; a fixed-order reduction turns them into dDelta and dA.
 // A dedicated MMA warp issues the contraction groups (tcgen05.mma blocks its
 // issuing thread) on ready barriers from the 8 epilogue warps, in the order
 // F1+B1, F2, B2, F4, B3-B5, dQ/dK/dV, so the readout chain (S, a~, P) and the
@@ -97,14 +101,16 @@ struct BwdArgs {
   const float* o;
   const float* den;
   const float* A;
+  const float* delta;
+  int dpm;
   const HeadTables* tabs;
   const uint8_t* R;  // [BH][nch] x (R_U, R_Gamma) fp16 swizzled tiles of 16 KB
   const float* Re;   // [BH][nch][128]
-  const float* dtab; // [H][128][64] d(E'')/dDelta rows, then [H][128] row sums
+  const float* dtab; // [3][H][128][64] d(E'')/dDelta, dRe A, dIm A rows, then [3][H][128] row sums
   float* dq;
   float* dk;
   float* dv;
-  float* dDelta;
+  float* gpart;      // [BH][M][3]: this (b,h)'s dL/dDelta_hm, dL/dRe A_m, dL/dIm A_m
   int* err;
   int H, N;
   long long BH;
@@ -172,12 +178,15 @@ __global__ void __launch_bounds__(NBWD, 1)
   const float2 lamC = T->lamC[m];
   const float ReA = a.A ? a.A[2 * m] : -0.5f;
   const float ImA = a.A ? a.A[2 * m + 1] : static_cast<float>(3.14159265358979323846 * m);
+  const float Dm = delta_hm(a.delta, a.dpm, kModesTC, h, m);
   const float r2 = T->r2[m];
   const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
   const float sgn = comp ? 1.f : -1.f;
-  // this row of d(E'')/dDelta over j (from the table prologue) and its sum
+  // this row of the three derivative tables over j (from the table prologue)
+  // and their sums: along Delta, Re A and Im A
+  const size_t tstride = static_cast<size_t>(a.H) * KR * C;
   const float* dErow = a.dtab + (static_cast<size_t>(h) * KR + k) * C;
-  const float dEsum_c = a.dtab[static_cast<size_t>(a.H) * KR * C + static_cast<size_t>(h) * KR + k];
+  auto dEsum = [&](int w) { return a.dtab[3 * tstride + (static_cast<size_t>(w) * a.H + h) * KR + k]; };
 
   // zero the state adjoint and the table adjoint
   if (warp < NEPI / 32) {
@@ -189,7 +198,12 @@ __global__ void __launch_bounds__(NBWD, 1)
     tmem_st_wait();
   }
   float de_c = 0.f;     // adjoint of the eta channel of the chunk-end state (this row)
-  float dD = 0.f;       // this thread's share of dDelta
+  // this thread's shares of dL/dDelta_hm, dL/dRe A_m, dL/dIm A_m, gathered as
+  //   gs  = sum dX a~ 2 (i-c) s                     (readout scale: Delta Re A in s)
+  //   zr, zn = sum over dR . R components            (Re z and -Im z of z = sum conj(dR) R,
+  //                                                    R = lambda^C S_hat0: C A and C Delta)
+  //   tD, tR, tI = the derivative-table contractions (E' and its chunk sum)
+  float gs = 0.f, zr = 0.f, zn = 0.f, tD = 0.f, tR = 0.f, tI = 0.f;
 
   auto issue_load = [&](int ch) {
     const int n0 = ch * C;
@@ -463,7 +477,7 @@ __global__ void __launch_bounds__(NBWD, 1)
           const int i = i0 + e;
           const float dx = fmaf(Reta, sDD[i], __uint_as_float(rx[e]));
           xs[e] = dx * s;
-          dD = fmaf(dx * __uint_as_float(ra[e]), 2.f * ReA * static_cast<float>(i - C / 2) * s, dD);
+          gs = fmaf(dx * __uint_as_float(ra[e]), 2.f * static_cast<float>(i - C / 2) * s, gs);
           s *= r2;
         }
         *reinterpret_cast<uint4*>(smem + B::S_DA + tile_off(k, i0, 1024)) = pack8(xs);
@@ -511,7 +525,8 @@ __global__ void __launch_bounds__(NBWD, 1)
           const float x = __uint_as_float(r[e]);
           const float y = __shfl_xor_sync(kFull, x, 1);
           const float rpart = __shfl_xor_sync(kFull, rv[e], 1);
-          dD = fmaf(static_cast<float>(C), fmaf(ReA, x * rv[e], ImA * sgn * x * rpart), dD);
+          zr = fmaf(x, rv[e], zr);
+          zn = fmaf(sgn * x, rpart, zn);
           w[e] = __float_as_uint(fmaf(lamC.x, x, -sgn * lamC.y * y));
         }
         tmem_st16(trow + B::T_ADJ + col0, w);
@@ -521,15 +536,20 @@ __global__ void __launch_bounds__(NBWD, 1)
       const float dRe = de_c + sRED[k] + sRED[KR + k];
       const float y = __shfl_xor_sync(kFull, dRe, 1);
       const float Rp = __shfl_xor_sync(kFull, Reta, 1);
-      float dEpart = dEsum_c;
+      float dEpart[3] = {dEsum(0), dEsum(1), dEsum(2)};
       if (nv < C) {   // ragged chunk: only the valid keys carry the constant channel
-        float acc = 0.f;
-        for (int j = 0; j < nv; ++j) acc += dErow[j];
-        dEpart = acc;
+        for (int w = 0; w < 3; ++w) {
+          float acc = 0.f;
+          for (int j = 0; j < nv; ++j) acc += dErow[w * tstride + j];
+          dEpart[w] = acc;
+        }
       }
       if (half == 0) {
-        dD = fmaf(static_cast<float>(C), fmaf(ReA, dRe * Reta, ImA * sgn * dRe * Rp), dD);
-        dD = fmaf(de_c, dEpart, dD);
+        zr = fmaf(dRe, Reta, zr);
+        zn = fmaf(sgn * dRe, Rp, zn);
+        tD = fmaf(de_c, dEpart[0], tD);
+        tR = fmaf(de_c, dEpart[1], tR);
+        tI = fmaf(de_c, dEpart[2], tI);
       }
       de_c = fmaf(lamC.x, dRe, -sgn * lamC.y * y);
     }
@@ -613,34 +633,44 @@ __global__ void __launch_bounds__(NBWD, 1)
   }
 
   if (!aborted) {
-    // contract the table adjoint with d(E'')/dDelta
+    // contract the table adjoint with the three derivative tables
 #pragma unroll
     for (int cb = 0; cb < 32; cb += 16) {
       const int j0 = 32 * half + cb;
       uint32_t r[16];
       tmem_ld16(trow + B::T_EBAR + j0, r);
       tmem_ld_wait16(r);
-      const float4* dq4 = reinterpret_cast<const float4*>(dErow + j0);
+      float* acc[3] = {&tD, &tR, &tI};
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 d = dq4[g];
-        dD = fmaf(__uint_as_float(r[4 * g]), d.x, dD);
-        dD = fmaf(__uint_as_float(r[4 * g + 1]), d.y, dD);
-        dD = fmaf(__uint_as_float(r[4 * g + 2]), d.z, dD);
-        dD = fmaf(__uint_as_float(r[4 * g + 3]), d.w, dD);
+      for (int w = 0; w < 3; ++w) {
+        const float4* dq4 = reinterpret_cast<const float4*>(dErow + w * tstride + j0);
+        float t = *acc[w];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 d = dq4[g];
+          t = fmaf(__uint_as_float(r[4 * g]), d.x, t);
+          t = fmaf(__uint_as_float(r[4 * g + 1]), d.y, t);
+          t = fmaf(__uint_as_float(r[4 * g + 2]), d.z, t);
+          t = fmaf(__uint_as_float(r[4 * g + 3]), d.w, t);
+        }
+        *acc[w] = t;
       }
     }
-    // block reduction -> one atomic per CTA
+    // this thread's shares, then the sum over the mode's four threads (two
+    // rows re/im in adjacent lanes, two column halves in warps w and w + 4),
+    // written for the fixed-order reduction over the batch
+    float g3[3];
+    g3[0] = fmaf(ReA, gs, fmaf(static_cast<float>(C), fmaf(ReA, zr, ImA * zn), tD));
+    g3[1] = fmaf(Dm, gs, fmaf(static_cast<float>(C) * Dm, zr, tR));
+    g3[2] = fmaf(static_cast<float>(C) * Dm, zn, tI);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dD += __shfl_xor_sync(kFull, dD, off);
+    for (int w = 0; w < 3; ++w) g3[w] += __shfl_xor_sync(kFull, g3[w], 1);
     named_sync(1, NEPI);
-    if (lane == 0) sRED[warp] = dD;
+    if (half == 1 && comp == 0)
+      for (int w = 0; w < 3; ++w) sRED[w * KR / 2 + m] = g3[w];
     named_sync(1, NEPI);
-    if (tid == 0) {
-      float s = 0.f;
-      for (int w = 0; w < NEPI / 32; ++w) s += sRED[w];
-      atomicAdd(a.dDelta + h, s);
-    }
+    if (half == 0 && comp == 0)
+      for (int w = 0; w < 3; ++w) a.gpart[(bh * kModesTC + m) * 3 + w] = g3[w] + sRED[w * KR / 2 + m];
   } else {   // let our own copies land before exiting (bounded)
     if (tid == 0 && tma_pending) mbar_wait(bar_tma, ph_tma, a.err);
     if (tid == 0 && r_pending) mbar_wait(bar_r, ph_r, a.err);
@@ -666,14 +696,15 @@ size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
   bytes += BH * nch * 2 * KR * 64 * 2;                        // R per chunk: two fp16 tiles
   bytes += BH * nch * KR * sizeof(float);                      // R_eta per chunk
   bytes += BH * s.N * sizeof(float) + 256;                     // den
-  bytes += static_cast<size_t>(s.H) * KR * (C + 1) * sizeof(float) + 256;   // dE/dDelta table
+  bytes += dtab_floats(s.H) * sizeof(float) + 256;              // derivative tables
+  bytes += grad_partials_bytes(s) + 256;                        // per-(b,h,m) gradient partials
   return bytes + 256;
 }
 
 cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A, const void* dO,
-                              float* o, float* dq, float* dk, float* dv, float* dDelta, void* ws,
-                              cudaStream_t st) {
+                              float* o, float* dq, float* dk, float* dv, float* dDelta, float* dA,
+                              void* ws, cudaStream_t st) {
   const size_t BH = static_cast<size_t>(s.B) * s.H;
   const size_t nch = (s.N + C - 1) / C;
   uint8_t* base = reinterpret_cast<uint8_t*>(tc_tables(ws));
@@ -684,10 +715,10 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   den = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(den) + 255) & ~static_cast<uintptr_t>(255));
   float* dtab = den + BH * s.N;
   dtab = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(dtab) + 255) & ~static_cast<uintptr_t>(255));
+  float* gpart = dtab + dtab_floats(s.H);
+  gpart = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(gpart) + 255) & ~static_cast<uintptr_t>(255));
   cudaError_t e = launch_tc_prefill(s, p, q, k, v, delta, A, nullptr, o, nullptr, den, nullptr, ws,
                                     st, dumpR, dumpRe, dtab);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(dDelta, 0, sizeof(float) * s.H, st);
   if (e != cudaSuccess) return e;
   BwdArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -697,6 +728,8 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   a.o = o;
   a.den = den;
   a.A = A;
+  a.delta = delta;
+  a.dpm = s.delta_per_mode;
   a.tabs = tc_tables(ws);
   a.R = dumpR;
   a.Re = dumpRe;
@@ -704,15 +737,15 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.dDelta = dDelta;
+  a.gpart = gpart;
   a.err = device_error_ptr();
   if (!a.err) return cudaErrorInvalidSymbol;
   a.H = s.H;
   a.N = s.N;
   a.BH = static_cast<long long>(BH);
   CUtensorMap tm_dq, tm_dk, tm_dv;
-  if (!encode_rows64_f32_map(&tm_dq, dq, a.BH, s.N) || !encode_rows64_f32_map(&tm_dk, dk, a.BH, s.N) ||
-      !encode_rows64_f32_map(&tm_dv, dv, a.BH, s.N))
+  if (!encode_rows64_f32_map(&tm_dq, dq, a.BH, s.N, 64) || !encode_rows64_f32_map(&tm_dk, dk, a.BH, s.N, 64) ||
+      !encode_rows64_f32_map(&tm_dv, dv, a.BH, s.N, 64))
     return cudaErrorNotSupported;
   e = cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B::SMEM);
   if (e != cudaSuccess) return e;
@@ -720,7 +753,8 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
   tc_bwd_kernel<<<static_cast<unsigned>(BH), NBWD, B::SMEM, st>>>(a, tm_dq, tm_dk, tm_dv);
   e = cudaGetLastError();
   mark_launch_end(st);
-  return e;
+  if (e != cudaSuccess) return e;
+  return launch_grad_reduce(s, gpart, dDelta, dA, st);
 }
 
 }  // namespace ia

@@ -40,7 +40,7 @@ __device__ __forceinline__ float xi_acc(float x) { return x > 0.f ? x + 1.f : ex
 template <typename T>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(
     int H, int DX, int DV, int M, int MG, const T* __restrict__ q, const T* __restrict__ k,
-    const T* __restrict__ v, const float* __restrict__ delta, const float* __restrict__ A,
+    const T* __restrict__ v, const float* __restrict__ delta, int dpm, const float* __restrict__ A,
     float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
     float* __restrict__ den, long long BH) {
   extern __shared__ float4 dsm[];
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(
     const int m = m0 + i;
     const float ar = A ? A[2 * m] : -0.5f;
     const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
-    const float d = delta[h];
+    const float d = delta_hm(delta, dpm, M, h, m);
     const float x = d * ar, y = d * ai;
     float sy, cy, sh, ch;
     sincosf(y, &sy, &cy);
@@ -203,7 +203,7 @@ constexpr int kBhWarps = 8;
 template <typename T>
 __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
     int H, int DX, int DV, int M, int D, const T* __restrict__ q, const T* __restrict__ k,
-    const T* __restrict__ v, const float* __restrict__ delta, const float* __restrict__ A,
+    const T* __restrict__ v, const float* __restrict__ delta, int dpm, const float* __restrict__ A,
     float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
     float* __restrict__ den, long long BH, int* err) {
   extern __shared__ float4 dsm[];
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
   for (int m = tid; m < M; m += kBhWarps * 32) {
     const float ar = A ? A[2 * m] : -0.5f;
     const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
-    const float d = delta[h];
+    const float d = delta_hm(delta, dpm, M, h, m);
     const float x = d * ar, y = d * ai;
     float sy, cy, sh, ch;
     sincosf(y, &sy, &cy);
@@ -383,7 +383,7 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
     mark_launch_begin(st);
     kern<<<static_cast<unsigned>(BHc), kBhWarps * 32, smem, st>>>(
         s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q), static_cast<const T*>(k),
-        static_cast<const T*>(v), delta, A, static_cast<float2*>(state), o, num, den, BHc, err);
+        static_cast<const T*>(v), delta, s.delta_per_mode, A, static_cast<float2*>(state), o, num, den, BHc, err);
     e = cudaGetLastError();
     mark_launch_end(st);
     return e;
@@ -410,7 +410,7 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   cfg.numAttrs = 1;
   mark_launch_begin(st);
   e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, MG, static_cast<const T*>(q),
-                         static_cast<const T*>(k), static_cast<const T*>(v), delta, A,
+                         static_cast<const T*>(k), static_cast<const T*>(v), delta, s.delta_per_mode, A,
                          static_cast<float2*>(state), o, num, den, BH);
   mark_launch_end(st);
   return e;

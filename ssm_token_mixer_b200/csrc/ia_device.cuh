@@ -291,6 +291,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
+// 32 lanes x 32 bit, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -329,6 +335,11 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_m
 }
 
 // ------------------------------------------------------------ small helpers
+// Delta of head h and mode m: delta [H] (dpm = 0) or [H,M] (dpm = 1).
+__device__ __forceinline__ float delta_hm(const float* delta, int dpm, int M, int h, int m) {
+  return dpm ? delta[static_cast<long long>(h) * M + m] : delta[h];
+}
+
 __device__ __forceinline__ float feat(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

@@ -11,8 +11,21 @@ namespace ia {
 
 struct HeadTables;
 
-cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
-                                cudaStream_t st, float* dtab = nullptr);
+// Per-head tables of the tensor-core path (and, with dtab, the Delta
+// derivative table of the reverse pass); also clears nflags look-back flags
+// of the chunk pass that follows.
+cudaError_t launch_param_tables(int H, const float* delta, int dpm, const float* A, HeadTables* tabs,
+                                cudaStream_t st, float* dtab = nullptr, int* flags = nullptr,
+                                int nflags = 0);
+// Floats of the three derivative tables of the reverse pass plus their row sums.
+inline size_t dtab_floats(int H) { return 3 * static_cast<size_t>(H) * 128 * (64 + 1); }
+
+// Reverse passes leave per-(b,h,m) partials of dL/dDelta_hm, dL/dRe A_m and
+// dL/dIm A_m ([B,H,M][3] fp32); this reduces them in a fixed order into
+// dDelta ([H] or [H,M]) and, if dA is not null, dA ([M] complex).
+size_t grad_partials_bytes(const ia_shape_t& s);
+cudaError_t launch_grad_reduce(const ia_shape_t& s, const float* gpart, float* dDelta, float* dA,
+                               cudaStream_t st);
 
 size_t seq_fwd_smem(int DX, int DV, int M);
 cudaError_t launch_seq_fwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
@@ -21,21 +34,25 @@ cudaError_t launch_seq_fwd(const ia_shape_t& s, const void* q, const void* k, co
 
 size_t seq_bwd_smem(int DX, int DV, int M);
 size_t seq_bwd_ws_per_bh(int N, int DX, int DV, int M);   // in float2 units
+size_t seq_bwd_workspace_bytes(const ia_shape_t& s);
 cudaError_t launch_seq_bwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
                            const float* delta, const float* A, const void* dO, float* o, float* dq,
-                           float* dk, float* dv, float* dDelta, void* ws, cudaStream_t st);
-
-cudaError_t launch_segment_scan(int B, int H, int DX, int DV, int nseg, int L,
-                                const HeadTables* tabs, const void* state_in, float* ws_state,
-                                float* ws_eta, cudaStream_t st);
+                           float* dk, float* dv, float* dDelta, float* dA, void* ws, cudaStream_t st);
 
 // Tensor-core chunked prefill (bf16 inputs, M = 64).
 bool tc_prefill_supported(const ia_shape_t& s);
 struct TcPlan {
-  int nseg;        // segments per (b,h) sequence
-  int seg_chunks;  // chunks per segment (all but the last)
+  int grid;   // CTAs of the chunk pass, each an equal range of the (stream, chunk) space
 };
 TcPlan tc_plan(const ia_shape_t& s, int num_sms);
+// One CTA per stream (whole value-block sequences, no look-back): the plan
+// of the no-allocation entry point.
+inline TcPlan tc_plan_whole_streams(const ia_shape_t& s) {
+  return TcPlan{static_cast<int>(static_cast<long long>(s.B) * s.H * (s.d_v / 64))};
+}
+// True if some CTA range of the plan starts inside a stream (the pass then
+// needs the look-back buffers of the workspace).
+bool tc_plan_splits(const ia_shape_t& s, const TcPlan& p);
 size_t tc_workspace_bytes(const ia_shape_t& s, const TcPlan& p);
 cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A,
@@ -46,24 +63,28 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
 
-// TMA tensor maps (ia_prefill_tc.cu): an fp32 [BH][N][64] array as
-// 32-column x 64-row boxes, 128-byte swizzled; q/k/v bf16 [BH][N][64] as
+// TMA tensor maps (ia_prefill_tc.cu): an fp32 [BH][N][W] array as
+// 32-column x 64-row boxes, 128-byte swizzled; q/k/v bf16 [BH][N][W] as
 // 64 x 64 boxes, 128-byte swizzled.  False if the driver refuses the map.
-bool encode_rows64_f32_map(CUtensorMap* m, float* x, long long BH, int N);
-bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N);
+bool encode_rows64_f32_map(CUtensorMap* m, float* x, long long BH, int N, int W);
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W);
 
 // Tensor-core training step (bf16, M = 64, d_xi = d_v = 64).
 bool tc_bwd_supported(const ia_shape_t& s);
 size_t tc_fwd_bwd_workspace_bytes(const ia_shape_t& s, const TcPlan& p);
 cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* q, const void* k,
                               const void* v, const float* delta, const float* A, const void* dO,
-                              float* o, float* dq, float* dk, float* dv, float* dDelta, void* ws,
-                              cudaStream_t st);
+                              float* o, float* dq, float* dk, float* dv, float* dDelta, float* dA,
+                              void* ws, cudaStream_t st);
 
 // Decode step.
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
                           const float* delta, const float* A, void* state, float* o, float* num,
                           float* den, cudaStream_t st);
+
+// IA_OK for cudaSuccess, else IA_ERR_CUDA after recording the error as this
+// thread's last CUDA error (ia_last_cuda_error).
+ia_status_t map_cuda(cudaError_t e);
 
 // Failure injection for host tests: with IA_INJECT_LAUNCH_FAILURE set (and
 // not "0"), every entry point returns IA_ERR_CUDA after its argument checks,

@@ -55,8 +55,7 @@ extern "C" IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* s, const v
     if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
   if (state_in && state_in == state_out) return IA_ERR_INVALID_ARG;
   if (!tc_prefill_supported(*s)) return IA_ERR_UNSUPPORTED;
-  const int nch = (s->N + kChunk - 1) / kChunk;
-  const TcPlan plan{1, nch};
+  const TcPlan plan = tc_plan_whole_streams(*s);   // one CTA per stream: tables only
   if (tc_workspace_bytes(*s, plan) > kStaticScratchBytes) return IA_ERR_WORKSPACE;
   if (inject_launch_failure()) return IA_ERR_CUDA;
   // Device address of the scratch array: in host code its name is only a
@@ -65,8 +64,7 @@ extern "C" IA_API ia_status_t ia_prefill_fwd_static(const ia_shape_t* s, const v
   static SymbolCache scratch_cache;
   cudaError_t e;
   void* scratch = scratch_cache.get(&g_static_scratch, &e);
-  if (!scratch) return IA_ERR_CUDA;
-  e = launch_tc_prefill(*s, plan, q, k, v, delta, A, state_in, o, num, den, state_out, scratch,
-                        static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? IA_OK : IA_ERR_CUDA;
+  if (!scratch) return map_cuda(e);
+  return map_cuda(launch_tc_prefill(*s, plan, q, k, v, delta, A, state_in, o, num, den, state_out,
+                                    scratch, static_cast<cudaStream_t>(stream)));
 }

@@ -7,13 +7,13 @@
 // summary's sec. A.2 describes.  Per (b,h) and chunk, with positions i, j in
 // [0, C), centre c = C/2 and the per-head table E'[j,m] = b_m lambda_m^(c-j):
 //
-//   S^T   = xi(K) xi(Q)^T                         GEMM1  (masked j <= i)
-//   a~^T  = E'^T S^T + R_U xi(Q)^T                GEMM2 + GEMM3   (a_i = lambda^(i-c) a~_i)
+//   S^T   = xi(K) xi(Q)^T                         G1  (masked j <= i)
+//   a~^T  = E'^T S^T + R_U xi(Q)^T                G2 + G3   (a_i = lambda^(i-c) a~_i)
 //   X     = |lambda|^(2(i-c)) a~                  (rows re/im; = conj(a) lambda^(i-c))
-//   P     = X E'^T                                GEMM4  (masked j <= i)
-//   num   = P V + X R_Gamma,  den = P 1 + X R_eta GEMM5,5b + GEMM6,6b
+//   P     = X E'^T                                G4  (masked j <= i)
+//   num   = P V + X R_Gamma,  den = P 1 + X R_eta G5 + G6
 //   o     = num / den
-//   S_hat <- R + E'^T [xi(K) | V]                 GEMM7  (accumulated onto R in TMEM)
+//   S_hat <- R + E'^T [xi(K) | V]                 G7  (accumulated onto R in TMEM)
 //
 // where the running state is kept scaled, S_hat = lambda^-(C-c-1) S, so that
 // R = lambda^C S_hat is both the decayed state the chunk adds to and the
@@ -21,24 +21,23 @@
 // split into real rows k = 2m (re) and 2m+1 (im), so every contraction is a
 // real fp16 x fp16 -> fp32 tcgen05 MMA with M = 64 or 128.
 //
-// Layouts: every shared-memory operand is in the no-swizzle canonical layout
-// (core matrices of 8 rows x 16 bytes, 128 contiguous bytes).  A tile with
-// rows r and columns x (x contiguous) of width W stores element (r, x) at
-//   (r/8)*(W*16) + (x/8)*128 + (r%8)*16 + (x%8)*2,
-// which serves as K-major (rows = M/N, lbo 128, sbo W*16) or as MN-major
-// (columns = M/N, lbo W*16, sbo 128) depending on the contraction.
-//
-// TMEM columns: [0,F) scaled state rows k; [F,F+64) a~^T (den aliases its
-// first 16 columns later in the chunk); [F+64,F+128) S^T then P (M=64
-// layout); [F+128, F+128+DV) num (M=64 layout).  F = d_xi + d_v.
-//
-// Sequences are split into segments when (b,h) pairs alone cannot fill the
-// GPU: a state-only pass produces each segment's local end state, a scan
-// combines them (S_in(s+1) = lambda^L S_in(s) + S_local(s)), and the full
-// pass recomputes every segment from its carried-in state -- the two
-// parallel passes around a sequential carry pass of the summary's sec. A.2.
+// Work split.  The value columns are cut into blocks of 64 (one per CTA at a
+// time), so a "stream" is one (b,h, value block): its CTA carries the whole
+// U (M x d_xi) but only its block of Gamma.  The grid is at most one CTA per
+// SM, and every CTA takes an equal contiguous range of the flattened
+// (stream, chunk) space, so all SMs get the same number of chunks whatever
+// the batch.  A range may start or end inside a stream.  The carried state
+// at such a boundary comes from the chunk algebra's linearity (the summary's
+// sec. A.2: parallel work within pieces, sequential state passing between
+// them): a CTA whose range ends inside a stream first runs the state-only
+// chain over that last piece from a zero state and publishes the result
+// (its local aggregate) to global memory; a CTA whose range starts inside a
+// stream composes its carry-in from its predecessors' published states,
+// S_in = sum over hops of lambda^(C n) A_p (a decoupled look-back, every
+// wait bounded), then runs the full chunk pass over its pieces.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 
@@ -67,14 +66,14 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// q, k or v [BH][N][64] bf16: one box is 64 rows x 64 columns (128 bytes) of
-// one (b,h), 128-byte swizzled in shared memory.  Rows >= N lie outside the
-// map and read as zero.
-bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
+// q, k or v [BH][N][W] bf16 (W a multiple of 64): one box is 64 rows x 64
+// columns (128 bytes) of one (b,h), 128-byte swizzled in shared memory.  Rows
+// >= N lie outside the map and read as zero.
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W) {
   const EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {64 * 2, static_cast<cuuint64_t>(N) * 64 * 2};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(W) * 2, static_cast<cuuint64_t>(N) * W * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kChunk), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
@@ -82,14 +81,15 @@ bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// An fp32 [BH][N][64] array (o, dq, dk, dv) seen as boxes of 32 columns x 64
+// An fp32 [BH][N][W] array (o, dq, dk, dv) seen as boxes of 32 columns x 64
 // rows of one (b,h), 128-byte swizzled in shared memory; rows >= N lie
 // outside the map (TMA stores skip them).
-bool encode_rows64_f32_map(CUtensorMap* m, float* o, long long BH, int N) {
+bool encode_rows64_f32_map(CUtensorMap* m, float* o, long long BH, int N, int W) {
   const EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {64 * sizeof(float), static_cast<cuuint64_t>(N) * 64 * sizeof(float)};
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(W) * sizeof(float),
+                                 static_cast<cuuint64_t>(N) * W * sizeof(float)};
   const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(kChunk), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -101,52 +101,67 @@ namespace {
 
 using namespace tc;
 
-constexpr int NT = 512;            // 16 warps: warp w owns TMEM lane quadrant w%4, column quarter w/4
-constexpr int NWARP = NT / 32;
+constexpr int kVB = 64;                  // value columns per stream (one CTA's block of Gamma)
+constexpr int kMinPiece = 4;             // fewest chunks per CTA the planner hands out
 
-template <int DX, int DV>
-struct Cfg {
-  static constexpr int F = DX + DV;
-  // den rides along the value contractions as an extra column when TMEM has room
-  static constexpr bool MERGE = F + 128 + DV + 16 <= 512;
-  static constexpr int WV = MERGE ? DV + 16 : DV;   // width of the V and R_Gamma tiles
-  static constexpr int NV = MERGE ? DV + 16 : DV;   // N of the value contractions
-  static constexpr uint32_t RSX = DX * 16;          // row-group stride of an [r][DX] fp16 tile
+// Four roles: 8 prepare warps (0-7) convert the inputs and rotate the carried
+// state into R; 8 output warps (8-15) run the masks, the readout scale and
+// o = num/den; warp 16 issues every tensor-core contraction; warp 17 brings
+// q, k, v in with TMA tensor loads that land in the operand layout.
+constexpr int GW = 8;                    // warps per epilogue group
+constexpr int GT = GW * 32;              // threads per epilogue group
+constexpr int NTH = 2 * GT + 64;         // + the MMA warp and the fetch warp
+
+template <int DX>
+struct PCfg {
+  static constexpr int F = DX + kVB;                // state columns: U | Gamma block
+  static constexpr int FH = F / 2;                  // state columns per prepare thread
+  static constexpr int WV = 80, NV = 80;            // [V | 1 0..] and [R_Gamma | R_eta 0..] widths
+  static constexpr int NB = DX == 64 ? 3 : 2;       // q, k, v and R_Gamma buffer sets
+  // d_xi = 128 needs 64 more state columns; S^T, a~ and P then share one tile
+  // (each is dead before the next is written within a chunk), at the price
+  // of issuing G1 of a chunk only after the previous chunk's P has been read.
+  static constexpr bool SHARED_SAP = DX == 128;
   static constexpr uint32_t RSV = WV * 16;
-  static constexpr uint32_t T_STATE = 0, T_A = F, T_SP = F + 64, T_NUM = F + 128;
-  static constexpr uint32_t T_DEN = MERGE ? T_NUM + DV : F;
-  static_assert(F + 128 + NV <= 512, "TMEM budget");
-  static_assert(DX % 64 == 0 && DV % 64 == 0, "feature widths must be multiples of 64");
-  static constexpr uint32_t STG_Q = 0;
-  static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
-  static constexpr uint32_t STG_V = STG_K + C * DX * 2;
-  static constexpr uint32_t S_Q = STG_V + C * DV * 2;
-  static constexpr uint32_t S_K = S_Q + C * DX * 2;
-  static constexpr uint32_t S_V = S_K + C * DX * 2;
-  static constexpr uint32_t S_E = S_V + C * WV * 2;
-  static constexpr uint32_t S_SP = S_E + KR * C * 2;
-  static constexpr uint32_t S_X = S_SP + C * C * 2;
-  static constexpr uint32_t S_RU = S_X + KR * C * 2;
-  static constexpr uint32_t S_RG = S_RU + KR * DX * 2;
-  static constexpr uint32_t S_RE = S_RG + KR * WV * 2;
-  static constexpr uint32_t S_ONES = S_RE + (MERGE ? 0 : KR * 16 * 2);
-  static constexpr uint32_t S_BAR = S_ONES + (MERGE ? 0 : C * 16 * 2);
-  static constexpr uint32_t S_TMEMH = S_BAR + 32;
+  static constexpr uint32_t T_STATE = 0;
+  static constexpr uint32_t T_A = F;
+  static constexpr uint32_t T_S = SHARED_SAP ? F : F + 64;
+  static constexpr uint32_t T_P = SHARED_SAP ? F : F + 128;
+  static constexpr uint32_t T_NUM = SHARED_SAP ? F + 64 : F + 192;
+  static constexpr uint32_t T_DEN = T_NUM + 64;
+  static constexpr uint32_t RU_COLS = DX / 2;       // R_U as fp16 pairs: columns per buffer
+  static constexpr uint32_t T_RU = SHARED_SAP ? 384 : 400;   // [2] x RU_COLS
+  static_assert(T_RU >= T_NUM + NV && T_RU + 2 * RU_COLS <= 512, "TMEM budget");
+  static constexpr uint32_t BOX = C * 64 * 2;       // one 64 x 64 bf16 box: 8 KB
+  static constexpr uint32_t TQ = C * DX * 2;        // q or k tile: DX / 64 boxes
+  static constexpr uint32_t TV = C * kVB * 2;
+  static constexpr uint32_t TRG = KR * WV * 2;
+  static constexpr uint32_t TO = C * kVB * 4;       // o block of one chunk: two 64 x 128-byte boxes
+  static constexpr uint32_t SW = 1024;              // one swizzle atom: 8 rows x 128 bytes
+  static constexpr uint32_t S_Q = 0;
+  static constexpr uint32_t S_K = S_Q + NB * TQ;
+  static constexpr uint32_t S_V = S_K + NB * TQ;
+  static constexpr uint32_t S_ONES = S_V + NB * TV;   // [V | 1]: MN-block 64..127 of G5's B operand
+  static constexpr uint32_t S_E = S_ONES + TV;
+  static constexpr uint32_t S_S = S_E + KR * C * 2;
+  static constexpr uint32_t S_P = S_S + C * C * 2;
+  static constexpr uint32_t S_X = S_P + C * C * 2;
+  static constexpr uint32_t S_O = S_X + KR * C * 2;   // [2] o staging, 128-byte swizzled
+  static constexpr uint32_t S_RG = S_O + 2 * TO;      // [NB]
+  static constexpr uint32_t S_BAR = S_RG + NB * TRG;  // mbarriers
+  static constexpr uint32_t S_FLAG = S_BAR + 256;     // abort flag, look-back exchange
+  static constexpr uint32_t S_TMEMH = S_FLAG + 16;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
-  // o of one chunk is staged (fp32, swizzled) over the sX and sRU tiles, both
-  // free while the output is written
-  static constexpr uint32_t S_OUT = S_X;
-  static_assert(KR * C * 2 + KR * DX * 2 >= C * DV * 4, "output staging fits");
+  static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
+  static_assert(S_O % 1024 == 0 && S_K % 1024 == 0 && S_V % 1024 == 0 && S_ONES % 1024 == 0,
+                "swizzled tiles start on the 128-byte swizzle period");
+  // byte offset of K-step kk (16 features) inside a K-major swizzled q/k tile
+  static __device__ __forceinline__ uint32_t kstep(int kk) { return (kk >> 2) * BOX + (kk & 3) * 32; }
 };
 
 struct TcArgs {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k;
-  const __nv_bfloat16* v;
   const HeadTables* tabs;
-  const float2* state_in;   // public layout, unscaled; seeds segment 0 of the full pass
-  float* seg_state;         // [BH][nseg-1][128][F] scaled: local end states, then carries
-  float* seg_eta;           // [BH][nseg-1][128]
+  const float2* state_in;   // public layout, unscaled
   float* o;
   float* num;
   float* den;
@@ -154,51 +169,12 @@ struct TcArgs {
   int* err;                 // device error flag
   uint8_t* dump_R;          // optional: R = lambda^C S_hat at every chunk start, fp16 tiles (dump_r16)
   float* dump_Re;           // optional: the eta part, [BH][nch][128] fp32
-  int H, N, nseg, seg_chunks;
-  long long BH;
+  float* agg;               // [G][128 * F + 128]: local end state of a CTA's last piece
+  float* incl;              // [G][128 * F + 128]: inclusive end state of a CTA's last piece
+  int* flags;               // [G]: 0 nothing yet, 1 agg published, 2 incl published
+  int H, N, DV, nch, nvb, G;
+  long long BH, total;      // total = BH * nvb * nch chunks
 };
-
-// bf16 staging rows [C][W] (row-major) -> fp16 canonical tile of row width WD,
-// applying xi when FEAT; rows >= nv become zero.  Work is split into warp
-// iterations of 8 rows x 4 column groups, the column group rotated by the row
-// so that staging reads and tile writes are bank-conflict free; all loads of
-// a thread are issued before any conversion.
-template <int W, int WD, bool FEAT, int NW = NWARP>
-__device__ __forceinline__ void convert_all(const uint8_t* stg, uint8_t* dst, int nv, int warp, int lane) {
-  constexpr int NCG = W / 8;
-  constexpr int ITERS = (C / 8) * (NCG / 4);
-  constexpr int PER = (ITERS + NW - 1) / NW;
-  const int r8 = lane & 7, slot = lane >> 3;
-  uint4 in[PER];
-  int rr[PER], cc[PER];
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int it = warp + u * NW;
-    const int rb = it & 7, rest = it >> 3;
-    rr[u] = rb * 8 + r8;
-    cc[u] = (rest >> 1) * 8 + ((slot + 4 * (rest & 1) + r8) & 7);
-    in[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (it < ITERS && rr[u] < nv) in[u] = *reinterpret_cast<const uint4*>(stg + rr[u] * (W * 2) + cc[u] * 16);
-  }
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int it = warp + u * NW;
-    if (it >= ITERS) break;
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (rr[u] < nv) {
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 f = __bfloat1622float2(p[e]);
-        if (FEAT) { f.x = feat(f.x); f.y = feat(f.y); }
-        w[e] = pack_half2(f.x, f.y);
-      }
-      out = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    *reinterpret_cast<uint4*>(dst + tile_off(rr[u], cc[u] * 8, WD * 16)) = out;
-  }
-}
 
 __device__ __forceinline__ uint4 pack8f(const uint32_t* r, float scale) {
   return make_uint4(pack_half2(__uint_as_float(r[0]) * scale, __uint_as_float(r[1]) * scale),
@@ -221,960 +197,335 @@ __device__ __forceinline__ void dump_r16(uint8_t* base, long long chunk, int k, 
     *reinterpret_cast<uint4*>(row + (((c0 + g) ^ (k & 7)) << 4)) = pack8f(w + 8 * g, 1.f);
 }
 
-template <int DX, int DV, bool FULL>
-__global__ void __launch_bounds__(NT, 1) tc_prefill_kernel(const TcArgs a) {
-  using K = Cfg<DX, DV>;
-  constexpr int F = K::F;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, part = warp >> 2;   // lane quadrant, column quarter
-  const int nrun = FULL ? a.nseg : a.nseg - 1;
-  const long long bh = blockIdx.x / nrun;
-  const int seg = static_cast<int>(blockIdx.x % nrun);
-  const int h = static_cast<int>(bh % a.H);
-  const HeadTables* T = a.tabs + h;
-  const int nch_total = (a.N + C - 1) / C;
-  const int ch0 = seg * a.seg_chunks;
-  const int ch1 = min(ch0 + a.seg_chunks, nch_total);
-
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
-  uint64_t* bar_mma = bar_tma + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
-  const uint32_t sbase = smem_u32(smem);
-
-  if (warp == 0) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
+// The CTA's schedule: its range [g0, g1) of the flattened (stream, chunk)
+// space; if the range ends inside a stream, the state-only items [gA, g1)
+// come first, then the full items [g0, g1).
+struct Sched {
+  long long g0, g1, gA;
+  int nA, nF, nch;
+  __device__ __forceinline__ Sched(long long total, int G, int c, int nch_) : nch(nch_) {
+    g0 = total * c / G;
+    g1 = total * (c + 1) / G;
+    const bool mid_end = g1 % nch != 0;
+    gA = mid_end ? max(g0, (g1 - 1) / nch * nch) : g1;
+    nA = static_cast<int>(g1 - gA);
+    nF = static_cast<int>(g1 - g0);
   }
-  if (tid == 0) {
-    mbar_init(bar_tma, 1);
-    mbar_init(bar_mma, 1);
-    fence_barrier_init();
+  __device__ __forceinline__ long long item(int i) const { return i < nA ? gA + i : g0 + (i - nA); }
+  __device__ __forceinline__ bool state_only(int i) const { return i < nA; }
+  __device__ __forceinline__ int items() const { return nA + nF; }
+};
+
+// Walks the items of a schedule in order without a 64-bit division per item:
+// (stream, chunk) advance by one chunk at a time, the stream splitting into
+// (b,h) and value block (nvb = 1 or 2 blocks, so lgv = nvb - 1) and the head
+// following the (b,h).
+struct Walker {
+  int ch, vb, bh, h;
+  __device__ __forceinline__ void seek(long long g, int nch, int nvb, int H) {
+    const long long stream = g / nch;
+    ch = static_cast<int>(g - stream * nch);
+    vb = static_cast<int>(stream & (nvb - 1));
+    bh = static_cast<int>(stream >> (nvb - 1));
+    h = bh % H;
   }
-  {  // E' table -> shared (already in canonical layout), constant tiles
-    const uint4* src = reinterpret_cast<const uint4*>(T->E);
-    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += NT) dst[i] = src[i];
-    if (FULL) {
-      const uint32_t one2 = 0x3C003C00u;   // two fp16 ones
-      if (K::MERGE) {
-        // V's extra column DV is 1 (gives den = P 1), R_Gamma's extra columns
-        // start at zero (column DV receives R_eta every chunk)
-        for (int r = tid; r < C; r += NT) {
-          *reinterpret_cast<uint4*>(smem + K::S_V + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(smem + K::S_V + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        for (int r = tid; r < KR; r += NT) {
-          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      } else {
-        uint4* ones = reinterpret_cast<uint4*>(smem + K::S_ONES);
-        for (int i = tid; i < C * 16 * 2 / 16; i += NT) ones[i] = make_uint4(one2, one2, one2, one2);
-        uint4* re = reinterpret_cast<uint4*>(smem + K::S_RE);
-        for (int i = tid; i < KR * 16 * 2 / 16; i += NT) re[i] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+  __device__ __forceinline__ void step(int nch, int nvb, int H) {
+    if (++ch < nch) return;
+    ch = 0;
+    if (++vb < nvb) return;
+    vb = 0;
+    ++bh;
+    if (++h == H) h = 0;
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  // Per-thread row constants: TMEM lane / state row k = 2m + comp.
-  const int k = 32 * quad + lane;
-  const int m = k >> 1, comp = k & 1;
-  const float2 lamC = T->lamC[m];
-  const float sgnLi = comp ? lamC.y : -lamC.y;
-  const float r2 = T->r2[m];
-  const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (16.0 * part - C / 2)));
-  const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
-  const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-  constexpr int FQ = F / 4;    // state columns per thread
-
-  // Initial (scaled) state into TMEM rows.
-  float eta_c = 0.f;
-  {
-    const float* carry = nullptr;
-    const float* carry_eta = nullptr;
-    if (FULL && seg > 0) {
-      carry = a.seg_state + ((bh * (a.nseg - 1) + (seg - 1)) * KR + k) * F;
-      carry_eta = a.seg_eta + (bh * (a.nseg - 1) + (seg - 1)) * KR + k;
-    }
-    const bool from_in = FULL && seg == 0 && a.state_in != nullptr;
-    const float2 si = T->sc_inv[m];
-#pragma unroll
-    for (int cb = 0; cb < FQ; cb += 16) {
-      const int col0 = part * FQ + cb;
-      uint32_t r[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float val = 0.f;
-        const int f = col0 + e;
-        if (carry) {
-          val = carry[f];
-        } else if (from_in) {
-          float2 x = f < DX ? a.state_in[(bh * 64 + m) * DX + f]
-                            : a.state_in[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)];
-          val = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-        }
-        r[e] = __float_as_uint(val);
-      }
-      tmem_st16(trow + K::T_STATE + col0, r);
-    }
-    if (carry_eta) {
-      eta_c = *carry_eta;
-    } else if (from_in) {
-      float2 x = a.state_in[a.BH * 64 * F + bh * 64 + m];
-      eta_c = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-    }
-    tmem_st_wait();
+  // position of item i + 1 of the schedule, after item i
+  __device__ __forceinline__ void next(const Sched& sc, int i, int nch, int nvb, int H) {
+    if (i + 1 == sc.nA) seek(sc.g0, nch, nvb, H);
+    else step(nch, nvb, H);
   }
+};
 
-  auto issue_load = [&](int ch) {
-    const int n0 = ch * C;
-    const int nv = min(C, a.N - n0);
-    const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
-    mbar_arrive_expect_tx(bar_tma, FULL ? 2 * bq + bv : bq + bv);
-    const long long row = bh * a.N + n0;
-    if (FULL) bulk_g2s(smem + K::STG_Q, a.q + row * DX, bq, bar_tma);
-    bulk_g2s(smem + K::STG_K, a.k + row * DX, bq, bar_tma);
-    bulk_g2s(smem + K::STG_V, a.v + row * DV, bv, bar_tma);
-  };
+// Range start of CTA c (same arithmetic as Sched).
+__device__ __forceinline__ long long range_lo(long long total, int G, int c) { return total * c / G; }
 
-  if (tid == 0 && ch0 < ch1) issue_load(ch0);
-  bool tma_pending = ch0 < ch1;
-  uint32_t ph_tma = 0, ph_mma = 0;
-  bool aborted = false;
-
-  auto mma_sync = [&](void) -> bool {   // wait for the last commit; uniform result
-    bool ok = mbar_wait(bar_mma, ph_mma, a.err);
-    ph_mma ^= 1u;
-    tc_fence_after();
-    return !__syncthreads_or(!ok);
-  };
-  auto to_tensor_core = [&]() {   // make thread smem / TMEM writes visible to the MMA issuer
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-  };
-
-  int nv = C;
-  for (int ch = ch0; ch < ch1; ++ch) {
-    const int n0 = ch * C;
-    nv = min(C, a.N - n0);
-    {
-      bool ok = mbar_wait(bar_tma, ph_tma, a.err);
-      ph_tma ^= 1u;
-      if (__syncthreads_or(!ok)) { aborted = true; break; }
-      tma_pending = false;
-    }
-    if (FULL) convert_all<DX, DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
-    convert_all<DX, DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
-    convert_all<DV, K::WV, false>(smem + K::STG_V, smem + K::S_V, nv, warp, lane);
-    __syncthreads();   // staging consumed
-    if (tid == 0 && ch + 1 < ch1) issue_load(ch + 1);
-    tma_pending = ch + 1 < ch1;
-
-    // ---- state: R = lambda^C S_hat -> TMEM (for GEMM7) and fp16 operands
-#pragma unroll
-    for (int cb = 0; cb < FQ; cb += 16) {
-      const int col0 = part * FQ + cb;
-      uint32_t r[16];
-      tmem_ld16(trow + K::T_STATE + col0, r);
-      tmem_ld_wait16(r);
-      uint32_t w[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float x = __uint_as_float(r[e]);
-        const float y = __shfl_xor_sync(kFull, x, 1);
-        w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
-      }
-      tmem_st16(trow + K::T_STATE + col0, w);
-      if (FULL && a.dump_R) dump_r16(a.dump_R, bh * nch_total + ch, k, col0, w);
-      if (FULL) {
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint4 pk = pack8f(w + 8 * g, 1.f);
-          const int f = col0 + 8 * g;
-          if (f < DX)
-            *reinterpret_cast<uint4*>(smem + K::S_RU + tile_off(k, f, K::RSX)) = pk;
-          else
-            *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(k, f - DX, K::RSV)) = pk;
-        }
-      }
-    }
-    tmem_st_wait();
-    {  // eta: R_eta = lambda^C eta_hat;  eta_hat <- R_eta + sum_{j<nv} E'[j]
-      const float y = __shfl_xor_sync(kFull, eta_c, 1);
-      const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
-      if (FULL && part == 0) {
-        if (a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
-        const uint4 pk = make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
-        if (K::MERGE)
-          *reinterpret_cast<uint4*>(smem + K::S_RG + tile_off(k, DV, K::RSV)) = pk;
-        else
-          *reinterpret_cast<uint4*>(smem + K::S_RE + tile_off(k, 0, 256)) = pk;
-      }
-      float add = esum_c;
-      if (nv < C) {   // ragged last chunk: partial sum of E' over the valid keys
-        double sr = 0.0, si = 0.0;
-        const double br = T->b[m].x, bi = T->b[m].y;
-        for (int j = 0; j < nv; ++j) {
-          const double e = exp((C / 2 - j) * T->re_dA[m]);
-          const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
-          double sn, cs;
-          sincos(ph, &sn, &cs);
-          const double pr = e * cs, pi = e * sn;
-          sr += br * pr - bi * pi;
-          si += br * pi + bi * pr;
-        }
-        add = static_cast<float>(comp ? si : sr);
-      }
-      eta_c = Re + add;
-    }
-    to_tensor_core();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sE = sbase + K::S_E, sK = sbase + K::S_K, sV = sbase + K::S_V;
-      if (FULL) {
-        const uint32_t sQ = sbase + K::S_Q;
-        gemm(tmem + K::T_SP, sK, 128, K::RSX, 256, sQ, 128, K::RSX, 256, idesc_f16(64, 64, 0, 0),
-             DX / 16, false);   // GEMM1: S^T
-      }
-      gemm(tmem + K::T_STATE, sE, 128, 1024, 256, sK, K::RSX, 128, 2 * K::RSX,
-           idesc_f16(128, DX, 0, 1), C / 16, true);   // GEMM7: U carry
-      gemm(tmem + K::T_STATE + DX, sE, 128, 1024, 256, sV, K::RSV, 128, 2 * K::RSV,
-           idesc_f16(128, DV, 0, 1), C / 16, true);   // GEMM7: Gamma carry
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-    if (!FULL) continue;
-
-    const int i0 = 16 * part;     // this warp's 16 columns of the 64-wide tiles
-    // The M = 64 accumulators (S^T, P, num) fill lanes 0-15 of each quadrant:
-    // thread t takes row 16 * quad + t % 16, the two half-warps splitting the
-    // warp's columns.
-    const int r16 = 16 * quad + (lane & 15), hb = lane >> 4;
-    const int c8 = i0 + 8 * hb;   // this thread's 8 columns
-    // ---- E1: S^T (M=64 rows j) -> masked fp16, MN-major B of GEMM2
-    {
-      const int j = r16;
-      uint32_t r[8];
-      tmem_ld8_halves<8>(trow + K::T_SP + i0, r);
-      tmem_ld_wait8(r);
-      const bool keep = j < nv;
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (!(keep && c8 + e >= j)) r[e] = 0u;
-      *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(j, c8, 1024)) = pack8f(r, 1.f);
-    }
-    to_tensor_core();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sE = sbase + K::S_E, sSP = sbase + K::S_SP, sQ = sbase + K::S_Q,
-                     sRU = sbase + K::S_RU;
-      gemm(tmem + K::T_A, sE, 128, 1024, 256, sSP, 1024, 128, 2048, idesc_f16(128, 64, 0, 1),
-           C / 16, false);   // GEMM2
-      gemm(tmem + K::T_A, sRU, 128, K::RSX, 256, sQ, 128, K::RSX, 256, idesc_f16(128, 64, 0, 0),
-           DX / 16, true);   // GEMM3
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-
-    // ---- E2: X = |lambda|^(2(i-c)) a~  (rows k, columns i) -> MN-major A of GEMM4/6
-    {
-      uint32_t r[16];
-      tmem_ld16(trow + K::T_A + i0, r);
-      tmem_ld_wait16(r);
-      float s = s_start;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
-        s *= r2;
-      }
-      *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0, 1024)) = pack8f(r, 1.f);
-      *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-    }
-    to_tensor_core();
-    if (tid == 0) {
-      tc_fence_after();
-      gemm(tmem + K::T_SP, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
-           idesc_f16(64, 64, 1, 1), KR / 16, false);   // GEMM4: P
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-
-    // ---- E3: P (M=64 rows i) -> masked fp16, K-major A of GEMM5
-    {
-      const int i = r16;
-      uint32_t r[8];
-      tmem_ld8_halves<8>(trow + K::T_SP + i0, r);
-      tmem_ld_wait8(r);
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (c8 + e > i) r[e] = 0u;
-      *reinterpret_cast<uint4*>(smem + K::S_SP + tile_off(i, c8, 1024)) = pack8f(r, 1.f);
-    }
-    to_tensor_core();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sSP = sbase + K::S_SP, sX = sbase + K::S_X;
-      gemm(tmem + K::T_NUM, sSP, 128, 1024, 256, sbase + K::S_V, K::RSV, 128, 2 * K::RSV,
-           idesc_f16(64, K::NV, 0, 1), C / 16, false);   // GEMM5: P [V | 1]
-      gemm(tmem + K::T_NUM, sX, 1024, 128, 2048, sbase + K::S_RG, K::RSV, 128, 2 * K::RSV,
-           idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // GEMM6: X [R_Gamma | R_eta]
-      if (!K::MERGE) {
-        gemm(tmem + K::T_DEN, sSP, 128, 1024, 256, sbase + K::S_ONES, 256, 128, 512,
-             idesc_f16(64, 16, 0, 1), C / 16, false);   // GEMM5b: P 1
-        gemm(tmem + K::T_DEN, sX, 1024, 128, 2048, sbase + K::S_RE, 256, 128, 512,
-             idesc_f16(64, 16, 1, 1), KR / 16, true);   // GEMM6b: X R_eta
-      }
-      mma_commit(bar_mma);
-    }
-    if (!mma_sync()) { aborted = true; break; }
-
-    // ---- E4: o = num / den, staged in shared memory, then written coalesced
-    {
-      const int i = r16;
-      uint32_t rd;
-      tmem_ld1(trow + K::T_DEN, rd);   // one column of all 32 lanes: rows in lanes 0-15
-      tmem_ld_wait1(rd);
-      const float dn = __shfl_sync(kFull, __uint_as_float(rd), lane & 15);
-      const float rdn = 1.0f / dn;
-      const long long row = bh * a.N + n0 + i;
-      const bool valid = i < nv;
-      if (valid && a.den && part == 0 && hb == 0) a.den[row] = dn;
-      constexpr int DQ = DV / 4;   // value columns per warp
-      static_assert(DQ == 16 || DQ == 32, "a warp's value columns split into two halves of 8 or 16");
-      constexpr int PH = DQ / 2;   // value columns per thread
-      const int f0 = part * DQ + PH * hb;
-      uint32_t r[PH];
-      if constexpr (PH == 16) {
-        tmem_ld16_halves<16>(trow + K::T_NUM + part * DQ, r);
-        tmem_ld_wait16(r);
-      } else {
-        tmem_ld8_halves<8>(trow + K::T_NUM + part * DQ, r);
-        tmem_ld_wait8(r);
-      }
-#pragma unroll
-      for (int g = 0; g < PH / 4; ++g) {
-        const int chunk = (f0 >> 2) + g;
-        *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
-            make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                        __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-      }
-      if (valid && a.num) {
-        float4* np = reinterpret_cast<float4*>(a.num + row * DV + f0);
-#pragma unroll
-        for (int g = 0; g < PH / 4; ++g)
-          np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                              __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
-      }
-      __syncthreads();
-      constexpr int CPR = DV / 4;  // 16-byte chunks per row
-      float* obase = a.o + (bh * a.N + n0) * DV;
-      for (int c = tid; c < nv * CPR; c += NT) {
-        const int rr = c / CPR, g = c % CPR;
-        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
-        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
-
-  if (!aborted) {
-    if (FULL) {
-      if (a.state_out && seg == a.nseg - 1) {
-        // state after the last token: sc * lambda^(nv - C) * S_hat = lambda^(nv-c-1) S_hat
-        const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
-        const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
-        double sn, cs;
-        sincos(ph, &sn, &cs);
-        const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
-#pragma unroll
-        for (int cb = 0; cb < FQ; cb += 16) {
-          const int col0 = part * FQ + cb;
-          uint32_t r[16];
-          tmem_ld16(trow + K::T_STATE + col0, r);
-          tmem_ld_wait16(r);
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const float x = __uint_as_float(r[e2]);
-            const float y = __shfl_xor_sync(kFull, x, 1);
-            if (comp == 0) {   // x = re, y = im
-              const float2 z = make_float2(fr * x - fi * y, fr * y + fi * x);
-              const int f = col0 + e2;
-              if (f < DX) a.state_out[(bh * 64 + m) * DX + f] = z;
-              else a.state_out[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)] = z;
-            }
-          }
-        }
-        const float y = __shfl_xor_sync(kFull, eta_c, 1);
-        if (comp == 0 && part == 0)
-          a.state_out[a.BH * 64 * F + bh * 64 + m] =
-              make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
-      }
-    } else {
-      float* dst = a.seg_state + ((bh * (a.nseg - 1) + seg) * KR + k) * F;
-#pragma unroll
-      for (int cb = 0; cb < FQ; cb += 16) {
-        const int col0 = part * FQ + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_STATE + col0, r);
-        tmem_ld_wait16(r);
-        float4* d4 = reinterpret_cast<float4*>(dst + col0);
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-          d4[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                              __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
-      }
-      if (part == 0) a.seg_eta[(bh * (a.nseg - 1) + seg) * KR + k] = eta_c;
-    }
-  } else if (tma_pending) {
-    mbar_wait(bar_tma, ph_tma, a.err);   // bounded: let our own copy land before exiting
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ---------------------------------------------------------------------------
-// Warp-specialized full pass for d_xi = d_v = 64.  tcgen05.mma issue blocks
-// the issuing thread for about as long as the tensor core works, so the
-// contractions are issued by a dedicated warp (warp 16, which also issues the
-// bulk copies) while 16 epilogue warps do the elementwise phases.  The two
-// sides hand over through mbarriers: "ready" barriers (512 epilogue-thread
-// arrivals after their shared/TMEM writes) and "done" barriers (one
-// tcgen05.commit).  Chunks are software-pipelined: the tail of chunk t-1
-// (mask P, value contractions, output) is interleaved with the head of chunk
-// t (Gram, decay contractions, readout scale), so the tensor core works on
-// one chunk while the epilogue warps work on the other.  V, R_Gamma and R_eta
-// are double-buffered; S, P, a~, num have their own TMEM tiles.
-constexpr int WS_EW = 16;                   // epilogue warps
-constexpr int WS_ET = WS_EW * 32;           // epilogue threads
-constexpr int WS_NT = WS_ET + 32;           // + one MMA / copy warp
-
-struct WCfg {
-  static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
-  static constexpr uint32_t RSX = DX * 16, RSV = WV * 16;
-  static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
-                            T_DEN = 320 + 64;
-  static constexpr uint32_t STG_Q = 0;
-  static constexpr uint32_t STG_K = STG_Q + C * DX * 2;
-  static constexpr uint32_t STG_V = STG_K + C * DX * 2;
-  static constexpr uint32_t S_Q = STG_V + C * DV * 2;
-  static constexpr uint32_t S_K = S_Q + C * DX * 2;
-  static constexpr uint32_t S_V0 = S_K + C * DX * 2;
-  static constexpr uint32_t S_V1 = S_V0 + C * WV * 2;
-  static constexpr uint32_t S_E = S_V1 + C * WV * 2;
-  static constexpr uint32_t S_S = S_E + KR * C * 2;
-  static constexpr uint32_t S_P = S_S + C * C * 2;
-  static constexpr uint32_t S_X = S_P + C * C * 2;
-  static constexpr uint32_t S_RU = S_X + KR * C * 2;
-  static constexpr uint32_t S_RG0 = S_RU + KR * DX * 2;
-  static constexpr uint32_t S_RG1 = S_RG0 + KR * WV * 2;
-  static constexpr uint32_t S_BAR = S_RG1 + KR * WV * 2;    // 10 mbarriers
-  static constexpr uint32_t S_FLAG = S_BAR + 80;
-  static constexpr uint32_t S_TMEMH = S_FLAG + 16;
-  static constexpr uint32_t SMEM = S_TMEMH + 16;
-  static constexpr uint32_t S_OUT = S_X;   // o of chunk t-1 is staged while sX is free
-  static_assert(KR * C * 2 >= C * DV * 4, "output staging fits in sX");
+// Cold paths of the prepare warps, kept out of line so that the chunk loop's
+// code stays small (the four roles run different code and share the SM's
+// instruction cache).  Each prepare thread owns TMEM lane / state row
+// k = 2m + comp and one half of the state columns.
+struct PrepThread {
+  uint32_t trow;   // this warp's TMEM lane quadrant
+  int tid, k, m, comp, half;
 };
 
-__global__ void __launch_bounds__(WS_NT, 1) tc_prefill_ws_kernel(const TcArgs a) {
-  using K = WCfg;
-  constexpr int DX = K::DX, DV = K::DV, F = K::F;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool mma_warp = warp == WS_EW;
-  const int quad = warp & 3, part = (warp >> 2) & 3;
-  const long long bh = blockIdx.x / a.nseg;
-  const int seg = static_cast<int>(blockIdx.x % a.nseg);
-  const int h = static_cast<int>(bh % a.H);
-  const HeadTables* T = a.tabs + h;
-  const int nch_total = (a.N + C - 1) / C;
-  const int ch0 = seg * a.seg_chunks;
-  const int ch1 = min(ch0 + a.seg_chunks, nch_total);
-
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
-  uint64_t* bar_tma = bars + 0;
-  uint64_t* rdy = bars + 1;     // rdy[0..3]: ready for G1+G7, G2+G3, G4, G5+G6
-  uint64_t* dne = bars + 5;     // dne[0..3]: done   "
-  uint64_t* bar_drain = bars + 9;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
-  const uint32_t sbase = smem_u32(smem);
-
-  if (warp == 0) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(bar_tma, 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(rdy + i, WS_ET);
-      mbar_init(dne + i, 1);
-    }
-    mbar_init(bar_drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(T->E);
-    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += WS_NT) dst[i] = src[i];
-    // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
-    for (int r = tid; r < C; r += WS_NT) {
-      for (int p = 0; p < 2; ++p) {
-        const uint32_t sv = p ? K::S_V1 : K::S_V0;
-        *reinterpret_cast<uint4*>(smem + sv + tile_off(r, DV, K::RSV)) = make_uint4(0x00003C00u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sv + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    for (int r = tid; r < KR; r += WS_NT) {
-      for (int p = 0; p < 2; ++p) {
-        const uint32_t sr = p ? K::S_RG1 : K::S_RG0;
-        *reinterpret_cast<uint4*>(smem + sr + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sr + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  if (mma_warp) {
-    // ------------------------------------------------ MMA and copy issuer
-    if (lane == 0) {
-      uint32_t pr[4] = {0u, 0u, 0u, 0u};
-      int issued = 0;
-      bool ok = true;
-      auto issue_load = [&](int ch) {
-        const int n0 = ch * C;
-        const int nv = min(C, a.N - n0);
-        const uint32_t bq = static_cast<uint32_t>(nv * DX * 2), bv = static_cast<uint32_t>(nv * DV * 2);
-        mbar_arrive_expect_tx(bar_tma, 2 * bq + bv);
-        const long long row = bh * a.N + n0;
-        bulk_g2s(smem + K::STG_Q, a.q + row * DX, bq, bar_tma);
-        bulk_g2s(smem + K::STG_K, a.k + row * DX, bq, bar_tma);
-        bulk_g2s(smem + K::STG_V, a.v + row * DV, bv, bar_tma);
-        ++issued;
-      };
-      auto wait_rdy = [&](int i) -> bool {
-        const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
-        pr[i] ^= 1u;
-        tc_fence_after();
-        return r;
-      };
-      auto g5g6 = [&](int pp) {
-        const uint32_t sv = sbase + (pp ? K::S_V1 : K::S_V0), srg = sbase + (pp ? K::S_RG1 : K::S_RG0);
-        gemm(tmem + K::T_NUM, sbase + K::S_P, 128, 1024, 256, sv, K::RSV, 128, 2 * K::RSV,
-             idesc_f16(64, K::NV, 0, 1), C / 16, false);   // G5: P [V | 1]
-        gemm(tmem + K::T_NUM, sbase + K::S_X, 1024, 128, 2048, srg, K::RSV, 128, 2 * K::RSV,
-             idesc_f16(64, K::NV, 1, 1), KR / 16, true);   // G6: X [R_Gamma | R_eta]
-        mma_commit(dne + 3);
-      };
-      if (ch0 < ch1) issue_load(ch0);
-      for (int t = ch0; t < ch1; ++t) {
-        const int p = (t - ch0) & 1;
-        if (!(ok = wait_rdy(0))) break;
-        if (t + 1 < ch1) issue_load(t + 1);   // staging was consumed before ready(0)
-        const uint32_t sv = sbase + (p ? K::S_V1 : K::S_V0);
-        gemm(tmem + K::T_S, sbase + K::S_K, 128, K::RSX, 256, sbase + K::S_Q, 128, K::RSX, 256,
-             idesc_f16(64, 64, 0, 0), DX / 16, false);   // G1: S^T
-        gemm(tmem + K::T_STATE, sbase + K::S_E, 128, 1024, 256, sbase + K::S_K, K::RSX, 128,
-             2 * K::RSX, idesc_f16(128, DX, 0, 1), C / 16, true);   // G7: U carry
-        gemm(tmem + K::T_STATE + DX, sbase + K::S_E, 128, 1024, 256, sv, K::RSV, 128, 2 * K::RSV,
-             idesc_f16(128, DV, 0, 1), C / 16, true);   // G7: Gamma carry
-        mma_commit(dne + 0);
-        if (t > ch0) {
-          if (!(ok = wait_rdy(3))) break;
-          g5g6(p ^ 1);
-        }
-        if (!(ok = wait_rdy(1))) break;
-        gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
-             idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
-        gemm(tmem + K::T_A, sbase + K::S_RU, 128, K::RSX, 256, sbase + K::S_Q, 128, K::RSX, 256,
-             idesc_f16(128, 64, 0, 0), DX / 16, true);   // G3
-        mma_commit(dne + 1);
-        if (!(ok = wait_rdy(2))) break;
-        gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
-             idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
-        mma_commit(dne + 2);
-      }
-      if (ok && ch0 < ch1) {
-        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) & 1);
-      }
-      if (!ok) {
-        // drain: every tensor-core group issued so far, and the last copy
-        mma_commit(bar_drain);
-        mbar_wait(bar_drain, 0u, a.err);
-        if (issued > 0) mbar_wait(bar_tma, static_cast<uint32_t>((issued - 1) & 1), a.err);
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------ epilogue warps
-    const int k = 32 * quad + lane;
-    const int m = k >> 1, comp = k & 1;
-    const float2 lamC = T->lamC[m];
-    const float sgnLi = comp ? lamC.y : -lamC.y;
-    const float r2 = T->r2[m];
-    const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (16.0 * part - C / 2)));
-    const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    constexpr int FQ = F / 4;
-    const int i0 = 16 * part;
-    uint32_t pd[4] = {0u, 0u, 0u, 0u};
-    uint32_t ptma = 0u;
-    auto wait_dne = [&](int i) -> bool {   // outcome made uniform across the epilogue warps
-      const bool r = mbar_wait_or_abort(dne + i, pd[i], a.err, abort_flag);
-      pd[i] ^= 1u;
-      tc_fence_after();
-      return !named_sync_or(2, WS_ET, !r);
-    };
-    auto signal = [&](int i) {   // my shared / TMEM writes are done: ready(i)
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(rdy + i);
-    };
-
-    float eta_c = 0.f;
-    {  // initial (scaled) state
-      const float* carry = nullptr;
-      const float* carry_eta = nullptr;
-      if (seg > 0) {
-        carry = a.seg_state + ((bh * (a.nseg - 1) + (seg - 1)) * KR + k) * F;
-        carry_eta = a.seg_eta + (bh * (a.nseg - 1) + (seg - 1)) * KR + k;
-      }
-      const bool from_in = seg == 0 && a.state_in != nullptr;
-      const float2 si = T->sc_inv[m];
-#pragma unroll
-      for (int cb = 0; cb < FQ; cb += 16) {
-        const int col0 = part * FQ + cb;
-        uint32_t r[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float val = 0.f;
-          const int f = col0 + e;
-          if (carry) {
-            val = carry[f];
-          } else if (from_in) {
-            float2 x = f < DX ? a.state_in[(bh * 64 + m) * DX + f]
-                              : a.state_in[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)];
-            val = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-          }
-          r[e] = __float_as_uint(val);
-        }
-        tmem_st16(trow + K::T_STATE + col0, r);
-      }
-      if (carry_eta) {
-        eta_c = *carry_eta;
-      } else if (from_in) {
-        float2 x = a.state_in[a.BH * 64 * F + bh * 64 + m];
-        eta_c = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-      }
-      tmem_st_wait();
-    }
-
-    int nv_last = C;
-    // chunk ch, buffer parity p: convert inputs, rotate the state, signal ready(0)
-    auto prepare = [&](int ch, int p) -> bool {
-      const int nv = min(C, a.N - ch * C);
-      nv_last = nv;
-      const bool r = mbar_wait_or_abort(bar_tma, ptma, a.err, abort_flag);
-      ptma ^= 1u;
-      if (named_sync_or(2, WS_ET, !r)) return false;
-      const uint32_t sv = p ? K::S_V1 : K::S_V0, srg = p ? K::S_RG1 : K::S_RG0;
-      convert_all<DX, DX, true>(smem + K::STG_Q, smem + K::S_Q, nv, warp, lane);
-      convert_all<DX, DX, true>(smem + K::STG_K, smem + K::S_K, nv, warp, lane);
-      convert_all<DV, K::WV, false>(smem + K::STG_V, smem + sv, nv, warp, lane);
-      static_assert(FQ == 32, "two 16-column blocks per thread");
-      uint32_t rs[2][16];
-      tmem_ld16(trow + K::T_STATE + part * FQ, rs[0]);
-      tmem_ld16(trow + K::T_STATE + part * FQ + 16, rs[1]);
-      tmem_ld_wait16(rs[0]);
-      tmem_ld_wait16(rs[1]);
-#pragma unroll
-      for (int cb = 0; cb < FQ; cb += 16) {
-        const int col0 = part * FQ + cb;
-        uint32_t (&rr)[16] = rs[cb / 16];
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float x = __uint_as_float(rr[e]);
-          const float y = __shfl_xor_sync(kFull, x, 1);
-          w[e] = __float_as_uint(fmaf(lamC.x, x, sgnLi * y));
-        }
-        tmem_st16(trow + K::T_STATE + col0, w);
-        if (a.dump_R) dump_r16(a.dump_R, bh * nch_total + ch, k, col0, w);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint4 pk = pack8f(w + 8 * g, 1.f);
-          const int f = col0 + 8 * g;
-          if (f < DX)
-            *reinterpret_cast<uint4*>(smem + K::S_RU + tile_off(k, f, K::RSX)) = pk;
-          else
-            *reinterpret_cast<uint4*>(smem + srg + tile_off(k, f - DX, K::RSV)) = pk;
-        }
-      }
-      tmem_st_wait();
-      {
-        const float y = __shfl_xor_sync(kFull, eta_c, 1);
-        const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
-        if (part == 0) {
-          if (a.dump_Re) a.dump_Re[(bh * nch_total + ch) * KR + k] = Re;
-          *reinterpret_cast<uint4*>(smem + srg + tile_off(k, DV, K::RSV)) =
-              make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
-        }
-        float add = esum_c;
-        if (nv < C) {
-          double sr = 0.0, si = 0.0;
-          const double br = T->b[m].x, bi = T->b[m].y;
-          for (int j = 0; j < nv; ++j) {
-            const double e = exp((C / 2 - j) * T->re_dA[m]);
-            const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
-            double sn, cs;
-            sincos(ph, &sn, &cs);
-            const double pr = e * cs, pi = e * sn;
-            sr += br * pr - bi * pi;
-            si += br * pi + bi * pr;
-          }
-          add = static_cast<float>(comp ? si : sr);
-        }
-        eta_c = Re + add;
-      }
-      signal(0);
-      return true;
-    };
-    auto e3 = [&]() {   // masked P -> [i][j]
-      const int i = 16 * quad + lane;
-      uint32_t r[16];
-      tmem_ld16(trow + K::T_P + i0, r);
-      tmem_ld_wait16(r);
-      if (lane < 16) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (i0 + e > i) r[e] = 0u;
-        *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0, 1024)) = pack8f(r, 1.f);
-        *reinterpret_cast<uint4*>(smem + K::S_P + tile_off(i, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-      }
-      signal(3);
-    };
-    auto e4 = [&](int ch, int nv) {   // o = num / den, staged then written coalesced
-      const int n0 = ch * C;
-      const int i = 16 * quad + lane;
-      uint32_t rd[16], r[16];
-      tmem_ld16(trow + K::T_DEN, rd);
-      tmem_ld16(trow + K::T_NUM + i0, r);
-      tmem_ld_wait16(rd);
-      tmem_ld_wait16(r);
-      const float dn = __uint_as_float(rd[0]);
-      const float rdn = 1.0f / dn;
-      const long long row = bh * a.N + n0 + i;
-      if (lane < 16) {
-        if (i < nv && a.den && part == 0) a.den[row] = dn;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int chunk = (i0 >> 2) + g;
-          *reinterpret_cast<float4*>(smem + K::S_OUT + i * DV * 4 + ((chunk ^ (i & 7)) << 4)) =
-              make_float4(__uint_as_float(r[4 * g]) * rdn, __uint_as_float(r[4 * g + 1]) * rdn,
-                          __uint_as_float(r[4 * g + 2]) * rdn, __uint_as_float(r[4 * g + 3]) * rdn);
-        }
-        if (i < nv && a.num) {
-          float4* np = reinterpret_cast<float4*>(a.num + row * DV + i0);
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-            np[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
-                                __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
-        }
-      }
-      named_sync(1, WS_ET);
-      constexpr int CPR = DV / 4;
-      float* obase = a.o + (bh * a.N + n0) * DV;
-      for (int c = tid; c < nv * CPR; c += WS_ET) {
-        const int rr = c / CPR, g = c % CPR;
-        const float4 x = *reinterpret_cast<const float4*>(smem + K::S_OUT + rr * DV * 4 + ((g ^ (rr & 7)) << 4));
-        *reinterpret_cast<float4*>(obase + rr * DV + 4 * g) = x;
-      }
-      named_sync(1, WS_ET);   // staging (sX) is read before E2 of the next chunk writes it
-    };
-
-    bool ok = true;
-    int prev = -1, prev_nv = C;
-    if (ch0 < ch1) ok = prepare(ch0, 0);
-    for (int t = ch0; ok && t < ch1; ++t) {
-      const int nv = min(C, a.N - t * C);
-      if (prev >= 0) {
-        if (!(ok = wait_dne(2))) break;   // G4(t-1)
-        e3();
-      }
-      if (!(ok = wait_dne(0))) break;     // G1 + G7(t)
-      {  // E1(t): masked S^T -> [j][i]
-        const int j = 16 * quad + lane;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_S + i0, r);
-        tmem_ld_wait16(r);
-        if (lane < 16) {
-          const bool keep = j < nv;
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (!(keep && i0 + e >= j)) r[e] = 0u;
-          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0, 1024)) = pack8f(r, 1.f);
-          *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-        }
-        signal(1);
-      }
-      if (prev >= 0) {
-        if (!(ok = wait_dne(3))) break;   // G5 + G6(t-1)
-        e4(prev, prev_nv);
-      }
-      if (!(ok = wait_dne(1))) break;     // G2 + G3(t)
-      {  // E2(t): X = |lambda|^(2(i-c)) a~
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_A + i0, r);
-        tmem_ld_wait16(r);
-        float s = s_start;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          r[e] = __float_as_uint(__uint_as_float(r[e]) * s);
-          s *= r2;
-        }
-        *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0, 1024)) = pack8f(r, 1.f);
-        *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 8, 1024)) = pack8f(r + 8, 1.f);
-        signal(2);
-      }
-      prev = t;
-      prev_nv = nv;
-      if (t + 1 < ch1) ok = prepare(t + 1, (t + 1 - ch0) & 1);
-    }
-    if (ok && prev >= 0) {
-      if ((ok = wait_dne(2))) e3();
-      if (ok && (ok = wait_dne(3))) e4(prev, prev_nv);
-    }
-    if (ok && a.state_out && seg == a.nseg - 1) {
-      const int nv = nv_last;
-      const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
-      const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
-      double sn, cs;
-      sincos(ph, &sn, &cs);
-      const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
-#pragma unroll
-      for (int cb = 0; cb < FQ; cb += 16) {
-        const int col0 = part * FQ + cb;
-        uint32_t r[16];
-        tmem_ld16(trow + K::T_STATE + col0, r);
-        tmem_ld_wait16(r);
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const float x = __uint_as_float(r[e2]);
-          const float y = __shfl_xor_sync(kFull, x, 1);
-          if (comp == 0) {
-            const float2 z = make_float2(fr * x - fi * y, fr * y + fi * x);
-            const int f = col0 + e2;
-            if (f < DX) a.state_out[(bh * 64 + m) * DX + f] = z;
-            else a.state_out[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)] = z;
-          }
-        }
-      }
-      const float y = __shfl_xor_sync(kFull, eta_c, 1);
-      if (comp == 0 && part == 0)
-        a.state_out[a.BH * 64 * F + bh * 64 + m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+// lambda_m^n in fp64 from the table's Delta A (phase reduced modulo 2 pi)
+__device__ __noinline__ void lam_pow(const HeadTables* T, int m, double n, double* pr, double* pi) {
+  const double e = exp(n * T->re_dA[m]);
+  const double ph = fmod(n * T->im_dA[m], 6.283185307179586476925);
+  double sn, cs;
+  sincos(ph, &sn, &cs);
+  *pr = e * cs;
+  *pi = e * sn;
 }
 
-// ---------------------------------------------------------------------------
-// Two-group warp-specialized full pass for d_xi = d_v = 64.  Four roles run
-// concurrently: 8 "prepare" warps (0-7) convert the inputs and rotate the
-// carried state into R(t); 8 "output" warps (8-15) run the masks, readout
-// scale and o = num/den of chunks t and t-1; warp 16 issues every
-// tensor-core contraction; warp 17 brings q, k, v in with TMA tensor loads
-// that land directly in the operand layout, where the prepare warps convert
-// them in place, so there is no staging area.  A 64-row box arrives as 64
-// rows of 128 bytes in the 128-byte swizzled layout, which the tensor core
-// reads as a K-major (features along K) or an MN-major (tokens along K)
-// operand alike.  Rows past the sequence arrive as zeros.
-// R_U, the A operand of G3, is written to tensor memory as fp16 pairs, and o
-// leaves through TMA tensor stores from a double-buffered staging area, so
-// neither waits on the other side.  q, k, v and R_Gamma have three buffer sets and
-// R_U two: the fetch warp refills a set as soon as the contractions of the
-// chunk it held are done, about two chunks ahead of its use.  Handover is by
-// mbarriers: loaded(set) from the copies, ready(0) from the prepare warps,
-// ready(1..3) from the output warps, done(0..3) and the buffer releases
-// (freeQK after G2+G3, freeVR after G5+G6) from tcgen05.commit.
-constexpr int W2_GW = 8;                       // warps per epilogue group
-constexpr int W2_GT = W2_GW * 32;              // threads per epilogue group
-constexpr int W2_NT = 2 * W2_GT + 64;          // + the MMA warp and the fetch warp
+// component comp of sum_{j < nv} E'[j, m]: the constant channel's carry of
+// a ragged last chunk
+__device__ __noinline__ float ragged_esum(const HeadTables* T, int m, int comp, int nv) {
+  double sr = 0.0, si = 0.0;
+  const double br = T->b[m].x, bi = T->b[m].y;
+  for (int j = 0; j < nv; ++j) {
+    double pr, pi;
+    lam_pow(T, m, C / 2 - j, &pr, &pi);
+    sr += br * pr - bi * pi;
+    si += br * pi + bi * pr;
+  }
+  return static_cast<float>(comp ? si : sr);
+}
 
-struct W2Cfg {
-  static constexpr int DX = 64, DV = 64, F = 128, WV = 80, NV = 80;
-  static constexpr uint32_t RSV = WV * 16;
-  static constexpr uint32_t T_STATE = 0, T_A = 128, T_S = 192, T_P = 256, T_NUM = 320,
-                            T_DEN = 320 + 64, T_RU = 400;   // T_RU: [2] x 32 columns of fp16 pairs
-  static constexpr uint32_t TQ = C * DX * 2, TV = C * DV * 2, TRG = KR * WV * 2;
-  static constexpr uint32_t TO = C * DV * 4;               // o of one chunk: two 64 x 128-byte boxes
-  static constexpr int NB = 3;                             // q, k, v and R_Gamma buffer sets
-  static constexpr uint32_t TIN = C * 64 * 2;              // bytes of one TMA box (64 rows x 64 bf16)
-  static constexpr uint32_t SW = 1024;                     // one swizzle atom: 8 rows x 128 bytes
-  static constexpr uint32_t S_Q = 0;                       // [NB]
-  static constexpr uint32_t S_K = S_Q + NB * TQ;           // [NB]
-  static constexpr uint32_t S_V = S_K + NB * TQ;           // [NB]
-  static constexpr uint32_t S_ONES = S_V + NB * TV;        // [V | 1]: MN-block 64..127 of G5's B operand
-  static constexpr uint32_t S_E = S_ONES + TV;
-  static constexpr uint32_t S_S = S_E + KR * C * 2;
-  static constexpr uint32_t S_P = S_S + C * C * 2;
-  static constexpr uint32_t S_X = S_P + C * C * 2;
-  static constexpr uint32_t S_O = S_X + KR * C * 2;        // [2] o staging, 128-byte swizzled
-  static constexpr uint32_t S_RG = S_O + 2 * TO;           // [NB]
-  static constexpr uint32_t S_BAR = S_RG + NB * TRG;       // 18 mbarriers
-  static constexpr uint32_t S_FLAG = S_BAR + 256;
-  static constexpr uint32_t S_TMEMH = S_FLAG + 16;
-  static constexpr uint32_t SMEM = S_TMEMH + 16;
-  static_assert(SMEM <= 232448, "fits one CTA's opt-in shared memory");
-  static_assert(S_O % 1024 == 0 && S_K % 1024 == 0 && S_V % 1024 == 0 && S_ONES % 1024 == 0,
-                "swizzled tiles start on the 128-byte swizzle period");
-};
+// state column f of row m in the public layout (complex): U for f < DX,
+// else column vb * 64 + f - DX of Gamma
+template <int DX>
+__device__ __forceinline__ long long pub_index(const TcArgs& a, long long bh, int m, int vb, int f) {
+  return f < DX ? (bh * 64 + m) * DX + f : a.BH * 64 * DX + (bh * 64 + m) * a.DV + vb * kVB + (f - DX);
+}
 
-__global__ void __launch_bounds__(W2_NT, 1)
-    tc_prefill_ws2_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
-                          const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                          const __grid_constant__ CUtensorMap tm_o) {
-  using K = W2Cfg;
-  constexpr int DX = K::DX, DV = K::DV, F = K::F, NB = K::NB;
+template <int DX>
+__device__ __noinline__ void prep_zero(const PrepThread& th) {
+  constexpr int FH = PCfg<DX>::FH;
+  uint32_t z[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) z[e] = 0u;
+  for (int cb = 0; cb < FH; cb += 16) tmem_st16(th.trow + PCfg<DX>::T_STATE + th.half * FH + cb, z);
+  tmem_st_wait();
+}
+
+// initial scaled state of a piece from state_in (zero without it); returns
+// this row's eta
+template <int DX>
+__device__ __noinline__ float prep_init_from_input(const TcArgs& a, const HeadTables* T, const PrepThread& th,
+                                                  long long bh, int vb) {
+  constexpr int FH = PCfg<DX>::FH;
+  if (!a.state_in) {
+    prep_zero<DX>(th);
+    return 0.f;
+  }
+  const float2 si = T->sc_inv[th.m];
+  for (int cb = 0; cb < FH; cb += 16) {
+    const int col0 = th.half * FH + cb;
+    uint32_t r[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float2 x = a.state_in[pub_index<DX>(a, bh, th.m, vb, col0 + e)];
+      r[e] = __float_as_uint(th.comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y));
+    }
+    tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
+  }
+  tmem_st_wait();
+  const float2 x = a.state_in[a.BH * 64 * (DX + a.DV) + bh * 64 + th.m];
+  return th.comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
+}
+
+// the state after the last token of a stream: sc lambda^(nv - C) S_hat = lambda^(nv-c-1) S_hat
+template <int DX>
+__device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTables* T, const PrepThread& th,
+                                                  long long bh, int vb, int ch, float eta_c) {
+  constexpr int FH = PCfg<DX>::FH;
+  const int nv = a.N - ch * C;
+  double pr, pi;
+  lam_pow(T, th.m, nv - C / 2 - 1, &pr, &pi);
+  const float fr = static_cast<float>(pr), fi = static_cast<float>(pi);
+  for (int cb = 0; cb < FH; cb += 16) {
+    const int col0 = th.half * FH + cb;
+    uint32_t r[16];
+    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_ld_wait16(r);
+#pragma unroll
+    for (int e2 = 0; e2 < 16; ++e2) {
+      const float x = __uint_as_float(r[e2]);
+      const float y = __shfl_xor_sync(kFull, x, 1);
+      const int f = col0 + e2;
+      if (th.comp == 0 && (f >= DX || vb == 0))   // U is the same in every value block
+        a.state_out[pub_index<DX>(a, bh, th.m, vb, f)] = make_float2(fr * x - fi * y, fr * y + fi * x);
+    }
+  }
+  const float y = __shfl_xor_sync(kFull, eta_c, 1);
+  if (th.comp == 0 && th.half == 0 && vb == 0)
+    a.state_out[a.BH * 64 * (DX + a.DV) + bh * 64 + th.m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
+}
+
+// this thread's part of the TMEM state (and eta) -> dst [128 * F + 128]
+template <int DX>
+__device__ __noinline__ void prep_publish(const PrepThread& th, float* dst, float eta_c) {
+  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  for (int cb = 0; cb < FH; cb += 16) {
+    const int col0 = th.half * FH + cb;
+    uint32_t r[16];
+    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_ld_wait16(r);
+    float4* d4 = reinterpret_cast<float4*>(dst + th.k * F + col0);
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      d4[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
+                          __uint_as_float(r[4 * g + 3]));
+  }
+  if (th.half == 0) dst[KR * F + th.k] = eta_c;
+}
+
+// every prepare thread's stores are visible GPU-wide before one thread raises
+// the flag (release)
+__device__ __noinline__ void prep_raise_flag(int* flag, int value, int tid) {
+  __threadfence();
+  named_sync(4, GT);
+  if (tid == 0) st_release(flag, value);
+}
+
+// TMEM state (and eta) += (mr + i mi) src, complex per mode (rows 2m, 2m+1)
+template <int DX>
+__device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* src, double mr, double mi, float* eta) {
+  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  const float fr = static_cast<float>(mr), fs = static_cast<float>(th.comp ? mi : -mi);
+  for (int cb = 0; cb < FH; cb += 16) {
+    const int col0 = th.half * FH + cb;
+    uint32_t r[16];
+    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    float x[16];
+    const float4* s4 = reinterpret_cast<const float4*>(src + th.k * F + col0);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const float4 v4 = __ldcg(s4 + g);
+      x[4 * g] = v4.x; x[4 * g + 1] = v4.y; x[4 * g + 2] = v4.z; x[4 * g + 3] = v4.w;
+    }
+    tmem_ld_wait16(r);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float y = __shfl_xor_sync(kFull, x[e], 1);
+      r[e] = __float_as_uint(__uint_as_float(r[e]) + fmaf(fr, x[e], fs * y));
+    }
+    tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
+  }
+  tmem_st_wait();
+  const float xe = __ldcg(src + KR * F + th.k);
+  const float ye = __shfl_xor_sync(kFull, xe, 1);
+  *eta += fmaf(fr, xe, fs * ye);
+}
+
+// Carry into a first piece that starts inside a stream: the sum over
+// predecessors p = c-1, c-2, ... of lambda^(C n) times their published end
+// states, n counting the chunks between p's piece and ours; stops at the
+// first inclusive state.  Leaves the carry in the TMEM state and *eta.
+// Returns false if a wait gave up (uniform over the prepare group).
+template <int DX>
+__device__ __noinline__ bool prep_look_back(const TcArgs& a, const HeadTables* T, const PrepThread& th,
+                                            volatile int* abort_flag, volatile int* xchg, float* eta) {
+  constexpr int STRIDE = KR * PCfg<DX>::F + KR;
+  prep_zero<DX>(th);
+  *eta = 0.f;
+  double mr = 1.0, mi = 0.0;
+  for (int p = static_cast<int>(blockIdx.x) - 1; p >= 0; --p) {
+    if (th.tid == 0) {   // poll the predecessor's flag (bounded)
+      int f = ld_acquire(a.flags + p);
+      const unsigned long long t0 = global_ns();
+      while (f == 0 && !*abort_flag) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          atomicOr(a.err, kErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        f = ld_acquire(a.flags + p);
+      }
+      *xchg = *abort_flag ? 0 : f;
+    }
+    named_sync(4, GT);
+    const int f = *xchg;
+    named_sync(4, GT);
+    if (f == 0) return false;
+    __threadfence();
+    prep_accumulate<DX>(th, (f == 2 ? a.incl : a.agg) + static_cast<long long>(p) * STRIDE, mr, mi, eta);
+    if (f == 2) return true;
+    // p published a local state only: its last piece starts inside the
+    // stream, so continue with p - 1 one piece further back
+    const long long p_lo = range_lo(a.total, a.G, p), p_hi = range_lo(a.total, a.G, p + 1);
+    const long long n = p_hi - max(p_lo, (p_hi - 1) / a.nch * a.nch);
+    double lr, li;
+    lam_pow(T, th.m, static_cast<double>(C) * n, &lr, &li);
+    const double nr = mr * lr - mi * li;
+    mi = mr * li + mi * lr;
+    mr = nr;
+  }
+  return false;   // unreachable: the stream's first piece publishes an inclusive state
+}
+
+// A CTA whose one piece lies inside a stream publishes its inclusive end
+// state once its carry (in TMEM, eta) is known: local + lambda^(C n) carry.
+template <int DX>
+__device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadTables* T, const PrepThread& th,
+                                                    int n, float eta_c) {
+  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH, STRIDE = KR * F + KR;
+  double lr, li;
+  lam_pow(T, th.m, static_cast<double>(C) * n, &lr, &li);
+  const float fr = static_cast<float>(lr), fs = static_cast<float>(th.comp ? li : -li);
+  const float* loc = a.agg + static_cast<long long>(blockIdx.x) * STRIDE;
+  float* dst = a.incl + static_cast<long long>(blockIdx.x) * STRIDE;
+  for (int cb = 0; cb < FH; cb += 16) {
+    const int col0 = th.half * FH + cb;
+    uint32_t r[16];
+    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_ld_wait16(r);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float x = __uint_as_float(r[e]);
+      const float y = __shfl_xor_sync(kFull, x, 1);
+      dst[th.k * F + col0 + e] = loc[th.k * F + col0 + e] + fmaf(fr, x, fs * y);
+    }
+  }
+  const float y = __shfl_xor_sync(kFull, eta_c, 1);
+  if (th.half == 0) dst[KR * F + th.k] = loc[KR * F + th.k] + fmaf(fr, eta_c, fs * y);
+  prep_raise_flag(a.flags + blockIdx.x, 2, th.tid);
+}
+
+// 576 threads: one SM sub-partition carries five of the 18 warps, so its
+// 16 K registers cap a thread at 96.
+template <int DX>
+__global__ void __launch_bounds__(NTH, 1)
+    tc_prefill_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o) {
+  using K = PCfg<DX>;
+  constexpr int F = K::F, FH = K::FH, NB = K::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int role = warp < 2 * W2_GW ? warp / W2_GW : warp - 2 * W2_GW + 2;   // prepare, output, mma, fetch
-  const int gw = warp & (W2_GW - 1);          // warp index within its epilogue group
+  const int role = warp < 2 * GW ? warp / GW : warp - 2 * GW + 2;   // prepare, output, mma, fetch
+  const int gw = warp & (GW - 1);          // warp index within its epilogue group
   const int quad = warp & 3, half = gw >> 2;
-  const long long bh = blockIdx.x / a.nseg;
-  const int seg = static_cast<int>(blockIdx.x % a.nseg);
-  const int h = static_cast<int>(bh % a.H);
-  const HeadTables* T = a.tabs + h;
-  const int nch_total = (a.N + C - 1) / C;
-  const int ch0 = seg * a.seg_chunks;
-  const int ch1 = min(ch0 + a.seg_chunks, nch_total);
+  const Sched sc(a.total, a.G, blockIdx.x, a.nch);
+  const int nI = sc.items();
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
-  uint64_t* rdy = bars + 0;       // [4]
-  uint64_t* dne = bars + 4;       // [4]
-  uint64_t* freeQK = bars + 8;    // [NB]: sQ, sK of that set (and the sR_U it was read with) reusable
-  uint64_t* freeVR = bars + 11;   // [NB]: sV, sR_Gamma of that set reusable
-  uint64_t* bar_drain = bars + 14;
-  uint64_t* loaded = bars + 15;   // [NB]: that set's q, k, v rows have landed
+  uint64_t* rdy = bars + 0;       // [4]: prepare -> G7 (+G1), output -> G2G3, G4, G5G6
+  uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
+  uint64_t* dneS = bars + 8;      // G1 done
+  uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
+  uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
+  uint64_t* bar_drain = bars + 15;
+  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
   const uint32_t sbase = smem_u32(smem);
   auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
   auto sK = [&](int b) { return K::S_K + b * K::TQ; };
   auto sV = [&](int b) { return K::S_V + b * K::TV; };
   auto sRG = [&](int b) { return K::S_RG + b * K::TRG; };
+  // stream s = bh * nvb + vb
+  auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
 
   if (warp == 0) {
     tmem_alloc(tmem_holder, 512);
@@ -1182,9 +533,10 @@ __global__ void __launch_bounds__(W2_NT, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) {
-      mbar_init(rdy + i, W2_GT);
+      mbar_init(rdy + i, i == 0 ? GT : GT);
       mbar_init(dne + i, 1);
     }
+    mbar_init(dneS, 1);
     for (int i = 0; i < NB; ++i) {
       mbar_init(freeQK + i, 1);
       mbar_init(freeVR + i, 1);
@@ -1195,29 +547,39 @@ __global__ void __launch_bounds__(W2_NT, 1)
     fence_barrier_init();
   }
   {
-    // V's extra column DV is 1 (den = P 1); R_Gamma's extra columns start at 0
-    // the ones column after V: MN element 64 (first of the second 64-block)
+    // the ones block after V: MN element 64 (first of the second 64-block)
     // is 1 in every row, the rest 0, in the swizzled layout
-    for (int i = tid; i < C * 8; i += W2_NT) {
+    for (int i = tid; i < C * 8; i += NTH) {
       const int r = i >> 3, c = i & 7;
       *reinterpret_cast<uint4*>(smem + K::S_ONES + r * 128 + c * 16) =
           make_uint4((c == (r & 7)) ? 0x00003C00u : 0u, 0u, 0u, 0u);
     }
-    for (int r = tid; r < KR; r += W2_NT) {
+    // R_Gamma's extra columns start at zero (column 64 receives R_eta every chunk)
+    for (int r = tid; r < KR; r += NTH) {
       for (int b = 0; b < NB; ++b) {
-        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, DV, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, DV + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     // Everything above touches only this CTA's own resources.  The kernel may
-    // have been launched while the previous kernel of the stream (the table
-    // prologue, or the segment carry scan) still runs: every global read of
-    // the tables, carries and inputs comes after this wait, and nothing global
-    // is written before it.
+    // have been launched while the table kernel before it still runs: every
+    // global read (tables, inputs, look-back flags, which the table kernel
+    // clears) comes after this wait, and nothing global is written before it.
     griddep_wait();
-    const uint4* src = reinterpret_cast<const uint4*>(T->E);
+  }
+  // The E' table depends on the head; a CTA may span heads, so it is copied
+  // per piece by the prepare warps (see load_table) -- except that the first
+  // item's head is loaded here by everyone.
+  int h_first = 0;
+  {
+    Walker w;
+    first_item(w);
+    h_first = w.h;
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h_first].E);
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += W2_NT) dst[i] = src[i];
+    for (int i = tid; i < KR * C * 2 / 16; i += NTH) dst[i] = src[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -1235,12 +597,24 @@ __global__ void __launch_bounds__(W2_NT, 1)
         tc_fence_after();
         return r;
       };
-      // contraction over ksteps K-steps of 16 with prebuilt descriptors; the
-      // start addresses advance by astep / bstep bytes per step
       auto gemm_d = [&](uint32_t d, uint64_t ad, uint32_t astep, uint64_t bd, uint32_t bstep, uint32_t idesc,
                         int ksteps, bool acc) {
         for (int kk = 0; kk < ksteps; ++kk)
           mma_f16(d, ad + ((kk * astep) >> 4), bd + ((kk * bstep) >> 4), idesc, (kk > 0 || acc) ? 1u : 0u);
+      };
+      auto g1 = [&](int b) {   // S^T = xi(K) xi(Q)^T, K-major swizzled tiles of DX / 64 boxes
+        for (int kk = 0; kk < DX / 16; ++kk)
+          mma_f16(tmem + K::T_S, smem_desc_sw128(sbase + sK(b) + K::kstep(kk), 16, K::SW),
+                  smem_desc_sw128(sbase + sQ(b) + K::kstep(kk), 16, K::SW), idesc_f16(64, 64, 0, 0),
+                  kk > 0 ? 1u : 0u);
+      };
+      auto g7 = [&](int b) {   // S_hat += E'^T [xi(K) | V]
+        gemm_d(tmem + K::T_STATE, smem_desc(sbase + K::S_E, 128, 1024), 256,
+               smem_desc_sw128(sbase + sK(b), K::BOX, K::SW), 2 * K::SW, idesc_f16(128, DX, 0, 1), C / 16,
+               true);
+        gemm_d(tmem + K::T_STATE + DX, smem_desc(sbase + K::S_E, 128, 1024), 256,
+               smem_desc_sw128(sbase + sV(b), K::S_ONES - sV(b), K::SW), 2 * K::SW, idesc_f16(128, kVB, 0, 1),
+               C / 16, true);
       };
       auto g5g6 = [&](int bb) {
         gemm_d(tmem + K::T_NUM, smem_desc(sbase + K::S_P, 128, 1024), 256,
@@ -1251,38 +625,51 @@ __global__ void __launch_bounds__(W2_NT, 1)
         mma_commit(dne + 3);
         mma_commit(freeVR + bb);
       };
-      for (int t = ch0; t < ch1; ++t) {
-        const int rel = t - ch0, b = rel % NB, p = rel & 1;
+      int t = 0, prev_b = 0;   // full items issued so far; set of the previous full item
+      for (int i = 0; i < nI; ++i) {
+        const int b = i % NB, p = i & 1;
         if (!(ok = wait_rdy(0))) break;
-        gemm_d(tmem + K::T_S, smem_desc_sw128(sbase + sK(b), 16, K::SW), 32,
-               smem_desc_sw128(sbase + sQ(b), 16, K::SW), 32, idesc_f16(64, 64, 0, 0), DX / 16,
-               false);   // G1: S^T
-        gemm_d(tmem + K::T_STATE, smem_desc(sbase + K::S_E, 128, 1024), 256,
-               smem_desc_sw128(sbase + sK(b), K::TQ, K::SW), 2 * K::SW, idesc_f16(128, DX, 0, 1), C / 16,
-               true);   // G7: U carry
-        gemm_d(tmem + K::T_STATE + DX, smem_desc(sbase + K::S_E, 128, 1024), 256,
-               smem_desc_sw128(sbase + sV(b), K::S_ONES - sV(b), K::SW), 2 * K::SW, idesc_f16(128, DV, 0, 1),
-               C / 16, true);   // G7: Gamma carry
+        if (sc.state_only(i)) {
+          g7(b);
+          mma_commit(dne + 0);
+          mma_commit(freeQK + b);
+          mma_commit(freeVR + b);
+          continue;
+        }
+        if (!K::SHARED_SAP) {
+          g1(b);
+          mma_commit(dneS);
+        }
+        g7(b);
         mma_commit(dne + 0);
-        if (t > ch0) {
-          if (!(ok = wait_rdy(3))) break;
-          g5g6((rel + NB - 1) % NB);
+        if (t > 0) {
+          if (!(ok = wait_rdy(3))) break;   // E3 of the previous chunk: P read
+          if (K::SHARED_SAP) {
+            g1(b);
+            mma_commit(dneS);
+          }
+          g5g6(prev_b);
+        } else if (K::SHARED_SAP) {
+          g1(b);
+          mma_commit(dneS);
         }
         if (!(ok = wait_rdy(1))) break;
         gemm(tmem + K::T_A, sbase + K::S_E, 128, 1024, 256, sbase + K::S_S, 1024, 128, 2048,
              idesc_f16(128, 64, 0, 1), C / 16, false);   // G2
         for (int kk = 0; kk < DX / 16; ++kk)   // G3: A = R_U from tensor memory
-          mma_f16_ts(tmem + K::T_A, tmem + K::T_RU + 32 * p + 8 * kk,
-                     smem_desc_sw128(sbase + sQ(b) + 32 * kk, 16, K::SW), idesc_f16(128, 64, 0, 0), 1u);
+          mma_f16_ts(tmem + K::T_A, tmem + K::T_RU + K::RU_COLS * p + 8 * kk,
+                     smem_desc_sw128(sbase + sQ(b) + K::kstep(kk), 16, K::SW), idesc_f16(128, 64, 0, 0), 1u);
         mma_commit(dne + 1);
         mma_commit(freeQK + b);
         if (!(ok = wait_rdy(2))) break;
         gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
              idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
         mma_commit(dne + 2);
+        prev_b = b;
+        ++t;
       }
-      if (ok && ch0 < ch1) {
-        if ((ok = wait_rdy(3))) g5g6((ch1 - 1 - ch0) % NB);
+      if (ok && t > 0) {
+        if ((ok = wait_rdy(3))) g5g6(prev_b);
       }
       if (!ok) {   // drain every tensor-core group issued so far
         mma_commit(bar_drain);
@@ -1294,110 +681,143 @@ __global__ void __launch_bounds__(W2_NT, 1)
     // ------------------------------------------------ prepare warps
     const int k = 32 * quad + lane;
     const int m = k >> 1, comp = k & 1;
-    const float2 lamC = T->lamC[m];
-    const float sgnLi = comp ? lamC.y : -lamC.y;
-    const uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
-    const float esum_c = comp ? T->esum[m].y : T->esum[m].x;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    constexpr int FH = F / 2;   // state columns per thread
-    uint32_t pd0 = 0u, pld[NB] = {0u, 0u, 0u};
+    uint32_t pd0 = 0u, pld = 0u;   // parities; pld bit b for buffer set b
+    int cur_h = h_first;
+    const HeadTables* T = a.tabs + cur_h;
+    float2 lamC = T->lamC[m];
+    float sgnLi = comp ? lamC.y : -lamC.y;
+    uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
+    float esum_c = comp ? T->esum[m].y : T->esum[m].x;
+    auto set_head = [&](int h) {   // per-mode constants of head h
+      cur_h = h;
+      T = a.tabs + h;
+      lamC = T->lamC[m];
+      sgnLi = comp ? lamC.y : -lamC.y;
+      lamC2 = f2_pack(lamC.x, lamC.x);
+      sgnLi2 = f2_pack(sgnLi, sgnLi);
+      esum_c = comp ? T->esum[m].y : T->esum[m].x;
+    };
     auto waitA = [&](uint64_t* bar, uint32_t& ph) -> bool {   // uniform over the prepare group
       const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
       ph ^= 1u;
       tc_fence_after();
-      return !named_sync_or(2, W2_GT, !r);
+      return !named_sync_or(2, GT, !r);
     };
-    // 16-byte pieces of a 64 x 64 input tile in address order (piece =
-    // row * 8 + slot); the map is elementwise, so the swizzle does not matter
-    auto piece = [](int pc, int& r, int& slot) {
-      r = pc >> 3;
-      slot = pc & 7;
+    auto waitLoaded = [&](int b) -> bool {
+      const bool r = mbar_wait_or_abort(loaded + b, (pld >> b) & 1u, a.err, abort_flag);
+      pld ^= 1u << b;
+      tc_fence_after();
+      return !named_sync_or(2, GT, !r);
     };
     // bf16 -> fp16 in place (q, k through the feature map); rows past the
-    // sequence become 0
-    auto convert = [&](int nv, int b) {
+    // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x 128
+    // bytes; the map is elementwise, so the swizzle does not matter.
+    auto convert = [&](int nv, int b, bool with_q) {
+      constexpr int PQ = K::TQ / 16 / GT;   // 16-byte pieces of a q or k tile per thread
+      constexpr int PV = K::TV / 16 / GT;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        int r, slot;
-        piece(tid + u * W2_GT, r, slot);   // this thread converts pieces tid, tid + 256
-        const uint32_t off = r * 128 + slot * 16;
-        uint4* ptr[3] = {reinterpret_cast<uint4*>(smem + sQ(b) + off),
-                         reinterpret_cast<uint4*>(smem + sK(b) + off),
-                         reinterpret_cast<uint4*>(smem + sV(b) + off)};
-        uint4 in[3] = {*ptr[0], *ptr[1], *ptr[2]};
+      for (int u = 0; u < 2 * PQ + PV; ++u) {
+        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
+        if (tsel == 0 && !with_q) continue;
+        const int pc = tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
+        const int r = (pc >> 3) & 63;                          // row within its box
+        const uint32_t base = tsel == 0 ? sQ(b) : (tsel == 1 ? sK(b) : sV(b));
+        uint4* ptr = reinterpret_cast<uint4*>(smem + base + pc * 16);
+        const uint4 in = *ptr;
+        uint4 out = make_uint4(0u, 0u, 0u, 0u);
+        if (r < nv) {
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in);
+          uint32_t w[4];
 #pragma unroll
-        for (int tsel = 0; tsel < 3; ++tsel) {
-          uint4 out = make_uint4(0u, 0u, 0u, 0u);
-          if (r < nv) {
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[tsel]);
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(x2[e]);
-              w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
-            }
-            out = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(x2[e]);
+            w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
           }
-          *ptr[tsel] = out;
+          out = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        *ptr = out;
       }
     };
+    const PrepThread th{trow, tid, k, m, comp, half};
     float eta_c = 0.f;
-    {  // initial (scaled) state
-      const float* carry = nullptr;
-      const float* carry_eta = nullptr;
-      if (seg > 0) {
-        carry = a.seg_state + ((bh * (a.nseg - 1) + (seg - 1)) * KR + k) * F;
-        carry_eta = a.seg_eta + (bh * (a.nseg - 1) + (seg - 1)) * KR + k;
-      }
-      const bool from_in = seg == 0 && a.state_in != nullptr;
-      const float2 si = T->sc_inv[m];
-#pragma unroll
-      for (int cb = 0; cb < FH; cb += 16) {
-        const int col0 = half * FH + cb;
-        uint32_t r[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float val = 0.f;
-          const int f = col0 + e;
-          if (carry) {
-            val = carry[f];
-          } else if (from_in) {
-            float2 x = f < DX ? a.state_in[(bh * 64 + m) * DX + f]
-                              : a.state_in[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)];
-            val = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-          }
-          r[e] = __float_as_uint(val);
-        }
-        tmem_st16(trow + K::T_STATE + col0, r);
-      }
-      if (carry_eta) {
-        eta_c = *carry_eta;
-      } else if (from_in) {
-        float2 x = a.state_in[a.BH * 64 * F + bh * 64 + m];
-        eta_c = comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y);
-      }
-      tmem_st_wait();
-    }
+    constexpr int STRIDE = KR * F + KR;   // floats per published state
+    auto load_table = [&](int h) {   // E' of head h into shared memory (prepare group)
+      const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h].E);
+      uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
+      for (int i = tid; i < KR * C * 2 / 16; i += GT) dst[i] = src[i];
+    };
+
     bool ok = true;
-    int nv_last = C;
-    for (int t = ch0; t < ch1; ++t) {
-      const int rel = t - ch0, b = rel % NB, p = rel & 1;
-      const int nv = min(C, a.N - t * C);
-      nv_last = nv;
-      if (!(ok = waitA(loaded + b, pld[b]))) break;
-      convert(nv, b);
-      if (rel >= 1 && !(ok = waitA(dne + 0, pd0))) break;   // G7(t-1): the state is current
-      uint32_t ru[16];
+    bool single_piece_pending = false;   // publish our inclusive state once the carry is known
+    Walker w;
+    first_item(w);
+    int prev_bh = 0, prev_vb = 0, prev_ch = 0;
+    int b = 0;   // buffer set of item i (i % NB)
+    for (int i = 0; ok && i < nI; ++i, w.next(sc, i - 1, a.nch, a.nvb, a.H), b = b + 1 == NB ? 0 : b + 1) {
+      const int p = i & 1;
+      const bool so = sc.state_only(i);
+      const int ch = w.ch;
+      const int nv = min(C, a.N - ch * C);
+      const long long bh = w.bh;
+      const int vb = w.vb;
+      if (!(ok = waitLoaded(b))) break;
+      convert(nv, b, !so);
+      const bool piece_start = so ? (i == 0) : (i == sc.nA || ch == 0);
+      if (i > 0 && !(ok = waitA(dne + 0, pd0))) break;   // G7 of the previous item: the state is current
+      if (piece_start) {
+        if (i > 0) {
+          if (sc.state_only(i - 1)) {
+            // end of the state-only chain: publish our last piece's state
+            const bool inclusive = sc.gA % a.nch == 0;
+            prep_publish<DX>(th, (inclusive ? a.incl : a.agg) + static_cast<long long>(blockIdx.x) * STRIDE, eta_c);
+            prep_raise_flag(a.flags + blockIdx.x, inclusive ? 2 : 1, tid);
+            single_piece_pending = !inclusive;
+          } else if (prev_ch == a.nch - 1 && a.state_out) {
+            prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
+          }
+        }
+        const int h = w.h;
+        if (h != cur_h) {
+          // A new head: its E' table replaces the old one once every
+          // contraction reading the old one is done.  G7 of the previous
+          // item is; G4 of the previous full item (issued after it) is waited
+          // for here by phase: at most that one phase can be pending.
+          const int t = i - sc.nA;
+          if (t >= 1) {
+            const bool r = mbar_wait_or_abort(dne + 2, static_cast<uint32_t>((t - 1) & 1), a.err, abort_flag);
+            tc_fence_after();
+            if (!(ok = !named_sync_or(2, GT, !r))) break;
+          }
+          load_table(h);
+          set_head(h);
+        }
+        if (so && sc.gA % a.nch != 0) {   // a local aggregate starts from zero
+          prep_zero<DX>(th);
+          eta_c = 0.f;
+        } else if (so || ch == 0) {        // a stream's start: state_in or zero
+          eta_c = prep_init_from_input<DX>(a, T, th, bh, vb);
+        } else {                           // inside a stream: the carry from the predecessors
+          if (!(ok = prep_look_back<DX>(a, T, th, abort_flag, xchg, &eta_c))) break;
+          if (single_piece_pending) {
+            prep_publish_inclusive<DX>(a, T, th, sc.nF, eta_c);
+            single_piece_pending = false;
+          }
+        }
+        fence_async_smem();   // a reloaded E' table is read by the next contractions
+      }
+      // R = lambda^C S_hat -> TMEM (the state G7 adds to); for full items also
+      // R_U (fp16 pairs in TMEM, A operand of G3) and R_Gamma (shared memory,
+      // B operand of G6)
 #pragma unroll
       for (int blk = 0; blk < FH / 16; ++blk) {
         const int col0 = half * FH + 16 * blk;
-        uint32_t rs[16], w[16];
-        tmem_ld16(trow + K::T_STATE + col0, rs);
-        tmem_ld_wait16(rs);
+        uint32_t w[16];
+        tmem_ld16(trow + K::T_STATE + col0, w);
+        tmem_ld_wait16(w);
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {   // w = Re/Im of lambda^C times the partner row, two columns at once
-          const float x0 = __uint_as_float(rs[e]), x1 = __uint_as_float(rs[e + 1]);
+        for (int e = 0; e < 16; e += 2) {   // in place: Re/Im of lambda^C times the partner row, two columns at once
+          const float x0 = __uint_as_float(w[e]), x1 = __uint_as_float(w[e + 1]);
           const uint64_t y = f2_pack(__shfl_xor_sync(kFull, x0, 1), __shfl_xor_sync(kFull, x1, 1));
           float w0, w1;
           f2_unpack(f2_fma(lamC2, f2_pack(x0, x1), f2_mul(sgnLi2, y)), w0, w1);
@@ -1405,95 +825,59 @@ __global__ void __launch_bounds__(W2_NT, 1)
           w[e + 1] = __float_as_uint(w1);
         }
         tmem_st16(trow + K::T_STATE + col0, w);
-        if (a.dump_R) dump_r16(a.dump_R, bh * nch_total + t, k, col0, w);
-        if (half == 0) {   // R_U: fp16 pairs into tensor memory, 16 columns per two blocks
+        if (!so) {
+          if (a.dump_R) dump_r16(a.dump_R, bh * a.nch + ch, k, col0, w);
+          if (col0 < DX) {   // R_U: fp16 pairs into tensor memory, 8 columns per block
+            uint32_t ru[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            ru[(blk & 1) * 8 + e] = pack_half2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
-          if (blk & 1) tmem_st16(trow + K::T_RU + 32 * p + 16 * (blk >> 1), ru);
-        } else {           // R_Gamma: shared memory, B operand of G6
+            for (int e = 0; e < 8; ++e)
+              ru[e] = pack_half2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+            tmem_st8(trow + K::T_RU + K::RU_COLS * p + col0 / 2, ru);
+          } else {           // R_Gamma: shared memory, B operand of G6
 #pragma unroll
-          for (int g = 0; g < 2; ++g)
-            *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, col0 - DX + 8 * g, K::RSV)) =
-                pack8f(w + 8 * g, 1.f);
+            for (int g2 = 0; g2 < 2; ++g2)
+              *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, col0 - DX + 8 * g2, K::RSV)) =
+                  pack8f(w + 8 * g2, 1.f);
+          }
         }
       }
       tmem_st_wait();
       {
         const float y = __shfl_xor_sync(kFull, eta_c, 1);
         const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
-        if (half == 0) {
-          if (a.dump_Re) a.dump_Re[(bh * nch_total + t) * KR + k] = Re;
-          *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, DV, K::RSV)) =
+        if (half == 0 && !so) {
+          if (a.dump_Re) a.dump_Re[(bh * a.nch + ch) * KR + k] = Re;
+          *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, kVB, K::RSV)) =
               make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
         }
-        float add = esum_c;
-        if (nv < C) {
-          double sr = 0.0, si = 0.0;
-          const double br = T->b[m].x, bi = T->b[m].y;
-          for (int j = 0; j < nv; ++j) {
-            const double e = exp((C / 2 - j) * T->re_dA[m]);
-            const double ph = fmod((C / 2 - j) * T->im_dA[m], 6.283185307179586476925);
-            double sn, cs;
-            sincos(ph, &sn, &cs);
-            const double pr = e * cs, pi = e * sn;
-            sr += br * pr - bi * pi;
-            si += br * pi + bi * pr;
-          }
-          add = static_cast<float>(comp ? si : sr);
-        }
-        eta_c = Re + add;
+        // ragged last chunk: partial sum of E' over the valid keys
+        eta_c = Re + (nv < C ? ragged_esum(T, m, comp, nv) : esum_c);
       }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(rdy + 0);
+      prev_bh = static_cast<int>(bh);
+      prev_vb = vb;
+      prev_ch = ch;
     }
-    if (ok && ch0 < ch1 && a.state_out && seg == a.nseg - 1) {
+    if (ok && nI > 0 && a.state_out && sc.g1 % a.nch == 0) {
       ok = waitA(dne + 0, pd0);   // G7 of the last chunk
-      if (ok) {
-        const int nv = nv_last;
-        const double ex = exp((nv - C / 2 - 1) * T->re_dA[m]);
-        const double ph = fmod((nv - C / 2 - 1) * T->im_dA[m], 6.283185307179586476925);
-        double sn, cs;
-        sincos(ph, &sn, &cs);
-        const float fr = static_cast<float>(ex * cs), fi = static_cast<float>(ex * sn);
-#pragma unroll
-        for (int cb = 0; cb < FH; cb += 16) {
-          const int col0 = half * FH + cb;
-          uint32_t r[16];
-          tmem_ld16(trow + K::T_STATE + col0, r);
-          tmem_ld_wait16(r);
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const float x = __uint_as_float(r[e2]);
-            const float y = __shfl_xor_sync(kFull, x, 1);
-            if (comp == 0) {
-              const float2 z = make_float2(fr * x - fi * y, fr * y + fi * x);
-              const int f = col0 + e2;
-              if (f < DX) a.state_out[(bh * 64 + m) * DX + f] = z;
-              else a.state_out[a.BH * 64 * DX + (bh * 64 + m) * DV + (f - DX)] = z;
-            }
-          }
-        }
-        const float y = __shfl_xor_sync(kFull, eta_c, 1);
-        if (comp == 0 && half == 0)
-          a.state_out[a.BH * 64 * F + bh * 64 + m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
-      }
+      if (ok) prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
     }
   } else if (role == 1) {
     // ------------------------------------------------ output warps
     const int k = 32 * quad + lane;
     const int m = k >> 1;
-    const float r2 = T->r2[m];
-    const float s_start = static_cast<float>(exp(2.0 * T->re_dA[m] * (32.0 * half - C / 2)));
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     const int i0 = 32 * half;     // this thread's 32 columns of the 64-wide tiles
-    uint32_t pd[4] = {0u, 0u, 0u, 0u};
-    auto waitB = [&](int i) -> bool {
-      const bool r = mbar_wait_or_abort(dne + i, pd[i], a.err, abort_flag);
-      pd[i] ^= 1u;
+    uint32_t pd[4] = {0u, 0u, 0u, 0u}, pS = 0u;
+    int cur_h = -1;
+    float r2 = 0.f, s_start = 0.f;
+    auto waitB = [&](uint64_t* bar, uint32_t& ph) -> bool {
+      const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
+      ph ^= 1u;
       tc_fence_after();
-      return !named_sync_or(3, W2_GT, !r);
+      return !named_sync_or(3, GT, !r);
     };
     auto signalB = [&](int i) {
       fence_async_smem();
@@ -1517,14 +901,14 @@ __global__ void __launch_bounds__(W2_NT, 1)
       signalB(3);
     };
     // o = num / den, staged as two boxes of 64 rows x 128 bytes (columns 0-31
-    // and 32-63) in the 128-byte swizzled layout, which keeps the row-per-lane
-    // writes free of bank conflicts, then written by one TMA store per box.
-    // Rows past the sequence lie outside the tensor map and are not written.
-    // Staging alternates between two buffers.  Before the barrier that
-    // precedes each store, the issuing thread waits until the store before it
-    // has finished reading its buffer; every thread passes that barrier before
-    // it writes that buffer again one chunk later.
-    auto e4 = [&](int ch, int nv) {
+    // and 32-63 of the value block) in the 128-byte swizzled layout, which
+    // keeps the row-per-lane writes free of bank conflicts, then written by
+    // one TMA store per box.  Rows past the sequence lie outside the tensor
+    // map and are not written.  Staging alternates between two buffers.
+    // Before the barrier that precedes each store, the issuing thread waits
+    // until the store before it has finished reading its buffer; every thread
+    // passes that barrier before it writes that buffer again one chunk later.
+    auto e4 = [&](long long bh, int vb, int ch, int nv, int t) {
       const int i = r16, hb = lane >> 4;
       uint32_t rd, rr[16];
       tmem_ld1(trow + K::T_DEN, rd);   // one column of all 32 lanes: rows in lanes 0-15
@@ -1535,46 +919,55 @@ __global__ void __launch_bounds__(W2_NT, 1)
       const float rdn = 1.0f / dn;
       const uint64_t rdn2 = f2_pack(rdn, rdn);
       const long long row = bh * a.N + ch * C + i;
-      const uint32_t stage = K::S_O + ((ch - ch0) & 1) * K::TO;
-      if (i < nv && a.den && half == 0 && hb == 0) a.den[row] = dn;
+      const uint32_t stage = K::S_O + (t & 1) * K::TO;
+      if (i < nv && a.den && half == 0 && hb == 0 && vb == 0) a.den[row] = dn;
       uint8_t* box = smem + stage + half * (K::TO / 2) + i * 128;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t* r = rr + 4 * g;
+      for (int gg = 0; gg < 4; ++gg) {
+        const uint32_t* r = rr + 4 * gg;
         float4 q;
         f2_unpack(f2_mul(f2_pack(__uint_as_float(r[0]), __uint_as_float(r[1])), rdn2), q.x, q.y);
         f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2]), __uint_as_float(r[3])), rdn2), q.z, q.w);
-        *reinterpret_cast<float4*>(box + (((4 * hb + g) ^ (i & 7)) << 4)) = q;
+        *reinterpret_cast<float4*>(box + (((4 * hb + gg) ^ (i & 7)) << 4)) = q;
       }
       if (i < nv && a.num) {
-        float4* np = reinterpret_cast<float4*>(a.num + row * DV + c0);
+        float4* np = reinterpret_cast<float4*>(a.num + row * a.DV + vb * kVB + c0);
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
-          np[g] = make_float4(__uint_as_float(rr[4 * g]), __uint_as_float(rr[4 * g + 1]),
-                              __uint_as_float(rr[4 * g + 2]), __uint_as_float(rr[4 * g + 3]));
+        for (int gg = 0; gg < 4; ++gg)
+          np[gg] = make_float4(__uint_as_float(rr[4 * gg]), __uint_as_float(rr[4 * gg + 1]),
+                               __uint_as_float(rr[4 * gg + 2]), __uint_as_float(rr[4 * gg + 3]));
       }
       fence_async_smem();
-      if (tid == W2_GT) bulk_wait_read_0();
-      named_sync(1, W2_GT);
-      if (tid == W2_GT) {
-        tma_store_3d(&tm_o, sbase + stage, 0, ch * C, static_cast<int>(bh));
-        tma_store_3d(&tm_o, sbase + stage + K::TO / 2, 32, ch * C, static_cast<int>(bh));
+      if (tid == GT) bulk_wait_read_0();
+      named_sync(1, GT);
+      if (tid == GT) {
+        tma_store_3d(&tm_o, sbase + stage, vb * kVB, ch * C, static_cast<int>(bh));
+        tma_store_3d(&tm_o, sbase + stage + K::TO / 2, vb * kVB + 32, ch * C, static_cast<int>(bh));
         bulk_commit();
       }
     };
     bool ok = true;
-    int prev = -1, prev_nv = C;
+    bool have_prev = false;
+    int prev_bh = 0, prev_vb = 0, prev_ch = 0, prev_nv = C, t = 0;
+    Walker w;
+    w.seek(sc.g0, a.nch, a.nvb, a.H);
     // E2(t) comes before E4(t-1) so that G4(t) can start while E4 runs;
-    // t == ch1 runs only the tail (E3, E4) of the last chunk
-    for (int t = ch0; ok && t <= ch1 && ch0 < ch1; ++t) {
-      const bool head = t < ch1;
-      const int nv = head ? min(C, a.N - t * C) : 0;
-      if (prev >= 0) {
-        if (!(ok = waitB(2))) break;   // G4(t-1)
+    // t == nF runs only the tail (E3, E4) of the last chunk
+    for (t = 0; ok && t <= sc.nF && sc.nF > 0; ++t) {
+      const bool head = t < sc.nF;
+      const int nv = head ? min(C, a.N - w.ch * C) : 0;
+      if (have_prev) {
+        if (!(ok = waitB(dne + 2, pd[2]))) break;   // G4(t-1)
         e3();
       }
       if (head) {
-        if (!(ok = waitB(0))) break;   // G1 + G7(t)
+        const int h = w.h;
+        if (h != cur_h) {
+          cur_h = h;
+          r2 = a.tabs[h].r2[m];
+          s_start = static_cast<float>(exp(2.0 * a.tabs[h].re_dA[m] * (32.0 * half - C / 2)));
+        }
+        if (!(ok = waitB(dneS, pS))) break;   // G1(t)
         {  // E1(t): masked S^T -> [j][i]
           const int j = r16;
           const bool keep = j < nv;
@@ -1588,16 +981,14 @@ __global__ void __launch_bounds__(W2_NT, 1)
           *reinterpret_cast<uint4*>(smem + K::S_S + tile_off(j, c0 + 8, 1024)) = pack8f(r + 8, 1.f);
           signalB(1);
         }
-      }
-      if (head) {
-        if (!(ok = waitB(1))) break;   // G2 + G3(t)
+        if (!(ok = waitB(dne + 1, pd[1]))) break;   // G2 + G3(t)
         {  // E2(t): X = |lambda|^(2(i-c)) a~
           uint64_t s2 = f2_pack(s_start, s_start * r2);   // scales of two adjacent columns
           const uint64_t r4 = f2_pack(r2 * r2, r2 * r2);
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
+          for (int bb = 0; bb < 2; ++bb) {
             uint32_t r[16];
-            tmem_ld16(trow + K::T_A + i0 + 16 * b, r);
+            tmem_ld16(trow + K::T_A + i0 + 16 * bb, r);
             tmem_ld_wait16(r);
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
@@ -1607,43 +998,54 @@ __global__ void __launch_bounds__(W2_NT, 1)
               r[e + 1] = __float_as_uint(x1);
               s2 = f2_mul(s2, r4);
             }
-            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b, 1024)) = pack8f(r, 1.f);
-            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * b + 8, 1024)) = pack8f(r + 8, 1.f);
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb, 1024)) = pack8f(r, 1.f);
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb + 8, 1024)) = pack8f(r + 8, 1.f);
           }
           signalB(2);
         }
       }
-      if (prev >= 0) {
-        if (!(ok = waitB(3))) break;   // G5 + G6(t-1)
-        e4(prev, prev_nv);
+      if (have_prev) {
+        if (!(ok = waitB(dne + 3, pd[3]))) break;   // G5 + G6(t-1)
+        e4(prev_bh, prev_vb, prev_ch, prev_nv, t - 1);
       }
-      prev = t;
+      have_prev = head;
+      prev_bh = w.bh;
+      prev_vb = w.vb;
+      prev_ch = w.ch;
       prev_nv = nv;
+      if (head) w.step(a.nch, a.nvb, a.H);
     }
-    if (tid == W2_GT) bulk_wait_all();   // o is in global memory before the block exits
+    if (tid == GT) bulk_wait_all();   // o is in global memory before the block exits
   }
   if (role == 3) {
     // ------------------------------------------------ fetch warp
     if (lane == 0) {
-      uint32_t pfq[NB] = {0u, 0u, 0u}, pfv[NB] = {0u, 0u, 0u};
-      int issued[NB] = {0, 0, 0};
-      for (int t = ch0; t < ch1; ++t) {
-        const int rel = t - ch0, b = rel % NB;
-        if (rel >= NB) {   // set b last held chunk t-3: wait until its contractions are done
-          bool ok = mbar_wait_or_abort(freeQK + b, pfq[b], a.err, abort_flag);
-          pfq[b] ^= 1u;
-          if (ok) ok = mbar_wait_or_abort(freeVR + b, pfv[b], a.err, abort_flag);
-          pfv[b] ^= 1u;
+      int issued = 0;
+      Walker w;
+      first_item(w);
+      for (int i = 0, b = 0; i < nI; ++i, w.next(sc, i - 1, a.nch, a.nvb, a.H), b = b + 1 == NB ? 0 : b + 1) {
+        const bool so = sc.state_only(i);
+        if (i >= NB) {   // set b last held item i - NB: wait until its contractions are done
+          const uint32_t par = static_cast<uint32_t>((i / NB - 1) & 1);   // that item's release phase
+          bool ok = mbar_wait_or_abort(freeQK + b, par, a.err, abort_flag);
+          if (ok) ok = mbar_wait_or_abort(freeVR + b, par, a.err, abort_flag);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(loaded + b, 3 * K::TIN);
-        tma_load_3d(sbase + sQ(b), &tm_q, 0, t * C, static_cast<int>(bh), loaded + b);
-        tma_load_3d(sbase + sK(b), &tm_k, 0, t * C, static_cast<int>(bh), loaded + b);
-        tma_load_3d(sbase + sV(b), &tm_v, 0, t * C, static_cast<int>(bh), loaded + b);
-        ++issued[b];
+        const int y = w.ch * C, z = w.bh;
+        mbar_arrive_expect_tx(loaded + b, (so ? 1 : 2) * K::TQ + K::TV);
+        for (int x = 0; x < DX / 64; ++x) {
+          if (!so) tma_load_3d(sbase + sQ(b) + x * K::BOX, &tm_q, 64 * x, y, z, loaded + b);
+          tma_load_3d(sbase + sK(b) + x * K::BOX, &tm_k, 64 * x, y, z, loaded + b);
+        }
+        tma_load_3d(sbase + sV(b), &tm_v, w.vb * kVB, y, z, loaded + b);
+        issued = i + 1;
       }
-      for (int b = 0; b < NB; ++b)   // no copy of ours lands after the block exits
-        if (issued[b] > 0) mbar_wait(loaded + b, static_cast<uint32_t>((issued[b] - 1) & 1), a.err);
+      // no copy of ours lands after the block exits: the last load into each
+      // set b was item i_b, the phase (i_b / NB) of loaded[b]
+      for (int b = 0; b < NB && b < issued; ++b) {
+        const int i_b = b + (issued - 1 - b) / NB * NB;
+        mbar_wait(loaded + b, static_cast<uint32_t>((i_b / NB) & 1), a.err);
+      }
     }
     __syncwarp();
   }
@@ -1652,70 +1054,49 @@ __global__ void __launch_bounds__(W2_NT, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Tuning switch IA_PREFILL_WS for d = 64: 0 the one-role loop, 1 one epilogue
-// group, unset or 2 the four-role kernel.
-bool ws2_selected() {
-  const char* ws = std::getenv("IA_PREFILL_WS");
-  return !ws || std::atoi(ws) >= 2;
+// Chunks a CTA carries under grid G: the largest range, plus the state-only
+// chain of a last piece that ends inside a stream (about a quarter of a full
+// chunk each), plus the hops of the look-back.
+double plan_cost(long long total, int nch, int G) {
+  constexpr double kStateOnly = 0.25, kHop = 0.5;
+  double worst = 0.0;
+  for (int c = 0; c < G; ++c) {
+    const long long g0 = total * c / G, g1 = total * (c + 1) / G;
+    double t = static_cast<double>(g1 - g0);
+    if (g1 % nch != 0) t += kStateOnly * static_cast<double>(g1 - std::max(g0, (g1 - 1) / nch * nch));
+    if (g0 % nch != 0) {   // hops back to the stream's first piece, roughly
+      const long long start = g0 / nch * nch;
+      t += kHop * std::ceil(static_cast<double>(g0 - start) * G / static_cast<double>(total));
+    }
+    worst = std::max(worst, t);
+  }
+  return worst;
 }
 
-template <int DX, int DV>
-cudaError_t launch_impl(const TcArgs& args, const ia_shape_t& s, const TcPlan& p, cudaStream_t st) {
-  using K = Cfg<DX, DV>;
-  cudaError_t e;
-  if (p.nseg > 1) {
-    auto k1 = tc_prefill_kernel<DX, DV, false>;
-    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
-    if (e != cudaSuccess) return e;
-    k1<<<static_cast<unsigned>(args.BH * (p.nseg - 1)), NT, K::SMEM, st>>>(args);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = launch_segment_scan(s.B, s.H, DX, DV, p.nseg, p.seg_chunks * C, args.tabs, args.state_in,
-                            args.seg_state, args.seg_eta, st);
-    if (e != cudaSuccess) return e;
-  }
-  if constexpr (DX == 64 && DV == 64) {
-    if (ws2_selected()) {
-      CUtensorMap tm_q, tm_k, tm_v, tm_o;
-      if (!encode_input_map(&tm_q, args.q, args.BH, args.N) || !encode_input_map(&tm_k, args.k, args.BH, args.N) ||
-          !encode_input_map(&tm_v, args.v, args.BH, args.N) || !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N))
-        return cudaErrorNotSupported;
-      e = cudaFuncSetAttribute(tc_prefill_ws2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, W2Cfg::SMEM);
-      if (e != cudaSuccess) return e;
-      // Programmatic dependent launch: the CTAs set up barriers, TMEM and
-      // constant tiles while the previous kernel finishes (see griddep_wait).
-      // Straight after the table kernel, the timing mark was set before it.
-      if (p.nseg > 1) mark_launch_begin(st);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(static_cast<unsigned>(args.BH * p.nseg));
-      cfg.blockDim = dim3(W2_NT);
-      cfg.dynamicSmemBytes = W2Cfg::SMEM;
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      e = cudaLaunchKernelEx(&cfg, tc_prefill_ws2_kernel, args, tm_q, tm_k, tm_v, tm_o);
-      mark_launch_end(st);
-      return e;
-    }
-    const char* ws = std::getenv("IA_PREFILL_WS");
-    if (std::atoi(ws) == 1) {
-      e = cudaFuncSetAttribute(tc_prefill_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WCfg::SMEM);
-      if (e != cudaSuccess) return e;
-      mark_launch_begin(st);
-      tc_prefill_ws_kernel<<<static_cast<unsigned>(args.BH * p.nseg), WS_NT, WCfg::SMEM, st>>>(args);
-      e = cudaGetLastError();
-      mark_launch_end(st);
-      return e;
-    }
-  }
-  auto k3 = tc_prefill_kernel<DX, DV, true>;
-  e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
+template <int DX>
+cudaError_t launch_impl(const TcArgs& args, const void* q, const void* k, const void* v, int DV,
+                        cudaStream_t st) {
+  using K = PCfg<DX>;
+  CUtensorMap tm_q, tm_k, tm_v, tm_o;
+  if (!encode_input_map(&tm_q, q, args.BH, args.N, DX) || !encode_input_map(&tm_k, k, args.BH, args.N, DX) ||
+      !encode_input_map(&tm_v, v, args.BH, args.N, DV) || !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N, DV))
+    return cudaErrorNotSupported;
+  auto kern = tc_prefill_kernel<DX>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
-  mark_launch_begin(st);
-  k3<<<static_cast<unsigned>(args.BH * p.nseg), NT, K::SMEM, st>>>(args);
-  e = cudaGetLastError();
+  // Programmatic dependent launch: the CTAs set up barriers, TMEM and
+  // constant tiles while the table kernel finishes (see griddep_wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(args.G));
+  cfg.blockDim = dim3(NTH);
+  cfg.dynamicSmemBytes = K::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, args, tm_q, tm_k, tm_v, tm_o);
   mark_launch_end(st);
   return e;
 }
@@ -1729,42 +1110,53 @@ bool tc_prefill_supported(const ia_shape_t& s) {
 }
 
 TcPlan tc_plan(const ia_shape_t& s, int num_sms) {
-  const long long BH = static_cast<long long>(s.B) * s.H;
-  const int nch = (s.N + C - 1) / C;
-  // Forced segment count (tuning and tests): IA_PREFILL_SEGMENTS=n.
-  if (const char* env = std::getenv("IA_PREFILL_SEGMENTS")) {
-    const int n = std::atoi(env);
-    if (n >= 1 && n <= nch) {
-      const int L = (nch + n - 1) / n;
-      return TcPlan{(nch + L - 1) / L, L};
-    }
+  const long long nch = (s.N + C - 1) / C;
+  const long long streams = static_cast<long long>(s.B) * s.H * (s.d_v / kVB);
+  const long long total = streams * nch;
+  // Forced grid (tuning and tests): IA_PREFILL_GRID=n.
+  if (const char* env = std::getenv("IA_PREFILL_GRID")) {
+    const long long n = std::atoll(env);
+    if (n >= 1) return TcPlan{static_cast<int>(std::min<long long>({n, total, static_cast<long long>(num_sms)}))};
   }
-  // Cost in units of one full chunk pass: waves x (chunks per CTA + per-CTA
-  // prologue/epilogue), a state-only chunk costing alpha, plus the scan.
-  const double alpha = 0.35, cta_overhead = 1.0, scan = 1.0;
-  const int min_len = 4;   // shorter segments spend more on state round trips than they save
-  TcPlan best{1, nch};
-  double best_t = 1e300;
-  for (int nseg = 1; nseg <= 32 && nseg <= nch; ++nseg) {
-    const int L = (nch + nseg - 1) / nseg;
-    if ((nch + L - 1) / L != nseg) continue;
-    if (nseg > 1 && L < min_len) continue;
-    const double w1 = nseg > 1 ? std::ceil(static_cast<double>(BH * (nseg - 1)) / num_sms) : 0.0;
-    const double w3 = std::ceil(static_cast<double>(BH * nseg) / num_sms);
-    const double t = w1 * (L * alpha + cta_overhead) + w3 * (L + cta_overhead) + (nseg > 1 ? scan : 0.0);
+  // The search below is O(num_sms^2); remember the last few answers.
+  struct Entry {
+    long long total, nch;
+    int num_sms, grid;
+  };
+  static thread_local Entry cache[4] = {};
+  static thread_local int next = 0;
+  for (const Entry& e : cache)
+    if (e.grid > 0 && e.total == total && e.nch == nch && e.num_sms == num_sms) return TcPlan{e.grid};
+  const int gmax = static_cast<int>(std::min<long long>(num_sms, (total + kMinPiece - 1) / kMinPiece));
+  // the largest grid first, so that ties keep every SM busy
+  TcPlan best{std::max(1, gmax)};
+  double best_t = plan_cost(total, static_cast<int>(nch), best.grid);
+  for (int G = gmax - 1; G >= 1; --G) {
+    const double t = plan_cost(total, static_cast<int>(nch), G);
     if (t < best_t - 1e-9) {
       best_t = t;
-      best = TcPlan{nseg, L};
+      best.grid = G;
     }
   }
+  cache[next] = Entry{total, nch, num_sms, best.grid};
+  next = (next + 1) % 4;
   return best;
 }
 
+bool tc_plan_splits(const ia_shape_t& s, const TcPlan& p) {
+  const long long nch = (s.N + C - 1) / C;
+  const long long total = static_cast<long long>(s.B) * s.H * (s.d_v / kVB) * nch;
+  for (int c = 1; c < p.grid; ++c)
+    if ((total * c / p.grid) % nch != 0) return true;
+  return false;
+}
+
 size_t tc_workspace_bytes(const ia_shape_t& s, const TcPlan& p) {
-  const size_t BH = static_cast<size_t>(s.B) * s.H;
   size_t bytes = sizeof(HeadTables) * static_cast<size_t>(s.H);
-  if (p.nseg > 1) {
-    bytes += BH * (p.nseg - 1) * (static_cast<size_t>(KR) * (s.d_xi + s.d_v) + KR) * sizeof(float);
+  if (tc_plan_splits(s, p)) {
+    const size_t F = static_cast<size_t>(s.d_xi) + kVB;
+    bytes += 2 * static_cast<size_t>(p.grid) * (KR * F + KR) * sizeof(float);   // agg, incl
+    bytes += static_cast<size_t>(p.grid) * sizeof(int) + 256;                    // flags
   }
   return bytes + 256;
 }
@@ -1778,25 +1170,27 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st, void* dump_R,
                               float* dump_Re, float* dtab) {
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  w = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(w) + 255) & ~static_cast<uintptr_t>(255));
+  uint8_t* w = reinterpret_cast<uint8_t*>(tc_tables(ws));
   HeadTables* tabs = reinterpret_cast<HeadTables*>(w);
-  float* seg_state = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);
-  const size_t BH = static_cast<size_t>(s.B) * s.H;
-  float* seg_eta = seg_state + BH * (p.nseg > 1 ? p.nseg - 1 : 0) * KR * (s.d_xi + s.d_v);
-  // the four-role d = 64 kernel directly after the tables overlaps them, so
-  // its timing mark goes before the table kernel
-  if (s.d_xi == 64 && s.d_v == 64 && p.nseg == 1 && ws2_selected()) mark_launch_begin(st);
-  cudaError_t e = launch_param_tables(s.H, delta, A, tabs, st, dtab);
-  if (e != cudaSuccess) return e;
   TcArgs args;
-  args.q = static_cast<const __nv_bfloat16*>(q);
-  args.k = static_cast<const __nv_bfloat16*>(k);
-  args.v = static_cast<const __nv_bfloat16*>(v);
+  args.agg = args.incl = nullptr;
+  args.flags = nullptr;
+  const size_t F = static_cast<size_t>(s.d_xi) + kVB;
+  if (tc_plan_splits(s, p)) {
+    float* agg = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);
+    args.agg = agg;
+    args.incl = agg + static_cast<size_t>(p.grid) * (KR * F + KR);
+    uint8_t* fl = reinterpret_cast<uint8_t*>(args.incl + static_cast<size_t>(p.grid) * (KR * F + KR));
+    args.flags = reinterpret_cast<int*>((reinterpret_cast<uintptr_t>(fl) + 255) & ~static_cast<uintptr_t>(255));
+  }
+  // the chunk pass starts under the table kernel, so its timing mark goes
+  // before the table kernel
+  mark_launch_begin(st);
+  cudaError_t e = launch_param_tables(s.H, delta, s.delta_per_mode, A, tabs, st, dtab, args.flags,
+                                      args.flags ? p.grid : 0);
+  if (e != cudaSuccess) return e;
   args.tabs = tabs;
   args.state_in = static_cast<const float2*>(state_in);
-  args.seg_state = seg_state;
-  args.seg_eta = seg_eta;
   args.o = o;
   args.num = num;
   args.den = den;
@@ -1807,13 +1201,14 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
   if (!args.err) return cudaErrorInvalidSymbol;
   args.H = s.H;
   args.N = s.N;
-  args.nseg = p.nseg;
-  args.seg_chunks = p.seg_chunks;
-  args.BH = static_cast<long long>(BH);
-  if (s.d_xi == 64 && s.d_v == 64) return launch_impl<64, 64>(args, s, p, st);
-  if (s.d_xi == 128 && s.d_v == 128) return launch_impl<128, 128>(args, s, p, st);
-  if (s.d_xi == 64 && s.d_v == 128) return launch_impl<64, 128>(args, s, p, st);
-  if (s.d_xi == 128 && s.d_v == 64) return launch_impl<128, 64>(args, s, p, st);
+  args.DV = s.d_v;
+  args.nch = (s.N + C - 1) / C;
+  args.nvb = s.d_v / kVB;
+  args.G = p.grid;
+  args.BH = static_cast<long long>(s.B) * s.H;
+  args.total = args.BH * args.nvb * args.nch;
+  if (s.d_xi == 64) return launch_impl<64>(args, q, k, v, s.d_v, st);
+  if (s.d_xi == 128) return launch_impl<128>(args, q, k, v, s.d_v, st);
   return cudaErrorInvalidValue;
 }
 

@@ -61,5 +61,5 @@ extern "C" IA_API ia_status_t ia_selftest_wait_expiry(unsigned long long limit_n
   int* err = device_error_ptr();
   if (!err) return IA_ERR_CUDA;
   wait_expiry_kernel<<<1, 96, 0, static_cast<cudaStream_t>(stream)>>>(err, limit_ns, out);
-  return cudaGetLastError() == cudaSuccess ? IA_OK : IA_ERR_CUDA;
+  return map_cuda(cudaGetLastError());
 }

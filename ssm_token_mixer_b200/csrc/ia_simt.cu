@@ -1,6 +1,6 @@
-// IA layer on CUDA cores in fp32: per-head parameter tables, the sequential
-// recurrence (forward), its reverse-mode adjoint (backward) and the
-// inter-segment carry scan of the chunked tensor-core path.
+// IA layer on CUDA cores in fp32: per-head parameter tables of the chunked
+// tensor-core path, the sequential recurrence (forward) and its reverse-mode
+// adjoint (backward).
 //
 // The recurrence and readout follow the paper 'Interdomain Attention: Beyond
 // Token-Level Key-Value Memory' (paperlayer.ai summary sec. 3.1-3.2; AI-radio
@@ -11,72 +11,10 @@
 #include "ia_device.cuh"
 #include "ia_internal.h"
 #include "ia_tables.cuh"
+#include "ia_simt_common.cuh"
 
 namespace ia {
 
-namespace {
-
-template <typename T>
-__device__ __forceinline__ float ldf(const T* p);
-template <>
-__device__ __forceinline__ float ldf<float>(const float* p) {
-  return *p;
-}
-template <>
-__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) {
-  return __bfloat162float(*p);
-}
-
-__device__ __forceinline__ float feat_acc(float x) { return x > 0.f ? x + 1.f : expf(x); }
-__device__ __forceinline__ float dfeat_acc(float x) { return x > 0.f ? 1.f : expf(x); }
-
-__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
-  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
-}
-__device__ __forceinline__ float2 cfma(float2 a, float2 b, float2 c) {  // a*b + c
-  return make_float2(fmaf(a.x, b.x, fmaf(-a.y, b.y, c.x)), fmaf(a.x, b.y, fmaf(a.y, b.x, c.y)));
-}
-__device__ __forceinline__ float re_conj_mul(float2 a, float2 b) {  // Re(conj(a) b)
-  return fmaf(a.x, b.x, a.y * b.y);
-}
-
-// Mode constants in fp64: A_m (S4D-Lin unless given), lambda = exp(Delta A),
-// b = (lambda - 1) / A (zero-order hold).
-struct ModeD {
-  double ar, ai, lr, li, br, bi;
-};
-__device__ __forceinline__ ModeD mode_consts(float delta, const float* A, int m) {
-  ModeD r;
-  r.ar = A ? static_cast<double>(A[2 * m]) : -0.5;
-  r.ai = A ? static_cast<double>(A[2 * m + 1]) : 3.14159265358979323846 * m;
-  double d = static_cast<double>(delta);
-  double e = exp(d * r.ar), s, c;
-  sincos(d * r.ai, &s, &c);
-  r.lr = e * c;
-  r.li = e * s;
-  double nr = r.lr - 1.0, ni = r.li, den = r.ar * r.ar + r.ai * r.ai;
-  r.br = (nr * r.ar + ni * r.ai) / den;
-  r.bi = (ni * r.ar - nr * r.ai) / den;
-  return r;
-}
-
-// lambda^n = exp(n Delta A) with the phase reduced in fp64.
-__device__ __forceinline__ void cpow_d(double re_dA, double im_dA, double n, double* pr, double* pi) {
-  double e = exp(n * re_dA);
-  double ph = fmod(n * im_dA, 6.283185307179586476925);
-  double s, c;
-  sincos(ph, &s, &c);
-  *pr = e * c;
-  *pi = e * s;
-}
-
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
-}  // namespace
 
 // ------------------------------------------------------------------------
 // Parameter prologue for the tensor-core path: one block per head, four
@@ -85,10 +23,14 @@ __device__ __forceinline__ float warp_sum(float x) {
 // power (relative error ~16 * 2^-53); the sum of E' over the chunk is reduced
 // across the four threads, and the remaining per-mode powers are shared out
 // among them.  The E' table is staged in shared memory and written out with
-// coalesced 16-byte stores.  With dtab, also the derivative table for the
-// reverse pass: dtab[h][k][j] = component (k & 1) of dE'[j, k/2]/dDelta =
-// lambda^n (lambda + n A b), n = c - j, fp32, followed by the row sums
-// dtab[H*128*64 + h*128 + k].
+// coalesced 16-byte stores.  With dtab, also the derivative tables of the
+// reverse pass, [3][H][128][64] fp32 followed by their row sums [3][H][128]:
+// table w, row k = 2m + comp, column j holds component comp of
+//   w = 0: dE'[j,m]/dDelta_hm = lambda^n (lambda + n A b)
+//   w = 1: dE'[j,m]/dA_m      = lambda^n ((Delta lambda - b)/A + n Delta b)
+//   w = 2: i dE'[j,m]/dA_m    (the derivative along Im A_m)
+// with n = c - j, so that the reverse pass contracts its adjoint of E' with
+// each table to get dL/dDelta, dL/dRe A and dL/dIm A.
 // The tensor-core operands carry factors up to |lambda_m|^(-C/2) =
 // exp(Delta |Re A_m| C/2) in fp16 (the centred decay table and the readout
 // scale); a head whose factor exceeds kMaxHalfChunkGrowth, or whose Delta is
@@ -100,53 +42,73 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
                                                                     const float* __restrict__ A,
                                                                     HeadTables* __restrict__ tabs,
                                                                     float* __restrict__ dtab,
-                                                                    int* __restrict__ err) {
+                                                                    int* __restrict__ err,
+                                                                    int* __restrict__ flags, int nflags,
+                                                                    int dpm) {
   __shared__ __align__(16) __half Es[2 * kModesTC * kChunk];
   griddep_launch_dependents();   // the chunk pass may start its table-free prologue now
   const int h = blockIdx.x;
+  if (h == 0)   // the chunk pass's look-back flags start at zero
+    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0;
   HeadTables* T = tabs + h;
-  const float dl = delta[h];
   constexpr int C = kChunk, c = kChunk / 2, JS = kChunk / 4;
   const int m = threadIdx.x >> 2, part = threadIdx.x & 3;   // four threads per mode, adjacent lanes
+  const float dl = delta_hm(delta, dpm, kModesTC, h, m);
   ModeD md = mode_consts(dl, A, m);
   const double rdA = dl * md.ar, idA = dl * md.ai;
   if (part == 0 && !(dl > 0.f && fabs(rdA) * (C / 2) <= log(kMaxHalfChunkGrowth))) atomicOr(err, kErrParamRange);
   double pr, pi, ir, ii;
   cpow_d(rdA, idA, c - JS * part, &pr, &pi);   // lambda^(c-j) at this thread's first j
   cpow_d(rdA, idA, -1.0, &ir, &ii);            // lambda^-1
-  double sr = 0.0, si = 0.0, dsr = 0.0, dsi = 0.0;
+  double sr = 0.0, si = 0.0;
+  double dsr[3] = {0.0, 0.0, 0.0}, dsi[3] = {0.0, 0.0, 0.0};
   char* base = reinterpret_cast<char*>(Es);
-  float* drow = dtab ? dtab + (static_cast<size_t>(h) * 2 * kModesTC + 2 * m) * C : nullptr;
+  const size_t tab_stride = static_cast<size_t>(H) * 2 * kModesTC * C;   // floats per derivative table
+  // (Delta lambda - b) / A: the A-derivative of b, less its n Delta b part
+  const double cr = dl * md.lr - md.br, ci = dl * md.li - md.bi, aa = md.ar * md.ar + md.ai * md.ai;
+  const double gr = (cr * md.ar + ci * md.ai) / aa, gi = (ci * md.ar - cr * md.ai) / aa;
   for (int j = JS * part; j < JS * (part + 1); ++j) {   // E'[j] = b lambda^(c-j)
     const double er = md.br * pr - md.bi * pi, ei = md.br * pi + md.bi * pr;
     *reinterpret_cast<__half*>(base + etab_offset(2 * m, j)) = __double2half(er);
     *reinterpret_cast<__half*>(base + etab_offset(2 * m + 1, j)) = __double2half(ei);
     sr += er;
     si += ei;
-    if (drow) {   // dE'[j]/dDelta = lambda^n (lambda + n A b), n = c - j
+    if (dtab) {
       const double n = c - j;
+      // dDelta: lambda^n (lambda + n A b)
       const double fr = md.lr + n * (md.ar * md.br - md.ai * md.bi), fi = md.li + n * (md.ar * md.bi + md.ai * md.br);
-      const double dr = pr * fr - pi * fi, di = pr * fi + pi * fr;
-      drow[j] = static_cast<float>(dr);
-      drow[C + j] = static_cast<float>(di);
-      dsr += dr;
-      dsi += di;
+      // dA: lambda^n ((Delta lambda - b)/A + n Delta b)
+      const double hr = gr + n * dl * md.br, hi = gi + n * dl * md.bi;
+      const double d0r = pr * fr - pi * fi, d0i = pr * fi + pi * fr;
+      const double d1r = pr * hr - pi * hi, d1i = pr * hi + pi * hr;
+      const double comp[3][2] = {{d0r, d0i}, {d1r, d1i}, {-d1i, d1r}};   // rows 2m, 2m+1 of each table
+      for (int w = 0; w < 3; ++w) {
+        float* row = dtab + w * tab_stride + (static_cast<size_t>(h) * 2 * kModesTC + 2 * m) * C;
+        row[j] = static_cast<float>(comp[w][0]);
+        row[C + j] = static_cast<float>(comp[w][1]);
+        dsr[w] += comp[w][0];
+        dsi[w] += comp[w][1];
+      }
     }
     const double nr = pr * ir - pi * ii;
     pi = pr * ii + pi * ir;
     pr = nr;
   }
-  // sum of E' over the chunk: the four partial sums of this mode
+  // sums over the chunk: the four partial sums of this mode
   for (int off = 1; off < 4; off <<= 1) {
     sr += __shfl_xor_sync(0xffffffffu, sr, off);
     si += __shfl_xor_sync(0xffffffffu, si, off);
-    dsr += __shfl_xor_sync(0xffffffffu, dsr, off);
-    dsi += __shfl_xor_sync(0xffffffffu, dsi, off);
+    for (int w = 0; w < 3; ++w) {
+      dsr[w] += __shfl_xor_sync(0xffffffffu, dsr[w], off);
+      dsi[w] += __shfl_xor_sync(0xffffffffu, dsi[w], off);
+    }
   }
-  if (dtab && part == 0) {   // row sums after the [H][128][64] table
-    float* dsum = dtab + static_cast<size_t>(H) * 2 * kModesTC * C + static_cast<size_t>(h) * 2 * kModesTC;
-    dsum[2 * m] = static_cast<float>(dsr);
-    dsum[2 * m + 1] = static_cast<float>(dsi);
+  if (dtab && part == 0) {   // row sums after the three tables
+    for (int w = 0; w < 3; ++w) {
+      float* dsum = dtab + 3 * tab_stride + (static_cast<size_t>(w) * H + h) * 2 * kModesTC;
+      dsum[2 * m] = static_cast<float>(dsr[w]);
+      dsum[2 * m + 1] = static_cast<float>(dsi[w]);
+    }
   }
   if (part == 0) {
     T->lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
@@ -179,7 +141,7 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
 template <typename T>
 __global__ void seq_fwd_kernel(int H, int N, int DX, int DV, int M, const T* __restrict__ q,
                                const T* __restrict__ k, const T* __restrict__ v,
-                               const float* __restrict__ delta, const float* __restrict__ A,
+                               const float* __restrict__ delta, int dpm, const float* __restrict__ A,
                                const float2* __restrict__ state_in, float* __restrict__ o,
                                float* __restrict__ num, float* __restrict__ den,
                                float2* __restrict__ state_out, long long BH) {
@@ -200,7 +162,7 @@ __global__ void seq_fwd_kernel(int H, int N, int DX, int DV, int M, const T* __r
   const int warp = tid >> 5, lane = tid & 31, nwarp = nthr >> 5;
 
   for (int m = tid; m < M; m += nthr) {
-    ModeD md = mode_consts(delta[h], A, m);
+    ModeD md = mode_consts(delta_hm(delta, dpm, M, h, m), A, m);
     lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
     bb[m] = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
   }
@@ -275,10 +237,10 @@ constexpr int kCk = 64;
 template <typename T>
 __global__ void seq_bwd_kernel(int H, int N, int DX, int DV, int M, const T* __restrict__ q,
                                const T* __restrict__ k, const T* __restrict__ v,
-                               const T* __restrict__ dO, const float* __restrict__ delta,
+                               const T* __restrict__ dO, const float* __restrict__ delta, int dpm,
                                const float* __restrict__ A, float* __restrict__ o,
                                float* __restrict__ dq, float* __restrict__ dk,
-                               float* __restrict__ dv, float* __restrict__ dDelta,
+                               float* __restrict__ dv, float* __restrict__ gpart,
                                float2* __restrict__ ws, long long per_bh) {
   extern __shared__ float4 smem_f4[];
   const int SL = M * (DX + DV + 1);
@@ -306,7 +268,7 @@ __global__ void seq_bwd_kernel(int H, int N, int DX, int DV, int M, const T* __r
   float* den_ws = reinterpret_cast<float*>(blk + static_cast<long long>(kCk + 1) * SL);  // [N]
 
   for (int m = tid; m < M; m += nthr) {
-    ModeD md = mode_consts(delta[h], A, m);
+    ModeD md = mode_consts(delta_hm(delta, dpm, M, h, m), A, m);
     lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
     bb[m] = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
     Am[m] = make_float2(static_cast<float>(md.ar), static_cast<float>(md.ai));
@@ -497,80 +459,32 @@ __global__ void seq_bwd_kernel(int H, int N, int DX, int DV, int M, const T* __r
       __syncthreads();
     }
   }
-  float dd = 0.f;
+  // this sequence's share of the parameter gradients, per mode:
+  //   dL/dDelta_hm = Re(conj(gbar_lambda) A lambda + conj(gbar_b) lambda)
+  //   dL/dA_m      = conj(Delta lambda) gbar_lambda + conj((Delta lambda - b)/A) gbar_b
   for (int m = tid; m < M; m += nthr) {
-    float2 Al = cmul(Am[m], lam[m]);
-    dd += re_conj_mul(glam[m], Al) + re_conj_mul(gbs[m], lam[m]);
-  }
-  dd = warp_sum(dd);
-  if (lane == 0) red[warp] = dd;
-  __syncthreads();
-  if (tid == 0) {
-    float s = 0.f;
-    for (int w = 0; w < nwarp; ++w) s += red[w];
-    atomicAdd(dDelta + h, s);
-  }
-}
-
-// ------------------------------------------------------------------------
-// Inter-segment carry scan of the chunked path (one thread per complex state
-// entry of one (b,h)): carry(s+1) = lambda^L carry(s) + local(s), in the
-// scaled representation S_hat (the per-mode scale commutes with the combine).
-// local and carry are [BH][nseg-1][F2] with F2 = 2M rows x (DX+DV) columns
-// fp32 in the kernel's row layout, plus eta [BH][nseg-1][2M].  carry slot s
-// receives the state entering segment s+1.  Optional state_in (unscaled,
-// public layout) seeds segment 0.
-__global__ void segment_scan_kernel(int H, int DX, int DV, int nseg, int L,
-                                    const HeadTables* __restrict__ tabs,
-                                    const float2* __restrict__ state_in, long long BH,
-                                    float* __restrict__ ws_state, float* __restrict__ ws_eta) {
-  const int F = DX + DV;
-  const long long per = 64LL * F;   // complex entries per (b,h) state (U and Gamma)
-  const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
-  const long long total = BH * (per + 64);
-  if (idx >= total) return;
-  long long bh, e;
-  bool is_eta = idx >= BH * per;
-  if (!is_eta) { bh = idx / per; e = idx % per; } else { bh = (idx - BH * per) / 64; e = (idx - BH * per) % 64; }
-  const int h = static_cast<int>(bh % H);
-  const HeadTables* T = tabs + h;
-  const int m = is_eta ? static_cast<int>(e) : static_cast<int>(e / F);
-  const int f = is_eta ? 0 : static_cast<int>(e % F);
-  double pr, pi;
-  cpow_d(T->re_dA[m], T->im_dA[m], static_cast<double>(L), &pr, &pi);
-  const float2 lamL = make_float2(static_cast<float>(pr), static_cast<float>(pi));
-  float2 carry = make_float2(0.f, 0.f);
-  if (state_in) {
-    float2 s;
-    if (is_eta) s = state_in[BH * 64 * F + bh * 64 + m];
-    else if (f < DX) s = state_in[bh * 64 * DX + m * DX + f];
-    else s = state_in[BH * 64 * DX + bh * 64 * DV + m * DV + (f - DX)];
-    carry = cmul(T->sc_inv[m], s);
-  }
-  for (int s = 0; s + 1 < nseg; ++s) {
-    float* pre;
-    float* pim;
-    if (is_eta) {
-      float* base = ws_eta + (bh * (nseg - 1) + s) * 128;
-      pre = base + 2 * m; pim = base + 2 * m + 1;
-    } else {
-      float* base = ws_state + (bh * (nseg - 1) + s) * 128LL * F;
-      pre = base + (2 * m) * F + f; pim = base + (2 * m + 1) * F + f;
-    }
-    float2 loc = make_float2(*pre, *pim);
-    carry = cfma(lamL, carry, loc);
-    *pre = carry.x;
-    *pim = carry.y;
+    const float dl = delta_hm(delta, dpm, M, h, m);
+    const float2 Al = cmul(Am[m], lam[m]);
+    const float2 dlam = make_float2(dl * lam[m].x, dl * lam[m].y);
+    const float2 num_ = make_float2(dlam.x - bb[m].x, dlam.y - bb[m].y);
+    const float aa = fmaf(Am[m].x, Am[m].x, Am[m].y * Am[m].y);
+    const float2 dbdA = make_float2(fmaf(num_.x, Am[m].x, num_.y * Am[m].y) / aa,
+                                    fmaf(num_.y, Am[m].x, -num_.x * Am[m].y) / aa);
+    float* out = gpart + (bh * M + m) * 3;
+    out[0] = re_conj_mul(glam[m], Al) + re_conj_mul(gbs[m], lam[m]);
+    // conj(x) g summed: real part Re(conj(x) g), imaginary part Im(conj(x) g)
+    out[1] = re_conj_mul(dlam, glam[m]) + re_conj_mul(dbdA, gbs[m]);
+    out[2] = (dlam.x * glam[m].y - dlam.y * glam[m].x) + (dbdA.x * gbs[m].y - dbdA.y * gbs[m].x);
   }
 }
 
 // ------------------------------------------------------------------------
 // host-side launchers
-cudaError_t launch_param_tables(int H, const float* delta, const float* A, HeadTables* tabs,
-                                cudaStream_t st, float* dtab) {
+cudaError_t launch_param_tables(int H, const float* delta, int dpm, const float* A, HeadTables* tabs,
+                                cudaStream_t st, float* dtab, int* flags, int nflags) {
   int* err = device_error_ptr();
   if (!err) return cudaErrorInvalidSymbol;
-  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs, dtab, err);
+  param_tables_kernel<<<H, 4 * kModesTC, 0, st>>>(H, delta, A, tabs, dtab, err, flags, nflags, dpm);
   return cudaGetLastError();
 }
 
@@ -591,7 +505,7 @@ static cudaError_t seq_fwd_impl(const ia_shape_t& s, const void* q, const void* 
   mark_launch_begin(st);
   kern<<<static_cast<unsigned>(BH), 256, smem, st>>>(
       s.H, s.N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
-      static_cast<const T*>(v), delta, A, static_cast<const float2*>(state_in), o, num, den,
+      static_cast<const T*>(v), delta, s.delta_per_mode, A, static_cast<const float2*>(state_in), o, num, den,
       static_cast<float2*>(state_out), BH);
   e = cudaGetLastError();
   mark_launch_end(st);
@@ -618,45 +532,82 @@ size_t seq_bwd_ws_per_bh(int N, int DX, int DV, int M) {   // in float2 units
   return (n + 31) & ~static_cast<size_t>(31);
 }
 
+size_t seq_bwd_workspace_bytes(const ia_shape_t& s) {
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  return sizeof(float2) * BH * seq_bwd_ws_per_bh(s.N, s.d_xi, s.d_v, s.M) + 256 +
+         grad_partials_bytes(s) + 256;
+}
+
 template <typename T>
 static cudaError_t seq_bwd_impl(const ia_shape_t& s, const void* q, const void* k, const void* v,
                                 const float* delta, const float* A, const void* dO, float* o,
-                                float* dq, float* dk, float* dv, float* dDelta, void* ws,
+                                float* dq, float* dk, float* dv, float* dDelta, float* dA, void* ws,
                                 cudaStream_t st) {
   size_t smem = seq_bwd_smem(s.d_xi, s.d_v, s.M);
   auto kern = seq_bwd_kernel<T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(dDelta, 0, sizeof(float) * s.H, st);
-  if (e != cudaSuccess) return e;
   long long BH = static_cast<long long>(s.B) * s.H;
+  const long long per_bh = static_cast<long long>(seq_bwd_ws_per_bh(s.N, s.d_xi, s.d_v, s.M));
+  float2* scratch = static_cast<float2*>(ws);
+  uintptr_t gp = reinterpret_cast<uintptr_t>(scratch + BH * per_bh);
+  float* gpart = reinterpret_cast<float*>((gp + 255) & ~static_cast<uintptr_t>(255));
   mark_launch_begin(st);
   kern<<<static_cast<unsigned>(BH), 256, smem, st>>>(
       s.H, s.N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k),
-      static_cast<const T*>(v), static_cast<const T*>(dO), delta, A, o, dq, dk, dv, dDelta,
-      static_cast<float2*>(ws), static_cast<long long>(seq_bwd_ws_per_bh(s.N, s.d_xi, s.d_v, s.M)));
+      static_cast<const T*>(v), static_cast<const T*>(dO), delta, s.delta_per_mode, A, o, dq, dk, dv, gpart,
+      scratch, per_bh);
   e = cudaGetLastError();
   mark_launch_end(st);
-  return e;
+  if (e != cudaSuccess) return e;
+  return launch_grad_reduce(s, gpart, dDelta, dA, st);
 }
 
 cudaError_t launch_seq_bwd(const ia_shape_t& s, const void* q, const void* k, const void* v,
                            const float* delta, const float* A, const void* dO, float* o, float* dq,
-                           float* dk, float* dv, float* dDelta, void* ws, cudaStream_t st) {
+                           float* dk, float* dv, float* dDelta, float* dA, void* ws, cudaStream_t st) {
   if (s.in_dtype == IA_F32)
-    return seq_bwd_impl<float>(s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, ws, st);
-  return seq_bwd_impl<__nv_bfloat16>(s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, ws, st);
+    return seq_bwd_impl<float>(s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, dA, ws, st);
+  return seq_bwd_impl<__nv_bfloat16>(s, q, k, v, delta, A, dO, o, dq, dk, dv, dDelta, dA, ws, st);
 }
 
-cudaError_t launch_segment_scan(int B, int H, int DX, int DV, int nseg, int L,
-                                const HeadTables* tabs, const void* state_in, float* ws_state,
-                                float* ws_eta, cudaStream_t st) {
-  long long BH = static_cast<long long>(B) * H;
-  long long total = BH * (64LL * (DX + DV) + 64);
-  unsigned blocks = static_cast<unsigned>((total + 255) / 256);
-  segment_scan_kernel<<<blocks, 256, 0, st>>>(H, DX, DV, nseg, L, tabs,
-                                               static_cast<const float2*>(state_in), BH, ws_state,
-                                               ws_eta);
+// ------------------------------------------------------------------------
+// dDelta and dA from the per-(b,h,m) partials of a reverse pass, summed in a
+// fixed order (b, then h, then m), so that the result is the same on every
+// run.  One thread per output: dDelta[h] or dDelta[h][m], then dA[m].
+__global__ void grad_reduce_kernel(int B, int H, int M, int dpm, const float* __restrict__ gpart,
+                                   float* __restrict__ dDelta, float* __restrict__ dA) {
+  const int nD = dpm ? H * M : H;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < nD) {
+    const int h = dpm ? idx / M : idx;
+    const int m0 = dpm ? idx % M : 0, m1 = dpm ? m0 + 1 : M;
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b)
+      for (int m = m0; m < m1; ++m) acc += gpart[((static_cast<long long>(b) * H + h) * M + m) * 3];
+    dDelta[idx] = acc;
+  } else if (dA && idx < nD + M) {
+    const int m = idx - nD;
+    float re = 0.f, im = 0.f;
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h) {
+        const float* p = gpart + ((static_cast<long long>(b) * H + h) * M + m) * 3;
+        re += p[1];
+        im += p[2];
+      }
+    dA[2 * m] = re;
+    dA[2 * m + 1] = im;
+  }
+}
+
+size_t grad_partials_bytes(const ia_shape_t& s) {
+  return sizeof(float) * 3 * static_cast<size_t>(s.B) * s.H * s.M;
+}
+
+cudaError_t launch_grad_reduce(const ia_shape_t& s, const float* gpart, float* dDelta, float* dA,
+                               cudaStream_t st) {
+  const int n = (s.delta_per_mode ? s.H * s.M : s.H) + s.M;
+  grad_reduce_kernel<<<(n + 127) / 128, 128, 0, st>>>(s.B, s.H, s.M, s.delta_per_mode, gpart, dDelta, dA);
   return cudaGetLastError();
 }
 

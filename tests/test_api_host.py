@@ -71,8 +71,17 @@ def test_workspace_checked_before_launch(lib):
     assert prefill(lib, s, ws=FAKE, wsb=need - 1) == 3
     fb = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(s))
     rc = lib.ia_fwd_bwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE,
-                        FAKE, FAKE, ctypes.c_size_t(fb - 1), None)
+                        FAKE, FAKE, FAKE, ctypes.c_size_t(fb - 1), None)
     assert rc == 3
+
+
+def test_delta_per_mode_flag_checked(lib):
+    s = shape()
+    s.delta_per_mode = 2                                # only 0 ([H]) and 1 ([H,M]) are defined
+    assert prefill(lib, s) == 1
+    assert lib.ia_state_bytes(ctypes.byref(s)) == 0
+    s.delta_per_mode = 1
+    assert prefill(lib, s) == 3                         # valid: fails later, on the missing workspace
 
 
 def test_decode_validation(lib):
@@ -93,8 +102,9 @@ def test_injected_launch_failure(lib, monkeypatch):
     assert rc == 4
     need = lib.ia_fwd_bwd_workspace_bytes(ctypes.byref(s))
     rc = lib.ia_fwd_bwd(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                        FAKE, ctypes.c_size_t(need), None)
+                        None, FAKE, ctypes.c_size_t(need), None)
     assert rc == 4
+    assert lib.ia_selftest_wait_expiry(ctypes.c_ulonglong(1000000), FAKE, None) == 4
     t = shape(B=1, H=2, N=100, dx=64, dv=64, M=64, dt=1)   # the no-allocation entry point: bf16, M = 64
     rc = lib.ia_prefill_fwd_static(ctypes.byref(t), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None,
                                    None, None)
@@ -156,38 +166,37 @@ def test_missing_library_fails_loudly(monkeypatch):
         ia.load_library()
 
 
-def _segments(lib, s, monkeypatch):
-    """Segments per sequence of the tensor-core plan, read from the workspace
-    size: each boundary between segments keeps one carried state per (b,h)."""
-    ws = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
-    monkeypatch.setenv("IA_PREFILL_SEGMENTS", "1")
-    ws1 = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
-    monkeypatch.delenv("IA_PREFILL_SEGMENTS")
-    per_bh = lib.ia_state_bytes(ctypes.byref(s)) // (s.B * s.H)
-    extra = ws - ws1
-    assert extra % (s.B * s.H * per_bh) == 0
-    return 1 + extra // (s.B * s.H * per_bh)
-
-
-@pytest.mark.parametrize("B,H,N,d,nseg", [
-    (8, 12, 2048, 64, 1),    # 125M prefill: 96 sequences, one pass
-    (8, 16, 2048, 64, 1),    # 350M training shape: 128 sequences
-    (4, 16, 2048, 128, 2),   # 1.3B prefill: 64 sequences of 32 chunks -> 2 x 16 chunks on 128 CTAs
-    (1, 16, 7168, 128, 9),   # 1.3B long context: 16 x 112 chunks -> 9 x 13 chunks on 144 CTAs
+@pytest.mark.parametrize("B,H,N,dx,dv,grid,splits", [
+    (8, 12, 2048, 64, 64, 148, True),      # 125M prefill: 96 sequences x 32 chunks over all 148 SMs
+    (8, 16, 2048, 64, 64, 128, False),     # 350M training shape: 128 whole streams beat 148 ranges of 27.7
+    (4, 16, 2048, 128, 128, 128, False),   # 1.3B prefill: 64 sequences x 2 value blocks, whole streams
+    (1, 16, 7168, 128, 128, 148, True),    # 1.3B long context: 32 streams x 112 chunks over 148 SMs
+    (37, 4, 256, 64, 64, 148, False),      # 148 streams of 4 chunks: one whole stream per SM
+    (1, 2, 200, 64, 64, 2, False),         # 2 streams of 4 chunks: pieces shorter than 4 do not pay
 ])
-def test_segment_plan_on_148_sms(lib, monkeypatch, B, H, N, d, nseg):
-    # With no GPU the planner assumes a B200's 148 SMs.  Splitting pays when
-    # the sequences alone leave SMs idle: a state-only pass and the carry scan
-    # then precede the full pass (4 launches instead of tables + full pass).
-    s = shape(B=B, H=H, N=N, dx=d, dv=d, M=64, dt=1)
-    assert _segments(lib, s, monkeypatch) == nseg
-    assert lib.ia_prefill_launches(ctypes.byref(s)) == (4 if nseg > 1 else 2)
+def test_chunk_pass_plan_on_148_sms(lib, B, H, N, dx, dv, grid, splits):
+    # With no GPU the planner assumes a B200's 148 SMs.  Each CTA takes an
+    # equal range of the (stream, chunk) space; when a range starts inside a
+    # stream the workspace also holds the look-back states (two per CTA).
+    # (the planner's cost model may trade a few CTAs for better-aligned ranges)
+    s = shape(B=B, H=H, N=N, dx=dx, dv=dv, M=64, dt=1)
+    got = lib.ia_prefill_grid(ctypes.byref(s))
+    assert (grid - 8 <= got <= grid) if splits else got == grid
+    assert lib.ia_prefill_launches(ctypes.byref(s)) == 2
+    tables = H * 20992 + 256
+    ws = lib.ia_prefill_workspace_bytes(ctypes.byref(s))
+    per_cta = 2 * (128 * (dx + 64) + 128) * 4 + 4
+    assert ws == (tables + got * per_cta + 256 if splits else tables)
 
 
-def test_segment_override_and_cuda_core_path(lib, monkeypatch):
+def test_grid_override_and_cuda_core_path(lib, monkeypatch):
     s = shape(B=8, H=12, N=2048, dx=64, dv=64, M=64, dt=1)
-    monkeypatch.setenv("IA_PREFILL_SEGMENTS", "4")
-    assert lib.ia_prefill_launches(ctypes.byref(s)) == 4
-    monkeypatch.delenv("IA_PREFILL_SEGMENTS")
-    # fp32 inputs run the sequential CUDA-core kernel: one launch, no segments
-    assert lib.ia_prefill_launches(ctypes.byref(shape(B=1, H=2, N=256, dx=16, dv=16, M=16, dt=0))) == 1
+    monkeypatch.setenv("IA_PREFILL_GRID", "7")
+    assert lib.ia_prefill_grid(ctypes.byref(s)) == 7
+    monkeypatch.setenv("IA_PREFILL_GRID", "100000")
+    assert lib.ia_prefill_grid(ctypes.byref(s)) == 148     # at most one CTA per SM
+    monkeypatch.delenv("IA_PREFILL_GRID")
+    # fp32 inputs run the sequential CUDA-core kernel: one launch, no chunk-pass grid
+    t = shape(B=1, H=2, N=256, dx=16, dv=16, M=16, dt=0)
+    assert lib.ia_prefill_launches(ctypes.byref(t)) == 1
+    assert lib.ia_prefill_grid(ctypes.byref(t)) == 0

@@ -1,4 +1,4 @@
-"""Training-step parity on the GPU: o, dq, dk, dv and dDelta against the
+"""Training-step parity on the GPU: o, dq, dk, dv, dDelta and dA against the
 oracle's reverse-mode adjoint (itself pinned by finite differences and the
 tangent/adjoint dot-product test)."""
 import numpy as np
@@ -26,12 +26,19 @@ def run(inp, M, dev):
     return {k: v.cpu() for k, v in r.items()}
 
 
+def vec_rel(x, r):
+    x = x.double().numpy() if hasattr(x, "double") else np.asarray(x)
+    return float(np.abs(x - r).max() / np.abs(r).max())
+
+
 def compare(r, g, tol):
     assert slice_rel(r["dq"], g["dq"], (-2, -1)) < tol
     assert slice_rel(r["dk"], g["dk"], (-2, -1)) < tol
     assert slice_rel(r["dv"], g["dv"], (-2, -1)) < tol
-    dd = np.abs(r["dDelta"].double().numpy() - g["dDelta"]).max() / np.abs(g["dDelta"]).max()
+    dd = vec_rel(r["dDelta"], g["dDelta"])
     assert dd < tol, dd
+    da = vec_rel(r["dA"], g["dA"])
+    assert da < tol, da
 
 
 @pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])

@@ -1,0 +1,110 @@
+"""The layer's optional parts on the GPU (ia_prefill_fwd_ex, ia_decode_step_ex)
+against the fp64 oracle's extended forward, itself pinned by mpmath brute
+force, closed forms and invariants: the RMSNorm with per-head gain and bias on
+the SSM input, a step per token (selective writing and memory decay), the
+complex readout matrix and the bidirectional layer."""
+import numpy as np
+import pytest
+import torch
+
+import ssm_token_mixer_b200 as ia
+from gpu_common import device
+from parity import TOL_BF16, TOL_F32, report, slice_rel
+from ssm_token_mixer_b200 import synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    return device()
+
+
+def options(B, H, N, dx, dv, M, seed, which):
+    g = torch.Generator().manual_seed(seed)
+    o = {}
+    if "selective" in which:
+        o["delta_t"] = torch.exp(np.log(5e-3) + torch.rand(B, H, N, generator=g) * (np.log(2e-1) - np.log(5e-3)))
+    if "norm" in which:
+        o["gain"] = 0.5 + torch.rand(H, dx + dv, generator=g)
+        o["bias"] = 0.3 * torch.randn(H, dx + dv, generator=g)
+    if "readout" in which:
+        o["W"] = (torch.randn(H, M, M, 2, generator=g) / np.sqrt(M)) + torch.eye(M)[None, :, :, None] * \
+            torch.tensor([1.0, 0.0])
+    return o
+
+
+def to_oracle(o):
+    r = {k: v for k, v in o.items() if k != "W"}
+    if "W" in o:
+        W = o["W"].double().numpy()
+        r["W"] = W[..., 0] + 1j * W[..., 1]
+    return r
+
+
+CASES = [("selective",), ("norm",), ("readout",), ("selective", "norm", "readout")]
+
+
+@pytest.mark.parametrize("which", CASES, ids=["+".join(c) for c in CASES])
+@pytest.mark.parametrize("dtype,dx,dv,M,tol", [("f32", 16, 12, 8, TOL_F32), ("bf16", 64, 64, 64, TOL_BF16)])
+def test_prefill_with_optional_parts(oracle_mod, dev, which, dtype, dx, dv, M, tol):
+    B, H, N = 2, 3, 130
+    inp = synthetic.layer_inputs(B, H, N, dx, dv, dtype, seed=80 + dx)
+    opt = options(B, H, N, dx, dv, M, 81, which)
+    delta = None if "selective" in which else inp["delta"]
+    g = lambda x: None if x is None else x.to(dev)
+    r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta=g(delta), want_num_den=True,
+                          want_state=True, **{k: g(v) for k, v in opt.items()})
+    ia.check_device_errors()
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=delta, **to_oracle(opt))
+    rep = report(r["num"].cpu(), r["den"].cpu(), r["o"].cpu(), ref)
+    assert max(rep.values()) < tol, rep
+    st = r["state"].cpu().double().numpy()
+    assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < tol
+
+
+def test_split_prefill_and_decode_with_optional_parts(oracle_mod, dev):
+    # P12/P13 with every part on: prefill(N1) -> state -> prefill(N2) and
+    # decode steps equal the oracle on the whole sequence
+    B, H, dx, dv, M, N1, N2, K = 2, 2, 16, 16, 8, 70, 40, 3
+    N = N1 + N2 + K
+    inp = synthetic.layer_inputs(B, H, N, dx, dv, "f32", seed=82)
+    opt = options(B, H, N, dx, dv, M, 83, ("selective", "norm", "readout"))
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, **to_oracle(opt))
+    g = lambda x: x.to(dev)
+    sl = lambda x, a, b: x[:, :, a:b].contiguous()
+    kw = lambda a, b: {"delta_t": g(sl(opt["delta_t"], a, b)), "gain": g(opt["gain"]), "bias": g(opt["bias"]),
+                       "W": g(opt["W"])}
+    r1 = ia.prefill_fwd_ex(*(g(sl(inp[n], 0, N1)) for n in ("q", "k", "v")), M, want_state=True, **kw(0, N1))
+    r2 = ia.prefill_fwd_ex(*(g(sl(inp[n], N1, N1 + N2)) for n in ("q", "k", "v")), M, want_state=True,
+                           state_in=r1["state"], **kw(N1, N1 + N2))
+    o = torch.cat([r1["o"].cpu(), r2["o"].cpu()], dim=2)
+    assert slice_rel(o, ref["o"][:, :, :N1 + N2], (-2, -1)) < TOL_F32
+    state = r2["state"]
+    for t in range(N1 + N2, N):
+        tok = lambda n: g(inp[n][:, :, t].contiguous())
+        r = ia.decode_step_ex(tok("q"), tok("k"), tok("v"), state, M, delta_t=g(opt["delta_t"][:, :, t].contiguous()),
+                              gain=g(opt["gain"]), bias=g(opt["bias"]), W=g(opt["W"]))
+        ia.check_device_errors()
+        assert slice_rel(r["o"].cpu(), ref["o"][:, :, t], (-1,)) < TOL_F32
+
+
+@pytest.mark.parametrize("dtype,tol", [("f32", TOL_F32), ("bf16", TOL_BF16)])
+def test_bidirectional_layer(oracle_mod, dev, dtype, tol):
+    B, H, N, d, M = 2, 3, 90, 16, 8
+    inp = synthetic.layer_inputs(B, H, N, d, d, dtype, seed=84)
+    opt = options(B, H, N, d, d, M, 85, ("selective",))
+    g = lambda x: x.to(dev)
+    r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta_t=g(opt["delta_t"]), bidirectional=True)
+    ia.check_device_errors()
+    ref = oracle_mod.forward_bidirectional(inp["q"], inp["k"], inp["v"], M, delta_t=opt["delta_t"])
+    assert slice_rel(r["o"].cpu(), ref, (-2, -1)) < tol
+
+
+def test_no_options_is_the_plain_layer(dev):
+    inp = synthetic.layer_inputs(2, 2, 150, 64, 64, "bf16", seed=86)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    a = ia.prefill_fwd(g["q"], g["k"], g["v"], g["delta"], 64, want_num_den=True)
+    b = ia.prefill_fwd_ex(g["q"], g["k"], g["v"], 64, delta=g["delta"], want_num_den=True)
+    ia.check_device_errors()
+    assert slice_rel(b["num"].cpu(), a["num"].cpu(), (-2, -1)) < TOL_BF16

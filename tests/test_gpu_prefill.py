@@ -2,8 +2,6 @@
 fp64 oracle on the same seeded inputs.  Bars: 1e-4 for fp32 inputs, 2e-2
 for bf16 inputs, normwise per (b,h) slice on num and den separately (o where
 den is away from zero) -- see parity.py."""
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -63,11 +61,12 @@ def test_tensor_core_prefill_small(oracle_mod, dev, dx, dv, N):
                 TOL_BF16)
 
 
-def test_tensor_core_segments_and_tail(oracle_mod, dev):
-    # few (b,h) pairs and a long ragged sequence: the planner splits it into
-    # segments, so the state-only pass and the carry scan both run
+def test_tensor_core_long_ragged_sequence(oracle_mod, dev):
+    # few (b,h) pairs and a long ragged sequence: the planner spreads the
+    # chunks over many CTAs, so most ranges start inside the sequence and
+    # take their carried state from the look-back
     B, H, N, d, M = 1, 2, 1000, 64, 64
-    assert ia.prefill_workspace_bytes(B, H, N, d, d, M, "bf16") > 2 * 21504
+    assert ia.prefill_grid(B, H, N, d, d, M, "bf16") > 2
     inp = synthetic.layer_inputs(B, H, N, d, d, "bf16", seed=11)
     r = gpu_prefill(inp, M, dev)
     ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
@@ -95,27 +94,31 @@ def test_state_in_and_split_prefill(oracle_mod, dev, dtype, tol):
     check_state(r2["state"], oracle_mod.split_state(ref["state"], B, H, M, d, d), B, H, M, d, d, tol)
 
 
-@pytest.mark.parametrize("variant", ["0", "1", "2"])
-@pytest.mark.parametrize("N,with_state", [(1, False), (37, True), (200, False), (1000, True)])
-def test_d64_chunk_pass_variants(oracle_mod, dev, monkeypatch, variant, N, with_state):
-    # the three d=64 full-pass kernels (one role for all warps, one epilogue
-    # group beside the MMA warp, two epilogue groups) against the oracle, on
-    # ragged lengths, a carried state and (N=1000, B*H=2) split segments
-    monkeypatch.setenv("IA_PREFILL_WS", variant)
-    B, H, d, M = 1, 2, 64, 64
-    N0 = 75 if with_state else 0
-    inp = synthetic.layer_inputs(B, H, N0 + N, d, d, "bf16", seed=31 + N)
-    st = None
-    if with_state:
-        head = {k: (v[:, :, :N0].contiguous() if k != "delta" else v) for k, v in inp.items()}
-        st = gpu_prefill(head, M, dev)["state"].to(dev)
+@pytest.mark.parametrize("dx,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("grid", [1, 2, 5, 7, 13, 29, 60])
+def test_chunk_pass_ranges(oracle_mod, dev, monkeypatch, dx, dv, grid):
+    # The chunk pass gives every CTA an equal range of the (stream, chunk)
+    # space.  Forcing the grid exercises every kind of range: many whole
+    # streams of different heads in one CTA (grid 1), ranges that start
+    # inside a stream and take their state from one or several predecessors,
+    # single-piece ranges inside a stream that publish an inclusive state for
+    # the next, and ragged last chunks -- all from a carried state_in, with
+    # the end state checked too.
+    B, H, M = 2, 3, 64
+    N0, N = 75, 300                   # 5 chunks per stream, the last one ragged
+    inp = synthetic.layer_inputs(B, H, N0 + N, dx, dv, "bf16", seed=31 + grid + dx + dv)
+    head = {k: (v[:, :, :N0].contiguous() if k != "delta" else v) for k, v in inp.items()}
+    st = gpu_prefill(head, M, dev)["state"].to(dev)
     tail = {k: (v[:, :, N0:].contiguous() if k != "delta" else v) for k, v in inp.items()}
+    monkeypatch.setenv("IA_PREFILL_GRID", str(grid))
+    total = B * H * (dv // 64) * ((N + 63) // 64)
+    assert ia.prefill_grid(B, H, N, dx, dv, M, "bf16") == min(grid, total)
     r = gpu_prefill(tail, M, dev, state_in=st)
     ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
     ref_tail = {"num": ref["num"][:, :, N0:], "den": ref["den"][:, :, N0:], "o": ref["o"][:, :, N0:]}
     rep = report(r["num"], r["den"], r["o"], ref_tail)
     assert max(rep.values()) < TOL_BF16, rep
-    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, d, d), B, H, M, d, d, TOL_BF16)
+    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, dx, dv), B, H, M, dx, dv, TOL_BF16)
 
 
 def test_first_token_returns_v(dev):
