@@ -50,6 +50,24 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Like mbar_test, but a thread whose phase is not complete sleeps until it
+// completes or about hint_ns have passed, instead of returning at once: a
+// waiting warp then takes no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Sleep per try in the bounded waits: short against the one-second limit and
+// the abort flag's reaction time, long against a chunk's work.
+constexpr uint32_t kSleepHintNs = 4000;
+
 // Device error flag bits (the library's flag, read and cleared by
 // ia_check_device_errors): a bounded wait expired; a parameter was outside
 // the range the tensor-core operands hold.
@@ -63,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
                                           unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   unsigned long long t0 = global_ns();
-  while (!mbar_test(bar, parity)) {
+  while (!mbar_test_sleep(bar, parity, kSleepHintNs)) {
     if (global_ns() - t0 > limit_ns) {
       atomicOr(err, kErrTimeout);
       return false;
@@ -84,7 +102,7 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
                                                    unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   unsigned long long t0 = global_ns();
-  while (!mbar_test(bar, parity)) {
+  while (!mbar_test_sleep(bar, parity, kSleepHintNs)) {
     if (*abort) return false;
     if (global_ns() - t0 > limit_ns) {
       atomicOr(err, kErrTimeout);

@@ -1055,10 +1055,13 @@ __global__ void __launch_bounds__(NTH, 1)
 }
 
 // Chunks a CTA carries under grid G: the largest range, plus the state-only
-// chain of a last piece that ends inside a stream (about a quarter of a full
-// chunk each), plus the hops of the look-back.
+// chain of a last piece that ends inside a stream, plus the hops of the
+// look-back.  A state-only chunk costs nearly as much as a full one (on a
+// B200, 96 whole 32-chunk streams of d = 64 take 115 us, the same work as 144
+// ranges with their state-only chains 155 us): the chain of conversion,
+// rotation and G7 that it runs is the latency-bound part of a full chunk.
 double plan_cost(long long total, int nch, int G) {
-  constexpr double kStateOnly = 0.25, kHop = 0.5;
+  constexpr double kStateOnly = 0.9, kHop = 0.5;
   double worst = 0.0;
   for (int c = 0; c < G; ++c) {
     const long long g0 = total * c / G, g1 = total * (c + 1) / G;

@@ -167,7 +167,7 @@ def test_missing_library_fails_loudly(monkeypatch):
 
 
 @pytest.mark.parametrize("B,H,N,dx,dv,grid,splits", [
-    (8, 12, 2048, 64, 64, 148, True),      # 125M prefill: 96 sequences x 32 chunks over all 148 SMs
+    (8, 12, 2048, 64, 64, 96, False),      # 125M prefill: 96 whole sequences beat 144 ranges and their state-only chains
     (8, 16, 2048, 64, 64, 128, False),     # 350M training shape: 128 whole streams beat 148 ranges of 27.7
     (4, 16, 2048, 128, 128, 128, False),   # 1.3B prefill: 64 sequences x 2 value blocks, whole streams
     (1, 16, 7168, 128, 128, 148, True),    # 1.3B long context: 32 streams x 112 chunks over 148 SMs
