@@ -50,6 +50,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Tests a phase without ever suspending the thread (mbar_test may wait a
+// while for the phase before it answers): for a thread that polls several
+// barriers in turn.
+__device__ __forceinline__ bool mbar_probe(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Like mbar_test, but a thread whose phase is not complete sleeps until it
 // completes or about hint_ns have passed, instead of returning at once: a
 // waiting warp then takes no issue slots from the warps doing the work.
