@@ -6,10 +6,10 @@
 //   a = U xi(q),  o = Re(a^H Gamma) / Re(a^H eta)
 //
 // The step is bound by state bytes: every state entry is read and written
-// once in fp32.  A thread-block cluster serves one (b,h); each CTA of the
-// cluster streams a group of modes with 16-byte loads and stores, keeps its
-// partial num/den in shared memory, and the cluster's rank-0 CTA sums the
-// partials over distributed shared memory and writes o.
+// once in fp32.  A cluster of 1-8 CTAs serves one (b,h); each CTA streams a
+// group of modes through shared memory with bulk copies and writes them back
+// with 16-byte stores, and the cluster's rank-0 CTA sums the partial num/den
+// over distributed shared memory and writes o.
 #include <cstdlib>
 #include <cooperative_groups.h>
 
@@ -21,9 +21,7 @@ namespace cg = cooperative_groups;
 namespace ia {
 namespace {
 
-constexpr int kDecThreads = 256;
 constexpr int kVecPerLane = 4;   // rows up to 256 complex entries (d <= 256)
-constexpr int kModesPerWarp = 2;  // up to 16 modes per CTA
 
 template <typename T>
 __device__ __forceinline__ float ldx(const T* p);
@@ -36,172 +34,20 @@ __device__ __forceinline__ float ldx<__nv_bfloat16>(const __nv_bfloat16* p) {
 
 __device__ __forceinline__ float xi_acc(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
-// shared: fq [DX] | fk [DX] | vv [DV] | part [8 warps][DV] | pden [8] | lam,b [MG] float2
-template <typename T>
-__global__ void __launch_bounds__(kDecThreads) decode_kernel(
-    int H, int DX, int DV, int M, int MG, const T* __restrict__ q, const T* __restrict__ k,
-    const T* __restrict__ v, const float* __restrict__ delta, int dpm, const float* __restrict__ A,
-    float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
-    float* __restrict__ den, long long BH) {
-  extern __shared__ float4 dsm[];
-  float* fq = reinterpret_cast<float*>(dsm);
-  float* fk = fq + DX;
-  float* vv = fk + DX;
-  float* part = vv + DV;                    // [8][DV]
-  float* pden = part + 8 * DV;              // [8]
-  float2* lamb = reinterpret_cast<float2*>(pden + 8);   // [MG] lambda, [MG] b
-  float2* bb = lamb + MG;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int g = static_cast<int>(cluster.block_rank());
-  const int G = static_cast<int>(cluster.num_blocks());
-  const long long bh = blockIdx.x / G;
-  const int h = static_cast<int>(bh % H);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = g * MG;
-  const int nu = DX / 2, ng = DV / 2;   // 16-byte vectors (two complex entries) per row
-
-  float2* Ub = state + bh * M * DX;
-  float2* Gb = state + BH * M * DX + bh * M * DV;
-  float2* Eb = state + BH * M * (DX + DV) + bh * M;
-
-  // Issue every state load of this warp's modes first, so that HBM latency
-  // overlaps the parameter and feature set-up below.
-  float4 uv[kModesPerWarp][kVecPerLane], gv[kModesPerWarp][kVecPerLane];
-  float2 ev[kModesPerWarp];
-#pragma unroll
-  for (int r = 0; r < kModesPerWarp; ++r) {
-    const int mi = warp + 8 * r, m = m0 + mi;
-    const bool ok = mi < MG && m < M;
-    const float4* Ur = reinterpret_cast<const float4*>(Ub + static_cast<long long>(m) * DX);
-    const float4* Gr = reinterpret_cast<const float4*>(Gb + static_cast<long long>(m) * DV);
-#pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i) {
-      const int p = lane + 32 * i;
-      if (ok && p < nu) uv[r][i] = Ur[p];
-      if (ok && p < ng) gv[r][i] = Gr[p];
-    }
-    ev[r] = (ok && lane == 0) ? Eb[m] : make_float2(0.f, 0.f);
-  }
-
-  for (int f = tid; f < DX; f += kDecThreads) {
-    fq[f] = xi_acc(ldx(q + bh * DX + f));
-    fk[f] = xi_acc(ldx(k + bh * DX + f));
-  }
-  for (int f = tid; f < DV; f += kDecThreads) vv[f] = ldx(v + bh * DV + f);
-  for (int i = tid; i < MG; i += kDecThreads) {
-    // lambda = exp(Delta A), b = (lambda - 1)/A in fp32; lambda - 1 is formed
-    // as expm1(x) cos(y) - 2 sin^2(y/2) + i e^x sin(y) so it keeps its
-    // relative accuracy for small Delta.
-    const int m = m0 + i;
-    const float ar = A ? A[2 * m] : -0.5f;
-    const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
-    const float d = delta_hm(delta, dpm, M, h, m);
-    const float x = d * ar, y = d * ai;
-    float sy, cy, sh, ch;
-    sincosf(y, &sy, &cy);
-    sincosf(0.5f * y, &sh, &ch);
-    const float ex = expf(x), em1 = expm1f(x);
-    const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;   // lambda - 1
-    const float dd = fmaf(ar, ar, ai * ai);
-    lamb[i] = make_float2(ex * cy, ex * sy);
-    bb[i] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
-  }
-  for (int i = tid; i < 8 * DV + 8; i += kDecThreads) part[i] = 0.f;
-  __syncthreads();
-
-  float* mypart = part + warp * DV;
-  float dpart = 0.f;
-#pragma unroll
-  for (int r = 0; r < kModesPerWarp; ++r) {
-    const int mi = warp + 8 * r, m = m0 + mi;
-    if (mi >= MG || m >= M) break;
-    const float2 L = lamb[mi], Bm = bb[mi];
-    float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
-    float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
-    float ar = 0.f, ai = 0.f;
-#pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i) {
-      const int p = lane + 32 * i;
-      if (p < nu) {
-        const float4 u = uv[r][i];
-        const float x0 = fk[2 * p], x1 = fk[2 * p + 1];
-        float4 w;
-        w.x = fmaf(L.x, u.x, fmaf(-L.y, u.y, Bm.x * x0));
-        w.y = fmaf(L.x, u.y, fmaf(L.y, u.x, Bm.y * x0));
-        w.z = fmaf(L.x, u.z, fmaf(-L.y, u.w, Bm.x * x1));
-        w.w = fmaf(L.x, u.w, fmaf(L.y, u.z, Bm.y * x1));
-        Ur[p] = w;
-        ar = fmaf(w.x, fq[2 * p], fmaf(w.z, fq[2 * p + 1], ar));
-        ai = fmaf(w.y, fq[2 * p], fmaf(w.w, fq[2 * p + 1], ai));
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      ar += __shfl_xor_sync(0xffffffffu, ar, off);
-      ai += __shfl_xor_sync(0xffffffffu, ai, off);
-    }
-#pragma unroll
-    for (int i = 0; i < kVecPerLane; ++i) {
-      const int p = lane + 32 * i;
-      if (p < ng) {
-        const float4 gq = gv[r][i];
-        const float x0 = vv[2 * p], x1 = vv[2 * p + 1];
-        float4 w;
-        w.x = fmaf(L.x, gq.x, fmaf(-L.y, gq.y, Bm.x * x0));
-        w.y = fmaf(L.x, gq.y, fmaf(L.y, gq.x, Bm.y * x0));
-        w.z = fmaf(L.x, gq.z, fmaf(-L.y, gq.w, Bm.x * x1));
-        w.w = fmaf(L.x, gq.w, fmaf(L.y, gq.z, Bm.y * x1));
-        Gr[p] = w;
-        mypart[2 * p] += fmaf(ar, w.x, ai * w.y);       // Re(conj(a) Gamma)
-        mypart[2 * p + 1] += fmaf(ar, w.z, ai * w.w);
-      }
-    }
-    if (lane == 0) {
-      const float2 e = ev[r];
-      const float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
-      Eb[m] = w;
-      dpart += fmaf(ar, w.x, ai * w.y);
-    }
-  }
-  if (lane == 0) pden[warp] = dpart;
-  __syncthreads();
-  // CTA partial: fold the 8 warp rows into row 0
-  for (int f = tid; f < DV; f += kDecThreads) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += part[w * DV + f];
-    part[f] = s;
-  }
-  if (tid == 0) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += pden[w];
-    pden[0] = s;
-  }
-  cluster.sync();
-  if (g == 0) {
-    float dn = 0.f;
-    for (int r = 0; r < G; ++r) dn += cluster.map_shared_rank(pden, r)[0];
-    for (int f = tid; f < DV; f += kDecThreads) {
-      float s = 0.f;
-      for (int r = 0; r < G; ++r) s += cluster.map_shared_rank(part, r)[f];
-      o[bh * DV + f] = s / dn;
-      if (num) num[bh * DV + f] = s;
-    }
-    if (den && tid == 0) den[bh] = dn;
-  }
-  cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
-}
-
-// Large-batch variant: one CTA per (b,h) covers all modes, so no cluster and
-// no cross-CTA reduction is needed.  Each warp walks its modes (warp, warp+8,
-// ...) through a ring of D shared-memory slots: bulk copies bring the U and
-// Gamma rows of the next D modes while it updates the current one, so each SM
-// keeps enough bytes in flight to cover the memory latency; the updated rows
-// go straight back to HBM and the partial Re(a^H Gamma) stays in registers.
+// Streaming variant: a cluster of S CTAs (S = 1, 2, 4 or 8) serves one
+// (b,h), CTA r taking modes [r M/S, (r+1) M/S).  Each warp walks its modes
+// (warp, warp+8, ... of that range) through a ring of D shared-memory slots:
+// bulk copies bring the U and Gamma rows of the next D modes while it
+// updates the current one, so each SM keeps enough bytes in flight to cover
+// the memory latency; the updated rows go straight back to HBM and the
+// partial Re(a^H Gamma) stays in registers.  Small batches take S > 1 so
+// that every SM holds several CTAs and each warp's rows are all in flight at
+// once; the cluster's rank-0 CTA then adds the partials of the others over
+// distributed shared memory, in rank order.
 constexpr int kBhWarps = 8;
 
 template <typename T>
-__global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
+__global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
     int H, int DX, int DV, int M, int D, const T* __restrict__ q, const T* __restrict__ k,
     const T* __restrict__ v, const float* __restrict__ delta, int dpm, const float* __restrict__ A,
     float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
@@ -219,24 +65,50 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
   float2* lamb = reinterpret_cast<float2*>(pden + kBhWarps);   // [M]
   float2* bb = lamb + M;
   float2* eta = bb + M;
-  const long long bh = blockIdx.x;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int S = static_cast<int>(cluster.num_blocks());
+  const long long bh = blockIdx.x / S;
   const int h = static_cast<int>(bh % H);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nu = DX / 2, ng = DV / 2;
+  const int MS = M / S, m_lo = rank * MS;   // this CTA's modes
   float2* Ub = state + bh * M * DX;
   float2* Gb = state + BH * M * DX + bh * M * DV;
   float2* Eb = state + BH * M * (DX + DV) + bh * M;
   uint8_t* myring = ring + warp * D * slot;
   uint64_t* mybar = bars + warp * D;
-  const int nj = warp < M ? (M - warp + kBhWarps - 1) / kBhWarps : 0;   // modes warp, warp + 8, ...
+  const int nj = warp < MS ? (MS - warp + kBhWarps - 1) / kBhWarps : 0;   // modes m_lo + warp, + 8, ...
 
   // each warp streams its own modes' state rows through its ring, D rows ahead
   auto issue = [&](int j) {
-    const int m = warp + kBhWarps * j, s = j % D;
+    const int m = m_lo + warp + kBhWarps * j, s = j % D;
     mbar_arrive_expect_tx(mybar + s, slot);
     bulk_g2s(myring + s * slot, Ub + static_cast<long long>(m) * DX, rowU, mybar + s);
     bulk_g2s(myring + s * slot + rowU, Gb + static_cast<long long>(m) * DV, rowG, mybar + s);
   };
+  // The per-(b,h) inputs (q, k, v, Delta, A, eta) are loaded first, in one
+  // round trip, ahead of the ring's bulk copies: behind them, each of these
+  // small dependent loads would wait out the copies' queue.
+  constexpr int NT = kBhWarps * 32;
+  float xq = 0.f, xk = 0.f, xv = 0.f, pd = 0.f, par = -0.5f, pai = 0.f;
+  float2 pe = make_float2(0.f, 0.f);
+  if (tid < DX) {
+    xq = ldx(q + bh * DX + tid);
+    xk = ldx(k + bh * DX + tid);
+  }
+  if (tid < DV) xv = ldx(v + bh * DV + tid);
+  if (tid < MS) {
+    const int m = m_lo + tid;
+    if (A) {
+      par = A[2 * m];
+      pai = A[2 * m + 1];
+    } else {
+      pai = 3.14159265358979f * static_cast<float>(m);
+    }
+    pd = delta_hm(delta, dpm, M, h, m);
+    pe = Eb[m];
+  }
   int issued = 0;
   if (lane == 0) {
     for (int s = 0; s < D; ++s) mbar_init(mybar + s, 1);
@@ -245,15 +117,10 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
   }
   __syncwarp();
 
-  for (int f = tid; f < DX; f += kBhWarps * 32) {
-    fq[f] = xi_acc(ldx(q + bh * DX + f));
-    fk[f] = xi_acc(ldx(k + bh * DX + f));
-  }
-  for (int f = tid; f < DV; f += kBhWarps * 32) vv[f] = ldx(v + bh * DV + f);
-  for (int m = tid; m < M; m += kBhWarps * 32) {
-    const float ar = A ? A[2 * m] : -0.5f;
-    const float ai = A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m);
-    const float d = delta_hm(delta, dpm, M, h, m);
+  // lambda = exp(Delta A), b = (lambda - 1)/A in fp32; lambda - 1 is formed as
+  // expm1(x) cos(y) - 2 sin^2(y/2) + i e^x sin(y), keeping its relative
+  // accuracy for small Delta
+  auto params = [&](int mi, float ar, float ai, float d, float2 e) {
     const float x = d * ar, y = d * ai;
     float sy, cy, sh, ch;
     sincosf(y, &sy, &cy);
@@ -261,9 +128,20 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
     const float ex = expf(x), em1 = expm1f(x);
     const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;
     const float dd = fmaf(ar, ar, ai * ai);
-    lamb[m] = make_float2(ex * cy, ex * sy);
-    bb[m] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
-    eta[m] = Eb[m];
+    lamb[mi] = make_float2(ex * cy, ex * sy);
+    bb[mi] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
+    eta[mi] = e;
+  };
+  if (tid < DX) {
+    fq[tid] = xi_acc(xq);
+    fk[tid] = xi_acc(xk);
+  }
+  if (tid < DV) vv[tid] = xv;
+  if (tid < MS) params(tid, par, pai, pd, pe);
+  for (int mi = tid + NT; mi < MS; mi += NT) {   // more modes per CTA than threads
+    const int m = m_lo + mi;
+    params(mi, A ? A[2 * m] : -0.5f, A ? A[2 * m + 1] : 3.14159265358979f * static_cast<float>(m),
+           delta_hm(delta, dpm, M, h, m), Eb[m]);
   }
   __syncthreads();
 
@@ -273,14 +151,14 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
   float dpart = 0.f;
   bool ok = true;
   for (int j = 0; j < nj; ++j) {
-    const int m = warp + kBhWarps * j, s = j % D;
+    const int mi = warp + kBhWarps * j, m = m_lo + mi, s = j % D;
     if (!mbar_wait(mybar + s, static_cast<uint32_t>((j / D) & 1), err)) {
       ok = false;
       break;
     }
     const float4* us = reinterpret_cast<const float4*>(myring + s * slot);
     const float4* gs = reinterpret_cast<const float4*>(myring + s * slot + rowU);
-    const float2 L = lamb[m], Bm = bb[m];
+    const float2 L = lamb[mi], Bm = bb[mi];
     float4* Ur = reinterpret_cast<float4*>(Ub + static_cast<long long>(m) * DX);
     float4* Gr = reinterpret_cast<float4*>(Gb + static_cast<long long>(m) * DV);
     float ar = 0.f, ai = 0.f;
@@ -322,7 +200,7 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
       }
     }
     if (lane == 0) {
-      const float2 e = eta[m];
+      const float2 e = eta[mi];
       const float2 w = make_float2(fmaf(L.x, e.x, fmaf(-L.y, e.y, Bm.x)), fmaf(L.x, e.y, fmaf(L.y, e.x, Bm.y)));
       Eb[m] = w;
       dpart = fmaf(ar, w.x, fmaf(ai, w.y, dpart));
@@ -348,15 +226,42 @@ __global__ void __launch_bounds__(kBhWarps * 32, 3) decode_bh_kernel(
   }
   if (lane == 0) pden[warp] = dpart;
   __syncthreads();
-  float dn = 0.f;
-  for (int w = 0; w < kBhWarps; ++w) dn += pden[w];
+  if (S == 1) {
+    float dn = 0.f;
+    for (int w = 0; w < kBhWarps; ++w) dn += pden[w];
+    for (int f = tid; f < DV; f += kBhWarps * 32) {
+      float s = 0.f;
+      for (int w = 0; w < kBhWarps; ++w) s += part[w * DV + f];
+      o[bh * DV + f] = s / dn;
+      if (num) num[bh * DV + f] = s;
+    }
+    if (den && tid == 0) den[bh] = dn;
+    return;
+  }
+  // fold this CTA's warps into row 0, then rank 0 adds the ranks in order
   for (int f = tid; f < DV; f += kBhWarps * 32) {
     float s = 0.f;
     for (int w = 0; w < kBhWarps; ++w) s += part[w * DV + f];
-    o[bh * DV + f] = s / dn;
-    if (num) num[bh * DV + f] = s;
+    part[f] = s;
   }
-  if (den && tid == 0) den[bh] = dn;
+  if (tid == 0) {
+    float s = 0.f;
+    for (int w = 0; w < kBhWarps; ++w) s += pden[w];
+    pden[0] = s;
+  }
+  cluster.sync();
+  if (rank == 0) {
+    float dn = 0.f;
+    for (int r = 0; r < S; ++r) dn += cluster.map_shared_rank(pden, r)[0];
+    for (int f = tid; f < DV; f += kBhWarps * 32) {
+      float s = 0.f;
+      for (int r = 0; r < S; ++r) s += cluster.map_shared_rank(part, r)[f];
+      o[bh * DV + f] = s / dn;
+      if (num) num[bh * DV + f] = s;
+    }
+    if (den && tid == 0) den[bh] = dn;
+  }
+  cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
 }
 
 template <typename T>
@@ -366,54 +271,53 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
   const long long BHc = static_cast<long long>(s.B) * s.H;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // tuning switch: the smallest B*H that takes the one-CTA-per-(b,h) kernel
-  const char* thr_env = std::getenv("IA_DECODE_BH_MIN");
-  const long long thr = thr_env ? std::atoll(thr_env) : static_cast<long long>(sms);
-  if (BHc >= thr) {   // at least one (b,h) per SM: no need to split the modes across CTAs
-    // ring depth: four mode rows per warp while several CTAs still fit on an SM
+  // Cluster size S: one CTA per (b,h) once there is a (b,h) for every SM,
+  // else the fewest CTAs per (b,h) that give every SM one (S divides M; on a
+  // B200 splitting the 256 (b,h) of a 16 x 16-head batch measured slower, each
+  // CTA repeating the per-(b,h) set-up).  IA_DECODE_SPLIT=n forces S.
+  int S = 1;
+  while (S < 8 && BHc * S < sms && s.M % (2 * S) == 0) S *= 2;
+  if (const char* env = std::getenv("IA_DECODE_SPLIT")) {
+    const int f = std::atoi(env);
+    if ((f == 1 || f == 2 || f == 4 || f == 8) && s.M % f == 0) S = f;
+  }
+  {
+    // ring depth: up to four mode rows per warp, within a quarter of an SM's
+    // shared memory per CTA so that four CTAs fit (a deeper ring for fewer
+    // CTAs per SM measured slower on a B200)
     const size_t row = static_cast<size_t>(s.d_xi + s.d_v) * 8;
-    const int D = kBhWarps * 4 * row <= 96 * 1024 ? 4 : 2;
-    const size_t smem = kBhWarps * D * (row + 8) + sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
-                        sizeof(float2) * 3 * s.M + 16;
+    const size_t fixed = sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
+                         sizeof(float2) * 3 * s.M + 16;
+    const int per_warp = (s.M / S + kBhWarps - 1) / kBhWarps;
+    const size_t budget = 56 * 1024;
+    int D = 4;
+    while (D > 1 && kBhWarps * D * (row + 8) + fixed > budget) --D;
+    D = std::max(1, std::min(D, per_warp));
+    const size_t smem = kBhWarps * D * (row + 8) + fixed;
     int* err = device_error_ptr();
     if (!err) return cudaErrorInvalidSymbol;
     auto kern = decode_bh_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(BHc * S), 1, 1);
+    cfg.blockDim = dim3(kBhWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     mark_launch_begin(st);
-    kern<<<static_cast<unsigned>(BHc), kBhWarps * 32, smem, st>>>(
-        s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q), static_cast<const T*>(k),
-        static_cast<const T*>(v), delta, s.delta_per_mode, A, static_cast<float2*>(state), o, num, den, BHc, err);
-    e = cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q),
+                           static_cast<const T*>(k), static_cast<const T*>(v), delta, s.delta_per_mode, A,
+                           static_cast<float2*>(state), o, num, den, BHc, err);
     mark_launch_end(st);
     return e;
   }
-  // 16 modes (two per warp) per CTA, up to 8 CTAs per cluster
-  const int G = (s.M + 15) / 16;
-  const int MG = (s.M + G - 1) / G;
-  const long long BH = static_cast<long long>(s.B) * s.H;
-  const size_t smem = sizeof(float) * (2 * s.d_xi + s.d_v + 8 * s.d_v + 8) + sizeof(float2) * 2 * MG + 16;
-  auto kern = decode_kernel<T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(G * BH), 1, 1);
-  cfg.blockDim = dim3(kDecThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = G;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  mark_launch_begin(st);
-  e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, MG, static_cast<const T*>(q),
-                         static_cast<const T*>(k), static_cast<const T*>(v), delta, s.delta_per_mode, A,
-                         static_cast<float2*>(state), o, num, den, BH);
-  mark_launch_end(st);
-  return e;
 }
 
 }  // namespace

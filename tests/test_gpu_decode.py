@@ -17,13 +17,14 @@ def dev():
     return device()
 
 
-@pytest.mark.parametrize("kernel", ["default", "cluster", "per_bh"])
+@pytest.mark.parametrize("split", ["default", "1", "2", "4", "8"])
 @pytest.mark.parametrize("B", [1, 16, 64])
-def test_decode_steps_match_oracle(oracle_mod, dev, monkeypatch, B, kernel):
-    # both decode kernels (a cluster of CTAs per (b,h) splitting the modes, and
-    # one CTA per (b,h)) are forced at every batch size, besides the default choice
-    if kernel != "default":
-        monkeypatch.setenv("IA_DECODE_BH_MIN", "1000000000" if kernel == "cluster" else "1")
+def test_decode_steps_match_oracle(oracle_mod, dev, monkeypatch, B, split):
+    # every cluster size (1, 2, 4 or 8 CTAs per (b,h), each taking a range of
+    # the modes, rank 0 adding the partials) is forced at every batch size,
+    # besides the default choice
+    if split != "default":
+        monkeypatch.setenv("IA_DECODE_SPLIT", split)
     H, d, M, N0 = 16, 128, 64, 96
     pre = synthetic.layer_inputs(B, H, N0, d, d, "bf16", seed=1004)
     ref = oracle_mod.forward(pre["q"], pre["k"], pre["v"], pre["delta"], M)
