@@ -491,6 +491,35 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
   prep_raise_flag(a.flags + blockIdx.x, 2, th.tid);
 }
 
+// bf16 -> fp16 in place over one tile of PIECES 16-byte pieces, by NT
+// threads (ct = 0 .. NT-1), through the feature map when FEAT; rows past the
+// sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x 128
+// bytes; the map is elementwise, so the swizzle does not matter.
+template <bool FEAT, int PIECES, int NT>
+__device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct) {
+  constexpr int U = PIECES / NT;
+  static_assert(PIECES % NT == 0 && U <= 8, "pieces per thread");
+  uint4 in[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) in[u] = *reinterpret_cast<const uint4*>(base + (ct + u * NT) * 16);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int pc = ct + u * NT;
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (((pc >> 3) & 63) < nv) {   // row within its box
+      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(x2[e]);
+        w[e] = FEAT ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
+      }
+      out = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *reinterpret_cast<uint4*>(base + pc * 16) = out;
+  }
+}
+
 // 576 threads: one SM sub-partition carries five of the 18 warps, so its
 // 16 K registers cap a thread at 96.
 template <int DX>
@@ -516,6 +545,11 @@ __global__ void __launch_bounds__(NTH, 1)
   uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
   uint64_t* bar_drain = bars + 15;
   uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  // [NB]: output warps -> G7 of a state-only item, that set's k and v are
+  // fp16 operands.  A set is refilled only after that G7, so no barrier runs
+  // a phase ahead of the MMA warp's wait.
+  uint64_t* rdyKV = bars + 19;
+  static_assert(NB <= 3 && (19 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
   // G4 groups known done: the output warps see each G4 complete, in order,
@@ -546,6 +580,7 @@ __global__ void __launch_bounds__(NTH, 1)
       mbar_init(loaded + i, 1);
     }
     mbar_init(bar_drain, 1);
+    for (int i = 0; i < NB; ++i) mbar_init(rdyKV + i, GT);
     *abort_flag = 0;
     *g4_seen = 0;
     fence_barrier_init();
@@ -649,12 +684,15 @@ __global__ void __launch_bounds__(NTH, 1)
         // The state chain then waits on the output warps only through E1(f-1).
         const int nA = sc.nA, nF = sc.nF;
         int i7 = 0, f1 = 0, f23 = 0, f4 = 0, f56 = 0;
+        uint32_t pKV = 0u;   // bit b: parity of rdyKV[b]
         unsigned long long t_last = global_ns();
         for (unsigned spin = 0; i7 < nI || f56 < nF; ++spin) {
-          if (i7 < nI && (i7 < nA || f23 >= i7 - nA) && mbar_probe(rdy + 0, pr[0])) {
+          if (i7 < nI && (i7 < nA || f23 >= i7 - nA) &&
+              (i7 >= nA || mbar_probe(rdyKV + i7 % NB, (pKV >> (i7 % NB)) & 1u)) && mbar_probe(rdy + 0, pr[0])) {
             pr[0] ^= 1u;
-            tc_fence_after();
             const int b = i7 % NB;
+            if (i7 < nA) pKV ^= 1u << b;
+            tc_fence_after();
             g7(b);
             mma_commit(dne + 0);
             if (i7 < nA) {
@@ -720,10 +758,15 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       } else {
         int t = 0, prev_b = 0;   // full items issued so far; set of the previous full item
+        uint32_t pKV = 0u;       // bit b: parity of rdyKV[b]
         for (int i = 0; i < nI; ++i) {
           const int b = i % NB, p = i & 1;
           if (!(ok = wait_rdy(0))) break;
           if (sc.state_only(i)) {
+            ok = mbar_wait_or_abort(rdyKV + b, (pKV >> b) & 1u, a.err, abort_flag);   // k, v converted
+            pKV ^= 1u << b;
+            tc_fence_after();
+            if (!ok) break;
             g7(b);
             mma_commit(dne + 0);
             mma_commit(freeQK + b);
@@ -867,7 +910,7 @@ __global__ void __launch_bounds__(NTH, 1)
       const long long bh = w.bh;
       const int vb = w.vb;
       if (!(ok = waitLoaded(b))) break;
-      convert(nv, b, !so);
+      if (!so) convert(nv, b, true);   // the output warps convert a state-only item's k, v
       const bool piece_start = so ? (i == 0) : (i == sc.nA || ch == 0);
       if (i > 0 && !(ok = waitA(dne + 0, pd0))) break;   // G7 of the previous item: the state is current
       if (piece_start) {
@@ -1065,6 +1108,27 @@ __global__ void __launch_bounds__(NTH, 1)
       }
     };
     bool ok = true;
+    {
+      // The state-only chain of the range's last piece (items 0 .. nA-1)
+      // runs before any full chunk, when these warps have no readout to do:
+      // they convert its k and v tiles, so that the prepare warps only rotate
+      // and the chain is the rotation and G7 alone.
+      Walker wa;
+      wa.seek(sc.gA, a.nch, a.nvb, a.H);
+      for (int i = 0; ok && i < sc.nA; ++i, wa.step(a.nch, a.nvb, a.H)) {
+        const int b = i % NB;
+        const bool r = mbar_wait_or_abort(loaded + b, static_cast<uint32_t>((i / NB) & 1), a.err, abort_flag);
+        if (named_sync_or(3, GT, !r)) {
+          ok = false;
+          break;
+        }
+        const int nv = min(C, a.N - wa.ch * C);
+        convert_tile<true, K::TQ / 16, GT>(smem + sK(b), nv, tid - GT);
+        convert_tile<false, K::TV / 16, GT>(smem + sV(b), nv, tid - GT);
+        fence_async_smem();
+        mbar_arrive(rdyKV + b);
+      }
+    }
     bool have_prev = false;
     int prev_bh = 0, prev_vb = 0, prev_ch = 0, prev_nv = C, t = 0;
     Walker w;
