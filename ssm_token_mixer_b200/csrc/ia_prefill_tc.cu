@@ -387,32 +387,39 @@ __device__ __noinline__ void prep_raise_flag(int* flag, int value, int tid) {
   if (tid == 0) st_release(flag, value);
 }
 
-// TMEM state (and eta) += (mr + i mi) src, complex per mode (rows 2m, 2m+1)
+// TMEM state (and eta) += (mr + i mi) src, complex per mode (rows 2m, 2m+1).
+// src was written by another SM: each load is an L2 round trip, so a
+// thread's row segment is fetched in two batches (not one block at a time).
 template <int DX>
 __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* src, double mr, double mi, float* eta) {
   constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  constexpr int HB = FH / 8;   // float4 per batch: half of this thread's segment
+  static_assert(HB % 4 == 0, "a batch holds whole 16-column blocks");
   const float fr = static_cast<float>(mr), fs = static_cast<float>(th.comp ? mi : -mi);
-  for (int cb = 0; cb < FH; cb += 16) {
-    const int col0 = th.half * FH + cb;
-    uint32_t r[16];
-    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
-    float x[16];
-    const float4* s4 = reinterpret_cast<const float4*>(src + th.k * F + col0);
+  const float4* s4 = reinterpret_cast<const float4*>(src + th.k * F + th.half * FH);
+  const float xe = __ldcg(src + KR * F + th.k);
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const float4 v4 = __ldcg(s4 + g);
-      x[4 * g] = v4.x; x[4 * g + 1] = v4.y; x[4 * g + 2] = v4.z; x[4 * g + 3] = v4.w;
-    }
-    tmem_ld_wait16(r);
+  for (int hb = 0; hb < 2; ++hb) {
+    float4 g[HB];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float y = __shfl_xor_sync(kFull, x[e], 1);
-      r[e] = __float_as_uint(__uint_as_float(r[e]) + fmaf(fr, x[e], fs * y));
+    for (int u = 0; u < HB; ++u) g[u] = __ldcg(s4 + hb * HB + u);
+#pragma unroll
+    for (int blk = 0; blk < HB / 4; ++blk) {
+      const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
+      uint32_t r[16];
+      tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+      tmem_ld_wait16(r);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float4 v4 = g[4 * blk + e / 4];
+        const float x = (e & 3) == 0 ? v4.x : ((e & 3) == 1 ? v4.y : ((e & 3) == 2 ? v4.z : v4.w));
+        const float y = __shfl_xor_sync(kFull, x, 1);
+        r[e] = __float_as_uint(__uint_as_float(r[e]) + fmaf(fr, x, fs * y));
+      }
+      tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
     }
-    tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
   }
   tmem_st_wait();
-  const float xe = __ldcg(src + KR * F + th.k);
   const float ye = __shfl_xor_sync(kFull, xe, 1);
   *eta += fmaf(fr, xe, fs * ye);
 }
@@ -474,16 +481,33 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
   const float fr = static_cast<float>(lr), fs = static_cast<float>(th.comp ? li : -li);
   const float* loc = a.agg + static_cast<long long>(blockIdx.x) * STRIDE;
   float* dst = a.incl + static_cast<long long>(blockIdx.x) * STRIDE;
-  for (int cb = 0; cb < FH; cb += 16) {
-    const int col0 = th.half * FH + cb;
-    uint32_t r[16];
-    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
-    tmem_ld_wait16(r);
+  constexpr int HB = FH / 8;   // float4 per batch (the local state is re-read from L2)
+  const float4* l4 = reinterpret_cast<const float4*>(loc + th.k * F + th.half * FH);
+  float4* d4 = reinterpret_cast<float4*>(dst + th.k * F + th.half * FH);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float x = __uint_as_float(r[e]);
-      const float y = __shfl_xor_sync(kFull, x, 1);
-      dst[th.k * F + col0 + e] = loc[th.k * F + col0 + e] + fmaf(fr, x, fs * y);
+  for (int hb = 0; hb < 2; ++hb) {
+    float4 g[HB];
+#pragma unroll
+    for (int u = 0; u < HB; ++u) g[u] = __ldcg(l4 + hb * HB + u);
+#pragma unroll
+    for (int blk = 0; blk < HB / 4; ++blk) {
+      const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
+      uint32_t r[16];
+      tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+      tmem_ld_wait16(r);
+      float o[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x = __uint_as_float(r[e]);
+        const float y = __shfl_xor_sync(kFull, x, 1);
+        o[e] = fmaf(fr, x, fs * y);
+      }
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) {
+        const float4 lv = g[4 * blk + gg];
+        d4[hb * HB + 4 * blk + gg] =
+            make_float4(lv.x + o[4 * gg], lv.y + o[4 * gg + 1], lv.z + o[4 * gg + 2], lv.w + o[4 * gg + 3]);
+      }
     }
   }
   const float y = __shfl_xor_sync(kFull, eta_c, 1);
