@@ -361,20 +361,26 @@ __device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTab
     a.state_out[a.BH * 64 * (DX + a.DV) + bh * 64 + th.m] = make_float2(fr * eta_c - fi * y, fr * y + fi * eta_c);
 }
 
+// A published state (workspace only) holds columns in groups of four, each
+// group row after row: float4 (c / 4) * KR + k is row k, columns c .. c + 3,
+// so the 32 rows of a warp read or write 512 contiguous bytes per
+// instruction; eta follows, one float per row.
+__device__ __forceinline__ int pub4(int c, int k) { return (c >> 2) * KR + k; }
+
 // this thread's part of the TMEM state (and eta) -> dst [128 * F + 128]
 template <int DX>
 __device__ __noinline__ void prep_publish(const PrepThread& th, float* dst, float eta_c) {
   constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  float4* d4 = reinterpret_cast<float4*>(dst);
   for (int cb = 0; cb < FH; cb += 16) {
     const int col0 = th.half * FH + cb;
     uint32_t r[16];
     tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
     tmem_ld_wait16(r);
-    float4* d4 = reinterpret_cast<float4*>(dst + th.k * F + col0);
 #pragma unroll
     for (int g = 0; g < 4; ++g)
-      d4[g] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]), __uint_as_float(r[4 * g + 2]),
-                          __uint_as_float(r[4 * g + 3]));
+      d4[pub4(col0 + 4 * g, th.k)] = make_float4(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1]),
+                                                 __uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3]));
   }
   if (th.half == 0) dst[KR * F + th.k] = eta_c;
 }
@@ -396,13 +402,13 @@ __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* 
   constexpr int HB = FH / 8;   // float4 per batch: half of this thread's segment
   static_assert(HB % 4 == 0, "a batch holds whole 16-column blocks");
   const float fr = static_cast<float>(mr), fs = static_cast<float>(th.comp ? mi : -mi);
-  const float4* s4 = reinterpret_cast<const float4*>(src + th.k * F + th.half * FH);
+  const float4* s4 = reinterpret_cast<const float4*>(src);
   const float xe = __ldcg(src + KR * F + th.k);
 #pragma unroll
   for (int hb = 0; hb < 2; ++hb) {
     float4 g[HB];
 #pragma unroll
-    for (int u = 0; u < HB; ++u) g[u] = __ldcg(s4 + hb * HB + u);
+    for (int u = 0; u < HB; ++u) g[u] = __ldcg(s4 + pub4(th.half * FH + 4 * (hb * HB + u), th.k));
 #pragma unroll
     for (int blk = 0; blk < HB / 4; ++blk) {
       const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
@@ -482,13 +488,13 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
   const float* loc = a.agg + static_cast<long long>(blockIdx.x) * STRIDE;
   float* dst = a.incl + static_cast<long long>(blockIdx.x) * STRIDE;
   constexpr int HB = FH / 8;   // float4 per batch (the local state is re-read from L2)
-  const float4* l4 = reinterpret_cast<const float4*>(loc + th.k * F + th.half * FH);
-  float4* d4 = reinterpret_cast<float4*>(dst + th.k * F + th.half * FH);
+  const float4* l4 = reinterpret_cast<const float4*>(loc);
+  float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int hb = 0; hb < 2; ++hb) {
     float4 g[HB];
 #pragma unroll
-    for (int u = 0; u < HB; ++u) g[u] = __ldcg(l4 + hb * HB + u);
+    for (int u = 0; u < HB; ++u) g[u] = __ldcg(l4 + pub4(th.half * FH + 4 * (hb * HB + u), th.k));
 #pragma unroll
     for (int blk = 0; blk < HB / 4; ++blk) {
       const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
@@ -505,7 +511,7 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
 #pragma unroll
       for (int gg = 0; gg < 4; ++gg) {
         const float4 lv = g[4 * blk + gg];
-        d4[hb * HB + 4 * blk + gg] =
+        d4[pub4(th.half * FH + 4 * (hb * HB + 4 * blk + gg), th.k)] =
             make_float4(lv.x + o[4 * gg], lv.y + o[4 * gg + 1], lv.z + o[4 * gg + 2], lv.w + o[4 * gg + 3]);
       }
     }
