@@ -61,6 +61,34 @@ def test_tensor_core_prefill_small(oracle_mod, dev, dx, dv, N):
                 TOL_BF16)
 
 
+@pytest.mark.parametrize("B,H,dx,dv", [(1, 3, 64, 64), (3, 5, 64, 64), (3, 1, 128, 128), (5, 3, 128, 64)])
+def test_tensor_core_odd_batch_times_heads(oracle_mod, dev, B, H, dx, dv):
+    # odd B*H on the tensor-core path: heads change between streams at
+    # arbitrary CTA boundaries, whole streams or ranges as the planner picks
+    M, N = 64, 150
+    assert ia.prefill_path(B, H, N, dx, dv, M, "bf16") == "tensor_core"
+    inp = synthetic.layer_inputs(B, H, N, dx, dv, "bf16", seed=13 * B + H + dx + dv)
+    r = gpu_prefill(inp, M, dev)
+    ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
+    rep = report(r["num"], r["den"], r["o"], ref)
+    assert max(rep.values()) < TOL_BF16, rep
+    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, dx, dv), B, H, M, dx, dv, TOL_BF16)
+
+
+@pytest.mark.parametrize("M", [1, 16, 48, 96])
+def test_bf16_prefill_other_mode_counts(oracle_mod, dev, M):
+    # bf16 inputs with M != 64 take the sequential CUDA-core path: same
+    # tolerance as the tensor-core path, which only M = 64 runs
+    B, H, N, d = 2, 3, 130, 64
+    assert ia.prefill_path(B, H, N, d, d, M, "bf16") == "sequential"
+    inp = synthetic.layer_inputs(B, H, N, d, d, "bf16", seed=300 + M)
+    r = gpu_prefill(inp, M, dev)
+    ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
+    rep = report(r["num"], r["den"], r["o"], ref)
+    assert max(rep.values()) < TOL_BF16, rep
+    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, d, d), B, H, M, d, d, TOL_BF16)
+
+
 def test_tensor_core_long_ragged_sequence(oracle_mod, dev):
     # few (b,h) pairs and a long ragged sequence: the planner spreads the
     # chunks over many CTAs, so most ranges start inside the sequence and
