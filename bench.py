@@ -532,14 +532,24 @@ def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, wor
         "readout": {"W": (torch.randn(w.H, w.M, w.M, 2, generator=g) / math.sqrt(w.M)).to(dev)},
         "bidirectional": {"bidirectional": True},
     }
+    parts["norm+bidirectional"] = {**parts["norm"], **parts["bidirectional"]}
     parts["all"] = {**parts["selective"], **parts["norm"], **parts["readout"]}
     tokens = w.B * w.N
     by = bytes_fwd(w.d_xi, w.d_v) * tokens * w.H
     out = {"workload": f"{w.name} (B{w.B} H{w.H} N{w.N} d_xi{w.d_xi} d_v{w.d_v} M{w.M}, bf16 inputs)",
-           "unit": "tokens/s", "kernel": "token-serial CUDA-core layer (ia_prefill_fwd_ex)", "parts": {}}
+           "unit": "tokens/s",
+           "kernel": "ia_prefill_fwd_ex: the tensor-core chunk pass with a prologue (and, bidirectional, a "
+                     "second pass and an epilogue) where the parts allow it, else the token-serial CUDA-core "
+                     "layer; `path` per part", "parts": {}}
     for name, kw in parts.items():
         d = None if "delta_t" in kw else delta
-        fn = lambda: ia.prefill_fwd_ex(q, k, v, w.M, delta=d, **kw)
+        present = dict(norm="gain" in kw, selective="delta_t" in kw, readout="W" in kw,
+                       bidirectional=bool(kw.get("bidirectional")))
+        path = ia.prefill_ex_path(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16", **present)
+        need = ia.prefill_ex_workspace_bytes(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16", **present)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+        o = torch.empty(w.B, w.H, w.N, w.d_v, dtype=torch.float32, device=dev)
+        fn = lambda: ia.prefill_fwd_ex(q, k, v, w.M, delta=d, workspace=ws, o=o, **kw)
         barrier(dev)
         step_ms, kern_ms = timer.run(fn, steps, warmup)
         barrier(dev)
@@ -547,8 +557,11 @@ def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, wor
         passes = 2 if kw.get("bidirectional") else 1
         rf = roofline(by * passes, flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H * passes, kern_ms, peaks,
                       peak_kind, None, sustained=False)
+        # tensor cores: the prologue, a table kernel and a chunk pass per direction, the epilogue
+        launches = ((1 if present["norm"] or present["bidirectional"] else 0) + passes * 2 +
+                    (1 if present["bidirectional"] else 0)) if path == "tensor_core" else passes
         out["parts"][name] = {"value": world * tokens * steps / (total * 1e-3), "ms_per_step": total / steps,
-                              "roofline": rf, "gpu_launches": passes * steps}
+                              "path": path, "roofline": rf, "gpu_launches": launches * steps}
     return out
 
 

@@ -235,15 +235,30 @@ typedef struct {
 
 /*
  * ia_prefill_fwd with the optional parts (NULL opt = the plain layer).
- * Runs the token-serial fp32 CUDA-core kernel (one CTA per (b,h), any input
- * dtype; the tensor-core chunk pass does not take these options), so it is
- * correct for every shape whose state fits in shared memory but slower than
- * ia_prefill_fwd.  Needs no workspace.
+ * Two forms, chosen per call (ia_prefill_ex_path tells which):
+ *   - bf16 inputs on a shape of the tensor-core chunk pass (M = 64, d_xi and
+ *     d_v in {64, 128}) with no delta_t and no W run on tensor cores: a
+ *     prologue kernel writes the stabilised SSM input z (when gain or bias is
+ *     given) as fp16 k and v operands, and the time-reversed q and z (for the
+ *     bidirectional layer); the chunk pass runs once, or twice for the
+ *     bidirectional layer, whose second output an epilogue kernel adds back
+ *     in forward order.  z is rounded to fp16 once more than in the
+ *     token-serial form.  Needs ia_prefill_ex_workspace_bytes of workspace.
+ *   - everything else runs the token-serial fp32 CUDA-core kernel (one CTA
+ *     per (b,h), any input dtype), correct for every shape whose state fits
+ *     in shared memory but much slower; it needs no workspace (workspace may
+ *     be NULL).
+ * workspace: device scratch of at least ia_prefill_ex_workspace_bytes bytes
+ * for the tensor-core form, any alignment; too small gives IA_ERR_WORKSPACE
+ * before anything is launched.
  */
+IA_API size_t ia_prefill_ex_workspace_bytes(const ia_shape_t* shape, const ia_options_t* opt);
+IA_API int ia_prefill_ex_path(const ia_shape_t* shape, const ia_options_t* opt);
 IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* shape, const ia_options_t* opt, const void* q,
                                      const void* k, const void* v, const float* delta, const float* A,
                                      const void* state_in, float* o, float* num, float* den,
-                                     void* state_out, void* stream);
+                                     void* state_out, void* workspace, size_t workspace_bytes,
+                                     void* stream);
 
 /*
  * ia_decode_step with the optional parts (bidirectional excluded: that layer

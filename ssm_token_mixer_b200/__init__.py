@@ -88,7 +88,11 @@ def load_library():
     lib.ia_decode_step.argtypes = [S] + [P] * 9 + [P]
     O = ctypes.POINTER(IAOptions)
     lib.ia_prefill_fwd_ex.restype = ctypes.c_int
-    lib.ia_prefill_fwd_ex.argtypes = [S, O] + [P] * 10 + [P]
+    lib.ia_prefill_fwd_ex.argtypes = [S, O] + [P] * 10 + [P, ctypes.c_size_t, P]
+    lib.ia_prefill_ex_workspace_bytes.restype = ctypes.c_size_t
+    lib.ia_prefill_ex_workspace_bytes.argtypes = [S, O]
+    lib.ia_prefill_ex_path.restype = ctypes.c_int
+    lib.ia_prefill_ex_path.argtypes = [S, O]
     lib.ia_decode_step_ex.restype = ctypes.c_int
     lib.ia_decode_step_ex.argtypes = [S, O] + [P] * 9 + [P]
     lib.ia_set_launch_events.restype = ctypes.c_int
@@ -161,6 +165,39 @@ def prefill_path(B, H, N, d_xi, d_v, M, dtype):
 def fwd_bwd_path(B, H, N, d_xi, d_v, M, dtype):
     """'tensor_core' or 'sequential': the reverse-pass kernels ia_fwd_bwd runs for this shape."""
     return PATHS[load_library().ia_fwd_bwd_path(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype)))]
+
+
+def _presence_options(norm, selective, readout, bidirectional):
+    """Options whose arrays are placeholder addresses: for the queries, which
+    test only which parts are present and read no array."""
+    opt = IAOptions()
+    some = ctypes.c_void_p(256)
+    if selective:
+        opt.delta_t = some
+    if norm:
+        opt.gain = some
+    if readout:
+        opt.W = some
+    opt.eps = 1e-6
+    opt.bidirectional = int(bool(bidirectional))
+    return opt
+
+
+def prefill_ex_path(B, H, N, d_xi, d_v, M, dtype, norm=False, selective=False, readout=False,
+                    bidirectional=False):
+    """'tensor_core' or 'sequential': the kernels ia_prefill_fwd_ex runs for this
+    shape and these optional parts."""
+    opt = _presence_options(norm, selective, readout, bidirectional)
+    shp = make_shape(B, H, N, d_xi, d_v, M, dtype)
+    return PATHS[load_library().ia_prefill_ex_path(ctypes.byref(shp), ctypes.byref(opt))]
+
+
+def prefill_ex_workspace_bytes(B, H, N, d_xi, d_v, M, dtype, norm=False, selective=False, readout=False,
+                               bidirectional=False) -> int:
+    """Workspace bytes ia_prefill_fwd_ex needs for this shape and these parts."""
+    opt = _presence_options(norm, selective, readout, bidirectional)
+    shp = make_shape(B, H, N, d_xi, d_v, M, dtype)
+    return int(load_library().ia_prefill_ex_workspace_bytes(ctypes.byref(shp), ctypes.byref(opt)))
 
 
 def prefill_static_max_heads() -> int:
@@ -381,11 +418,14 @@ def _options(named_shapes, delta_t, gain, bias, eps, W, bidirectional, B, H, M, 
 
 
 def prefill_fwd_ex(q, k, v, M, delta=None, A=None, delta_t=None, gain=None, bias=None, eps=1e-6, W=None,
-                   bidirectional=False, state_in=None, want_num_den=False, want_state=False, stream=None):
+                   bidirectional=False, state_in=None, want_num_den=False, want_state=False, stream=None,
+                   workspace=None, o=None):
     """The layer with its optional parts (see ia_prefill_fwd_ex in include/ia.h):
     delta_t [B,H,N] a step per token, gain/bias [H, d_xi+d_v] the RMSNorm on the
     SSM input, W [H,M,M,2] (re, im) the complex readout matrix, bidirectional
-    the two-direction layer.  Returns dict(o, num, den, state)."""
+    the two-direction layer.  workspace: a uint8 device tensor of at least
+    prefill_ex_workspace_bytes (allocated here when None).  Returns dict(o,
+    num, den, state)."""
     lib = load_library()
     _need("q", q)
     if q.dim() != 4:
@@ -408,12 +448,20 @@ def prefill_fwd_ex(q, k, v, M, delta=None, A=None, delta_t=None, gain=None, bias
     opt = _options(None, delta_t, gain, bias, eps, W, bidirectional, B, H, M, d_xi, d_v, (N,))
     dev = _cuda_device([("q", q), ("k", k), ("v", v), ("delta", delta), ("A", A), ("delta_t", delta_t),
                         ("gain", gain), ("bias", bias), ("W", W), ("state_in", state_in)])
-    o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    if o is None:
+        o = torch.empty(B, H, N, d_v, dtype=torch.float32, device=dev)
+    else:
+        _need("o", o, (B, H, N, d_v), torch.float32)
     num = torch.empty_like(o) if want_num_den else None
     den = torch.empty(B, H, N, dtype=torch.float32, device=dev) if want_num_den else None
     st = torch.empty(n_state, dtype=torch.float32, device=dev) if want_state else None
+    need = int(lib.ia_prefill_ex_workspace_bytes(ctypes.byref(shp), ctypes.byref(opt)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     rc = lib.ia_prefill_fwd_ex(ctypes.byref(shp), ctypes.byref(opt), _ptr(q), _ptr(k), _ptr(v), _ptr(delta),
-                               _ptr(A), _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st), _stream(stream))
+                               _ptr(A), _ptr(state_in), _ptr(o), _ptr(num), _ptr(den), _ptr(st),
+                               _ptr(workspace), nbytes, _stream(stream))
     _check(rc, "ia_prefill_fwd_ex")
     return {"o": o, "num": num, "den": den, "state": st}
 

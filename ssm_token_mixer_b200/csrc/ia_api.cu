@@ -26,15 +26,6 @@ bool env_set(const char* name) {
   return s && s[0] && std::strcmp(s, "0") != 0;
 }
 
-int num_sms() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-    cudaGetLastError();   // clear a sticky "no device" error; plan for a B200
-    return 148;
-  }
-  return n;
-}
 
 bool use_tc(const ia_shape_t& s) {
   if (env_set("IA_PREFILL_SIMT")) return false;   // debug switch: force the CUDA-core path
@@ -49,6 +40,16 @@ bool use_tc_bwd(const ia_shape_t& s) {
 cudaEvent_t g_ev_begin = nullptr, g_ev_end = nullptr;
 
 }  // namespace
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();   // clear a sticky "no device" error; plan for a B200
+    return 148;
+  }
+  return n;
+}
 
 bool valid_dims(const ia_shape_t* s, bool need_n) {
   if (!s) return false;
@@ -114,11 +115,13 @@ void* SymbolCache::get(const void* symbol, cudaError_t* err) {
   return p;
 }
 
+thread_local bool g_marks_held = false;
+void hold_launch_marks(bool hold) { g_marks_held = hold; }
 void mark_launch_begin(cudaStream_t st) {
-  if (g_ev_begin) cudaEventRecord(g_ev_begin, st);
+  if (g_ev_begin && !g_marks_held) cudaEventRecord(g_ev_begin, st);
 }
 void mark_launch_end(cudaStream_t st) {
-  if (g_ev_end) cudaEventRecord(g_ev_end, st);
+  if (g_ev_end && !g_marks_held) cudaEventRecord(g_ev_end, st);
 }
 
 int* device_error_ptr() {

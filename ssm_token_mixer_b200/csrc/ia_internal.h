@@ -59,7 +59,7 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st,
                               void* dump_R = nullptr, float* dump_Re = nullptr,
-                              float* dtab = nullptr);
+                              float* dtab = nullptr, bool kv_ready = false);
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
 
@@ -67,7 +67,7 @@ HeadTables* tc_tables(void* ws);
 // 32-column x 64-row boxes, 128-byte swizzled; q/k/v bf16 [BH][N][W] as
 // 64 x 64 boxes, 128-byte swizzled.  False if the driver refuses the map.
 bool encode_rows64_f32_map(CUtensorMap* m, float* x, long long BH, int N, int W);
-bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W);
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W, bool fp16 = false);
 
 // Tensor-core training step (bf16, M = 64, d_xi = d_v = 64).
 bool tc_bwd_supported(const ia_shape_t& s);
@@ -94,6 +94,20 @@ bool inject_launch_failure();
 // Caller-registered events bracketing the dominant kernel launch (profiling).
 void mark_launch_begin(cudaStream_t st);
 void mark_launch_end(cudaStream_t st);
+// While held, mark_launch_begin/end do nothing: an entry point that runs
+// several passes marks its whole sequence once.
+void hold_launch_marks(bool hold);
+
+// The optional parts on the tensor-core chunk pass (ia_layer_tc.cu): input
+// stabilisation and the bidirectional layer, for the shapes the chunk pass
+// runs; no per-token step and no readout matrix.
+bool ex_tc_supported(const ia_shape_t& s, const ia_options_t* opt);
+size_t ex_tc_workspace_bytes(const ia_shape_t& s, const ia_options_t* opt, const TcPlan& p);
+cudaError_t launch_ex_tc(const ia_shape_t& s, const ia_options_t* opt, const TcPlan& p, const void* q,
+                         const void* k, const void* v, const float* delta, const float* A,
+                         const void* state_in, float* o, float* num, float* den, void* state_out, void* ws,
+                         cudaStream_t st);
+int num_sms();
 
 // Shape check shared by every entry point: positive dims (N only when
 // need_n), a known dtype, and B*H within int range.

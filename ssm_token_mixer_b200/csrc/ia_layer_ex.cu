@@ -16,6 +16,8 @@
 //     second launch that reads and writes the sequence back to front and adds
 //     its output to the first.
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 
 #include "ia_device.cuh"
 #include "ia_internal.h"
@@ -214,6 +216,15 @@ ExArgs make_args(const ia_shape_t* s, const ia_options_t* opt, const float* delt
   return a;
 }
 
+// The tensor-core form (ia_layer_tc.cu) serves bf16 shapes of the chunk pass
+// whose options are only the input stabilisation and / or the bidirectional
+// layer; IA_PREFILL_SIMT forces the token-serial kernel, as for the plain layer.
+bool ex_use_tc(const ia_shape_t& s, const ia_options_t* opt) {
+  const char* env = std::getenv("IA_PREFILL_SIMT");
+  if (env && env[0] && std::strcmp(env, "0") != 0) return false;
+  return ex_tc_supported(s, opt);
+}
+
 bool valid_options(const ia_options_t* opt) {
   if (!opt) return true;
   const void* ptrs[] = {opt->delta_t, opt->gain, opt->bias, opt->W};
@@ -230,10 +241,20 @@ using namespace ia;
 
 extern "C" {
 
+IA_API size_t ia_prefill_ex_workspace_bytes(const ia_shape_t* s, const ia_options_t* opt) {
+  if (!valid_dims(s, true) || !valid_options(opt) || !ex_use_tc(*s, opt)) return 0;
+  return ex_tc_workspace_bytes(*s, opt, tc_plan(*s, num_sms()));
+}
+
+IA_API int ia_prefill_ex_path(const ia_shape_t* s, const ia_options_t* opt) {
+  if (!valid_dims(s, true) || !valid_options(opt)) return IA_PATH_NONE;
+  return ex_use_tc(*s, opt) ? IA_PATH_TENSOR_CORE : IA_PATH_SEQUENTIAL;
+}
+
 IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* s, const ia_options_t* opt, const void* q,
                                      const void* k, const void* v, const float* delta, const float* A,
                                      const void* state_in, float* o, float* num, float* den,
-                                     void* state_out, void* stream) {
+                                     void* state_out, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dims(s, true) || !valid_options(opt)) return IA_ERR_INVALID_ARG;
   if (!q || !k || !v || !o || (!delta && !(opt && opt->delta_t))) return IA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, delta, A, state_in, o, num, den, state_out};
@@ -244,9 +265,24 @@ IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* s, const ia_options_t* op
   // the two directions of the bidirectional layer have no single state, and
   // their num / den do not combine into o
   if (bidir && (state_in || state_out || num || den)) return IA_ERR_INVALID_ARG;
-  if (ex_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  const bool tc = ex_use_tc(*s, opt);
+  if (!tc && ex_smem(s->d_xi, s->d_v, s->M) > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  TcPlan plan{1};
+  if (tc) {
+    plan = tc_plan(*s, num_sms());
+    if (!workspace || workspace_bytes < ex_tc_workspace_bytes(*s, opt, plan)) return IA_ERR_WORKSPACE;
+  }
   if (inject_launch_failure()) return IA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc) {   // the marks bracket every pass of the call
+    mark_launch_begin(st);
+    hold_launch_marks(true);
+    const cudaError_t e = launch_ex_tc(*s, opt, plan, q, k, v, delta, A, state_in, o, num, den, state_out,
+                                       workspace, st);
+    hold_launch_marks(false);
+    mark_launch_end(st);
+    return map_cuda(e);
+  }
   ExArgs a = make_args(s, opt, delta, A);
   a.state_in = static_cast<const float2*>(state_in);
   a.state_out = static_cast<float2*>(state_out);

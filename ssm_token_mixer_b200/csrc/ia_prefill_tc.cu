@@ -69,14 +69,15 @@ EncodeTiledFn encode_tiled() {
 // q, k or v [BH][N][W] bf16 (W a multiple of 64): one box is 64 rows x 64
 // columns (128 bytes) of one (b,h), 128-byte swizzled in shared memory.  Rows
 // >= N lie outside the map and read as zero.
-bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W) {
+bool encode_input_map(CUtensorMap* m, const void* x, long long BH, int N, int W, bool fp16) {
   const EncodeTiledFn enc = encode_tiled();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(W) * 2, static_cast<cuuint64_t>(N) * W * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kChunk), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+  return enc(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x),
+             dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -172,6 +173,7 @@ struct TcArgs {
   float* agg;               // [G][128 * F + 128]: local end state of a CTA's last piece
   float* incl;              // [G][128 * F + 128]: inclusive end state of a CTA's last piece
   int* flags;               // [G]: 0 nothing yet, 1 agg published, 2 incl published
+  int kv_ready;             // 1: k, v arrive as fp16 operands (k already through the feature map)
   int H, N, DV, nch, nvb, G;
   long long BH, total;      // total = BH * nvb * nch chunks
 };
@@ -526,7 +528,7 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
 // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x 128
 // bytes; the map is elementwise, so the swizzle does not matter.
 template <bool FEAT, int PIECES, int NT>
-__device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct) {
+__device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct, bool ready = false) {
   constexpr int U = PIECES / NT;
   static_assert(PIECES % NT == 0 && U <= 8, "pieces per thread");
   uint4 in[U];
@@ -537,14 +539,18 @@ __device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct) {
     const int pc = ct + u * NT;
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (((pc >> 3) & 63) < nv) {   // row within its box
-      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
-      uint32_t w[4];
+      if (ready) {
+        out = in[u];
+      } else {
+        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
+        uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(x2[e]);
-        w[e] = FEAT ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(x2[e]);
+          w[e] = FEAT ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
+        }
+        out = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      out = make_uint4(w[0], w[1], w[2], w[3]);
     }
     *reinterpret_cast<uint4*>(base + pc * 16) = out;
   }
@@ -904,7 +910,9 @@ __global__ void __launch_bounds__(NTH, 1)
         const uint32_t base = tsel == 0 ? sQ(b) : (tsel == 1 ? sK(b) : sV(b));
         uint4* ptr = reinterpret_cast<uint4*>(smem + base + pc * 16);
         uint4 out = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nv) {
+        if (r < nv && tsel > 0 && a.kv_ready) {   // k, v already fp16 operands
+          out = in[u];
+        } else if (r < nv) {
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
           uint32_t w[4];
 #pragma unroll
@@ -1153,8 +1161,8 @@ __global__ void __launch_bounds__(NTH, 1)
           break;
         }
         const int nv = min(C, a.N - wa.ch * C);
-        convert_tile<true, K::TQ / 16, GT>(smem + sK(b), nv, tid - GT);
-        convert_tile<false, K::TV / 16, GT>(smem + sV(b), nv, tid - GT);
+        convert_tile<true, K::TQ / 16, GT>(smem + sK(b), nv, tid - GT, a.kv_ready);
+        convert_tile<false, K::TV / 16, GT>(smem + sV(b), nv, tid - GT, a.kv_ready);
         fence_async_smem();
         mbar_arrive(rdyKV + b);
       }
@@ -1297,8 +1305,10 @@ cudaError_t launch_impl(const TcArgs& args, const void* q, const void* k, const 
                         cudaStream_t st) {
   using K = PCfg<DX>;
   CUtensorMap tm_q, tm_k, tm_v, tm_o;
-  if (!encode_input_map(&tm_q, q, args.BH, args.N, DX) || !encode_input_map(&tm_k, k, args.BH, args.N, DX) ||
-      !encode_input_map(&tm_v, v, args.BH, args.N, DV) || !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N, DV))
+  const bool f16 = args.kv_ready != 0;
+  if (!encode_input_map(&tm_q, q, args.BH, args.N, DX) || !encode_input_map(&tm_k, k, args.BH, args.N, DX, f16) ||
+      !encode_input_map(&tm_v, v, args.BH, args.N, DV, f16) ||
+      !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N, DV))
     return cudaErrorNotSupported;
   auto kern = tc_prefill_kernel<DX>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
@@ -1388,12 +1398,13 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st, void* dump_R,
-                              float* dump_Re, float* dtab) {
+                              float* dump_Re, float* dtab, bool kv_ready) {
   uint8_t* w = reinterpret_cast<uint8_t*>(tc_tables(ws));
   HeadTables* tabs = reinterpret_cast<HeadTables*>(w);
   TcArgs args;
   args.agg = args.incl = nullptr;
   args.flags = nullptr;
+  args.kv_ready = kv_ready ? 1 : 0;
   const size_t F = static_cast<size_t>(s.d_xi) + kVB;
   if (tc_plan_splits(s, p)) {
     float* agg = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);

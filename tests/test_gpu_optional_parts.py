@@ -108,3 +108,73 @@ def test_no_options_is_the_plain_layer(dev):
     b = ia.prefill_fwd_ex(g["q"], g["k"], g["v"], 64, delta=g["delta"], want_num_den=True)
     ia.check_device_errors()
     assert slice_rel(b["num"].cpu(), a["num"].cpu(), (-2, -1)) < TOL_BF16
+
+
+TC_CASES = [("norm",), ("bidirectional",), ("norm", "bidirectional")]
+
+
+@pytest.mark.parametrize("which", TC_CASES, ids=["+".join(c) for c in TC_CASES])
+@pytest.mark.parametrize("dx,dv,N", [(64, 64, 150), (128, 128, 200), (64, 128, 64), (128, 64, 1)])
+def test_tensor_core_optional_parts(oracle_mod, dev, which, dx, dv, N):
+    # input stabilisation and the bidirectional layer on the tensor-core chunk
+    # pass (a prologue writes the normalised and / or reversed operands; the
+    # bidirectional second pass is added back by an epilogue), ragged lengths
+    B, H, M = 2, 3, 64
+    norm, bidir = "norm" in which, "bidirectional" in which
+    assert ia.prefill_ex_path(B, H, N, dx, dv, M, "bf16", norm=norm, bidirectional=bidir) == "tensor_core"
+    inp = synthetic.layer_inputs(B, H, N, dx, dv, "bf16", seed=90 + dx + dv + N)
+    opt = options(B, H, N, dx, dv, M, 91, which)
+    g = lambda x: None if x is None else x.to(dev)
+    kw = {k: g(v) for k, v in opt.items()}
+    if bidir:
+        r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta=g(inp["delta"]), bidirectional=True,
+                              **kw)
+        ia.check_device_errors()
+        ref = oracle_mod.forward_bidirectional(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **opt)
+        assert slice_rel(r["o"].cpu(), ref, (-2, -1)) < TOL_BF16
+        return
+    r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta=g(inp["delta"]), want_num_den=True,
+                          want_state=True, **kw)
+    ia.check_device_errors()
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **opt)
+    rep = report(r["num"].cpu(), r["den"].cpu(), r["o"].cpu(), ref)
+    assert max(rep.values()) < TOL_BF16, rep
+    st = r["state"].cpu().double().numpy()
+    assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < TOL_BF16
+
+
+def test_tensor_core_and_token_serial_optional_parts_agree(dev, monkeypatch):
+    # the same call through both forms of ia_prefill_fwd_ex
+    B, H, N, d, M = 2, 2, 300, 64, 64
+    inp = synthetic.layer_inputs(B, H, N, d, d, "bf16", seed=92)
+    opt = options(B, H, N, d, d, M, 93, ("norm",))
+    g = {k: v.to(dev) for k, v in inp.items()}
+    kw = {k: v.to(dev) for k, v in opt.items()}
+    a = ia.prefill_fwd_ex(g["q"], g["k"], g["v"], M, delta=g["delta"], bidirectional=True, **kw)
+    monkeypatch.setenv("IA_PREFILL_SIMT", "1")
+    assert ia.prefill_ex_path(B, H, N, d, d, M, "bf16", norm=True, bidirectional=True) == "sequential"
+    b = ia.prefill_fwd_ex(g["q"], g["k"], g["v"], M, delta=g["delta"], bidirectional=True, **kw)
+    ia.check_device_errors()
+    assert slice_rel(a["o"].cpu(), b["o"].cpu(), (-2, -1)) < TOL_BF16
+
+
+def test_optional_parts_paths_and_workspace(dev):
+    B, H, N = 2, 3, 150
+    tc = lambda **kw: ia.prefill_ex_path(B, H, N, 64, 64, 64, "bf16", **kw)
+    assert tc() == "tensor_core"
+    assert tc(norm=True) == tc(bidirectional=True) == tc(norm=True, bidirectional=True) == "tensor_core"
+    assert tc(selective=True) == tc(readout=True) == tc(norm=True, readout=True) == "sequential"
+    assert ia.prefill_ex_path(B, H, N, 64, 64, 48, "bf16", norm=True) == "sequential"    # M != 64
+    assert ia.prefill_ex_path(B, H, N, 64, 64, 64, "f32", norm=True) == "sequential"     # fp32 inputs
+    # a workspace one byte short is refused before anything runs
+    inp = synthetic.layer_inputs(B, H, N, 64, 64, "bf16", seed=94)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    shp = ia.make_shape(B, H, N, 64, 64, 64, "bf16")
+    opt = ia.IAOptions()
+    opt.bidirectional = 1
+    need = ia.load_library().ia_prefill_ex_workspace_bytes(ia.ctypes.byref(shp), ia.ctypes.byref(opt))
+    assert need > 0
+    ws = torch.empty(need - 1, dtype=torch.uint8, device=dev)
+    with pytest.raises(ia.IAError) as err:
+        ia.prefill_fwd_ex(g["q"], g["k"], g["v"], 64, delta=g["delta"], bidirectional=True, workspace=ws)
+    assert err.value.status == 3   # IA_ERR_WORKSPACE
