@@ -238,9 +238,7 @@ ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, co
     if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
   if ((s->d_xi & 1) || (s->d_v & 1)) return IA_ERR_UNSUPPORTED;   // 16-byte state vectors
   if (s->d_xi > 256 || s->d_v > 256) return IA_ERR_UNSUPPORTED;     // one register pass per row
-  if (s->M > 128) return IA_ERR_UNSUPPORTED;                        // at most 8 CTAs x 16 modes
-  const size_t smem = sizeof(float) * (2 * s->d_xi + 9 * s->d_v + 8) + 2 * sizeof(float2) * s->M + 16;
-  if (smem > kMaxSmem) return IA_ERR_UNSUPPORTED;
+  if (decode_smem_bytes(*s) > kMaxSmem) return IA_ERR_UNSUPPORTED;
   if (inject_launch_failure()) return IA_ERR_CUDA;
   return map_cuda(launch_decode(*s, q, k, v, delta, A, state, o, num, den,
                                 static_cast<cudaStream_t>(stream)));

@@ -264,6 +264,11 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
   cluster.sync();   // keep every CTA's shared memory alive until rank 0 has read it
 }
 
+// shared memory besides the ring: features, partial sums, mode parameters
+size_t decode_fixed_smem(const ia_shape_t& s) {
+  return sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) + sizeof(float2) * 3 * s.M + 16;
+}
+
 template <typename T>
 cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const void* v,
                         const float* delta, const float* A, void* state, float* o, float* num,
@@ -286,8 +291,7 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
     // shared memory per CTA so that four CTAs fit (a deeper ring for fewer
     // CTAs per SM measured slower on a B200)
     const size_t row = static_cast<size_t>(s.d_xi + s.d_v) * 8;
-    const size_t fixed = sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) +
-                         sizeof(float2) * 3 * s.M + 16;
+    const size_t fixed = decode_fixed_smem(s);
     const int per_warp = (s.M / S + kBhWarps - 1) / kBhWarps;
     const size_t budget = 56 * 1024;
     int D = 4;
@@ -321,6 +325,10 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
 }
 
 }  // namespace
+
+size_t decode_smem_bytes(const ia_shape_t& s) {
+  return kBhWarps * (static_cast<size_t>(s.d_xi + s.d_v) * 8 + 8) + decode_fixed_smem(s);
+}
 
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
                           const float* delta, const float* A, void* state, float* o, float* num,

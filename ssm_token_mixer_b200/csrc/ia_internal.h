@@ -78,6 +78,8 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
                               void* ws, cudaStream_t st);
 
 // Decode step.
+// Shared memory of the decode kernel with a one-row ring: the least it needs.
+size_t decode_smem_bytes(const ia_shape_t& s);
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
                           const float* delta, const float* A, void* state, float* o, float* num,
                           float* den, cudaStream_t st);

@@ -90,6 +90,10 @@ def test_decode_validation(lib):
     assert rc == 2
     rc = lib.ia_decode_step(ctypes.byref(shape()), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None, None)
     assert rc == 1
+    # rows past 256 entries, or mode parameters past shared memory, are refused
+    for bad in (shape(dx=258), shape(dv=258), shape(M=12000)):
+        rc = lib.ia_decode_step(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, None, None)
+        assert rc == 2
 
 
 def test_injected_launch_failure(lib, monkeypatch):
@@ -108,6 +112,25 @@ def test_injected_launch_failure(lib, monkeypatch):
     t = shape(B=1, H=2, N=100, dx=64, dv=64, M=64, dt=1)   # the no-allocation entry point: bf16, M = 64
     rc = lib.ia_prefill_fwd_static(ctypes.byref(t), FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None,
                                    None, None)
+    assert rc == 4
+    # the optional parts: token-serial (fp32, no workspace) and tensor-core
+    # (bf16 stabilisation + bidirectional, with its workspace) forms
+    import ssm_token_mixer_b200 as ia
+    opt = ia.IAOptions()
+    opt.gain = FAKE
+    opt.eps = 1e-6
+    rc = lib.ia_prefill_fwd_ex(ctypes.byref(s), ctypes.byref(opt), FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                               None, None, None, None, ctypes.c_size_t(0), None)
+    assert rc == 4
+    opt.bidirectional = 1
+    assert lib.ia_prefill_ex_path(ctypes.byref(t), ctypes.byref(opt)) == 1
+    need = lib.ia_prefill_ex_workspace_bytes(ctypes.byref(t), ctypes.byref(opt))
+    rc = lib.ia_prefill_fwd_ex(ctypes.byref(t), ctypes.byref(opt), FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                               None, None, None, FAKE, ctypes.c_size_t(need), None)
+    assert rc == 4
+    opt.bidirectional = 0
+    rc = lib.ia_decode_step_ex(ctypes.byref(s), ctypes.byref(opt), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+                               None, None, None)
     assert rc == 4
     # without the switch, argument errors still come first
     monkeypatch.setenv("IA_INJECT_LAUNCH_FAILURE", "0")
