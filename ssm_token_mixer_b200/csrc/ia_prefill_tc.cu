@@ -107,8 +107,12 @@ constexpr int kMinPiece = 4;             // fewest chunks per CTA the planner ha
 
 // Four roles: 8 prepare warps (0-7) convert the inputs and rotate the carried
 // state into R; 8 output warps (8-15) run the masks, the readout scale and
-// o = num/den; warp 16 issues every tensor-core contraction; warp 17 brings
-// q, k, v in with TMA tensor loads that land in the operand layout.
+// o = num/den, and convert the k and v tiles of the state-only chain that
+// precedes their first chunk; warp 16 issues every tensor-core contraction;
+// warp 17 brings q, k, v in with TMA tensor loads that land in the operand
+// layout.  The inputs are bf16 (q, k through the feature map on the way to
+// fp16), or, for the layer's input stabilisation, k and v arrive as ready
+// fp16 operands and only their rows past the sequence are cleared.
 constexpr int GW = 8;                    // warps per epilogue group
 constexpr int GT = GW * 32;              // threads per epilogue group
 constexpr int NTH = 2 * GT + 64;         // + the MMA warp and the fetch warp
@@ -213,7 +217,6 @@ struct Sched {
     nA = static_cast<int>(g1 - gA);
     nF = static_cast<int>(g1 - g0);
   }
-  __device__ __forceinline__ long long item(int i) const { return i < nA ? gA + i : g0 + (i - nA); }
   __device__ __forceinline__ bool state_only(int i) const { return i < nA; }
   __device__ __forceinline__ int items() const { return nA + nF; }
 };
