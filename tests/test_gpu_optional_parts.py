@@ -178,3 +178,26 @@ def test_optional_parts_paths_and_workspace(dev):
     with pytest.raises(ia.IAError) as err:
         ia.prefill_fwd_ex(g["q"], g["k"], g["v"], 64, delta=g["delta"], bidirectional=True, workspace=ws)
     assert err.value.status == 3   # IA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("dx,dv", [(64, 64), (128, 128)])
+def test_tensor_core_stabilised_split_prefill(oracle_mod, dev, dx, dv):
+    # P13 on the tensor-core form of the stabilised layer: prefill(N1) ->
+    # state -> prefill(N2, state_in) equals the oracle on N1 + N2 (ragged N1)
+    B, H, M, N1, N2 = 2, 3, 64, 100, 90
+    inp = synthetic.layer_inputs(B, H, N1 + N2, dx, dv, "bf16", seed=95 + dx)
+    opt = options(B, H, N1 + N2, dx, dv, M, 96, ("norm",))
+    assert ia.prefill_ex_path(B, H, N1, dx, dv, M, "bf16", norm=True) == "tensor_core"
+    g = lambda x: x.to(dev)
+    sl = lambda x, a, b: x[:, :, a:b].contiguous()
+    kw = {k: g(v) for k, v in opt.items()}
+    r1 = ia.prefill_fwd_ex(*(g(sl(inp[n], 0, N1)) for n in ("q", "k", "v")), M, delta=g(inp["delta"]),
+                           want_state=True, **kw)
+    r2 = ia.prefill_fwd_ex(*(g(sl(inp[n], N1, N1 + N2)) for n in ("q", "k", "v")), M, delta=g(inp["delta"]),
+                           state_in=r1["state"], want_state=True, **kw)
+    ia.check_device_errors()
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **opt)
+    o = torch.cat([r1["o"].cpu(), r2["o"].cpu()], dim=2)
+    assert slice_rel(o, ref["o"], (-2, -1)) < TOL_BF16
+    st = r2["state"].cpu().double().numpy()
+    assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < TOL_BF16
