@@ -200,6 +200,24 @@ IA_API ia_status_t ia_decode_step(const ia_shape_t* shape, const void* q, const 
                            float* o, float* num, float* den, void* stream);
 
 /*
+ * Carry composition for one sequence split into consecutive spans (summary
+ * sec. A.2: parallel passes over pieces with sequential state passing
+ * between them; across GPUs, the spans' local end states are exchanged once
+ * and each span's carry-in is composed from them).  The recurrence is linear
+ * in its state, so
+ *     out = lambda^L * carry_in + local
+ * per (b,h) and mode over U, Gamma and eta, with lambda = exp(Delta A) as in
+ * ia_prefill_fwd (A NULL = S4D-Lin).  L >= 0 is the length in tokens of the
+ * span whose end state from a zero start is `local` (an ia_prefill_fwd
+ * state_out); carry_in is the state before that span (NULL = zero).  All
+ * three are states in the ia_state_bytes layout, device memory, 16-byte
+ * aligned; out may alias carry_in or local.  shape: B, H, d_xi, d_v, M,
+ * delta_per_mode (N ignored).  Errors as for the other entry points.
+ */
+IA_API ia_status_t ia_state_carry(const ia_shape_t* shape, const float* delta, const float* A, long long L,
+                                  const void* carry_in, const void* local, void* out, void* stream);
+
+/*
  * Optional parts of the layer that the pages name beside the plain readout.
  * Every pointer is a caller-owned device array; NULL (or 0) leaves that part
  * out, so an all-zero ia_options_t is the plain layer.

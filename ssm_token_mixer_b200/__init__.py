@@ -95,6 +95,8 @@ def load_library():
     lib.ia_prefill_ex_path.argtypes = [S, O]
     lib.ia_decode_step_ex.restype = ctypes.c_int
     lib.ia_decode_step_ex.argtypes = [S, O] + [P] * 9 + [P]
+    lib.ia_state_carry.restype = ctypes.c_int
+    lib.ia_state_carry.argtypes = [S, P, P, ctypes.c_longlong, P, P, P, P]
     lib.ia_set_launch_events.restype = ctypes.c_int
     lib.ia_set_launch_events.argtypes = [P, P]
     lib.ia_check_device_errors.restype = ctypes.c_int
@@ -165,6 +167,30 @@ def prefill_path(B, H, N, d_xi, d_v, M, dtype):
 def fwd_bwd_path(B, H, N, d_xi, d_v, M, dtype):
     """'tensor_core' or 'sequential': the reverse-pass kernels ia_fwd_bwd runs for this shape."""
     return PATHS[load_library().ia_fwd_bwd_path(ctypes.byref(make_shape(B, H, N, d_xi, d_v, M, dtype)))]
+
+
+def state_carry(local, delta, M, L, B, H, d_xi, d_v, carry_in=None, A=None, out=None, stream=None):
+    """lambda^L * carry_in + local over whole states (flat fp32, the
+    ia_state_bytes layout; see ia_state_carry): the state before a span
+    decayed across it plus what the span built from zero.  Returns out."""
+    lib = load_library()
+    dpm = _check_delta(delta, H, M)
+    shp = make_shape(B, H, 1, d_xi, d_v, M, "f32", dpm)
+    n = lib.ia_state_bytes(ctypes.byref(shp)) // 4
+    _need("local", local, dtype=torch.float32, numel=n)
+    if carry_in is not None:
+        _need("carry_in", carry_in, dtype=torch.float32, numel=n)
+    if A is not None:
+        _need("A", A, dtype=torch.float32, numel=2 * int(M))
+    dev = _cuda_device([("local", local), ("delta", delta), ("carry_in", carry_in), ("A", A), ("out", out)])
+    if out is None:
+        out = torch.empty_like(local)
+    else:
+        _need("out", out, dtype=torch.float32, numel=n)
+    rc = lib.ia_state_carry(ctypes.byref(shp), _ptr(delta), _ptr(A), int(L), _ptr(carry_in), _ptr(local),
+                            _ptr(out), _stream(stream))
+    _check(rc, "ia_state_carry")
+    return out
 
 
 def _presence_options(norm, selective, readout, bidirectional):

@@ -244,6 +244,18 @@ ia_status_t ia_decode_step(const ia_shape_t* s, const void* q, const void* k, co
                                 static_cast<cudaStream_t>(stream)));
 }
 
+ia_status_t ia_state_carry(const ia_shape_t* s, const float* delta, const float* A, long long L,
+                           const void* carry_in, const void* local, void* out, void* stream) {
+  if (!valid_dims(s, false)) return IA_ERR_INVALID_ARG;
+  if (!delta || !local || !out || L < 0) return IA_ERR_INVALID_ARG;
+  const void* ptrs[] = {delta, A, carry_in, local, out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return IA_ERR_INVALID_ARG;
+  if (static_cast<long long>(s->B) * s->H * s->M > (1LL << 31) - 1) return IA_ERR_UNSUPPORTED;   // one block per row
+  if (inject_launch_failure()) return IA_ERR_CUDA;
+  return map_cuda(launch_state_carry(*s, delta, A, L, carry_in, local, out, static_cast<cudaStream_t>(stream)));
+}
+
 ia_status_t ia_set_launch_events(void* begin, void* end) {
   if ((begin == nullptr) != (end == nullptr)) return IA_ERR_INVALID_ARG;
   g_ev_begin = static_cast<cudaEvent_t>(begin);

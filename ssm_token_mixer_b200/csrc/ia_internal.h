@@ -78,6 +78,10 @@ cudaError_t launch_tc_fwd_bwd(const ia_shape_t& s, const TcPlan& p, const void* 
                               void* ws, cudaStream_t st);
 
 // Decode step.
+// out = lambda^L carry_in + local over a whole state (ia_carry.cu).
+cudaError_t launch_state_carry(const ia_shape_t& s, const float* delta, const float* A, long long L,
+                               const void* carry_in, const void* local, void* out, cudaStream_t st);
+
 // Shared memory of the decode kernel with a one-row ring: the least it needs.
 size_t decode_smem_bytes(const ia_shape_t& s);
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
