@@ -526,6 +526,238 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
   prep_raise_flag(a.flags + blockIdx.x, 2, th.tid);
 }
 
+// What a piece start hands back to the chunk loop.
+struct PieceStart {
+  float eta;      // this row's eta of the piece's initial state
+  bool ok;        // false if a wait gave up (uniform over the prepare group)
+  bool pending;   // the CTA still owes its inclusive state
+};
+
+// Everything the prepare warps do at a piece start, between the G7 wait of
+// the previous item and the rotation of the piece's first item: publish the
+// end of the state-only chain or write state_out of the stream that ended,
+// reload E' on a change of head (once every contraction reading the old one
+// is done), and set the piece's initial state (zero, state_in, or the carry
+// from the look-back).  One call out of the chunk loop, so that the loop keeps
+// its registers for the per-chunk work.
+template <int DX>
+__device__ __noinline__ PieceStart prep_piece_start(const TcArgs& a, const PrepThread& th, int i, int nA, long long gA,
+                                                    int nF, bool so, int ch, long long bh, int vb, int h,
+                                                    int prev_bh, int prev_vb, int prev_ch, int cur_h, float eta_c,
+                                                    bool pending, volatile int* abort_flag, volatile int* xchg,
+                                                    volatile int* g4_seen, uint8_t* sE) {
+  constexpr int STRIDE = KR * PCfg<DX>::F + KR;   // floats per published state
+  PieceStart r{eta_c, true, pending};
+  const HeadTables* T = a.tabs + cur_h;
+  if (i > 0) {
+    if (i - 1 < nA) {
+      // end of the state-only chain: publish our last piece's state
+      const bool inclusive = gA % a.nch == 0;
+      prep_publish<DX>(th, (inclusive ? a.incl : a.agg) + static_cast<long long>(blockIdx.x) * STRIDE, eta_c);
+      prep_raise_flag(a.flags + blockIdx.x, inclusive ? 2 : 1, th.tid);
+      r.pending = !inclusive;
+    } else if (prev_ch == a.nch - 1 && a.state_out) {
+      prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
+    }
+  }
+  if (h != cur_h) {
+    // A new head: its E' table replaces the old one once every contraction
+    // reading the old one is done.  G7 of the previous item is; every G2 and
+    // G4 of the previous full items is once the output warps have seen G4 of
+    // the last of them complete.
+    const int t = i - nA;
+    if (t >= 1) {
+      bool ok = true;
+      if (th.tid == 0) {
+        const unsigned long long t0 = global_ns();
+        while (*g4_seen < t) {
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(a.err, kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          __nanosleep(64);
+        }
+        __threadfence_block();
+      }
+      if (named_sync_or(2, GT, !ok)) {
+        r.ok = false;
+        return r;
+      }
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h].E);
+    uint4* dst = reinterpret_cast<uint4*>(sE);
+    for (int x = th.tid; x < KR * C * 2 / 16; x += GT) dst[x] = src[x];
+    T = a.tabs + h;
+  }
+  if (so && gA % a.nch != 0) {   // a local aggregate starts from zero
+    prep_zero<DX>(th);
+    r.eta = 0.f;
+  } else if (so || ch == 0) {    // a stream's start: state_in or zero
+    r.eta = prep_init_from_input<DX>(a, T, th, bh, vb);
+  } else {                       // inside a stream: the carry from the predecessors
+    float e = 0.f;
+    if (!prep_look_back<DX>(a, T, th, abort_flag, xchg, &e)) {
+      r.ok = false;
+      return r;
+    }
+    r.eta = e;
+    if (r.pending) {
+      prep_publish_inclusive<DX>(a, T, th, nF, e);
+      r.pending = false;
+    }
+  }
+  fence_async_smem();   // a reloaded E' table is read by the next contractions
+  return r;
+}
+
+// The prepare warps' chunk loop over the n items of one piece: for each,
+// wait for its tiles, convert them (a full item's q, k, v; the output warps
+// convert a state-only item's k, v), wait for G7 of the item before (except
+// for the piece's first item, whose wait comes before the piece start),
+// rotate the carried state into R and signal the MMA warp.  It sits out of
+// line, apart from the piece starts and their calls, so that its registers
+// hold only what the chunks need.
+struct PrepRun {
+  float eta;
+  uint32_t pd0, pld;   // parities of the G7 barrier and of the loaded barriers (bit per set)
+  bool ok;
+};
+
+template <int DX>
+__device__ __noinline__ PrepRun prep_chunks(const TcArgs& a_in, uint8_t* smem, const PrepThread th, const HeadTables* T,
+                                            int i, int n, int b, bool so, long long bh, int ch, float eta_c,
+                                            uint32_t pd0, uint32_t pld, float esum_tail) {
+  const TcArgs a = a_in;
+  using K = PCfg<DX>;
+  constexpr int FH = K::FH, NB = K::NB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* rdy0 = bars + 0;
+  uint64_t* dne0 = bars + 4;
+  uint64_t* loaded = bars + 16;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  const float2 lamC = T->lamC[th.m];
+  const float sgnLi = th.comp ? lamC.y : -lamC.y;
+  const uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
+  const float esum_c = th.comp ? T->esum[th.m].y : T->esum[th.m].x;
+  PrepRun r{eta_c, pd0, pld, true};
+  for (int j = 0; j < n; ++j, ++i, ++ch, b = b + 1 == NB ? 0 : b + 1) {
+    const int p = i & 1;
+    const int nv = min(C, a.N - ch * C);
+    {
+      const bool ok = mbar_wait_or_abort(loaded + b, (r.pld >> b) & 1u, a.err, abort_flag);
+      r.pld ^= 1u << b;
+      tc_fence_after();
+      if (named_sync_or(2, GT, !ok)) {
+        r.ok = false;
+        return r;
+      }
+    }
+    if (!so) {
+      // bf16 -> fp16 in place (q, k through the feature map); rows past the
+      // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x
+      // 128 bytes; the map is elementwise, so the swizzle does not matter.
+      constexpr int PQ = K::TQ / 16 / GT;   // 16-byte pieces of a q or k tile per thread
+      constexpr int PV = K::TV / 16 / GT;
+      constexpr int NP = 2 * PQ + PV;
+      // every load first (a store may alias a later load, so loads issued in
+      // between would queue behind it), then convert and store
+      uint4 in[NP];
+#pragma unroll
+      for (int u = 0; u < NP; ++u) {
+        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
+        const int pc = th.tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
+        const uint32_t base = tsel == 0 ? K::S_Q + b * K::TQ : (tsel == 1 ? K::S_K + b * K::TQ : K::S_V + b * K::TV);
+        in[u] = *reinterpret_cast<const uint4*>(smem + base + pc * 16);
+      }
+#pragma unroll
+      for (int u = 0; u < NP; ++u) {
+        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
+        const int pc = th.tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
+        const int row = (pc >> 3) & 63;                          // row within its box
+        const uint32_t base = tsel == 0 ? K::S_Q + b * K::TQ : (tsel == 1 ? K::S_K + b * K::TQ : K::S_V + b * K::TV);
+        uint4 out = make_uint4(0u, 0u, 0u, 0u);
+        if (row < nv && tsel > 0 && a.kv_ready) {   // k, v already fp16 operands
+          out = in[u];
+        } else if (row < nv) {
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(x2[e]);
+            w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
+          }
+          out = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *reinterpret_cast<uint4*>(smem + base + pc * 16) = out;
+      }
+    }
+    if (j > 0) {   // G7 of the previous item: the state is current
+      const bool ok = mbar_wait_or_abort(dne0, r.pd0, a.err, abort_flag);
+      r.pd0 ^= 1u;
+      tc_fence_after();
+      if (named_sync_or(2, GT, !ok)) {
+        r.ok = false;
+        return r;
+      }
+    }
+    // R = lambda^C S_hat -> TMEM (the state G7 adds to); for full items also
+    // R_U (fp16 pairs in TMEM, A operand of G3) and R_Gamma (shared memory,
+    // B operand of G6)
+    uint8_t* sRG = smem + K::S_RG + b * K::TRG;
+#pragma unroll
+    for (int blk = 0; blk < FH / 16; ++blk) {
+      const int col0 = th.half * FH + 16 * blk;
+      uint32_t w[16];
+      tmem_ld16(th.trow + K::T_STATE + col0, w);
+      tmem_ld_wait16(w);
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {   // in place: Re/Im of lambda^C times the partner row, two columns at once
+        const float x0 = __uint_as_float(w[e]), x1 = __uint_as_float(w[e + 1]);
+        const uint64_t y = f2_pack(__shfl_xor_sync(kFull, x0, 1), __shfl_xor_sync(kFull, x1, 1));
+        float w0, w1;
+        f2_unpack(f2_fma(lamC2, f2_pack(x0, x1), f2_mul(sgnLi2, y)), w0, w1);
+        w[e] = __float_as_uint(w0);
+        w[e + 1] = __float_as_uint(w1);
+      }
+      tmem_st16(th.trow + K::T_STATE + col0, w);
+      if (!so) {
+        if (a.dump_R) dump_r16(a.dump_R, bh * a.nch + ch, th.k, col0, w);
+        if (col0 < DX) {   // R_U: fp16 pairs into tensor memory, 8 columns per block
+          uint32_t ru[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ru[e] = pack_half2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+          tmem_st8(th.trow + K::T_RU + K::RU_COLS * p + col0 / 2, ru);
+        } else {           // R_Gamma: shared memory, B operand of G6
+#pragma unroll
+          for (int g2 = 0; g2 < 2; ++g2)
+            *reinterpret_cast<uint4*>(sRG + tile_off(th.k, col0 - DX + 8 * g2, K::RSV)) = pack8f(w + 8 * g2, 1.f);
+        }
+      }
+    }
+    tmem_st_wait();
+    {
+      const float y = __shfl_xor_sync(kFull, r.eta, 1);
+      const float Re = fmaf(lamC.x, r.eta, sgnLi * y);
+      if (th.half == 0 && !so) {
+        if (a.dump_Re) a.dump_Re[(bh * a.nch + ch) * KR + th.k] = Re;
+        *reinterpret_cast<uint4*>(sRG + tile_off(th.k, kVB, K::RSV)) = make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
+      }
+      // ragged last chunk: partial sum of E' over the valid keys
+      r.eta = Re + (nv < C ? esum_tail : esum_c);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    mbar_arrive(rdy0);
+  }
+  return r;
+}
+
 // bf16 -> fp16 in place over one tile of PIECES 16-byte pieces, by NT
 // threads (ct = 0 .. NT-1), through the feature map when FEAT; rows past the
 // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x 128
@@ -559,23 +791,18 @@ __device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct, bool
   }
 }
 
-// 576 threads: one SM sub-partition carries five of the 18 warps, so its
-// 16 K registers cap a thread at 96.
+// The four roles of the chunk pass, each out of line so that its registers
+// are allocated for its own loop alone (the prepare warps' piece starts call
+// out of line, and the spills around those calls stay in that role).  Each
+// derives its barriers, tiles and schedule from shared memory and the
+// arguments; the barriers are described where the kernel initialises them.
 template <int DX>
-__global__ void __launch_bounds__(NTH, 1)
-    tc_prefill_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                      const __grid_constant__ CUtensorMap tm_o) {
+__device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_first) {
   using K = PCfg<DX>;
-  constexpr int F = K::F, FH = K::FH, NB = K::NB;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int role = warp < 2 * GW ? warp / GW : warp - 2 * GW + 2;   // prepare, output, mma, fetch
-  const int gw = warp & (GW - 1);          // warp index within its epilogue group
-  const int quad = warp & 3, half = gw >> 2;
+  constexpr int NB = K::NB;
+  const int tid = threadIdx.x, lane = tid & 31;
   const Sched sc(a.total, a.G, blockIdx.x, a.nch);
   const int nI = sc.items();
-
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
   uint64_t* rdy = bars + 0;       // [4]: prepare -> G7 (+G1), output -> G2G3, G4, G5G6
   uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
@@ -583,88 +810,14 @@ __global__ void __launch_bounds__(NTH, 1)
   uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
   uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
   uint64_t* bar_drain = bars + 15;
-  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
-  // [NB]: output warps -> G7 of a state-only item, that set's k and v are
-  // fp16 operands.  A set is refilled only after that G7, so no barrier runs
-  // a phase ahead of the MMA warp's wait.
-  uint64_t* rdyKV = bars + 19;
-  static_assert(NB <= 3 && (19 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
+  uint64_t* rdyKV = bars + 19;    // [NB]: output warps -> G7 of a state-only item (k, v converted)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
-  volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
-  // G4 groups known done: the output warps see each G4 complete, in order,
-  // before E3 of its chunk, and count them here for the prepare warps
-  volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
   const uint32_t sbase = smem_u32(smem);
   auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
   auto sK = [&](int b) { return K::S_K + b * K::TQ; };
   auto sV = [&](int b) { return K::S_V + b * K::TV; };
   auto sRG = [&](int b) { return K::S_RG + b * K::TRG; };
-  // stream s = bh * nvb + vb
-  auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
-
-  if (warp == 0) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(rdy + i, i == 0 ? GT : GT);
-      mbar_init(dne + i, 1);
-    }
-    mbar_init(dneS, 1);
-    for (int i = 0; i < NB; ++i) {
-      mbar_init(freeQK + i, 1);
-      mbar_init(freeVR + i, 1);
-      mbar_init(loaded + i, 1);
-    }
-    mbar_init(bar_drain, 1);
-    for (int i = 0; i < NB; ++i) mbar_init(rdyKV + i, GT);
-    *abort_flag = 0;
-    *g4_seen = 0;
-    fence_barrier_init();
-  }
-  {
-    // the ones block after V: MN element 64 (first of the second 64-block)
-    // is 1 in every row, the rest 0, in the swizzled layout
-    for (int i = tid; i < C * 8; i += NTH) {
-      const int r = i >> 3, c = i & 7;
-      *reinterpret_cast<uint4*>(smem + K::S_ONES + r * 128 + c * 16) =
-          make_uint4((c == (r & 7)) ? 0x00003C00u : 0u, 0u, 0u, 0u);
-    }
-    // R_Gamma's extra columns start at zero (column 64 receives R_eta every chunk)
-    for (int r = tid; r < KR; r += NTH) {
-      for (int b = 0; b < NB; ++b) {
-        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-    // Everything above touches only this CTA's own resources.  The kernel may
-    // have been launched while the table kernel before it still runs: every
-    // global read (tables, inputs, look-back flags, which the table kernel
-    // clears) comes after this wait, and nothing global is written before it.
-    griddep_wait();
-  }
-  // The E' table depends on the head; a CTA may span heads, so it is copied
-  // per piece by the prepare warps (see load_table) -- except that the first
-  // item's head is loaded here by everyone.
-  int h_first = 0;
-  {
-    Walker w;
-    first_item(w);
-    h_first = w.h;
-  }
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h_first].E);
-    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-    for (int i = tid; i < KR * C * 2 / 16; i += NTH) dst[i] = src[i];
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  if (role == 2) {
+  const uint32_t tmem = *reinterpret_cast<const uint32_t*>(smem + K::S_TMEMH);
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t pr[4] = {0u, 0u, 0u, 0u};
@@ -854,7 +1007,25 @@ __global__ void __launch_bounds__(NTH, 1)
       }
     }
     __syncwarp();
-  } else if (role == 0) {
+}
+
+template <int DX>
+__device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int h_first) {
+  using K = PCfg<DX>;
+  constexpr int NB = K::NB;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gw = warp & (GW - 1);          // warp index within its epilogue group
+  const int quad = warp & 3, half = gw >> 2;
+  const Sched sc(a.total, a.G, blockIdx.x, a.nch);
+  const int nI = sc.items();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
+  volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);   // G4 groups seen done
+  // stream s = bh * nvb + vb
+  auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
+  const uint32_t tmem = *reinterpret_cast<const uint32_t*>(smem + K::S_TMEMH);
     // ------------------------------------------------ prepare warps
     const int k = 32 * quad + lane;
     const int m = k >> 1, comp = k & 1;
@@ -862,18 +1033,9 @@ __global__ void __launch_bounds__(NTH, 1)
     uint32_t pd0 = 0u, pld = 0u;   // parities; pld bit b for buffer set b
     int cur_h = h_first;
     const HeadTables* T = a.tabs + cur_h;
-    float2 lamC = T->lamC[m];
-    float sgnLi = comp ? lamC.y : -lamC.y;
-    uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
-    float esum_c = comp ? T->esum[m].y : T->esum[m].x;
-    auto set_head = [&](int h) {   // per-mode constants of head h
+    auto set_head = [&](int h) {
       cur_h = h;
       T = a.tabs + h;
-      lamC = T->lamC[m];
-      sgnLi = comp ? lamC.y : -lamC.y;
-      lamC2 = f2_pack(lamC.x, lamC.x);
-      sgnLi2 = f2_pack(sgnLi, sgnLi);
-      esum_c = comp ? T->esum[m].y : T->esum[m].x;
     };
     auto waitA = [&](uint64_t* bar, uint32_t& ph) -> bool {   // uniform over the prepare group
       const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
@@ -881,61 +1043,8 @@ __global__ void __launch_bounds__(NTH, 1)
       tc_fence_after();
       return !named_sync_or(2, GT, !r);
     };
-    auto waitLoaded = [&](int b) -> bool {
-      const bool r = mbar_wait_or_abort(loaded + b, (pld >> b) & 1u, a.err, abort_flag);
-      pld ^= 1u << b;
-      tc_fence_after();
-      return !named_sync_or(2, GT, !r);
-    };
-    // bf16 -> fp16 in place (q, k through the feature map); rows past the
-    // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x 128
-    // bytes; the map is elementwise, so the swizzle does not matter.
-    auto convert = [&](int nv, int b, bool with_q) {
-      constexpr int PQ = K::TQ / 16 / GT;   // 16-byte pieces of a q or k tile per thread
-      constexpr int PV = K::TV / 16 / GT;
-      constexpr int NP = 2 * PQ + PV;
-      // every load first (a store may alias a later load, so loads issued in
-      // between would queue behind it), then convert and store
-      uint4 in[NP];
-#pragma unroll
-      for (int u = 0; u < NP; ++u) {
-        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
-        const int pc = tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
-        const uint32_t base = tsel == 0 ? sQ(b) : (tsel == 1 ? sK(b) : sV(b));
-        if (tsel != 0 || with_q) in[u] = *reinterpret_cast<const uint4*>(smem + base + pc * 16);
-      }
-#pragma unroll
-      for (int u = 0; u < NP; ++u) {
-        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
-        if (tsel == 0 && !with_q) continue;
-        const int pc = tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
-        const int r = (pc >> 3) & 63;                          // row within its box
-        const uint32_t base = tsel == 0 ? sQ(b) : (tsel == 1 ? sK(b) : sV(b));
-        uint4* ptr = reinterpret_cast<uint4*>(smem + base + pc * 16);
-        uint4 out = make_uint4(0u, 0u, 0u, 0u);
-        if (r < nv && tsel > 0 && a.kv_ready) {   // k, v already fp16 operands
-          out = in[u];
-        } else if (r < nv) {
-          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(x2[e]);
-            w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
-          }
-          out = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        *ptr = out;
-      }
-    };
     const PrepThread th{trow, tid, k, m, comp, half};
     float eta_c = 0.f;
-    constexpr int STRIDE = KR * F + KR;   // floats per published state
-    auto load_table = [&](int h) {   // E' of head h into shared memory (prepare group)
-      const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h].E);
-      uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
-      for (int i = tid; i < KR * C * 2 / 16; i += GT) dst[i] = src[i];
-    };
 
     bool ok = true;
     bool single_piece_pending = false;   // publish our inclusive state once the carry is known
@@ -943,130 +1052,60 @@ __global__ void __launch_bounds__(NTH, 1)
     first_item(w);
     int prev_bh = 0, prev_vb = 0, prev_ch = 0;
     int b = 0;   // buffer set of item i (i % NB)
-    for (int i = 0; ok && i < nI; ++i, w.next(sc, i - 1, a.nch, a.nvb, a.H), b = b + 1 == NB ? 0 : b + 1) {
-      const int p = i & 1;
+    // One piece at a time: the state-only chain, then each run of a stream's
+    // chunks in the range.  Its start runs after G7 of the item before.
+    for (int i = 0; ok && i < nI;) {
       const bool so = sc.state_only(i);
-      const int ch = w.ch;
-      const int nv = min(C, a.N - ch * C);
-      const long long bh = w.bh;
-      const int vb = w.vb;
-      if (!(ok = waitLoaded(b))) break;
-      if (!so) convert(nv, b, true);   // the output warps convert a state-only item's k, v
-      const bool piece_start = so ? (i == 0) : (i == sc.nA || ch == 0);
+      const int n = so ? sc.nA : min(a.nch - w.ch, nI - i);
       if (i > 0 && !(ok = waitA(dne + 0, pd0))) break;   // G7 of the previous item: the state is current
-      if (piece_start) {
-        if (i > 0) {
-          if (sc.state_only(i - 1)) {
-            // end of the state-only chain: publish our last piece's state
-            const bool inclusive = sc.gA % a.nch == 0;
-            prep_publish<DX>(th, (inclusive ? a.incl : a.agg) + static_cast<long long>(blockIdx.x) * STRIDE, eta_c);
-            prep_raise_flag(a.flags + blockIdx.x, inclusive ? 2 : 1, tid);
-            single_piece_pending = !inclusive;
-          } else if (prev_ch == a.nch - 1 && a.state_out) {
-            prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
-          }
-        }
-        const int h = w.h;
-        if (h != cur_h) {
-          // A new head: its E' table replaces the old one once every
-          // contraction reading the old one is done.  G7 of the previous
-          // item is; every G2 and G4 of the previous full items is once the
-          // output warps have seen G4 of the last of them complete.
-          const int t = i - sc.nA;
-          if (t >= 1) {
-            bool r = true;
-            if (tid == 0) {
-              const unsigned long long t0 = global_ns();
-              while (*g4_seen < t) {
-                if (*abort_flag) { r = false; break; }
-                if (global_ns() - t0 > kWaitLimitNs) {
-                  atomicOr(a.err, kErrTimeout);
-                  *abort_flag = 1;
-                  r = false;
-                  break;
-                }
-                __nanosleep(64);
-              }
-              __threadfence_block();
-            }
-            if (!(ok = !named_sync_or(2, GT, !r))) break;
-          }
-          load_table(h);
-          set_head(h);
-        }
-        if (so && sc.gA % a.nch != 0) {   // a local aggregate starts from zero
-          prep_zero<DX>(th);
-          eta_c = 0.f;
-        } else if (so || ch == 0) {        // a stream's start: state_in or zero
-          eta_c = prep_init_from_input<DX>(a, T, th, bh, vb);
-        } else {                           // inside a stream: the carry from the predecessors
-          if (!(ok = prep_look_back<DX>(a, T, th, abort_flag, xchg, &eta_c))) break;
-          if (single_piece_pending) {
-            prep_publish_inclusive<DX>(a, T, th, sc.nF, eta_c);
-            single_piece_pending = false;
-          }
-        }
-        fence_async_smem();   // a reloaded E' table is read by the next contractions
-      }
-      // R = lambda^C S_hat -> TMEM (the state G7 adds to); for full items also
-      // R_U (fp16 pairs in TMEM, A operand of G3) and R_Gamma (shared memory,
-      // B operand of G6)
-#pragma unroll
-      for (int blk = 0; blk < FH / 16; ++blk) {
-        const int col0 = half * FH + 16 * blk;
-        uint32_t w[16];
-        tmem_ld16(trow + K::T_STATE + col0, w);
-        tmem_ld_wait16(w);
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {   // in place: Re/Im of lambda^C times the partner row, two columns at once
-          const float x0 = __uint_as_float(w[e]), x1 = __uint_as_float(w[e + 1]);
-          const uint64_t y = f2_pack(__shfl_xor_sync(kFull, x0, 1), __shfl_xor_sync(kFull, x1, 1));
-          float w0, w1;
-          f2_unpack(f2_fma(lamC2, f2_pack(x0, x1), f2_mul(sgnLi2, y)), w0, w1);
-          w[e] = __float_as_uint(w0);
-          w[e + 1] = __float_as_uint(w1);
-        }
-        tmem_st16(trow + K::T_STATE + col0, w);
-        if (!so) {
-          if (a.dump_R) dump_r16(a.dump_R, bh * a.nch + ch, k, col0, w);
-          if (col0 < DX) {   // R_U: fp16 pairs into tensor memory, 8 columns per block
-            uint32_t ru[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              ru[e] = pack_half2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
-            tmem_st8(trow + K::T_RU + K::RU_COLS * p + col0 / 2, ru);
-          } else {           // R_Gamma: shared memory, B operand of G6
-#pragma unroll
-            for (int g2 = 0; g2 < 2; ++g2)
-              *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, col0 - DX + 8 * g2, K::RSV)) =
-                  pack8f(w + 8 * g2, 1.f);
-          }
-        }
-      }
-      tmem_st_wait();
-      {
-        const float y = __shfl_xor_sync(kFull, eta_c, 1);
-        const float Re = fmaf(lamC.x, eta_c, sgnLi * y);
-        if (half == 0 && !so) {
-          if (a.dump_Re) a.dump_Re[(bh * a.nch + ch) * KR + k] = Re;
-          *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(k, kVB, K::RSV)) =
-              make_uint4(pack_half2(Re, 0.f), 0u, 0u, 0u);
-        }
-        // ragged last chunk: partial sum of E' over the valid keys
-        eta_c = Re + (nv < C ? ragged_esum(T, m, comp, nv) : esum_c);
-      }
-      fence_async_smem();
-      tc_fence_before();
-      mbar_arrive(rdy + 0);
-      prev_bh = static_cast<int>(bh);
-      prev_vb = vb;
-      prev_ch = ch;
+      const PieceStart ps = prep_piece_start<DX>(a, th, i, sc.nA, sc.gA, sc.nF, so, w.ch, w.bh, w.vb, w.h, prev_bh,
+                                                 prev_vb, prev_ch, cur_h, eta_c, single_piece_pending, abort_flag,
+                                                 xchg, g4_seen, smem + K::S_E);
+      if (!(ok = ps.ok)) break;
+      eta_c = ps.eta;
+      single_piece_pending = ps.pending;
+      if (w.h != cur_h) set_head(w.h);
+      const int last_nv = min(C, a.N - (w.ch + n - 1) * C);
+      const float esum_tail = last_nv < C ? ragged_esum(T, m, comp, last_nv) : 0.f;
+      const PrepRun run = prep_chunks<DX>(a, smem, th, T, i, n, b, so, w.bh, w.ch, eta_c, pd0, pld, esum_tail);
+      eta_c = run.eta;
+      pd0 = run.pd0;
+      pld = run.pld;
+      if (!(ok = run.ok)) break;
+      prev_bh = w.bh;
+      prev_vb = w.vb;
+      prev_ch = w.ch + n - 1;
+      i += n;
+      b = (b + n) % NB;
+      if (i < nI) w.seek(i < sc.nA ? sc.gA + i : sc.g0 + (i - sc.nA), a.nch, a.nvb, a.H);
     }
     if (ok && nI > 0 && a.state_out && sc.g1 % a.nch == 0) {
       ok = waitA(dne + 0, pd0);   // G7 of the last chunk
       if (ok) prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
     }
-  } else if (role == 1) {
+}
+
+template <int DX>
+__device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int h_first,
+                                          const CUtensorMap& tm_o) {
+  using K = PCfg<DX>;
+  constexpr int NB = K::NB;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gw = warp & (GW - 1);          // warp index within its epilogue group
+  const int quad = warp & 3, half = gw >> 2;
+  const Sched sc(a.total, a.G, blockIdx.x, a.nch);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* rdy = bars + 0;       // [4]: prepare -> G7 (+G1), output -> G2G3, G4, G5G6
+  uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
+  uint64_t* dneS = bars + 8;      // G1 done
+  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  uint64_t* rdyKV = bars + 19;    // [NB]: output warps -> G7 of a state-only item (k, v converted)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);   // G4 groups seen done
+  const uint32_t sbase = smem_u32(smem);
+  auto sK = [&](int b) { return K::S_K + b * K::TQ; };
+  auto sV = [&](int b) { return K::S_V + b * K::TV; };
+  const uint32_t tmem = *reinterpret_cast<const uint32_t*>(smem + K::S_TMEMH);
     // ------------------------------------------------ output warps
     const int k = 32 * quad + lane;
     const int m = k >> 1;
@@ -1243,8 +1282,27 @@ __global__ void __launch_bounds__(NTH, 1)
       if (head) w.step(a.nch, a.nvb, a.H);
     }
     if (tid == GT) bulk_wait_all();   // o is in global memory before the block exits
-  }
-  if (role == 3) {
+}
+
+template <int DX>
+__device__ __noinline__ void tc_role_fetch(const TcArgs& a, uint8_t* smem, int h_first, const CUtensorMap& tm_q,
+                                         const CUtensorMap& tm_k, const CUtensorMap& tm_v) {
+  using K = PCfg<DX>;
+  constexpr int NB = K::NB;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const Sched sc(a.total, a.G, blockIdx.x, a.nch);
+  const int nI = sc.items();
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
+  uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
+  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  const uint32_t sbase = smem_u32(smem);
+  auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
+  auto sK = [&](int b) { return K::S_K + b * K::TQ; };
+  auto sV = [&](int b) { return K::S_V + b * K::TV; };
+  // stream s = bh * nvb + vb
+  auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
     // ------------------------------------------------ fetch warp
     if (lane == 0) {
       int issued = 0;
@@ -1275,7 +1333,116 @@ __global__ void __launch_bounds__(NTH, 1)
       }
     }
     __syncwarp();
+}
+
+
+// 576 threads: one SM sub-partition carries five of the 18 warps, so its
+// 16 K registers cap a thread at 96.
+template <int DX>
+__global__ void __launch_bounds__(NTH, 1)
+    tc_prefill_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o) {
+  using K = PCfg<DX>;
+  constexpr int NB = K::NB;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int role = warp < 2 * GW ? warp / GW : warp - 2 * GW + 2;   // prepare, output, mma, fetch
+  const Sched sc(a.total, a.G, blockIdx.x, a.nch);
+  const int nI = sc.items();
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
+  uint64_t* rdy = bars + 0;       // [4]: prepare -> G7 (+G1), output -> G2G3, G4, G5G6
+  uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
+  uint64_t* dneS = bars + 8;      // G1 done
+  uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
+  uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
+  uint64_t* bar_drain = bars + 15;
+  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  // [NB]: output warps -> G7 of a state-only item, that set's k and v are
+  // fp16 operands.  A set is refilled only after that G7, so no barrier runs
+  // a phase ahead of the MMA warp's wait.
+  uint64_t* rdyKV = bars + 19;
+  static_assert(NB <= 3 && (19 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
+  volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
+  // G4 groups known done: the output warps see each G4 complete, in order,
+  // before E3 of its chunk, and count them here for the prepare warps
+  volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + K::S_TMEMH);
+  const uint32_t sbase = smem_u32(smem);
+  auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
+  auto sK = [&](int b) { return K::S_K + b * K::TQ; };
+  auto sV = [&](int b) { return K::S_V + b * K::TV; };
+  auto sRG = [&](int b) { return K::S_RG + b * K::TRG; };
+  // stream s = bh * nvb + vb
+  auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
+
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
   }
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(rdy + i, i == 0 ? GT : GT);
+      mbar_init(dne + i, 1);
+    }
+    mbar_init(dneS, 1);
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(freeQK + i, 1);
+      mbar_init(freeVR + i, 1);
+      mbar_init(loaded + i, 1);
+    }
+    mbar_init(bar_drain, 1);
+    for (int i = 0; i < NB; ++i) mbar_init(rdyKV + i, GT);
+    *abort_flag = 0;
+    *g4_seen = 0;
+    fence_barrier_init();
+  }
+  {
+    // the ones block after V: MN element 64 (first of the second 64-block)
+    // is 1 in every row, the rest 0, in the swizzled layout
+    for (int i = tid; i < C * 8; i += NTH) {
+      const int r = i >> 3, c = i & 7;
+      *reinterpret_cast<uint4*>(smem + K::S_ONES + r * 128 + c * 16) =
+          make_uint4((c == (r & 7)) ? 0x00003C00u : 0u, 0u, 0u, 0u);
+    }
+    // R_Gamma's extra columns start at zero (column 64 receives R_eta every chunk)
+    for (int r = tid; r < KR; r += NTH) {
+      for (int b = 0; b < NB; ++b) {
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(smem + sRG(b) + tile_off(r, kVB + 8, K::RSV)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    // Everything above touches only this CTA's own resources.  The kernel may
+    // have been launched while the table kernel before it still runs: every
+    // global read (tables, inputs, look-back flags, which the table kernel
+    // clears) comes after this wait, and nothing global is written before it.
+    griddep_wait();
+  }
+  // The E' table depends on the head; a CTA may span heads, so it is copied
+  // per piece by the prepare warps (see load_table) -- except that the first
+  // item's head is loaded here by everyone.
+  int h_first = 0;
+  {
+    Walker w;
+    first_item(w);
+    h_first = w.h;
+  }
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h_first].E);
+    uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
+    for (int i = tid; i < KR * C * 2 / 16; i += NTH) dst[i] = src[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (role == 2) tc_role_mma<DX>(a, smem, h_first);
+  else if (role == 0) tc_role_prepare<DX>(a, smem, h_first);
+  else if (role == 1) tc_role_output<DX>(a, smem, h_first, tm_o);
+  else tc_role_fetch<DX>(a, smem, h_first, tm_q, tm_k, tm_v);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
