@@ -435,48 +435,71 @@ __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* 
   *eta += fmaf(fr, xe, fs * ye);
 }
 
-// Carry into a first piece that starts inside a stream: the sum over
-// predecessors p = c-1, c-2, ... of lambda^(C n) times their published end
-// states, n counting the chunks between p's piece and ours; stops at the
-// first inclusive state.  Leaves the carry in the TMEM state and *eta.
-// Returns false if a wait gave up (uniform over the prepare group).
+// Carry into a first piece that starts inside a stream: the sum over the
+// predecessors q = c-1, c-2, ... in the stream of lambda^(C d_q) times their
+// published end states, d_q the chunks from q's range end to our start,
+// down to the first inclusive state.  The flags of up to kLookBackWindow
+// predecessors are awaited together and their states summed in one round,
+// so a CTA pays one wait for all of them instead of one per hop.  Leaves the
+// carry in the TMEM state and *eta.  Returns false if a wait gave up
+// (uniform over the prepare group).
+constexpr int kLookBackWindow = 8;
+
 template <int DX>
 __device__ __noinline__ bool prep_look_back(const TcArgs& a, const HeadTables* T, const PrepThread& th,
                                             volatile int* abort_flag, volatile int* xchg, float* eta) {
   constexpr int STRIDE = KR * PCfg<DX>::F + KR;
+  const double re_dA = T->re_dA[th.m], im_dA = T->im_dA[th.m];
   prep_zero<DX>(th);
   *eta = 0.f;
-  double mr = 1.0, mi = 0.0;
-  for (int p = static_cast<int>(blockIdx.x) - 1; p >= 0; --p) {
-    if (th.tid == 0) {   // poll the predecessor's flag (bounded)
-      int f = ld_acquire(a.flags + p);
+  const long long g0 = range_lo(a.total, a.G, blockIdx.x);
+  for (int p = static_cast<int>(blockIdx.x) - 1; p >= 0;) {
+    if (th.tid == 0) {   // await p, p-1, ... (bounded): stop at an inclusive state or the window's end
+      int lo = -1, incl = 0;
       const unsigned long long t0 = global_ns();
-      while (f == 0 && !*abort_flag) {
-        if (global_ns() - t0 > kWaitLimitNs) {
-          atomicOr(a.err, kErrTimeout);
-          *abort_flag = 1;
+      for (int q = p; q >= 0 && q > p - kLookBackWindow; --q) {
+        int f = ld_acquire(a.flags + q);
+        while (f == 0 && !*abort_flag) {
+          if (global_ns() - t0 > kWaitLimitNs) {
+            atomicOr(a.err, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          f = ld_acquire(a.flags + q);
+        }
+        if (f == 0) {
+          lo = -1;
           break;
         }
-        f = ld_acquire(a.flags + p);
+        lo = q;
+        if (f == 2) {
+          incl = 1;
+          break;
+        }
       }
-      *xchg = *abort_flag ? 0 : f;
+      *xchg = lo < 0 ? 0 : (((lo + 1) << 1) | incl);
     }
     named_sync(4, GT);
-    const int f = *xchg;
+    const int v = *xchg;
     named_sync(4, GT);
-    if (f == 0) return false;
+    if (v == 0) return false;
+    const int lo = (v >> 1) - 1;
+    const bool incl = (v & 1) != 0;
     __threadfence();
-    prep_accumulate<DX>(th, (f == 2 ? a.incl : a.agg) + static_cast<long long>(p) * STRIDE, mr, mi, eta);
-    if (f == 2) return true;
-    // p published a local state only: its last piece starts inside the
-    // stream, so continue with p - 1 one piece further back
-    const long long p_lo = range_lo(a.total, a.G, p), p_hi = range_lo(a.total, a.G, p + 1);
-    const long long n = p_hi - max(p_lo, (p_hi - 1) / a.nch * a.nch);
-    double lr, li;
-    lam_pow(T, th.m, static_cast<double>(C) * n, &lr, &li);
-    const double nr = mr * lr - mi * li;
-    mi = mr * li + mi * lr;
-    mr = nr;
+    for (int q = p; q >= lo; --q) {
+      const double n = static_cast<double>(C) * static_cast<double>(g0 - range_lo(a.total, a.G, q + 1));
+      double lr = 1.0, li = 0.0;
+      if (n > 0.0) {
+        const double e = exp(n * re_dA);
+        double sn, cs;
+        sincos(fmod(n * im_dA, 6.283185307179586476925), &sn, &cs);
+        lr = e * cs;
+        li = e * sn;
+      }
+      prep_accumulate<DX>(th, (q == lo && incl ? a.incl : a.agg) + static_cast<long long>(q) * STRIDE, lr, li, eta);
+    }
+    if (incl) return true;
+    p = lo - 1;
   }
   return false;   // unreachable: the stream's first piece publishes an inclusive state
 }
