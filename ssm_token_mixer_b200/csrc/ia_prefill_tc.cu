@@ -648,64 +648,71 @@ __device__ __noinline__ PieceStart prep_piece_start(const TcArgs& a, const PrepT
 // hold only what the chunks need.
 struct PrepRun {
   float eta;
-  uint32_t pd0, pld;   // parities of the G7 barrier and of the loaded barriers (bit per set)
+  uint32_t pd0, pld, pldv;   // parities of the G7 barrier and of the q,k / v loaded barriers (bit per set)
   bool ok;
 };
 
 template <int DX>
 __device__ __noinline__ PrepRun prep_chunks(const TcArgs& a_in, uint8_t* smem, const PrepThread th, const HeadTables* T,
                                             int i, int n, int b, bool so, long long bh, int ch, float eta_c,
-                                            uint32_t pd0, uint32_t pld, float esum_tail) {
+                                            uint32_t pd0, uint32_t pld, uint32_t pldv, float esum_tail) {
   const TcArgs a = a_in;
   using K = PCfg<DX>;
   constexpr int FH = K::FH, NB = K::NB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
   uint64_t* rdy0 = bars + 0;
   uint64_t* dne0 = bars + 4;
-  uint64_t* loaded = bars + 16;
+  uint64_t* loadedQK = bars + 16;
+  uint64_t* loadedV = bars + 22;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   const float2 lamC = T->lamC[th.m];
   const float sgnLi = th.comp ? lamC.y : -lamC.y;
   const uint64_t lamC2 = f2_pack(lamC.x, lamC.x), sgnLi2 = f2_pack(sgnLi, sgnLi);
   const float esum_c = th.comp ? T->esum[th.m].y : T->esum[th.m].x;
-  PrepRun r{eta_c, pd0, pld, true};
+  PrepRun r{eta_c, pd0, pld, pldv, true};
+  // waits for set b's q, k (QK) or v tiles, uniform over the prepare group
+  auto wait_tiles = [&](uint64_t* bar, uint32_t& bits) -> bool {
+    const bool ok = mbar_wait_or_abort(bar + b, (bits >> b) & 1u, a.err, abort_flag);
+    bits ^= 1u << b;
+    tc_fence_after();
+    return !named_sync_or(2, GT, !ok);
+  };
   for (int j = 0; j < n; ++j, ++i, ++ch, b = b + 1 == NB ? 0 : b + 1) {
     const int p = i & 1;
     const int nv = min(C, a.N - ch * C);
-    {
-      const bool ok = mbar_wait_or_abort(loaded + b, (r.pld >> b) & 1u, a.err, abort_flag);
-      r.pld ^= 1u << b;
-      tc_fence_after();
-      if (named_sync_or(2, GT, !ok)) {
-        r.ok = false;
-        return r;
-      }
+    if (!wait_tiles(loadedQK, r.pld)) {
+      r.ok = false;
+      return r;
     }
-    if (!so) {
-      // bf16 -> fp16 in place (q, k through the feature map); rows past the
-      // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x
-      // 128 bytes; the map is elementwise, so the swizzle does not matter.
-      constexpr int PQ = K::TQ / 16 / GT;   // 16-byte pieces of a q or k tile per thread
-      constexpr int PV = K::TV / 16 / GT;
-      constexpr int NP = 2 * PQ + PV;
+    // bf16 -> fp16 in place (q, k through the feature map); rows past the
+    // sequence become 0.  A tile is a sequence of 8 KB boxes of 64 rows x
+    // 128 bytes; the map is elementwise, so the swizzle does not matter.
+    // q and k land before v (their buffers are released one contraction
+    // group earlier), so they are converted first.
+    constexpr int PQ = K::TQ / 16 / GT;   // 16-byte pieces of a q or k tile per thread
+    constexpr int PV = K::TV / 16 / GT;
+    auto convert = [&](const int tsel, const int NPIECE) {
       // every load first (a store may alias a later load, so loads issued in
       // between would queue behind it), then convert and store
-      uint4 in[NP];
+      uint4 in[2 * PQ];
+      const uint32_t base = tsel == 0 ? K::S_Q + b * K::TQ : (tsel == 1 ? K::S_K + b * K::TQ : K::S_V + b * K::TV);
 #pragma unroll
-      for (int u = 0; u < NP; ++u) {
-        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
-        const int pc = th.tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
-        const uint32_t base = tsel == 0 ? K::S_Q + b * K::TQ : (tsel == 1 ? K::S_K + b * K::TQ : K::S_V + b * K::TV);
-        in[u] = *reinterpret_cast<const uint4*>(smem + base + pc * 16);
+      for (int u = 0; u < 2 * PQ; ++u) {
+        if (u >= NPIECE) break;
+        const int t = tsel == 0 && u >= PQ ? 1 : tsel;   // tsel 0 converts q then k
+        const uint32_t bs = t == 0 ? base : (t == 1 ? K::S_K + b * K::TQ : base);
+        const int pc = th.tid + (tsel == 0 ? u % PQ : u) * GT;
+        in[u] = *reinterpret_cast<const uint4*>(smem + bs + pc * 16);
       }
 #pragma unroll
-      for (int u = 0; u < NP; ++u) {
-        const int tsel = u < PQ ? 0 : (u < 2 * PQ ? 1 : 2);   // q, k, v
-        const int pc = th.tid + (u - (tsel == 0 ? 0 : (tsel == 1 ? PQ : 2 * PQ))) * GT;
-        const int row = (pc >> 3) & 63;                          // row within its box
-        const uint32_t base = tsel == 0 ? K::S_Q + b * K::TQ : (tsel == 1 ? K::S_K + b * K::TQ : K::S_V + b * K::TV);
+      for (int u = 0; u < 2 * PQ; ++u) {
+        if (u >= NPIECE) break;
+        const int t = tsel == 0 && u >= PQ ? 1 : tsel;
+        const uint32_t bs = t == 0 ? base : (t == 1 ? K::S_K + b * K::TQ : base);
+        const int pc = th.tid + (tsel == 0 ? u % PQ : u) * GT;
+        const int row = (pc >> 3) & 63;   // row within its box
         uint4 out = make_uint4(0u, 0u, 0u, 0u);
-        if (row < nv && tsel > 0 && a.kv_ready) {   // k, v already fp16 operands
+        if (row < nv && t > 0 && a.kv_ready) {   // k, v already fp16 operands
           out = in[u];
         } else if (row < nv) {
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&in[u]);
@@ -713,13 +720,19 @@ __device__ __noinline__ PrepRun prep_chunks(const TcArgs& a_in, uint8_t* smem, c
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(x2[e]);
-            w[e] = tsel < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
+            w[e] = t < 2 ? feat_h2(f.x, f.y) : pack_half2(f.x, f.y);
           }
           out = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *reinterpret_cast<uint4*>(smem + base + pc * 16) = out;
+        *reinterpret_cast<uint4*>(smem + bs + pc * 16) = out;
       }
+    };
+    if (!so) convert(0, 2 * PQ);   // the output warps convert a state-only item's k, v
+    if (!wait_tiles(loadedV, r.pldv)) {
+      r.ok = false;
+      return r;
     }
+    if (!so) convert(2, PV);
     if (j > 0) {   // G7 of the previous item: the state is current
       const bool ok = mbar_wait_or_abort(dne0, r.pd0, a.err, abort_flag);
       r.pd0 ^= 1u;
@@ -1053,7 +1066,7 @@ __device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int
     const int k = 32 * quad + lane;
     const int m = k >> 1, comp = k & 1;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
-    uint32_t pd0 = 0u, pld = 0u;   // parities; pld bit b for buffer set b
+    uint32_t pd0 = 0u, pld = 0u, pldv = 0u;   // parities; pld, pldv bit b for buffer set b
     int cur_h = h_first;
     const HeadTables* T = a.tabs + cur_h;
     auto set_head = [&](int h) {
@@ -1090,10 +1103,11 @@ __device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int
       if (w.h != cur_h) set_head(w.h);
       const int last_nv = min(C, a.N - (w.ch + n - 1) * C);
       const float esum_tail = last_nv < C ? ragged_esum(T, m, comp, last_nv) : 0.f;
-      const PrepRun run = prep_chunks<DX>(a, smem, th, T, i, n, b, so, w.bh, w.ch, eta_c, pd0, pld, esum_tail);
+      const PrepRun run = prep_chunks<DX>(a, smem, th, T, i, n, b, so, w.bh, w.ch, eta_c, pd0, pld, pldv, esum_tail);
       eta_c = run.eta;
       pd0 = run.pd0;
       pld = run.pld;
+      pldv = run.pldv;
       if (!(ok = run.ok)) break;
       prev_bh = w.bh;
       prev_vb = w.vb;
@@ -1121,7 +1135,8 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
   uint64_t* rdy = bars + 0;       // [4]: prepare -> G7 (+G1), output -> G2G3, G4, G5G6
   uint64_t* dne = bars + 4;       // [4]: G7 done, G2G3 done, G4 done, G5G6 done
   uint64_t* dneS = bars + 8;      // G1 done
-  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  uint64_t* loadedQK = bars + 16;   // [NB]: that set's q, k rows have landed
+  uint64_t* loadedV = bars + 22;    // [NB]: that set's v rows have landed
   uint64_t* rdyKV = bars + 19;    // [NB]: output warps -> G7 of a state-only item (k, v converted)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);   // G4 groups seen done
@@ -1220,13 +1235,19 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
       wa.seek(sc.gA, a.nch, a.nvb, a.H);
       for (int i = 0; ok && i < sc.nA; ++i, wa.step(a.nch, a.nvb, a.H)) {
         const int b = i % NB;
-        const bool r = mbar_wait_or_abort(loaded + b, static_cast<uint32_t>((i / NB) & 1), a.err, abort_flag);
+        const uint32_t par = static_cast<uint32_t>((i / NB) & 1);
+        const int nv = min(C, a.N - wa.ch * C);
+        bool r = mbar_wait_or_abort(loadedQK + b, par, a.err, abort_flag);
         if (named_sync_or(3, GT, !r)) {
           ok = false;
           break;
         }
-        const int nv = min(C, a.N - wa.ch * C);
         convert_tile<true, K::TQ / 16, GT>(smem + sK(b), nv, tid - GT, a.kv_ready);
+        r = mbar_wait_or_abort(loadedV + b, par, a.err, abort_flag);
+        if (named_sync_or(3, GT, !r)) {
+          ok = false;
+          break;
+        }
         convert_tile<false, K::TV / 16, GT>(smem + sV(b), nv, tid - GT, a.kv_ready);
         fence_async_smem();
         mbar_arrive(rdyKV + b);
@@ -1318,7 +1339,8 @@ __device__ __noinline__ void tc_role_fetch(const TcArgs& a, uint8_t* smem, int h
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
   uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
   uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
-  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  uint64_t* loadedQK = bars + 16;   // [NB]: that set's q, k rows have landed
+  uint64_t* loadedV = bars + 22;    // [NB]: that set's v rows have landed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   const uint32_t sbase = smem_u32(smem);
   auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
@@ -1328,31 +1350,38 @@ __device__ __noinline__ void tc_role_fetch(const TcArgs& a, uint8_t* smem, int h
   auto first_item = [&](Walker& w) { w.seek(sc.nA > 0 ? sc.gA : sc.g0, a.nch, a.nvb, a.H); };
     // ------------------------------------------------ fetch warp
     if (lane == 0) {
-      int issued = 0;
+      int issued_qk = 0, issued_v = 0;
       Walker w;
       first_item(w);
+      // q, k of an item go as soon as the contractions reading that set's q,
+      // k are done (G2+G3 of the item that last held it); v waits for G5+G6
       for (int i = 0, b = 0; i < nI; ++i, w.next(sc, i - 1, a.nch, a.nvb, a.H), b = b + 1 == NB ? 0 : b + 1) {
         const bool so = sc.state_only(i);
-        if (i >= NB) {   // set b last held item i - NB: wait until its contractions are done
-          const uint32_t par = static_cast<uint32_t>((i / NB - 1) & 1);   // that item's release phase
-          bool ok = mbar_wait_or_abort(freeQK + b, par, a.err, abort_flag);
-          if (ok) ok = mbar_wait_or_abort(freeVR + b, par, a.err, abort_flag);
-          if (!ok) break;
-        }
+        const uint32_t par = static_cast<uint32_t>((i / NB - 1) & 1);   // release phase of the set's last item
         const int y = w.ch * C, z = w.bh;
-        mbar_arrive_expect_tx(loaded + b, (so ? 1 : 2) * K::TQ + K::TV);
+        if (i >= NB && !mbar_wait_or_abort(freeQK + b, par, a.err, abort_flag)) break;
+        mbar_arrive_expect_tx(loadedQK + b, (so ? 1 : 2) * K::TQ);
         for (int x = 0; x < DX / 64; ++x) {
-          if (!so) tma_load_3d(sbase + sQ(b) + x * K::BOX, &tm_q, 64 * x, y, z, loaded + b);
-          tma_load_3d(sbase + sK(b) + x * K::BOX, &tm_k, 64 * x, y, z, loaded + b);
+          if (!so) tma_load_3d(sbase + sQ(b) + x * K::BOX, &tm_q, 64 * x, y, z, loadedQK + b);
+          tma_load_3d(sbase + sK(b) + x * K::BOX, &tm_k, 64 * x, y, z, loadedQK + b);
         }
-        tma_load_3d(sbase + sV(b), &tm_v, w.vb * kVB, y, z, loaded + b);
-        issued = i + 1;
+        issued_qk = i + 1;
+        if (i >= NB && !mbar_wait_or_abort(freeVR + b, par, a.err, abort_flag)) break;
+        mbar_arrive_expect_tx(loadedV + b, K::TV);
+        tma_load_3d(sbase + sV(b), &tm_v, w.vb * kVB, y, z, loadedV + b);
+        issued_v = i + 1;
       }
       // no copy of ours lands after the block exits: the last load into each
-      // set b was item i_b, the phase (i_b / NB) of loaded[b]
-      for (int b = 0; b < NB && b < issued; ++b) {
-        const int i_b = b + (issued - 1 - b) / NB * NB;
-        mbar_wait(loaded + b, static_cast<uint32_t>((i_b / NB) & 1), a.err);
+      // set b was item i_b, the phase (i_b / NB) of its barrier
+      for (int b = 0; b < NB; ++b) {
+        if (b < issued_qk) {
+          const int i_b = b + (issued_qk - 1 - b) / NB * NB;
+          mbar_wait(loadedQK + b, static_cast<uint32_t>((i_b / NB) & 1), a.err);
+        }
+        if (b < issued_v) {
+          const int i_b = b + (issued_v - 1 - b) / NB * NB;
+          mbar_wait(loadedV + b, static_cast<uint32_t>((i_b / NB) & 1), a.err);
+        }
       }
     }
     __syncwarp();
@@ -1381,12 +1410,13 @@ __global__ void __launch_bounds__(NTH, 1)
   uint64_t* freeQK = bars + 9;    // [NB]: sQ, sK of that set reusable
   uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
   uint64_t* bar_drain = bars + 15;
-  uint64_t* loaded = bars + 16;   // [NB]: that set's q, k, v rows have landed
+  uint64_t* loadedQK = bars + 16;   // [NB]: that set's q, k rows have landed
+  uint64_t* loadedV = bars + 22;    // [NB]: that set's v rows have landed
   // [NB]: output warps -> G7 of a state-only item, that set's k and v are
   // fp16 operands.  A set is refilled only after that G7, so no barrier runs
   // a phase ahead of the MMA warp's wait.
   uint64_t* rdyKV = bars + 19;
-  static_assert(NB <= 3 && (19 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
+  static_assert(NB <= 3 && (22 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
   // G4 groups known done: the output warps see each G4 complete, in order,
@@ -1414,7 +1444,8 @@ __global__ void __launch_bounds__(NTH, 1)
     for (int i = 0; i < NB; ++i) {
       mbar_init(freeQK + i, 1);
       mbar_init(freeVR + i, 1);
-      mbar_init(loaded + i, 1);
+      mbar_init(loadedQK + i, 1);
+      mbar_init(loadedV + i, 1);
     }
     mbar_init(bar_drain, 1);
     for (int i = 0; i < NB; ++i) mbar_init(rdyKV + i, GT);
