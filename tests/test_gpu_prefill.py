@@ -149,6 +149,29 @@ def test_chunk_pass_ranges(oracle_mod, dev, monkeypatch, dx, dv, grid):
     check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, dx, dv), B, H, M, dx, dv, TOL_BF16)
 
 
+@pytest.mark.parametrize("grid", [20, 37])
+def test_look_back_across_many_predecessors(oracle_mod, dev, monkeypatch, grid):
+    # One stream of 40 chunks (the last one ragged) over 20 or 37 CTAs: a
+    # range's carry sums the published states of up to 36 predecessors, more
+    # than the eight awaited per round, so the look-back takes several rounds
+    # (and single-piece CTAs publish inclusive states that cut later ones
+    # short), from a nonzero state_in.
+    B, H, M, dx, dv = 1, 1, 64, 64, 64
+    N0, N = 50, 64 * 39 + 23
+    inp = synthetic.layer_inputs(B, H, N0 + N, dx, dv, "bf16", seed=400 + grid)
+    head = {k: (v[:, :, :N0].contiguous() if k != "delta" else v) for k, v in inp.items()}
+    st = gpu_prefill(head, M, dev)["state"].to(dev)
+    tail = {k: (v[:, :, N0:].contiguous() if k != "delta" else v) for k, v in inp.items()}
+    monkeypatch.setenv("IA_PREFILL_GRID", str(grid))
+    assert ia.prefill_grid(B, H, N, dx, dv, M, "bf16") == grid
+    r = gpu_prefill(tail, M, dev, state_in=st)
+    ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], inp["delta"], M)
+    ref_tail = {"num": ref["num"][:, :, N0:], "den": ref["den"][:, :, N0:], "o": ref["o"][:, :, N0:]}
+    rep = report(r["num"], r["den"], r["o"], ref_tail)
+    assert max(rep.values()) < TOL_BF16, rep
+    check_state(r["state"], oracle_mod.split_state(ref["state"], B, H, M, dx, dv), B, H, M, dx, dv, TOL_BF16)
+
+
 def test_first_token_returns_v(dev):
     # P3 on the GPU path: o_1 = v_1 whatever q_1 and k_1
     inp = synthetic.layer_inputs(3, 4, 70, 64, 64, "bf16", seed=3)
