@@ -52,6 +52,25 @@ def test_prefill_per_mode_delta_and_A(oracle_mod, dev, dtype, dx, dv, M, tol):
     assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < tol
 
 
+@pytest.mark.parametrize("dx,grid", [(64, 14), (128, 25)])
+def test_look_back_with_per_mode_delta_and_A(oracle_mod, dev, monkeypatch, dx, grid):
+    # ranges that start inside a stream compose their carry with
+    # lambda_m^(C d) from each mode's own Delta and A
+    B, H, M, N = 1, 2, 64, 64 * 20 + 17
+    inp = synthetic.layer_inputs(B, H, N, dx, dx, "bf16", seed=90 + dx)
+    delta, A = modes_params(H, M, 91)
+    monkeypatch.setenv("IA_PREFILL_GRID", str(grid))
+    assert ia.prefill_grid(B, H, N, dx, dx, M, "bf16") == grid
+    r = ia.prefill_fwd(inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev), delta.to(dev), M, A=A.to(dev),
+                       want_num_den=True, want_state=True)
+    ia.check_device_errors()
+    ref = oracle_mod.forward(inp["q"], inp["k"], inp["v"], delta, M, A=A)
+    rep = report(r["num"].cpu(), r["den"].cpu(), r["o"].cpu(), ref)
+    assert max(rep.values()) < TOL_BF16, rep
+    st = r["state"].cpu().double().numpy()
+    assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < TOL_BF16
+
+
 def test_decode_per_mode_delta_and_A(oracle_mod, dev):
     B, H, d, M = 4, 3, 128, 64
     pre = synthetic.layer_inputs(B, H, 70, d, d, "bf16", seed=62)
