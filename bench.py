@@ -559,8 +559,10 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
 def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world):
     """The layer's optional parts (RMSNorm on the SSM input, a step per token,
     the complex readout matrix, the bidirectional layer) through
-    ia_prefill_fwd_ex on the same workload: the token-serial CUDA-core kernel,
-    one CTA per (b,h).  Each part is timed alone and all together."""
+    ia_prefill_fwd_ex on the same workload: the tensor-core chunk pass where
+    the parts allow it, else the token-serial CUDA-core kernel over segments
+    of each sequence in two passes around a carry.  Each part is timed alone
+    and some together."""
     import torch
     import ssm_token_mixer_b200 as ia
     from ssm_token_mixer_b200 import synthetic
@@ -601,11 +603,14 @@ def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, wor
         passes = 2 if kw.get("bidirectional") else 1
         rf = roofline(by * passes, flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H * passes, kern_ms, peaks,
                       peak_kind, None, sustained=False)
-        # tensor cores: the prologue, a table kernel and a chunk pass per direction, the epilogue
+        # tensor cores: the prologue, a table kernel and a chunk pass per direction, the epilogue;
+        # token-serial: one pass per direction, or pass 1, the carry (past two segments) and pass 2
+        nseg = ia.prefill_ex_segments(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16", need, **present)
         launches = ((1 if present["norm"] or present["bidirectional"] else 0) + passes * 2 +
-                    (1 if present["bidirectional"] else 0)) if path == "tensor_core" else passes
+                    (1 if present["bidirectional"] else 0)) if path == "tensor_core" else \
+            passes * (1 if nseg == 1 else 2 if nseg == 2 else 3)
         out["parts"][name] = {"value": world * tokens * steps / (total * 1e-3), "ms_per_step": total / steps,
-                              "path": path, "roofline": rf, "gpu_launches": launches * steps}
+                              "path": path, "segments": nseg, "roofline": rf, "gpu_launches": launches * steps}
     return out
 
 

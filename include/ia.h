@@ -262,16 +262,37 @@ typedef struct {
  *     bidirectional layer, whose second output an epilogue kernel adds back
  *     in forward order.  z is rounded to fp16 once more than in the
  *     token-serial form.  Needs ia_prefill_ex_workspace_bytes of workspace.
- *   - everything else runs the token-serial fp32 CUDA-core kernel (one CTA
- *     per (b,h), any input dtype), correct for every shape whose state fits
- *     in shared memory but much slower; it needs no workspace (workspace may
- *     be NULL).
- * workspace: device scratch of at least ia_prefill_ex_workspace_bytes bytes
- * for the tensor-core form, any alignment; too small gives IA_ERR_WORKSPACE
+ *   - everything else runs the token-serial fp32 CUDA-core kernel (any
+ *     input dtype), correct for every shape whose state fits in shared memory
+ *     but much slower.  With ia_prefill_ex_workspace_bytes of workspace it
+ *     cuts each sequence into segments of at least 64 tokens, one CTA each,
+ *     enough to fill the GPU's resident CTA slots: a first pass runs every
+ *     segment but the last from a zero state (the first from state_in) for
+ *     its end state, a carry kernel composes those into the state entering
+ *     each segment (the decay over a segment is exp(A times its summed
+ *     steps)), and a second pass runs every segment from its entering state
+ *     with the readout (paper summary sec. A.2: parallel passes over pieces
+ *     of the sequence, the state passed between them).  A smaller workspace,
+ *     or NULL, gives fewer segments, down to one CTA per (b,h) token after
+ *     token; results differ from one segment count to another only by fp32
+ *     rounding.
+ * workspace: device scratch of at least ia_prefill_ex_workspace_bytes bytes,
+ * any alignment; for the tensor-core form too small gives IA_ERR_WORKSPACE
  * before anything is launched.
  */
 IA_API size_t ia_prefill_ex_workspace_bytes(const ia_shape_t* shape, const ia_options_t* opt);
 IA_API int ia_prefill_ex_path(const ia_shape_t* shape, const ia_options_t* opt);
+/*
+ * Segments per sequence that ia_prefill_fwd_ex runs with this workspace
+ * (pointer and size as the call would get them; only the pointer's being
+ * non-NULL matters): 1 for the tensor-core form and for a single token-serial
+ * pass, else the count of the two-pass form, whose call then launches pass 1,
+ * the carry kernel (when more than two segments) and pass 2 per direction.
+ * 0 for an invalid shape or options.  Asks the device for the kernel's
+ * resident CTAs per SM (1 when no device answers).
+ */
+IA_API int ia_prefill_ex_segments(const ia_shape_t* shape, const ia_options_t* opt, const void* workspace,
+                                  size_t workspace_bytes);
 IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* shape, const ia_options_t* opt, const void* q,
                                      const void* k, const void* v, const float* delta, const float* A,
                                      const void* state_in, float* o, float* num, float* den,

@@ -93,6 +93,8 @@ def load_library():
     lib.ia_prefill_ex_workspace_bytes.argtypes = [S, O]
     lib.ia_prefill_ex_path.restype = ctypes.c_int
     lib.ia_prefill_ex_path.argtypes = [S, O]
+    lib.ia_prefill_ex_segments.restype = ctypes.c_int
+    lib.ia_prefill_ex_segments.argtypes = [S, O, P, ctypes.c_size_t]
     lib.ia_decode_step_ex.restype = ctypes.c_int
     lib.ia_decode_step_ex.argtypes = [S, O] + [P] * 9 + [P]
     lib.ia_state_carry.restype = ctypes.c_int
@@ -216,6 +218,18 @@ def prefill_ex_path(B, H, N, d_xi, d_v, M, dtype, norm=False, selective=False, r
     opt = _presence_options(norm, selective, readout, bidirectional)
     shp = make_shape(B, H, N, d_xi, d_v, M, dtype)
     return PATHS[load_library().ia_prefill_ex_path(ctypes.byref(shp), ctypes.byref(opt))]
+
+
+def prefill_ex_segments(B, H, N, d_xi, d_v, M, dtype, workspace_bytes, norm=False, selective=False,
+                        readout=False, bidirectional=False) -> int:
+    """Segments per sequence ia_prefill_fwd_ex runs with a workspace of that
+    many bytes (0 bytes: none given): 1 for the tensor-core form and a single
+    token-serial pass."""
+    opt = _presence_options(norm, selective, readout, bidirectional)
+    shp = make_shape(B, H, N, d_xi, d_v, M, dtype)
+    ws = ctypes.c_void_p(16) if workspace_bytes else None   # only the pointer's presence counts
+    return int(load_library().ia_prefill_ex_segments(ctypes.byref(shp), ctypes.byref(opt), ws,
+                                                     ctypes.c_size_t(workspace_bytes)))
 
 
 def prefill_ex_workspace_bytes(B, H, N, d_xi, d_v, M, dtype, norm=False, selective=False, readout=False,

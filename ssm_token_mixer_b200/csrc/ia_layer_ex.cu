@@ -15,6 +15,7 @@
 //     bidirectional handling): o = f(x) + flip(f(flip x)), the second term a
 //     second launch that reads and writes the sequence back to front and adds
 //     its output to the first.
+#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -27,10 +28,12 @@ namespace ia {
 namespace {
 
 // shared (float2): U [M*DX] | G [M*DV] | eta [M] | lam [M] | b [M] | a [M] | a~ [M]
-// then floats: fq [DX] | z [DX + DV] | red [32]
+// then floats: fq [DX] | z [DX + DV] | red [32]; then, when it fits, the
+// head's readout matrix W_h [M*M] (float2)
 size_t ex_smem(int DX, int DV, int M) {
   return sizeof(float2) * (static_cast<size_t>(M) * (DX + DV) + 5 * M) + sizeof(float) * (2 * DX + DV + 32) + 16;
 }
+size_t ex_smem_w(int M) { return sizeof(float2) * static_cast<size_t>(M) * M; }
 
 struct ExArgs {
   const float* delta;     // [H] or [H,M] (unused with delta_t)
@@ -48,10 +51,21 @@ struct ExArgs {
   float* den;
   int reverse;            // read and write tokens back to front
   int accumulate;         // add o to what is there instead of overwriting it
+  int w_smem;             // W_h is staged in shared memory
+  // The sequence may be cut into nseg segments of seg_len steps, one CTA
+  // each, in two passes around a carry composition (the summary's sec. A.2):
+  // pass 1 runs segments 0 .. nseg-2 for their end states only (segment 0
+  // from state_in, the others from zero) into seg, and the step sums of
+  // delta into dsum; ex_carry_kernel turns slot s of seg into the state
+  // entering segment s+1; pass 2 (or the single pass, nseg = 1) runs every
+  // segment from its entering state with the readout.
+  int nseg, seg_len, pass;
+  float2* seg;            // [BH][nseg-1][M (DX + DV + 1)]
+  double* dsum;           // [BH][nseg]: sum of delta_t over the segment's tokens
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256) seq_fwd_ex_kernel(int H, int N, int DX, int DV, int M, const T* __restrict__ q,
+__global__ void __launch_bounds__(256, 3) seq_fwd_ex_kernel(int H, int N, int DX, int DV, int M, const T* __restrict__ q,
                                                          const T* __restrict__ k, const T* __restrict__ v,
                                                          const ExArgs a, long long BH) {
   extern __shared__ float4 smem_f4[];
@@ -65,10 +79,18 @@ __global__ void __launch_bounds__(256) seq_fwd_ex_kernel(int H, int N, int DX, i
   float* fq = reinterpret_cast<float*>(at + M);
   float* z = fq + DX;            // [DX + DV]: xi(k) then v, normalised when asked
   float* red = z + DX + DV;      // [32]
+  // W_h after the floats, on a 16-byte boundary
+  float2* Ws = reinterpret_cast<float2*>((reinterpret_cast<uintptr_t>(red + 32) + 15) & ~static_cast<uintptr_t>(15));
 
-  const long long bh = blockIdx.x;
+  const long long bh = blockIdx.x / a.nseg;
+  const int sg = static_cast<int>(blockIdx.x - bh * a.nseg);
   const int h = static_cast<int>(bh % H);
   const int tid = threadIdx.x, nthr = blockDim.x;
+  const int step0 = sg * a.seg_len, step1 = min(N, step0 + a.seg_len);
+  const bool readout = a.pass != 1;
+  if (!readout && sg == a.nseg - 1) return;   // pass 1: the last segment's end state is not needed
+  const int SW = M * (DX + DV + 1);   // complex entries of one (b,h) state
+  float2* slot_in = sg > 0 ? a.seg + (bh * (a.nseg - 1) + (sg - 1)) * SW : nullptr;
   const int warp = tid >> 5, lane = tid & 31, nwarp = nthr >> 5;
   const int D = DX + DV;
   const bool norm = a.gain || a.bias;
@@ -81,28 +103,93 @@ __global__ void __launch_bounds__(256) seq_fwd_ex_kernel(int H, int N, int DX, i
     }
   }
   const long long u0 = bh * M * DX, g0 = BH * M * DX + bh * M * DV, e0 = BH * M * (DX + DV) + bh * M;
-  for (int i = tid; i < M * DX; i += nthr) U[i] = a.state_in ? a.state_in[u0 + i] : make_float2(0.f, 0.f);
-  for (int i = tid; i < M * DV; i += nthr) G[i] = a.state_in ? a.state_in[g0 + i] : make_float2(0.f, 0.f);
-  for (int i = tid; i < M; i += nthr) eta[i] = a.state_in ? a.state_in[e0 + i] : make_float2(0.f, 0.f);
+  if (sg == 0) {   // the caller's state (public layout), or zero
+    for (int i = tid; i < M * DX; i += nthr) U[i] = a.state_in ? a.state_in[u0 + i] : make_float2(0.f, 0.f);
+    for (int i = tid; i < M * DV; i += nthr) G[i] = a.state_in ? a.state_in[g0 + i] : make_float2(0.f, 0.f);
+    for (int i = tid; i < M; i += nthr) eta[i] = a.state_in ? a.state_in[e0 + i] : make_float2(0.f, 0.f);
+  } else {         // pass 2: the composed carry; pass 1: zero
+    for (int i = tid; i < SW; i += nthr) U[i] = readout ? slot_in[i] : make_float2(0.f, 0.f);
+  }
+  if (a.W && a.w_smem && readout) {
+    const float2* Wg = reinterpret_cast<const float2*>(a.W) + static_cast<long long>(h) * M * M;
+    for (int i = tid; i < M * M; i += nthr) Ws[i] = Wg[i];
+  }
   __syncthreads();
 
   const T* qb = q + bh * N * DX;
   const T* kb = k + bh * N * DX;
   const T* vb = v + bh * N * DV;
-  for (int step = 0; step < N; ++step) {
+  // A step per token: this thread's mode's A (tid < M), and lambda_t, b_t in
+  // fp32 in the decode step's form (lambda - 1 = expm1(x) cos(y) - 2 sin^2(y/2)
+  // + i e^x sin(y), so that b keeps its relative accuracy at small Delta_t).
+  float m_ar = -0.5f, m_ai = 0.f;
+  if (a.delta_t && tid < M) {
+    m_ar = a.A ? a.A[2 * tid] : -0.5f;
+    m_ai = a.A ? a.A[2 * tid + 1] : 3.14159265358979323846f * static_cast<float>(tid);
+  }
+  auto step_params = [&](float dt) {
+    const float x = dt * m_ar, y = dt * m_ai;
+    float sy, cy, sh, ch;
+    sincosf(y, &sy, &cy);
+    sincosf(0.5f * y, &sh, &ch);
+    const float ex = expf(x), em1 = expm1f(x);
+    const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;
+    const float dd = fmaf(m_ar, m_ar, m_ai * m_ai);
+    lam[tid] = make_float2(ex * cy, ex * sy);
+    bb[tid] = make_float2(fmaf(nr, m_ar, ni * m_ai) / dd, fmaf(ni, m_ar, -nr * m_ai) / dd);
+  };
+  // The next token's inputs are loaded while this one is processed: each
+  // thread holds entries f = tid and tid + 256 of k|v and of q.
+  constexpr int kPre = 2;
+  const bool pre = D <= kPre * nthr && DX <= kPre * nthr;
+  float rz[kPre] = {0.f, 0.f}, rq[kPre] = {0.f, 0.f}, rdt = 0.f;
+  auto fetch = [&](int tt) {
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+      const int f = tid + i * nthr;
+      if (f < DX) {
+        rz[i] = ldf(kb + static_cast<long long>(tt) * DX + f);
+        rq[i] = ldf(qb + static_cast<long long>(tt) * DX + f);
+      } else if (f < D) {
+        rz[i] = ldf(vb + static_cast<long long>(tt) * DV + (f - DX));
+      }
+    }
+    if (a.delta_t && tid < M) rdt = a.delta_t[bh * N + tt];
+  };
+  double dt_sum = 0.0;   // pass 1, thread 0: the segment's sum of delta_t
+  if (pre && step1 > step0) fetch(a.reverse ? N - 1 - step0 : step0);
+  for (int step = step0; step < step1; ++step) {
     const int t = a.reverse ? N - 1 - step : step;
     // the SSM input z = (xi(k_t), v_t) and the query features
     float ss = 0.f;
-    for (int f = tid; f < D; f += nthr) {
-      const float x = f < DX ? feat_acc(ldf(kb + static_cast<long long>(t) * DX + f))
-                             : ldf(vb + static_cast<long long>(t) * DV + (f - DX));
-      z[f] = x;
-      ss = fmaf(x, x, ss);
+    if (pre) {
+#pragma unroll
+      for (int i = 0; i < kPre; ++i) {
+        const int f = tid + i * nthr;
+        if (f < D) {
+          const float x = f < DX ? feat_acc(rz[i]) : rz[i];
+          z[f] = x;
+          ss = fmaf(x, x, ss);
+        }
+        if (f < DX) fq[f] = feat_acc(rq[i]);
+      }
+      if (a.delta_t && tid < M) step_params(rdt);
+      if (a.delta_t && tid == 0) dt_sum += rdt;
+      if (step + 1 < step1) fetch(a.reverse ? N - 2 - step : step + 1);
+    } else {
+      for (int f = tid; f < D; f += nthr) {
+        const float x = f < DX ? feat_acc(ldf(kb + static_cast<long long>(t) * DX + f))
+                               : ldf(vb + static_cast<long long>(t) * DV + (f - DX));
+        z[f] = x;
+        ss = fmaf(x, x, ss);
+      }
+      for (int f = tid; f < DX; f += nthr) fq[f] = feat_acc(ldf(qb + static_cast<long long>(t) * DX + f));
+      if (a.delta_t && tid < M) step_params(a.delta_t[bh * N + t]);
+      if (a.delta_t && tid == 0) dt_sum += a.delta_t[bh * N + t];
     }
-    for (int f = tid; f < DX; f += nthr) fq[f] = feat_acc(ldf(qb + static_cast<long long>(t) * DX + f));
-    if (a.delta_t) {   // this token's step for every mode
+    if (a.delta_t && M > nthr) {   // modes past the block's threads
       const float dt = a.delta_t[bh * N + t];
-      for (int m = tid; m < M; m += nthr) {
+      for (int m = tid + nthr; m < M; m += nthr) {
         const ModeD md = mode_consts(dt, a.A, m);
         lam[m] = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
         bb[m] = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
@@ -122,72 +209,211 @@ __global__ void __launch_bounds__(256) seq_fwd_ex_kernel(int H, int N, int DX, i
       }
     }
     __syncthreads();
-    for (int m = warp; m < M; m += nwarp) {
-      const float2 L = lam[m], Bm = bb[m];
-      float ar = 0.f, ai = 0.f;
-      for (int f = lane; f < DX; f += 32) {
-        const float2 u = cfma(L, U[m * DX + f], make_float2(Bm.x * z[f], Bm.y * z[f]));
-        U[m * DX + f] = u;
-        ar = fmaf(u.x, fq[f], ar);
-        ai = fmaf(u.y, fq[f], ai);
+    // state update and a = U xi(q): four modes per warp at a time, their
+    // eight warp sums reduced together
+    constexpr int MB = 4;
+    for (int mb = warp * MB; mb < M; mb += nwarp * MB) {
+      float pr[MB], pi[MB];
+      float2 L[MB], Bm[MB];
+#pragma unroll
+      for (int u = 0; u < MB; ++u) {
+        pr[u] = pi[u] = 0.f;
+        const int m = min(mb + u, M - 1);   // a mode past M repeats the last one and is not stored
+        L[u] = lam[m];
+        Bm[u] = bb[m];
       }
-      for (int f = lane; f < DV; f += 32)
-        G[m * DV + f] = cfma(L, G[m * DV + f], make_float2(Bm.x * z[DX + f], Bm.y * z[DX + f]));
-      ar = warp_sum(ar);
-      ai = warp_sum(ai);
+      const int nu = min(MB, M - mb);
+      // each column's z and xi(q) are read once for the warp's modes
+      for (int f = lane; f < DX; f += 32) {
+        const float zf = z[f], qf = fq[f];
+#pragma unroll
+        for (int u = 0; u < MB; ++u) {
+          if (u >= nu) break;
+          float2* up = U + (mb + u) * DX + f;
+          const float2 uu = cfma(L[u], *up, make_float2(Bm[u].x * zf, Bm[u].y * zf));
+          *up = uu;
+          if (readout) {
+            pr[u] = fmaf(uu.x, qf, pr[u]);
+            pi[u] = fmaf(uu.y, qf, pi[u]);
+          }
+        }
+      }
+      for (int f = lane; f < DV; f += 32) {
+        const float zv = z[DX + f];
+#pragma unroll
+        for (int u = 0; u < MB; ++u) {
+          if (u >= nu) break;
+          float2* gp = G + (mb + u) * DV + f;
+          *gp = cfma(L[u], *gp, make_float2(Bm[u].x * zv, Bm[u].y * zv));
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+        for (int u = 0; u < MB; ++u) {
+          pr[u] += __shfl_xor_sync(0xffffffffu, pr[u], off);
+          pi[u] += __shfl_xor_sync(0xffffffffu, pi[u], off);
+        }
+      }
       if (lane == 0) {
-        av[m] = make_float2(ar, ai);
-        eta[m] = cfma(L, eta[m], Bm);
+#pragma unroll
+        for (int u = 0; u < MB; ++u) {
+          const int m = mb + u;
+          if (m < M) {
+            av[m] = make_float2(pr[u], pi[u]);
+            eta[m] = cfma(L[u], eta[m], Bm[u]);
+          }
+        }
       }
     }
     __syncthreads();
-    // readout matrix: a~ = W_h a (row m of W dotted with a, one warp per row)
+    if (!readout) continue;   // pass 1: the state only (uniform over the block)
+    // readout matrix: a~ = W_h a (row m of W dotted with a), four rows per
+    // warp at a time
     if (a.W) {
-      const float2* Wh = reinterpret_cast<const float2*>(a.W) + static_cast<long long>(h) * M * M;
-      for (int m = warp; m < M; m += nwarp) {
-        float sr = 0.f, si = 0.f;
-        for (int mp = lane; mp < M; mp += 32) {
-          const float2 w = Wh[static_cast<long long>(m) * M + mp], x = av[mp];
-          sr = fmaf(w.x, x.x, fmaf(-w.y, x.y, sr));
-          si = fmaf(w.x, x.y, fmaf(w.y, x.x, si));
+      const float2* Wh = a.w_smem ? Ws : reinterpret_cast<const float2*>(a.W) + static_cast<long long>(h) * M * M;
+      for (int mb = warp * MB; mb < M; mb += nwarp * MB) {
+        float sr[MB], si[MB];
+#pragma unroll
+        for (int u = 0; u < MB; ++u) {
+          sr[u] = si[u] = 0.f;
+          const int m = mb + u;
+          if (m >= M) continue;
+          for (int mp = lane; mp < M; mp += 32) {
+            const float2 w = Wh[static_cast<long long>(m) * M + mp], x = av[mp];
+            sr[u] = fmaf(w.x, x.x, fmaf(-w.y, x.y, sr[u]));
+            si[u] = fmaf(w.x, x.y, fmaf(w.y, x.x, si[u]));
+          }
         }
-        sr = warp_sum(sr);
-        si = warp_sum(si);
-        if (lane == 0) at[m] = make_float2(sr, si);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+          for (int u = 0; u < MB; ++u) {
+            sr[u] += __shfl_xor_sync(0xffffffffu, sr[u], off);
+            si[u] += __shfl_xor_sync(0xffffffffu, si[u], off);
+          }
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int u = 0; u < MB; ++u)
+            if (mb + u < M) at[mb + u] = make_float2(sr[u], si[u]);
+        }
       }
       __syncthreads();
     }
+    // num and den: P threads per value column, each summing every P-th mode
+    // (four interleaved partial sums), then a shuffle sum over the P lanes
     const float2* rd = a.W ? at : av;
-    float dn = 0.f;
-    for (int m = 0; m < M; ++m) dn += re_conj_mul(rd[m], eta[m]);
+    int P = 1;
+    while (P < 8 && 2 * P * DV <= nthr) P *= 2;
+    const int part = tid % P, S = nthr / P;
     const long long row = bh * N + t;
-    for (int f = tid; f < DV; f += nthr) {
-      float nf = 0.f;
-      for (int m = 0; m < M; ++m) nf += re_conj_mul(rd[m], G[m * DV + f]);
-      const float of = nf / dn;
-      a.o[row * DV + f] = a.accumulate ? a.o[row * DV + f] + of : of;
-      if (a.num) a.num[row * DV + f] = nf;
+    const int rounds = (DV + S - 1) / S;   // the same for every thread: the shuffles below see whole warps
+    for (int rr = 0; rr < rounds; ++rr) {
+      const int f0 = rr * S + tid / P;
+      const int f = f0 < DV ? f0 : DV - 1;
+      float n0 = 0.f, n1 = 0.f, e0 = 0.f, e1 = 0.f;
+      int m = part;
+      for (; m + P < M; m += 2 * P) {
+        n0 += re_conj_mul(rd[m], G[m * DV + f]);
+        e0 += re_conj_mul(rd[m], eta[m]);
+        n1 += re_conj_mul(rd[m + P], G[(m + P) * DV + f]);
+        e1 += re_conj_mul(rd[m + P], eta[m + P]);
+      }
+      if (m < M) {
+        n0 += re_conj_mul(rd[m], G[m * DV + f]);
+        e0 += re_conj_mul(rd[m], eta[m]);
+      }
+      float nf = n0 + n1, dn = e0 + e1;
+      for (int off = 1; off < P; off <<= 1) {
+        nf += __shfl_xor_sync(0xffffffffu, nf, off);
+        dn += __shfl_xor_sync(0xffffffffu, dn, off);
+      }
+      if (part == 0 && f0 < DV) {
+        const float of = nf / dn;
+        a.o[row * DV + f] = a.accumulate ? a.o[row * DV + f] + of : of;
+        if (a.num) a.num[row * DV + f] = nf;
+        if (a.den && f == 0) a.den[row] = dn;
+      }
     }
-    if (a.den && tid == 0) a.den[row] = dn;
     __syncthreads();
   }
-  if (a.state_out) {
+  if (!readout) {   // pass 1: this segment's end state into its slot
+    float2* slot = a.seg + (bh * (a.nseg - 1) + sg) * SW;
+    for (int i = tid; i < SW; i += nthr) slot[i] = U[i];
+    if (tid == 0 && a.dsum) a.dsum[bh * a.nseg + sg] = dt_sum;
+  } else if (a.state_out && sg == a.nseg - 1) {
     for (int i = tid; i < M * DX; i += nthr) a.state_out[u0 + i] = U[i];
     for (int i = tid; i < M * DV; i += nthr) a.state_out[g0 + i] = G[i];
     for (int i = tid; i < M; i += nthr) a.state_out[e0 + i] = eta[i];
   }
 }
 
+// Turns the pass-1 end states into the states entering each segment, per
+// (b,h) and mode: slot 0 already is the state entering segment 1 (segment 0
+// started from state_in); slot s (s >= 1) becomes Lambda_s slot(s-1) +
+// slot s, Lambda_s the decay over segment s, exp(A_m D_s) with D_s its sum of
+// steps (delta_t summed in pass 1, or Delta_hm times its length), in fp64.
+__global__ void __launch_bounds__(128) ex_carry_kernel(int H, int N, int DX, int DV, int M, const float* delta,
+                                                       int dpm, const float* A, const double* dsum, int nseg,
+                                                       int seg_len, float2* seg) {
+  extern __shared__ double2 lamS[];   // [nseg]
+  const long long bh = blockIdx.x / M;
+  const int m = static_cast<int>(blockIdx.x - bh * M);
+  const int h = static_cast<int>(bh % H);
+  const double ar = A ? A[2 * m] : -0.5;
+  const double ai = A ? A[2 * m + 1] : 3.14159265358979323846 * m;
+  for (int sgi = threadIdx.x + 1; sgi < nseg - 1; sgi += blockDim.x) {
+    const int len = min(N, (sgi + 1) * seg_len) - sgi * seg_len;
+    const double D = dsum ? dsum[bh * nseg + sgi] : static_cast<double>(delta_hm(delta, dpm, M, h, m)) * len;
+    const double e = exp(D * ar);
+    double sn, cs;
+    sincos(fmod(D * ai, 6.283185307179586476925), &sn, &cs);
+    lamS[sgi] = make_double2(e * cs, e * sn);
+  }
+  __syncthreads();
+  const int SW = M * (DX + DV + 1);
+  float2* base = seg + bh * (nseg - 1) * SW;
+  auto walk = [&](int e) {   // one state entry through the segments
+    double cr = base[e].x, ci = base[e].y;
+    for (int sgi = 1; sgi < nseg - 1; ++sgi) {
+      const double2 L = lamS[sgi];
+      const float2 loc = base[sgi * SW + e];
+      const double nr = L.x * cr - L.y * ci + loc.x;
+      ci = L.x * ci + L.y * cr + loc.y;
+      cr = nr;
+      base[sgi * SW + e] = make_float2(static_cast<float>(cr), static_cast<float>(ci));
+    }
+  };
+  for (int f = threadIdx.x; f < DX; f += blockDim.x) walk(m * DX + f);
+  for (int f = threadIdx.x; f < DV; f += blockDim.x) walk(M * DX + m * DV + f);
+  if (threadIdx.x == 0) walk(M * (DX + DV) + m);
+}
+
+constexpr int kExThreads = 256;
+
+// dynamic shared memory of one launch: W_h is staged when it fits and the
+// launch reads out (pass 1 keeps the state only)
+size_t ex_launch_smem(const ia_shape_t& s, bool with_w, bool* w_smem) {
+  size_t smem = ex_smem(s.d_xi, s.d_v, s.M);
+  *w_smem = with_w && smem + 16 + ex_smem_w(s.M) <= 232448;
+  return *w_smem ? smem + 16 + ex_smem_w(s.M) : smem;
+}
+
 template <typename T>
 cudaError_t launch_ex(const ia_shape_t& s, int N, const void* q, const void* k, const void* v, const ExArgs& a,
                       cudaStream_t st) {
-  const size_t smem = ex_smem(s.d_xi, s.d_v, s.M);
+  ExArgs args = a;
+  bool ws = false;
+  const size_t smem = ex_launch_smem(s, a.W && a.pass != 1, &ws);
+  args.w_smem = ws ? 1 : 0;
   auto kern = seq_fwd_ex_kernel<T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long BH = static_cast<long long>(s.B) * s.H;
-  kern<<<static_cast<unsigned>(BH), 256, smem, st>>>(s.H, N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q),
-                                                     static_cast<const T*>(k), static_cast<const T*>(v), a, BH);
+  kern<<<static_cast<unsigned>(BH * args.nseg), kExThreads, smem, st>>>(
+      s.H, N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), args,
+      BH);
   return cudaGetLastError();
 }
 
@@ -197,12 +423,81 @@ cudaError_t launch_ex_any(const ia_shape_t& s, int N, const void* q, const void*
   return launch_ex<__nv_bfloat16>(s, N, q, k, v, a, st);
 }
 
+// CTAs of the reading-out launch resident per SM (1 when no device answers)
+int ex_resident(const ia_shape_t& s, bool with_w) {
+  bool ws = false;
+  const size_t smem = ex_launch_smem(s, with_w, &ws);
+  const void* fn = s.in_dtype == IA_F32 ? reinterpret_cast<const void*>(seq_fwd_ex_kernel<float>)
+                                        : reinterpret_cast<const void*>(seq_fwd_ex_kernel<__nv_bfloat16>);
+  int n = 0;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kExThreads, smem) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 1;
+  }
+  return n;
+}
+
+// Segments per sequence of the token-serial form: enough that the grid of
+// B H nseg CTAs fills the SMs' resident slots once, each segment at least
+// kMinSegment tokens, at most kMaxSegments (the carry walks them in turn).
+constexpr int kMinSegment = 64, kMaxSegments = 64;
+
+int ex_segments(const ia_shape_t& s, const ia_options_t* opt) {
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  const long long by_len = std::min<long long>(s.N / kMinSegment, kMaxSegments);
+  if (by_len < 2) return 1;
+  const long long slots = static_cast<long long>(num_sms()) * ex_resident(s, opt && opt->W);
+  return static_cast<int>(std::max<long long>(1, std::min(by_len, slots / BH)));
+}
+
+// workspace of nseg segments: the end-state slots, then the delta_t sums, with
+// 16 bytes of slack to align the caller's pointer
+size_t ex_seg_bytes(const ia_shape_t& s, const ia_options_t* opt, int nseg) {
+  if (nseg <= 1) return 0;
+  const size_t BH = static_cast<size_t>(s.B) * s.H;
+  const size_t SW = static_cast<size_t>(s.M) * (s.d_xi + s.d_v + 1);
+  return 16 + BH * (nseg - 1) * SW * sizeof(float2) + (opt && opt->delta_t ? BH * nseg * sizeof(double) : 0);
+}
+
+// the planned count, lowered until the caller's workspace holds it
+int ex_fit_segments(const ia_shape_t& s, const ia_options_t* opt, const void* workspace, size_t workspace_bytes) {
+  int nseg = ex_segments(s, opt);
+  while (nseg > 1 && (!workspace || ex_seg_bytes(s, opt, nseg) > workspace_bytes)) --nseg;
+  return nseg;
+}
+
+cudaError_t launch_ex_carry(const ia_shape_t& s, const ExArgs& a, cudaStream_t st) {
+  const long long rows = static_cast<long long>(s.B) * s.H * s.M;
+  ex_carry_kernel<<<static_cast<unsigned>(rows), 128, sizeof(double2) * a.nseg, st>>>(
+      s.H, s.N, s.d_xi, s.d_v, s.M, a.delta, a.dpm, a.A, a.dsum, a.nseg, a.seg_len, a.seg);
+  return cudaGetLastError();
+}
+
+// one direction of the token-serial form: a single pass, or pass 1, the carry
+// and pass 2 over the segments
+cudaError_t run_ex_direction(const ia_shape_t& s, const void* q, const void* k, const void* v, ExArgs a,
+                             cudaStream_t st) {
+  if (a.nseg <= 1) {
+    a.pass = 0;
+    return launch_ex_any(s, s.N, q, k, v, a, st);
+  }
+  a.pass = 1;
+  cudaError_t e = launch_ex_any(s, s.N, q, k, v, a, st);
+  if (e == cudaSuccess && a.nseg > 2) e = launch_ex_carry(s, a, st);
+  if (e != cudaSuccess) return e;
+  a.pass = 2;
+  return launch_ex_any(s, s.N, q, k, v, a, st);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr size_t kMaxSmem = 232448;
 
 ExArgs make_args(const ia_shape_t* s, const ia_options_t* opt, const float* delta, const float* A) {
   ExArgs a = {};
+  a.nseg = 1;
+  a.seg_len = 1 << 30;
   a.delta = delta;
   a.dpm = s->delta_per_mode;
   a.A = A;
@@ -242,8 +537,16 @@ using namespace ia;
 extern "C" {
 
 IA_API size_t ia_prefill_ex_workspace_bytes(const ia_shape_t* s, const ia_options_t* opt) {
-  if (!valid_dims(s, true) || !valid_options(opt) || !ex_use_tc(*s, opt)) return 0;
+  if (!valid_dims(s, true) || !valid_options(opt)) return 0;
+  if (!ex_use_tc(*s, opt)) return ex_seg_bytes(*s, opt, ex_segments(*s, opt));
   return ex_tc_workspace_bytes(*s, opt, tc_plan(*s, num_sms()));
+}
+
+IA_API int ia_prefill_ex_segments(const ia_shape_t* s, const ia_options_t* opt, const void* workspace,
+                                  size_t workspace_bytes) {
+  if (!valid_dims(s, true) || !valid_options(opt)) return 0;
+  if (ex_use_tc(*s, opt)) return 1;
+  return ex_fit_segments(*s, opt, workspace, workspace_bytes);
 }
 
 IA_API int ia_prefill_ex_path(const ia_shape_t* s, const ia_options_t* opt) {
@@ -289,12 +592,22 @@ IA_API ia_status_t ia_prefill_fwd_ex(const ia_shape_t* s, const ia_options_t* op
   a.o = o;
   a.num = num;
   a.den = den;
+  const int nseg = ex_fit_segments(*s, opt, workspace, workspace_bytes);
+  if (nseg > 1) {
+    const uintptr_t base = (reinterpret_cast<uintptr_t>(workspace) + 15) & ~static_cast<uintptr_t>(15);
+    const size_t BH = static_cast<size_t>(s->B) * s->H;
+    const size_t slots = BH * (nseg - 1) * s->M * (s->d_xi + s->d_v + 1) * sizeof(float2);
+    a.nseg = nseg;
+    a.seg_len = (s->N + nseg - 1) / nseg;
+    a.seg = reinterpret_cast<float2*>(base);
+    a.dsum = a.delta_t ? reinterpret_cast<double*>(base + slots) : nullptr;
+  }
   mark_launch_begin(st);
-  cudaError_t e = launch_ex_any(*s, s->N, q, k, v, a, st);
+  cudaError_t e = run_ex_direction(*s, q, k, v, a, st);
   if (e == cudaSuccess && bidir) {
     a.reverse = 1;
     a.accumulate = 1;
-    e = launch_ex_any(*s, s->N, q, k, v, a, st);
+    e = run_ex_direction(*s, q, k, v, a, st);
   }
   mark_launch_end(st);
   return map_cuda(e);

@@ -223,3 +223,23 @@ def test_grid_override_and_cuda_core_path(lib, monkeypatch):
     t = shape(B=1, H=2, N=256, dx=16, dv=16, M=16, dt=0)
     assert lib.ia_prefill_launches(ctypes.byref(t)) == 1
     assert lib.ia_prefill_grid(ctypes.byref(t)) == 0
+
+
+def test_token_serial_segments_follow_the_workspace():
+    # the token-serial form's segment count: at most one per 64 tokens, at
+    # most the planned count, and only as many as the workspace holds (none
+    # given: one CTA per (b,h)); the tensor-core form is always 1
+    import ssm_token_mixer_b200 as ia
+    B, H, N, d, M = 1, 2, 357, 16, 8
+    need = ia.prefill_ex_workspace_bytes(B, H, N, d, d, M, "f32", selective=True)
+    full = ia.prefill_ex_segments(B, H, N, d, d, M, "f32", need, selective=True)
+    assert 2 <= full <= N // 64
+    assert ia.prefill_ex_segments(B, H, N, d, d, M, "f32", 0, selective=True) == 1
+    assert ia.prefill_ex_segments(B, H, N, d, d, M, "f32", need - 1, selective=True) == full - 1
+    assert ia.prefill_ex_segments(B, H, 127, d, d, M, "f32", 1 << 30, selective=True) == 1
+    # bytes grow by one end state per extra segment, plus a step sum per segment with delta_t
+    per_seg = B * H * M * (2 * d + 1) * 8
+    assert need == 16 + (full - 1) * per_seg + B * H * full * 8
+    plain = ia.prefill_ex_workspace_bytes(B, H, N, d, d, M, "f32", readout=True)
+    assert plain == 16 + (ia.prefill_ex_segments(B, H, N, d, d, M, "f32", plain, readout=True) - 1) * per_seg
+    assert ia.prefill_ex_segments(B, H, 4096, 64, 64, 64, "bf16", 1 << 30, norm=True) == 1   # tensor cores

@@ -201,3 +201,71 @@ def test_tensor_core_stabilised_split_prefill(oracle_mod, dev, dx, dv):
     assert slice_rel(o, ref["o"], (-2, -1)) < TOL_BF16
     st = r2["state"].cpu().double().numpy()
     assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < TOL_BF16
+
+
+def mode_params(H, M, seed):
+    """Delta [H,M] in the S4D-Lin step range and a general decaying A [2M]."""
+    g = torch.Generator().manual_seed(seed)
+    delta = torch.exp(np.log(2e-2) + torch.rand(H, M, generator=g) * (np.log(1.2e-1) - np.log(2e-2)))
+    A = torch.empty(2 * M)
+    A[0::2] = -0.2 - 0.6 * torch.rand(M, generator=g)
+    A[1::2] = np.pi * torch.arange(M) + 0.7 * torch.rand(M, generator=g)
+    return delta.float(), A.float()
+
+
+SEG_CASES = [("selective", "norm", "readout"), ("readout",), ("norm",)]
+
+
+@pytest.mark.parametrize("which", SEG_CASES, ids=["+".join(c) for c in SEG_CASES])
+def test_segmented_token_serial_pass(oracle_mod, dev, which):
+    # The token-serial form cuts 357 tokens into five segments (the last one
+    # ragged) around the carry kernel, from the state a 50-token prefix left,
+    # with a general A and, without a step per token, a Delta per (head, mode):
+    # o and the end state against the oracle on the whole sequence, and o
+    # against the single pass that a one-byte workspace leaves
+    B, H, P, N, dx, dv, M = 1, 2, 50, 357, 16, 12, 8
+    inp = synthetic.layer_inputs(B, H, P + N, dx, dv, "f32", seed=88)
+    opt = options(B, H, P + N, dx, dv, M, 89, which)
+    delta, A = mode_params(H, M, 90)
+    if "selective" in which:
+        delta = None
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=delta, A=A, **to_oracle(opt))
+    pre = oracle_mod.forward_ex(*(x[:, :, :P] for x in (inp["q"], inp["k"], inp["v"])), M, delta=delta, A=A,
+                                **to_oracle({k: (x[:, :, :P] if k == "delta_t" else x) for k, x in opt.items()}))
+    g = lambda x: None if x is None else x.to(dev)
+    tail = lambda x: g(x[:, :, P:].contiguous())
+    kw = {k: (tail(x) if k == "delta_t" else g(x)) for k, x in opt.items()}
+    state_in = g(torch.from_numpy(np.asarray(pre["state"], dtype=np.float32).ravel()))
+    need = ia.prefill_ex_workspace_bytes(B, H, N, dx, dv, M, "f32", norm="gain" in opt, selective="delta_t" in opt,
+                                         readout="W" in opt)
+    assert need > 0
+    outs = {}
+    for name, ws in (("segmented", torch.empty(need, dtype=torch.uint8, device=dev)),
+                     ("single", torch.empty(1, dtype=torch.uint8, device=dev))):
+        r = ia.prefill_fwd_ex(tail(inp["q"]), tail(inp["k"]), tail(inp["v"]), M, delta=g(delta), A=g(A),
+                              state_in=state_in, want_state=True, workspace=ws, **kw)
+        ia.check_device_errors()
+        outs[name] = r
+        assert slice_rel(r["o"].cpu(), ref["o"][:, :, P:], (-2, -1)) < TOL_F32, name
+        st = r["state"].cpu().double().numpy()
+        want = np.asarray(ref["state"]).ravel()
+        assert np.abs(st - want).max() / np.abs(want).max() < TOL_F32, name
+    assert slice_rel(outs["segmented"]["o"].cpu(), outs["single"]["o"].cpu().double().numpy(), (-2, -1)) < TOL_F32
+
+
+def test_segmented_bidirectional_layer(oracle_mod, dev):
+    # both directions of the bidirectional layer cut into segments, a step per
+    # token (the carry's decay from the summed steps, summed back to front in
+    # the second direction)
+    B, H, N, d, M = 2, 2, 300, 16, 8
+    inp = synthetic.layer_inputs(B, H, N, d, d, "f32", seed=91)
+    opt = options(B, H, N, d, d, M, 92, ("selective", "norm"))
+    g = lambda x: x.to(dev)
+    need = ia.prefill_ex_workspace_bytes(B, H, N, d, d, M, "f32", norm=True, selective=True, bidirectional=True)
+    assert need > 0
+    r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, bidirectional=True,
+                          workspace=torch.empty(need, dtype=torch.uint8, device=dev),
+                          **{k: g(v) for k, v in opt.items()})
+    ia.check_device_errors()
+    ref = oracle_mod.forward_bidirectional(inp["q"], inp["k"], inp["v"], M, **to_oracle(opt))
+    assert slice_rel(r["o"].cpu(), ref, (-2, -1)) < TOL_F32
