@@ -482,13 +482,20 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
         toks = [tuple(x.to(dev) for x in synthetic.decode_token(B, w.H, w.d_xi, w.d_v, "bf16", step=i))
                 for i in range(steps)]
         o = torch.empty(B, w.H, w.d_v, dtype=torch.float32, device=dev)
-        # one captured graph per timed step (its own inputs and state replica)
+        # the K timed steps captured in one CUDA graph, each step with its own
+        # inputs and state replica: kernel after kernel inside a graph, as a
+        # layer's decode kernel runs inside a per-token graph of a whole model;
+        # for comparison the same steps as K graphs of one step each
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             for i in range(3):   # warm-up outside capture
                 ia.decode_step(*toks[i % len(toks)], delta, states[i % R], w.M, o=o, stream=s)
         torch.cuda.current_stream().wait_stream(s)
+        loop = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(loop, stream=s):
+            for i in range(steps):
+                ia.decode_step(*toks[i], delta, states[i % R], w.M, o=o, stream=s)
         graphs = []
         for i in range(steps):
             gr = torch.cuda.CUDAGraph()
@@ -500,8 +507,11 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
         fn = lambda: graphs[next(it) % steps].replay()
         barrier(dev)
         # the K steps run back to back (a decode loop); the state replicas
-        # rotate through more than L2, so no flush is needed between them
-        step_ms = timer.run_batch(fn, steps, warmup)
+        # rotate through more than L2, so no flush is needed between them.
+        # Warm-up: W replays of the K-step graph.
+        t_loop = timer.run_batch(loop.replay, 1, max(1, warmup))[0]
+        step_ms = [t_loop / steps] * steps
+        per_graph_ms = timer.run_batch(fn, steps, warmup)
         barrier(dev)
         total = max_over_ranks(sum(step_ms), dev)
         by = bytes_decode(w.d_xi, w.d_v, w.M) * B * w.H
@@ -512,9 +522,10 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
         rf["peak"] = float(peaks["hbm_gbs"])
         rf["frac"] = rf["achieved"] / rf["peak"]
         rf.pop("tensor_frac", None)
-        rf["note"] = (f"one graph replay per step, the steps back to back between two events (kernel only); "
+        rf["note"] = (f"the K steps in one captured graph, between two events (kernel only); "
                       f"{R} state replicas rotate so each step reads HBM")
         entry = {"value": world * B * steps / (total * 1e-3), "ms_per_step": total / steps,
+                 "ms_per_step_one_graph_per_step": statistics.mean(per_graph_ms),
                  "roofline": rf, "gpu_launches": steps}
         # end to end with host buffers (no graph): H2D q,k,v, step, D2H o
         hq = [tuple(x.pin_memory() for x in synthetic.decode_token(B, w.H, w.d_xi, w.d_v, "bf16", step=i))
@@ -537,7 +548,7 @@ def leg_decode(dev, w, steps, warmup, timer, peaks, peak_kind, rank, world, cpu_
                         "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in hq[0])),
                         "d2h_bytes_per_step": int(oh.numel() * 4)}
         out["batches"][str(B)] = entry
-        del graphs, states, pre
+        del graphs, loop, states, pre
         torch.cuda.empty_cache()
     if cpu_leg and rank == 0 and world == 1:
         import numpy as np

@@ -10,6 +10,7 @@
 // group of modes through shared memory with bulk copies and writes them back
 // with 16-byte stores, and the cluster's rank-0 CTA sums the partial num/den
 // over distributed shared memory and writes o.
+#include <algorithm>
 #include <cstdlib>
 #include <cooperative_groups.h>
 
@@ -44,14 +45,18 @@ __device__ __forceinline__ float xi_acc(float x) { return x > 0.f ? x + 1.f : ex
 // that every SM holds several CTAs and each warp's rows are all in flight at
 // once; the cluster's rank-0 CTA then adds the partials of the others over
 // distributed shared memory, in rank order.
-constexpr int kBhWarps = 8;
-
-template <typename T>
-__global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
+// NW warps per CTA (8).  Smaller CTAs (4 warps, each (b,h) split over 2, 4
+// or 8 of them so that every SM gets an even share of mode rows) measured
+// slower on a B200 at every batch of the 1.3B shape: at B = 16 the 256 whole
+// (b,h) already stream at about 0.9 of HBM in the main phase, and the split
+// repeats the per-(b,h) set-up.
+template <typename T, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == 8 ? 4 : 8) decode_bh_kernel(
     int H, int DX, int DV, int M, int D, const T* __restrict__ q, const T* __restrict__ k,
     const T* __restrict__ v, const float* __restrict__ delta, int dpm, const float* __restrict__ A,
     float2* __restrict__ state, float* __restrict__ o, float* __restrict__ num,
     float* __restrict__ den, long long BH, int* err) {
+  constexpr int kBhWarps = NW;
   extern __shared__ float4 dsm[];
   const uint32_t rowU = static_cast<uint32_t>(DX) * 8, rowG = static_cast<uint32_t>(DV) * 8, slot = rowU + rowG;
   // ring of D mode rows (U row then Gamma row) per warp, then its mbarriers
@@ -79,6 +84,10 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
   uint8_t* myring = ring + warp * D * slot;
   uint64_t* mybar = bars + warp * D;
   const int nj = warp < MS ? (MS - warp + kBhWarps - 1) / kBhWarps : 0;   // modes m_lo + warp, + 8, ...
+  // Programmatic dependent launch: this grid may have become resident while
+  // the previous kernel in the stream finished; nothing global is read before
+  // that kernel has completed and its writes are visible.
+  griddep_wait();
 
   // each warp streams its own modes' state rows through its ring, D rows ahead
   auto issue = [&](int j) {
@@ -91,13 +100,16 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
   // round trip, ahead of the ring's bulk copies: behind them, each of these
   // small dependent loads would wait out the copies' queue.
   constexpr int NT = kBhWarps * 32;
-  float xq = 0.f, xk = 0.f, xv = 0.f, pd = 0.f, par = -0.5f, pai = 0.f;
+  constexpr int R = (2 * 32 * kVecPerLane + NT - 1) / NT;   // features per thread (d <= 256)
+  float xq[R], xk[R], xv[R], pd = 0.f, par = -0.5f, pai = 0.f;
   float2 pe = make_float2(0.f, 0.f);
-  if (tid < DX) {
-    xq = ldx(q + bh * DX + tid);
-    xk = ldx(k + bh * DX + tid);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int f = tid + r * NT;
+    xq[r] = f < DX ? ldx(q + bh * DX + f) : 0.f;
+    xk[r] = f < DX ? ldx(k + bh * DX + f) : 0.f;
+    xv[r] = f < DV ? ldx(v + bh * DV + f) : 0.f;
   }
-  if (tid < DV) xv = ldx(v + bh * DV + tid);
   if (tid < MS) {
     const int m = m_lo + tid;
     if (A) {
@@ -132,11 +144,15 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
     bb[mi] = make_float2(fmaf(nr, ar, ni * ai) / dd, fmaf(ni, ar, -nr * ai) / dd);
     eta[mi] = e;
   };
-  if (tid < DX) {
-    fq[tid] = xi_acc(xq);
-    fk[tid] = xi_acc(xk);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int f = tid + r * NT;
+    if (f < DX) {
+      fq[f] = xi_acc(xq[r]);
+      fk[f] = xi_acc(xk[r]);
+    }
+    if (f < DV) vv[f] = xv[r];
   }
-  if (tid < DV) vv[tid] = xv;
   if (tid < MS) params(tid, par, pai, pd, pe);
   for (int mi = tid + NT; mi < MS; mi += NT) {   // more modes per CTA than threads
     const int m = m_lo + mi;
@@ -211,6 +227,9 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
       issue(issued++);
     }
   }
+  // the next kernel in the stream may launch once every CTA has streamed its
+  // rows (it still waits for this grid's completion before reading memory)
+  griddep_launch_dependents();
   if (!ok) {   // let this warp's copies in flight land (bounded) before the block exits
     if (lane == 0)
       for (int j = 0; j < issued; ++j) mbar_wait(mybar + j % D, static_cast<uint32_t>((j / D) & 1), err);
@@ -265,8 +284,51 @@ __global__ void __launch_bounds__(kBhWarps * 32, 4) decode_bh_kernel(
 }
 
 // shared memory besides the ring: features, partial sums, mode parameters
-size_t decode_fixed_smem(const ia_shape_t& s) {
-  return sizeof(float) * (2 * s.d_xi + s.d_v + kBhWarps * s.d_v + kBhWarps) + sizeof(float2) * 3 * s.M + 16;
+size_t decode_fixed_smem(const ia_shape_t& s, int nw) {
+  return sizeof(float) * (2 * s.d_xi + s.d_v + nw * s.d_v + nw) + sizeof(float2) * 3 * s.M + 16;
+}
+
+template <typename T, int NW>
+cudaError_t decode_launch(const ia_shape_t& s, int S, const void* q, const void* k, const void* v,
+                          const float* delta, const float* A, void* state, float* o, float* num, float* den,
+                          cudaStream_t st) {
+  const long long BHc = static_cast<long long>(s.B) * s.H;
+  // ring depth: up to four mode rows per warp, within a quarter of an SM's
+  // shared memory per CTA so that four fit (a deeper ring for fewer CTAs per
+  // SM measured slower on a B200)
+  const size_t row = static_cast<size_t>(s.d_xi + s.d_v) * 8;
+  const size_t fixed = decode_fixed_smem(s, NW);
+  const int per_warp = (s.M / S + NW - 1) / NW;
+  const size_t budget = 56 * 1024;
+  int D = 4;
+  while (D > 1 && NW * D * (row + 8) + fixed > budget) --D;
+  D = std::max(1, std::min(D, per_warp));
+  const size_t smem = NW * D * (row + 8) + fixed;
+  int* err = device_error_ptr();
+  if (!err) return cudaErrorInvalidSymbol;
+  auto kern = decode_bh_kernel<T, NW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(BHc * S), 1, 1);
+  cfg.blockDim = dim3(NW * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  mark_launch_begin(st);
+  e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q), static_cast<const T*>(k),
+                         static_cast<const T*>(v), delta, s.delta_per_mode, A, static_cast<float2*>(state), o, num,
+                         den, BHc, err);
+  mark_launch_end(st);
+  return e;
 }
 
 template <typename T>
@@ -286,48 +348,13 @@ cudaError_t decode_impl(const ia_shape_t& s, const void* q, const void* k, const
     const int f = std::atoi(env);
     if ((f == 1 || f == 2 || f == 4 || f == 8) && s.M % f == 0) S = f;
   }
-  {
-    // ring depth: up to four mode rows per warp, within a quarter of an SM's
-    // shared memory per CTA so that four CTAs fit (a deeper ring for fewer
-    // CTAs per SM measured slower on a B200)
-    const size_t row = static_cast<size_t>(s.d_xi + s.d_v) * 8;
-    const size_t fixed = decode_fixed_smem(s);
-    const int per_warp = (s.M / S + kBhWarps - 1) / kBhWarps;
-    const size_t budget = 56 * 1024;
-    int D = 4;
-    while (D > 1 && kBhWarps * D * (row + 8) + fixed > budget) --D;
-    D = std::max(1, std::min(D, per_warp));
-    const size_t smem = kBhWarps * D * (row + 8) + fixed;
-    int* err = device_error_ptr();
-    if (!err) return cudaErrorInvalidSymbol;
-    auto kern = decode_bh_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(BHc * S), 1, 1);
-    cfg.blockDim = dim3(kBhWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    mark_launch_begin(st);
-    e = cudaLaunchKernelEx(&cfg, kern, s.H, s.d_xi, s.d_v, s.M, D, static_cast<const T*>(q),
-                           static_cast<const T*>(k), static_cast<const T*>(v), delta, s.delta_per_mode, A,
-                           static_cast<float2*>(state), o, num, den, BHc, err);
-    mark_launch_end(st);
-    return e;
-  }
+  return decode_launch<T, 8>(s, S, q, k, v, delta, A, state, o, num, den, st);
 }
 
 }  // namespace
 
-size_t decode_smem_bytes(const ia_shape_t& s) {
-  return kBhWarps * (static_cast<size_t>(s.d_xi + s.d_v) * 8 + 8) + decode_fixed_smem(s);
+size_t decode_smem_bytes(const ia_shape_t& s) {   // the larger CTA's least ring
+  return 8 * (static_cast<size_t>(s.d_xi + s.d_v) * 8 + 8) + decode_fixed_smem(s, 8);
 }
 
 cudaError_t launch_decode(const ia_shape_t& s, const void* q, const void* k, const void* v,
