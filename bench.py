@@ -614,11 +614,12 @@ def leg_optional_parts(dev, w, steps, warmup, timer, peaks, peak_kind, rank, wor
         passes = 2 if kw.get("bidirectional") else 1
         rf = roofline(by * passes, flops_fwd(w.d_xi, w.d_v, w.M) * tokens * w.H * passes, kern_ms, peaks,
                       peak_kind, None, sustained=False)
-        # tensor cores: the prologue, a table kernel and a chunk pass per direction, the epilogue;
-        # token-serial: one pass per direction, or pass 1, the carry (past two segments) and pass 2
+        # tensor cores: the prologue, the W' conversion, a table kernel and a chunk pass per direction,
+        # the epilogue; token-serial: one pass per direction, or pass 1, the carry (past two segments)
+        # and pass 2
         nseg = ia.prefill_ex_segments(w.B, w.H, w.N, w.d_xi, w.d_v, w.M, "bf16", need, **present)
-        launches = ((1 if present["norm"] or present["bidirectional"] else 0) + passes * 2 +
-                    (1 if present["bidirectional"] else 0)) if path == "tensor_core" else \
+        launches = ((1 if present["norm"] or present["bidirectional"] else 0) + (1 if present["readout"] else 0) +
+                    passes * 2 + (1 if present["bidirectional"] else 0)) if path == "tensor_core" else \
             passes * (1 if nseg == 1 else 2 if nseg == 2 else 3)
         out["parts"][name] = {"value": world * tokens * steps / (total * 1e-3), "ms_per_step": total / steps,
                               "path": path, "segments": nseg, "roofline": rf, "gpu_launches": launches * steps}

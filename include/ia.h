@@ -255,13 +255,17 @@ typedef struct {
  * ia_prefill_fwd with the optional parts (NULL opt = the plain layer).
  * Two forms, chosen per call (ia_prefill_ex_path tells which):
  *   - bf16 inputs on a shape of the tensor-core chunk pass (M = 64, d_xi and
- *     d_v in {64, 128}) with no delta_t and no W run on tensor cores: a
- *     prologue kernel writes the stabilised SSM input z (when gain or bias is
- *     given) as fp16 k and v operands, and the time-reversed q and z (for the
- *     bidirectional layer); the chunk pass runs once, or twice for the
- *     bidirectional layer, whose second output an epilogue kernel adds back
- *     in forward order.  z is rounded to fp16 once more than in the
- *     token-serial form.  Needs ia_prefill_ex_workspace_bytes of workspace.
+ *     d_v in {64, 128}) with no delta_t, and W only at d_xi = 64, run on
+ *     tensor cores: a prologue kernel writes the stabilised SSM input z (when
+ *     gain or bias is given) as fp16 k and v operands, and the time-reversed
+ *     q and z (for the bidirectional layer); a second kernel writes W as the
+ *     real fp16 matrix [[Re W, -Im W], [Im W, Re W]] (rows and columns
+ *     interleaved by mode), and the chunk pass then runs one more contraction
+ *     per chunk, W times the readout vectors of its 64 tokens; the chunk pass
+ *     runs once, or twice for the bidirectional layer, whose second output an
+ *     epilogue kernel adds back in forward order.  z, and with W the readout
+ *     vectors and W, are rounded to fp16 once more than in the token-serial
+ *     form.  Needs ia_prefill_ex_workspace_bytes of workspace.
  *   - everything else runs the token-serial fp32 CUDA-core kernel (any
  *     input dtype), correct for every shape whose state fits in shared memory
  *     but much slower.  With ia_prefill_ex_workspace_bytes of workspace it

@@ -59,7 +59,7 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st,
                               void* dump_R = nullptr, float* dump_Re = nullptr,
-                              float* dtab = nullptr, bool kv_ready = false);
+                              float* dtab = nullptr, bool kv_ready = false, const void* Wt = nullptr);
 // Byte offset of the per-head tables inside a tensor-core workspace (256-aligned start).
 HeadTables* tc_tables(void* ws);
 

@@ -512,8 +512,9 @@ ExArgs make_args(const ia_shape_t* s, const ia_options_t* opt, const float* delt
 }
 
 // The tensor-core form (ia_layer_tc.cu) serves bf16 shapes of the chunk pass
-// whose options are only the input stabilisation and / or the bidirectional
-// layer; IA_PREFILL_SIMT forces the token-serial kernel, as for the plain layer.
+// without a per-token step (the input stabilisation, the bidirectional layer
+// and, at d_xi = 64, the readout matrix); IA_PREFILL_SIMT forces the
+// token-serial kernel, as for the plain layer.
 bool ex_use_tc(const ia_shape_t& s, const ia_options_t* opt) {
   const char* env = std::getenv("IA_PREFILL_SIMT");
   if (env && env[0] && std::strcmp(env, "0") != 0) return false;

@@ -9,14 +9,22 @@
 //     The prologue also writes the time-reversed q (bf16) and z (fp16), a
 //     second chunk pass runs the causal layer on them, and an epilogue adds
 //     its output, reversed back, to the first pass's.
-// The per-token step (selective writing) and the readout matrix change the
-// chunk algebra itself and stay on the token-serial kernel (ia_layer_ex.cu).
+//   - the complex readout matrix (summary sec. A.3), d_xi = 64: a~_t = W_h a_t
+//     before the readout.  wprime_kernel writes W_h as the real fp16 matrix W'
+//     (ia_tables.cuh) and the chunk pass runs one more contraction per chunk,
+//     G_W: a~~ = W' a, between its key-state read and its score matrix (the
+//     readout factor then is a complex rotation per entry instead of a real
+//     row scale).  W' and a are fp16 operands, one rounding more than the
+//     plain layer's.
+// The per-token step (selective writing) changes the chunk decay itself and
+// stays on the token-serial kernel (ia_layer_ex.cu).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "ia_device.cuh"
 #include "ia_internal.h"
 #include "ia_simt_common.cuh"
+#include "ia_tables.cuh"
 
 namespace ia {
 namespace {
@@ -83,6 +91,18 @@ __global__ void __launch_bounds__(kPrepWarps * 32) ex_prep_kernel(
   }
 }
 
+// W [H][M][M] complex (re, im pairs) -> W' per head (wprime_offset layout):
+// one block per (h, row k of W'), one thread per column k'.
+__global__ void __launch_bounds__(2 * kModesTC) wprime_kernel(const float* __restrict__ W, __half* __restrict__ Wt) {
+  const int h = blockIdx.x / (2 * kModesTC), k = blockIdx.x % (2 * kModesTC), kp = threadIdx.x;
+  const int m = k >> 1, mp = kp >> 1;
+  const float2 w = reinterpret_cast<const float2*>(W)[(static_cast<long long>(h) * kModesTC + m) * kModesTC + mp];
+  // [re -im; im re] in the (k, k') parities
+  const float x = (k & 1) == (kp & 1) ? w.x : ((k & 1) ? w.y : -w.y);
+  *reinterpret_cast<__half*>(reinterpret_cast<uint8_t*>(Wt) + static_cast<size_t>(h) * kWprimeBytes +
+                             wprime_offset(k, kp)) = __float2half_rn(x);
+}
+
 // o[bh][t] += orv[bh][N-1-t], four floats per thread (DV a multiple of 4)
 __global__ void __launch_bounds__(256) add_reversed_kernel(int N, int DV, float* __restrict__ o,
                                                           const float* __restrict__ orv, long long n4) {
@@ -101,7 +121,7 @@ __global__ void __launch_bounds__(256) add_reversed_kernel(int N, int DV, float*
 size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
 struct ExLayout {   // byte offsets inside the workspace (after the chunk pass's own)
-  size_t tc, kz, vz, qr, kr, vr, orv, total;
+  size_t tc, kz, vz, qr, kr, vr, orv, wt, total;
 };
 
 ExLayout ex_layout(const ia_shape_t& s, const ia_options_t& opt, const TcPlan& p) {
@@ -122,6 +142,7 @@ ExLayout ex_layout(const ia_shape_t& s, const ia_options_t& opt, const TcPlan& p
   L.kr = take(flip, tokens * s.d_xi * 2);
   L.vr = take(flip, tokens * s.d_v * 2);
   L.orv = take(flip, tokens * s.d_v * 4);
+  L.wt = take(opt.W != nullptr, static_cast<size_t>(s.H) * kWprimeBytes);
   L.total = at + 256;   // the caller's pointer may need rounding up to 256
   return L;
 }
@@ -130,7 +151,8 @@ ExLayout ex_layout(const ia_shape_t& s, const ia_options_t& opt, const TcPlan& p
 
 bool ex_tc_supported(const ia_shape_t& s, const ia_options_t* opt) {
   if (!tc_prefill_supported(s)) return false;
-  if (opt && (opt->delta_t || opt->W)) return false;
+  if (opt && opt->delta_t) return false;
+  if (opt && opt->W && s.d_xi != 64) return false;   // W' takes the shared memory of d_xi = 128's tiles
   return s.d_xi + s.d_v <= 256;
 }
 
@@ -156,6 +178,12 @@ cudaError_t launch_ex_tc(const ia_shape_t& s, const ia_options_t* opt, const TcP
   __half* kr = reinterpret_cast<__half*>(at(L.kr));
   __half* vr = reinterpret_cast<__half*>(at(L.vr));
   float* orv = reinterpret_cast<float*>(at(L.orv));
+  __half* wt = op.W ? reinterpret_cast<__half*>(at(L.wt)) : nullptr;
+  if (wt) {
+    wprime_kernel<<<static_cast<unsigned>(s.H * 2 * kModesTC), 2 * kModesTC, 0, st>>>(op.W, wt);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (norm || flip) {
     const unsigned grid = static_cast<unsigned>((tokens + kPrepWarps - 1) / kPrepWarps);
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
@@ -176,11 +204,11 @@ cudaError_t launch_ex_tc(const ia_shape_t& s, const ia_options_t* opt, const TcP
   // the causal pass over the sequence as given (z normalised when asked)
   cudaError_t e = launch_tc_prefill(s, p, q, norm ? static_cast<const void*>(kz) : k,
                                     norm ? static_cast<const void*>(vz) : v, delta, A, state_in, o, num, den,
-                                    state_out, ws, st, nullptr, nullptr, nullptr, norm);
+                                    state_out, ws, st, nullptr, nullptr, nullptr, norm, wt);
   if (e != cudaSuccess || !flip) return e;
   // the causal pass over the reversed sequence, added back in forward order
   e = launch_tc_prefill(s, p, qr, kr, vr, delta, A, nullptr, orv, nullptr, nullptr, nullptr, ws, st, nullptr,
-                        nullptr, nullptr, true);
+                        nullptr, nullptr, true, wt);
   if (e != cudaSuccess) return e;
   const long long n4 = tokens * s.d_v / 4;
   add_reversed_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(s.N, s.d_v, o, orv, n4);

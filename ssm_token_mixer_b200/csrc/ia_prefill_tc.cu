@@ -117,12 +117,15 @@ constexpr int GW = 8;                    // warps per epilogue group
 constexpr int GT = GW * 32;              // threads per epilogue group
 constexpr int NTH = 2 * GT + 64;         // + the MMA warp and the fetch warp
 
-template <int DX>
+template <int DX, bool RW>
 struct PCfg {
   static constexpr int F = DX + kVB;                // state columns: U | Gamma block
   static constexpr int FH = F / 2;                  // state columns per prepare thread
   static constexpr int WV = 80, NV = 80;            // [V | 1 0..] and [R_Gamma | R_eta 0..] widths
-  static constexpr int NB = DX == 64 ? 3 : 2;       // q, k, v and R_Gamma buffer sets
+  // q, k, v and R_Gamma buffer sets: two when the readout matrix W' takes
+  // its 32 KB of shared memory (d_xi = 64 only)
+  static constexpr int NB = DX == 64 && !RW ? 3 : 2;
+  static_assert(!RW || DX == 64, "the readout matrix runs at d_xi = 64");
   // d_xi = 128 needs 64 more state columns; S^T, a~ and P then share one tile
   // (each is dead before the next is written within a chunk), at the price
   // of issuing G1 of a chunk only after the previous chunk's P has been read.
@@ -153,7 +156,8 @@ struct PCfg {
   static constexpr uint32_t S_X = S_P + C * C * 2;
   static constexpr uint32_t S_O = S_X + KR * C * 2;   // [2] o staging, 128-byte swizzled
   static constexpr uint32_t S_RG = S_O + 2 * TO;      // [NB]
-  static constexpr uint32_t S_BAR = S_RG + NB * TRG;  // mbarriers
+  static constexpr uint32_t S_W = S_RG + NB * TRG;    // W' [2M x 2M] fp16, no-swizzle K-major (RW)
+  static constexpr uint32_t S_BAR = S_W + (RW ? KR * KR * 2 : 0);   // mbarriers
   static constexpr uint32_t S_FLAG = S_BAR + 256;     // abort flag, look-back exchange
   static constexpr uint32_t S_TMEMH = S_FLAG + 16;
   static constexpr uint32_t SMEM = S_TMEMH + 16;
@@ -178,6 +182,7 @@ struct TcArgs {
   float* incl;              // [G][128 * F + 128]: inclusive end state of a CTA's last piece
   int* flags;               // [G]: 0 nothing yet, 1 agg published, 2 incl published
   int kv_ready;             // 1: k, v arrive as fp16 operands (k already through the feature map)
+  const __half* Wt;         // readout matrix per head as W' tiles (wprime_offset layout), RW only
   int H, N, DV, nch, nvb, G;
   long long BH, total;      // total = BH * nvb * nch chunks
 };
@@ -297,29 +302,29 @@ __device__ __noinline__ float ragged_esum(const HeadTables* T, int m, int comp, 
 
 // state column f of row m in the public layout (complex): U for f < DX,
 // else column vb * 64 + f - DX of Gamma
-template <int DX>
+template <int DX, bool RW>
 __device__ __forceinline__ long long pub_index(const TcArgs& a, long long bh, int m, int vb, int f) {
   return f < DX ? (bh * 64 + m) * DX + f : a.BH * 64 * DX + (bh * 64 + m) * a.DV + vb * kVB + (f - DX);
 }
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void prep_zero(const PrepThread& th) {
-  constexpr int FH = PCfg<DX>::FH;
+  constexpr int FH = PCfg<DX, RW>::FH;
   uint32_t z[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) z[e] = 0u;
-  for (int cb = 0; cb < FH; cb += 16) tmem_st16(th.trow + PCfg<DX>::T_STATE + th.half * FH + cb, z);
+  for (int cb = 0; cb < FH; cb += 16) tmem_st16(th.trow + PCfg<DX, RW>::T_STATE + th.half * FH + cb, z);
   tmem_st_wait();
 }
 
 // initial scaled state of a piece from state_in (zero without it); returns
 // this row's eta
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ float prep_init_from_input(const TcArgs& a, const HeadTables* T, const PrepThread& th,
                                                   long long bh, int vb) {
-  constexpr int FH = PCfg<DX>::FH;
+  constexpr int FH = PCfg<DX, RW>::FH;
   if (!a.state_in) {
-    prep_zero<DX>(th);
+    prep_zero<DX, RW>(th);
     return 0.f;
   }
   const float2 si = T->sc_inv[th.m];
@@ -328,10 +333,10 @@ __device__ __noinline__ float prep_init_from_input(const TcArgs& a, const HeadTa
     uint32_t r[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      const float2 x = a.state_in[pub_index<DX>(a, bh, th.m, vb, col0 + e)];
+      const float2 x = a.state_in[pub_index<DX, RW>(a, bh, th.m, vb, col0 + e)];
       r[e] = __float_as_uint(th.comp ? fmaf(si.x, x.y, si.y * x.x) : fmaf(si.x, x.x, -si.y * x.y));
     }
-    tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_st16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
   }
   tmem_st_wait();
   const float2 x = a.state_in[a.BH * 64 * (DX + a.DV) + bh * 64 + th.m];
@@ -339,10 +344,10 @@ __device__ __noinline__ float prep_init_from_input(const TcArgs& a, const HeadTa
 }
 
 // the state after the last token of a stream: sc lambda^(nv - C) S_hat = lambda^(nv-c-1) S_hat
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTables* T, const PrepThread& th,
                                                   long long bh, int vb, int ch, float eta_c) {
-  constexpr int FH = PCfg<DX>::FH;
+  constexpr int FH = PCfg<DX, RW>::FH;
   const int nv = a.N - ch * C;
   double pr, pi;
   lam_pow(T, th.m, nv - C / 2 - 1, &pr, &pi);
@@ -350,7 +355,7 @@ __device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTab
   for (int cb = 0; cb < FH; cb += 16) {
     const int col0 = th.half * FH + cb;
     uint32_t r[16];
-    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_ld16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
     tmem_ld_wait16(r);
 #pragma unroll
     for (int e2 = 0; e2 < 16; ++e2) {
@@ -358,7 +363,7 @@ __device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTab
       const float y = __shfl_xor_sync(kFull, x, 1);
       const int f = col0 + e2;
       if (th.comp == 0 && (f >= DX || vb == 0))   // U is the same in every value block
-        a.state_out[pub_index<DX>(a, bh, th.m, vb, f)] = make_float2(fr * x - fi * y, fr * y + fi * x);
+        a.state_out[pub_index<DX, RW>(a, bh, th.m, vb, f)] = make_float2(fr * x - fi * y, fr * y + fi * x);
     }
   }
   const float y = __shfl_xor_sync(kFull, eta_c, 1);
@@ -373,14 +378,14 @@ __device__ __noinline__ void prep_write_state_out(const TcArgs& a, const HeadTab
 __device__ __forceinline__ int pub4(int c, int k) { return (c >> 2) * KR + k; }
 
 // this thread's part of the TMEM state (and eta) -> dst [128 * F + 128]
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void prep_publish(const PrepThread& th, float* dst, float eta_c) {
-  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  constexpr int F = PCfg<DX, RW>::F, FH = PCfg<DX, RW>::FH;
   float4* d4 = reinterpret_cast<float4*>(dst);
   for (int cb = 0; cb < FH; cb += 16) {
     const int col0 = th.half * FH + cb;
     uint32_t r[16];
-    tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+    tmem_ld16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
     tmem_ld_wait16(r);
 #pragma unroll
     for (int g = 0; g < 4; ++g)
@@ -401,9 +406,9 @@ __device__ __noinline__ void prep_raise_flag(int* flag, int value, int tid) {
 // TMEM state (and eta) += (mr + i mi) src, complex per mode (rows 2m, 2m+1).
 // src was written by another SM: each load is an L2 round trip, so a
 // thread's row segment is fetched in two batches (not one block at a time).
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* src, double mr, double mi, float* eta) {
-  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH;
+  constexpr int F = PCfg<DX, RW>::F, FH = PCfg<DX, RW>::FH;
   constexpr int HB = FH / 8;   // float4 per batch: half of this thread's segment
   static_assert(HB % 4 == 0, "a batch holds whole 16-column blocks");
   const float fr = static_cast<float>(mr), fs = static_cast<float>(th.comp ? mi : -mi);
@@ -418,7 +423,7 @@ __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* 
     for (int blk = 0; blk < HB / 4; ++blk) {
       const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
       uint32_t r[16];
-      tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+      tmem_ld16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
       tmem_ld_wait16(r);
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
@@ -427,7 +432,7 @@ __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* 
         const float y = __shfl_xor_sync(kFull, x, 1);
         r[e] = __float_as_uint(__uint_as_float(r[e]) + fmaf(fr, x, fs * y));
       }
-      tmem_st16(th.trow + PCfg<DX>::T_STATE + col0, r);
+      tmem_st16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
     }
   }
   tmem_st_wait();
@@ -445,12 +450,12 @@ __device__ __noinline__ void prep_accumulate(const PrepThread& th, const float* 
 // (uniform over the prepare group).
 constexpr int kLookBackWindow = 8;
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ bool prep_look_back(const TcArgs& a, const HeadTables* T, const PrepThread& th,
                                             volatile int* abort_flag, volatile int* xchg, float* eta) {
-  constexpr int STRIDE = KR * PCfg<DX>::F + KR;
+  constexpr int STRIDE = KR * PCfg<DX, RW>::F + KR;
   const double re_dA = T->re_dA[th.m], im_dA = T->im_dA[th.m];
-  prep_zero<DX>(th);
+  prep_zero<DX, RW>(th);
   *eta = 0.f;
   const long long g0 = range_lo(a.total, a.G, blockIdx.x);
   for (int p = static_cast<int>(blockIdx.x) - 1; p >= 0;) {
@@ -496,7 +501,7 @@ __device__ __noinline__ bool prep_look_back(const TcArgs& a, const HeadTables* T
         lr = e * cs;
         li = e * sn;
       }
-      prep_accumulate<DX>(th, (q == lo && incl ? a.incl : a.agg) + static_cast<long long>(q) * STRIDE, lr, li, eta);
+      prep_accumulate<DX, RW>(th, (q == lo && incl ? a.incl : a.agg) + static_cast<long long>(q) * STRIDE, lr, li, eta);
     }
     if (incl) return true;
     p = lo - 1;
@@ -506,10 +511,10 @@ __device__ __noinline__ bool prep_look_back(const TcArgs& a, const HeadTables* T
 
 // A CTA whose one piece lies inside a stream publishes its inclusive end
 // state once its carry (in TMEM, eta) is known: local + lambda^(C n) carry.
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadTables* T, const PrepThread& th,
                                                     int n, float eta_c) {
-  constexpr int F = PCfg<DX>::F, FH = PCfg<DX>::FH, STRIDE = KR * F + KR;
+  constexpr int F = PCfg<DX, RW>::F, FH = PCfg<DX, RW>::FH, STRIDE = KR * F + KR;
   double lr, li;
   lam_pow(T, th.m, static_cast<double>(C) * n, &lr, &li);
   const float fr = static_cast<float>(lr), fs = static_cast<float>(th.comp ? li : -li);
@@ -527,7 +532,7 @@ __device__ __noinline__ void prep_publish_inclusive(const TcArgs& a, const HeadT
     for (int blk = 0; blk < HB / 4; ++blk) {
       const int col0 = th.half * FH + (hb * HB + 4 * blk) * 4;
       uint32_t r[16];
-      tmem_ld16(th.trow + PCfg<DX>::T_STATE + col0, r);
+      tmem_ld16(th.trow + PCfg<DX, RW>::T_STATE + col0, r);
       tmem_ld_wait16(r);
       float o[16];
 #pragma unroll
@@ -563,31 +568,31 @@ struct PieceStart {
 // is done), and set the piece's initial state (zero, state_in, or the carry
 // from the look-back).  One call out of the chunk loop, so that the loop keeps
 // its registers for the per-chunk work.
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ PieceStart prep_piece_start(const TcArgs& a, const PrepThread& th, int i, int nA, long long gA,
                                                     int nF, bool so, int ch, long long bh, int vb, int h,
                                                     int prev_bh, int prev_vb, int prev_ch, int cur_h, float eta_c,
                                                     bool pending, volatile int* abort_flag, volatile int* xchg,
-                                                    volatile int* g4_seen, uint8_t* sE) {
-  constexpr int STRIDE = KR * PCfg<DX>::F + KR;   // floats per published state
+                                                    volatile int* g4_seen, uint8_t* sE, uint8_t* sW) {
+  constexpr int STRIDE = KR * PCfg<DX, RW>::F + KR;   // floats per published state
   PieceStart r{eta_c, true, pending};
   const HeadTables* T = a.tabs + cur_h;
   if (i > 0) {
     if (i - 1 < nA) {
       // end of the state-only chain: publish our last piece's state
       const bool inclusive = gA % a.nch == 0;
-      prep_publish<DX>(th, (inclusive ? a.incl : a.agg) + static_cast<long long>(blockIdx.x) * STRIDE, eta_c);
+      prep_publish<DX, RW>(th, (inclusive ? a.incl : a.agg) + static_cast<long long>(blockIdx.x) * STRIDE, eta_c);
       prep_raise_flag(a.flags + blockIdx.x, inclusive ? 2 : 1, th.tid);
       r.pending = !inclusive;
     } else if (prev_ch == a.nch - 1 && a.state_out) {
-      prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
+      prep_write_state_out<DX, RW>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
     }
   }
   if (h != cur_h) {
-    // A new head: its E' table replaces the old one once every contraction
-    // reading the old one is done.  G7 of the previous item is; every G2 and
-    // G4 of the previous full items is once the output warps have seen G4 of
-    // the last of them complete.
+    // A new head: its E' table (and W') replaces the old one once every
+    // contraction reading the old one is done.  G7 of the previous item is;
+    // every G2, G_W and G4 of the previous full items is once the output warps
+    // have seen G4 of the last of them complete.
     const int t = i - nA;
     if (t >= 1) {
       bool ok = true;
@@ -616,22 +621,27 @@ __device__ __noinline__ PieceStart prep_piece_start(const TcArgs& a, const PrepT
     const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h].E);
     uint4* dst = reinterpret_cast<uint4*>(sE);
     for (int x = th.tid; x < KR * C * 2 / 16; x += GT) dst[x] = src[x];
+    if constexpr (RW) {   // the head's readout matrix, read by G_W between G2+G3 and G4
+      const uint4* ws = reinterpret_cast<const uint4*>(a.Wt) + static_cast<size_t>(h) * (kWprimeBytes / 16);
+      uint4* wd = reinterpret_cast<uint4*>(sW);
+      for (int x = th.tid; x < static_cast<int>(kWprimeBytes / 16); x += GT) wd[x] = ws[x];
+    }
     T = a.tabs + h;
   }
   if (so && gA % a.nch != 0) {   // a local aggregate starts from zero
-    prep_zero<DX>(th);
+    prep_zero<DX, RW>(th);
     r.eta = 0.f;
   } else if (so || ch == 0) {    // a stream's start: state_in or zero
-    r.eta = prep_init_from_input<DX>(a, T, th, bh, vb);
+    r.eta = prep_init_from_input<DX, RW>(a, T, th, bh, vb);
   } else {                       // inside a stream: the carry from the predecessors
     float e = 0.f;
-    if (!prep_look_back<DX>(a, T, th, abort_flag, xchg, &e)) {
+    if (!prep_look_back<DX, RW>(a, T, th, abort_flag, xchg, &e)) {
       r.ok = false;
       return r;
     }
     r.eta = e;
     if (r.pending) {
-      prep_publish_inclusive<DX>(a, T, th, nF, e);
+      prep_publish_inclusive<DX, RW>(a, T, th, nF, e);
       r.pending = false;
     }
   }
@@ -652,12 +662,12 @@ struct PrepRun {
   bool ok;
 };
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ PrepRun prep_chunks(const TcArgs& a_in, uint8_t* smem, const PrepThread th, const HeadTables* T,
                                             int i, int n, int b, bool so, long long bh, int ch, float eta_c,
                                             uint32_t pd0, uint32_t pld, uint32_t pldv, float esum_tail) {
   const TcArgs a = a_in;
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int FH = K::FH, NB = K::NB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K::S_BAR);
   uint64_t* rdy0 = bars + 0;
@@ -832,9 +842,9 @@ __device__ __forceinline__ void convert_tile(uint8_t* base, int nv, int ct, bool
 // out of line, and the spills around those calls stay in that role).  Each
 // derives its barriers, tiles and schedule from shared memory and the
 // arguments; the barriers are described where the kernel initialises them.
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_first) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int NB = K::NB;
   const int tid = threadIdx.x, lane = tid & 31;
   const Sched sc(a.total, a.G, blockIdx.x, a.nch);
@@ -847,6 +857,8 @@ __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_f
   uint64_t* freeVR = bars + 12;   // [NB]: sV, sR_Gamma of that set reusable
   uint64_t* bar_drain = bars + 15;
   uint64_t* rdyKV = bars + 19;    // [NB]: output warps -> G7 of a state-only item (k, v converted)
+  uint64_t* rdyW = bars + 25;     // output warps -> G_W (a staged in the X tile)
+  uint64_t* dneW = bars + 26;     // G_W done
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   const uint32_t sbase = smem_u32(smem);
   auto sQ = [&](int b) { return K::S_Q + b * K::TQ; };
@@ -856,7 +868,7 @@ __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_f
   const uint32_t tmem = *reinterpret_cast<const uint32_t*>(smem + K::S_TMEMH);
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t pr[4] = {0u, 0u, 0u, 0u};
+      uint32_t pr[4] = {0u, 0u, 0u, 0u}, prW = 0u;
       bool ok = true;
       auto wait_rdy = [&](int i) -> bool {
         const bool r = mbar_wait_or_abort(rdy + i, pr[i], a.err, abort_flag);
@@ -892,6 +904,7 @@ __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_f
         mma_commit(dne + 3);
         mma_commit(freeVR + bb);
       };
+      static_assert(!(RW && K::SHARED_SAP), "G_W is issued by the in-order loop");
       if constexpr (K::SHARED_SAP) {
         // d_xi = 128 (measured on a B200: the 1.3B prefill 11% faster
         // than with the in-order issue below, which is faster at d_xi = 64)
@@ -1026,6 +1039,15 @@ __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_f
                        smem_desc_sw128(sbase + sQ(b) + K::kstep(kk), 16, K::SW), idesc_f16(128, 64, 0, 0), 1u);
           mma_commit(dne + 1);
           mma_commit(freeQK + b);
+          if constexpr (RW) {   // G_W: a~~ = W' a, over the a~ columns E2 has read
+            ok = mbar_wait_or_abort(rdyW, prW, a.err, abort_flag);
+            prW ^= 1u;
+            tc_fence_after();
+            if (!ok) break;
+            gemm(tmem + K::T_A, sbase + K::S_W, 128, 2048, 256, sbase + K::S_X, 1024, 128, 2048,
+                 idesc_f16(128, 64, 0, 1), KR / 16, false);
+            mma_commit(dneW);
+          }
           if (!(ok = wait_rdy(2))) break;
           gemm(tmem + K::T_P, sbase + K::S_X, 1024, 128, 2048, sbase + K::S_E, 1024, 128, 2048,
                idesc_f16(64, 64, 1, 1), KR / 16, false);   // G4: P
@@ -1045,9 +1067,9 @@ __device__ __noinline__ void tc_role_mma(const TcArgs& a, uint8_t* smem, int h_f
     __syncwarp();
 }
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int h_first) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int NB = K::NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gw = warp & (GW - 1);          // warp index within its epilogue group
@@ -1094,16 +1116,16 @@ __device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int
       const bool so = sc.state_only(i);
       const int n = so ? sc.nA : min(a.nch - w.ch, nI - i);
       if (i > 0 && !(ok = waitA(dne + 0, pd0))) break;   // G7 of the previous item: the state is current
-      const PieceStart ps = prep_piece_start<DX>(a, th, i, sc.nA, sc.gA, sc.nF, so, w.ch, w.bh, w.vb, w.h, prev_bh,
+      const PieceStart ps = prep_piece_start<DX, RW>(a, th, i, sc.nA, sc.gA, sc.nF, so, w.ch, w.bh, w.vb, w.h, prev_bh,
                                                  prev_vb, prev_ch, cur_h, eta_c, single_piece_pending, abort_flag,
-                                                 xchg, g4_seen, smem + K::S_E);
+                                                 xchg, g4_seen, smem + K::S_E, smem + K::S_W);
       if (!(ok = ps.ok)) break;
       eta_c = ps.eta;
       single_piece_pending = ps.pending;
       if (w.h != cur_h) set_head(w.h);
       const int last_nv = min(C, a.N - (w.ch + n - 1) * C);
       const float esum_tail = last_nv < C ? ragged_esum(T, m, comp, last_nv) : 0.f;
-      const PrepRun run = prep_chunks<DX>(a, smem, th, T, i, n, b, so, w.bh, w.ch, eta_c, pd0, pld, pldv, esum_tail);
+      const PrepRun run = prep_chunks<DX, RW>(a, smem, th, T, i, n, b, so, w.bh, w.ch, eta_c, pd0, pld, pldv, esum_tail);
       eta_c = run.eta;
       pd0 = run.pd0;
       pld = run.pld;
@@ -1118,14 +1140,14 @@ __device__ __noinline__ void tc_role_prepare(const TcArgs& a, uint8_t* smem, int
     }
     if (ok && nI > 0 && a.state_out && sc.g1 % a.nch == 0) {
       ok = waitA(dne + 0, pd0);   // G7 of the last chunk
-      if (ok) prep_write_state_out<DX>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
+      if (ok) prep_write_state_out<DX, RW>(a, T, th, prev_bh, prev_vb, prev_ch, eta_c);
     }
 }
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int h_first,
                                           const CUtensorMap& tm_o) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int NB = K::NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gw = warp & (GW - 1);          // warp index within its epilogue group
@@ -1138,6 +1160,8 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
   uint64_t* loadedQK = bars + 16;   // [NB]: that set's q, k rows have landed
   uint64_t* loadedV = bars + 22;    // [NB]: that set's v rows have landed
   uint64_t* rdyKV = bars + 19;    // [NB]: output warps -> G7 of a state-only item (k, v converted)
+  uint64_t* rdyW = bars + 25;     // output warps -> G_W (a staged in the X tile)
+  uint64_t* dneW = bars + 26;     // G_W done
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   volatile int* g4_seen = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 8);   // G4 groups seen done
   const uint32_t sbase = smem_u32(smem);
@@ -1149,9 +1173,10 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
     const int m = k >> 1;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quad) << 16);
     const int i0 = 32 * half;     // this thread's 32 columns of the 64-wide tiles
-    uint32_t pd[4] = {0u, 0u, 0u, 0u}, pS = 0u;
+    uint32_t pd[4] = {0u, 0u, 0u, 0u}, pS = 0u, pW = 0u;
     int cur_h = -1;
     float r2 = 0.f, s_start = 0.f;
+    float2 p_start = make_float2(0.f, 0.f), lam_m = make_float2(0.f, 0.f);   // RW: lambda_m^(i0 - c), lambda_m
     auto waitB = [&](uint64_t* bar, uint32_t& ph) -> bool {
       const bool r = mbar_wait_or_abort(bar, ph, a.err, abort_flag);
       ph ^= 1u;
@@ -1276,6 +1301,14 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
           cur_h = h;
           r2 = a.tabs[h].r2[m];
           s_start = static_cast<float>(exp(2.0 * a.tabs[h].re_dA[m] * (32.0 * half - C / 2)));
+          if constexpr (RW) {
+            const double n = 32.0 * half - C / 2;
+            const double mag = exp(n * a.tabs[h].re_dA[m]);
+            double sn, cs;
+            sincos(fmod(n * a.tabs[h].im_dA[m], 6.283185307179586476925), &sn, &cs);
+            p_start = make_float2(static_cast<float>(mag * cs), static_cast<float>(mag * sn));
+            lam_m = a.tabs[h].lam[m];
+          }
         }
         if (!(ok = waitB(dneS, pS))) break;   // G1(t)
         {  // E1(t): masked S^T -> [j][i]
@@ -1292,7 +1325,50 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
           signalB(1);
         }
         if (!(ok = waitB(dne + 1, pd[1]))) break;   // G2 + G3(t)
-        {  // E2(t): X = |lambda|^(2(i-c)) a~
+        if constexpr (RW) {
+          // E2a(t): a = lambda^(i-c) a~ into the X tile (G_W's B operand);
+          // each complex product takes the other part from the partner lane
+          // (rows 2m and 2m+1 sit in adjacent lanes)
+          const float sg = (k & 1) ? 1.f : -1.f;
+          float2 pw = p_start;
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            uint32_t r[16];
+            tmem_ld16(trow + K::T_A + i0 + 16 * bb, r);
+            tmem_ld_wait16(r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x = __uint_as_float(r[e]);
+              const float y = __shfl_xor_sync(kFull, x, 1);
+              r[e] = __float_as_uint(fmaf(pw.x, x, sg * pw.y * y));
+              pw = make_float2(fmaf(pw.x, lam_m.x, -pw.y * lam_m.y), fmaf(pw.x, lam_m.y, pw.y * lam_m.x));
+            }
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb, 1024)) = pack8f(r, 1.f);
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb + 8, 1024)) = pack8f(r + 8, 1.f);
+          }
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(rdyW);
+          if (!(ok = waitB(dneW, pW))) break;   // G_W(t): a~~ = W' a in the a~ columns
+          // E2b(t): X = conj(lambda^(i-c)) a~~
+          pw = p_start;
+#pragma unroll
+          for (int bb = 0; bb < 2; ++bb) {
+            uint32_t r[16];
+            tmem_ld16(trow + K::T_A + i0 + 16 * bb, r);
+            tmem_ld_wait16(r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x = __uint_as_float(r[e]);
+              const float y = __shfl_xor_sync(kFull, x, 1);
+              r[e] = __float_as_uint(fmaf(pw.x, x, -sg * pw.y * y));
+              pw = make_float2(fmaf(pw.x, lam_m.x, -pw.y * lam_m.y), fmaf(pw.x, lam_m.y, pw.y * lam_m.x));
+            }
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb, 1024)) = pack8f(r, 1.f);
+            *reinterpret_cast<uint4*>(smem + K::S_X + tile_off(k, i0 + 16 * bb + 8, 1024)) = pack8f(r + 8, 1.f);
+          }
+          signalB(2);
+        } else {  // E2(t): X = |lambda|^(2(i-c)) a~
           uint64_t s2 = f2_pack(s_start, s_start * r2);   // scales of two adjacent columns
           const uint64_t r4 = f2_pack(r2 * r2, r2 * r2);
 #pragma unroll
@@ -1328,10 +1404,10 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
     if (tid == GT) bulk_wait_all();   // o is in global memory before the block exits
 }
 
-template <int DX>
+template <int DX, bool RW>
 __device__ __noinline__ void tc_role_fetch(const TcArgs& a, uint8_t* smem, int h_first, const CUtensorMap& tm_q,
                                          const CUtensorMap& tm_k, const CUtensorMap& tm_v) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int NB = K::NB;
   const int tid = threadIdx.x, lane = tid & 31;
   const Sched sc(a.total, a.G, blockIdx.x, a.nch);
@@ -1390,12 +1466,12 @@ __device__ __noinline__ void tc_role_fetch(const TcArgs& a, uint8_t* smem, int h
 
 // 576 threads: one SM sub-partition carries five of the 18 warps, so its
 // 16 K registers cap a thread at 96.
-template <int DX>
+template <int DX, bool RW>
 __global__ void __launch_bounds__(NTH, 1)
     tc_prefill_kernel(const __grid_constant__ TcArgs a, const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   constexpr int NB = K::NB;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -1416,7 +1492,9 @@ __global__ void __launch_bounds__(NTH, 1)
   // fp16 operands.  A set is refilled only after that G7, so no barrier runs
   // a phase ahead of the MMA warp's wait.
   uint64_t* rdyKV = bars + 19;
-  static_assert(NB <= 3 && (22 + 3) * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
+  uint64_t* rdyW = bars + 25;     // output warps -> G_W (the readout's input a staged), RW only
+  uint64_t* dneW = bars + 26;     // G_W done
+  static_assert(NB <= 3 && 27 * 8 <= K::S_FLAG - K::S_BAR, "the mbarriers fit their slot");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + K::S_FLAG);
   volatile int* xchg = reinterpret_cast<volatile int*>(smem + K::S_FLAG + 4);   // look-back result
   // G4 groups known done: the output warps see each G4 complete, in order,
@@ -1449,6 +1527,8 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     mbar_init(bar_drain, 1);
     for (int i = 0; i < NB; ++i) mbar_init(rdyKV + i, GT);
+    mbar_init(rdyW, GT);
+    mbar_init(dneW, 1);
     *abort_flag = 0;
     *g4_seen = 0;
     fence_barrier_init();
@@ -1487,16 +1567,21 @@ __global__ void __launch_bounds__(NTH, 1)
     const uint4* src = reinterpret_cast<const uint4*>(a.tabs[h_first].E);
     uint4* dst = reinterpret_cast<uint4*>(smem + K::S_E);
     for (int i = tid; i < KR * C * 2 / 16; i += NTH) dst[i] = src[i];
+    if constexpr (RW) {
+      const uint4* ws = reinterpret_cast<const uint4*>(a.Wt) + static_cast<size_t>(h_first) * (kWprimeBytes / 16);
+      uint4* wd = reinterpret_cast<uint4*>(smem + K::S_W);
+      for (int i = tid; i < static_cast<int>(kWprimeBytes / 16); i += NTH) wd[i] = ws[i];
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (role == 2) tc_role_mma<DX>(a, smem, h_first);
-  else if (role == 0) tc_role_prepare<DX>(a, smem, h_first);
-  else if (role == 1) tc_role_output<DX>(a, smem, h_first, tm_o);
-  else tc_role_fetch<DX>(a, smem, h_first, tm_q, tm_k, tm_v);
+  if (role == 2) tc_role_mma<DX, RW>(a, smem, h_first);
+  else if (role == 0) tc_role_prepare<DX, RW>(a, smem, h_first);
+  else if (role == 1) tc_role_output<DX, RW>(a, smem, h_first, tm_o);
+  else tc_role_fetch<DX, RW>(a, smem, h_first, tm_q, tm_k, tm_v);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1524,17 +1609,17 @@ double plan_cost(long long total, int nch, int G) {
   return worst;
 }
 
-template <int DX>
+template <int DX, bool RW>
 cudaError_t launch_impl(const TcArgs& args, const void* q, const void* k, const void* v, int DV,
                         cudaStream_t st) {
-  using K = PCfg<DX>;
+  using K = PCfg<DX, RW>;
   CUtensorMap tm_q, tm_k, tm_v, tm_o;
   const bool f16 = args.kv_ready != 0;
   if (!encode_input_map(&tm_q, q, args.BH, args.N, DX) || !encode_input_map(&tm_k, k, args.BH, args.N, DX, f16) ||
       !encode_input_map(&tm_v, v, args.BH, args.N, DV, f16) ||
       !encode_rows64_f32_map(&tm_o, args.o, args.BH, args.N, DV))
     return cudaErrorNotSupported;
-  auto kern = tc_prefill_kernel<DX>;
+  auto kern = tc_prefill_kernel<DX, RW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, K::SMEM);
   if (e != cudaSuccess) return e;
   // Programmatic dependent launch: the CTAs set up barriers, TMEM and
@@ -1622,13 +1707,14 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
                               const void* v, const float* delta, const float* A,
                               const void* state_in, float* o, float* num, float* den,
                               void* state_out, void* ws, cudaStream_t st, void* dump_R,
-                              float* dump_Re, float* dtab, bool kv_ready) {
+                              float* dump_Re, float* dtab, bool kv_ready, const void* Wt) {
   uint8_t* w = reinterpret_cast<uint8_t*>(tc_tables(ws));
   HeadTables* tabs = reinterpret_cast<HeadTables*>(w);
   TcArgs args;
   args.agg = args.incl = nullptr;
   args.flags = nullptr;
   args.kv_ready = kv_ready ? 1 : 0;
+  args.Wt = static_cast<const __half*>(Wt);
   const size_t F = static_cast<size_t>(s.d_xi) + kVB;
   if (tc_plan_splits(s, p)) {
     float* agg = reinterpret_cast<float*>(w + sizeof(HeadTables) * s.H);
@@ -1661,8 +1747,12 @@ cudaError_t launch_tc_prefill(const ia_shape_t& s, const TcPlan& p, const void* 
   args.G = p.grid;
   args.BH = static_cast<long long>(s.B) * s.H;
   args.total = args.BH * args.nvb * args.nch;
-  if (s.d_xi == 64) return launch_impl<64>(args, q, k, v, s.d_v, st);
-  if (s.d_xi == 128) return launch_impl<128>(args, q, k, v, s.d_v, st);
+  if (Wt) {   // the readout matrix: d_xi = 64, no saved states
+    if (s.d_xi != 64 || dump_R) return cudaErrorInvalidValue;
+    return launch_impl<64, true>(args, q, k, v, s.d_v, st);
+  }
+  if (s.d_xi == 64) return launch_impl<64, false>(args, q, k, v, s.d_v, st);
+  if (s.d_xi == 128) return launch_impl<128, false>(args, q, k, v, s.d_v, st);
   return cudaErrorInvalidValue;
 }
 

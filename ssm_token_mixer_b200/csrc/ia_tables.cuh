@@ -41,4 +41,14 @@ __host__ __device__ constexpr uint32_t etab_offset(int k, int j) {
   return static_cast<uint32_t>((k >> 3) * 1024 + (j >> 3) * 128 + (k & 7) * 16 + (j & 7) * 2);
 }
 
+// The complex readout matrix W_h [M x M] as the real [2M x 2M] matrix W' of
+// rows k = 2m + {0: re, 1: im} and columns k' = 2m' + {0, 1}
+// (W'[2m][2m'] = W'[2m+1][2m'+1] = Re W[m][m'], W'[2m][2m'+1] = -Im W[m][m'],
+// W'[2m+1][2m'] = Im W[m][m']), fp16 in the no-swizzle K-major core-matrix
+// layout with K = 2M: byte (k/8)*2048 + (k'/8)*128 + (k%8)*16 + (k'%8)*2.
+constexpr uint32_t kWprimeBytes = 2 * kModesTC * 2 * kModesTC * 2;
+__host__ __device__ constexpr uint32_t wprime_offset(int k, int kp) {
+  return static_cast<uint32_t>((k >> 3) * 2048 + (kp >> 3) * 128 + (k & 7) * 16 + (kp & 7) * 2);
+}
+
 }  // namespace ia

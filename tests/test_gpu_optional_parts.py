@@ -163,7 +163,9 @@ def test_optional_parts_paths_and_workspace(dev):
     tc = lambda **kw: ia.prefill_ex_path(B, H, N, 64, 64, 64, "bf16", **kw)
     assert tc() == "tensor_core"
     assert tc(norm=True) == tc(bidirectional=True) == tc(norm=True, bidirectional=True) == "tensor_core"
-    assert tc(selective=True) == tc(readout=True) == tc(norm=True, readout=True) == "sequential"
+    assert tc(readout=True) == tc(norm=True, readout=True) == tc(readout=True, bidirectional=True) == "tensor_core"
+    assert tc(selective=True) == tc(selective=True, readout=True) == "sequential"
+    assert ia.prefill_ex_path(B, H, N, 128, 128, 64, "bf16", readout=True) == "sequential"   # d_xi = 128
     assert ia.prefill_ex_path(B, H, N, 64, 64, 48, "bf16", norm=True) == "sequential"    # M != 64
     assert ia.prefill_ex_path(B, H, N, 64, 64, 64, "f32", norm=True) == "sequential"     # fp32 inputs
     # a workspace one byte short is refused before anything runs
@@ -269,3 +271,51 @@ def test_segmented_bidirectional_layer(oracle_mod, dev):
     ia.check_device_errors()
     ref = oracle_mod.forward_bidirectional(inp["q"], inp["k"], inp["v"], M, **to_oracle(opt))
     assert slice_rel(r["o"].cpu(), ref, (-2, -1)) < TOL_F32
+
+
+TC_W_CASES = [("readout",), ("norm", "readout"), ("readout", "bidirectional")]
+
+
+@pytest.mark.parametrize("which", TC_W_CASES, ids=["+".join(c) for c in TC_W_CASES])
+@pytest.mark.parametrize("dv", [64, 128])
+def test_tensor_core_readout_matrix(oracle_mod, dev, which, dv):
+    # the readout matrix on the chunk pass (G_W between the key-state read and
+    # the score matrix), d_xi = 64, a ragged N over several chunks, with the
+    # stabilisation or the bidirectional layer beside it: o, num, den and the
+    # end state against the oracle
+    B, H, N, dx, M = 2, 3, 333, 64, 64
+    bidir = "bidirectional" in which
+    inp = synthetic.layer_inputs(B, H, N, dx, dv, "bf16", seed=97 + dv)
+    opt = options(B, H, N, dx, dv, M, 98, which)
+    present = dict(norm="gain" in opt, readout=True, bidirectional=bidir)
+    assert ia.prefill_ex_path(B, H, N, dx, dv, M, "bf16", **present) == "tensor_core"
+    g = lambda x: x.to(dev)
+    r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta=g(inp["delta"]), bidirectional=bidir,
+                          want_num_den=not bidir, want_state=not bidir, **{k: g(v) for k, v in opt.items()})
+    ia.check_device_errors()
+    if bidir:
+        ref = oracle_mod.forward_bidirectional(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **to_oracle(opt))
+        assert slice_rel(r["o"].cpu(), ref, (-2, -1)) < TOL_BF16
+        return
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **to_oracle(opt))
+    rep = report(r["num"].cpu(), r["den"].cpu(), r["o"].cpu(), ref)
+    assert max(rep.values()) < TOL_BF16, rep
+    st = r["state"].cpu().double().numpy()
+    assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < TOL_BF16
+
+
+def test_tensor_core_readout_matrix_across_heads_and_ranges(oracle_mod, dev, monkeypatch):
+    # forced grids put several heads in one CTA (W' reloaded per head) and
+    # start ranges inside streams (look-back; the state-only chain reads no W)
+    B, H, N, d, M = 1, 4, 700, 64, 64
+    inp = synthetic.layer_inputs(B, H, N, d, d, "bf16", seed=99)
+    opt = options(B, H, N, d, d, M, 100, ("readout",))
+    ref = oracle_mod.forward_ex(inp["q"], inp["k"], inp["v"], M, delta=inp["delta"], **to_oracle(opt))
+    g = lambda x: x.to(dev)
+    for grid in ("1", "3", "7"):
+        monkeypatch.setenv("IA_PREFILL_GRID", grid)
+        r = ia.prefill_fwd_ex(g(inp["q"]), g(inp["k"]), g(inp["v"]), M, delta=g(inp["delta"]), want_num_den=True,
+                              W=g(opt["W"]))
+        ia.check_device_errors()
+        rep = report(r["num"].cpu(), r["den"].cpu(), r["o"].cpu(), ref)
+        assert max(rep.values()) < TOL_BF16, (grid, rep)
