@@ -1,5 +1,6 @@
-// The layer with its optional parts, on CUDA cores in fp32 (one CTA per (b,h),
-// token after token), behind ia_prefill_fwd_ex and ia_decode_step_ex.
+// The layer with its optional parts, on CUDA cores in fp32 (one CTA per
+// segment of a (b,h), token after token), behind ia_prefill_fwd_ex where its
+// tensor-core form does not apply, and behind ia_decode_step_ex.
 //
 // The optional parts are the ones the pages name beside the plain layer
 // (paper 'Interdomain Attention: Beyond Token-Level Key-Value Memory'):

@@ -1331,7 +1331,7 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
           // (rows 2m and 2m+1 sit in adjacent lanes)
           const float sg = (k & 1) ? 1.f : -1.f;
           float2 pw = p_start;
-#pragma unroll
+#pragma unroll 1
           for (int bb = 0; bb < 2; ++bb) {
             uint32_t r[16];
             tmem_ld16(trow + K::T_A + i0 + 16 * bb, r);
@@ -1352,7 +1352,7 @@ __device__ __noinline__ void tc_role_output(const TcArgs& a, uint8_t* smem, int 
           if (!(ok = waitB(dneW, pW))) break;   // G_W(t): a~~ = W' a in the a~ columns
           // E2b(t): X = conj(lambda^(i-c)) a~~
           pw = p_start;
-#pragma unroll
+#pragma unroll 1
           for (int bb = 0; bb < 2; ++bb) {
             uint32_t r[16];
             tmem_ld16(trow + K::T_A + i0 + 16 * bb, r);
