@@ -350,6 +350,236 @@ __global__ void __launch_bounds__(256, 3) seq_fwd_ex_kernel(int H, int N, int DX
   }
 }
 
+// Register-resident form for d_xi = d_v = M = 64 (the same arithmetic, the
+// same segments and passes): 16 warps, warp w owning modes 4w .. 4w+3 and
+// lane l the state columns 2l, 2l+1 of U and Gamma in registers (every lane
+// keeps its warp's four eta), so that the state does not pass through shared
+// memory every token.  Warps 0-3 stage the token's z and xi(q) (and threads
+// 0-63 its lambda_t, b_t) in shared memory, double-buffered by token parity:
+// one block barrier per token orders the update, a second one the sum of the
+// warps' partial num and den (a third, with W, the exchange of a).
+constexpr int kRegWarps = 16, kRegModes = 4, kRegD = 64, kRegM = 64;
+
+bool ex_reg_form(const ia_shape_t& s) { return s.d_xi == kRegD && s.d_v == kRegD && s.M == kRegM; }
+
+template <typename T>
+__global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, int N, const T* __restrict__ q,
+                                                                        const T* __restrict__ k,
+                                                                        const T* __restrict__ v, const ExArgs a,
+                                                                        long long BH) {
+  constexpr int DX = kRegD, DV = kRegD, M = kRegM, D = DX + DV;
+  __shared__ __align__(16) float zs[2][D];     // xi(k) | v, normalised when asked
+  __shared__ __align__(16) float qs[2][DX];    // xi(q)
+  __shared__ float2 lamS[2][M], bS[2][M];
+  __shared__ float2 aS[M];                     // a, for the readout matrix
+  __shared__ __align__(16) float part[2][kRegWarps][DV];
+  __shared__ float dpart[2][kRegWarps];
+  __shared__ float red[4];
+  extern __shared__ float4 wsm[];              // W_h [M*M] (float2), when given and reading out
+  float2* Ws = reinterpret_cast<float2*>(wsm);
+
+  const long long bh = blockIdx.x / a.nseg;
+  const int sg = static_cast<int>(blockIdx.x - bh * a.nseg);
+  const int h = static_cast<int>(bh % H);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int step0 = sg * a.seg_len, step1 = min(N, step0 + a.seg_len);
+  const bool readout = a.pass != 1;
+  if (!readout && sg == a.nseg - 1) return;   // pass 1: the last segment's end state is not needed
+  constexpr int SW = M * (DX + DV + 1);
+  const int m0 = warp * kRegModes, f0 = 2 * lane;
+  const bool norm = a.gain || a.bias;
+
+  // this thread's state entries: (public layout for segment 0, else the slot)
+  float2 U[kRegModes][2], G[kRegModes][2], E[kRegModes];
+  {
+    const float2* su = nullptr;
+    const float2* sgm = nullptr;
+    const float2* se = nullptr;
+    if (sg == 0 && a.state_in) {
+      su = a.state_in + bh * M * DX;
+      sgm = a.state_in + BH * M * DX + bh * M * DV;
+      se = a.state_in + BH * M * (DX + DV) + bh * M;
+    } else if (sg > 0 && readout) {
+      const float2* slot = a.seg + (bh * (a.nseg - 1) + (sg - 1)) * SW;
+      su = slot;
+      sgm = slot + M * DX;
+      se = slot + M * (DX + DV);
+    }
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const int m = m0 + u;
+      float4 x = su ? *reinterpret_cast<const float4*>(su + m * DX + f0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      U[u][0] = make_float2(x.x, x.y);
+      U[u][1] = make_float2(x.z, x.w);
+      x = sgm ? *reinterpret_cast<const float4*>(sgm + m * DV + f0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      G[u][0] = make_float2(x.x, x.y);
+      G[u][1] = make_float2(x.z, x.w);
+      E[u] = se ? se[m] : make_float2(0.f, 0.f);
+    }
+  }
+  if (a.W && readout) {
+    const float2* Wg = reinterpret_cast<const float2*>(a.W) + static_cast<long long>(h) * M * M;
+    for (int i = tid; i < M * M; i += kRegWarps * 32) Ws[i] = Wg[i];
+  }
+  // thread m < M: its mode's A; lambda, b once for a constant step
+  float m_ar = -0.5f, m_ai = 0.f;
+  if (tid < M) {
+    m_ar = a.A ? a.A[2 * tid] : -0.5f;
+    m_ai = a.A ? a.A[2 * tid + 1] : 3.14159265358979323846f * static_cast<float>(tid);
+    if (!a.delta_t) {
+      const ModeD md = mode_consts(delta_hm(a.delta, a.dpm, M, h, tid), a.A, tid);
+      const float2 l = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
+      const float2 b = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
+      lamS[0][tid] = lamS[1][tid] = l;
+      bS[0][tid] = bS[1][tid] = b;
+    }
+  }
+  const T* qb = q + bh * N * DX;
+  const T* kb = k + bh * N * DX;
+  const T* vb = v + bh * N * DV;
+  // the next token's inputs, loaded while this one is processed
+  float rz = 0.f, rq = 0.f, rdt = 0.f;
+  auto fetch = [&](int tt) {
+    if (tid < DX) {
+      rz = ldf(kb + static_cast<long long>(tt) * DX + tid);
+      rq = ldf(qb + static_cast<long long>(tt) * DX + tid);
+    } else if (tid < D) {
+      rz = ldf(vb + static_cast<long long>(tt) * DV + (tid - DX));
+    }
+    if (a.delta_t && tid < M) rdt = a.delta_t[bh * N + tt];
+  };
+  double dt_sum = 0.0;
+  if (step1 > step0) fetch(a.reverse ? N - 1 - step0 : step0);
+  for (int step = step0; step < step1; ++step) {
+    const int t = a.reverse ? N - 1 - step : step;
+    const int p = (step - step0) & 1;
+    if (tid < D) {   // warps 0-3: z_t and xi(q_t)
+      float x = tid < DX ? feat_acc(rz) : rz;
+      if (norm) {
+        const float ss = warp_sum(x * x);
+        if (lane == 0) red[warp] = ss;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const float r = rsqrtf((red[0] + red[1] + red[2] + red[3]) / static_cast<float>(D) + a.eps);
+        const float g = a.gain ? a.gain[static_cast<long long>(h) * D + tid] : 1.f;
+        const float c = a.bias ? a.bias[static_cast<long long>(h) * D + tid] : 0.f;
+        x = fmaf(x * r, g, c);
+      }
+      zs[p][tid] = x;
+      if (tid < DX) qs[p][tid] = feat_acc(rq);
+    }
+    if (a.delta_t && tid < M) {   // lambda_t, b_t as in the decode step (b through expm1)
+      const float x = rdt * m_ar, y = rdt * m_ai;
+      float sy, cy, sh, ch;
+      sincosf(y, &sy, &cy);
+      sincosf(0.5f * y, &sh, &ch);
+      const float ex = expf(x), em1 = expm1f(x);
+      const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;
+      const float dd = fmaf(m_ar, m_ar, m_ai * m_ai);
+      lamS[p][tid] = make_float2(ex * cy, ex * sy);
+      bS[p][tid] = make_float2(fmaf(nr, m_ar, ni * m_ai) / dd, fmaf(ni, m_ar, -nr * m_ai) / dd);
+      if (tid == 0) dt_sum += rdt;
+    }
+    if (step + 1 < step1) fetch(a.reverse ? N - 2 - step : step + 1);
+    __syncthreads();
+    // the update, and this lane's part of a = U xi(q) for the warp's modes
+    const float2 zk = *reinterpret_cast<const float2*>(&zs[p][f0]);
+    const float2 zv = *reinterpret_cast<const float2*>(&zs[p][DX + f0]);
+    const float2 zq = *reinterpret_cast<const float2*>(&qs[p][f0]);
+    float ar[kRegModes], ai[kRegModes];
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const float2 L = lamS[p][m0 + u], B = bS[p][m0 + u];
+      U[u][0] = cfma(L, U[u][0], make_float2(B.x * zk.x, B.y * zk.x));
+      U[u][1] = cfma(L, U[u][1], make_float2(B.x * zk.y, B.y * zk.y));
+      G[u][0] = cfma(L, G[u][0], make_float2(B.x * zv.x, B.y * zv.x));
+      G[u][1] = cfma(L, G[u][1], make_float2(B.x * zv.y, B.y * zv.y));
+      E[u] = cfma(L, E[u], B);
+      ar[u] = fmaf(U[u][0].x, zq.x, U[u][1].x * zq.y);
+      ai[u] = fmaf(U[u][0].y, zq.x, U[u][1].y * zq.y);
+    }
+    if (!readout) continue;   // pass 1: the state only (uniform over the block)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int u = 0; u < kRegModes; ++u) {
+        ar[u] += __shfl_xor_sync(0xffffffffu, ar[u], off);
+        ai[u] += __shfl_xor_sync(0xffffffffu, ai[u], off);
+      }
+    }
+    if (a.W) {   // a~ = W_h a: every warp needs all of a
+      if (lane == 0) {
+#pragma unroll
+        for (int u = 0; u < kRegModes; ++u) aS[m0 + u] = make_float2(ar[u], ai[u]);
+      }
+      __syncthreads();
+      const float2 a0 = aS[f0], a1 = aS[f0 + 1];
+#pragma unroll
+      for (int u = 0; u < kRegModes; ++u) {
+        const float4 w = *reinterpret_cast<const float4*>(Ws + (m0 + u) * M + f0);   // W[m][2l], W[m][2l+1]
+        ar[u] = fmaf(w.x, a0.x, fmaf(-w.y, a0.y, fmaf(w.z, a1.x, -w.w * a1.y)));
+        ai[u] = fmaf(w.x, a0.y, fmaf(w.y, a0.x, fmaf(w.z, a1.y, w.w * a1.x)));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+        for (int u = 0; u < kRegModes; ++u) {
+          ar[u] += __shfl_xor_sync(0xffffffffu, ar[u], off);
+          ai[u] += __shfl_xor_sync(0xffffffffu, ai[u], off);
+        }
+      }
+    }
+    // this lane's two columns of num over the warp's modes, and den
+    float n0 = 0.f, n1 = 0.f, dn = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const float2 at = make_float2(ar[u], ai[u]);
+      n0 += re_conj_mul(at, G[u][0]);
+      n1 += re_conj_mul(at, G[u][1]);
+      dn += re_conj_mul(at, E[u]);
+    }
+    *reinterpret_cast<float2*>(&part[p][warp][f0]) = make_float2(n0, n1);
+    if (lane == 0) dpart[p][warp] = dn;
+    __syncthreads();
+    if (tid < DV) {
+      float nf = 0.f, d = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRegWarps; ++w) {
+        nf += part[p][w][tid];
+        d += dpart[p][w];
+      }
+      const long long row = bh * N + t;
+      const float of = nf / d;
+      a.o[row * DV + tid] = a.accumulate ? a.o[row * DV + tid] + of : of;
+      if (a.num) a.num[row * DV + tid] = nf;
+      if (a.den && tid == 0) a.den[row] = d;
+    }
+  }
+  // end state: pass 1 into this segment's slot, else the last segment's state_out
+  float2* du = nullptr;
+  float2* dg = nullptr;
+  float2* de = nullptr;
+  if (!readout) {
+    float2* slot = a.seg + (bh * (a.nseg - 1) + sg) * SW;
+    du = slot;
+    dg = slot + M * DX;
+    de = slot + M * (DX + DV);
+    if (tid == 0 && a.dsum) a.dsum[bh * a.nseg + sg] = dt_sum;
+  } else if (a.state_out && sg == a.nseg - 1) {
+    du = a.state_out + bh * M * DX;
+    dg = a.state_out + BH * M * DX + bh * M * DV;
+    de = a.state_out + BH * M * (DX + DV) + bh * M;
+  }
+  if (du) {
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const int m = m0 + u;
+      *reinterpret_cast<float4*>(du + m * DX + f0) = make_float4(U[u][0].x, U[u][0].y, U[u][1].x, U[u][1].y);
+      *reinterpret_cast<float4*>(dg + m * DV + f0) = make_float4(G[u][0].x, G[u][0].y, G[u][1].x, G[u][1].y);
+      if (lane == 0) de[m] = E[u];
+    }
+  }
+}
+
 // Turns the pass-1 end states into the states entering each segment, per
 // (b,h) and mode: slot 0 already is the state entering segment 1 (segment 0
 // started from state_in); slot s (s >= 1) becomes Lambda_s slot(s-1) +
@@ -404,6 +634,16 @@ size_t ex_launch_smem(const ia_shape_t& s, bool with_w, bool* w_smem) {
 template <typename T>
 cudaError_t launch_ex(const ia_shape_t& s, int N, const void* q, const void* k, const void* v, const ExArgs& a,
                       cudaStream_t st) {
+  const long long BH = static_cast<long long>(s.B) * s.H;
+  if (ex_reg_form(s)) {
+    const size_t wsm = a.W && a.pass != 1 ? sizeof(float2) * kRegM * kRegM : 0;
+    auto kern = seq_ex_reg_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(wsm));
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(BH * a.nseg), kRegWarps * 32, wsm, st>>>(
+        s.H, N, static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), a, BH);
+    return cudaGetLastError();
+  }
   ExArgs args = a;
   bool ws = false;
   const size_t smem = ex_launch_smem(s, a.W && a.pass != 1, &ws);
@@ -411,7 +651,6 @@ cudaError_t launch_ex(const ia_shape_t& s, int N, const void* q, const void* k, 
   auto kern = seq_fwd_ex_kernel<T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const long long BH = static_cast<long long>(s.B) * s.H;
   kern<<<static_cast<unsigned>(BH * args.nseg), kExThreads, smem, st>>>(
       s.H, N, s.d_xi, s.d_v, s.M, static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), args,
       BH);
@@ -426,6 +665,7 @@ cudaError_t launch_ex_any(const ia_shape_t& s, int N, const void* q, const void*
 
 // CTAs of the reading-out launch resident per SM (1 when no device answers)
 int ex_resident(const ia_shape_t& s, bool with_w) {
+  if (ex_reg_form(s)) return 1;   // 512 threads of up to 128 registers
   bool ws = false;
   const size_t smem = ex_launch_smem(s, with_w, &ws);
   const void* fn = s.in_dtype == IA_F32 ? reinterpret_cast<const void*>(seq_fwd_ex_kernel<float>)

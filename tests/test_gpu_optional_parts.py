@@ -63,10 +63,12 @@ def test_prefill_with_optional_parts(oracle_mod, dev, which, dtype, dx, dv, M, t
     assert np.abs(st - ref["state"]).max() / np.abs(ref["state"]).max() < tol
 
 
-def test_split_prefill_and_decode_with_optional_parts(oracle_mod, dev):
+@pytest.mark.parametrize("dx,dv,M", [(16, 16, 8), (64, 64, 64)], ids=["small", "register_form"])
+def test_split_prefill_and_decode_with_optional_parts(oracle_mod, dev, dx, dv, M):
     # P12/P13 with every part on: prefill(N1) -> state -> prefill(N2) and
-    # decode steps equal the oracle on the whole sequence
-    B, H, dx, dv, M, N1, N2, K = 2, 2, 16, 16, 8, 70, 40, 3
+    # decode steps equal the oracle on the whole sequence (d_xi = d_v = M =
+    # 64: the register-resident kernel, also for the in-place decode step)
+    B, H, N1, N2, K = 2, 2, 70, 140, 3
     N = N1 + N2 + K
     inp = synthetic.layer_inputs(B, H, N, dx, dv, "f32", seed=82)
     opt = options(B, H, N, dx, dv, M, 83, ("selective", "norm", "readout"))
@@ -219,13 +221,15 @@ SEG_CASES = [("selective", "norm", "readout"), ("readout",), ("norm",)]
 
 
 @pytest.mark.parametrize("which", SEG_CASES, ids=["+".join(c) for c in SEG_CASES])
-def test_segmented_token_serial_pass(oracle_mod, dev, which):
+@pytest.mark.parametrize("dx,dv,M", [(16, 12, 8), (64, 64, 64)], ids=["small", "register_form"])
+def test_segmented_token_serial_pass(oracle_mod, dev, which, dx, dv, M):
     # The token-serial form cuts 357 tokens into five segments (the last one
     # ragged) around the carry kernel, from the state a 50-token prefix left,
     # with a general A and, without a step per token, a Delta per (head, mode):
     # o and the end state against the oracle on the whole sequence, and o
-    # against the single pass that a one-byte workspace leaves
-    B, H, P, N, dx, dv, M = 1, 2, 50, 357, 16, 12, 8
+    # against the single pass that a one-byte workspace leaves.  d_xi = d_v =
+    # M = 64 runs the register-resident kernel.
+    B, H, P, N = 1, 2, 50, 357
     inp = synthetic.layer_inputs(B, H, P + N, dx, dv, "f32", seed=88)
     opt = options(B, H, P + N, dx, dv, M, 89, which)
     delta, A = mode_params(H, M, 90)
