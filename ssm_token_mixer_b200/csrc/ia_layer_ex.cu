@@ -354,10 +354,11 @@ __global__ void __launch_bounds__(256, 3) seq_fwd_ex_kernel(int H, int N, int DX
 // same segments and passes): 16 warps, warp w owning modes 4w .. 4w+3 and
 // lane l the state columns 2l, 2l+1 of U and Gamma in registers (every lane
 // keeps its warp's four eta), so that the state does not pass through shared
-// memory every token.  Warps 0-3 stage the token's z and xi(q) (and threads
-// 0-63 its lambda_t, b_t) in shared memory, double-buffered by token parity:
-// one block barrier per token orders the update, a second one the sum of the
-// warps' partial num and den (a third, with W, the exchange of a).
+// memory every token.  Warps 0-3 stage the token's z and xi(q), warps 4-5 its
+// lambda_t, b_t, in shared memory, double-buffered by token parity: one block
+// barrier per token orders the update, a second one the sum of the warps'
+// partial num and den (a third, with W, the exchange of a), which warps 14-15
+// finish while warps 0-5 stage the next token.
 constexpr int kRegWarps = 16, kRegModes = 4, kRegD = 64, kRegM = 64;
 
 bool ex_reg_form(const ia_shape_t& s) { return s.d_xi == kRegD && s.d_v == kRegD && s.M == kRegM; }
@@ -421,17 +422,20 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     const float2* Wg = reinterpret_cast<const float2*>(a.W) + static_cast<long long>(h) * M * M;
     for (int i = tid; i < M * M; i += kRegWarps * 32) Ws[i] = Wg[i];
   }
-  // thread m < M: its mode's A; lambda, b once for a constant step
+  // warps 4-5 (mode pm = tid - 128): its A; lambda, b once for a constant step
+  constexpr int kParamT0 = 4 * 32, kSumT0 = kRegWarps * 32 - DV;
+  const int pm = tid - kParamT0;
+  const bool param_thread = pm >= 0 && pm < M;
   float m_ar = -0.5f, m_ai = 0.f;
-  if (tid < M) {
-    m_ar = a.A ? a.A[2 * tid] : -0.5f;
-    m_ai = a.A ? a.A[2 * tid + 1] : 3.14159265358979323846f * static_cast<float>(tid);
+  if (param_thread) {
+    m_ar = a.A ? a.A[2 * pm] : -0.5f;
+    m_ai = a.A ? a.A[2 * pm + 1] : 3.14159265358979323846f * static_cast<float>(pm);
     if (!a.delta_t) {
-      const ModeD md = mode_consts(delta_hm(a.delta, a.dpm, M, h, tid), a.A, tid);
+      const ModeD md = mode_consts(delta_hm(a.delta, a.dpm, M, h, pm), a.A, pm);
       const float2 l = make_float2(static_cast<float>(md.lr), static_cast<float>(md.li));
       const float2 b = make_float2(static_cast<float>(md.br), static_cast<float>(md.bi));
-      lamS[0][tid] = lamS[1][tid] = l;
-      bS[0][tid] = bS[1][tid] = b;
+      lamS[0][pm] = lamS[1][pm] = l;
+      bS[0][pm] = bS[1][pm] = b;
     }
   }
   const T* qb = q + bh * N * DX;
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     } else if (tid < D) {
       rz = ldf(vb + static_cast<long long>(tt) * DV + (tid - DX));
     }
-    if (a.delta_t && tid < M) rdt = a.delta_t[bh * N + tt];
+    if (a.delta_t && param_thread) rdt = a.delta_t[bh * N + tt];
   };
   double dt_sum = 0.0;
   if (step1 > step0) fetch(a.reverse ? N - 1 - step0 : step0);
@@ -467,7 +471,7 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
       zs[p][tid] = x;
       if (tid < DX) qs[p][tid] = feat_acc(rq);
     }
-    if (a.delta_t && tid < M) {   // lambda_t, b_t as in the decode step (b through expm1)
+    if (a.delta_t && param_thread) {   // lambda_t, b_t as in the decode step (b through expm1)
       const float x = rdt * m_ar, y = rdt * m_ai;
       float sy, cy, sh, ch;
       sincosf(y, &sy, &cy);
@@ -475,9 +479,9 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
       const float ex = expf(x), em1 = expm1f(x);
       const float nr = fmaf(em1, cy, -2.f * sh * sh), ni = ex * sy;
       const float dd = fmaf(m_ar, m_ar, m_ai * m_ai);
-      lamS[p][tid] = make_float2(ex * cy, ex * sy);
-      bS[p][tid] = make_float2(fmaf(nr, m_ar, ni * m_ai) / dd, fmaf(ni, m_ar, -nr * m_ai) / dd);
-      if (tid == 0) dt_sum += rdt;
+      lamS[p][pm] = make_float2(ex * cy, ex * sy);
+      bS[p][pm] = make_float2(fmaf(nr, m_ar, ni * m_ai) / dd, fmaf(ni, m_ar, -nr * m_ai) / dd);
+      if (pm == 0) dt_sum += rdt;
     }
     if (step + 1 < step1) fetch(a.reverse ? N - 2 - step : step + 1);
     __syncthreads();
@@ -540,18 +544,19 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     *reinterpret_cast<float2*>(&part[p][warp][f0]) = make_float2(n0, n1);
     if (lane == 0) dpart[p][warp] = dn;
     __syncthreads();
-    if (tid < DV) {
+    if (tid >= kSumT0) {   // warps 14-15: column f of num, den, o
+      const int f = tid - kSumT0;
       float nf = 0.f, d = 0.f;
 #pragma unroll
       for (int w = 0; w < kRegWarps; ++w) {
-        nf += part[p][w][tid];
+        nf += part[p][w][f];
         d += dpart[p][w];
       }
       const long long row = bh * N + t;
       const float of = nf / d;
-      a.o[row * DV + tid] = a.accumulate ? a.o[row * DV + tid] + of : of;
-      if (a.num) a.num[row * DV + tid] = nf;
-      if (a.den && tid == 0) a.den[row] = d;
+      a.o[row * DV + f] = a.accumulate ? a.o[row * DV + f] + of : of;
+      if (a.num) a.num[row * DV + f] = nf;
+      if (a.den && f == 0) a.den[row] = d;
     }
   }
   // end state: pass 1 into this segment's slot, else the last segment's state_out
@@ -563,7 +568,7 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     du = slot;
     dg = slot + M * DX;
     de = slot + M * (DX + DV);
-    if (tid == 0 && a.dsum) a.dsum[bh * a.nseg + sg] = dt_sum;
+    if (pm == 0 && a.dsum) a.dsum[bh * a.nseg + sg] = dt_sum;
   } else if (a.state_out && sg == a.nseg - 1) {
     du = a.state_out + bh * M * DX;
     dg = a.state_out + BH * M * DX + bh * M * DV;
