@@ -355,10 +355,10 @@ __global__ void __launch_bounds__(256, 3) seq_fwd_ex_kernel(int H, int N, int DX
 // lane l the state columns 2l, 2l+1 of U and Gamma in registers (every lane
 // keeps its warp's four eta), so that the state does not pass through shared
 // memory every token.  Warps 0-3 stage the token's z and xi(q), warps 4-5 its
-// lambda_t, b_t, in shared memory, double-buffered by token parity: one block
-// barrier per token orders the update, a second one the sum of the warps'
-// partial num and den (a third, with W, the exchange of a), which warps 14-15
-// finish while warps 0-5 stage the next token.
+// lambda_t, b_t, in shared memory, double-buffered by token parity, and so are
+// the warps' partial num and den: one block barrier per token orders the
+// update (a second, with W, the exchange of a), and warps 14-15 sum the
+// previous token's partials right after it.
 constexpr int kRegWarps = 16, kRegModes = 4, kRegD = 64, kRegM = 64;
 
 bool ex_reg_form(const ia_shape_t& s) { return s.d_xi == kRegD && s.d_v == kRegD && s.M == kRegM; }
@@ -452,7 +452,24 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     }
     if (a.delta_t && param_thread) rdt = a.delta_t[bh * N + tt];
   };
+  // warps 14-15: column f of num, den and o of token tt from the partials in
+  // buffer pp (written before the block barrier that precedes this call)
+  auto finish = [&](int pp, int tt) {
+    const int f = tid - kSumT0;
+    float nf = 0.f, d = 0.f;
+#pragma unroll
+    for (int w = 0; w < kRegWarps; ++w) {
+      nf += part[pp][w][f];
+      d += dpart[pp][w];
+    }
+    const long long row = bh * N + tt;
+    const float of = nf / d;
+    a.o[row * DV + f] = a.accumulate ? a.o[row * DV + f] + of : of;
+    if (a.num) a.num[row * DV + f] = nf;
+    if (a.den && f == 0) a.den[row] = d;
+  };
   double dt_sum = 0.0;
+  int prev_t = -1, prev_p = 0;   // the token whose partials are pending
   if (step1 > step0) fetch(a.reverse ? N - 1 - step0 : step0);
   for (int step = step0; step < step1; ++step) {
     const int t = a.reverse ? N - 1 - step : step;
@@ -485,6 +502,7 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     }
     if (step + 1 < step1) fetch(a.reverse ? N - 2 - step : step + 1);
     __syncthreads();
+    if (prev_t >= 0 && tid >= kSumT0) finish(prev_p, prev_t);
     // the update, and this lane's part of a = U xi(q) for the warp's modes
     const float2 zk = *reinterpret_cast<const float2*>(&zs[p][f0]);
     const float2 zv = *reinterpret_cast<const float2*>(&zs[p][DX + f0]);
@@ -543,21 +561,12 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     }
     *reinterpret_cast<float2*>(&part[p][warp][f0]) = make_float2(n0, n1);
     if (lane == 0) dpart[p][warp] = dn;
+    prev_t = t;
+    prev_p = p;
+  }
+  if (prev_t >= 0) {   // the last token's sum (uniform: readout and a non-empty range)
     __syncthreads();
-    if (tid >= kSumT0) {   // warps 14-15: column f of num, den, o
-      const int f = tid - kSumT0;
-      float nf = 0.f, d = 0.f;
-#pragma unroll
-      for (int w = 0; w < kRegWarps; ++w) {
-        nf += part[p][w][f];
-        d += dpart[p][w];
-      }
-      const long long row = bh * N + t;
-      const float of = nf / d;
-      a.o[row * DV + f] = a.accumulate ? a.o[row * DV + f] + of : of;
-      if (a.num) a.num[row * DV + f] = nf;
-      if (a.den && f == 0) a.den[row] = d;
-    }
+    if (tid >= kSumT0) finish(prev_p, prev_t);
   }
   // end state: pass 1 into this segment's slot, else the last segment's state_out
   float2* du = nullptr;
