@@ -356,9 +356,10 @@ __global__ void __launch_bounds__(256, 3) seq_fwd_ex_kernel(int H, int N, int DX
 // keeps its warp's four eta), so that the state does not pass through shared
 // memory every token.  Warps 0-3 stage the token's z and xi(q), warps 4-5 its
 // lambda_t, b_t, in shared memory, double-buffered by token parity, and so are
-// the warps' partial num and den: one block barrier per token orders the
-// update (a second, with W, the exchange of a), and warps 14-15 sum the
-// previous token's partials right after it.
+// a and the warps' partial num and den: one block barrier per token orders
+// the update, warps 14-15 sum the previous token's partials right after it,
+// and with W a token's readout (which needs every warp's a) is formed after
+// the next token's barrier, from its a and the state before that update.
 constexpr int kRegWarps = 16, kRegModes = 4, kRegD = 64, kRegM = 64;
 
 bool ex_reg_form(const ia_shape_t& s) { return s.d_xi == kRegD && s.d_v == kRegD && s.M == kRegM; }
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
   __shared__ __align__(16) float zs[2][D];     // xi(k) | v, normalised when asked
   __shared__ __align__(16) float qs[2][DX];    // xi(q)
   __shared__ float2 lamS[2][M], bS[2][M];
-  __shared__ float2 aS[M];                     // a, for the readout matrix
+  __shared__ float2 aS[2][M];                  // a, for the readout matrix
   __shared__ __align__(16) float part[2][kRegWarps][DV];
   __shared__ float dpart[2][kRegWarps];
   __shared__ float red[4];
@@ -468,8 +469,39 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     if (a.num) a.num[row * DV + f] = nf;
     if (a.den && f == 0) a.den[row] = d;
   };
+  // W: this warp's rows of a~ = W_h a from buffer pp, then its partial num
+  // and den with the current state, into the partial buffer pp
+  auto w_partials = [&](int pp) {
+    const float2 a0 = aS[pp][f0], a1 = aS[pp][f0 + 1];
+    float sr[kRegModes], si[kRegModes];
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const float4 w = *reinterpret_cast<const float4*>(Ws + (m0 + u) * M + f0);   // W[m][2l], W[m][2l+1]
+      sr[u] = fmaf(w.x, a0.x, fmaf(-w.y, a0.y, fmaf(w.z, a1.x, -w.w * a1.y)));
+      si[u] = fmaf(w.x, a0.y, fmaf(w.y, a0.x, fmaf(w.z, a1.y, w.w * a1.x)));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int u = 0; u < kRegModes; ++u) {
+        sr[u] += __shfl_xor_sync(0xffffffffu, sr[u], off);
+        si[u] += __shfl_xor_sync(0xffffffffu, si[u], off);
+      }
+    }
+    float n0 = 0.f, n1 = 0.f, dn = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRegModes; ++u) {
+      const float2 at = make_float2(sr[u], si[u]);
+      n0 += re_conj_mul(at, G[u][0]);
+      n1 += re_conj_mul(at, G[u][1]);
+      dn += re_conj_mul(at, E[u]);
+    }
+    *reinterpret_cast<float2*>(&part[pp][warp][f0]) = make_float2(n0, n1);
+    if (lane == 0) dpart[pp][warp] = dn;
+  };
   double dt_sum = 0.0;
-  int prev_t = -1, prev_p = 0;   // the token whose partials are pending
+  int prev_t = -1, prev_p = 0;   // the token whose partials are written, not yet summed
+  int wpend_t = -1, wpend_p = 0;  // W: the token whose a is staged, its readout not yet formed
   if (step1 > step0) fetch(a.reverse ? N - 1 - step0 : step0);
   for (int step = step0; step < step1; ++step) {
     const int t = a.reverse ? N - 1 - step : step;
@@ -503,6 +535,12 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     if (step + 1 < step1) fetch(a.reverse ? N - 2 - step : step + 1);
     __syncthreads();
     if (prev_t >= 0 && tid >= kSumT0) finish(prev_p, prev_t);
+    if (wpend_t >= 0) {   // W: the previous token's readout, with the state before this update
+      w_partials(wpend_p);
+      prev_t = wpend_t;
+      prev_p = wpend_p;
+      wpend_t = -1;
+    }
     // the update, and this lane's part of a = U xi(q) for the warp's modes
     const float2 zk = *reinterpret_cast<const float2*>(&zs[p][f0]);
     const float2 zv = *reinterpret_cast<const float2*>(&zs[p][DX + f0]);
@@ -528,27 +566,14 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
         ai[u] += __shfl_xor_sync(0xffffffffu, ai[u], off);
       }
     }
-    if (a.W) {   // a~ = W_h a: every warp needs all of a
+    if (a.W) {   // a~ = W_h a needs every warp's a: staged, formed after the next barrier
       if (lane == 0) {
 #pragma unroll
-        for (int u = 0; u < kRegModes; ++u) aS[m0 + u] = make_float2(ar[u], ai[u]);
+        for (int u = 0; u < kRegModes; ++u) aS[p][m0 + u] = make_float2(ar[u], ai[u]);
       }
-      __syncthreads();
-      const float2 a0 = aS[f0], a1 = aS[f0 + 1];
-#pragma unroll
-      for (int u = 0; u < kRegModes; ++u) {
-        const float4 w = *reinterpret_cast<const float4*>(Ws + (m0 + u) * M + f0);   // W[m][2l], W[m][2l+1]
-        ar[u] = fmaf(w.x, a0.x, fmaf(-w.y, a0.y, fmaf(w.z, a1.x, -w.w * a1.y)));
-        ai[u] = fmaf(w.x, a0.y, fmaf(w.y, a0.x, fmaf(w.z, a1.y, w.w * a1.x)));
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-#pragma unroll
-        for (int u = 0; u < kRegModes; ++u) {
-          ar[u] += __shfl_xor_sync(0xffffffffu, ar[u], off);
-          ai[u] += __shfl_xor_sync(0xffffffffu, ai[u], off);
-        }
-      }
+      wpend_t = t;
+      wpend_p = p;
+      continue;
     }
     // this lane's two columns of num over the warp's modes, and den
     float n0 = 0.f, n1 = 0.f, dn = 0.f;
@@ -564,9 +589,14 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) seq_ex_reg_kernel(int H, in
     prev_t = t;
     prev_p = p;
   }
-  if (prev_t >= 0) {   // the last token's sum (uniform: readout and a non-empty range)
+  if (prev_t >= 0 || wpend_t >= 0) {   // the pending sums (uniform: readout and a non-empty range)
     __syncthreads();
-    if (tid >= kSumT0) finish(prev_p, prev_t);
+    if (prev_t >= 0 && tid >= kSumT0) finish(prev_p, prev_t);
+    if (wpend_t >= 0) {   // the last token's readout with W (the other partial buffer)
+      w_partials(wpend_p);
+      __syncthreads();
+      if (tid >= kSumT0) finish(wpend_p, wpend_t);
+    }
   }
   // end state: pass 1 into this segment's slot, else the last segment's state_out
   float2* du = nullptr;
