@@ -57,9 +57,37 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
   ModeD md = mode_consts(dl, A, m);
   const double rdA = dl * md.ar, idA = dl * md.ai;
   if (part == 0 && !(dl > 0.f && fabs(rdA) * (C / 2) <= log(kMaxHalfChunkGrowth))) atomicOr(err, kErrParamRange);
-  double pr, pi, ir, ii;
-  cpow_d(rdA, idA, c - JS * part, &pr, &pi);   // lambda^(c-j) at this thread's first j
-  cpow_d(rdA, idA, -1.0, &ir, &ii);            // lambda^-1
+  // The powers of lambda the tables need, from lambda itself by complex
+  // squarings, products and inverses in fp64 (relative error about n eps for
+  // lambda^n, far below the fp16 and fp32 the tables store).
+  auto cm = [](double ar, double ai, double br, double bi, double* r, double* i) {
+    *r = ar * br - ai * bi;
+    *i = ar * bi + ai * br;
+  };
+  auto cinv = [](double ar, double ai, double* r, double* i) {   // 1 / a = conj(a) / |a|^2
+    const double n = ar * ar + ai * ai;
+    *r = ar / n;
+    *i = -ai / n;
+  };
+  double l16r = md.lr, l16i = md.li;
+  for (int sq = 0; sq < 4; ++sq) cm(l16r, l16i, l16r, l16i, &l16r, &l16i);   // lambda^16
+  double l32r, l32i, ir, ii;
+  cm(l16r, l16i, l16r, l16i, &l32r, &l32i);                                 // lambda^32
+  cinv(md.lr, md.li, &ir, &ii);                                              // lambda^-1
+  static_assert(c == 32 && JS == 16, "the first powers below are lambda^32, ^16, ^0, ^-16");
+  double pr, pi;   // lambda^(c-j) at this thread's first j
+  if (part == 0) {
+    pr = l32r;
+    pi = l32i;
+  } else if (part == 1) {
+    pr = l16r;
+    pi = l16i;
+  } else if (part == 2) {
+    pr = 1.0;
+    pi = 0.0;
+  } else {
+    cinv(l16r, l16i, &pr, &pi);
+  }
   double sr = 0.0, si = 0.0;
   double dsr[3] = {0.0, 0.0, 0.0}, dsi[3] = {0.0, 0.0, 0.0};
   char* base = reinterpret_cast<char*>(Es);
@@ -117,15 +145,18 @@ __global__ void __launch_bounds__(4 * kModesTC) param_tables_kernel(int H, const
     T->re_dA[m] = rdA;
     T->im_dA[m] = idA;
   } else if (part == 1) {
-    cpow_d(rdA, idA, C, &pr, &pi);
+    static_assert(C == 64, "lambda^C is lambda^32 squared");
+    cm(l32r, l32i, l32r, l32i, &pr, &pi);
     T->lamC[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
-    T->r2[m] = static_cast<float>(exp(2.0 * rdA));
+    T->r2[m] = static_cast<float>(md.lr * md.lr + md.li * md.li);   // |lambda|^2
   } else if (part == 2) {
-    cpow_d(rdA, idA, C - c - 1, &pr, &pi);
+    cm(l32r, l32i, ir, ii, &pr, &pi);   // lambda^(C-c-1) = lambda^31
     T->sc[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
-    T->s0[m] = static_cast<float>(exp(-2.0 * c * rdA));
+    T->s0[m] = static_cast<float>(1.0 / (l32r * l32r + l32i * l32i));   // |lambda|^(-2c)
   } else {
-    cpow_d(rdA, idA, -(C - c - 1), &pr, &pi);
+    double tr, ti;
+    cm(l32r, l32i, ir, ii, &tr, &ti);
+    cinv(tr, ti, &pr, &pi);   // lambda^-(C-c-1)
     T->sc_inv[m] = make_float2(static_cast<float>(pr), static_cast<float>(pi));
   }
   __syncthreads();
