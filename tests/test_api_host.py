@@ -243,3 +243,18 @@ def test_token_serial_segments_follow_the_workspace():
     plain = ia.prefill_ex_workspace_bytes(B, H, N, d, d, M, "f32", readout=True)
     assert plain == 16 + (ia.prefill_ex_segments(B, H, N, d, d, M, "f32", plain, readout=True) - 1) * per_seg
     assert ia.prefill_ex_segments(B, H, 4096, 64, 64, 64, "bf16", 1 << 30, norm=True) == 1   # tensor cores
+
+
+def test_optional_parts_path_selection_and_readout_workspace():
+    # host logic only: which kernels ia_prefill_fwd_ex runs, and the W'
+    # operands (32 KB per head) in the tensor-core form's workspace
+    import ssm_token_mixer_b200 as ia
+    B, H, N = 2, 3, 300
+    tc = lambda dx, **kw: ia.prefill_ex_path(B, H, N, dx, 64, 64, "bf16", **kw)
+    assert tc(64, readout=True) == tc(64, readout=True, norm=True, bidirectional=True) == "tensor_core"
+    assert tc(128, readout=True) == "sequential"          # W' does not fit beside the d_xi = 128 tiles
+    assert tc(64, selective=True) == tc(64, selective=True, readout=True) == "sequential"
+    assert ia.prefill_ex_path(B, H, N, 64, 64, 64, "f32", readout=True) == "sequential"
+    plain = ia.prefill_ex_workspace_bytes(B, H, N, 64, 64, 64, "bf16", norm=True)
+    with_w = ia.prefill_ex_workspace_bytes(B, H, N, 64, 64, 64, "bf16", norm=True, readout=True)
+    assert with_w - plain == H * 32768
