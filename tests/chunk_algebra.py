@@ -21,6 +21,10 @@ same product R = lambda^C S_hat0 = lambda^(c+1) S0.  For one chunk:
     num_i  = sum_j P_ij v_j + Re sum_m X[i,m] R_Gamma[m]
     den_i  = sum_j P_ij     + Re sum_m X[i,m] R_eta[m]
     S_hat1 = R + sum_j E'[j] x_j^T          (x = xi(k), v, 1)
+With a complex readout matrix W (summary sec. A.3: a~~_i = W a_i before the
+readout) the readout factor mixes modes, so X is formed from a itself:
+    a[i]   = lambda^(i-c) a~[i];  a~~[i] = W a[i];  X[i] = lambda^(i-c) conj(a~~[i])
+and P, num, den follow as above (the kernels' extra contraction G_W).
 A ragged last chunk is zero-padded; its padded tokens add nothing but still
 decay the state, which the end state undoes with lambda^(n_valid - C).
 Segments: the local end states of equal segments of L tokens combine as
@@ -41,8 +45,9 @@ def tables(lam, b, C):
     return Ep, s, c
 
 
-def chunk_pass(fq, fk, v, lam, b, C, S0=None, with_outputs=True, rnd=None):
-    """One (b,h) sequence.  fq, fk [N,d], v [N,dv]; S0 = (U, G, eta) unscaled.
+def chunk_pass(fq, fk, v, lam, b, C, S0=None, with_outputs=True, rnd=None, W=None):
+    """One (b,h) sequence.  fq, fk [N,d], v [N,dv]; S0 = (U, G, eta) unscaled;
+    W [M,M] complex, the readout matrix, or None.
 
     rnd, if given, is a function applied to every tensor-core operand (to
     emulate fp16/bf16 rounding); accumulations stay fp64 here.
@@ -74,7 +79,13 @@ def chunk_pass(fq, fk, v, lam, b, C, S0=None, with_outputs=True, rnd=None):
             Sb = r(np.where(causal & (ii[None, :] < nv), S, 0.0))
             RUr = r(RU.real) + 1j * r(RU.imag)
             at = Sb @ Epr + Q @ RUr.T                            # a~ [C, M]
-            X = s * np.conj(at)
+            if W is None:
+                X = s * np.conj(at)
+            else:
+                lic = lam[None, :] ** (ii[:, None] - c)          # lambda^(i-c) [C, M]
+                a = lic * at
+                aw = (r(a.real) + 1j * r(a.imag)) @ (r(W.real) + 1j * r(W.imag)).T   # a~~ = W a
+                X = lic * np.conj(aw)
             Xr = r(X.real) + 1j * r(X.imag)
             P = np.where(causal, (Xr @ Epr.T).real, 0.0)
             Pr = r(P)

@@ -76,3 +76,44 @@ def test_p7_chunked_reverse_mode_equals_oracle_adjoint(oracle_mod, N, C):
     assert rel(dxk * dfeat(k[0, 0]), ref["dk"][0, 0]) < 1e-9
     assert rel(dvv, ref["dv"][0, 0]) < 1e-9
     assert abs(dD - ref["dDelta"][0]) < 1e-9 * max(1.0, abs(ref["dDelta"][0]))
+
+
+@pytest.mark.parametrize("N", [1, 64, 77, 200])
+def test_p7_chunked_with_readout_matrix(oracle_mod, N):
+    # the readout matrix in the chunked form (a = lambda^(i-c) a~, a~~ = W a,
+    # X = lambda^(i-c) conj(a~~)) equals the oracle's extended forward with W,
+    # also from a prefix's state; with fp16-rounded operands it stays within
+    # the bf16 tolerance
+    rng = np.random.default_rng(900 + N)
+    d, dv, M, P = 4, 3, 6, 30
+    q = rng.standard_normal((1, 1, P + N, d)); k = rng.standard_normal((1, 1, P + N, d))
+    v = rng.standard_normal((1, 1, P + N, dv))
+    delta = np.array([0.05])
+    W = (rng.standard_normal((1, M, M)) + 1j * rng.standard_normal((1, M, M))) / np.sqrt(M) + np.eye(M)
+    ref = oracle_mod.forward_ex(q, k, v, M, delta=delta, W=W)
+    pre = oracle_mod.forward_ex(q[:, :, :P], k[:, :, :P], v[:, :, :P], M, delta=delta, W=W)
+    U0, G0, e0 = oracle_mod.split_state(pre["state"], 1, 1, M, d, dv)
+    lam, b = oracle_mod.params(M, delta[0])
+    sl = slice(P, P + N)
+    o, num, den, (U, G, e) = chunk_pass(feat(q[0, 0, sl]), feat(k[0, 0, sl]), v[0, 0, sl], lam, b, 64,
+                                        S0=(U0[0, 0], G0[0, 0], e0[0, 0]), W=W[0])
+    assert rel(num, ref["num"][0, 0, sl]) < 1e-10
+    assert rel(den, ref["den"][0, 0, sl]) < 1e-10
+    Ur, Gr, er = oracle_mod.split_state(ref["state"], 1, 1, M, d, dv)
+    assert rel(U, Ur[0, 0]) < 1e-10 and rel(G, Gr[0, 0]) < 1e-10 and rel(e, er[0, 0]) < 1e-10
+    f16 = lambda x: np.asarray(x, np.float16).astype(np.float64)
+    _, num16, den16, _ = chunk_pass(feat(q[0, 0, sl]), feat(k[0, 0, sl]), v[0, 0, sl], lam, b, 64,
+                                    S0=(U0[0, 0], G0[0, 0], e0[0, 0]), W=W[0], rnd=f16)
+    assert rel(num16, ref["num"][0, 0, sl]) < 1e-2 and rel(den16, ref["den"][0, 0, sl]) < 1e-2
+
+
+def test_p7_readout_matrix_identity_is_the_plain_chunked_form(oracle_mod):
+    # W = I through the a -> a~~ -> X route gives the plain X = s conj(a~)
+    rng = np.random.default_rng(7)
+    N, d, dv, M = 100, 3, 2, 5
+    fq, fk = feat(rng.standard_normal((N, d))), feat(rng.standard_normal((N, d)))
+    v = rng.standard_normal((N, dv))
+    lam, b = oracle_mod.params(M, 0.08)
+    plain = chunk_pass(fq, fk, v, lam, b, 64)
+    ident = chunk_pass(fq, fk, v, lam, b, 64, W=np.eye(M, dtype=complex))
+    assert rel(ident[1], plain[1]) < 1e-12 and rel(ident[2], plain[2]) < 1e-12
