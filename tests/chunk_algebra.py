@@ -104,6 +104,66 @@ def chunk_pass(fq, fk, v, lam, b, C, S0=None, with_outputs=True, rnd=None, W=Non
     return o, num, den, end
 
 
+def chunk_pass_selective(fq, fk, v, dts, A, C, S0=None, rnd=None):
+    """The chunked form with a step per token (selective writing and memory
+    decay, summary sec. 3.3): lambda_t = exp(Delta_t A), b_t = (lambda_t - 1)/A.
+    With cs the inclusive cumulative sum of Delta_t inside a chunk, the decay
+    from token j to token i is exp(A (cs_i - cs_j)) = exp(A (cs_i - cs_c))
+    exp(A (cs_c - cs_j)), so the plain chunk algebra holds with tables per
+    chunk instead of per head:
+        E'_t[j,m] = b_{j,m} exp(A_m (cs_c - cs_j))
+        s_t[i,m]  = |exp(A_m (cs_i - cs_c))|^2
+        R         = exp(A cs_c) S0       end: exp(A (cs_last - cs_c)) (R + E'_t^T x)
+    Padded tokens take Delta = 0 (lambda = 1, b = 0): they neither write nor
+    decay, so a ragged chunk needs no end correction.  The state is kept
+    unscaled here.  fq, fk [N,d], v [N,dv], dts [N], A [M] complex."""
+    N, d = fq.shape
+    dv = v.shape[1]
+    M = A.shape[0]
+    c = C // 2
+    r = rnd if rnd is not None else (lambda x: x)
+    if S0 is None:
+        U = np.zeros((M, d), complex); G = np.zeros((M, dv), complex); eta = np.zeros(M, complex)
+    else:
+        U, G, eta = (np.array(x, complex) for x in S0)
+    o = np.zeros((N, dv)); num = np.zeros((N, dv)); den = np.zeros(N)
+    ii = np.arange(C)
+    causal = ii[None, :] <= ii[:, None]
+    for n0 in range(0, N, C):
+        nv = min(C, N - n0)
+        Q = np.zeros((C, d)); K = np.zeros((C, d)); V = np.zeros((C, dv)); one = np.zeros(C); dt = np.zeros(C)
+        Q[:nv] = fq[n0:n0 + nv]; K[:nv] = fk[n0:n0 + nv]; V[:nv] = v[n0:n0 + nv]; one[:nv] = 1.0
+        dt[:nv] = dts[n0:n0 + nv]
+        Q, K, V = r(Q), r(K), r(V)
+        cs = np.cumsum(dt)
+        lam_t = np.exp(dt[:, None] * A[None, :])
+        b_t = (lam_t - 1.0) / A[None, :]
+        Ep = b_t * np.exp(A[None, :] * (cs[c] - cs[:, None]))
+        Epr = r(Ep.real) + 1j * r(Ep.imag)
+        s = np.abs(np.exp(A[None, :] * (cs[:, None] - cs[c]))) ** 2
+        rc = np.exp(A * cs[c])
+        RU, RG, Re_ = rc[:, None] * U, rc[:, None] * G, rc * eta
+        S = Q @ K.T
+        Sb = r(np.where(causal & (ii[None, :] < nv), S, 0.0))
+        RUr = r(RU.real) + 1j * r(RU.imag)
+        at = Sb @ Epr + Q @ RUr.T
+        X = s * np.conj(at)
+        Xr = r(X.real) + 1j * r(X.imag)
+        P = r(np.where(causal, (Xr @ Epr.T).real, 0.0))
+        RGr = r(RG.real) + 1j * r(RG.imag)
+        Rer = r(Re_.real) + 1j * r(Re_.imag)
+        nm = P @ V + (Xr @ RGr).real
+        dn = P @ one + (Xr @ Rer).real
+        o[n0:n0 + nv] = nm[:nv] / dn[:nv, None]
+        num[n0:n0 + nv] = nm[:nv]
+        den[n0:n0 + nv] = dn[:nv]
+        rend = np.exp(A * (cs[-1] - cs[c]))
+        U = rend[:, None] * (RU + Epr.T @ K)
+        G = rend[:, None] * (RG + Epr.T @ V)
+        eta = rend * (Re_ + Epr.T @ one)
+    return o, num, den, (U, G, eta)
+
+
 def segmented_pass(fq, fk, v, lam, b, C, L):
     """Two-pass form over segments of L tokens (L a multiple of C):
     local end states from zero, an exclusive scan of the carries, then every

@@ -117,3 +117,49 @@ def test_p7_readout_matrix_identity_is_the_plain_chunked_form(oracle_mod):
     plain = chunk_pass(fq, fk, v, lam, b, 64)
     ident = chunk_pass(fq, fk, v, lam, b, 64, W=np.eye(M, dtype=complex))
     assert rel(ident[1], plain[1]) < 1e-12 and rel(ident[2], plain[2]) < 1e-12
+
+
+@pytest.mark.parametrize("N", [1, 64, 77, 200])
+def test_p7_chunked_with_steps_per_token(oracle_mod, N):
+    # selective writing and memory decay in the chunked form: per-chunk
+    # tables from the cumulative sum of the steps, the same contractions;
+    # equals the oracle's extended forward with delta_t and a general A, from
+    # a prefix's state, in fp64; fp16-rounded operands stay within 1e-2 over
+    # the bench's step range [5e-3, 1e-1]
+    from chunk_algebra import chunk_pass_selective
+    rng = np.random.default_rng(1300 + N)
+    d, dv, M, P = 4, 3, 6, 30
+    q = rng.standard_normal((1, 1, P + N, d)); k = rng.standard_normal((1, 1, P + N, d))
+    v = rng.standard_normal((1, 1, P + N, dv))
+    dts = np.exp(np.log(5e-3) + rng.random((1, 1, P + N)) * (np.log(1e-1) - np.log(5e-3)))
+    Ac = -(0.2 + 0.6 * rng.random(M)) + 1j * (np.pi * np.arange(M) + 0.7 * rng.random(M))
+    A = np.empty(2 * M); A[0::2] = Ac.real; A[1::2] = Ac.imag
+    ref = oracle_mod.forward_ex(q, k, v, M, A=A, delta_t=dts)
+    pre = oracle_mod.forward_ex(q[:, :, :P], k[:, :, :P], v[:, :, :P], M, A=A, delta_t=dts[:, :, :P])
+    U0, G0, e0 = oracle_mod.split_state(pre["state"], 1, 1, M, d, dv)
+    sl = slice(P, P + N)
+    args = (feat(q[0, 0, sl]), feat(k[0, 0, sl]), v[0, 0, sl], dts[0, 0, sl], Ac, 64)
+    S0 = (U0[0, 0], G0[0, 0], e0[0, 0])
+    o, num, den, (U, G, e) = chunk_pass_selective(*args, S0=S0)
+    assert rel(num, ref["num"][0, 0, sl]) < 1e-10
+    assert rel(den, ref["den"][0, 0, sl]) < 1e-10
+    Ur, Gr, er = oracle_mod.split_state(ref["state"], 1, 1, M, d, dv)
+    assert rel(U, Ur[0, 0]) < 1e-10 and rel(G, Gr[0, 0]) < 1e-10 and rel(e, er[0, 0]) < 1e-10
+    f16 = lambda x: np.asarray(x, np.float16).astype(np.float64)
+    _, num16, den16, _ = chunk_pass_selective(*args, S0=S0, rnd=f16)
+    assert rel(num16, ref["num"][0, 0, sl]) < 1e-2 and rel(den16, ref["den"][0, 0, sl]) < 1e-2
+
+
+def test_p7_steps_per_token_constant_step_is_the_plain_chunked_form(oracle_mod):
+    # a constant step reduces the per-chunk tables to the per-head ones
+    from chunk_algebra import chunk_pass_selective
+    rng = np.random.default_rng(11)
+    N, d, dv, M, delta = 150, 3, 2, 5, 0.07
+    fq, fk = feat(rng.standard_normal((N, d))), feat(rng.standard_normal((N, d)))
+    v = rng.standard_normal((N, dv))
+    lam, b = oracle_mod.params(M, delta)
+    Ac = -0.5 + 1j * np.pi * np.arange(M)
+    plain = chunk_pass(fq, fk, v, lam, b, 64)
+    sel = chunk_pass_selective(fq, fk, v, np.full(N, delta), Ac, 64)
+    assert rel(sel[1], plain[1]) < 1e-11 and rel(sel[2], plain[2]) < 1e-11
+    assert all(rel(x, y) < 1e-11 for x, y in zip(sel[3], plain[3]))
